@@ -1,0 +1,221 @@
+"""CPU oracle for the group-wise INT4 weight-only linear layer (W4A16, AWQ style).
+
+TEST INFRASTRUCTURE ONLY. This module is the plain, slow, obviously correct
+statement of what the CUDA library computes. Only the test suite, the smoke
+check in ``__graft_entry__`` and the CPU-baseline / reference arm of
+``bench.py`` may import it. The CUDA product path never imports, links or
+calls it, and it shares no code, table or constant generator with the CUDA
+sources: the nibble order below is restated here from the documented
+format, not imported.
+
+Sources (cited by page title and section):
+
+* "AutoAWQ" code tour (pyshine.com), section "The Quantization Flow Up
+  Close": pseudo-quantization rounds each group of weights to integer
+  levels against a per-group scale and zero point; section "From Install to
+  Your First Model": ``zero_point`` selects asymmetric vs symmetric,
+  ``q_group_size`` = 128 weights share one scale (and zero), ``w_bit`` = 4.
+* "AWQ > Implementation" (Language AI Handbook), section "Understanding the
+  Quantization Structure": ``qweight`` holds eight 4-bit codes per int32,
+  scales are fp16, one scale and zero per group of 128 weights.
+* "AWQ Quantization Support" (fak explainer), section "Dequantization
+  Formula": weight = scale x (code - 8) for the symmetric variant, codes
+  0..15.
+* "AutoAWQ" code tour, section "The big picture": dividing an input channel
+  of x by a constant and multiplying the matching weight column by it leaves
+  the layer output unchanged (used as a pin on the matmul, not here).
+
+Readings where the pages are silent (each is listed in the design doc):
+
+* Asymmetric scale/zero follow the plain per-group min/max affine rule on
+  the levels 0..15; the range is not widened to include 0.
+* Quantize arithmetic is IEEE fp32 with round-to-nearest-even, and the
+  fp16-rounded scale is the one used to derive the zero point and the codes.
+* The fp32 scale is floored at 1e-5 before the fp16 cast (constant groups).
+* ``rint`` (ties to even) for every rounding to an integer.
+* Symmetric scale = max|w| / 7 (largest positive level 7); codes are
+  clamp(rint(w/s), -8, 7) + 8.
+* Zero points are stored as fp16 values holding the integers 0..15.
+* Packing is along K, eight consecutive k per int32 word; nibble slot i
+  (bits 4i..4i+3) of the word covering k = 8w..8w+7 holds k = 8w + SLOT_K[i]
+  with SLOT_K = (0, 2, 4, 6, 1, 3, 5, 7).
+
+Every function below works on NumPy arrays. fp16 tensors are numpy.float16,
+packed words are numpy.int32 (the uint32 bit pattern reinterpreted).
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+GROUP_SIZE = 128
+W_BIT = 4
+LEVELS = 2 ** W_BIT - 1            # highest code, 15
+SYM_ZERO = 8                       # fixed zero point of the symmetric variant
+SCALE_FLOOR = np.float32(1e-5)     # reading: floor on the fp32 scale
+# Nibble slot i of a packed word holds k offset SLOT_K[i] (documented format).
+SLOT_K = (0, 2, 4, 6, 1, 3, 5, 7)
+
+
+def _groups_f32(W: np.ndarray, group_size: int) -> np.ndarray:
+    """View fp16 W[N, K] as fp32 [N, K/g, g] (exact widening)."""
+    W = np.asarray(W)
+    if W.dtype != np.float16:
+        raise TypeError("W must be float16")
+    N, K = W.shape
+    if group_size <= 0 or K % group_size:
+        raise ValueError("K must be a positive multiple of the group size")
+    return W.astype(np.float32).reshape(N, K // group_size, group_size)
+
+
+def quantize_asym(W: np.ndarray, group_size: int = GROUP_SIZE):
+    """Asymmetric (zero-point) group quantization of fp16 W[N, K].
+
+    Follows the AutoAWQ tour, "The Quantization Flow Up Close" (round each
+    group to integer levels against its scale and zero point) with the
+    min/max reading. Per row n and group j, with w the group's values in
+    fp32:
+
+      1. mx = max(w), mn = min(w)
+      2. s32 = max((mx - mn) / 15, 1e-5)            fp32, round to nearest even
+      3. s = fp16(s32); sf = float(s)
+      4. z = clamp(-rint(mn / sf), 0, 15)
+      5. q = clamp(rint(w / sf) + z, 0, 15)
+
+    Returns (codes uint8 [N, K], scales fp16 [N, G], zeros fp16 [N, G]).
+    """
+    w = _groups_f32(W, group_size)
+    mx = w.max(axis=2)
+    mn = w.min(axis=2)
+    s32 = np.maximum((mx - mn) / np.float32(LEVELS), SCALE_FLOOR)
+    scales = s32.astype(np.float16)
+    sf = scales.astype(np.float32)
+    z = np.clip(-np.rint(mn / sf), 0, LEVELS).astype(np.float32)
+    q = np.clip(np.rint(w / sf[..., None]) + z[..., None], 0, LEVELS)
+    codes = q.astype(np.uint8).reshape(W.shape)
+    return codes, scales, z.astype(np.float16)
+
+
+def quantize_sym(W: np.ndarray, group_size: int = GROUP_SIZE):
+    """Symmetric group quantization, zero point fixed at 8.
+
+    The fak explainer, "Dequantization Formula", fixes the decode as
+    scale x (code - 8) with codes 0..15; the scale rule is the reading
+    s = max|w| / 7. Per row n and group j:
+
+      1. a = max|w|
+      2. s32 = max(a / 7, 1e-5); s = fp16(s32); sf = float(s)
+      3. c = clamp(rint(w / sf), -8, 7); q = c + 8
+
+    With this scale |w / sf| stays below 7.5 (the fp16 rounding of the scale
+    is far smaller than the margin, and the 1e-5 floor only lowers the
+    ratio), so code 0 (c = -8) is never produced: 15 of the 16 levels are
+    used, as the max/7 reading implies.
+
+    Returns (codes uint8 [N, K], scales fp16 [N, G]).
+    """
+    w = _groups_f32(W, group_size)
+    a = np.abs(w).max(axis=2)
+    s32 = np.maximum(a / np.float32(7.0), SCALE_FLOOR)
+    scales = s32.astype(np.float16)
+    sf = scales.astype(np.float32)
+    c = np.clip(np.rint(w / sf[..., None]), -8, 7)
+    codes = (c + SYM_ZERO).astype(np.uint8).reshape(W.shape)
+    return codes, scales
+
+
+def pseudo_quantize(W: np.ndarray, group_size: int = GROUP_SIZE, zero_point: bool = True):
+    """Quantize with the variant ``zero_point`` selects (AutoAWQ tour, "From
+    Install to Your First Model"). Returns (codes, scales, zeros-or-None)."""
+    if zero_point:
+        return quantize_asym(W, group_size)
+    codes, scales = quantize_sym(W, group_size)
+    return codes, scales, None
+
+
+def pack(codes: np.ndarray) -> np.ndarray:
+    """Pack 4-bit codes [N, K] into int32 words [N, K/8], eight per word
+    ("AWQ > Implementation", "Understanding the Quantization Structure").
+
+    Word w of a row covers k = 8w .. 8w+7; nibble slot i holds k = 8w +
+    SLOT_K[i].
+    """
+    codes = np.asarray(codes)
+    N, K = codes.shape
+    if K % 8:
+        raise ValueError("K must be a multiple of 8")
+    if codes.size and (codes.min() < 0 or codes.max() > LEVELS):
+        raise ValueError("codes must lie in 0..15")
+    c = codes.astype(np.uint32).reshape(N, K // 8, 8)
+    word = np.zeros((N, K // 8), dtype=np.uint32)
+    for slot, koff in enumerate(SLOT_K):
+        word |= c[:, :, koff] << np.uint32(4 * slot)
+    return word.view(np.int32)
+
+
+def unpack(qweight: np.ndarray) -> np.ndarray:
+    """Inverse of :func:`pack`: int32 words [N, K/8] -> uint8 codes [N, K]."""
+    qweight = np.asarray(qweight)
+    if qweight.dtype != np.int32:
+        raise TypeError("qweight must be int32")
+    N, W = qweight.shape
+    word = qweight.view(np.uint32)
+    codes = np.zeros((N, W, 8), dtype=np.uint8)
+    for slot, koff in enumerate(SLOT_K):
+        codes[:, :, koff] = (word >> np.uint32(4 * slot)) & np.uint32(0xF)
+    return codes.reshape(N, W * 8)
+
+
+def dequant(codes: np.ndarray, scales: np.ndarray, zeros, group_size: int = GROUP_SIZE) -> np.ndarray:
+    """fp16 weights w' = fp16((q - z) * s); z = 8 when ``zeros`` is None.
+
+    Asymmetric: (q - z[n, j]) * s[n, j] (the zero-point decode the AutoAWQ
+    tour names); symmetric: scale x (code - 8) (fak explainer,
+    "Dequantization Formula"). (q - z) * s is exact in fp32 (|q - z| <= 15
+    times an 11-bit significand), so the only rounding is the one cast to
+    fp16, round to nearest even.
+    """
+    codes = np.asarray(codes)
+    N, K = codes.shape
+    G = K // group_size
+    q = codes.astype(np.float32).reshape(N, G, group_size)
+    sf = np.asarray(scales).astype(np.float32).reshape(N, G, 1)
+    if zeros is None:
+        z = np.float32(SYM_ZERO)
+    else:
+        z = np.asarray(zeros).astype(np.float32).reshape(N, G, 1)
+    return ((q - z) * sf).astype(np.float16).reshape(N, K)
+
+
+def matmul_f64(x: np.ndarray, Wd: np.ndarray) -> np.ndarray:
+    """y[m, n] = sum_k x[m, k] * w'[n, k], the plain definition in float64."""
+    return np.asarray(x).astype(np.float64) @ np.asarray(Wd).astype(np.float64).T
+
+
+def linear(x: np.ndarray, qweight: np.ndarray, scales: np.ndarray, zeros,
+           group_size: int = GROUP_SIZE) -> np.ndarray:
+    """The W4A16 linear layer: unpack, dequantize, then the float64 matmul."""
+    return matmul_f64(x, dequant(unpack(qweight), scales, zeros, group_size))
+
+
+def quantize_pack(W: np.ndarray, group_size: int = GROUP_SIZE, zero_point: bool = True):
+    """Quantize then pack: (qweight int32 [N, K/8], scales, zeros-or-None)."""
+    codes, scales, zeros = pseudo_quantize(W, group_size, zero_point)
+    return pack(codes), scales, zeros
+
+
+def rel_frobenius(y: np.ndarray, y_ref: np.ndarray) -> float:
+    """||y - y_ref||_F / ||y_ref||_F in float64."""
+    y = np.asarray(y, dtype=np.float64)
+    y_ref = np.asarray(y_ref, dtype=np.float64)
+    den = np.linalg.norm(y_ref)
+    return float(np.linalg.norm(y - y_ref) / den) if den > 0 else float(np.linalg.norm(y))
+
+
+def max_abs_ratio(y: np.ndarray, y_ref: np.ndarray) -> float:
+    """max|y - y_ref| / max|y_ref| in float64."""
+    y = np.asarray(y, dtype=np.float64)
+    y_ref = np.asarray(y_ref, dtype=np.float64)
+    den = np.abs(y_ref).max() if y_ref.size else 0.0
+    num = np.abs(y - y_ref).max() if y_ref.size else 0.0
+    return float(num / den) if den > 0 else float(num)
