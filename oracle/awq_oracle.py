@@ -93,7 +93,9 @@ def quantize_asym(W: np.ndarray, group_size: int = GROUP_SIZE):
     z = np.clip(-np.rint(mn / sf), 0, LEVELS).astype(np.float32)
     q = np.clip(np.rint(w / sf[..., None]) + z[..., None], 0, LEVELS)
     codes = q.astype(np.uint8).reshape(W.shape)
-    return codes, scales, z.astype(np.float16)
+    # z is an integer level; storing it through an integer keeps 0 as +0
+    # (-rint of a non-negative minimum is -0.0 in floating point).
+    return codes, scales, z.astype(np.int32).astype(np.float16)
 
 
 def quantize_sym(W: np.ndarray, group_size: int = GROUP_SIZE):

@@ -138,6 +138,19 @@ def test_asym_group_golden(golden_dir):
     assert deq[0, :len(vals)].astype(np.float64).tolist() == [float(v) for v in rows["dequant"]]
 
 
+def test_zero_points_are_positive_integers():
+    """Zero points are the integers 0..15 stored as fp16, zero as +0 (an
+    all-positive group has -rint(min/s) = -0)."""
+    W = np.abs(np.random.default_rng(11).normal(0, 0.02, (8, 256))).astype(np.float16)
+    _, _, zeros = O.quantize_asym(W, 128)
+    zb = bits16(zeros)
+    assert np.all(zb == 0)
+    W2 = np.random.default_rng(12).normal(0, 0.02, (64, 256)).astype(np.float16)
+    _, _, z2 = O.quantize_asym(W2, 128)
+    assert np.array_equal(bits16(z2), f16_bits_nearest(np.round(z2.astype(np.float64))))
+    assert np.all((z2.astype(np.float64) >= 0) & (z2.astype(np.float64) <= 15))
+
+
 def test_constant_groups_golden(golden_dir):
     for variant, c, sbits, z, q, wq in _read_golden(golden_dir, "constant_groups.txt"):
         w = np.full((1, 128), float(c), dtype=np.float16)
