@@ -1,0 +1,190 @@
+/*
+ * awq.h -- C ABI of libawq_b200, a W4A16 linear layer for NVIDIA B200 (sm_100a).
+ *
+ * The layer is y = x . W'^T where W' is decoded on the fly from group-wise
+ * 4-bit codes: w' = (q - z) * s (asymmetric, zero point z) or w' = s * (q - 8)
+ * (symmetric). Groups are 128 consecutive input channels of one output
+ * channel. Activations and outputs are fp16, accumulation is fp32.
+ *
+ * Sources, by page and section:
+ *   "AutoAWQ" code tour (pyshine.com): "The Quantization Flow Up Close"
+ *     (pseudo-quantization rounds each group to integer levels against its
+ *     scale and zero point), "The big picture" (WQLinear_GEMM for batched
+ *     requests, WQLinear_GEMV for single-token decode), "From Install to Your
+ *     First Model" (zero_point, q_group_size = 128, w_bit = 4).
+ *   "AutoAWQ" capability page (unfragile.ai): the WQLinear kernels dequantize
+ *     inside the fused matmul and never materialize fp16 weights.
+ *   "AWQ > Implementation" (Language AI Handbook), "Understanding the
+ *     Quantization Structure": eight 4-bit codes per int32, fp16 scales, one
+ *     scale and zero per 128 weights.
+ *   "AWQ Quantization Support" (fak explainer), "Dequantization Formula":
+ *     weight = scale x (code - 8); "Integration with Forward Pass": a
+ *     matrix-vector entry for decode and a batched matmul entry for P tokens.
+ *
+ * ---------------------------------------------------------------------------
+ * Data layout (all row-major, K contiguous; N output channels, K input
+ * channels, G = K / group_size groups per row):
+ *
+ *   W        fp16   [N][K]      (quantizer input; awq_dequant output)
+ *   x        fp16   [M][K]
+ *   y        fp16   [M][N]
+ *   qweight  int32  [N][K/8]    word w of row n covers k = 8w .. 8w+7; nibble
+ *                               slot i (bits 4i .. 4i+3) holds the code of
+ *                               k = 8w + {0,2,4,6,1,3,5,7}[i]. With this
+ *                               order, (word >> 4j) & 0x000F000F holds the
+ *                               codes of the consecutive pair k = 8w+2j,
+ *                               8w+2j+1 in its low and high 16-bit halves.
+ *   scales   fp16   [N][G]      s[n][j] for k in [128j, 128j + 128)
+ *   zeros    fp16   [N][G]      integer zero points 0..15 stored as fp16
+ *                               (asymmetric only; NULL for symmetric)
+ *
+ * fp16 buffers are passed as uint16_t pointers holding IEEE binary16 bits.
+ *
+ * Ownership and execution: every pointer is device memory owned by the
+ * caller (the library allocates nothing and keeps no per-call state). Every
+ * entry point validates its arguments on the host, then enqueues its work on
+ * `stream` (a cudaStream_t; NULL = the legacy default stream) and returns
+ * without synchronizing. A non-OK status means nothing was enqueued, except
+ * AWQ_ERR_CUDA, which reports a launch error from the CUDA runtime.
+ * Device pointers must be 16-byte aligned. Sizes are element counts.
+ * Inputs must be finite (no NaN or infinity); the results for non-finite
+ * inputs are unspecified.
+ * ---------------------------------------------------------------------------
+ */
+#ifndef AWQ_B200_H
+#define AWQ_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define AWQ_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define AWQ_API __attribute__((visibility("default")))
+#else
+#define AWQ_API
+#endif
+
+typedef enum awq_status {
+  AWQ_OK = 0,
+  AWQ_ERR_NULL = 1,        /* a required pointer is NULL                     */
+  AWQ_ERR_SHAPE = 2,       /* a size is negative, out of range or mismatched */
+  AWQ_ERR_ALIGN = 3,       /* a device pointer is not 16-byte aligned        */
+  AWQ_ERR_UNSUPPORTED = 4, /* group size / variant not implemented           */
+  AWQ_ERR_CUDA = 5,        /* the CUDA runtime reported an error             */
+  AWQ_ERR_WORKSPACE = 6    /* workspace missing or smaller than required     */
+} awq_status_t;
+
+/* Quantization configuration ("AutoAWQ" code tour, "From Install to Your
+ * First Model": q_group_size, zero_point; w_bit is fixed at 4).
+ * group_size must be 128. zero_point: 1 = asymmetric, 0 = symmetric. */
+typedef struct awq_qconfig {
+  int32_t group_size;
+  int32_t zero_point;
+} awq_qconfig_t;
+
+/* ABI version of the loaded library (AWQ_ABI_VERSION at build time). */
+AWQ_API int awq_abi_version(void);
+
+/* Static description of a status code. Never NULL. */
+AWQ_API const char* awq_status_string(awq_status_t status);
+
+/*
+ * awq_pseudo_quantize_pack -- quantize fp16 W[N][K] group-wise and pack it.
+ * ("AutoAWQ" code tour, "The Quantization Flow Up Close": each group of
+ * weights is rounded to integer levels against its scale and zero point.)
+ *
+ * Per row n and group j, with w the 128 values in fp32 and IEEE fp32
+ * arithmetic rounded to nearest even:
+ *   asymmetric: s = fp16(max((max w - min w) / 15, 1e-5)),
+ *               z = clamp(-rint(min w / s), 0, 15),
+ *               q = clamp(rint(w / s) + z, 0, 15)
+ *   symmetric:  s = fp16(max(max|w| / 7, 1e-5)),
+ *               q = clamp(rint(w / s), -8, 7) + 8
+ * rint rounds half to even; s is used at its fp16 value.
+ *
+ * In:  W [N][K] fp16.  Out: qweight [N][K/8], scales [N][G], zeros [N][G]
+ * (asymmetric; must be NULL for symmetric).
+ * N >= 0 (N == 0: no work), K > 0 and K % group_size == 0.
+ * Results are bit-exact: a given W always yields the same bits.
+ */
+AWQ_API awq_status_t awq_pseudo_quantize_pack(const uint16_t* W, int64_t N, int64_t K,
+                                      awq_qconfig_t cfg, int32_t* qweight,
+                                      uint16_t* scales, uint16_t* zeros,
+                                      void* stream);
+
+/*
+ * awq_dequant -- decode packed weights to fp16 W'[N][K] (for checks).
+ * ("AWQ Quantization Support", "Dequantization Formula": weight =
+ * scale x (code - 8); asymmetric: (q - z) x s.)
+ * w'[n][k] = fp16((q - z) * s), one rounding to nearest even ((q - z) * s is
+ * exact in fp32), z = 8 for symmetric. Bit-exact.
+ * N >= 0, K > 0, K % group_size == 0; zeros NULL iff symmetric.
+ */
+AWQ_API awq_status_t awq_dequant(const int32_t* qweight, const uint16_t* scales,
+                         const uint16_t* zeros, int64_t N, int64_t K,
+                         awq_qconfig_t cfg, uint16_t* W_out, void* stream);
+
+/*
+ * awq_workspace_bytes -- bytes of workspace awq_gemv / awq_gemm need for
+ * (M, N, K) on the current device. *bytes is 0 when none is needed.
+ * The workspace holds split-K partial sums and arrival counters. It must be
+ * zero-filled before its first use; every call that completes leaves it
+ * zero-filled again, so one memset at allocation suffices. Calls that may
+ * run concurrently need separate workspaces.
+ */
+AWQ_API awq_status_t awq_workspace_bytes(int64_t M, int64_t N, int64_t K,
+                                 awq_qconfig_t cfg, size_t* bytes);
+
+/*
+ * awq_gemv -- y[M][N] = x[M][K] . W'^T for small batches (decode), 1 <= M <= 16.
+ * ("AutoAWQ" code tour, "The big picture": the GEMV variant for single-token
+ * decoding; "AutoAWQ" capability page: dequantization fused into the matmul.)
+ * y[m][n] = fp16( sum_k x[m][k] * (q[n][k] - z[n][k/128]) * s[n][k/128] ),
+ * products and sums in fp32 (the per-group factor s is applied to the fp32
+ * partial sum of each group). The summation order is fixed for a given
+ * device and shape, so results are reproducible run to run.
+ * M in [1, 16]; N >= 0 (0: no work); K > 0, K % group_size == 0.
+ * workspace: at least awq_workspace_bytes(M, N, K) bytes, zero-filled before
+ * first use (see above); may be NULL when that size is 0.
+ */
+AWQ_API awq_status_t awq_gemv(const uint16_t* x, const int32_t* qweight,
+                      const uint16_t* scales, const uint16_t* zeros,
+                      int64_t M, int64_t N, int64_t K, awq_qconfig_t cfg,
+                      uint16_t* y, void* workspace, size_t workspace_bytes,
+                      void* stream);
+
+/*
+ * awq_gemm -- y[M][N] = x[M][K] . W'^T for any M >= 1 (prefill).
+ * ("AutoAWQ" code tour, "The big picture": the GEMM variant for batched
+ * requests; "AWQ Quantization Support", "Integration with Forward Pass":
+ * the batched product over P tokens.)
+ * Tiles of W' are decoded bit-exactly (as awq_dequant) into shared memory and
+ * multiplied on the tensor cores (tcgen05, fp16 inputs, fp32 accumulation in
+ * tensor memory); y = fp16 of the fp32 sum.
+ * M >= 0, N >= 0 (either 0: no work); K > 0, K % group_size == 0.
+ * Workspace as for awq_gemv.
+ */
+AWQ_API awq_status_t awq_gemm(const uint16_t* x, const int32_t* qweight,
+                      const uint16_t* scales, const uint16_t* zeros,
+                      int64_t M, int64_t N, int64_t K, awq_qconfig_t cfg,
+                      uint16_t* y, void* workspace, size_t workspace_bytes,
+                      void* stream);
+
+/*
+ * awq_device_error -- read and clear the device-side error word of the
+ * current device (synchronizes `stream`). Bit 0: a pipeline wait inside
+ * awq_gemm exceeded its iteration limit and the kernel abandoned its tile
+ * (the output is then incomplete). 0 means no error was recorded.
+ */
+AWQ_API awq_status_t awq_device_error(uint32_t* error_word, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AWQ_B200_H */

@@ -1,0 +1,124 @@
+"""C ABI checks that need no GPU: the library loads, exports every symbol the
+header declares, and rejects bad arguments on the host before any CUDA call.
+
+Every call below fails validation before the library touches the CUDA
+runtime (null pointers, bad sizes, bad configuration, misalignment), so the
+pointers passed are never dereferenced."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import weight_only_int4_gemv_b200 as awq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "awq.h")
+
+OK, NULL, SHAPE, ALIGN, UNSUP, CUDA, WS = range(7)
+A = 0x10000          # a 16-byte aligned fake address (never dereferenced)
+MIS = 0x10002        # a misaligned fake address
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"AWQ_API\s+[\w\s\*]+?\b(awq_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    if not os.path.exists(awq.LIB_PATH):
+        from weight_only_int4_gemv_b200 import build
+        build.build()
+    return awq.lib()
+
+
+def cfg(g=128, zp=1):
+    return awq.QConfig(g, zp)
+
+
+def test_header_declares_the_entry_points():
+    syms = declared_symbols()
+    for s in ["awq_pseudo_quantize_pack", "awq_dequant", "awq_gemv", "awq_gemm",
+              "awq_workspace_bytes", "awq_status_string", "awq_abi_version", "awq_device_error"]:
+        assert s in syms
+
+
+def test_library_exports_every_declared_symbol(L):
+    for s in declared_symbols():
+        assert hasattr(L, s), s
+        assert ctypes.cast(getattr(L, s), ctypes.c_void_p).value
+
+
+def test_abi_version_matches_header(L):
+    m = re.search(r"#define AWQ_ABI_VERSION (\d+)", open(HEADER).read())
+    assert L.awq_abi_version() == int(m.group(1))
+
+
+def test_status_strings(L):
+    for st in range(7):
+        assert L.awq_status_string(st)
+    assert L.awq_status_string(99) == b"unknown status"
+
+
+def _gemv(L, x=A, q=A, s=A, z=A, M=1, N=64, K=256, c=None, y=A, entry="awq_gemv"):
+    fn = getattr(L, entry)
+    return fn(ctypes.c_void_p(x), ctypes.c_void_p(q), ctypes.c_void_p(s),
+              ctypes.c_void_p(z) if z else None, M, N, K, c or cfg(), ctypes.c_void_p(y),
+              None, 0, None)
+
+
+@pytest.mark.parametrize("entry", ["awq_gemv", "awq_gemm"])
+def test_product_validation(L, entry):
+    assert _gemv(L, c=cfg(g=64), entry=entry) == UNSUP          # only g = 128 is built
+    assert _gemv(L, c=cfg(zp=2), entry=entry) == UNSUP
+    assert _gemv(L, K=200, entry=entry) == SHAPE                # K % 128 != 0
+    assert _gemv(L, K=0, entry=entry) == SHAPE
+    assert _gemv(L, N=-1, entry=entry) == SHAPE
+    assert _gemv(L, x=0, entry=entry) == NULL
+    assert _gemv(L, q=0, entry=entry) == NULL
+    assert _gemv(L, y=0, entry=entry) == NULL
+    assert _gemv(L, z=0, entry=entry) == NULL                   # asym needs zeros
+    assert _gemv(L, z=A, c=cfg(zp=0), entry=entry) == SHAPE     # sym takes no zeros
+    assert _gemv(L, x=MIS, entry=entry) == ALIGN
+    assert _gemv(L, y=MIS, entry=entry) == ALIGN
+    assert _gemv(L, N=0, entry=entry) == OK                     # empty: no work, no CUDA call
+
+
+def test_gemv_batch_range(L):
+    assert _gemv(L, M=0) == SHAPE
+    assert _gemv(L, M=17) == SHAPE
+    assert _gemv(L, M=0, entry="awq_gemm") == OK                # empty batch
+    assert _gemv(L, M=-3, entry="awq_gemm") == SHAPE
+
+
+def test_quantize_and_dequant_validation(L):
+    q = L.awq_pseudo_quantize_pack
+    P = ctypes.c_void_p
+    assert q(None, 8, 256, cfg(), P(A), P(A), P(A), None) == NULL
+    assert q(P(A), 8, 256, cfg(), P(A), P(A), None, None) == NULL
+    assert q(P(A), 8, 256, cfg(zp=0), P(A), P(A), P(A), None) == SHAPE
+    assert q(P(A), 8, 100, cfg(), P(A), P(A), P(A), None) == SHAPE
+    assert q(P(MIS), 8, 256, cfg(), P(A), P(A), P(A), None) == ALIGN
+    assert q(P(A), 0, 256, cfg(), P(A), P(A), P(A), None) == OK
+    d = L.awq_dequant
+    assert d(None, P(A), P(A), 8, 256, cfg(), P(A), None) == NULL
+    assert d(P(A), P(A), P(A), 8, 256, cfg(g=32), P(A), None) == UNSUP
+    assert d(P(A), P(A), P(A), 8, 256, cfg(), P(MIS), None) == ALIGN
+    assert d(P(A), P(A), P(A), 0, 256, cfg(), P(A), None) == OK
+
+
+def test_workspace_query_validation(L):
+    n = ctypes.c_size_t(7)
+    assert L.awq_workspace_bytes(1, 64, 256, cfg(), None) == NULL
+    assert L.awq_workspace_bytes(1, 64, 250, cfg(), ctypes.byref(n)) == SHAPE
+    assert L.awq_workspace_bytes(0, 64, 256, cfg(), ctypes.byref(n)) == OK and n.value == 0
+    assert L.awq_workspace_bytes(4, 0, 256, cfg(), ctypes.byref(n)) == OK and n.value == 0
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(1, 256, dtype=torch.float16)
+    with pytest.raises(ValueError, match="CUDA"):
+        awq.awq_gemv(x, torch.zeros(8, 32, dtype=torch.int32), torch.zeros(8, 2, dtype=torch.float16), None)

@@ -1,0 +1,102 @@
+"""GPU parity of awq_gemm (tcgen05 tensor-core path) against the float64 oracle.
+
+Small and ragged shapes are compared on every output; the prefill and 70B
+configurations at full size on sampled output channels (all rows of x)."""
+
+import numpy as np
+import pytest
+import torch
+
+import weight_only_int4_gemv_b200 as awq
+from oracle import awq_oracle as O
+from parity_util import (activations, assert_close, bits, dev, host, oracle_layer, sample_rows)
+from workloads import make_packed_random, make_weight
+
+pytestmark = pytest.mark.gpu
+
+
+def run_gemm(x, qweight, scales, zeros):
+    y = awq.awq_gemm(dev(x), dev(qweight), dev(scales), dev(zeros) if zeros is not None else None)
+    torch.cuda.synchronize()
+    return host(y)
+
+
+@pytest.fixture(autouse=True)
+def no_device_error():
+    yield
+    assert awq.awq_device_error() == 0, "a pipeline wait inside awq_gemm timed out"
+
+
+@pytest.mark.parametrize("zp", [True, False])
+@pytest.mark.parametrize("N,K,Ms", [
+    (512, 512, (1, 16, 17, 128, 129, 300)),
+    (256, 128, (128,)),                 # one tile, one k-block pair
+    (40, 256, (7, 200)),                # ragged N smaller than a tile
+    (1000, 1024, (128, 257)),           # ragged N and M
+    (4096, 4096, (128,)),
+])
+def test_gemm_full_compare(N, K, Ms, zp):
+    _, qweight, scales, zeros, Wd = oracle_layer(N, K, 0.02, 0.01, zp)
+    for M in Ms:
+        x = activations(M, K, seed=M)
+        y = run_gemm(x, qweight, scales, zeros)
+        assert_close(y, O.matmul_f64(x, Wd), f"N={N} K={K} M={M} zp={zp}")
+
+
+def test_gemm_odd_n_scalar_epilogue():
+    """N not a multiple of 8 takes the element-wise store path."""
+    qweight, scales, zeros = make_packed_random(301, 512, 128, True, seed=9)
+    Wd = O.dequant(O.unpack(qweight), scales, zeros, 128)
+    x = activations(130, 512, seed=2)
+    assert_close(run_gemm(x, qweight, scales, zeros), O.matmul_f64(x, Wd), "N=301")
+
+
+@pytest.mark.parametrize("N,K", [(4096, 4096), (14336, 4096)])
+def test_gemm_prefill_sampled(N, K):
+    """Prefill: M in {128, 512, 2048}; sampled output channels, every row of x."""
+    _, qweight, scales, zeros, Wd = oracle_layer(N, K, 0.02, 0.0, True)
+    cols = sample_rows(N, 384)
+    for M in (128, 512, 2048):
+        x = activations(M, K, seed=30 + M)
+        y = run_gemm(x, qweight, scales, zeros)
+        assert_close(y[:, cols], O.matmul_f64(x, Wd[cols]), f"N={N} K={K} M={M}")
+
+
+@pytest.mark.parametrize("N,K", [(8192, 8192), (28672, 8192), (8192, 28672)])
+def test_gemm_llama3_70b_sampled(N, K):
+    W = make_weight(N, K, 0.015, 0.01, seed=0)
+    qg, sg, zg = awq.awq_pseudo_quantize_pack(dev(W), zero_point=True)
+    cols = sample_rows(N, 256)
+    codes, scales, zeros = O.pseudo_quantize(W[cols], 128, True)
+    assert np.array_equal(bits(host(qg)[cols]), bits(O.pack(codes)))
+    Wd = O.dequant(codes, scales, zeros, 128)
+    x = activations(2048, K, seed=40)
+    y = host(awq.awq_gemm(dev(x), qg, sg, zg))
+    assert_close(y[:, cols], O.matmul_f64(x, Wd), f"N={N} K={K} M=2048")
+
+
+def test_gemm_matches_gemv_at_small_m():
+    _, qweight, scales, zeros, Wd = oracle_layer(4096, 4096, 0.02, 0.01, True)
+    for M in (1, 8, 16):
+        x = activations(M, 4096, seed=M)
+        ws = awq.alloc_workspace(M, 4096, 4096, True)
+        yv = host(awq.awq_gemv(dev(x), dev(qweight), dev(scales), dev(zeros), workspace=ws))
+        yg = run_gemm(x, qweight, scales, zeros)
+        ref = O.matmul_f64(x, Wd)
+        assert_close(yv, ref, f"gemv M={M}")
+        assert_close(yg, ref, f"gemm M={M}")
+
+
+def test_gemm_is_deterministic():
+    _, qweight, scales, zeros, _ = oracle_layer(1000, 1024, 0.02, 0.01, True)
+    x = activations(300, 1024, seed=1)
+    a = bits(run_gemm(x, qweight, scales, zeros))
+    b = bits(run_gemm(x, qweight, scales, zeros))
+    assert np.array_equal(a, b)
+
+
+def test_gemm_empty_batch():
+    _, qweight, scales, zeros, _ = oracle_layer(512, 512, 0.02, 0.01, True)
+    y = awq.awq_gemm(torch.empty((0, 512), dtype=torch.float16, device="cuda"), dev(qweight), dev(scales),
+                     dev(zeros))
+    assert y.shape == (0, 512)

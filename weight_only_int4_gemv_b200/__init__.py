@@ -1,0 +1,211 @@
+"""Python binding of libawq_b200: a W4A16 (group-wise INT4 weight, fp16
+activation) linear layer for NVIDIA B200.
+
+Every function marshals torch tensors into the C ABI declared in
+``include/awq.h`` and enqueues the library's CUDA kernels on the current
+torch stream. Nothing here computes: there is no CPU fallback, and using the
+binding without the built library or without a CUDA device raises.
+
+Layouts (row-major, K contiguous): W fp16 [N, K]; x fp16 [M, K]; y fp16
+[M, N]; qweight int32 [N, K/8] (eight 4-bit codes per word, nibble slot i of
+word w holds k = 8w + (0, 2, 4, 6, 1, 3, 5, 7)[i]); scales fp16 [N, K/128];
+zeros fp16 [N, K/128] holding integers 0..15 (None for the symmetric
+variant, whose zero point is 8).
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+__all__ = [
+    "LIB_PATH", "AwqError", "lib", "GROUP_SIZE",
+    "awq_pseudo_quantize_pack", "awq_dequant", "awq_workspace_bytes",
+    "awq_gemv", "awq_gemm", "awq_device_error", "awq_linear", "GEMV_MAX_M",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libawq_b200.so")
+GROUP_SIZE = 128
+GEMV_MAX_M = 16
+
+AWQ_OK = 0
+STATUS_NAMES = {0: "AWQ_OK", 1: "AWQ_ERR_NULL", 2: "AWQ_ERR_SHAPE", 3: "AWQ_ERR_ALIGN",
+                4: "AWQ_ERR_UNSUPPORTED", 5: "AWQ_ERR_CUDA", 6: "AWQ_ERR_WORKSPACE"}
+
+
+class AwqError(RuntimeError):
+    def __init__(self, fn: str, status: int, text: str):
+        super().__init__(f"{fn}: {STATUS_NAMES.get(status, status)} ({text})")
+        self.status = status
+
+
+class QConfig(ctypes.Structure):
+    _fields_ = [("group_size", ctypes.c_int32), ("zero_point", ctypes.c_int32)]
+
+
+_lib = None
+_lock = threading.Lock()
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_SIGS = {
+    "awq_abi_version": (ctypes.c_int, []),
+    "awq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "awq_pseudo_quantize_pack": (ctypes.c_int, [_P, _I64, _I64, QConfig, _P, _P, _P, _P]),
+    "awq_dequant": (ctypes.c_int, [_P, _P, _P, _I64, _I64, QConfig, _P, _P]),
+    "awq_workspace_bytes": (ctypes.c_int, [_I64, _I64, _I64, QConfig, ctypes.POINTER(ctypes.c_size_t)]),
+    "awq_gemv": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, QConfig, _P, _P, ctypes.c_size_t, _P]),
+    "awq_gemm": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, QConfig, _P, _P, ctypes.c_size_t, _P]),
+    "awq_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), _P]),
+}
+
+
+def lib():
+    """The loaded shared library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        with _lock:
+            if _lib is None:
+                if not os.path.exists(LIB_PATH):
+                    raise RuntimeError(
+                        f"{LIB_PATH} is missing: build it with "
+                        "`python -m weight_only_int4_gemv_b200.build` (there is no fallback)")
+                h = ctypes.CDLL(LIB_PATH)
+                for name, (res, args) in _SIGS.items():
+                    f = getattr(h, name)
+                    f.restype = res
+                    f.argtypes = args
+                _lib = h
+    return _lib
+
+
+def _check(fn: str, st: int):
+    if st != AWQ_OK:
+        raise AwqError(fn, st, lib().awq_status_string(st).decode())
+
+
+def _cfg(zero_point: bool, group_size: int) -> QConfig:
+    return QConfig(group_size, 1 if zero_point else 0)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (no CPU path exists)")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {ndim}-d tensor")
+
+
+def awq_pseudo_quantize_pack(W: torch.Tensor, zero_point: bool = True, group_size: int = GROUP_SIZE):
+    """Quantize fp16 W[N, K] and pack it: returns (qweight, scales, zeros or None)."""
+    _need(W, "W", torch.float16, 2)
+    N, K = W.shape
+    G = K // group_size if group_size > 0 else 0
+    qweight = torch.empty((N, K // 8), dtype=torch.int32, device=W.device)
+    scales = torch.empty((N, G), dtype=torch.float16, device=W.device)
+    zeros = torch.empty((N, G), dtype=torch.float16, device=W.device) if zero_point else None
+    with torch.cuda.device(W.device):
+        _check("awq_pseudo_quantize_pack", lib().awq_pseudo_quantize_pack(
+            _ptr(W), N, K, _cfg(zero_point, group_size), _ptr(qweight), _ptr(scales), _ptr(zeros),
+            _stream(W.device)))
+    return qweight, scales, zeros
+
+
+def awq_dequant(qweight: torch.Tensor, scales: torch.Tensor, zeros, group_size: int = GROUP_SIZE,
+                out: torch.Tensor | None = None) -> torch.Tensor:
+    """Decode packed weights to fp16 W'[N, K] (bit-exact)."""
+    _need(qweight, "qweight", torch.int32, 2)
+    _need(scales, "scales", torch.float16, 2)
+    if zeros is not None:
+        _need(zeros, "zeros", torch.float16, 2)
+    N, K = qweight.shape[0], qweight.shape[1] * 8
+    if out is None:
+        out = torch.empty((N, K), dtype=torch.float16, device=qweight.device)
+    _need(out, "out", torch.float16, 2)
+    with torch.cuda.device(qweight.device):
+        _check("awq_dequant", lib().awq_dequant(
+            _ptr(qweight), _ptr(scales), _ptr(zeros), N, K, _cfg(zeros is not None, group_size),
+            _ptr(out), _stream(qweight.device)))
+    return out
+
+
+def awq_workspace_bytes(M: int, N: int, K: int, zero_point: bool = True, group_size: int = GROUP_SIZE,
+                        device=None) -> int:
+    """Workspace bytes awq_gemv / awq_gemm need on `device` for this shape."""
+    n = ctypes.c_size_t(0)
+    with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
+        _check("awq_workspace_bytes", lib().awq_workspace_bytes(M, N, K, _cfg(zero_point, group_size),
+                                                                ctypes.byref(n)))
+    return int(n.value)
+
+
+def alloc_workspace(M: int, N: int, K: int, zero_point: bool = True, device=None) -> torch.Tensor | None:
+    """Zero-filled workspace for (M, N, K), or None when none is needed."""
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    nbytes = awq_workspace_bytes(M, N, K, zero_point, device=dev)
+    return torch.zeros(nbytes, dtype=torch.uint8, device=dev) if nbytes else None
+
+
+def _product(entry: str, x, qweight, scales, zeros, workspace, out, group_size):
+    _need(x, "x", torch.float16, 2)
+    _need(qweight, "qweight", torch.int32, 2)
+    _need(scales, "scales", torch.float16, 2)
+    if zeros is not None:
+        _need(zeros, "zeros", torch.float16, 2)
+    M, K = x.shape
+    N = qweight.shape[0]
+    if qweight.shape[1] * 8 != K:
+        raise ValueError("qweight must be [N, K/8] for x [M, K]")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float16, device=x.device)
+    _need(out, "out", torch.float16, 2)
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        if not workspace.is_cuda or not workspace.is_contiguous():
+            raise ValueError("workspace must be a contiguous CUDA tensor")
+        ws_ptr, ws_bytes = _ptr(workspace), workspace.numel() * workspace.element_size()
+    with torch.cuda.device(x.device):
+        fn = getattr(lib(), entry)
+        _check(entry, fn(_ptr(x), _ptr(qweight), _ptr(scales), _ptr(zeros), M, N, K,
+                         _cfg(zeros is not None, group_size), _ptr(out), ws_ptr, ws_bytes,
+                         _stream(x.device)))
+    return out
+
+
+def awq_gemv(x, qweight, scales, zeros, workspace=None, out=None, group_size: int = GROUP_SIZE):
+    """y = x . W'^T for 1 <= M <= 16 (decode). `workspace` from alloc_workspace()."""
+    return _product("awq_gemv", x, qweight, scales, zeros, workspace, out, group_size)
+
+
+def awq_gemm(x, qweight, scales, zeros, workspace=None, out=None, group_size: int = GROUP_SIZE):
+    """y = x . W'^T for any M (prefill), on the tcgen05 tensor cores."""
+    return _product("awq_gemm", x, qweight, scales, zeros, workspace, out, group_size)
+
+
+def awq_linear(x, qweight, scales, zeros, workspace=None, out=None, group_size: int = GROUP_SIZE):
+    """The layer with the documented M threshold: awq_gemv for M <= 16, else awq_gemm."""
+    entry = "awq_gemv" if x.shape[0] <= GEMV_MAX_M else "awq_gemm"
+    return _product(entry, x, qweight, scales, zeros, workspace, out, group_size)
+
+
+def awq_device_error(device=None) -> int:
+    """Read and clear the device error word (bit 0: a bounded wait in awq_gemm gave up)."""
+    v = ctypes.c_uint32(0)
+    dev = device if device is not None else torch.cuda.current_device()
+    with torch.cuda.device(dev):
+        _check("awq_device_error", lib().awq_device_error(ctypes.byref(v), _stream(dev)))
+    return int(v.value)

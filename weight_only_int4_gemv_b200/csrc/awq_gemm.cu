@@ -1,0 +1,541 @@
+// W4A16 prefill product y[M][N] = x[M][K] . W'^T on the sm_100a tensor cores.
+//
+// ("AutoAWQ" code tour, "The big picture": WQLinear_GEMM serves batched
+// requests; "AutoAWQ" capability page: the weights stay INT4 in memory and
+// are decoded inside the fused matmul.)
+//
+// For M beyond a few tens the layer is a dense contraction, so W' tiles are
+// decoded into shared memory and multiplied by tcgen05.mma with fp32
+// accumulators in tensor memory. One persistent CTA per SM walks output tiles
+// of 128 (rows of x) x 256 (output channels); K advances in blocks of 64.
+//
+// Warp roles (448 threads):
+//   warps 0-7   decode: thread i owns row i of the 256-row weight tile; it
+//               reads the row's 32 code bytes of the k block from shared
+//               memory, decodes w' = (q - z) * s exactly as awq_dequant does
+//               (HSUB2 gives q - z exactly, HMUL2 rounds the product once),
+//               and writes 128 bytes in the 128-byte-swizzled K-major layout
+//               the tensor core reads.
+//   warps 8-11  epilogue: tcgen05.ld of the fp32 accumulator (lane = row of
+//               x), fp16 conversion, stores to y.
+//   warp 12     TMA: x tile (128 x 64 fp16, 128B swizzle) and code tile
+//               (256 rows x 32 bytes, 32B swizzle) per k block.
+//   warp 13     MMA: one thread issues 4 x tcgen05.mma (M=128, N=256, K=16)
+//               per k block, commits stage release and accumulator-ready
+//               barriers. Warp 13 also allocates and frees tensor memory.
+// Pipelines: 4 shared-memory stages (x + codes in, decoded W' out) and two
+// 256-column accumulators, so the epilogue of one tile overlaps the main
+// loop of the next.
+//
+// Every mbarrier wait is bounded by a wall-clock limit. When a wait runs
+// out, the CTA records bit 0 in the device error word, every role leaves its
+// loop, in-flight copies and MMAs are waited for (again bounded), and tensor
+// memory is freed before the kernel returns.
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "awq_common.cuh"
+
+namespace awq {
+
+__device__ uint32_t g_awq_error_word = 0;
+
+namespace {
+
+constexpr int BM = 128;                 // rows of x per tile (MMA M)
+constexpr int BN = 256;                 // output channels per tile (MMA N)
+constexpr int BK = 64;                  // k per stage (one 128-byte swizzle row of fp16)
+constexpr int kStages = 4;
+constexpr int kDecodeWarps = BN / 32;   // 8
+constexpr int kEpiWarp0 = kDecodeWarps; // 8..11
+constexpr int kTmaWarp = kEpiWarp0 + 4; // 12
+constexpr int kMmaWarp = kTmaWarp + 1;  // 13
+constexpr int kGemmThreads = (kMmaWarp + 1) * 32;
+constexpr int kTmemCols = 2 * BN;       // two accumulators
+
+constexpr int kABytes = BM * BK * 2;        // 16 KB
+constexpr int kBBytes = BN * BK * 2;        // 32 KB
+constexpr int kCBytes = BN * (BK / 8) * 4;  // 8 KB of packed codes
+constexpr int kSmemTiles = kStages * (kABytes + kBBytes + kCBytes);
+constexpr int kSmemBytes = kSmemTiles + 1024 /*barriers*/ + 1024 /*alignment*/;
+
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s per wait
+
+// instruction descriptor: F16 x F16 -> F32, both K-major, M = 128, N = 256
+constexpr uint32_t kIdesc = (1u << 4) | (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
+
+struct SmemLayout {
+  // offsets from the 1024-aligned base
+  static constexpr int a(int s) { return s * kABytes; }
+  static constexpr int b(int s) { return kStages * kABytes + s * kBBytes; }
+  static constexpr int c(int s) { return kStages * (kABytes + kBBytes) + s * kCBytes; }
+  static constexpr int bar = kSmemTiles;
+};
+
+struct Bars {
+  uint64_t full_a[kStages];    // TMA bytes of x + codes landed
+  uint64_t full_b[kStages];    // decoded W' tile written (8 warp arrivals)
+  uint64_t empty[kStages];     // MMAs that read the stage finished
+  uint64_t tmem_full[2];       // accumulator complete
+  uint64_t tmem_empty[2];      // accumulator drained (4 warp arrivals)
+  uint64_t mma_done;           // final commit before teardown
+  uint32_t tmem_base;
+  int abort;
+};
+
+// ---------------------------------------------------------------------------
+// PTX wrappers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t now_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for the phase of `parity` to complete. Returns false when the CTA is
+// aborting or the wait ran past its limit (which starts the abort).
+__device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = now_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 63) == 0) {
+      if (*abort) return false;
+      if (now_ns() - t0 > kWaitLimitNs) {
+        *abort = 1;
+        atomicOr(&g_awq_error_word, 1u);
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 32 lanes x 32 consecutive fp32 columns
+__device__ __forceinline__ void tc_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart (stride byte offset), sm100 descriptor version 1.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  return uint64_t((saddr >> 4) & 0x3FFF) | (uint64_t(1) << 16) | (uint64_t(1024 >> 4) << 32) |
+         (uint64_t(1) << 46) | (uint64_t(2) << 61);
+}
+
+struct GemmParams {
+  uint16_t* y;
+  const uint16_t* scales;
+  const uint16_t* zeros;
+  int M, N, K, G;
+  int m_tiles, n_tiles, k_blocks;
+};
+
+template <bool ZP>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_q,
+            const GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  Bars* bars = reinterpret_cast<Bars*>(smem + SmemLayout::bar);
+  volatile int* abort = &bars->abort;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int num_tiles = p.m_tiles * p.n_tiles;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bars->full_a[s], 1);
+      mbar_init(&bars->full_b[s], kDecodeWarps);
+      mbar_init(&bars->empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&bars->tmem_full[a], 1);
+      mbar_init(&bars->tmem_empty[a], 4);
+    }
+    mbar_init(&bars->mma_done, 1);
+    bars->abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    fence_proxy_async_smem();
+  }
+  if (warp == kMmaWarp) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&bars->tmem_base)),
+                 "r"(kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = bars->tmem_base;
+
+  if (warp < kDecodeWarps) {
+    // ------------------------------------------------------------ decode
+    const int i = threadIdx.x;  // row of the weight tile
+    int s = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      const int n0 = (tile / p.m_tiles) * BN;
+      const int64_t row = int64_t(n0) + i;
+      const bool valid = row < p.N;
+      const uint16_t* srow = p.scales + (valid ? row : 0) * p.G;
+      const uint16_t* zrow = ZP ? p.zeros + (valid ? row : 0) * p.G : nullptr;
+      uint32_t zb1024 = 0, zb64 = 0, sc2 = 0;
+      // scale and zero of group 0, then always one group ahead
+      uint16_t s_next = valid ? ld_nc_u16(srow) : uint16_t(0);
+      uint16_t z_next = (ZP && valid) ? ld_nc_u16(zrow) : uint16_t(0);
+      for (int kb = 0; kb < p.k_blocks; ++kb) {
+        if ((kb & 1) == 0) {  // new group of 128 k
+          const uint16_t sb = s_next;
+          const float z = ZP ? half_bits_to_float(z_next) : 8.0f;
+          const int gn = (kb >> 1) + 1;
+          if (valid && gn < p.G) {
+            s_next = ld_nc_u16(srow + gn);
+            if (ZP) z_next = ld_nc_u16(zrow + gn);
+          }
+          zero_bias_pairs(z, zb1024, zb64);
+          sc2 = uint32_t(sb) | (uint32_t(sb) << 16);
+        }
+        if (!wait_bounded(&bars->full_a[s], ph, abort)) { ok = false; break; }
+        // codes of row i: 32 bytes, 16-byte halves swapped on rows with bit 2 set (32B swizzle)
+        const uint8_t* crow = smem + SmemLayout::c(s) + i * 32;
+        const int sw = (i >> 2) & 1;
+        const uint4 c0 = *reinterpret_cast<const uint4*>(crow + (sw << 4));
+        const uint4 c1 = *reinterpret_cast<const uint4*>(crow + ((sw ^ 1) << 4));
+        uint8_t* brow = smem + SmemLayout::b(s) + i * 128;
+        const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+          uint32_t pq[4];
+          decode_word_qz(words[w], zb1024, zb64, pq);
+          uint4 v;
+          v.x = hmul2_u32(pq[0], sc2);
+          v.y = hmul2_u32(pq[1], sc2);
+          v.z = hmul2_u32(pq[2], sc2);
+          v.w = hmul2_u32(pq[3], sc2);
+          *reinterpret_cast<uint4*>(brow + ((w ^ (i & 7)) << 4)) = v;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->full_b[s]);
+        if (++s == kStages) { s = 0; ph ^= 1; }
+      }
+    }
+  } else if (warp < kEpiWarp0 + 4) {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp - kEpiWarp0;            // TMEM lane quadrant (warp % 4)
+    int it = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+      const int m0 = (tile % p.m_tiles) * BM;
+      const int n0 = (tile / p.m_tiles) * BN;
+      const int acc = it & 1;
+      const uint32_t aph = (it >> 1) & 1;
+      if (!wait_bounded(&bars->tmem_full[acc], aph, abort)) break;
+      tc_fence_after();
+      const int64_t m = int64_t(m0) + q * 32 + lane;
+      uint16_t* yrow = p.y + m * p.N;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        tc_ld_32x32b_x32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * BN + c * 32), r);
+        const int nc = n0 + c * 32;
+        if (m < p.M && nc < p.N) {
+          uint32_t h[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const uint32_t lo = __half_as_ushort(__float2half_rn(__uint_as_float(r[2 * e])));
+            const uint32_t hi = __half_as_ushort(__float2half_rn(__uint_as_float(r[2 * e + 1])));
+            h[e] = lo | (hi << 16);
+          }
+          if (nc + 32 <= p.N && (p.N & 7) == 0) {
+            uint4* dst = reinterpret_cast<uint4*>(yrow + nc);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) dst[v] = make_uint4(h[4 * v], h[4 * v + 1], h[4 * v + 2], h[4 * v + 3]);
+          } else {
+            for (int e = 0; e < 32 && nc + e < p.N; ++e)
+              yrow[nc + e] = uint16_t((h[e >> 1] >> ((e & 1) * 16)) & 0xFFFF);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->tmem_empty[acc]);
+    }
+  } else if (warp == kTmaWarp) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      bool issued[kStages] = {};
+      uint32_t issued_ph[kStages] = {};
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const int m0 = (tile % p.m_tiles) * BM;
+        const int n0 = (tile / p.m_tiles) * BN;
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          if (!wait_bounded(&bars->empty[s], ph ^ 1, abort)) { ok = false; break; }
+          mbar_arrive_expect_tx(&bars->full_a[s], kABytes + kCBytes);
+          tma_load_2d(smem + SmemLayout::a(s), &tmap_x, kb * BK, m0, &bars->full_a[s]);
+          tma_load_2d(smem + SmemLayout::c(s), &tmap_q, kb * (BK / 8), n0, &bars->full_a[s]);
+          issued[s] = true;
+          issued_ph[s] = ph;
+          if (++s == kStages) { s = 0; ph ^= 1; }
+        }
+      }
+      // The copies still in flight land before the CTA's shared memory goes away.
+      for (int t = 0; t < kStages; ++t)
+        if (issued[t]) {
+          const uint64_t t0 = now_ns();
+          while (!mbar_try_wait(&bars->full_a[t], issued_ph[t]) && now_ns() - t0 < kWaitLimitNs) {}
+        }
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
+        const int acc = it & 1;
+        const uint32_t aph = (it >> 1) & 1;
+        if (!wait_bounded(&bars->tmem_empty[acc], aph ^ 1, abort)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + uint32_t(acc * BN);
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          if (!wait_bounded(&bars->full_a[s], ph, abort) ||
+              !wait_bounded(&bars->full_b[s], ph, abort)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + SmemLayout::a(s));
+          const uint32_t b_addr = smem_u32(smem + SmemLayout::b(s));
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)
+            tc_mma_f16(d_tmem, sw128_desc(a_addr + k * 32), sw128_desc(b_addr + k * 32), kIdesc,
+                       (kb | k) != 0);
+          tc_commit(&bars->empty[s]);
+          if (++s == kStages) { s = 0; ph ^= 1; }
+        }
+        if (ok) tc_commit(&bars->tmem_full[acc]);
+      }
+      // every MMA this thread issued completes before tensor memory is freed
+      tc_commit(&bars->mma_done);
+      const uint64_t t0 = now_ns();
+      while (!mbar_try_wait(&bars->mma_done, 0) && now_ns() - t0 < kWaitLimitNs) {}
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(kTmemCols));
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode;
+}
+
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_sms[kMaxDevices];
+std::atomic<int> g_attr_set[kMaxDevices][2];
+
+}  // namespace
+
+awq_status_t gemm_workspace_bytes(int64_t, int64_t, int64_t, bool, size_t* bytes) {
+  *bytes = 0;
+  return AWQ_OK;
+}
+
+}  // namespace awq
+
+using namespace awq;
+
+extern "C" awq_status_t awq_gemm(const uint16_t* x, const int32_t* qweight,
+                                 const uint16_t* scales, const uint16_t* zeros, int64_t M,
+                                 int64_t N, int64_t K, awq_qconfig_t cfg, uint16_t* y,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  awq_status_t st = check_cfg(cfg);
+  if (st != AWQ_OK) return st;
+  if ((st = check_nk(N, K)) != AWQ_OK) return st;
+  if (M < 0 || M > (int64_t(1) << 31) - 1) return AWQ_ERR_SHAPE;
+  if (M == 0 || N == 0) return AWQ_OK;
+  if (!x || !qweight || !scales || !y) return AWQ_ERR_NULL;
+  if (cfg.zero_point && !zeros) return AWQ_ERR_NULL;
+  if (!cfg.zero_point && zeros) return AWQ_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(qweight) || !aligned16(scales) || !aligned16(y) ||
+      (zeros && !aligned16(zeros)))
+    return AWQ_ERR_ALIGN;
+
+  PFN_cuTensorMapEncodeTiled_v12000 encode = get_encode();
+  if (!encode) return AWQ_ERR_CUDA;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return AWQ_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return AWQ_ERR_UNSUPPORTED;
+  int sms = g_sms[dev].load(std::memory_order_relaxed);
+  if (sms == 0) {
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return AWQ_ERR_CUDA;
+    g_sms[dev].store(sms, std::memory_order_relaxed);
+  }
+  auto kernel = cfg.zero_point ? gemm_kernel<true> : gemm_kernel<false>;
+  const int zi = cfg.zero_point ? 1 : 0;
+  if (!g_attr_set[dev][zi].load(std::memory_order_acquire)) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
+        cudaSuccess)
+      return AWQ_ERR_CUDA;
+    g_attr_set[dev][zi].store(1, std::memory_order_release);
+  }
+
+  // x: fp16 [M][K], box 64 (k) x 128 (rows), 128-byte swizzle; rows past M read as 0.
+  CUtensorMap tmap_x, tmap_q;
+  {
+    const cuuint64_t dims[2] = {cuuint64_t(K), cuuint64_t(M)};
+    const cuuint64_t strides[1] = {cuuint64_t(K) * 2};
+    const cuuint32_t box[2] = {BK, BM};
+    const cuuint32_t estr[2] = {1, 1};
+    if (encode(&tmap_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<uint16_t*>(x), dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return AWQ_ERR_CUDA;
+  }
+  // codes: int32 [N][K/8], box 8 words x 256 rows, 32-byte swizzle; rows past N read as 0.
+  {
+    const cuuint64_t dims[2] = {cuuint64_t(K / 8), cuuint64_t(N)};
+    const cuuint64_t strides[1] = {cuuint64_t(K / 8) * 4};
+    const cuuint32_t box[2] = {BK / 8, BN};
+    const cuuint32_t estr[2] = {1, 1};
+    if (encode(&tmap_q, CU_TENSOR_MAP_DATA_TYPE_INT32, 2, const_cast<int32_t*>(qweight), dims,
+               strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return AWQ_ERR_CUDA;
+  }
+  GemmParams p;
+  p.y = y;
+  p.scales = scales;
+  p.zeros = zeros;
+  p.M = int(M);
+  p.N = int(N);
+  p.K = int(K);
+  p.G = int(K / kGroup);
+  p.m_tiles = int((M + BM - 1) / BM);
+  p.n_tiles = int((N + BN - 1) / BN);
+  p.k_blocks = int(K / BK);
+  const int64_t tiles = int64_t(p.m_tiles) * p.n_tiles;
+  if (tiles > (int64_t(1) << 31) - 1) return AWQ_ERR_SHAPE;
+  const int grid = int(tiles < sms ? tiles : sms);
+  kernel<<<grid, kGemmThreads, kSmemBytes, static_cast<cudaStream_t>(stream)>>>(tmap_x, tmap_q, p);
+  return launch_status();
+}
+
+extern "C" awq_status_t awq_device_error(uint32_t* error_word, void* stream) {
+  if (!error_word) return AWQ_ERR_NULL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t zero = 0;
+  if (cudaMemcpyFromSymbolAsync(error_word, g_awq_error_word, sizeof(uint32_t), 0,
+                                cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return AWQ_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return AWQ_ERR_CUDA;
+  if (cudaMemcpyToSymbolAsync(g_awq_error_word, &zero, sizeof(uint32_t), 0, cudaMemcpyHostToDevice,
+                              s) != cudaSuccess)
+    return AWQ_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return AWQ_ERR_CUDA;
+  return AWQ_OK;
+}

@@ -1,0 +1,180 @@
+// Group-wise INT4 quantize + pack, and dequant, for sm_100a.
+//
+// Quantization rule ("AutoAWQ" code tour, "The Quantization Flow Up Close":
+// each group of weights is rounded to integer levels against its scale and
+// zero point; symmetric decode from "AWQ Quantization Support", section
+// "Dequantization Formula"): per (row n, group j), IEEE fp32 arithmetic with
+// round to nearest even,
+//   asymmetric: s = fp16(max((max - min) / 15, 1e-5)), z = clamp(-rint(min / s), 0, 15),
+//               q = clamp(rint(w / s) + z, 0, 15)
+//   symmetric:  s = fp16(max(max|w| / 7, 1e-5)),        q = clamp(rint(w / s), -8, 7) + 8
+// The explicit _rn intrinsics keep every operation a single IEEE rounding,
+// so the codes are bit-exact whatever contraction flags the file is built with.
+
+#include "awq_common.cuh"
+
+namespace awq {
+namespace {
+
+constexpr int kQuantThreads = 256;
+
+// One warp per (row, group) unit. Lane l holds k = 4l .. 4l+3 of the group:
+// a coalesced 256-byte read per warp, min/max by butterfly shuffles, and
+// the packed word of k = 8w .. 8w+7 assembled from lanes 2w and 2w+1.
+template <bool ZP>
+__global__ void __launch_bounds__(kQuantThreads)
+quantize_pack_kernel(const uint16_t* __restrict__ W, int64_t N, int64_t K,
+                     int32_t* __restrict__ qweight, uint16_t* __restrict__ scales,
+                     uint16_t* __restrict__ zeros) {
+  const int lane = threadIdx.x & 31;
+  const int64_t G = K / kGroup;
+  const int64_t units = N * G;
+  const int64_t nwarps = (int64_t(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t u = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; u < units; u += nwarps) {
+    const int64_t n = u / G;
+    const int64_t j = u - n * G;
+    const uint2 raw = *reinterpret_cast<const uint2*>(W + n * K + j * kGroup + lane * 4);
+    float w[4];
+    w[0] = half_bits_to_float(uint16_t(raw.x & 0xFFFF));
+    w[1] = half_bits_to_float(uint16_t(raw.x >> 16));
+    w[2] = half_bits_to_float(uint16_t(raw.y & 0xFFFF));
+    w[3] = half_bits_to_float(uint16_t(raw.y >> 16));
+
+    int q[4];
+    float sf;
+    float zf = 0.0f;
+    if (ZP) {
+      float mx = fmaxf(fmaxf(w[0], w[1]), fmaxf(w[2], w[3]));
+      float mn = fminf(fminf(w[0], w[1]), fminf(w[2], w[3]));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+      }
+      const float s32 = fmaxf(__fdiv_rn(__fsub_rn(mx, mn), 15.0f), 1e-5f);
+      sf = __half2float(__float2half_rn(s32));
+      zf = fminf(fmaxf(-rintf(__fdiv_rn(mn, sf)), 0.0f), 15.0f);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        q[i] = int(fminf(fmaxf(__fadd_rn(rintf(__fdiv_rn(w[i], sf)), zf), 0.0f), 15.0f));
+    } else {
+      float a = fmaxf(fmaxf(fabsf(w[0]), fabsf(w[1])), fmaxf(fabsf(w[2]), fabsf(w[3])));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+      const float s32 = fmaxf(__fdiv_rn(a, 7.0f), 1e-5f);
+      sf = __half2float(__float2half_rn(s32));
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        q[i] = int(fminf(fmaxf(rintf(__fdiv_rn(w[i], sf)), -8.0f), 7.0f)) + 8;
+    }
+
+    // k offset o of the word goes to slot (o even ? o/2 : 4 + o/2).
+    // Even lane: offsets 0..3 -> slots 0,4,1,5; odd lane: offsets 4..7 -> slots 2,6,3,7.
+    uint32_t part;
+    if ((lane & 1) == 0)
+      part = uint32_t(q[0]) | (uint32_t(q[1]) << 16) | (uint32_t(q[2]) << 4) | (uint32_t(q[3]) << 20);
+    else
+      part = (uint32_t(q[0]) << 8) | (uint32_t(q[1]) << 24) | (uint32_t(q[2]) << 12) |
+             (uint32_t(q[3]) << 28);
+    const uint32_t other = __shfl_xor_sync(0xffffffffu, part, 1);
+    if ((lane & 1) == 0)
+      qweight[n * (K / 8) + j * kWordsPerGroup + (lane >> 1)] = int32_t(part | other);
+    if (lane == 0) {
+      scales[n * G + j] = __half_as_ushort(__float2half_rn(sf));
+      if (ZP) zeros[n * G + j] = __half_as_ushort(__int2half_rn(int(zf)));
+    }
+  }
+}
+
+// One thread per packed word: eight fp16 outputs written as one 16-byte store.
+// w' = fp16((q - z) * s): the fp32 product is exact, so one rounding.
+template <bool ZP>
+__global__ void __launch_bounds__(256)
+dequant_kernel(const int32_t* __restrict__ qweight, const uint16_t* __restrict__ scales,
+               const uint16_t* __restrict__ zeros, int64_t N, int64_t K,
+               uint16_t* __restrict__ out) {
+  const int64_t wpr = K / 8;
+  const int64_t G = K / kGroup;
+  const int64_t words = N * wpr;
+  const int64_t stride = int64_t(gridDim.x) * blockDim.x;
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < words; i += stride) {
+    const int64_t n = i / wpr;
+    const int64_t wi = i - n * wpr;
+    const int64_t g = n * G + (wi * 8) / kGroup;
+    const float sf = half_bits_to_float(scales[g]);
+    const float zf = ZP ? half_bits_to_float(zeros[g]) : 8.0f;
+    const uint32_t word = uint32_t(qweight[i]);
+    uint32_t h[8];
+#pragma unroll
+    for (int o = 0; o < 8; ++o) {
+      const int slot = (o & 1) ? 4 + (o >> 1) : (o >> 1);
+      const float q = float((word >> (4 * slot)) & 0xFu);
+      h[o] = __half_as_ushort(__float2half_rn(__fmul_rn(__fsub_rn(q, zf), sf)));
+    }
+    uint4 v;
+    v.x = h[0] | (h[1] << 16);
+    v.y = h[2] | (h[3] << 16);
+    v.z = h[4] | (h[5] << 16);
+    v.w = h[6] | (h[7] << 16);
+    *reinterpret_cast<uint4*>(out + i * 8) = v;
+  }
+}
+
+int grid_for(int64_t work_items, int threads_per_item, int threads_per_block) {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t want = (work_items * threads_per_item + threads_per_block - 1) / threads_per_block;
+  const int64_t cap = int64_t(sms) * 8;
+  return int(want < cap ? (want > 0 ? want : 1) : cap);
+}
+
+}  // namespace
+}  // namespace awq
+
+using namespace awq;
+
+extern "C" awq_status_t awq_pseudo_quantize_pack(const uint16_t* W, int64_t N, int64_t K,
+                                                 awq_qconfig_t cfg, int32_t* qweight,
+                                                 uint16_t* scales, uint16_t* zeros,
+                                                 void* stream) {
+  awq_status_t st = check_cfg(cfg);
+  if (st != AWQ_OK) return st;
+  if ((st = check_nk(N, K)) != AWQ_OK) return st;
+  if (N == 0) return AWQ_OK;
+  if (!W || !qweight || !scales) return AWQ_ERR_NULL;
+  if (cfg.zero_point && !zeros) return AWQ_ERR_NULL;
+  if (!cfg.zero_point && zeros) return AWQ_ERR_SHAPE;
+  if (!aligned16(W) || !aligned16(qweight) || !aligned16(scales) || (zeros && !aligned16(zeros)))
+    return AWQ_ERR_ALIGN;
+  const int64_t units = N * (K / kGroup);
+  const int grid = grid_for(units, 32, kQuantThreads);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cfg.zero_point)
+    quantize_pack_kernel<true><<<grid, kQuantThreads, 0, s>>>(W, N, K, qweight, scales, zeros);
+  else
+    quantize_pack_kernel<false><<<grid, kQuantThreads, 0, s>>>(W, N, K, qweight, scales, nullptr);
+  return launch_status();
+}
+
+extern "C" awq_status_t awq_dequant(const int32_t* qweight, const uint16_t* scales,
+                                    const uint16_t* zeros, int64_t N, int64_t K,
+                                    awq_qconfig_t cfg, uint16_t* W_out, void* stream) {
+  awq_status_t st = check_cfg(cfg);
+  if (st != AWQ_OK) return st;
+  if ((st = check_nk(N, K)) != AWQ_OK) return st;
+  if (N == 0) return AWQ_OK;
+  if (!qweight || !scales || !W_out) return AWQ_ERR_NULL;
+  if (cfg.zero_point && !zeros) return AWQ_ERR_NULL;
+  if (!cfg.zero_point && zeros) return AWQ_ERR_SHAPE;
+  if (!aligned16(qweight) || !aligned16(scales) || !aligned16(W_out) || (zeros && !aligned16(zeros)))
+    return AWQ_ERR_ALIGN;
+  const int64_t words = N * (K / 8);
+  const int grid = grid_for(words, 1, 256);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cfg.zero_point)
+    dequant_kernel<true><<<grid, 256, 0, s>>>(qweight, scales, zeros, N, K, W_out);
+  else
+    dequant_kernel<false><<<grid, 256, 0, s>>>(qweight, scales, nullptr, N, K, W_out);
+  return launch_status();
+}
