@@ -36,6 +36,9 @@ Readings where the pages are silent (each is listed in the design doc):
 * Symmetric scale = max|w| / 7 (largest positive level 7); codes are
   clamp(rint(w/s), -8, 7) + 8.
 * Zero points are stored as fp16 values holding the integers 0..15.
+* Scales and zero points are stored group-major, [K/g, N] (entry [j, n] is
+  the group of k in [128j, 128j + 128) of output channel n), the orientation
+  AutoAWQ's checkpoints use for ``scales``.
 * Packing is along K, eight consecutive k per int32 word; nibble slot i
   (bits 4i..4i+3) of the word covering k = 8w..8w+7 holds k = 8w + SLOT_K[i]
   with SLOT_K = (0, 2, 4, 6, 1, 3, 5, 7).
@@ -82,7 +85,7 @@ def quantize_asym(W: np.ndarray, group_size: int = GROUP_SIZE):
       4. z = clamp(-rint(mn / sf), 0, 15)
       5. q = clamp(rint(w / sf) + z, 0, 15)
 
-    Returns (codes uint8 [N, K], scales fp16 [N, G], zeros fp16 [N, G]).
+    Returns (codes uint8 [N, K], scales fp16 [G, N], zeros fp16 [G, N]).
     """
     w = _groups_f32(W, group_size)
     mx = w.max(axis=2)
@@ -95,7 +98,8 @@ def quantize_asym(W: np.ndarray, group_size: int = GROUP_SIZE):
     codes = q.astype(np.uint8).reshape(W.shape)
     # z is an integer level; storing it through an integer keeps 0 as +0
     # (-rint of a non-negative minimum is -0.0 in floating point).
-    return codes, scales, z.astype(np.int32).astype(np.float16)
+    zeros = z.astype(np.int32).astype(np.float16)
+    return codes, np.ascontiguousarray(scales.T), np.ascontiguousarray(zeros.T)
 
 
 def quantize_sym(W: np.ndarray, group_size: int = GROUP_SIZE):
@@ -114,7 +118,7 @@ def quantize_sym(W: np.ndarray, group_size: int = GROUP_SIZE):
     ratio), so code 0 (c = -8) is never produced: 15 of the 16 levels are
     used, as the max/7 reading implies.
 
-    Returns (codes uint8 [N, K], scales fp16 [N, G]).
+    Returns (codes uint8 [N, K], scales fp16 [G, N]).
     """
     w = _groups_f32(W, group_size)
     a = np.abs(w).max(axis=2)
@@ -123,7 +127,7 @@ def quantize_sym(W: np.ndarray, group_size: int = GROUP_SIZE):
     sf = scales.astype(np.float32)
     c = np.clip(np.rint(w / sf[..., None]), -8, 7)
     codes = (c + SYM_ZERO).astype(np.uint8).reshape(W.shape)
-    return codes, scales
+    return codes, np.ascontiguousarray(scales.T)
 
 
 def pseudo_quantize(W: np.ndarray, group_size: int = GROUP_SIZE, zero_point: bool = True):
@@ -170,6 +174,7 @@ def unpack(qweight: np.ndarray) -> np.ndarray:
 
 def dequant(codes: np.ndarray, scales: np.ndarray, zeros, group_size: int = GROUP_SIZE) -> np.ndarray:
     """fp16 weights w' = fp16((q - z) * s); z = 8 when ``zeros`` is None.
+    ``scales`` and ``zeros`` are [G, N].
 
     Asymmetric: (q - z[n, j]) * s[n, j] (the zero-point decode the AutoAWQ
     tour names); symmetric: scale x (code - 8) (fak explainer,
@@ -181,11 +186,11 @@ def dequant(codes: np.ndarray, scales: np.ndarray, zeros, group_size: int = GROU
     N, K = codes.shape
     G = K // group_size
     q = codes.astype(np.float32).reshape(N, G, group_size)
-    sf = np.asarray(scales).astype(np.float32).reshape(N, G, 1)
+    sf = np.asarray(scales).astype(np.float32).reshape(G, N).T.reshape(N, G, 1)
     if zeros is None:
         z = np.float32(SYM_ZERO)
     else:
-        z = np.asarray(zeros).astype(np.float32).reshape(N, G, 1)
+        z = np.asarray(zeros).astype(np.float32).reshape(G, N).T.reshape(N, G, 1)
     return ((q - z) * sf).astype(np.float16).reshape(N, K)
 
 

@@ -101,8 +101,8 @@ def test_dequant_closed_form_exhaustive(z):
     sbits = _scale_sweep()
     S = len(sbits)
     codes = np.tile(np.tile(np.arange(16, dtype=np.uint8), 8), (S, 1))      # [S, 128]
-    scales = sbits.view(np.float16).reshape(S, 1)
-    zeros = None if z is None else np.full((S, 1), z, dtype=np.float16)
+    scales = sbits.view(np.float16).reshape(1, S)                           # [G=1, N=S]
+    zeros = None if z is None else np.full((1, S), z, dtype=np.float16)
     with warnings.catch_warnings():
         warnings.simplefilter("ignore")
         got = bits16(O.dequant(codes, scales, zeros, 128))
@@ -196,8 +196,8 @@ def test_asym_codes_are_nearest_level():
     with warnings.catch_warnings():
         warnings.simplefilter("ignore")
         codes, scales, zeros = O.quantize_asym(W, 128)
-    sf = f16_value(bits16(scales))[:, 0]
-    z = zeros.astype(np.float64)[:, 0]
+    sf = f16_value(bits16(scales))[0, :]       # one group per row: scales [1, n]
+    z = zeros.astype(np.float64)[0, :]
     w = W.astype(np.float64)
     levels = np.arange(16, dtype=np.float64)
     # each code minimizes |(q - z) s - w| over q in 0..15; ties -> even (q - z)
@@ -216,7 +216,7 @@ def test_sym_codes_are_nearest_level():
     with warnings.catch_warnings():
         warnings.simplefilter("ignore")
         codes, scales = O.quantize_sym(W, 128)
-    sf = f16_value(bits16(scales))[:, 0]
+    sf = f16_value(bits16(scales))[0, :]
     w = W.astype(np.float64)
     c = np.arange(-8, 8, dtype=np.float64)
     err = np.abs(c[None, None, :] * sf[:, None, None] - w[:, :, None])
@@ -248,8 +248,8 @@ def test_scale_rule_asym_and_sym():
     floor = float(np.float32(1e-5))
     r_a = np.maximum((w.max(1) - w.min(1)) / 15.0, floor)
     r_s = np.maximum(np.abs(w).max(1) / 7.0, floor)
-    _check_scale(bits16(s_a)[:, 0], r_a)
-    _check_scale(bits16(s_s)[:, 0], r_s)
+    _check_scale(bits16(s_a)[0, :], r_a)
+    _check_scale(bits16(s_s)[0, :], r_s)
 
 
 def test_dequant_error_bound():
@@ -262,8 +262,8 @@ def test_dequant_error_bound():
         for zp in (True, False):
             codes, scales, zeros = O.pseudo_quantize(W, 128, zp)
             wq = O.dequant(codes, scales, zeros, 128).astype(np.float64)
-            sf = f16_value(bits16(scales)).repeat(128, axis=1)
-            z = (zeros.astype(np.float64) if zp else np.full(scales.shape, 8.0)).repeat(128, axis=1)
+            sf = f16_value(bits16(scales)).T.repeat(128, axis=1)      # [n, 128]
+            z = (zeros.astype(np.float64).T if zp else np.full(scales.T.shape, 8.0)).repeat(128, axis=1)
             w = W.astype(np.float64)
             lo, hi = (0 - z) * sf, (15 - z) * sf
             inside = (w >= lo - sf / 2) & (w <= hi + sf / 2)
@@ -285,7 +285,7 @@ def test_quantize_scale_equivariance():
         c1, s1, z1 = O.pseudo_quantize(W, 128, zp)
         c2, s2, z2 = O.pseudo_quantize(W2, 128, zp)
         assert np.array_equal(c1, c2)
-        assert np.array_equal(s2.astype(np.float64), s1.astype(np.float64) * np.ldexp(1.0, e))
+        assert np.array_equal(s2.astype(np.float64), s1.astype(np.float64) * np.ldexp(1.0, e).T)
         if zp:
             assert np.array_equal(z1, z2)
 
@@ -338,7 +338,7 @@ def test_compression_arithmetic():
     int4_size = qweight.size * 4
     assert fp16_size / int4_size == 4
     assert qweight.nbytes == int4_size
-    assert scales.shape == zeros.shape == (512, 4)
+    assert scales.shape == zeros.shape == (4, 512)        # group-major [K/128, N]
 
 
 # ----------------------------------------------------------------------------
@@ -371,8 +371,8 @@ def test_linear_bruteforce_tiny():
             wrow = []
             for k in range(K):
                 q = (int(words[n, k // 8]) >> (4 * _slot_of_k(k % 8))) & 0xF
-                zz = float(zeros[n, k // 128]) if zp else 8.0
-                wrow.append(f16_value(f16_bits_nearest((q - zz) * sv[n, k // 128])))
+                zz = float(zeros[k // 128, n]) if zp else 8.0
+                wrow.append(f16_value(f16_bits_nearest((q - zz) * sv[k // 128, n])))
             for m in range(M):
                 exact = sum(Fraction(float(x[m, k])) * Fraction(float(wrow[k])) for k in range(K))
                 assert abs(y[m, n] - float(exact)) <= 1e-12 * max(1.0, abs(float(exact)))

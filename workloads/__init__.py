@@ -63,14 +63,15 @@ def make_packed_random(N: int, K: int, group_size: int = 128, zero_point: bool =
                        seed: int = 0, scale_lo: float = 1e-3, scale_hi: float = 4e-3):
     """Random packed weights without any quantizer: uniform int32 words (every
     bit pattern is a valid set of eight 4-bit codes), fp16 scales uniform in
-    [scale_lo, scale_hi], zero points uniform integers 0..15 stored as fp16.
+    [scale_lo, scale_hi], zero points uniform integers 0..15 stored as fp16;
+    scales and zeros are group-major [K/group_size, N].
     Used where a test wants arbitrary codes rather than codes of some W."""
     rng = np.random.default_rng(seed)
     words = rng.integers(0, 2 ** 32, size=(N, K // 8), dtype=np.uint64).astype(np.uint32)
     qweight = words.view(np.int32)
     G = K // group_size
-    scales = rng.uniform(scale_lo, scale_hi, size=(N, G)).astype(np.float16)
-    zeros = rng.integers(0, 16, size=(N, G)).astype(np.float16) if zero_point else None
+    scales = rng.uniform(scale_lo, scale_hi, size=(G, N)).astype(np.float16)
+    zeros = rng.integers(0, 16, size=(G, N)).astype(np.float16) if zero_point else None
     return qweight, scales, zeros
 
 
