@@ -1,0 +1,582 @@
+"""Benchmark of the W4A16 linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+                    [--workload llama3_8b_decode|decode_sweep|prefill|llama3_70b]
+
+Default workload: Llama-3-8B-shaped decode layers at M = 1 (q_proj 4096x4096,
+gate_proj and up_proj 14336x4096, down_proj 4096x14336; W ~ N(0, 0.02) with
+1% of input channels x10, asymmetric zero points, g = 128). One step is one
+layer's four GEMVs; the steps walk through 32 layer copies (3.3 GB of packed
+weights), so no step finds its weights in L2 (126 MB). Steps are replayed
+from CUDA graphs. The timed region is bracketed by a barrier and a device
+synchronize on both sides and timed with CUDA events; with several GPUs each
+rank runs its own replica and the time is the max over ranks.
+
+Printed: one JSON line (rank 0) with the effective HBM GB/s of the whole job
+(algorithmic bytes / time), the roofline object of the GEMV kernel (per-launch
+durations from CUDA events captured inside the timed graphs), the oracle
+timed on the host cores (cpu_baseline), the end-to-end number through the
+public API with host buffers (e2e), SM clocks sampled during the timed region,
+and the tensor-core GEMM measured on the prefill shape (M = 2048).
+
+--impl reference times the CPU oracle (the only other implementation of this
+method here) on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from workloads import LLAMA3_8B_DECODE, WORKLOADS, make_weight  # noqa: E402
+
+METRIC = "W4A16 GEMV/GEMM TFLOP/s and effective HBM GB/s (fraction of roofline), M=1..2048"
+HBM_FALLBACK_GBS = 6650.0
+TENSOR_FALLBACK_TFLOPS = 1590.0
+GEMV_PROFILE = os.path.join(ROOT, "profiles", "awq_gemv_llama3_8b_decode_m1.md")
+GEMM_PROFILE = os.path.join(ROOT, "profiles", "awq_gemm_prefill_m2048.md")
+
+
+# ----------------------------------------------------------------------------
+# work accounting (per launch)
+# ----------------------------------------------------------------------------
+def algo_bytes(M: int, N: int, K: int, zp: bool = True) -> int:
+    """Bytes a W4A16 product must move at least once: packed codes, scales,
+    zero points (asymmetric), x and y."""
+    G = K // 128
+    return N * K // 2 + 2 * N * G + (2 * N * G if zp else 0) + 2 * M * K + 2 * M * N
+
+
+def algo_flops(M: int, N: int, K: int) -> int:
+    return 2 * M * N * K
+
+
+# ----------------------------------------------------------------------------
+# distributed plumbing (replicas only: the layer is independent per GPU)
+# ----------------------------------------------------------------------------
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def init_dist(backend: str):
+    import torch.distributed as dist
+    ws, rank, _ = dist_env()
+    if ws > 1 and not dist.is_initialized():
+        from datetime import timedelta
+        dist.init_process_group(backend=backend, timeout=timedelta(seconds=120))
+    return dist if ws > 1 else None
+
+
+def reduce_max(value: float, dist, device=None) -> float:
+    """Max of a scalar over ranks (identity without a process group)."""
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def reduce_sum(value: float, dist, device=None) -> float:
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def aggregate(units_local: float, seconds_local: float, dist, device=None):
+    """Whole-job throughput: the units all ranks processed over the slowest
+    rank's time. Returns (total_units, max_seconds)."""
+    return reduce_sum(units_local, dist, device), reduce_max(seconds_local, dist, device)
+
+
+# ----------------------------------------------------------------------------
+# peaks, profiles, clocks
+# ----------------------------------------------------------------------------
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", 0)), "measured"
+    except Exception:
+        return HBM_FALLBACK_GBS, TENSOR_FALLBACK_TFLOPS, 0.0, "fallback"
+
+
+def source_sha(path: str) -> str:
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def profile_traffic(profile_path: str, source_path: str):
+    """Per-launch DRAM bytes from a committed ncu summary, or None when the
+    summary is missing or the kernel source changed since it was taken."""
+    try:
+        text = open(profile_path).read()
+    except OSError:
+        return None
+    m = re.search(r"source_sha256_16:\s*([0-9a-f]{16})", text)
+    t = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not m or not t or m.group(1) != source_sha(source_path):
+        return None
+    return float(t.group(1))
+
+
+class ClockSampler:
+    """SM clock and throttle reasons sampled through NVML while running."""
+
+    REASONS = {
+        "sw_power_cap": "nvmlClocksEventReasonSwPowerCap",
+        "hw_slowdown": "nvmlClocksEventReasonHwSlowdown",
+        "hw_thermal_slowdown": "nvmlClocksEventReasonHwThermalSlowdown",
+        "sw_thermal_slowdown": "nvmlClocksEventReasonSwThermalSlowdown",
+        "hw_power_brake": "nvmlClocksEventReasonHwPowerBrakeSlowdown",
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.002):
+        self.period = period_s
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, const in self.REASONS.items():
+                    if r & getattr(nv, const, 0):
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------
+# the CPU oracle on a bounded sample (baseline / reference arm)
+# ----------------------------------------------------------------------------
+def oracle_sample(shapes, M: int, rows: int, zp: bool = True, seed: int = 0):
+    """Per shape: a sample of `rows` output channels quantized by the oracle,
+    plus x. Returns [(x, qweight, scales, zeros, bytes)]."""
+    from oracle import awq_oracle as O
+    out = []
+    rng = np.random.default_rng(seed)
+    for sh in shapes:
+        W = make_weight(rows, sh.K, 0.02, 0.01, seed=seed)
+        qweight, scales, zeros = O.quantize_pack(W, 128, zp)
+        x = rng.standard_normal((M, sh.K), dtype=np.float32).astype(np.float16)
+        out.append((x, qweight, scales, zeros, algo_bytes(M, rows, sh.K, zp)))
+    return out
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def time_oracle(sample, budget_s: float):
+    """Run the oracle's layer (unpack, dequant, float64 matmul) over the sample
+    until `budget_s` has passed; returns (bytes, seconds, passes)."""
+    from oracle import awq_oracle as O
+    done_bytes, passes = 0, 0
+    t0 = time.perf_counter()
+    while True:
+        for x, q, s, z, b in sample:
+            O.linear(x, q, s, z, 128)
+            done_bytes += b
+        passes += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    return done_bytes, time.perf_counter() - t0, passes
+
+
+def cpu_baseline(shapes, M: int, budget_s: float = 10.0, rows: int = 1024):
+    sample = oracle_sample(shapes, M, rows)
+    b, s, passes = time_oracle(sample, budget_s)
+    return {"value": round(b / s / 1e9, 4), "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{rows} output channels of each of {len(shapes)} layer shapes, M={M}, "
+                      f"{passes} passes in {s:.1f} s (numpy unpack/dequant single-threaded, "
+                      f"float64 matmul on {blas_threads()} BLAS threads, {os.cpu_count()} host cores)"}
+
+
+# ----------------------------------------------------------------------------
+# native arm
+# ----------------------------------------------------------------------------
+class DecodeLayer:
+    """One layer copy: packed weights of each shape plus its x / y buffers."""
+
+    def __init__(self, packed, xs, ys, workspaces):
+        self.packed, self.xs, self.ys, self.ws = packed, xs, ys, workspaces
+
+
+def build_decode(awq, torch, device, shapes, M: int, n_layers: int, zp: bool):
+    """Quantize each shape once on the GPU (recipe W, seed 0), then clone the
+    packed tensors into n_layers copies at distinct addresses."""
+    base, quant_ms, quant_bytes = [], 0.0, 0
+    for sh in shapes:
+        W = torch.from_numpy(make_weight(sh.N, sh.K, 0.02, 0.01, seed=0)).to(device)
+        torch.cuda.synchronize(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        q, s, z = awq.awq_pseudo_quantize_pack(W, zero_point=zp)
+        e1.record()
+        torch.cuda.synchronize(device)
+        quant_ms += e0.elapsed_time(e1)
+        quant_bytes += 2 * sh.N * sh.K + algo_bytes(0, sh.N, sh.K, zp)
+        base.append((q, s, z))
+        del W
+    rng = np.random.default_rng(1)
+    layers = []
+    for _ in range(n_layers):
+        packed = [(q.clone(), s.clone(), z.clone() if z is not None else None) for q, s, z in base]
+        xs = [torch.from_numpy(rng.standard_normal((M, sh.K), dtype=np.float32).astype(np.float16)).to(device)
+              for sh in shapes]
+        ys = [torch.empty((M, sh.N), dtype=torch.float16, device=device) for sh in shapes]
+        wss = [awq.alloc_workspace(M, sh.N, sh.K, zp, device=device) for sh in shapes]
+        layers.append(DecodeLayer(packed, xs, ys, wss))
+    return layers, {"ms": round(quant_ms, 4), "GB/s": round(quant_bytes / (quant_ms * 1e-3) / 1e9, 1)}
+
+
+def run_native(args, dist):
+    import torch
+    import weight_only_int4_gemv_b200 as awq
+
+    ws_, rank, local = dist_env()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    awq.lib()
+    hbm_peak, tc_peak, tc_sust, peak_src = measured_peaks()
+    wl = WORKLOADS[args.workload]
+    zp = True
+    if args.workload == "llama3_8b_decode":
+        shapes, M = LLAMA3_8B_DECODE, 1
+    else:
+        shapes, M = wl.shapes, min(wl.Ms)
+    if M > awq.GEMV_MAX_M:
+        raise SystemExit("the decode bench runs the GEMV path; use --workload llama3_8b_decode or decode_sweep")
+
+    layers, quant = build_decode(awq, torch, device, shapes, M, args.layers, zp)
+    step_bytes = sum(algo_bytes(M, sh.N, sh.K, zp) for sh in shapes)
+    step_flops = sum(algo_flops(M, sh.N, sh.K) for sh in shapes)
+    stream = torch.cuda.Stream(device)
+
+    # one CUDA graph per layer copy; external event nodes around every GEMV
+    graphs, evs = [], []
+    with torch.cuda.stream(stream):
+        for L in layers:     # warm the plan caches outside capture
+            for i in range(len(shapes)):
+                awq.awq_gemv(L.xs[i], *L.packed[i], workspace=L.ws[i], out=L.ys[i])
+        torch.cuda.synchronize(device)
+        for L in layers:
+            g = torch.cuda.CUDAGraph()
+            pairs = [(torch.cuda.Event(enable_timing=True, external=True),
+                      torch.cuda.Event(enable_timing=True, external=True)) for _ in shapes]
+            with torch.cuda.graph(g, stream=stream):
+                for i in range(len(shapes)):
+                    pairs[i][0].record()
+                    awq.awq_gemv(L.xs[i], *L.packed[i], workspace=L.ws[i], out=L.ys[i])
+                    pairs[i][1].record()
+            graphs.append(g)
+            evs.append(pairs)
+    torch.cuda.synchronize(device)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    n = len(graphs)
+    with torch.cuda.stream(stream):
+        for s in range(args.warmup):
+            graphs[s % n].replay()
+    torch.cuda.synchronize(device)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(device.index if device.index is not None else 0)
+    barrier()
+    torch.cuda.synchronize(device)
+    with sampler:
+        with torch.cuda.stream(stream):
+            t0.record()
+            for s in range(args.steps):
+                graphs[(args.warmup + s) % n].replay()
+            t1.record()
+        torch.cuda.synchronize(device)
+    barrier()
+    elapsed_s = t0.elapsed_time(t1) * 1e-3
+
+    # per-launch kernel durations: the last replay of each graph inside the timed region
+    used = sorted({(args.warmup + s) % n for s in range(args.steps)})
+    launch_ms, launch_bytes = [], []
+    for gi in used:
+        for i, sh in enumerate(shapes):
+            launch_ms.append(evs[gi][i][0].elapsed_time(evs[gi][i][1]))
+            launch_bytes.append(algo_bytes(M, sh.N, sh.K, zp))
+    kernel_gbs = sum(launch_bytes) / (sum(launch_ms) * 1e-3) / 1e9
+
+    total_bytes, max_s = aggregate(step_bytes * args.steps, elapsed_s, dist, device)
+    value = total_bytes / max_s / 1e9
+
+    # end to end through the public API: pinned host x in, pinned host y out, every step
+    e2e = run_e2e(awq, torch, device, stream, layers, shapes, M, args, dist, step_bytes)
+
+    gemm = None
+    if ws_ == 1 and not args.no_gemm:
+        gemm = run_gemm_prefill(awq, torch, device, tc_peak, peak_src, args)
+
+    cpu = None
+    if ws_ == 1 and rank == 0 and not args.no_cpu:
+        cpu = cpu_baseline(shapes, M, budget_s=args.cpu_seconds)
+
+    if rank == 0:
+        gemv_src = os.path.join(ROOT, "weight_only_int4_gemv_b200", "csrc", "awq_gemv.cu")
+        traffic = profile_traffic(GEMV_PROFILE, gemv_src)
+        line = {
+            "metric": METRIC,
+            "value": round(value, 2),
+            "unit": "GB/s",
+            "n_gpus": ws_,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": round(max_s * 1e3 / args.steps, 6),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "f16",
+            "data": "synthetic (seeded N(0,0.02) weights, 1% salient input channels x10, N(0,1) x; no checkpoint)",
+            "config": {
+                "workload": f"{args.workload}_m{M}",
+                "layers": [f"{sh.name} {sh.N}x{sh.K}" for sh in shapes],
+                "M": M, "group_size": 128, "zero_point": zp,
+                "step": "one layer: one GEMV per listed projection",
+                "l2": f"inputs larger than L2: steps rotate over {args.layers} layer copies "
+                      f"({args.layers * step_bytes / 1e9:.2f} GB of packed weights)",
+                "parallelism": f"replicas x{ws_}",
+            },
+            "tflops": round(reduce_sum(step_flops * args.steps, dist, device) / max_s / 1e12, 4),
+            "roofline": {
+                "bound": "hbm", "achieved": round(kernel_gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+                "frac": round(kernel_gbs / hbm_peak, 4),
+                "traffic": traffic, "peak_source": peak_src,
+                "kernel": "awq_gemv (gemv_kernel<1,2,true>)",
+                "launches_timed": len(launch_ms),
+                "algorithmic_bytes_per_launch": round(sum(launch_bytes) / len(launch_bytes)),
+                "mean_launch_us": round(1e3 * sum(launch_ms) / len(launch_ms), 3),
+                "frac_of_nominal_8TBs": round(kernel_gbs / 8000.0, 4),
+            },
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": args.steps * len(shapes),
+            "clocks": sampler.summary(),
+            "quantize": quant,
+        }
+        if gemm is not None:
+            line["prefill_gemm"] = gemm
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(awq, torch, device, stream, layers, shapes, M, args, dist, step_bytes):
+    """Same metric through the Python API with host buffers: every step copies
+    its x from pinned host memory and reads its y back into pinned host
+    memory, then synchronizes."""
+    steps = max(1, min(args.steps, args.e2e_steps))
+    hx = [torch.empty((M, sh.K), dtype=torch.float16).pin_memory() for sh in shapes]
+    hy = [torch.empty((M, sh.N), dtype=torch.float16).pin_memory() for sh in shapes]
+    for i in range(len(shapes)):
+        hx[i].copy_(layers[0].xs[i].cpu())
+    h2d = sum(t.numel() * 2 for t in hx)
+    d2h = sum(t.numel() * 2 for t in hy)
+    n = len(layers)
+
+    def step(s):
+        L = layers[s % n]
+        for i in range(len(shapes)):
+            L.xs[i].copy_(hx[i], non_blocking=True)
+            awq.awq_gemv(L.xs[i], *L.packed[i], workspace=L.ws[i], out=L.ys[i])
+            hy[i].copy_(L.ys[i], non_blocking=True)
+        torch.cuda.current_stream(device).synchronize()
+
+    with torch.cuda.stream(stream):
+        for s in range(min(args.warmup, 20)):
+            step(s)
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize(device)
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record()
+        for s in range(steps):
+            step(s)
+        t1.record()
+        torch.cuda.synchronize(device)
+    sec = t0.elapsed_time(t1) * 1e-3
+    total, max_s = aggregate(step_bytes * steps, sec, dist, device)
+    return {"value": round(total / max_s / 1e9, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": steps,
+            "note": "effective HBM GB/s of the same algorithmic bytes, time includes the copies and a "
+                    "host synchronize per step"}
+
+
+def run_gemm_prefill(awq, torch, device, tc_peak, peak_src, args):
+    """awq_gemm at M = 2048 on gate_proj 14336x4096 (the prefill shape), four
+    weight/activation copies in rotation (180 MB > L2), events per launch."""
+    M, N, K = 2048, 14336, 4096
+    W = torch.from_numpy(make_weight(N, K, 0.02, 0.0, seed=0)).to(device)
+    q, s, z = awq.awq_pseudo_quantize_pack(W, zero_point=True)
+    del W
+    rng = np.random.default_rng(2)
+    copies = []
+    for _ in range(4):
+        x = torch.from_numpy(rng.standard_normal((M, K), dtype=np.float32).astype(np.float16)).to(device)
+        copies.append((x, q.clone(), s.clone(), z.clone(), torch.empty((M, N), dtype=torch.float16, device=device)))
+    reps = max(8, min(args.gemm_steps, 400))
+    for i in range(4):
+        x, qq, ss, zz, y = copies[i]
+        awq.awq_gemm(x, qq, ss, zz, out=y)
+    torch.cuda.synchronize(device)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    sampler = ClockSampler(device.index if device.index is not None else 0)
+    with sampler:
+        for r in range(reps):
+            x, qq, ss, zz, y = copies[r % 4]
+            evs[r][0].record()
+            awq.awq_gemm(x, qq, ss, zz, out=y)
+            evs[r][1].record()
+        torch.cuda.synchronize(device)
+    ms = [a.elapsed_time(b) for a, b in evs]
+    mean_ms = sum(ms) / len(ms)
+    tflops = algo_flops(M, N, K) / (mean_ms * 1e-3) / 1e12
+    err = awq.awq_device_error(device)
+    gemm_src = os.path.join(ROOT, "weight_only_int4_gemv_b200", "csrc", "awq_gemm.cu")
+    return {"workload": f"prefill_m{M} gate_proj {N}x{K}", "launches": reps,
+            "mean_launch_us": round(mean_ms * 1e3, 2), "min_launch_us": round(min(ms) * 1e3, 2),
+            "tflops": round(tflops, 1),
+            "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": tc_peak, "unit": "TFLOP/s",
+                         "frac": round(tflops / tc_peak, 4), "peak_source": f"{peak_src} (bf16 burst; fp16 same rate)",
+                         "traffic": profile_traffic(GEMM_PROFILE, gemm_src)},
+            "clocks": sampler.summary(), "device_error": err}
+
+
+# ----------------------------------------------------------------------------
+# reference arm: the CPU oracle
+# ----------------------------------------------------------------------------
+def run_reference(args, dist):
+    ws_, rank, _ = dist_env()
+    if rank != 0:
+        return
+    if args.workload == "llama3_8b_decode":
+        shapes, M = LLAMA3_8B_DECODE, 1
+    else:
+        wl = WORKLOADS[args.workload]
+        shapes, M = wl.shapes, min(wl.Ms)
+    rows = args.ref_rows
+    sample = oracle_sample(shapes, M, rows)
+    for _ in range(args.warmup):
+        time_oracle(sample, 0.0)
+    b, s, passes = 0, 0.0, 0
+    for _ in range(args.steps):
+        bb, ss, _p = time_oracle(sample, 0.0)
+        b += bb
+        s += ss
+        passes += 1
+    value = b / s / 1e9
+    desc = (f"each step: the oracle layer on {rows} output channels of each of {len(shapes)} shapes "
+            f"({', '.join(f'{sh.name} {sh.N}x{sh.K}' for sh in shapes)}), M={M}")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": ws_,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(s * 1e3 / args.steps, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": f"{args.workload}_m{M}", "sample": desc},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "kind": "oracle", "cores": blas_threads(),
+                         "sample": desc},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=64)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--workload", choices=["llama3_8b_decode", "decode_sweep"], default="llama3_8b_decode")
+    ap.add_argument("--layers", type=int, default=32, help="layer copies the steps rotate over")
+    ap.add_argument("--e2e-steps", type=int, default=500)
+    ap.add_argument("--gemm-steps", type=int, default=100)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--ref-rows", type=int, default=256)
+    ap.add_argument("--no-gemm", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    a = ap.parse_args(argv)
+    if a.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if a.steps < 1:
+        ap.error("--steps must be >= 1")
+    return a
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    ws_, _, _ = dist_env()
+    if args.impl == "reference":
+        run_reference(args, None)
+        return 0
+    dist = init_dist("nccl")
+    try:
+        run_native(args, dist)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -34,9 +34,11 @@
  *                               order, (word >> 4j) & 0x000F000F holds the
  *                               codes of the consecutive pair k = 8w+2j,
  *                               8w+2j+1 in its low and high 16-bit halves.
- *   scales   fp16   [N][G]      s[n][j] for k in [128j, 128j + 128)
- *   zeros    fp16   [N][G]      integer zero points 0..15 stored as fp16
- *                               (asymmetric only; NULL for symmetric)
+ *   scales   fp16   [G][N]      s[j][n] for k in [128j, 128j + 128) of row n
+ *                               (group-major, as AutoAWQ stores scales)
+ *   zeros    fp16   [G][N]      integer zero points 0..15 stored as fp16,
+ *                               group-major (asymmetric only; NULL for
+ *                               symmetric)
  *
  * fp16 buffers are passed as uint16_t pointers holding IEEE binary16 bits.
  *
@@ -107,7 +109,7 @@ AWQ_API const char* awq_status_string(awq_status_t status);
  *               q = clamp(rint(w / s), -8, 7) + 8
  * rint rounds half to even; s is used at its fp16 value.
  *
- * In:  W [N][K] fp16.  Out: qweight [N][K/8], scales [N][G], zeros [N][G]
+ * In:  W [N][K] fp16.  Out: qweight [N][K/8], scales [G][N], zeros [G][N]
  * (asymmetric; must be NULL for symmetric).
  * N >= 0 (N == 0: no work), K > 0 and K % group_size == 0.
  * Results are bit-exact: a given W always yields the same bits.
@@ -144,11 +146,12 @@ AWQ_API awq_status_t awq_workspace_bytes(int64_t M, int64_t N, int64_t K,
  * awq_gemv -- y[M][N] = x[M][K] . W'^T for small batches (decode), 1 <= M <= 16.
  * ("AutoAWQ" code tour, "The big picture": the GEMV variant for single-token
  * decoding; "AutoAWQ" capability page: dequantization fused into the matmul.)
- * y[m][n] = fp16( sum_k x[m][k] * (q[n][k] - z[n][k/128]) * s[n][k/128] ),
+ * y[m][n] = fp16( sum_k x[m][k] * (q[n][k] - z[k/128][n]) * s[k/128][n] ),
  * products and sums in fp32 (the per-group factor s is applied to the fp32
  * partial sum of each group). The summation order is fixed for a given
  * device and shape, so results are reproducible run to run.
- * M in [1, 16]; N >= 0 (0: no work); K > 0, K % group_size == 0.
+ * M in [1, 16]; N >= 0 and N % 8 == 0 (0: no work); K > 0, K % group_size == 0.
+ * (N % 8 keeps every 8-row run of scales and zero points 16-byte aligned.)
  * workspace: at least awq_workspace_bytes(M, N, K) bytes, zero-filled before
  * first use (see above); may be NULL when that size is 0.
  */

@@ -86,7 +86,7 @@ def test_gemv_llama3_70b_sampled(N, K):
 def test_gemv_random_codes_and_extreme_zero_points():
     """Arbitrary words (every code value in every slot) and zero points 0..15."""
     for zp in (True, False):
-        qweight, scales, zeros = make_packed_random(300, 2048, 128, zp, seed=4)
+        qweight, scales, zeros = make_packed_random(296, 2048, 128, zp, seed=4)
         Wd = O.dequant(O.unpack(qweight), scales, zeros, 128)
         for M in (1, 5, 16):
             x = activations(M, 2048, seed=M)
@@ -128,6 +128,10 @@ def test_gemv_edge_cases():
     # M out of range
     with pytest.raises(awq.AwqError, match="SHAPE"):
         awq.awq_gemv(dev(activations(17, 512)), dev(qweight), dev(scales), dev(zeros))
+    # N must be a multiple of 8 (16-byte runs of scales and zero points)
+    q2, s2, z2 = make_packed_random(300, 512, 128, True, seed=1)
+    with pytest.raises(awq.AwqError, match="SHAPE"):
+        awq.awq_gemv(dev(activations(1, 512)), dev(q2), dev(s2), dev(z2))
     # unsupported group size
     with pytest.raises(awq.AwqError, match="UNSUPPORTED"):
         awq.awq_gemv(dev(activations(1, 512)), dev(qweight), dev(scales), dev(zeros), group_size=64)

@@ -8,9 +8,9 @@ binding without the built library or without a CUDA device raises.
 
 Layouts (row-major, K contiguous): W fp16 [N, K]; x fp16 [M, K]; y fp16
 [M, N]; qweight int32 [N, K/8] (eight 4-bit codes per word, nibble slot i of
-word w holds k = 8w + (0, 2, 4, 6, 1, 3, 5, 7)[i]); scales fp16 [N, K/128];
-zeros fp16 [N, K/128] holding integers 0..15 (None for the symmetric
-variant, whose zero point is 8).
+word w holds k = 8w + (0, 2, 4, 6, 1, 3, 5, 7)[i]); scales fp16 [K/128, N];
+zeros fp16 [K/128, N] holding integers 0..15 (None for the symmetric
+variant, whose zero point is 8); scales and zeros are group-major.
 """
 
 from __future__ import annotations
@@ -116,8 +116,8 @@ def awq_pseudo_quantize_pack(W: torch.Tensor, zero_point: bool = True, group_siz
     N, K = W.shape
     G = K // group_size if group_size > 0 else 0
     qweight = torch.empty((N, K // 8), dtype=torch.int32, device=W.device)
-    scales = torch.empty((N, G), dtype=torch.float16, device=W.device)
-    zeros = torch.empty((N, G), dtype=torch.float16, device=W.device) if zero_point else None
+    scales = torch.empty((G, N), dtype=torch.float16, device=W.device)          # group-major
+    zeros = torch.empty((G, N), dtype=torch.float16, device=W.device) if zero_point else None
     with torch.cuda.device(W.device):
         _check("awq_pseudo_quantize_pack", lib().awq_pseudo_quantize_pack(
             _ptr(W), N, K, _cfg(zero_point, group_size), _ptr(qweight), _ptr(scales), _ptr(zeros),
@@ -133,6 +133,9 @@ def awq_dequant(qweight: torch.Tensor, scales: torch.Tensor, zeros, group_size: 
     if zeros is not None:
         _need(zeros, "zeros", torch.float16, 2)
     N, K = qweight.shape[0], qweight.shape[1] * 8
+    if group_size == GROUP_SIZE and (scales.shape != (K // group_size, N) or
+                                     (zeros is not None and zeros.shape != scales.shape)):
+        raise ValueError("scales / zeros must be [K/group_size, N]")
     if out is None:
         out = torch.empty((N, K), dtype=torch.float16, device=qweight.device)
     _need(out, "out", torch.float16, 2)
@@ -170,6 +173,9 @@ def _product(entry: str, x, qweight, scales, zeros, workspace, out, group_size):
     N = qweight.shape[0]
     if qweight.shape[1] * 8 != K:
         raise ValueError("qweight must be [N, K/8] for x [M, K]")
+    if group_size == GROUP_SIZE and (scales.shape != (K // group_size, N) or
+                                     (zeros is not None and zeros.shape != scales.shape)):
+        raise ValueError("scales / zeros must be [K/group_size, N]")
     if out is None:
         out = torch.empty((M, N), dtype=torch.float16, device=x.device)
     _need(out, "out", torch.float16, 2)

@@ -259,20 +259,21 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
       const int n0 = (tile / p.m_tiles) * BN;
       const int64_t row = int64_t(n0) + i;
       const bool valid = row < p.N;
-      const uint16_t* srow = p.scales + (valid ? row : 0) * p.G;
-      const uint16_t* zrow = ZP ? p.zeros + (valid ? row : 0) * p.G : nullptr;
+      // group-major metadata: consecutive threads read consecutive rows
+      const uint16_t* scol = p.scales + (valid ? row : 0);
+      const uint16_t* zcol = ZP ? p.zeros + (valid ? row : 0) : nullptr;
       uint32_t zb1024 = 0, zb64 = 0, sc2 = 0;
       // scale and zero of group 0, then always one group ahead
-      uint16_t s_next = valid ? ld_nc_u16(srow) : uint16_t(0);
-      uint16_t z_next = (ZP && valid) ? ld_nc_u16(zrow) : uint16_t(0);
+      uint16_t s_next = valid ? ld_nc_u16(scol) : uint16_t(0);
+      uint16_t z_next = (ZP && valid) ? ld_nc_u16(zcol) : uint16_t(0);
       for (int kb = 0; kb < p.k_blocks; ++kb) {
         if ((kb & 1) == 0) {  // new group of 128 k
           const uint16_t sb = s_next;
           const float z = ZP ? half_bits_to_float(z_next) : 8.0f;
           const int gn = (kb >> 1) + 1;
           if (valid && gn < p.G) {
-            s_next = ld_nc_u16(srow + gn);
-            if (ZP) z_next = ld_nc_u16(zrow + gn);
+            s_next = ld_nc_u16(scol + int64_t(gn) * p.N);
+            if (ZP) z_next = ld_nc_u16(zcol + int64_t(gn) * p.N);
           }
           zero_bias_pairs(z, zb1024, zb64);
           sc2 = uint32_t(sb) | (uint32_t(sb) << 16);

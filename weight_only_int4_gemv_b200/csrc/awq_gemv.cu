@@ -5,27 +5,31 @@
 // matmul and never written back as fp16.)
 //
 // The layer is bound by HBM: every packed code byte is read once and feeds
-// only M multiply-adds. Design:
+// only M multiply-adds, so the kernel is built around keeping enough bytes
+// in flight on every SM.
 //
 // * Work unit = (row block of 16*RT output channels, one group of 128 k).
-//   The units are ordered block-major and split evenly over every warp of a
-//   grid sized to the resident capacity of the GPU (a stream-K split), so all
-//   148 SMs stream the same number of bytes whatever N and K are.
-// * Each lane streams its codes with 16-byte non-allocating loads, one group
-//   ahead of the arithmetic: lane (g, t) of a warp reads 16 bytes (32 codes)
-//   of rows g and g+8 of each 16-row tile; the four lanes of a quad cover one
-//   whole group of a row.
+//   Units are ordered block-major and split evenly over every warp of a grid
+//   sized to the resident capacity of the GPU (a stream-K split): all SMs
+//   stream the same number of bytes whatever N and K are.
+// * Each warp owns an S-stage ring in shared memory and fills it with 16-byte
+//   cp.async copies S-1 units ahead of the arithmetic: the unit's packed
+//   codes (lane (g, t) copies 16 bytes of rows g and g+8 of each 16-row
+//   tile, the bytes it will decode itself), the 16-row runs of scales and
+//   zero points (group-major metadata makes them contiguous), and the
+//   unit's slice of x (128 k of every batch row, 16-byte chunks swizzled so
+//   the fragment reads are free of bank conflicts).
 // * Decode: the packed nibble order puts consecutive k pairs in the low and
 //   high halves of a word, so one LOP3 turns a word into two fp16 values
-//   1024+q (or 64+q) and one HSUB2 subtracts 1024+z, leaving q - z exactly.
+//   1024+q (or 64+q) and one HSUB2 subtracts 1024+z (64+z), leaving q - z
+//   exactly.
 // * Multiply: the decoded 16x16 weight tile is the A operand of
 //   mma.m16n8k16 straight from registers; x is the B operand (batch in the
 //   n dimension, two n8 tiles for M > 8). The k positions inside an MMA are
 //   a permutation of the word's k (each lane owns whole words), matched by
-//   loading x[m][8w .. 8w+7] for the same words, which is one 16-byte load
-//   covering two MMAs. Accumulation is fp32.
-// * The scale is applied once per group: sum_k x (q - z) s = s * sum_k x (q - z),
-//   the group's fp32 partial is multiplied by s and added to the fp32 total.
+//   reading x[m][8w .. 8w+7] for the same words: one 16-byte read covers two
+//   MMAs. Accumulation is fp32.
+// * The scale is applied once per group: sum_k x (q - z) s = s * sum_k x (q - z).
 // * A row block split between warps is finished by the last warp to arrive
 //   (arrival counter per block): it sums the contributors' fp32 partials in
 //   a fixed order, so results do not depend on timing, and resets the
@@ -51,7 +55,27 @@ struct GemvParams {
   uint32_t* counters;    // [nb]
   int64_t units;         // nb * G
   int M, N, K, G, nb, total_warps;
+  int stage_bytes;       // codes + metadata + x slice of one unit
+  int x_offset;          // offset of the x slice inside a stage
 };
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// 16-byte async copy global -> shared; src_bytes = 0 writes zeros.
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ uint4 lds128(const uint8_t* p) { return *reinterpret_cast<const uint4*>(p); }
+__device__ __forceinline__ uint16_t lds16(const uint8_t* p) { return *reinterpret_cast<const uint16_t*>(p); }
 
 __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                           uint32_t a3, uint32_t b0, uint32_t b1) {
@@ -66,11 +90,21 @@ __device__ __forceinline__ uint32_t word_of(const uint4& v, int i) {
   return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
 
-template <int RT>
-struct Stage {
-  uint4 c_lo[RT], c_hi[RT];
-  uint16_t s_lo[RT], s_hi[RT], z_lo[RT], z_hi[RT];
-};
+// (1024 + z, 1024 + z) and (64 + z, 64 + z) from the fp16 bits of an
+// integer zero point z in 0..15: both sums are exact in fp16.
+__device__ __forceinline__ void zero_bias_from_bits(uint16_t zbits, uint32_t& zb1024, uint32_t& zb64) {
+  const uint32_t zz = uint32_t(zbits) | (uint32_t(zbits) << 16);
+  uint32_t a, b;
+  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(a) : "r"(zz), "r"(0x64006400u));
+  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(b) : "r"(zz), "r"(0x54005400u));
+  zb1024 = a;
+  zb64 = b;
+}
+
+// Position of 16-byte chunk c (0..15) of batch row m inside a stage's x
+// slice: spreads the 8 lanes of each quarter-warp fragment read over all
+// 32 banks.
+__device__ __forceinline__ int x_chunk_pos(int m, int c) { return c ^ ((c >> 3) & 1) ^ ((m & 1) << 1); }
 
 // First unit of warp w in the even split of `units` over `warps`.
 __device__ __forceinline__ int64_t warp_start(int64_t units, int64_t w, int64_t warps) {
@@ -99,185 +133,210 @@ __device__ __forceinline__ void store_y(const GemvParams& p, int64_t row0, int g
   }
 }
 
-template <int MT, int RT, bool ZP>
-__global__ void __launch_bounds__(kGemvThreads)
-gemv_kernel(const GemvParams p) {
-  const int lane = threadIdx.x & 31;
-  const int g = lane >> 2;
-  const int t = lane & 3;
-  const int64_t gw = int64_t(blockIdx.x) * kGemvWarps + (threadIdx.x >> 5);
-  const int64_t W = p.total_warps;
+// Finish row block b after this warp summed groups [j0, j1) of it.
+template <int MT, int RT>
+__device__ __forceinline__ void finish_block(const GemvParams& p, int64_t b, int j0, int j1, int64_t gw,
+                                             int64_t first_block, int lane, int g, int t,
+                                             const float (&acc)[RT][MT][4]) {
+  const int64_t row0 = b * (16 * RT);
   const int64_t G = p.G;
-  const int64_t u_begin = warp_start(p.units, gw, W);
-  const int64_t u_end = warp_start(p.units, gw + 1, W);
-  if (u_begin >= u_end) return;
-  const int64_t first_block = u_begin / G;
-  const int64_t row_vec = p.K / 32;       // 16-byte vectors per packed row
-  const uint4* qv = reinterpret_cast<const uint4*>(p.qweight);
-
-  // activation rows served by this lane (batch index m = 8 mt + g)
-  const uint16_t* xrow[MT];
-  bool xok[MT];
-#pragma unroll
-  for (int mt = 0; mt < MT; ++mt) {
-    const int m = 8 * mt + g;
-    xok[mt] = m < p.M;
-    xrow[mt] = p.x + int64_t(xok[mt] ? m : 0) * p.K + 32 * t;
+  if (j0 == 0 && j1 == G) {
+    store_y<MT, RT>(p, row0, g, t, acc);
+    return;
   }
-
-  for (int64_t u = u_begin; u < u_end;) {
-    const int64_t b = u / G;
-    const int j0 = int(u - b * G);
-    const int j1 = int(u_end - b * G < G ? u_end - b * G : G);
-    const int64_t row0 = b * (16 * RT);
-
-    const uint4* cp_lo[RT];
-    const uint4* cp_hi[RT];
-    const uint16_t* sp_lo[RT];
-    const uint16_t* sp_hi[RT];
-    bool ok_lo[RT], ok_hi[RT];
+  // Partial block: publish this warp's fp32 sums, count its groups in.
+  constexpr int kSlot = RT * MT * 4 * 32;
+  const int slot = (b == first_block) ? 0 : 1;
+  float* sp = p.partials + (gw * 2 + slot) * kSlot;
+  int idx = 0;
 #pragma unroll
-    for (int rt = 0; rt < RT; ++rt) {
-      const int64_t r_lo = row0 + 16 * rt + g;
-      const int64_t r_hi = r_lo + 8;
-      ok_lo[rt] = r_lo < p.N;
-      ok_hi[rt] = r_hi < p.N;
-      cp_lo[rt] = qv + (ok_lo[rt] ? r_lo : 0) * row_vec + t;
-      cp_hi[rt] = qv + (ok_hi[rt] ? r_hi : 0) * row_vec + t;
-      sp_lo[rt] = p.scales + (ok_lo[rt] ? r_lo : 0) * G;
-      sp_hi[rt] = p.scales + (ok_hi[rt] ? r_hi : 0) * G;
-    }
-
-    auto load_stage = [&](Stage<RT>& s, int j) {
+  for (int rt = 0; rt < RT; ++rt)
 #pragma unroll
-      for (int rt = 0; rt < RT; ++rt) {
-        s.c_lo[rt] = ok_lo[rt] ? ld_stream_v4(cp_lo[rt] + 4 * j) : make_uint4(0, 0, 0, 0);
-        s.c_hi[rt] = ok_hi[rt] ? ld_stream_v4(cp_hi[rt] + 4 * j) : make_uint4(0, 0, 0, 0);
-        s.s_lo[rt] = ok_lo[rt] ? ld_nc_u16(sp_lo[rt] + j) : uint16_t(0);
-        s.s_hi[rt] = ok_hi[rt] ? ld_nc_u16(sp_hi[rt] + j) : uint16_t(0);
-        if (ZP) {
-          s.z_lo[rt] = ok_lo[rt] ? ld_nc_u16(p.zeros + (sp_lo[rt] - p.scales) + j) : uint16_t(0);
-          s.z_hi[rt] = ok_hi[rt] ? ld_nc_u16(p.zeros + (sp_hi[rt] - p.scales) + j) : uint16_t(0);
-        }
-      }
-    };
-
-    float acc[RT][MT][4];
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i, ++idx) __stcg(sp + idx * 32 + lane, acc[rt][mt][i]);
+  __threadfence();
+  __syncwarp();
+  uint32_t last = 0;
+  if (lane == 0) {
+    const uint32_t mine = uint32_t(j1 - j0);
+    const uint32_t old = atomicAdd(p.counters + b, mine);
+    last = (old + mine == uint32_t(G)) ? 1u : 0u;
+  }
+  last = __shfl_sync(0xffffffffu, last, 0);
+  if (!last) return;
+  __threadfence();
+  // contributors: every non-empty warp range overlapping block b, in warp order
+  const int64_t W = p.total_warps;
+  const int64_t w_first = ((b * G + 1) * W - 1) / p.units;
+  const int64_t w_last = ((b * G + G) * W - 1) / p.units;
+  float tot[RT][MT][4];
+#pragma unroll
+  for (int rt = 0; rt < RT; ++rt)
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) tot[rt][mt][i] = 0.0f;
+  for (int64_t w = w_first; w <= w_last; ++w) {
+    const int64_t ws = warp_start(p.units, w, W);
+    if (ws >= warp_start(p.units, w + 1, W)) continue;   // empty range
+    const int s = (ws / G == b) ? 0 : 1;
+    const float* rp = p.partials + (w * 2 + s) * kSlot;
+    int k = 0;
 #pragma unroll
     for (int rt = 0; rt < RT; ++rt)
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) acc[rt][mt][i] = 0.0f;
+        for (int i = 0; i < 4; ++i, ++k) tot[rt][mt][i] += __ldcg(rp + k * 32 + lane);
+  }
+  store_y<MT, RT>(p, row0, g, t, tot);
+  if (lane == 0) p.counters[b] = 0u;
+}
 
-    Stage<RT> cur;
-    load_stage(cur, j0);
-    for (int j = j0; j < j1; ++j) {
-      Stage<RT> nxt;
-      if (j + 1 < j1) load_stage(nxt, j + 1);
+template <int MT, int RT, bool ZP, int S>
+__global__ void __launch_bounds__(kGemvThreads)
+gemv_kernel(const GemvParams p) {
+  extern __shared__ __align__(16) uint8_t gemv_smem[];
+  constexpr int kCodeBytes = RT * 2 * 32 * 16;   // [rt][row half][lane] x 16 B
+  constexpr int kMetaBytes = RT * 16 * 2;         // one fp16 per row of the block
+  const int lane = threadIdx.x & 31;
+  const int g = lane >> 2;
+  const int t = lane & 3;
+  const int wi = threadIdx.x >> 5;
+  const int64_t gw = int64_t(blockIdx.x) * kGemvWarps + wi;
+  const int64_t W = p.total_warps;
+  const int64_t G = p.G;
+  const int64_t u_begin = warp_start(p.units, gw, W);
+  const int64_t u_end = warp_start(p.units, gw + 1, W);
+  if (u_begin >= u_end) return;
+  const int stage_bytes = p.stage_bytes;
+  uint8_t* ring = gemv_smem + int64_t(wi) * S * stage_bytes;
+  const uint32_t ring_s = smem_addr(ring);
+  const int64_t words_per_row = p.K / 8;
+  const int x_chunks = p.M * 16;
 
-      uint4 xf[MT][4];
+  auto issue = [&](int64_t u, int slot) {
+    if (u < u_end) {
+      const int64_t b = u / G;
+      const int64_t j = u - b * G;
+      const int64_t r0 = b * (16 * RT);
+      const uint32_t st = ring_s + uint32_t(slot * stage_bytes);
 #pragma unroll
-      for (int mt = 0; mt < MT; ++mt)
+      for (int rt = 0; rt < RT; ++rt)
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj)
-          xf[mt][jj] = xok[mt] ? ld_nc_v4(xrow[mt] + int64_t(j) * kGroup + 8 * jj) : make_uint4(0, 0, 0, 0);
-
-#pragma unroll
-      for (int rt = 0; rt < RT; ++rt) {
-        uint32_t zl1024, zl64, zh1024, zh64;
-        if (ZP) {
-          zero_bias_pairs(half_bits_to_float(cur.z_lo[rt]), zl1024, zl64);
-          zero_bias_pairs(half_bits_to_float(cur.z_hi[rt]), zh1024, zh64);
-        } else {
-          zero_bias_pairs(8.0f, zl1024, zl64);
-          zh1024 = zl1024;
-          zh64 = zl64;
+        for (int h = 0; h < 2; ++h) {
+          const int64_t row = r0 + 16 * rt + 8 * h + g;
+          const bool v = row < p.N;
+          const int32_t* src = p.qweight + (v ? row : 0) * words_per_row + j * kWordsPerGroup + t * 4;
+          cp_async_16(st + uint32_t(((rt * 2 + h) * 32 + lane) * 16), src, v ? 16u : 0u);
         }
-        float grp[MT][4];
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-          for (int i = 0; i < 4; ++i) grp[mt][i] = 0.0f;
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-          uint32_t plo[4], phi[4];
-          decode_word_qz(word_of(cur.c_lo[rt], jj), zl1024, zl64, plo);
-          decode_word_qz(word_of(cur.c_hi[rt], jj), zh1024, zh64, phi);
-#pragma unroll
-          for (int mt = 0; mt < MT; ++mt) {
-            mma_16816(grp[mt], plo[0], phi[0], plo[1], phi[1], xf[mt][jj].x, xf[mt][jj].y);
-            mma_16816(grp[mt], plo[2], phi[2], plo[3], phi[3], xf[mt][jj].z, xf[mt][jj].w);
-          }
-        }
-        const float s_lo = half_bits_to_float(cur.s_lo[rt]);
-        const float s_hi = half_bits_to_float(cur.s_hi[rt]);
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-          acc[rt][mt][0] = fmaf(s_lo, grp[mt][0], acc[rt][mt][0]);
-          acc[rt][mt][1] = fmaf(s_lo, grp[mt][1], acc[rt][mt][1]);
-          acc[rt][mt][2] = fmaf(s_hi, grp[mt][2], acc[rt][mt][2]);
-          acc[rt][mt][3] = fmaf(s_hi, grp[mt][3], acc[rt][mt][3]);
-        }
+      constexpr int kMetaLanes = 2 * RT * (ZP ? 2 : 1);
+      if (lane < kMetaLanes) {   // runs of 8 rows: N % 8 == 0 makes each run all in or all out
+        const int which = lane / (2 * RT);   // 0 scales, 1 zero points
+        const int rt = (lane >> 1) % RT;
+        const int h = lane & 1;
+        const int64_t rowc = r0 + 16 * rt + 8 * h;
+        const bool v = rowc < p.N;
+        const uint16_t* src = (which ? p.zeros : p.scales) + j * p.N + (v ? rowc : 0);
+        cp_async_16(st + uint32_t(kCodeBytes + which * kMetaBytes + (rt * 16 + 8 * h) * 2), src, v ? 16u : 0u);
       }
-      cur = nxt;
+      for (int c = lane; c < x_chunks; c += 32) {
+        const int m = c >> 4;
+        const int cc = c & 15;
+        const uint16_t* src = p.x + int64_t(m) * p.K + j * kGroup + cc * 8;
+        cp_async_16(st + uint32_t(p.x_offset + m * 256 + x_chunk_pos(m, cc) * 16), src, 16u);
+      }
     }
+    cp_async_commit();   // one group per unit, empty past the range, so counts stay uniform
+  };
 
-    if (j0 == 0 && j1 == G) {
-      store_y<MT, RT>(p, row0, g, t, acc);
-    } else {
-      // Partial block: publish this warp's fp32 sums, count the groups in.
-      constexpr int kSlot = RT * MT * 4 * 32;
-      const int slot = (b == first_block) ? 0 : 1;
-      float* sp = p.partials + (gw * 2 + slot) * kSlot;
-      int idx = 0;
+#pragma unroll
+  for (int i = 0; i < S - 1; ++i) issue(u_begin + i, i);
+
+  const int64_t first_block = u_begin / G;
+  int64_t cur_b = first_block;
+  int jstart = int(u_begin - cur_b * G);
+  float acc[RT][MT][4];
+#pragma unroll
+  for (int rt = 0; rt < RT; ++rt)
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[rt][mt][i] = 0.0f;
+
+  int slot = 0;
+  for (int64_t u = u_begin; u < u_end; ++u) {
+    issue(u + S - 1, slot == 0 ? S - 1 : slot - 1);
+    cp_async_wait<S - 1>();
+    __syncwarp();   // metadata and x were copied by other lanes
+    const int64_t b = u / G;
+    if (b != cur_b) {
+      finish_block<MT, RT>(p, cur_b, jstart, int(G), gw, first_block, lane, g, t, acc);
+      cur_b = b;
+      jstart = 0;
 #pragma unroll
       for (int rt = 0; rt < RT; ++rt)
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-          for (int i = 0; i < 4; ++i, ++idx) __stcg(sp + idx * 32 + lane, acc[rt][mt][i]);
-      __threadfence();
-      __syncwarp();
-      uint32_t last = 0;
-      if (lane == 0) {
-        const uint32_t mine = uint32_t(j1 - j0);
-        const uint32_t old = atomicAdd(p.counters + b, mine);
-        last = (old + mine == uint32_t(G)) ? 1u : 0u;
+          for (int i = 0; i < 4; ++i) acc[rt][mt][i] = 0.0f;
+    }
+    const uint8_t* st = ring + slot * stage_bytes;
+
+    uint4 xf[MT][4];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      const int m = 8 * mt + g;
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj)
+        xf[mt][jj] = m < p.M ? lds128(st + p.x_offset + m * 256 + x_chunk_pos(m, 4 * t + jj) * 16)
+                             : make_uint4(0, 0, 0, 0);
+    }
+
+#pragma unroll
+    for (int rt = 0; rt < RT; ++rt) {
+      const uint4 c_lo = lds128(st + ((rt * 2 + 0) * 32 + lane) * 16);
+      const uint4 c_hi = lds128(st + ((rt * 2 + 1) * 32 + lane) * 16);
+      const float s_lo = half_bits_to_float(lds16(st + kCodeBytes + (rt * 16 + g) * 2));
+      const float s_hi = half_bits_to_float(lds16(st + kCodeBytes + (rt * 16 + 8 + g) * 2));
+      uint32_t zl1024, zl64, zh1024, zh64;
+      if (ZP) {
+        zero_bias_from_bits(lds16(st + kCodeBytes + kMetaBytes + (rt * 16 + g) * 2), zl1024, zl64);
+        zero_bias_from_bits(lds16(st + kCodeBytes + kMetaBytes + (rt * 16 + 8 + g) * 2), zh1024, zh64);
+      } else {
+        zl1024 = zh1024 = 0x64086408u;   // 1032 = 1024 + 8
+        zl64 = zh64 = 0x54805480u;       // 72 = 64 + 8
       }
-      last = __shfl_sync(0xffffffffu, last, 0);
-      if (last) {
-        __threadfence();
-        // contributors: every non-empty warp range that overlaps block b,
-        // summed in warp order
-        const int64_t w_first = ((b * G + 1) * W - 1) / p.units;
-        const int64_t w_last = ((b * G + G) * W - 1) / p.units;
-        float tot[RT][MT][4];
+      float grp[MT][4];
 #pragma unroll
-        for (int rt = 0; rt < RT; ++rt)
+      for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-          for (int mt = 0; mt < MT; ++mt)
+        for (int i = 0; i < 4; ++i) grp[mt][i] = 0.0f;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) tot[rt][mt][i] = 0.0f;
-        for (int64_t w = w_first; w <= w_last; ++w) {
-          const int64_t ws = warp_start(p.units, w, W);
-          if (ws >= warp_start(p.units, w + 1, W)) continue;   // empty range
-          const int s = (ws / G == b) ? 0 : 1;
-          const float* rp = p.partials + (w * 2 + s) * kSlot;
-          int k = 0;
+      for (int jj = 0; jj < 4; ++jj) {
+        uint32_t plo[4], phi[4];
+        decode_word_qz(word_of(c_lo, jj), zl1024, zl64, plo);
+        decode_word_qz(word_of(c_hi, jj), zh1024, zh64, phi);
 #pragma unroll
-          for (int rt = 0; rt < RT; ++rt)
-#pragma unroll
-            for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-              for (int i = 0; i < 4; ++i, ++k) tot[rt][mt][i] += __ldcg(rp + k * 32 + lane);
+        for (int mt = 0; mt < MT; ++mt) {
+          mma_16816(grp[mt], plo[0], phi[0], plo[1], phi[1], xf[mt][jj].x, xf[mt][jj].y);
+          mma_16816(grp[mt], plo[2], phi[2], plo[3], phi[3], xf[mt][jj].z, xf[mt][jj].w);
         }
-        store_y<MT, RT>(p, row0, g, t, tot);
-        if (lane == 0) p.counters[b] = 0u;
+      }
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) {
+        acc[rt][mt][0] = fmaf(s_lo, grp[mt][0], acc[rt][mt][0]);
+        acc[rt][mt][1] = fmaf(s_lo, grp[mt][1], acc[rt][mt][1]);
+        acc[rt][mt][2] = fmaf(s_hi, grp[mt][2], acc[rt][mt][2]);
+        acc[rt][mt][3] = fmaf(s_hi, grp[mt][3], acc[rt][mt][3]);
       }
     }
-    u = b * G + j1;
+    __syncwarp();   // every lane is done with the slot before it is refilled
+    slot = (slot + 1 == S) ? 0 : slot + 1;
   }
+  finish_block<MT, RT>(p, cur_b, jstart, int(u_end - cur_b * G), gw, first_block, lane, g, t, acc);
+  cp_async_wait<0>();
 }
 
 // ---------------------------------------------------------------------------
@@ -287,20 +346,27 @@ using KernelFn = void (*)(const GemvParams);
 
 struct Variant {
   KernelFn fn;
-  int mt, rt;
+  int mt, rt, stages, id;
 };
 
+constexpr int kNumVariants = 4;
+
 Variant pick_variant(int64_t M, bool zp) {
-  // x fragments cost MT*256 bytes of L1 traffic per 16x128 weight tile; a
-  // 32-row block halves that, so two row tiles per warp.
-  if (M <= 8) return zp ? Variant{gemv_kernel<1, 2, true>, 1, 2} : Variant{gemv_kernel<1, 2, false>, 1, 2};
-  return zp ? Variant{gemv_kernel<2, 2, true>, 2, 2} : Variant{gemv_kernel<2, 2, false>, 2, 2};
+  if (M <= 8)
+    return zp ? Variant{gemv_kernel<1, 2, true, 4>, 1, 2, 4, 0} : Variant{gemv_kernel<1, 2, false, 4>, 1, 2, 4, 1};
+  return zp ? Variant{gemv_kernel<2, 2, true, 3>, 2, 2, 3, 2} : Variant{gemv_kernel<2, 2, false, 3>, 2, 2, 3, 3};
+}
+
+int stage_bytes_for(const Variant& v, int64_t M, bool zp) {
+  return v.rt * 2 * 32 * 16 + v.rt * 16 * 2 * (zp ? 2 : 1) + int(M) * 256;
 }
 
 struct Plan {
   Variant v;
   int grid;
   int nb;
+  int smem;
+  int stage_bytes;
   int64_t units;
   size_t counter_bytes;
   size_t partial_bytes;
@@ -308,28 +374,35 @@ struct Plan {
 
 constexpr int kMaxDevices = 64;
 std::atomic<int> g_sm_count[kMaxDevices];
-std::atomic<int> g_occ[kMaxDevices][4];
-
-int variant_index(const Variant& v, bool zp) { return (v.mt - 1) * 2 + (zp ? 1 : 0); }
+std::atomic<int> g_smem_attr[kMaxDevices][kNumVariants];
+std::atomic<int> g_occ[kMaxDevices][kNumVariants][17];   // by M
 
 awq_status_t make_plan(int64_t M, int64_t N, int64_t K, bool zp, Plan& pl) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return AWQ_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return AWQ_ERR_UNSUPPORTED;
   pl.v = pick_variant(M, zp);
+  pl.stage_bytes = stage_bytes_for(pl.v, M, zp);
+  pl.smem = kGemvWarps * pl.v.stages * pl.stage_bytes;
   int sms = g_sm_count[dev].load(std::memory_order_relaxed);
   if (sms == 0) {
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return AWQ_ERR_CUDA;
     g_sm_count[dev].store(sms, std::memory_order_relaxed);
   }
-  const int vi = variant_index(pl.v, zp);
-  int occ = g_occ[dev][vi].load(std::memory_order_relaxed);
-  if (occ == 0) {
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, pl.v.fn, kGemvThreads, 0) != cudaSuccess)
+  if (!g_smem_attr[dev][pl.v.id].load(std::memory_order_acquire)) {
+    // the largest ring any M asks of this variant
+    const int most = kGemvWarps * pl.v.stages * stage_bytes_for(pl.v, pl.v.mt * 8, zp);
+    if (cudaFuncSetAttribute(pl.v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, most) != cudaSuccess)
       return AWQ_ERR_CUDA;
-    if (occ < 1) occ = 1;
-    g_occ[dev][vi].store(occ, std::memory_order_relaxed);
+    g_smem_attr[dev][pl.v.id].store(1, std::memory_order_release);
+  }
+  int occ = g_occ[dev][pl.v.id][M].load(std::memory_order_relaxed);
+  if (occ == 0) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, pl.v.fn, kGemvThreads, pl.smem) != cudaSuccess)
+      return AWQ_ERR_CUDA;
+    if (occ < 1) return AWQ_ERR_UNSUPPORTED;
+    g_occ[dev][pl.v.id][M].store(occ, std::memory_order_relaxed);
   }
   const int64_t rows_per_block = 16 * pl.v.rt;
   const int64_t G = K / kGroup;
@@ -357,6 +430,7 @@ awq_status_t check_gemv_args(const uint16_t* x, const int32_t* qweight, const ui
   if (st != AWQ_OK) return st;
   if ((st = check_nk(N, K)) != AWQ_OK) return st;
   if (M < 1 || M > 16) return AWQ_ERR_SHAPE;
+  if (N % 8) return AWQ_ERR_SHAPE;
   if (N == 0) return AWQ_OK;
   if (!x || !qweight || !scales || !y) return AWQ_ERR_NULL;
   if (cfg.zero_point && !zeros) return AWQ_ERR_NULL;
@@ -412,6 +486,8 @@ extern "C" awq_status_t awq_gemv(const uint16_t* x, const int32_t* qweight,
   p.G = int(K / kGroup);
   p.nb = pl.nb;
   p.total_warps = pl.grid * kGemvWarps;
-  pl.v.fn<<<pl.grid, kGemvThreads, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  p.stage_bytes = pl.stage_bytes;
+  p.x_offset = pl.v.rt * 2 * 32 * 16 + pl.v.rt * 16 * 2 * (cfg.zero_point ? 2 : 1);
+  pl.v.fn<<<pl.grid, kGemvThreads, pl.smem, static_cast<cudaStream_t>(stream)>>>(p);
   return launch_status();
 }

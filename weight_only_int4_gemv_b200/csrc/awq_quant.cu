@@ -79,9 +79,9 @@ quantize_pack_kernel(const uint16_t* __restrict__ W, int64_t N, int64_t K,
     const uint32_t other = __shfl_xor_sync(0xffffffffu, part, 1);
     if ((lane & 1) == 0)
       qweight[n * (K / 8) + j * kWordsPerGroup + (lane >> 1)] = int32_t(part | other);
-    if (lane == 0) {
-      scales[n * G + j] = __half_as_ushort(__float2half_rn(sf));
-      if (ZP) zeros[n * G + j] = __half_as_ushort(__int2half_rn(int(zf)));
+    if (lane == 0) {  // metadata is group-major: [j][n]
+      scales[j * N + n] = __half_as_ushort(__float2half_rn(sf));
+      if (ZP) zeros[j * N + n] = __half_as_ushort(__int2half_rn(int(zf)));
     }
   }
 }
@@ -94,13 +94,12 @@ dequant_kernel(const int32_t* __restrict__ qweight, const uint16_t* __restrict__
                const uint16_t* __restrict__ zeros, int64_t N, int64_t K,
                uint16_t* __restrict__ out) {
   const int64_t wpr = K / 8;
-  const int64_t G = K / kGroup;
   const int64_t words = N * wpr;
   const int64_t stride = int64_t(gridDim.x) * blockDim.x;
   for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < words; i += stride) {
     const int64_t n = i / wpr;
     const int64_t wi = i - n * wpr;
-    const int64_t g = n * G + (wi * 8) / kGroup;
+    const int64_t g = ((wi * 8) / kGroup) * N + n;   // group-major metadata
     const float sf = half_bits_to_float(scales[g]);
     const float zf = ZP ? half_bits_to_float(zeros[g]) : 8.0f;
     const uint32_t word = uint32_t(qweight[i]);
