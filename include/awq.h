@@ -181,8 +181,10 @@ AWQ_API awq_status_t awq_gemm(const uint16_t* x, const int32_t* qweight,
 /*
  * awq_device_error -- read and clear the device-side error word of the
  * current device (synchronizes `stream`). Bit 0: a pipeline wait inside
- * awq_gemm exceeded its iteration limit and the kernel abandoned its tile
- * (the output is then incomplete). 0 means no error was recorded.
+ * awq_gemm passed its time limit (2 s) and the kernel abandoned its tiles;
+ * bit 1: the same inside awq_gemv. The output is then incomplete. 0 means
+ * no error was recorded. No kernel traps: a wait that gives up records the
+ * bit, lets its copies in flight land, frees what it holds and returns.
  */
 AWQ_API awq_status_t awq_device_error(uint32_t* error_word, void* stream);
 

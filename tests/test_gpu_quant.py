@@ -32,11 +32,13 @@ def check_quantize(W: np.ndarray, zp: bool, rows=None):
     torch.cuda.synchronize()
     Wr = W if rows is None else W[rows]
     codes, scales, zeros = O.pseudo_quantize(Wr, 128, zp)
-    sel = (lambda t: host(t)) if rows is None else (lambda t: host(t)[rows])
-    assert np.array_equal(bits(sel(qg)), bits(O.pack(codes))), "packed codes differ"
-    assert np.array_equal(bits(sel(sg)), bits(scales)), "scales differ"
+    # packed codes are [N, K/8]; scales and zero points are group-major [K/128, N]
+    sel_rows = (lambda t: host(t)) if rows is None else (lambda t: host(t)[rows])
+    sel_cols = (lambda t: host(t)) if rows is None else (lambda t: host(t)[:, rows])
+    assert np.array_equal(bits(sel_rows(qg)), bits(O.pack(codes))), "packed codes differ"
+    assert np.array_equal(bits(sel_cols(sg)), bits(scales)), "scales differ"
     if zp:
-        assert np.array_equal(bits(sel(zg)), bits(zeros)), "zero points differ"
+        assert np.array_equal(bits(sel_cols(zg)), bits(zeros)), "zero points differ"
     else:
         assert zg is None
     return qg, sg, zg
@@ -84,7 +86,7 @@ def test_dequant_roundtrip_of_gpu_codes(zp):
 def test_quantize_empty_rows_is_a_no_op():
     W = torch.empty((0, 256), dtype=torch.float16, device="cuda")
     q, s, z = awq.awq_pseudo_quantize_pack(W)
-    assert q.shape == (0, 32) and s.shape == (0, 2) and z.shape == (0, 2)
+    assert q.shape == (0, 32) and s.shape == (2, 0) and z.shape == (2, 0)
 
 
 def test_quantize_rejects_bad_group():

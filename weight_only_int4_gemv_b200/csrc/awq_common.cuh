@@ -106,12 +106,106 @@ __device__ __forceinline__ void decode_word_qz(uint32_t w, uint32_t zb1024, uint
   p[3] = hsub2_u32(lop3_and_or(w8, 0x00F000F0u, 0x54005400u), zb64);
 }
 
+// Codes of one packed word as four fp16 pairs without the zero point: the
+// pairs (0,1) and (4,5) come out as 1024 + q, the pairs (2,3) and (6,7) as
+// 64 + q (same masks and magic numbers as decode_word_qz). The offsets are
+// removed later in fp32, once per group, by the caller.
+__device__ __forceinline__ void decode_word_magic(uint32_t w, uint32_t (&p)[4]) {
+  const uint32_t w8 = w >> 8;
+  p[0] = lop3_and_or(w, 0x000F000Fu, 0x64006400u);
+  p[1] = lop3_and_or(w, 0x00F000F0u, 0x54005400u);
+  p[2] = lop3_and_or(w8, 0x000F000Fu, 0x64006400u);
+  p[3] = lop3_and_or(w8, 0x00F000F0u, 0x54005400u);
+}
+
 // (1024 + z) and (64 + z) in both fp16 halves for an integer zero point z.
 __device__ __forceinline__ void zero_bias_pairs(float z, uint32_t& zb1024, uint32_t& zb64) {
   const uint32_t a = __half_as_ushort(__float2half_rn(1024.0f + z));
   const uint32_t b = __half_as_ushort(__float2half_rn(64.0f + z));
   zb1024 = a | (a << 16);
   zb64 = b | (b << 16);
+}
+
+// ---------------------------------------------------------------------------
+// mbarrier / TMA wrappers (PTX ISA: mbarrier, cp.async.bulk(.tensor))
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t now_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s for any single wait
+
+// Wait for the phase of `parity` to complete. Gives up (returns false) when
+// *abort is set by another thread or the wait passes kWaitLimitNs, in which
+// case it sets *abort and ORs `err_bit` into *err.
+__device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                             uint32_t* err, uint32_t err_bit) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = now_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 63) == 0) {
+      if (*abort) return false;
+      if (now_ns() - t0 > kWaitLimitNs) {
+        *abort = 1;
+        atomicOr(err, err_bit);
+        return false;
+      }
+    }
+  }
+}
+
+// Bounded wait with no abort protocol (teardown of copies already issued).
+__device__ __forceinline__ void wait_teardown(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = now_ns();
+  while (!mbar_try_wait(bar, parity) && now_ns() - t0 < kWaitLimitNs) {
+  }
+}
+
+// 2-D tiled TMA load of one box into shared memory, completing on `bar`.
+__device__ __forceinline__ void tma_load_2d(void* dst, const void* tensor_map, int x, int y,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tensor_map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 }  // namespace awq

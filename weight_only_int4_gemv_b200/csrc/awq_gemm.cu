@@ -36,9 +36,9 @@
 #include <cudaTypedefs.h>
 
 #include <atomic>
-#include <mutex>
 
 #include "awq_common.cuh"
+#include "awq_tma_host.h"
 
 namespace awq {
 
@@ -62,8 +62,6 @@ constexpr int kBBytes = BN * BK * 2;        // 32 KB
 constexpr int kCBytes = BN * (BK / 8) * 4;  // 8 KB of packed codes
 constexpr int kSmemTiles = kStages * (kABytes + kBBytes + kCBytes);
 constexpr int kSmemBytes = kSmemTiles + 1024 /*barriers*/ + 1024 /*alignment*/;
-
-constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s per wait
 
 // instruction descriptor: F16 x F16 -> F32, both K-major, M = 128, N = 256
 constexpr uint32_t kIdesc = (1u << 4) | (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
@@ -90,73 +88,6 @@ struct Bars {
 // ---------------------------------------------------------------------------
 // PTX wrappers
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ uint64_t now_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
-               "r"(bytes)
-               : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Wait for the phase of `parity` to complete. Returns false when the CTA is
-// aborting or the wait ran past its limit (which starts the abort).
-__device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = now_ns();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63) == 0) {
-      if (*abort) return false;
-      if (now_ns() - t0 > kWaitLimitNs) {
-        *abort = 1;
-        atomicOr(&g_awq_error_word, 1u);
-        return false;
-      }
-    }
-  }
-}
-
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
-                                            uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
-      "[%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
-      : "memory");
-}
-
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -278,7 +209,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
           zero_bias_pairs(z, zb1024, zb64);
           sc2 = uint32_t(sb) | (uint32_t(sb) << 16);
         }
-        if (!wait_bounded(&bars->full_a[s], ph, abort)) { ok = false; break; }
+        if (!wait_bounded(&bars->full_a[s], ph, abort, &g_awq_error_word, 1u)) { ok = false; break; }
         // codes of row i: 32 bytes, 16-byte halves swapped on rows with bit 2 set (32B swizzle)
         const uint8_t* crow = smem + SmemLayout::c(s) + i * 32;
         const int sw = (i >> 2) & 1;
@@ -312,7 +243,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
       const int n0 = (tile / p.m_tiles) * BN;
       const int acc = it & 1;
       const uint32_t aph = (it >> 1) & 1;
-      if (!wait_bounded(&bars->tmem_full[acc], aph, abort)) break;
+      if (!wait_bounded(&bars->tmem_full[acc], aph, abort, &g_awq_error_word, 1u)) break;
       tc_fence_after();
       const int64_t m = int64_t(m0) + q * 32 + lane;
       uint16_t* yrow = p.y + m * p.N;
@@ -355,7 +286,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         const int m0 = (tile % p.m_tiles) * BM;
         const int n0 = (tile / p.m_tiles) * BN;
         for (int kb = 0; kb < p.k_blocks; ++kb) {
-          if (!wait_bounded(&bars->empty[s], ph ^ 1, abort)) { ok = false; break; }
+          if (!wait_bounded(&bars->empty[s], ph ^ 1, abort, &g_awq_error_word, 1u)) { ok = false; break; }
           mbar_arrive_expect_tx(&bars->full_a[s], kABytes + kCBytes);
           tma_load_2d(smem + SmemLayout::a(s), &tmap_x, kb * BK, m0, &bars->full_a[s]);
           tma_load_2d(smem + SmemLayout::c(s), &tmap_q, kb * (BK / 8), n0, &bars->full_a[s]);
@@ -366,10 +297,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
       }
       // The copies still in flight land before the CTA's shared memory goes away.
       for (int t = 0; t < kStages; ++t)
-        if (issued[t]) {
-          const uint64_t t0 = now_ns();
-          while (!mbar_try_wait(&bars->full_a[t], issued_ph[t]) && now_ns() - t0 < kWaitLimitNs) {}
-        }
+        if (issued[t]) wait_teardown(&bars->full_a[t], issued_ph[t]);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
@@ -381,12 +309,12 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
         const int acc = it & 1;
         const uint32_t aph = (it >> 1) & 1;
-        if (!wait_bounded(&bars->tmem_empty[acc], aph ^ 1, abort)) break;
+        if (!wait_bounded(&bars->tmem_empty[acc], aph ^ 1, abort, &g_awq_error_word, 1u)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + uint32_t(acc * BN);
         for (int kb = 0; kb < p.k_blocks; ++kb) {
-          if (!wait_bounded(&bars->full_a[s], ph, abort) ||
-              !wait_bounded(&bars->full_b[s], ph, abort)) { ok = false; break; }
+          if (!wait_bounded(&bars->full_a[s], ph, abort, &g_awq_error_word, 1u) ||
+              !wait_bounded(&bars->full_b[s], ph, abort, &g_awq_error_word, 1u)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + SmemLayout::a(s));
           const uint32_t b_addr = smem_u32(smem + SmemLayout::b(s));
@@ -401,8 +329,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
       }
       // every MMA this thread issued completes before tensor memory is freed
       tc_commit(&bars->mma_done);
-      const uint64_t t0 = now_ns();
-      while (!mbar_try_wait(&bars->mma_done, 0) && now_ns() - t0 < kWaitLimitNs) {}
+      wait_teardown(&bars->mma_done, 0);
     }
   }
 
@@ -418,25 +345,13 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
-std::once_flag g_encode_once;
-
-PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
-  std::call_once(g_encode_once, [] {
-    void* fn = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-  });
-  return g_encode;
-}
-
 constexpr int kMaxDevices = 64;
 std::atomic<int> g_sms[kMaxDevices];
 std::atomic<int> g_attr_set[kMaxDevices][2];
 
 }  // namespace
+
+awq_status_t gemv_take_error(uint32_t* word, cudaStream_t s);
 
 awq_status_t gemm_workspace_bytes(int64_t, int64_t, int64_t, bool, size_t* bytes) {
   *bytes = 0;
@@ -465,8 +380,6 @@ extern "C" awq_status_t awq_gemm(const uint16_t* x, const int32_t* qweight,
       (zeros && !aligned16(zeros)))
     return AWQ_ERR_ALIGN;
 
-  PFN_cuTensorMapEncodeTiled_v12000 encode = get_encode();
-  if (!encode) return AWQ_ERR_CUDA;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return AWQ_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return AWQ_ERR_UNSUPPORTED;
@@ -486,28 +399,13 @@ extern "C" awq_status_t awq_gemm(const uint16_t* x, const int32_t* qweight,
   }
 
   // x: fp16 [M][K], box 64 (k) x 128 (rows), 128-byte swizzle; rows past M read as 0.
-  CUtensorMap tmap_x, tmap_q;
-  {
-    const cuuint64_t dims[2] = {cuuint64_t(K), cuuint64_t(M)};
-    const cuuint64_t strides[1] = {cuuint64_t(K) * 2};
-    const cuuint32_t box[2] = {BK, BM};
-    const cuuint32_t estr[2] = {1, 1};
-    if (encode(&tmap_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<uint16_t*>(x), dims, strides,
-               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return AWQ_ERR_CUDA;
-  }
   // codes: int32 [N][K/8], box 8 words x 256 rows, 32-byte swizzle; rows past N read as 0.
-  {
-    const cuuint64_t dims[2] = {cuuint64_t(K / 8), cuuint64_t(N)};
-    const cuuint64_t strides[1] = {cuuint64_t(K / 8) * 4};
-    const cuuint32_t box[2] = {BK / 8, BN};
-    const cuuint32_t estr[2] = {1, 1};
-    if (encode(&tmap_q, CU_TENSOR_MAP_DATA_TYPE_INT32, 2, const_cast<int32_t*>(qweight), dims,
-               strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return AWQ_ERR_CUDA;
-  }
+  CUtensorMap tmap_x, tmap_q;
+  if (!make_tensor_map_2d(&tmap_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x, uint64_t(K), uint64_t(M),
+                          uint64_t(K) * 2, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tensor_map_2d(&tmap_q, CU_TENSOR_MAP_DATA_TYPE_INT32, qweight, uint64_t(K / 8), uint64_t(N),
+                          uint64_t(K / 8) * 4, BK / 8, BN, CU_TENSOR_MAP_SWIZZLE_32B))
+    return AWQ_ERR_CUDA;
   GemmParams p;
   p.y = y;
   p.scales = scales;
@@ -529,8 +427,8 @@ extern "C" awq_status_t awq_gemm(const uint16_t* x, const int32_t* qweight,
 extern "C" awq_status_t awq_device_error(uint32_t* error_word, void* stream) {
   if (!error_word) return AWQ_ERR_NULL;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  uint32_t zero = 0;
-  if (cudaMemcpyFromSymbolAsync(error_word, g_awq_error_word, sizeof(uint32_t), 0,
+  uint32_t gemm_word = 0, gemv_word = 0, zero = 0;
+  if (cudaMemcpyFromSymbolAsync(&gemm_word, g_awq_error_word, sizeof(uint32_t), 0,
                                 cudaMemcpyDeviceToHost, s) != cudaSuccess)
     return AWQ_ERR_CUDA;
   if (cudaStreamSynchronize(s) != cudaSuccess) return AWQ_ERR_CUDA;
@@ -538,5 +436,8 @@ extern "C" awq_status_t awq_device_error(uint32_t* error_word, void* stream) {
                               s) != cudaSuccess)
     return AWQ_ERR_CUDA;
   if (cudaStreamSynchronize(s) != cudaSuccess) return AWQ_ERR_CUDA;
+  awq_status_t st = gemv_take_error(&gemv_word, s);
+  if (st != AWQ_OK) return st;
+  *error_word = gemm_word | gemv_word;
   return AWQ_OK;
 }

@@ -5,74 +5,68 @@
 // matmul and never written back as fp16.)
 //
 // The layer is bound by HBM: every packed code byte is read once and feeds
-// only M multiply-adds, so the kernel is built around keeping enough bytes
-// in flight on every SM.
+// only M multiply-adds. Design:
 //
 // * Work unit = (row block of 16*RT output channels, one group of 128 k).
 //   Units are ordered block-major and split evenly over every warp of a grid
 //   sized to the resident capacity of the GPU (a stream-K split): all SMs
 //   stream the same number of bytes whatever N and K are.
-// * Each warp owns an S-stage ring in shared memory and fills it with 16-byte
-//   cp.async copies S-1 units ahead of the arithmetic: the unit's packed
-//   codes (lane (g, t) copies 16 bytes of rows g and g+8 of each 16-row
-//   tile, the bytes it will decode itself), the 16-row runs of scales and
-//   zero points (group-major metadata makes them contiguous), and the
-//   unit's slice of x (128 k of every batch row, 16-byte chunks swizzled so
-//   the fragment reads are free of bank conflicts).
+// * Each warp owns an S-stage ring in shared memory. Lane 0 fills a stage
+//   with TMA: one 2-D box of packed codes (16*RT rows x 64 bytes), one box
+//   of x (M rows x 128 k), and the 16*RT-long runs of scales and zero points
+//   (group-major metadata makes them contiguous), all completing on the
+//   stage's mbarrier. Units S-1 ahead of the arithmetic stay in flight
+//   without holding registers or L1 request slots.
 // * Decode: the packed nibble order puts consecutive k pairs in the low and
-//   high halves of a word, so one LOP3 turns a word into two fp16 values
-//   1024+q (or 64+q) and one HSUB2 subtracts 1024+z (64+z), leaving q - z
-//   exactly.
+//   high halves of a word, so one LOP3 turns a word into two exact fp16
+//   integers, 1024+q for the pairs (0,1), (4,5) and 64+q for (2,3), (6,7):
+//   five instructions per eight weights.
 // * Multiply: the decoded 16x16 weight tile is the A operand of
 //   mma.m16n8k16 straight from registers; x is the B operand (batch in the
 //   n dimension, two n8 tiles for M > 8). The k positions inside an MMA are
 //   a permutation of the word's k (each lane owns whole words), matched by
 //   reading x[m][8w .. 8w+7] for the same words: one 16-byte read covers two
-//   MMAs. Accumulation is fp32.
-// * The scale is applied once per group: sum_k x (q - z) s = s * sum_k x (q - z).
+//   MMAs. Products are exact and accumulation is fp32. The RT row tiles are
+//   independent accumulator chains, interleaved.
+// * Offsets and scale, once per group and batch row, in fp32:
+//   sum_k x (q - z) = raw - C(m) - z S(m), with raw the MMA sum over the
+//   magic-offset values, C(m) = 1024 sum_{k: 1024 pairs} x + 64 sum_{k: 64
+//   pairs} x and S(m) = sum_k x. C and S come from two more MMAs against a
+//   constant tile (rows 0 and 1), shared by all rows of the unit. Then
+//   acc += s (raw - C - z S): the scale multiplies the group's partial sum.
 // * A row block split between warps is finished by the last warp to arrive
 //   (arrival counter per block): it sums the contributors' fp32 partials in
 //   a fixed order, so results do not depend on timing, and resets the
 //   counter for the next call. No warp ever waits on another.
+// * Every mbarrier wait is bounded (2 s); a warp that gives up records bit 1
+//   of the device error word, waits (bounded) for its copies in flight and
+//   leaves its rows unwritten.
 
 #include <atomic>
 
 #include "awq_common.cuh"
+#include "awq_tma_host.h"
 
 namespace awq {
+
+__device__ uint32_t g_awq_gemv_error = 0;
+
 namespace {
 
-constexpr int kGemvWarps = 8;
+constexpr int kGemvWarps = 4;
 constexpr int kGemvThreads = kGemvWarps * 32;
+constexpr int kBarRegion = 1024;   // mbarriers of all warps, ahead of the rings
 
 struct GemvParams {
-  const uint16_t* x;
-  const int32_t* qweight;
-  const uint16_t* scales;
-  const uint16_t* zeros;
   uint16_t* y;
-  float* partials;       // [total_warps][2][slot floats]
+  float* partials;       // [total_warps][2][32 lanes][RT*MT*4]
   uint32_t* counters;    // [nb]
   int64_t units;         // nb * G
   int M, N, K, G, nb, total_warps;
-  int stage_bytes;       // codes + metadata + x slice of one unit
+  int stage_bytes;       // codes + metadata + x slice of one unit (multiple of 128)
   int x_offset;          // offset of the x slice inside a stage
+  uint32_t tx_bytes;     // bytes the TMA copies of one unit deliver
 };
-
-__device__ __forceinline__ uint32_t smem_addr(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-// 16-byte async copy global -> shared; src_bytes = 0 writes zeros.
-__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
 
 __device__ __forceinline__ uint4 lds128(const uint8_t* p) { return *reinterpret_cast<const uint4*>(p); }
 __device__ __forceinline__ uint16_t lds16(const uint8_t* p) { return *reinterpret_cast<const uint16_t*>(p); }
@@ -89,22 +83,6 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a
 __device__ __forceinline__ uint32_t word_of(const uint4& v, int i) {
   return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
-
-// (1024 + z, 1024 + z) and (64 + z, 64 + z) from the fp16 bits of an
-// integer zero point z in 0..15: both sums are exact in fp16.
-__device__ __forceinline__ void zero_bias_from_bits(uint16_t zbits, uint32_t& zb1024, uint32_t& zb64) {
-  const uint32_t zz = uint32_t(zbits) | (uint32_t(zbits) << 16);
-  uint32_t a, b;
-  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(a) : "r"(zz), "r"(0x64006400u));
-  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(b) : "r"(zz), "r"(0x54005400u));
-  zb1024 = a;
-  zb64 = b;
-}
-
-// Position of 16-byte chunk c (0..15) of batch row m inside a stage's x
-// slice: spreads the 8 lanes of each quarter-warp fragment read over all
-// 32 banks.
-__device__ __forceinline__ int x_chunk_pos(int m, int c) { return c ^ ((c >> 3) & 1) ^ ((m & 1) << 1); }
 
 // First unit of warp w in the even split of `units` over `warps`.
 __device__ __forceinline__ int64_t warp_start(int64_t units, int64_t w, int64_t warps) {
@@ -134,6 +112,8 @@ __device__ __forceinline__ void store_y(const GemvParams& p, int64_t row0, int g
 }
 
 // Finish row block b after this warp summed groups [j0, j1) of it.
+// Partials are stored lane-major ([lane][RT*MT*4] floats) so each lane moves
+// its values with 16-byte accesses.
 template <int MT, int RT>
 __device__ __forceinline__ void finish_block(const GemvParams& p, int64_t b, int j0, int j1, int64_t gw,
                                              int64_t first_block, int lane, int g, int t,
@@ -144,62 +124,95 @@ __device__ __forceinline__ void finish_block(const GemvParams& p, int64_t b, int
     store_y<MT, RT>(p, row0, g, t, acc);
     return;
   }
-  // Partial block: publish this warp's fp32 sums, count its groups in.
-  constexpr int kSlot = RT * MT * 4 * 32;
+  constexpr int kVals = RT * MT * 4;           // floats per lane
+  constexpr int kVec = kVals / 4;              // float4 per lane
+  constexpr int kSlot = kVals * 32;
   const int slot = (b == first_block) ? 0 : 1;
-  float* sp = p.partials + (gw * 2 + slot) * kSlot;
-  int idx = 0;
+  float4* sp = reinterpret_cast<float4*>(p.partials + (gw * 2 + slot) * kSlot) + lane * kVec;
 #pragma unroll
   for (int rt = 0; rt < RT; ++rt)
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-      for (int i = 0; i < 4; ++i, ++idx) __stcg(sp + idx * 32 + lane, acc[rt][mt][i]);
-  __threadfence();
-  __syncwarp();
+      __stcg(sp + rt * MT + mt, make_float4(acc[rt][mt][0], acc[rt][mt][1], acc[rt][mt][2], acc[rt][mt][3]));
+  __syncwarp();   // every lane's stores happen before lane 0's release below
   uint32_t last = 0;
   if (lane == 0) {
     const uint32_t mine = uint32_t(j1 - j0);
-    const uint32_t old = atomicAdd(p.counters + b, mine);
+    uint32_t old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;"
+                 : "=r"(old) : "l"(p.counters + b), "r"(mine) : "memory");
     last = (old + mine == uint32_t(G)) ? 1u : 0u;
   }
   last = __shfl_sync(0xffffffffu, last, 0);
   if (!last) return;
-  __threadfence();
-  // contributors: every non-empty warp range overlapping block b, in warp order
+  // Sum every contributor in warp order (fixed order: reproducible bits),
+  // four contributors' loads in flight at a time.
   const int64_t W = p.total_warps;
   const int64_t w_first = ((b * G + 1) * W - 1) / p.units;
   const int64_t w_last = ((b * G + G) * W - 1) / p.units;
-  float tot[RT][MT][4];
+  float4 tot[kVec];
+#pragma unroll
+  for (int v = 0; v < kVec; ++v) tot[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int64_t w0 = w_first; w0 <= w_last; w0 += 4) {
+    float4 part[4][kVec];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int64_t w = w0 + c;
+      const int64_t ws = warp_start(p.units, w, W);
+      const bool live = w <= w_last && ws < warp_start(p.units, w + 1, W);   // skip empty ranges
+      const int s = (ws / G == b) ? 0 : 1;
+      const float4* rp = reinterpret_cast<const float4*>(p.partials + (w * 2 + s) * kSlot) + lane * kVec;
+#pragma unroll
+      for (int v = 0; v < kVec; ++v) part[c][v] = live ? __ldcg(rp + v) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+#pragma unroll
+      for (int v = 0; v < kVec; ++v) {
+        tot[v].x += part[c][v].x;
+        tot[v].y += part[c][v].y;
+        tot[v].z += part[c][v].z;
+        tot[v].w += part[c][v].w;
+      }
+  }
+  float sum[RT][MT][4];
 #pragma unroll
   for (int rt = 0; rt < RT; ++rt)
 #pragma unroll
-    for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) tot[rt][mt][i] = 0.0f;
-  for (int64_t w = w_first; w <= w_last; ++w) {
-    const int64_t ws = warp_start(p.units, w, W);
-    if (ws >= warp_start(p.units, w + 1, W)) continue;   // empty range
-    const int s = (ws / G == b) ? 0 : 1;
-    const float* rp = p.partials + (w * 2 + s) * kSlot;
-    int k = 0;
-#pragma unroll
-    for (int rt = 0; rt < RT; ++rt)
-#pragma unroll
-      for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-        for (int i = 0; i < 4; ++i, ++k) tot[rt][mt][i] += __ldcg(rp + k * 32 + lane);
-  }
-  store_y<MT, RT>(p, row0, g, t, tot);
+    for (int mt = 0; mt < MT; ++mt) {
+      const float4 v = tot[rt * MT + mt];
+      sum[rt][mt][0] = v.x;
+      sum[rt][mt][1] = v.y;
+      sum[rt][mt][2] = v.z;
+      sum[rt][mt][3] = v.w;
+    }
+  store_y<MT, RT>(p, row0, g, t, sum);
   if (lane == 0) p.counters[b] = 0u;
 }
 
+// A fragment of the constant 16x16 tile that turns two extra MMAs into the
+// per-batch-row sums the decode offsets need: row 0 holds 1024 at the k
+// slots fed by (1024 + q) pairs and 64 at the slots fed by (64 + q) pairs,
+// row 1 holds 1; every other row is 0. Lane (g, t) owns rows g and g+8.
+__device__ __forceinline__ void offset_tile(int g, uint32_t& a0, uint32_t& a2) {
+  a0 = g == 0 ? 0x64006400u : (g == 1 ? 0x3C003C00u : 0u);
+  a2 = g == 0 ? 0x54005400u : (g == 1 ? 0x3C003C00u : 0u);
+}
+
+template <int RT>
+struct StageLayout {
+  static constexpr int kCodeBytes = 16 * RT * 64;   // [16*RT rows][16 words]
+  static constexpr int kMetaBytes = 16 * RT * 2;    // one fp16 per row of the block
+  static constexpr int kMetaStride = (kMetaBytes + 127) / 128 * 128;
+};
+
 template <int MT, int RT, bool ZP, int S>
 __global__ void __launch_bounds__(kGemvThreads)
-gemv_kernel(const GemvParams p) {
-  extern __shared__ __align__(16) uint8_t gemv_smem[];
-  constexpr int kCodeBytes = RT * 2 * 32 * 16;   // [rt][row half][lane] x 16 B
-  constexpr int kMetaBytes = RT * 16 * 2;         // one fp16 per row of the block
+gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_x,
+            const __grid_constant__ CUtensorMap tmap_s, const __grid_constant__ CUtensorMap tmap_z,
+            const GemvParams p) {
+  extern __shared__ __align__(1024) uint8_t gemv_smem[];
+  using L = StageLayout<RT>;
   const int lane = threadIdx.x & 31;
   const int g = lane >> 2;
   const int t = lane & 3;
@@ -211,48 +224,48 @@ gemv_kernel(const GemvParams p) {
   const int64_t u_end = warp_start(p.units, gw + 1, W);
   if (u_begin >= u_end) return;
   const int stage_bytes = p.stage_bytes;
-  uint8_t* ring = gemv_smem + int64_t(wi) * S * stage_bytes;
-  const uint32_t ring_s = smem_addr(ring);
-  const int64_t words_per_row = p.K / 8;
-  const int x_chunks = p.M * 16;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(gemv_smem) + wi * S;
+  uint8_t* ring = gemv_smem + kBarRegion + wi * S * stage_bytes;
 
+  if (lane == 0) {
+#pragma unroll
+    for (int i = 0; i < S; ++i) mbar_init(&bars[i], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    fence_proxy_async_smem();
+  }
+  __syncwarp();
+
+  // lane 0: fill `slot` with unit u (codes box, x box, scale and zero runs)
   auto issue = [&](int64_t u, int slot) {
     if (u < u_end) {
       const int64_t b = u / G;
-      const int64_t j = u - b * G;
-      const int64_t r0 = b * (16 * RT);
-      const uint32_t st = ring_s + uint32_t(slot * stage_bytes);
-#pragma unroll
-      for (int rt = 0; rt < RT; ++rt)
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int64_t row = r0 + 16 * rt + 8 * h + g;
-          const bool v = row < p.N;
-          const int32_t* src = p.qweight + (v ? row : 0) * words_per_row + j * kWordsPerGroup + t * 4;
-          cp_async_16(st + uint32_t(((rt * 2 + h) * 32 + lane) * 16), src, v ? 16u : 0u);
-        }
-      constexpr int kMetaLanes = 2 * RT * (ZP ? 2 : 1);
-      if (lane < kMetaLanes) {   // runs of 8 rows: N % 8 == 0 makes each run all in or all out
-        const int which = lane / (2 * RT);   // 0 scales, 1 zero points
-        const int rt = (lane >> 1) % RT;
-        const int h = lane & 1;
-        const int64_t rowc = r0 + 16 * rt + 8 * h;
-        const bool v = rowc < p.N;
-        const uint16_t* src = (which ? p.zeros : p.scales) + j * p.N + (v ? rowc : 0);
-        cp_async_16(st + uint32_t(kCodeBytes + which * kMetaBytes + (rt * 16 + 8 * h) * 2), src, v ? 16u : 0u);
-      }
-      for (int c = lane; c < x_chunks; c += 32) {
-        const int m = c >> 4;
-        const int cc = c & 15;
-        const uint16_t* src = p.x + int64_t(m) * p.K + j * kGroup + cc * 8;
-        cp_async_16(st + uint32_t(p.x_offset + m * 256 + x_chunk_pos(m, cc) * 16), src, 16u);
-      }
+      const int j = int(u - b * G);
+      const int r0 = int(b * (16 * RT));
+      uint8_t* st = ring + slot * stage_bytes;
+      mbar_arrive_expect_tx(&bars[slot], p.tx_bytes);
+      tma_load_2d(st, &tmap_q, j * kWordsPerGroup, r0, &bars[slot]);
+      tma_load_2d(st + p.x_offset, &tmap_x, j * kGroup, 0, &bars[slot]);
+      tma_load_2d(st + L::kCodeBytes, &tmap_s, r0, j, &bars[slot]);
+      if (ZP) tma_load_2d(st + L::kCodeBytes + L::kMetaStride, &tmap_z, r0, j, &bars[slot]);
     }
-    cp_async_commit();   // one group per unit, empty past the range, so counts stay uniform
   };
-
+  if (lane == 0) {
 #pragma unroll
-  for (int i = 0; i < S - 1; ++i) issue(u_begin + i, i);
+    for (int i = 0; i < S - 1; ++i) issue(u_begin + i, i);
+  }
+
+  // x fragment offsets inside a stage: batch row m = 8 mt + g, chunk 4t + jj
+  int xoff[MT];
+  bool xok[MT];
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt) {
+    const int m = 8 * mt + g;
+    xok[mt] = m < p.M;
+    xoff[mt] = p.x_offset + m * 256 + t * 64;
+  }
+  uint32_t ca0, ca2;
+  offset_tile(g, ca0, ca2);
+  volatile int abort_flag = 0;
 
   const int64_t first_block = u_begin / G;
   int64_t cur_b = first_block;
@@ -266,10 +279,13 @@ gemv_kernel(const GemvParams p) {
       for (int i = 0; i < 4; ++i) acc[rt][mt][i] = 0.0f;
 
   int slot = 0;
-  for (int64_t u = u_begin; u < u_end; ++u) {
-    issue(u + S - 1, slot == 0 ? S - 1 : slot - 1);
-    cp_async_wait<S - 1>();
-    __syncwarp();   // metadata and x were copied by other lanes
+  uint32_t phase = 0;
+  bool ok = true;
+  int64_t u = u_begin;
+  for (; u < u_end; ++u) {
+    if (lane == 0) issue(u + S - 1, slot == 0 ? S - 1 : slot - 1);
+    const bool got = wait_bounded(&bars[slot], phase, &abort_flag, &g_awq_gemv_error, 2u);
+    if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
     const int64_t b = u / G;
     if (b != cur_b) {
       finish_block<MT, RT>(p, cur_b, jstart, int(G), gw, first_block, lane, g, t, acc);
@@ -284,65 +300,103 @@ gemv_kernel(const GemvParams p) {
     }
     const uint8_t* st = ring + slot * stage_bytes;
 
+    // x fragments and packed codes of the unit
     uint4 xf[MT][4];
 #pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
-      const int m = 8 * mt + g;
+    for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj)
-        xf[mt][jj] = m < p.M ? lds128(st + p.x_offset + m * 256 + x_chunk_pos(m, 4 * t + jj) * 16)
-                             : make_uint4(0, 0, 0, 0);
-    }
-
+      for (int jj = 0; jj < 4; ++jj) xf[mt][jj] = xok[mt] ? lds128(st + xoff[mt] + jj * 16) : make_uint4(0, 0, 0, 0);
+    uint4 c_lo[RT], c_hi[RT];
 #pragma unroll
     for (int rt = 0; rt < RT; ++rt) {
-      const uint4 c_lo = lds128(st + ((rt * 2 + 0) * 32 + lane) * 16);
-      const uint4 c_hi = lds128(st + ((rt * 2 + 1) * 32 + lane) * 16);
-      const float s_lo = half_bits_to_float(lds16(st + kCodeBytes + (rt * 16 + g) * 2));
-      const float s_hi = half_bits_to_float(lds16(st + kCodeBytes + (rt * 16 + 8 + g) * 2));
-      uint32_t zl1024, zl64, zh1024, zh64;
-      if (ZP) {
-        zero_bias_from_bits(lds16(st + kCodeBytes + kMetaBytes + (rt * 16 + g) * 2), zl1024, zl64);
-        zero_bias_from_bits(lds16(st + kCodeBytes + kMetaBytes + (rt * 16 + 8 + g) * 2), zh1024, zh64);
-      } else {
-        zl1024 = zh1024 = 0x64086408u;   // 1032 = 1024 + 8
-        zl64 = zh64 = 0x54805480u;       // 72 = 64 + 8
+      c_lo[rt] = lds128(st + (16 * rt + g) * 64 + t * 16);
+      c_hi[rt] = lds128(st + (16 * rt + 8 + g) * 64 + t * 16);
+    }
+
+    float grp[RT][MT][4];
+    float cs[MT][4];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        cs[mt][i] = 0.0f;
+#pragma unroll
+        for (int rt = 0; rt < RT; ++rt) grp[rt][mt][i] = 0.0f;
       }
-      float grp[MT][4];
 #pragma unroll
-      for (int mt = 0; mt < MT; ++mt)
+    for (int jj = 0; jj < 4; ++jj) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) grp[mt][i] = 0.0f;
+      for (int mt = 0; mt < MT; ++mt) {
+        mma_16816(cs[mt], ca0, 0u, ca2, 0u, xf[mt][jj].x, xf[mt][jj].y);
+        mma_16816(cs[mt], ca0, 0u, ca2, 0u, xf[mt][jj].z, xf[mt][jj].w);
+      }
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj) {
+      for (int rt = 0; rt < RT; ++rt) {
         uint32_t plo[4], phi[4];
-        decode_word_qz(word_of(c_lo, jj), zl1024, zl64, plo);
-        decode_word_qz(word_of(c_hi, jj), zh1024, zh64, phi);
+        decode_word_magic(word_of(c_lo[rt], jj), plo);
+        decode_word_magic(word_of(c_hi[rt], jj), phi);
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt) {
-          mma_16816(grp[mt], plo[0], phi[0], plo[1], phi[1], xf[mt][jj].x, xf[mt][jj].y);
-          mma_16816(grp[mt], plo[2], phi[2], plo[3], phi[3], xf[mt][jj].z, xf[mt][jj].w);
+          mma_16816(grp[rt][mt], plo[0], phi[0], plo[1], phi[1], xf[mt][jj].x, xf[mt][jj].y);
+          mma_16816(grp[rt][mt], plo[2], phi[2], plo[3], phi[3], xf[mt][jj].z, xf[mt][jj].w);
         }
+      }
+    }
+    // row 0 of the constant tile (lanes 0..3) holds C, row 1 (lanes 4..7) holds S
+    float cm[MT][2], sm[MT][2];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      cm[mt][0] = __shfl_sync(0xffffffffu, cs[mt][0], t);
+      cm[mt][1] = __shfl_sync(0xffffffffu, cs[mt][1], t);
+      sm[mt][0] = __shfl_sync(0xffffffffu, cs[mt][0], 4 + t);
+      sm[mt][1] = __shfl_sync(0xffffffffu, cs[mt][1], 4 + t);
+    }
+    // sum_k x (q - z) = raw - C(m) - z S(m); then the group's scale
+#pragma unroll
+    for (int rt = 0; rt < RT; ++rt) {
+      const float s_lo = half_bits_to_float(lds16(st + L::kCodeBytes + (16 * rt + g) * 2));
+      const float s_hi = half_bits_to_float(lds16(st + L::kCodeBytes + (16 * rt + 8 + g) * 2));
+      float z_lo = 8.0f, z_hi = 8.0f;
+      if (ZP) {
+        z_lo = half_bits_to_float(lds16(st + L::kCodeBytes + L::kMetaStride + (16 * rt + g) * 2));
+        z_hi = half_bits_to_float(lds16(st + L::kCodeBytes + L::kMetaStride + (16 * rt + 8 + g) * 2));
       }
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) {
-        acc[rt][mt][0] = fmaf(s_lo, grp[mt][0], acc[rt][mt][0]);
-        acc[rt][mt][1] = fmaf(s_lo, grp[mt][1], acc[rt][mt][1]);
-        acc[rt][mt][2] = fmaf(s_hi, grp[mt][2], acc[rt][mt][2]);
-        acc[rt][mt][3] = fmaf(s_hi, grp[mt][3], acc[rt][mt][3]);
+        acc[rt][mt][0] = fmaf(s_lo, fmaf(-z_lo, sm[mt][0], grp[rt][mt][0] - cm[mt][0]), acc[rt][mt][0]);
+        acc[rt][mt][1] = fmaf(s_lo, fmaf(-z_lo, sm[mt][1], grp[rt][mt][1] - cm[mt][1]), acc[rt][mt][1]);
+        acc[rt][mt][2] = fmaf(s_hi, fmaf(-z_hi, sm[mt][0], grp[rt][mt][2] - cm[mt][0]), acc[rt][mt][2]);
+        acc[rt][mt][3] = fmaf(s_hi, fmaf(-z_hi, sm[mt][1], grp[rt][mt][3] - cm[mt][1]), acc[rt][mt][3]);
       }
     }
-    __syncwarp();   // every lane is done with the slot before it is refilled
-    slot = (slot + 1 == S) ? 0 : slot + 1;
+    __syncwarp();   // every lane is done with the slot before lane 0 refills it
+    if (++slot == S) {
+      slot = 0;
+      phase ^= 1u;
+    }
   }
-  finish_block<MT, RT>(p, cur_b, jstart, int(u_end - cur_b * G), gw, first_block, lane, g, t, acc);
-  cp_async_wait<0>();
+  if (ok) {
+    finish_block<MT, RT>(p, cur_b, jstart, int(u_end - cur_b * G), gw, first_block, lane, g, t, acc);
+  } else if (lane == 0) {
+    // Gave up: let the copies already issued for units u .. u+S-1 land
+    // before this warp's shared memory can be reused.
+    int s = slot;
+    uint32_t ph = phase;
+    for (int64_t v = u; v < u_end && v < u + S; ++v) {
+      wait_teardown(&bars[s], ph);
+      if (++s == S) {
+        s = 0;
+        ph ^= 1u;
+      }
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------
 // host side: plan (variant, grid, workspace) for a shape
 // ---------------------------------------------------------------------------
-using KernelFn = void (*)(const GemvParams);
+using KernelFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap,
+                          const GemvParams);
 
 struct Variant {
   KernelFn fn;
@@ -353,20 +407,33 @@ constexpr int kNumVariants = 4;
 
 Variant pick_variant(int64_t M, bool zp) {
   if (M <= 8)
-    return zp ? Variant{gemv_kernel<1, 2, true, 4>, 1, 2, 4, 0} : Variant{gemv_kernel<1, 2, false, 4>, 1, 2, 4, 1};
-  return zp ? Variant{gemv_kernel<2, 2, true, 3>, 2, 2, 3, 2} : Variant{gemv_kernel<2, 2, false, 3>, 2, 2, 3, 3};
+    return zp ? Variant{gemv_kernel<1, 4, true, 4>, 1, 4, 4, 0} : Variant{gemv_kernel<1, 4, false, 4>, 1, 4, 4, 1};
+  return zp ? Variant{gemv_kernel<2, 4, true, 3>, 2, 4, 3, 2} : Variant{gemv_kernel<2, 4, false, 3>, 2, 4, 3, 3};
 }
 
-int stage_bytes_for(const Variant& v, int64_t M, bool zp) {
-  return v.rt * 2 * 32 * 16 + v.rt * 16 * 2 * (zp ? 2 : 1) + int(M) * 256;
+int round128(int v) { return (v + 127) / 128 * 128; }
+
+struct StageGeometry {
+  int code_bytes, meta_stride, x_offset, stage_bytes;
+  uint32_t tx_bytes;
+};
+
+StageGeometry stage_geometry(const Variant& v, int64_t M, bool zp) {
+  StageGeometry sg;
+  sg.code_bytes = 16 * v.rt * 64;
+  sg.meta_stride = round128(16 * v.rt * 2);
+  sg.x_offset = sg.code_bytes + sg.meta_stride * (zp ? 2 : 1);
+  sg.stage_bytes = round128(sg.x_offset + int(M) * 256);
+  sg.tx_bytes = uint32_t(sg.code_bytes + 16 * v.rt * 2 * (zp ? 2 : 1) + int(M) * 256);
+  return sg;
 }
 
 struct Plan {
   Variant v;
+  StageGeometry sg;
   int grid;
   int nb;
   int smem;
-  int stage_bytes;
   int64_t units;
   size_t counter_bytes;
   size_t partial_bytes;
@@ -382,8 +449,8 @@ awq_status_t make_plan(int64_t M, int64_t N, int64_t K, bool zp, Plan& pl) {
   if (cudaGetDevice(&dev) != cudaSuccess) return AWQ_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return AWQ_ERR_UNSUPPORTED;
   pl.v = pick_variant(M, zp);
-  pl.stage_bytes = stage_bytes_for(pl.v, M, zp);
-  pl.smem = kGemvWarps * pl.v.stages * pl.stage_bytes;
+  pl.sg = stage_geometry(pl.v, M, zp);
+  pl.smem = kBarRegion + kGemvWarps * pl.v.stages * pl.sg.stage_bytes;
   int sms = g_sm_count[dev].load(std::memory_order_relaxed);
   if (sms == 0) {
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
@@ -392,7 +459,7 @@ awq_status_t make_plan(int64_t M, int64_t N, int64_t K, bool zp, Plan& pl) {
   }
   if (!g_smem_attr[dev][pl.v.id].load(std::memory_order_acquire)) {
     // the largest ring any M asks of this variant
-    const int most = kGemvWarps * pl.v.stages * stage_bytes_for(pl.v, pl.v.mt * 8, zp);
+    const int most = kBarRegion + kGemvWarps * pl.v.stages * stage_geometry(pl.v, pl.v.mt * 8, zp).stage_bytes;
     if (cudaFuncSetAttribute(pl.v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, most) != cudaSuccess)
       return AWQ_ERR_CUDA;
     g_smem_attr[dev][pl.v.id].store(1, std::memory_order_release);
@@ -453,6 +520,19 @@ awq_status_t gemv_workspace_bytes(int64_t M, int64_t N, int64_t K, bool zp, size
   return AWQ_OK;
 }
 
+// Read and clear this file's device error word (stream-ordered).
+awq_status_t gemv_take_error(uint32_t* word, cudaStream_t s) {
+  uint32_t zero = 0;
+  if (cudaMemcpyFromSymbolAsync(word, g_awq_gemv_error, sizeof(uint32_t), 0, cudaMemcpyDeviceToHost, s) !=
+      cudaSuccess)
+    return AWQ_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return AWQ_ERR_CUDA;
+  if (cudaMemcpyToSymbolAsync(g_awq_gemv_error, &zero, sizeof(uint32_t), 0, cudaMemcpyHostToDevice, s) !=
+      cudaSuccess)
+    return AWQ_ERR_CUDA;
+  return cudaStreamSynchronize(s) == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA;
+}
+
 }  // namespace awq
 
 using namespace awq;
@@ -463,13 +543,10 @@ extern "C" awq_status_t awq_gemv(const uint16_t* x, const int32_t* qweight,
                                  void* workspace, size_t workspace_bytes, void* stream) {
   awq_status_t st = check_gemv_args(x, qweight, scales, zeros, M, N, K, cfg, y);
   if (st != AWQ_OK || N == 0) return st;
+  const bool zp = cfg.zero_point != 0;
   Plan pl;
-  if ((st = make_plan(M, N, K, cfg.zero_point != 0, pl)) != AWQ_OK) return st;
+  if ((st = make_plan(M, N, K, zp, pl)) != AWQ_OK) return st;
   GemvParams p;
-  p.x = x;
-  p.qweight = qweight;
-  p.scales = scales;
-  p.zeros = zeros;
   p.y = y;
   p.counters = nullptr;
   p.partials = nullptr;
@@ -479,15 +556,35 @@ extern "C" awq_status_t awq_gemv(const uint16_t* x, const int32_t* qweight,
     p.counters = static_cast<uint32_t*>(workspace);
     p.partials = reinterpret_cast<float*>(static_cast<char*>(workspace) + pl.counter_bytes);
   }
+  const int G = int(K / kGroup);
+  // codes: int32 [N][K/8], box 16 words (one group) x 16*RT rows
+  // x: fp16 [M][K], box 128 k x M rows; scales / zeros: fp16 [G][N], box 16*RT x 1
+  CUtensorMap tq, tx, ts, tz;
+  const uint32_t rows = uint32_t(16 * pl.v.rt);
+  if (!make_tensor_map_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_INT32, qweight, uint64_t(K / 8), uint64_t(N),
+                          uint64_t(K / 8) * 4, kWordsPerGroup, rows, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_tensor_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x, uint64_t(K), uint64_t(M),
+                          uint64_t(K) * 2, kGroup, uint32_t(M), CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_tensor_map_2d(&ts, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, scales, uint64_t(N), uint64_t(G),
+                          uint64_t(N) * 2, rows, 1, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return AWQ_ERR_CUDA;
+  if (zp) {
+    if (!make_tensor_map_2d(&tz, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, zeros, uint64_t(N), uint64_t(G),
+                            uint64_t(N) * 2, rows, 1, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return AWQ_ERR_CUDA;
+  } else {
+    tz = ts;   // never read by the symmetric kernels
+  }
   p.units = pl.units;
   p.M = int(M);
   p.N = int(N);
   p.K = int(K);
-  p.G = int(K / kGroup);
+  p.G = G;
   p.nb = pl.nb;
   p.total_warps = pl.grid * kGemvWarps;
-  p.stage_bytes = pl.stage_bytes;
-  p.x_offset = pl.v.rt * 2 * 32 * 16 + pl.v.rt * 16 * 2 * (cfg.zero_point ? 2 : 1);
-  pl.v.fn<<<pl.grid, kGemvThreads, pl.smem, static_cast<cudaStream_t>(stream)>>>(p);
+  p.stage_bytes = pl.sg.stage_bytes;
+  p.x_offset = pl.sg.x_offset;
+  p.tx_bytes = pl.sg.tx_bytes;
+  pl.v.fn<<<pl.grid, kGemvThreads, pl.smem, static_cast<cudaStream_t>(stream)>>>(tq, tx, ts, tz, p);
   return launch_status();
 }
