@@ -162,6 +162,33 @@ AWQ_API awq_status_t awq_gemv(const uint16_t* x, const int32_t* qweight,
                       void* stream);
 
 /*
+ * awq_gemv_noalloc -- awq_gemv without a caller-provided workspace, for
+ * callers that cannot allocate device memory when they run the layer: for
+ * example a plugin inside a host engine that owns all device memory and
+ * passes in only the input and output buffers, or a decode loop that must
+ * not allocate after start-up. The AWQ pages have no counterpart to this
+ * entry point.
+ *
+ * Same arguments, limits, arithmetic and results as awq_gemv; the split-K
+ * scratch lives in one fixed array of AWQ_GEMV_STATIC_WORKSPACE_BYTES inside
+ * the library, which every GPU that loads the library keeps until the
+ * process exits. Shapes whose scratch would not fit return
+ * AWQ_ERR_WORKSPACE. The call allocates nothing: it does not call cudaMalloc,
+ * cudaFree or any allocating routine. It enqueues a cudaMemsetAsync of the
+ * array's counter region and then the GEMV kernel, both on `stream`.
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current and caches it; make that
+ * first call before any stream capture. All calls on a device share the
+ * array: calls that may overlap on the GPU (different streams, or
+ * concurrent host threads) race and must be serialized by the caller.
+ */
+#define AWQ_GEMV_STATIC_WORKSPACE_BYTES (16u << 20)
+AWQ_API awq_status_t awq_gemv_noalloc(const uint16_t* x, const int32_t* qweight,
+                                      const uint16_t* scales, const uint16_t* zeros,
+                                      int64_t M, int64_t N, int64_t K, awq_qconfig_t cfg,
+                                      uint16_t* y, void* stream);
+
+/*
  * awq_gemm -- y[M][N] = x[M][K] . W'^T for any M >= 1 (prefill).
  * ("AutoAWQ" code tour, "The big picture": the GEMM variant for batched
  * requests; "AWQ Quantization Support", "Integration with Forward Pass":

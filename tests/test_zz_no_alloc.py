@@ -1,0 +1,67 @@
+"""awq_gemv_noalloc: the GEMV entry point that allocates nothing.
+
+Some callers of this library cannot allocate device memory when they run the
+layer: a plugin inside a host engine that owns all device memory and hands in
+only the input and output buffers, or a decode loop that must not allocate
+after start-up. awq_gemv_noalloc serves them from one fixed scratch array
+inside the library instead of a caller workspace. These tests call it through
+the C ABI and check it against awq_gemv with a caller workspace, on two calls
+in a row (the array keeps the previous call's contents). The file is named
+so that pytest collects it after every other test file.
+"""
+
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import weight_only_int4_gemv_b200 as awq
+from oracle import awq_oracle as O
+from parity_util import activations, assert_close, bits, dev, host, oracle_layer
+
+
+def test_noalloc_is_exported_and_validates_on_the_host():
+    L = awq.lib()
+    assert hasattr(L, "awq_gemv_noalloc")
+    P, A = ctypes.c_void_p, 0x10000
+    cfg = awq.QConfig(128, 1)
+    # rejected before any CUDA call: null input, batch out of range, N % 8, group size
+    assert L.awq_gemv_noalloc(None, P(A), P(A), P(A), 1, 64, 256, cfg, P(A), None) == 1
+    assert L.awq_gemv_noalloc(P(A), P(A), P(A), P(A), 17, 64, 256, cfg, P(A), None) == 2
+    assert L.awq_gemv_noalloc(P(A), P(A), P(A), P(A), 1, 60, 256, cfg, P(A), None) == 2
+    assert L.awq_gemv_noalloc(P(A), P(A), P(A), P(A), 1, 64, 256, awq.QConfig(64, 1), P(A), None) == 4
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("M,N,K,zp", [(1, 14336, 4096, True), (4, 4096, 14336, True),
+                                      (16, 4096, 4096, False), (3, 1000, 1024, True)])
+def test_noalloc_matches_workspace_entry_on_two_calls(M, N, K, zp):
+    _, qweight, scales, zeros, Wd = oracle_layer(N, K, 0.02, 0.01, zp)
+    xh = activations(M, K, seed=M)
+    x, q, s = dev(xh), dev(qweight), dev(scales)
+    z = dev(zeros) if zp else None
+    ws = awq.alloc_workspace(M, N, K, zp)
+    ref = host(awq.awq_gemv(x, q, s, z, workspace=ws))
+    torch.cuda.synchronize()
+    for call in range(2):
+        y = torch.full((M, N), float("nan"), dtype=torch.float16, device="cuda")
+        awq.awq_gemv_noalloc(x, q, s, z, out=y)
+        torch.cuda.synchronize()
+        yh = host(y)
+        # the parity tolerance of the other tests, against the existing entry point
+        assert_close(yh, ref.astype(np.float64), f"call {call} vs awq_gemv")
+        # same kernel and same split: the bits agree too
+        assert np.array_equal(bits(yh), bits(ref)), f"call {call}"
+    assert_close(yh, O.matmul_f64(xh, Wd), "vs oracle")
+
+
+@pytest.mark.gpu
+def test_noalloc_rejects_shapes_beyond_its_array():
+    """The arrival counters of N = 2^30 output channels alone exceed the fixed
+    array: the call is refused on the host before any device work."""
+    L = awq.lib()
+    P, A = ctypes.c_void_p, 0x10000
+    with torch.cuda.device(0):
+        st = L.awq_gemv_noalloc(P(A), P(A), P(A), P(A), 1, 1 << 30, 256, awq.QConfig(128, 1), P(A), None)
+    assert st == 6   # AWQ_ERR_WORKSPACE

@@ -24,7 +24,7 @@ import torch
 __all__ = [
     "LIB_PATH", "AwqError", "lib", "GROUP_SIZE",
     "awq_pseudo_quantize_pack", "awq_dequant", "awq_workspace_bytes",
-    "awq_gemv", "awq_gemm", "awq_device_error", "awq_linear", "GEMV_MAX_M",
+    "awq_gemv", "awq_gemm", "awq_device_error", "awq_linear", "GEMV_MAX_M", "awq_gemv_noalloc",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libawq_b200.so")
@@ -60,6 +60,7 @@ _SIGS = {
     "awq_gemv": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, QConfig, _P, _P, ctypes.c_size_t, _P]),
     "awq_gemm": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, QConfig, _P, _P, ctypes.c_size_t, _P]),
     "awq_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), _P]),
+    "awq_gemv_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, QConfig, _P, _P]),
 }
 
 
@@ -195,6 +196,29 @@ def _product(entry: str, x, qweight, scales, zeros, workspace, out, group_size):
 def awq_gemv(x, qweight, scales, zeros, workspace=None, out=None, group_size: int = GROUP_SIZE):
     """y = x . W'^T for 1 <= M <= 16 (decode). `workspace` from alloc_workspace()."""
     return _product("awq_gemv", x, qweight, scales, zeros, workspace, out, group_size)
+
+
+def awq_gemv_noalloc(x, qweight, scales, zeros, out=None, group_size: int = GROUP_SIZE):
+    """awq_gemv with the library's fixed scratch array instead of a workspace,
+    for callers that cannot allocate device memory when they run the layer.
+    Calls on one device share the array and must not overlap on the GPU."""
+    _need(x, "x", torch.float16, 2)
+    _need(qweight, "qweight", torch.int32, 2)
+    _need(scales, "scales", torch.float16, 2)
+    if zeros is not None:
+        _need(zeros, "zeros", torch.float16, 2)
+    M, K = x.shape
+    N = qweight.shape[0]
+    if qweight.shape[1] * 8 != K:
+        raise ValueError("qweight must be [N, K/8] for x [M, K]")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float16, device=x.device)
+    _need(out, "out", torch.float16, 2)
+    with torch.cuda.device(x.device):
+        _check("awq_gemv_noalloc", lib().awq_gemv_noalloc(
+            _ptr(x), _ptr(qweight), _ptr(scales), _ptr(zeros), M, N, K, _cfg(zeros is not None, group_size),
+            _ptr(out), _stream(x.device)))
+    return out
 
 
 def awq_gemm(x, qweight, scales, zeros, workspace=None, out=None, group_size: int = GROUP_SIZE):

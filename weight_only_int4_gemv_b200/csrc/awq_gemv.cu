@@ -588,3 +588,60 @@ extern "C" awq_status_t awq_gemv(const uint16_t* x, const int32_t* qweight,
   pl.v.fn<<<pl.grid, kGemvThreads, pl.smem, static_cast<cudaStream_t>(stream)>>>(tq, tx, ts, tz, p);
   return launch_status();
 }
+
+// ---------------------------------------------------------------------------
+// awq_gemv_noalloc: awq_gemv with its scratch in a fixed array of this
+// library instead of caller memory. The AWQ pages have no counterpart; it
+// exists for callers that cannot allocate device memory at the point of
+// the call (see awq.h).
+// ---------------------------------------------------------------------------
+namespace awq {
+namespace {
+
+constexpr size_t kStaticScratchBytes = AWQ_GEMV_STATIC_WORKSPACE_BYTES;
+
+// Split-K partials and arrival counters of awq_gemv_noalloc. Every GPU that
+// loads the library holds this array until the process exits; all calls on
+// a device share it.
+static __device__ __align__(256) uint8_t g_gemv_scratch[kStaticScratchBytes];
+
+std::atomic<uintptr_t> g_scratch_addr[kMaxDevices];
+
+// Device address of g_gemv_scratch on the current device. In host code the
+// array's name is only a host-side stand-in, so the address is looked up once
+// per device (with that device current) and cached.
+awq_status_t scratch_address(int dev, void** out) {
+  uintptr_t a = g_scratch_addr[dev].load(std::memory_order_acquire);
+  if (a == 0) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_gemv_scratch) != cudaSuccess || p == nullptr) return AWQ_ERR_CUDA;
+    a = reinterpret_cast<uintptr_t>(p);
+    g_scratch_addr[dev].store(a, std::memory_order_release);
+  }
+  *out = reinterpret_cast<void*>(a);
+  return AWQ_OK;
+}
+
+}  // namespace
+}  // namespace awq
+
+extern "C" awq_status_t awq_gemv_noalloc(const uint16_t* x, const int32_t* qweight,
+                                         const uint16_t* scales, const uint16_t* zeros, int64_t M,
+                                         int64_t N, int64_t K, awq_qconfig_t cfg, uint16_t* y,
+                                         void* stream) {
+  awq_status_t st = check_gemv_args(x, qweight, scales, zeros, M, N, K, cfg, y);
+  if (st != AWQ_OK || N == 0) return st;
+  Plan pl;
+  if ((st = make_plan(M, N, K, cfg.zero_point != 0, pl)) != AWQ_OK) return st;
+  const size_t need = pl.partial_bytes ? pl.counter_bytes + pl.partial_bytes : 0;
+  if (need > kStaticScratchBytes) return AWQ_ERR_WORKSPACE;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return AWQ_ERR_CUDA;
+  void* scratch = nullptr;
+  if ((st = scratch_address(dev, &scratch)) != AWQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // The arrival counters must start at zero. A completed call leaves them at
+  // zero, but one that gave up part-way may not, so clear them every call.
+  if (need && cudaMemsetAsync(scratch, 0, pl.counter_bytes, s) != cudaSuccess) return AWQ_ERR_CUDA;
+  return awq_gemv(x, qweight, scales, zeros, M, N, K, cfg, y, scratch, kStaticScratchBytes, stream);
+}
