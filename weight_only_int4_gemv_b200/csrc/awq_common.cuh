@@ -204,6 +204,15 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const void* tensor_map, i
       : "memory");
 }
 
+// Prefetch one 2-D box of a tensor from global memory into L2 (no data
+// reaches shared memory; no barrier is involved).
+__device__ __forceinline__ void tma_prefetch_l2_2d(const void* tensor_map, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(tensor_map)),
+               "r"(x), "r"(y)
+               : "memory");
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }

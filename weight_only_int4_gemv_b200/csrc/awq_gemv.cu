@@ -38,6 +38,12 @@
 //   (arrival counter per block): it sums the contributors' fp32 partials in
 //   a fixed order, so results do not depend on timing, and resets the
 //   counter for the next call. No warp ever waits on another.
+// * Programmatic dependent launch: every CTA lets the next kernel launch as
+//   soon as it runs, and prefetches its first weight units from HBM into L2
+//   before waiting for the previous kernel (griddepcontrol.wait); loads into
+//   shared memory, workspace accesses and y stores come after the wait.
+//   Back-to-back layers overlap their launch and HBM ramp-up with the
+//   previous layer's tail. The L2 prefetch runs kPrefetchUnits ahead.
 // * Every mbarrier wait is bounded (2 s); a warp that gives up records bit 1
 //   of the device error word, waits (bounded) for its copies in flight and
 //   leaves its rows unwritten.
@@ -56,6 +62,7 @@ namespace {
 constexpr int kGemvWarps = 4;
 constexpr int kGemvThreads = kGemvWarps * 32;
 constexpr int kBarRegion = 1024;   // mbarriers of all warps, ahead of the rings
+constexpr int kPrefetchUnits = 8;  // L2 prefetch distance, in units, per warp
 
 struct GemvParams {
   uint16_t* y;
@@ -220,6 +227,10 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
   const int64_t gw = int64_t(blockIdx.x) * kGemvWarps + wi;
   const int64_t W = p.total_warps;
   const int64_t G = p.G;
+  // Let the next kernel in the stream (if launched as a programmatic
+  // dependent) start as soon as every CTA of this one is running; it waits
+  // for this grid's completion before it reads anything this grid writes.
+  asm volatile("griddepcontrol.launch_dependents;");
   const int64_t u_begin = warp_start(p.units, gw, W);
   const int64_t u_end = warp_start(p.units, gw + 1, W);
   if (u_begin >= u_end) return;
@@ -249,6 +260,29 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
       if (ZP) tma_load_2d(st + L::kCodeBytes + L::kMetaStride, &tmap_z, r0, j, &bars[slot]);
     }
   };
+  // lane 0: pull unit u's weight side (codes, scales, zero points) from HBM
+  // into L2. L2 is where all writes meet, so a prefetch is safe even while
+  // an earlier kernel may still be writing these bytes: the loads into
+  // shared memory that consume them happen after griddepcontrol.wait.
+  auto prefetch = [&](int64_t u) {
+    if (u < u_end) {
+      const int64_t b = u / G;
+      const int j = int(u - b * G);
+      const int r0 = int(b * (16 * RT));
+      tma_prefetch_l2_2d(&tmap_q, j * kWordsPerGroup, r0);
+      tma_prefetch_l2_2d(&tmap_s, r0, j);
+      if (ZP) tma_prefetch_l2_2d(&tmap_z, r0, j);
+    }
+  };
+  // Start the HBM stream for the first units, then wait for the kernels this
+  // one depends on (programmatic dependent launch: x may be their output,
+  // the weights may have just been written, the workspace and y may still
+  // be in use) before any load into shared memory or any store.
+  if (lane == 0) {
+#pragma unroll
+    for (int i = 0; i < kPrefetchUnits; ++i) prefetch(u_begin + i);
+  }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   if (lane == 0) {
 #pragma unroll
     for (int i = 0; i < S - 1; ++i) issue(u_begin + i, i);
@@ -283,7 +317,10 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
   bool ok = true;
   int64_t u = u_begin;
   for (; u < u_end; ++u) {
-    if (lane == 0) issue(u + S - 1, slot == 0 ? S - 1 : slot - 1);
+    if (lane == 0) {
+      issue(u + S - 1, slot == 0 ? S - 1 : slot - 1);
+      prefetch(u + kPrefetchUnits);
+    }
     const bool got = wait_bounded(&bars[slot], phase, &abort_flag, &g_awq_gemv_error, 2u);
     if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
     const int64_t b = u / G;
@@ -585,7 +622,20 @@ extern "C" awq_status_t awq_gemv(const uint16_t* x, const int32_t* qweight,
   p.stage_bytes = pl.sg.stage_bytes;
   p.x_offset = pl.sg.x_offset;
   p.tx_bytes = pl.sg.tx_bytes;
-  pl.v.fn<<<pl.grid, kGemvThreads, pl.smem, static_cast<cudaStream_t>(stream)>>>(tq, tx, ts, tz, p);
+  // Programmatic dependent launch: this grid may start while the previous
+  // kernel in the stream finishes; the kernel waits for it (griddepcontrol)
+  // before reading x or writing y and the workspace.
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(pl.grid);
+  lc.blockDim = dim3(kGemvThreads);
+  lc.dynamicSmemBytes = size_t(pl.smem);
+  lc.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  if (cudaLaunchKernelEx(&lc, pl.v.fn, tq, tx, ts, tz, p) != cudaSuccess) return AWQ_ERR_CUDA;
   return launch_status();
 }
 
