@@ -59,17 +59,20 @@ __device__ uint32_t g_awq_gemv_error = 0;
 
 namespace {
 
-constexpr int kGemvWarps = 4;
-constexpr int kGemvThreads = kGemvWarps * 32;
-constexpr int kBarRegion = 1024;   // mbarriers of all warps, ahead of the rings
-constexpr int kPrefetchUnits = 8;  // L2 prefetch distance, in units, per warp
+constexpr int kMaxConsumers = 12;
+constexpr int kMaxStages = 8;
+constexpr int kBarRegion = 2 * kMaxConsumers * kMaxStages * 8;   // full + empty mbarriers
+constexpr int kPrefetchUnits = 6;  // L2 prefetch distance, in units, per consumer
 
 struct GemvParams {
   uint16_t* y;
-  float* partials;       // [total_warps][2][32 lanes][RT*MT*4]
+  float* partials;       // [total consumers][2][16*RT*M] floats, [row][m]
   uint32_t* counters;    // [nb]
   int64_t units;         // nb * G
-  int M, N, K, G, nb, total_warps;
+  int M, N, K, G, nb;
+  int consumers;         // consumer warps per CTA
+  int total_consumers;   // grid * consumers
+  int stages;            // ring stages per consumer
   int stage_bytes;       // codes + metadata + x slice of one unit (multiple of 128)
   int x_offset;          // offset of the x slice inside a stage
   uint32_t tx_bytes;     // bytes the TMA copies of one unit deliver
@@ -91,9 +94,9 @@ __device__ __forceinline__ uint32_t word_of(const uint4& v, int i) {
   return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
 
-// First unit of warp w in the even split of `units` over `warps`.
-__device__ __forceinline__ int64_t warp_start(int64_t units, int64_t w, int64_t warps) {
-  return units * w / warps;
+// First unit of consumer w in the even split of `units` over `consumers`.
+__device__ __forceinline__ int64_t range_start(int64_t units, int64_t w, int64_t consumers) {
+  return units * w / consumers;
 }
 
 template <int MT, int RT>
@@ -118,11 +121,13 @@ __device__ __forceinline__ void store_y(const GemvParams& p, int64_t row0, int g
   }
 }
 
-// Finish row block b after this warp summed groups [j0, j1) of it.
-// Partials are stored lane-major ([lane][RT*MT*4] floats) so each lane moves
-// its values with 16-byte accesses.
+// Finish row block b after consumer gc summed groups [j0, j1) of it.
+// A split block's partial sums are stored compactly (the block's 16*RT rows
+// x M batch rows, [row][m]); the consumer that completes the block's group
+// count sums every contributor's values in consumer order (reproducible
+// bits), loading many contributors at once.
 template <int MT, int RT>
-__device__ __forceinline__ void finish_block(const GemvParams& p, int64_t b, int j0, int j1, int64_t gw,
+__device__ __forceinline__ void finish_block(const GemvParams& p, int64_t b, int j0, int j1, int64_t gc,
                                              int64_t first_block, int lane, int g, int t,
                                              const float (&acc)[RT][MT][4]) {
   const int64_t row0 = b * (16 * RT);
@@ -131,16 +136,25 @@ __device__ __forceinline__ void finish_block(const GemvParams& p, int64_t b, int
     store_y<MT, RT>(p, row0, g, t, acc);
     return;
   }
-  constexpr int kVals = RT * MT * 4;           // floats per lane
-  constexpr int kVec = kVals / 4;              // float4 per lane
-  constexpr int kSlot = kVals * 32;
+  const int M = p.M;
+  const int V = 16 * RT * M;                     // values of one partial
   const int slot = (b == first_block) ? 0 : 1;
-  float4* sp = reinterpret_cast<float4*>(p.partials + (gw * 2 + slot) * kSlot) + lane * kVec;
+  float* sp = p.partials + (gc * 2 + slot) * int64_t(V);
 #pragma unroll
   for (int rt = 0; rt < RT; ++rt)
 #pragma unroll
-    for (int mt = 0; mt < MT; ++mt)
-      __stcg(sp + rt * MT + mt, make_float4(acc[rt][mt][0], acc[rt][mt][1], acc[rt][mt][2], acc[rt][mt][3]));
+    for (int mt = 0; mt < MT; ++mt) {
+      const int m0 = 8 * mt + 2 * t;
+      const int r_lo = 16 * rt + g, r_hi = r_lo + 8;
+      if (m0 < M) {
+        __stcg(sp + r_lo * M + m0, acc[rt][mt][0]);
+        __stcg(sp + r_hi * M + m0, acc[rt][mt][2]);
+      }
+      if (m0 + 1 < M) {
+        __stcg(sp + r_lo * M + m0 + 1, acc[rt][mt][1]);
+        __stcg(sp + r_hi * M + m0 + 1, acc[rt][mt][3]);
+      }
+    }
   __syncwarp();   // every lane's stores happen before lane 0's release below
   uint32_t last = 0;
   if (lane == 0) {
@@ -152,48 +166,55 @@ __device__ __forceinline__ void finish_block(const GemvParams& p, int64_t b, int
   }
   last = __shfl_sync(0xffffffffu, last, 0);
   if (!last) return;
-  // Sum every contributor in warp order (fixed order: reproducible bits),
-  // four contributors' loads in flight at a time.
-  const int64_t W = p.total_warps;
+  // Contributors: every non-empty consumer range overlapping block b, in
+  // consumer order. Range starts floor(units * w / W) advance by
+  // floor(units / W) plus a carry, so no division happens per contributor.
+  const int64_t W = p.total_consumers;
   const int64_t w_first = ((b * G + 1) * W - 1) / p.units;
   const int64_t w_last = ((b * G + G) * W - 1) / p.units;
-  float4 tot[kVec];
+  const int64_t q_step = p.units / W, r_step = p.units % W;
+  const int64_t bG = b * G;
+  constexpr int kChunk = 16;                     // contributors loaded at once
+  const int nv = V / 32;                         // values per lane (V = 64 M), two per pass
+  for (int v0 = 0; v0 < nv; v0 += 2) {
+    int64_t ws = range_start(p.units, w_first, W);
+    int64_t rem = (p.units * w_first) % W;
+    float acc2[2] = {0.0f, 0.0f};
+    for (int64_t w0 = w_first; w0 <= w_last; w0 += kChunk) {
+      float part[kChunk][2];
 #pragma unroll
-  for (int v = 0; v < kVec; ++v) tot[v] = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int64_t w0 = w_first; w0 <= w_last; w0 += 4) {
-    float4 part[4][kVec];
+      for (int c = 0; c < kChunk; ++c) {
+        const int64_t w = w0 + c;
+        int64_t we = ws + q_step;                // start of range w + 1
+        int64_t rem2 = rem + r_step;
+        if (rem2 >= W) { rem2 -= W; ++we; }
+        const bool live = w <= w_last && ws < we;
+        const int s = ws >= bG ? 0 : 1;          // block b is the range's first block, or its last
+        const float* src = p.partials + (w * 2 + s) * int64_t(V);
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const int64_t w = w0 + c;
-      const int64_t ws = warp_start(p.units, w, W);
-      const bool live = w <= w_last && ws < warp_start(p.units, w + 1, W);   // skip empty ranges
-      const int s = (ws / G == b) ? 0 : 1;
-      const float4* rp = reinterpret_cast<const float4*>(p.partials + (w * 2 + s) * kSlot) + lane * kVec;
-#pragma unroll
-      for (int v = 0; v < kVec; ++v) part[c][v] = live ? __ldcg(rp + v) : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-#pragma unroll
-    for (int c = 0; c < 4; ++c)
-#pragma unroll
-      for (int v = 0; v < kVec; ++v) {
-        tot[v].x += part[c][v].x;
-        tot[v].y += part[c][v].y;
-        tot[v].z += part[c][v].z;
-        tot[v].w += part[c][v].w;
+        for (int e = 0; e < 2; ++e) {
+          const int v = lane + 32 * (v0 + e);
+          part[c][e] = (live && v < V) ? __ldcg(src + v) : 0.0f;
+        }
+        ws = we;
+        rem = rem2;
       }
-  }
-  float sum[RT][MT][4];
 #pragma unroll
-  for (int rt = 0; rt < RT; ++rt)
-#pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
-      const float4 v = tot[rt * MT + mt];
-      sum[rt][mt][0] = v.x;
-      sum[rt][mt][1] = v.y;
-      sum[rt][mt][2] = v.z;
-      sum[rt][mt][3] = v.w;
+      for (int c = 0; c < kChunk; ++c) {
+        acc2[0] += part[c][0];
+        acc2[1] += part[c][1];
+      }
     }
-  store_y<MT, RT>(p, row0, g, t, sum);
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int v = lane + 32 * (v0 + e);
+      if (v < V) {
+        const int row = v / M, m = v - row * M;
+        if (row0 + row < p.N)
+          p.y[int64_t(m) * p.N + row0 + row] = __half_as_ushort(__float2half_rn(acc2[e]));
+      }
+    }
+  }
   if (lane == 0) p.counters[b] = 0u;
 }
 
@@ -213,80 +234,114 @@ struct StageLayout {
   static constexpr int kMetaStride = (kMetaBytes + 127) / 128 * 128;
 };
 
-template <int MT, int RT, bool ZP, int S>
-__global__ void __launch_bounds__(kGemvThreads)
+// Consumer warps per CTA. Each SM sub-partition has its own quarter of the
+// register file, so the warp count (consumers + producer) is kept a multiple
+// of 4: 12 warps leave 168 registers per thread for one n8 batch tile, 8
+// warps leave 255 for two.
+template <int MT>
+struct Consumers {
+  static constexpr int value = MT == 1 ? 11 : 7;
+};
+
+template <int MT, int RT, bool ZP>
+__global__ void __launch_bounds__(32 * (1 + Consumers<MT>::value), 1)
 gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_x,
             const __grid_constant__ CUtensorMap tmap_s, const __grid_constant__ CUtensorMap tmap_z,
             const GemvParams p) {
   extern __shared__ __align__(1024) uint8_t gemv_smem[];
   using L = StageLayout<RT>;
   const int lane = threadIdx.x & 31;
-  const int g = lane >> 2;
-  const int t = lane & 3;
-  const int wi = threadIdx.x >> 5;
-  const int64_t gw = int64_t(blockIdx.x) * kGemvWarps + wi;
-  const int64_t W = p.total_warps;
+  const int warp = threadIdx.x >> 5;
+  const int C = p.consumers;
+  const int S = p.stages;
+  const int64_t W = p.total_consumers;
   const int64_t G = p.G;
+  const int stage_bytes = p.stage_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(gemv_smem);            // [consumer][stage]
+  uint64_t* empty = full + kMaxConsumers * kMaxStages;                // [consumer][stage]
+  uint8_t* rings = gemv_smem + kBarRegion;                            // consumer c: c * S stages
   // Let the next kernel in the stream (if launched as a programmatic
   // dependent) start as soon as every CTA of this one is running; it waits
   // for this grid's completion before it reads anything this grid writes.
   asm volatile("griddepcontrol.launch_dependents;");
-  const int64_t u_begin = warp_start(p.units, gw, W);
-  const int64_t u_end = warp_start(p.units, gw + 1, W);
-  if (u_begin >= u_end) return;
-  const int stage_bytes = p.stage_bytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(gemv_smem) + wi * S;
-  uint8_t* ring = gemv_smem + kBarRegion + wi * S * stage_bytes;
 
-  if (lane == 0) {
-#pragma unroll
-    for (int i = 0; i < S; ++i) mbar_init(&bars[i], 1);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C * S; ++i) {
+      mbar_init(&full[(i / S) * kMaxStages + i % S], 1);
+      mbar_init(&empty[(i / S) * kMaxStages + i % S], 1);
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     fence_proxy_async_smem();
   }
-  __syncwarp();
+  __syncthreads();
 
-  // lane 0: fill `slot` with unit u (codes box, x box, scale and zero runs)
-  auto issue = [&](int64_t u, int slot) {
-    if (u < u_end) {
-      const int64_t b = u / G;
-      const int j = int(u - b * G);
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    // Lane c feeds consumer c. All lanes step through their rounds together,
+    // so round r of every consumer is issued before round r+1 and data
+    // returns roughly in the order it is consumed.
+    if (lane >= C) return;
+    const int64_t gc = int64_t(blockIdx.x) * C + lane;
+    const int64_t ub = range_start(p.units, gc, W);
+    const int64_t n = range_start(p.units, gc + 1, W) - ub;
+    if (n <= 0) return;
+    // (block, group) of the consumer's first unit; later units advance by one group
+    int64_t b0 = ub / G;
+    int j0 = int(ub - b0 * G);
+    // Before the dependency wait only L2 prefetches: they are safe even
+    // while an earlier kernel may still be writing these bytes.
+    {
+      int64_t b = b0;
+      int j = j0;
+      for (int64_t r = 0; r < n && r < kPrefetchUnits; ++r) {
+        const int r0 = int(b * (16 * RT));
+        tma_prefetch_l2_2d(&tmap_q, j * kWordsPerGroup, r0);
+        tma_prefetch_l2_2d(&tmap_s, r0, j);
+        if (ZP) tma_prefetch_l2_2d(&tmap_z, r0, j);
+        if (++j == G) { j = 0; ++b; }
+      }
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    uint64_t* fb0 = &full[lane * kMaxStages];
+    uint64_t* eb0 = &empty[lane * kMaxStages];
+    uint8_t* ring = rings + lane * S * stage_bytes;
+    volatile int abort_flag = 0;
+    int64_t b = b0;
+    int j = j0;
+    int slot = 0;
+    uint32_t ephase = 1;   // parity of the empty phase to wait for in the slot's next reuse
+    int64_t r = 0;
+    for (; r < n; ++r) {
+      if (r >= S && !wait_bounded(&eb0[slot], ephase, &abort_flag, &g_awq_gemv_error, 2u)) break;
       const int r0 = int(b * (16 * RT));
       uint8_t* st = ring + slot * stage_bytes;
-      mbar_arrive_expect_tx(&bars[slot], p.tx_bytes);
-      tma_load_2d(st, &tmap_q, j * kWordsPerGroup, r0, &bars[slot]);
-      tma_load_2d(st + p.x_offset, &tmap_x, j * kGroup, 0, &bars[slot]);
-      tma_load_2d(st + L::kCodeBytes, &tmap_s, r0, j, &bars[slot]);
-      if (ZP) tma_load_2d(st + L::kCodeBytes + L::kMetaStride, &tmap_z, r0, j, &bars[slot]);
+      mbar_arrive_expect_tx(&fb0[slot], p.tx_bytes);
+      tma_load_2d(st, &tmap_q, j * kWordsPerGroup, r0, &fb0[slot]);
+      tma_load_2d(st + p.x_offset, &tmap_x, j * kGroup, 0, &fb0[slot]);
+      tma_load_2d(st + L::kCodeBytes, &tmap_s, r0, j, &fb0[slot]);
+      if (ZP) tma_load_2d(st + L::kCodeBytes + L::kMetaStride, &tmap_z, r0, j, &fb0[slot]);
+      if (++j == G) { j = 0; ++b; }
+      if (++slot == S) { slot = 0; ephase ^= 1u; }
     }
-  };
-  // lane 0: pull unit u's weight side (codes, scales, zero points) from HBM
-  // into L2. L2 is where all writes meet, so a prefetch is safe even while
-  // an earlier kernel may still be writing these bytes: the loads into
-  // shared memory that consume them happen after griddepcontrol.wait.
-  auto prefetch = [&](int64_t u) {
-    if (u < u_end) {
-      const int64_t b = u / G;
-      const int j = int(u - b * G);
-      const int r0 = int(b * (16 * RT));
-      tma_prefetch_l2_2d(&tmap_q, j * kWordsPerGroup, r0);
-      tma_prefetch_l2_2d(&tmap_s, r0, j);
-      if (ZP) tma_prefetch_l2_2d(&tmap_z, r0, j);
+    // Gave up: the copies already issued (the last S rounds before r) land
+    // before the CTA's shared memory can be reused.
+    if (r < n) {
+      for (int64_t q = r - S > 0 ? r - S : 0; q < r; ++q)
+        wait_teardown(&fb0[int(q % S)], uint32_t((q / S) & 1));
     }
-  };
-  // Start the HBM stream for the first units, then wait for the kernels this
-  // one depends on (programmatic dependent launch: x may be their output,
-  // the weights may have just been written, the workspace and y may still
-  // be in use) before any load into shared memory or any store.
-  if (lane == 0) {
-#pragma unroll
-    for (int i = 0; i < kPrefetchUnits; ++i) prefetch(u_begin + i);
+    return;
   }
+
+  // -------------------------------------------------------------- consumer
+  const int cw = warp - 1;
+  const int g = lane >> 2;
+  const int t = lane & 3;
+  const int64_t gc = int64_t(blockIdx.x) * C + cw;
+  const int64_t u_begin = range_start(p.units, gc, W);
+  const int64_t u_end = range_start(p.units, gc + 1, W);
+  if (u_begin >= u_end) return;
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  if (lane == 0) {
-#pragma unroll
-    for (int i = 0; i < S - 1; ++i) issue(u_begin + i, i);
-  }
+  uint8_t* ring = rings + cw * S * stage_bytes;
 
   // x fragment offsets inside a stage: batch row m = 8 mt + g, chunk 4t + jj
   int xoff[MT];
@@ -304,6 +359,8 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
   const int64_t first_block = u_begin / G;
   int64_t cur_b = first_block;
   int jstart = int(u_begin - cur_b * G);
+  int64_t ub_ = cur_b;   // block of the unit being consumed
+  int jg = jstart;       // its group
   float acc[RT][MT][4];
 #pragma unroll
   for (int rt = 0; rt < RT; ++rt)
@@ -314,18 +371,13 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
 
   int slot = 0;
   uint32_t phase = 0;
-  bool ok = true;
-  int64_t u = u_begin;
-  for (; u < u_end; ++u) {
-    if (lane == 0) {
-      issue(u + S - 1, slot == 0 ? S - 1 : slot - 1);
-      prefetch(u + kPrefetchUnits);
-    }
-    const bool got = wait_bounded(&bars[slot], phase, &abort_flag, &g_awq_gemv_error, 2u);
-    if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-    const int64_t b = u / G;
+  for (int64_t u = u_begin; u < u_end; ++u) {
+    const bool got = wait_bounded(&full[cw * kMaxStages + slot], phase, &abort_flag, &g_awq_gemv_error, 2u);
+    if (!__all_sync(0xffffffffu, got)) return;   // producer gave up or timed out: rows stay unwritten
+    const int64_t b = ub_;
+    if (++jg == G) { jg = 0; ++ub_; }
     if (b != cur_b) {
-      finish_block<MT, RT>(p, cur_b, jstart, int(G), gw, first_block, lane, g, t, acc);
+      finish_block<MT, RT>(p, cur_b, jstart, int(G), gc, first_block, lane, g, t, acc);
       cur_b = b;
       jstart = 0;
 #pragma unroll
@@ -349,7 +401,6 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
       c_lo[rt] = lds128(st + (16 * rt + g) * 64 + t * 16);
       c_hi[rt] = lds128(st + (16 * rt + 8 + g) * 64 + t * 16);
     }
-
     float grp[RT][MT][4];
     float cs[MT][4];
 #pragma unroll
@@ -388,45 +439,33 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
       sm[mt][0] = __shfl_sync(0xffffffffu, cs[mt][0], 4 + t);
       sm[mt][1] = __shfl_sync(0xffffffffu, cs[mt][1], 4 + t);
     }
-    // sum_k x (q - z) = raw - C(m) - z S(m); then the group's scale
+    float s_lo[RT], s_hi[RT], z_lo[RT], z_hi[RT];
 #pragma unroll
     for (int rt = 0; rt < RT; ++rt) {
-      const float s_lo = half_bits_to_float(lds16(st + L::kCodeBytes + (16 * rt + g) * 2));
-      const float s_hi = half_bits_to_float(lds16(st + L::kCodeBytes + (16 * rt + 8 + g) * 2));
-      float z_lo = 8.0f, z_hi = 8.0f;
-      if (ZP) {
-        z_lo = half_bits_to_float(lds16(st + L::kCodeBytes + L::kMetaStride + (16 * rt + g) * 2));
-        z_hi = half_bits_to_float(lds16(st + L::kCodeBytes + L::kMetaStride + (16 * rt + 8 + g) * 2));
-      }
-#pragma unroll
-      for (int mt = 0; mt < MT; ++mt) {
-        acc[rt][mt][0] = fmaf(s_lo, fmaf(-z_lo, sm[mt][0], grp[rt][mt][0] - cm[mt][0]), acc[rt][mt][0]);
-        acc[rt][mt][1] = fmaf(s_lo, fmaf(-z_lo, sm[mt][1], grp[rt][mt][1] - cm[mt][1]), acc[rt][mt][1]);
-        acc[rt][mt][2] = fmaf(s_hi, fmaf(-z_hi, sm[mt][0], grp[rt][mt][2] - cm[mt][0]), acc[rt][mt][2]);
-        acc[rt][mt][3] = fmaf(s_hi, fmaf(-z_hi, sm[mt][1], grp[rt][mt][3] - cm[mt][1]), acc[rt][mt][3]);
-      }
+      s_lo[rt] = half_bits_to_float(lds16(st + L::kCodeBytes + (16 * rt + g) * 2));
+      s_hi[rt] = half_bits_to_float(lds16(st + L::kCodeBytes + (16 * rt + 8 + g) * 2));
+      z_lo[rt] = ZP ? half_bits_to_float(lds16(st + L::kCodeBytes + L::kMetaStride + (16 * rt + g) * 2)) : 8.0f;
+      z_hi[rt] = ZP ? half_bits_to_float(lds16(st + L::kCodeBytes + L::kMetaStride + (16 * rt + 8 + g) * 2)) : 8.0f;
     }
-    __syncwarp();   // every lane is done with the slot before lane 0 refills it
+    // everything the unit needs is in registers: release the slot
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[cw * kMaxStages + slot]);
     if (++slot == S) {
       slot = 0;
       phase ^= 1u;
     }
-  }
-  if (ok) {
-    finish_block<MT, RT>(p, cur_b, jstart, int(u_end - cur_b * G), gw, first_block, lane, g, t, acc);
-  } else if (lane == 0) {
-    // Gave up: let the copies already issued for units u .. u+S-1 land
-    // before this warp's shared memory can be reused.
-    int s = slot;
-    uint32_t ph = phase;
-    for (int64_t v = u; v < u_end && v < u + S; ++v) {
-      wait_teardown(&bars[s], ph);
-      if (++s == S) {
-        s = 0;
-        ph ^= 1u;
+    // sum_k x (q - z) = raw - C(m) - z S(m); then the group's scale
+#pragma unroll
+    for (int rt = 0; rt < RT; ++rt)
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) {
+        acc[rt][mt][0] = fmaf(s_lo[rt], fmaf(-z_lo[rt], sm[mt][0], grp[rt][mt][0] - cm[mt][0]), acc[rt][mt][0]);
+        acc[rt][mt][1] = fmaf(s_lo[rt], fmaf(-z_lo[rt], sm[mt][1], grp[rt][mt][1] - cm[mt][1]), acc[rt][mt][1]);
+        acc[rt][mt][2] = fmaf(s_hi[rt], fmaf(-z_hi[rt], sm[mt][0], grp[rt][mt][2] - cm[mt][0]), acc[rt][mt][2]);
+        acc[rt][mt][3] = fmaf(s_hi[rt], fmaf(-z_hi[rt], sm[mt][1], grp[rt][mt][3] - cm[mt][1]), acc[rt][mt][3]);
       }
-    }
   }
+  finish_block<MT, RT>(p, cur_b, jstart, int(u_end - cur_b * G), gc, first_block, lane, g, t, acc);
 }
 
 // ---------------------------------------------------------------------------
@@ -437,21 +476,25 @@ using KernelFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMa
 
 struct Variant {
   KernelFn fn;
-  int mt, rt, stages, id;
+  int mt, rt, consumers, id;
 };
 
 constexpr int kNumVariants = 4;
+constexpr int kRT = 4;
+constexpr int kSmemBudget = 232448;   // largest dynamic shared memory of one sm_100 CTA
 
 Variant pick_variant(int64_t M, bool zp) {
   if (M <= 8)
-    return zp ? Variant{gemv_kernel<1, 4, true, 4>, 1, 4, 4, 0} : Variant{gemv_kernel<1, 4, false, 4>, 1, 4, 4, 1};
-  return zp ? Variant{gemv_kernel<2, 4, true, 3>, 2, 4, 3, 2} : Variant{gemv_kernel<2, 4, false, 3>, 2, 4, 3, 3};
+    return zp ? Variant{gemv_kernel<1, kRT, true>, 1, kRT, Consumers<1>::value, 0}
+              : Variant{gemv_kernel<1, kRT, false>, 1, kRT, Consumers<1>::value, 1};
+  return zp ? Variant{gemv_kernel<2, kRT, true>, 2, kRT, Consumers<2>::value, 2}
+            : Variant{gemv_kernel<2, kRT, false>, 2, kRT, Consumers<2>::value, 3};
 }
 
 int round128(int v) { return (v + 127) / 128 * 128; }
 
 struct StageGeometry {
-  int code_bytes, meta_stride, x_offset, stage_bytes;
+  int code_bytes, meta_stride, x_offset, stage_bytes, stages;
   uint32_t tx_bytes;
 };
 
@@ -462,6 +505,8 @@ StageGeometry stage_geometry(const Variant& v, int64_t M, bool zp) {
   sg.x_offset = sg.code_bytes + sg.meta_stride * (zp ? 2 : 1);
   sg.stage_bytes = round128(sg.x_offset + int(M) * 256);
   sg.tx_bytes = uint32_t(sg.code_bytes + 16 * v.rt * 2 * (zp ? 2 : 1) + int(M) * 256);
+  int st = (kSmemBudget - kBarRegion) / (v.consumers * sg.stage_bytes);
+  sg.stages = st > kMaxStages ? kMaxStages : st;
   return sg;
 }
 
@@ -479,7 +524,6 @@ struct Plan {
 constexpr int kMaxDevices = 64;
 std::atomic<int> g_sm_count[kMaxDevices];
 std::atomic<int> g_smem_attr[kMaxDevices][kNumVariants];
-std::atomic<int> g_occ[kMaxDevices][kNumVariants][17];   // by M
 
 awq_status_t make_plan(int64_t M, int64_t N, int64_t K, bool zp, Plan& pl) {
   int dev = 0;
@@ -487,7 +531,8 @@ awq_status_t make_plan(int64_t M, int64_t N, int64_t K, bool zp, Plan& pl) {
   if (dev < 0 || dev >= kMaxDevices) return AWQ_ERR_UNSUPPORTED;
   pl.v = pick_variant(M, zp);
   pl.sg = stage_geometry(pl.v, M, zp);
-  pl.smem = kBarRegion + kGemvWarps * pl.v.stages * pl.sg.stage_bytes;
+  if (pl.sg.stages < 2) return AWQ_ERR_UNSUPPORTED;
+  pl.smem = kBarRegion + pl.v.consumers * pl.sg.stages * pl.sg.stage_bytes;
   int sms = g_sm_count[dev].load(std::memory_order_relaxed);
   if (sms == 0) {
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
@@ -495,35 +540,27 @@ awq_status_t make_plan(int64_t M, int64_t N, int64_t K, bool zp, Plan& pl) {
     g_sm_count[dev].store(sms, std::memory_order_relaxed);
   }
   if (!g_smem_attr[dev][pl.v.id].load(std::memory_order_acquire)) {
-    // the largest ring any M asks of this variant
-    const int most = kBarRegion + kGemvWarps * pl.v.stages * stage_geometry(pl.v, pl.v.mt * 8, zp).stage_bytes;
-    if (cudaFuncSetAttribute(pl.v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, most) != cudaSuccess)
+    if (cudaFuncSetAttribute(pl.v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBudget) != cudaSuccess)
       return AWQ_ERR_CUDA;
     g_smem_attr[dev][pl.v.id].store(1, std::memory_order_release);
-  }
-  int occ = g_occ[dev][pl.v.id][M].load(std::memory_order_relaxed);
-  if (occ == 0) {
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, pl.v.fn, kGemvThreads, pl.smem) != cudaSuccess)
-      return AWQ_ERR_CUDA;
-    if (occ < 1) return AWQ_ERR_UNSUPPORTED;
-    g_occ[dev][pl.v.id][M].store(occ, std::memory_order_relaxed);
   }
   const int64_t rows_per_block = 16 * pl.v.rt;
   const int64_t G = K / kGroup;
   pl.nb = int((N + rows_per_block - 1) / rows_per_block);
   pl.units = int64_t(pl.nb) * G;
-  const int64_t want = (pl.units + kGemvWarps - 1) / kGemvWarps;
-  const int64_t cap = int64_t(sms) * occ;
-  pl.grid = int(want < cap ? (want > 0 ? want : 1) : cap);
-  const int64_t total_warps = int64_t(pl.grid) * kGemvWarps;
-  // units * warps must fit the kernel's 64-bit split arithmetic
-  if (pl.units > 0 && total_warps > (int64_t(1) << 62) / pl.units) return AWQ_ERR_SHAPE;
-  const size_t slot_floats = size_t(pl.v.rt) * pl.v.mt * 4 * 32;
+  // one CTA per SM (the ring takes the SM's shared memory); fewer when
+  // there are fewer units than consumers
+  const int64_t want = (pl.units + pl.v.consumers - 1) / pl.v.consumers;
+  pl.grid = int(want < sms ? (want > 0 ? want : 1) : sms);
+  const int64_t total = int64_t(pl.grid) * pl.v.consumers;
+  // units * consumers must fit the kernel's 64-bit split arithmetic
+  if (pl.units > 0 && total > (int64_t(1) << 62) / pl.units) return AWQ_ERR_SHAPE;
   pl.counter_bytes = ((size_t(pl.nb) * 4 + 255) / 256) * 256;
   // With one group per row (G == 1) every unit is a whole block and no
-  // block is ever split; otherwise warps may share blocks. A warp holds at
-  // most two partial blocks: the first and the last of its range.
-  pl.partial_bytes = G > 1 ? size_t(total_warps) * 2 * slot_floats * 4 : 0;
+  // block is ever split; otherwise consumers may share blocks. A consumer
+  // holds at most two partial blocks: the first and the last of its range,
+  // each 16*RT rows x M values.
+  pl.partial_bytes = G > 1 ? size_t(total) * 2 * size_t(16 * pl.v.rt) * size_t(M) * 4 : 0;
   return AWQ_OK;
 }
 
@@ -618,16 +655,18 @@ extern "C" awq_status_t awq_gemv(const uint16_t* x, const int32_t* qweight,
   p.K = int(K);
   p.G = G;
   p.nb = pl.nb;
-  p.total_warps = pl.grid * kGemvWarps;
+  p.consumers = pl.v.consumers;
+  p.total_consumers = pl.grid * pl.v.consumers;
+  p.stages = pl.sg.stages;
   p.stage_bytes = pl.sg.stage_bytes;
   p.x_offset = pl.sg.x_offset;
   p.tx_bytes = pl.sg.tx_bytes;
   // Programmatic dependent launch: this grid may start while the previous
   // kernel in the stream finishes; the kernel waits for it (griddepcontrol)
-  // before reading x or writing y and the workspace.
+  // before any load into shared memory, workspace access or store.
   cudaLaunchConfig_t lc = {};
   lc.gridDim = dim3(pl.grid);
-  lc.blockDim = dim3(kGemvThreads);
+  lc.blockDim = dim3(32 * (1 + pl.v.consumers));
   lc.dynamicSmemBytes = size_t(pl.smem);
   lc.stream = static_cast<cudaStream_t>(stream);
   cudaLaunchAttribute attr[1];
