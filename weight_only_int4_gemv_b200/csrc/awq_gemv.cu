@@ -234,17 +234,21 @@ struct StageLayout {
   static constexpr int kMetaStride = (kMetaBytes + 127) / 128 * 128;
 };
 
-// Consumer warps per CTA. Each SM sub-partition has its own quarter of the
-// register file, so the warp count (consumers + producer) is kept a multiple
-// of 4: 12 warps leave 168 registers per thread for one n8 batch tile, 8
-// warps leave 255 for two.
+// Consumer warps per CTA: 7, plus the producer, so each SM sub-partition's
+// quarter of the register file holds a whole number of warps. With one n8
+// batch tile a CTA is built to take half an SM (<= 128 registers per thread,
+// <= 113 KB of shared memory): one CTA per SM streams this layer while the
+// other half hosts the next kernel's CTA, which starts prefetching its
+// weights before this one finishes. With two batch tiles a CTA takes the
+// whole SM (255 registers per thread).
 template <int MT>
 struct Consumers {
-  static constexpr int value = MT == 1 ? 11 : 7;
+  static constexpr int value = 7;
+  static constexpr int ctas_per_sm = MT == 1 ? 2 : 1;
 };
 
 template <int MT, int RT, bool ZP>
-__global__ void __launch_bounds__(32 * (1 + Consumers<MT>::value), 1)
+__global__ void __launch_bounds__(32 * (1 + Consumers<MT>::value), Consumers<MT>::ctas_per_sm)
 gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_x,
             const __grid_constant__ CUtensorMap tmap_s, const __grid_constant__ CUtensorMap tmap_z,
             const GemvParams p) {
@@ -482,6 +486,9 @@ struct Variant {
 constexpr int kNumVariants = 4;
 constexpr int kRT = 4;
 constexpr int kSmemBudget = 232448;   // largest dynamic shared memory of one sm_100 CTA
+constexpr int kHalfSmBudget = 115712; // half of an SM's 228 KB, less the 1 KB reserved per CTA
+
+int smem_budget(const Variant& v);
 
 Variant pick_variant(int64_t M, bool zp) {
   if (M <= 8)
@@ -505,10 +512,12 @@ StageGeometry stage_geometry(const Variant& v, int64_t M, bool zp) {
   sg.x_offset = sg.code_bytes + sg.meta_stride * (zp ? 2 : 1);
   sg.stage_bytes = round128(sg.x_offset + int(M) * 256);
   sg.tx_bytes = uint32_t(sg.code_bytes + 16 * v.rt * 2 * (zp ? 2 : 1) + int(M) * 256);
-  int st = (kSmemBudget - kBarRegion) / (v.consumers * sg.stage_bytes);
+  int st = (smem_budget(v) - kBarRegion) / (v.consumers * sg.stage_bytes);
   sg.stages = st > kMaxStages ? kMaxStages : st;
   return sg;
 }
+
+int smem_budget(const Variant& v) { return v.mt == 1 ? kHalfSmBudget : kSmemBudget; }
 
 struct Plan {
   Variant v;
@@ -540,7 +549,7 @@ awq_status_t make_plan(int64_t M, int64_t N, int64_t K, bool zp, Plan& pl) {
     g_sm_count[dev].store(sms, std::memory_order_relaxed);
   }
   if (!g_smem_attr[dev][pl.v.id].load(std::memory_order_acquire)) {
-    if (cudaFuncSetAttribute(pl.v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBudget) != cudaSuccess)
+    if (cudaFuncSetAttribute(pl.v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_budget(pl.v)) != cudaSuccess)
       return AWQ_ERR_CUDA;
     g_smem_attr[dev][pl.v.id].store(1, std::memory_order_release);
   }
@@ -548,8 +557,9 @@ awq_status_t make_plan(int64_t M, int64_t N, int64_t K, bool zp, Plan& pl) {
   const int64_t G = K / kGroup;
   pl.nb = int((N + rows_per_block - 1) / rows_per_block);
   pl.units = int64_t(pl.nb) * G;
-  // one CTA per SM (the ring takes the SM's shared memory); fewer when
-  // there are fewer units than consumers
+  // one CTA per SM (for one batch tile it takes half the SM, leaving the
+  // other half to the next kernel); fewer when there are fewer units than
+  // consumers
   const int64_t want = (pl.units + pl.v.consumers - 1) / pl.v.consumers;
   pl.grid = int(want < sms ? (want > 0 ? want : 1) : sms);
   const int64_t total = int64_t(pl.grid) * pl.v.consumers;
