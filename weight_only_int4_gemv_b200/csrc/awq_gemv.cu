@@ -62,7 +62,7 @@ namespace {
 constexpr int kMaxConsumers = 12;
 constexpr int kMaxStages = 8;
 constexpr int kBarRegion = 2 * kMaxConsumers * kMaxStages * 8;   // full + empty mbarriers
-constexpr int kPrefetchUnits = 6;  // L2 prefetch distance, in units, per consumer
+constexpr int kPrefetchUnits = 1;  // L2 prefetch distance, in units, per consumer
 
 struct GemvParams {
   uint16_t* y;
