@@ -121,9 +121,17 @@ def measured_peaks():
         return HBM_FALLBACK_GBS, TENSOR_FALLBACK_TFLOPS, 0.0, "fallback"
 
 
+COMMON_SRC = os.path.join(ROOT, "weight_only_int4_gemv_b200", "csrc", "awq_common.cuh")
+
+
 def source_sha(path: str) -> str:
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    """First 16 hex digits of the SHA-256 of a kernel's .cu file followed by
+    the device helpers it includes, so a profile goes stale when either changes."""
+    h = hashlib.sha256()
+    for p in (path, COMMON_SRC):
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def profile_traffic(profile_path: str, source_path: str):
@@ -400,7 +408,7 @@ def run_native(args, dist):
                 "bound": "hbm", "achieved": round(kernel_gbs, 1), "peak": hbm_peak, "unit": "GB/s",
                 "frac": round(kernel_gbs / hbm_peak, 4),
                 "traffic": traffic, "peak_source": peak_src,
-                "kernel": "awq_gemv (gemv_kernel<1,2,true>)",
+                "kernel": "awq_gemv (gemv_kernel, M tile 1, asymmetric)",
                 "launches_timed": n_launch,
                 "algorithmic_bytes_per_launch": round(step_bytes / len(shapes)),
                 "mean_launch_us": round(1e6 * mean_launch_s, 3),
