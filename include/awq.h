@@ -63,7 +63,7 @@
 extern "C" {
 #endif
 
-#define AWQ_ABI_VERSION 1
+#define AWQ_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define AWQ_API __attribute__((visibility("default")))
@@ -83,11 +83,22 @@ typedef enum awq_status {
 
 /* Quantization configuration ("AutoAWQ" code tour, "From Install to Your
  * First Model": q_group_size, zero_point; w_bit is fixed at 4).
- * group_size must be 128. zero_point: 1 = asymmetric, 0 = symmetric. */
+ * group_size must be 128. zero_point: 1 = asymmetric, 0 = symmetric.
+ * flags: a bitwise OR of AWQ_FLAG_* values (0 for none); bits this library
+ * does not define are rejected with AWQ_ERR_UNSUPPORTED. */
 typedef struct awq_qconfig {
   int32_t group_size;
   int32_t zero_point;
+  uint32_t flags;
 } awq_qconfig_t;
+
+/* awq_gemv / awq_gemv_noalloc may start reading qweight, scales and zeros
+ * before the kernel launched just before them on the same stream has
+ * finished (it still waits for that kernel before it reads x or writes y).
+ * Set it only when no work still running on the stream writes those three
+ * arrays, for instance in a decode loop over weights loaded once. The other
+ * entry points ignore it. */
+#define AWQ_FLAG_WEIGHTS_STATIC 1u
 
 /* ABI version of the loaded library (AWQ_ABI_VERSION at build time). */
 AWQ_API int awq_abi_version(void);
@@ -152,8 +163,10 @@ AWQ_API awq_status_t awq_workspace_bytes(int64_t M, int64_t N, int64_t K,
  * device and shape, so results are reproducible run to run.
  * M in [1, 16]; N >= 0 and N % 8 == 0 (0: no work); K > 0, K % group_size == 0.
  * (N % 8 keeps every 8-row run of scales and zero points 16-byte aligned.)
+ * cfg.flags may hold AWQ_FLAG_WEIGHTS_STATIC (see there).
  * workspace: at least awq_workspace_bytes(M, N, K) bytes, zero-filled before
- * first use (see above); may be NULL when that size is 0.
+ * first use (see above); may be NULL when that size is 0, which is the case
+ * whenever N / 16 is at least the device's SM count.
  */
 AWQ_API awq_status_t awq_gemv(const uint16_t* x, const int32_t* qweight,
                       const uint16_t* scales, const uint16_t* zeros,
@@ -182,7 +195,7 @@ AWQ_API awq_status_t awq_gemv(const uint16_t* x, const int32_t* qweight,
  * array: calls that may overlap on the GPU (different streams, or
  * concurrent host threads) race and must be serialized by the caller.
  */
-#define AWQ_GEMV_STATIC_WORKSPACE_BYTES (16u << 20)
+#define AWQ_GEMV_STATIC_WORKSPACE_BYTES (1u << 20)
 AWQ_API awq_status_t awq_gemv_noalloc(const uint16_t* x, const int32_t* qweight,
                                       const uint16_t* scales, const uint16_t* zeros,
                                       int64_t M, int64_t N, int64_t K, awq_qconfig_t cfg,

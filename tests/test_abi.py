@@ -34,8 +34,8 @@ def L():
     return awq.lib()
 
 
-def cfg(g=128, zp=1):
-    return awq.QConfig(g, zp)
+def cfg(g=128, zp=1, flags=0):
+    return awq.QConfig(g, zp, flags)
 
 
 def test_header_declares_the_entry_points():
@@ -84,6 +84,9 @@ def test_product_validation(L, entry):
     assert _gemv(L, x=MIS, entry=entry) == ALIGN
     assert _gemv(L, y=MIS, entry=entry) == ALIGN
     assert _gemv(L, N=0, entry=entry) == OK                     # empty: no work, no CUDA call
+    assert _gemv(L, c=cfg(flags=2), entry=entry) == UNSUP       # undefined flag bits
+    assert _gemv(L, c=cfg(flags=0x80000000), entry=entry) == UNSUP
+    assert _gemv(L, N=0, c=cfg(flags=awq.FLAG_WEIGHTS_STATIC), entry=entry) == OK
 
 
 def test_gemv_batch_range(L):
@@ -102,6 +105,7 @@ def test_quantize_and_dequant_validation(L):
     assert q(P(A), 8, 100, cfg(), P(A), P(A), P(A), None) == SHAPE
     assert q(P(MIS), 8, 256, cfg(), P(A), P(A), P(A), None) == ALIGN
     assert q(P(A), 0, 256, cfg(), P(A), P(A), P(A), None) == OK
+    assert q(P(A), 8, 256, cfg(flags=4), P(A), P(A), P(A), None) == UNSUP
     d = L.awq_dequant
     assert d(None, P(A), P(A), 8, 256, cfg(), P(A), None) == NULL
     assert d(P(A), P(A), P(A), 8, 256, cfg(g=32), P(A), None) == UNSUP

@@ -18,12 +18,12 @@ from workloads import make_layer, make_packed_random, make_weight
 pytestmark = pytest.mark.gpu
 
 
-def run_gemv(x, qweight, scales, zeros):
+def run_gemv(x, qweight, scales, zeros, weights_static=False):
     M, K = x.shape
     N = qweight.shape[0]
     ws = awq.alloc_workspace(M, N, K, zeros is not None)
     y = awq.awq_gemv(dev(x), dev(qweight), dev(scales), dev(zeros) if zeros is not None else None,
-                     workspace=ws)
+                     workspace=ws, weights_static=weights_static)
     torch.cuda.synchronize()
     return host(y), ws
 
@@ -95,16 +95,18 @@ def test_gemv_random_codes_and_extreme_zero_points():
 
 
 def test_gemv_is_deterministic_and_reuses_its_workspace():
-    """Repeated calls on one workspace give identical bits and stay correct:
-    a split block is finished only when its arrival counter reaches the
-    group count, so a counter left non-zero would leave blocks unfinished."""
-    _, qweight, scales, zeros, Wd = oracle_layer(4096, 14336, 0.02, 0.0, True)
+    """Repeated calls on one workspace give identical bits and stay correct.
+    N = 1024 has fewer 16-channel tiles than the GPU has SMs, so K is cut
+    into slices that different CTAs sum; a tile is finished only when its
+    arrival counter reaches the slice count, so a counter left non-zero would
+    leave tiles unfinished."""
+    _, qweight, scales, zeros, Wd = oracle_layer(1024, 14336, 0.02, 0.0, True)
     x = activations(4, 14336, seed=3)
-    ws = awq.alloc_workspace(4, 4096, 14336, True)
+    ws = awq.alloc_workspace(4, 1024, 14336, True)
     assert ws is not None
     ys = []
     for _ in range(4):
-        y = torch.full((4, 4096), float("nan"), dtype=torch.float16, device="cuda")
+        y = torch.full((4, 1024), float("nan"), dtype=torch.float16, device="cuda")
         awq.awq_gemv(dev(x), dev(qweight), dev(scales), dev(zeros), workspace=ws, out=y)
         torch.cuda.synchronize()
         ys.append(bits(y))
@@ -113,10 +115,54 @@ def test_gemv_is_deterministic_and_reuses_its_workspace():
     assert_close(ys[-1].view(np.float16), O.matmul_f64(x, Wd), "4th call")
 
 
+def test_gemv_whole_tiles_need_no_workspace():
+    """With at least one 16-channel tile per SM every CTA covers all of K for
+    its tiles: no workspace, and the call works without one."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    for M, N, K in [(1, 16 * sms, 4096), (8, 4096, 14336), (16, 14336, 4096)]:
+        assert awq.awq_workspace_bytes(M, N, K, True) == 0
+    _, qweight, scales, zeros, Wd = oracle_layer(16 * sms, 1024, 0.02, 0.01, True)
+    x = activations(2, 1024, seed=7)
+    y = host(awq.awq_gemv(dev(x), dev(qweight), dev(scales), dev(zeros), workspace=None))
+    assert_close(y, O.matmul_f64(x, Wd), "N = 16 x SMs")
+
+
+@pytest.mark.parametrize("zp", [True, False])
+@pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (1, 14336, 4096), (8, 4096, 14336), (16, 1000, 2048),
+                                   (3, 40, 256), (1, 2360, 1024)])
+def test_gemv_weights_static_gives_the_same_bits(M, N, K, zp):
+    """AWQ_FLAG_WEIGHTS_STATIC only moves when the weights are read (before
+    the previous kernel on the stream completes), never what is computed."""
+    _, qweight, scales, zeros, Wd = oracle_layer(N, K, 0.02, 0.01, zp)
+    x = activations(M, K, seed=5)
+    y0, _ = run_gemv(x, qweight, scales, zeros)
+    y1, _ = run_gemv(x, qweight, scales, zeros, weights_static=True)
+    assert np.array_equal(bits(y0), bits(y1))
+    assert_close(y1, O.matmul_f64(x, Wd), f"static M={M} N={N} K={K}")
+
+
+def test_gemv_back_to_back_layers_weights_static():
+    """A chain of dependent layers on one stream with the flag set: each
+    layer's x is the previous layer's y, written by the kernel just before."""
+    layers = [oracle_layer(1024, 1024, 0.02, 0.01, True, seed=s) for s in range(4)]
+    x0 = activations(2, 1024, seed=9)
+    xs = [dev(x0)]
+    for (_, q, s, z, _) in layers:
+        y = awq.awq_gemv(xs[-1], dev(q), dev(s), dev(z), workspace=awq.alloc_workspace(2, 1024, 1024, True),
+                         weights_static=True)
+        xs.append(y)
+    torch.cuda.synchronize()
+    xr = x0.astype(np.float64)
+    for i, (_, _, _, _, Wd) in enumerate(layers):
+        yr = O.matmul_f64(xr.astype(np.float16), Wd)
+        assert_close(host(xs[i + 1]), yr, f"layer {i}")
+        xr = host(xs[i + 1]).astype(np.float64)
+
+
 def test_gemv_workspace_required_and_checked():
-    _, qweight, scales, zeros, _ = oracle_layer(4096, 4096, 0.02, 0.01, True)
+    _, qweight, scales, zeros, _ = oracle_layer(1024, 4096, 0.02, 0.01, True)
     x = dev(activations(2, 4096))
-    need = awq.awq_workspace_bytes(2, 4096, 4096, True)
+    need = awq.awq_workspace_bytes(2, 1024, 4096, True)
     assert need > 0
     small = torch.zeros(need - 16, dtype=torch.uint8, device="cuda")
     with pytest.raises(awq.AwqError, match="WORKSPACE"):

@@ -42,8 +42,17 @@ class AwqError(RuntimeError):
         self.status = status
 
 
+ABI_VERSION = 2   # awq_abi_version() of a library this binding matches
+
+
 class QConfig(ctypes.Structure):
-    _fields_ = [("group_size", ctypes.c_int32), ("zero_point", ctypes.c_int32)]
+    _fields_ = [("group_size", ctypes.c_int32), ("zero_point", ctypes.c_int32), ("flags", ctypes.c_uint32)]
+
+
+# awq_qconfig_t.flags bit: qweight / scales / zeros are not written by work
+# still running on the stream, so the GEMV may read them before the previous
+# kernel finishes (it still waits for that kernel before reading x).
+FLAG_WEIGHTS_STATIC = 1
 
 
 _lib = None
@@ -79,6 +88,9 @@ def lib():
                     f = getattr(h, name)
                     f.restype = res
                     f.argtypes = args
+                if h.awq_abi_version() != ABI_VERSION:
+                    raise RuntimeError(f"{LIB_PATH} has ABI version {h.awq_abi_version()}, this binding "
+                                       f"needs {ABI_VERSION}: rebuild it")
                 _lib = h
     return _lib
 
@@ -88,8 +100,8 @@ def _check(fn: str, st: int):
         raise AwqError(fn, st, lib().awq_status_string(st).decode())
 
 
-def _cfg(zero_point: bool, group_size: int) -> QConfig:
-    return QConfig(group_size, 1 if zero_point else 0)
+def _cfg(zero_point: bool, group_size: int, flags: int = 0) -> QConfig:
+    return QConfig(group_size, 1 if zero_point else 0, flags)
 
 
 def _ptr(t):
@@ -164,7 +176,7 @@ def alloc_workspace(M: int, N: int, K: int, zero_point: bool = True, device=None
     return torch.zeros(nbytes, dtype=torch.uint8, device=dev) if nbytes else None
 
 
-def _product(entry: str, x, qweight, scales, zeros, workspace, out, group_size):
+def _product(entry: str, x, qweight, scales, zeros, workspace, out, group_size, flags=0):
     _need(x, "x", torch.float16, 2)
     _need(qweight, "qweight", torch.int32, 2)
     _need(scales, "scales", torch.float16, 2)
@@ -188,17 +200,23 @@ def _product(entry: str, x, qweight, scales, zeros, workspace, out, group_size):
     with torch.cuda.device(x.device):
         fn = getattr(lib(), entry)
         _check(entry, fn(_ptr(x), _ptr(qweight), _ptr(scales), _ptr(zeros), M, N, K,
-                         _cfg(zeros is not None, group_size), _ptr(out), ws_ptr, ws_bytes,
+                         _cfg(zeros is not None, group_size, flags), _ptr(out), ws_ptr, ws_bytes,
                          _stream(x.device)))
     return out
 
 
-def awq_gemv(x, qweight, scales, zeros, workspace=None, out=None, group_size: int = GROUP_SIZE):
-    """y = x . W'^T for 1 <= M <= 16 (decode). `workspace` from alloc_workspace()."""
-    return _product("awq_gemv", x, qweight, scales, zeros, workspace, out, group_size)
+def awq_gemv(x, qweight, scales, zeros, workspace=None, out=None, group_size: int = GROUP_SIZE,
+             weights_static: bool = False):
+    """y = x . W'^T for 1 <= M <= 16 (decode). `workspace` from alloc_workspace().
+    weights_static: no work still running on the stream writes qweight, scales
+    or zeros (a decode loop over loaded weights), so the kernel may start
+    streaming them before the previous kernel on the stream has finished."""
+    return _product("awq_gemv", x, qweight, scales, zeros, workspace, out, group_size,
+                    FLAG_WEIGHTS_STATIC if weights_static else 0)
 
 
-def awq_gemv_noalloc(x, qweight, scales, zeros, out=None, group_size: int = GROUP_SIZE):
+def awq_gemv_noalloc(x, qweight, scales, zeros, out=None, group_size: int = GROUP_SIZE,
+                     weights_static: bool = False):
     """awq_gemv with the library's fixed scratch array instead of a workspace,
     for callers that cannot allocate device memory when they run the layer.
     Calls on one device share the array and must not overlap on the GPU."""
@@ -216,7 +234,8 @@ def awq_gemv_noalloc(x, qweight, scales, zeros, out=None, group_size: int = GROU
     _need(out, "out", torch.float16, 2)
     with torch.cuda.device(x.device):
         _check("awq_gemv_noalloc", lib().awq_gemv_noalloc(
-            _ptr(x), _ptr(qweight), _ptr(scales), _ptr(zeros), M, N, K, _cfg(zeros is not None, group_size),
+            _ptr(x), _ptr(qweight), _ptr(scales), _ptr(zeros), M, N, K,
+            _cfg(zeros is not None, group_size, FLAG_WEIGHTS_STATIC if weights_static else 0),
             _ptr(out), _stream(x.device)))
     return out
 
@@ -226,10 +245,12 @@ def awq_gemm(x, qweight, scales, zeros, workspace=None, out=None, group_size: in
     return _product("awq_gemm", x, qweight, scales, zeros, workspace, out, group_size)
 
 
-def awq_linear(x, qweight, scales, zeros, workspace=None, out=None, group_size: int = GROUP_SIZE):
+def awq_linear(x, qweight, scales, zeros, workspace=None, out=None, group_size: int = GROUP_SIZE,
+               weights_static: bool = False):
     """The layer with the documented M threshold: awq_gemv for M <= 16, else awq_gemm."""
     entry = "awq_gemv" if x.shape[0] <= GEMV_MAX_M else "awq_gemm"
-    return _product(entry, x, qweight, scales, zeros, workspace, out, group_size)
+    return _product(entry, x, qweight, scales, zeros, workspace, out, group_size,
+                    FLAG_WEIGHTS_STATIC if weights_static else 0)
 
 
 def awq_device_error(device=None) -> int:

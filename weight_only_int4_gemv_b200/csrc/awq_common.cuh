@@ -20,6 +20,7 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 inline awq_status_t check_cfg(awq_qconfig_t cfg) {
   if (cfg.group_size != kGroup) return AWQ_ERR_UNSUPPORTED;
   if (cfg.zero_point != 0 && cfg.zero_point != 1) return AWQ_ERR_UNSUPPORTED;
+  if (cfg.flags & ~AWQ_FLAG_WEIGHTS_STATIC) return AWQ_ERR_UNSUPPORTED;
   return AWQ_OK;
 }
 
@@ -202,6 +203,24 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const void* tensor_map, i
       "[%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(tensor_map)), "r"(x), "r"(y), "r"(smem_u32(bar))
       : "memory");
+}
+
+// 3-D tiled TMA load of one box into shared memory, completing on `bar`.
+__device__ __forceinline__ void tma_load_3d(void* dst, const void* tensor_map, int x, int y, int z,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tensor_map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Prefetch one 3-D box of a tensor from global memory into L2.
+__device__ __forceinline__ void tma_prefetch_l2_3d(const void* tensor_map, int x, int y, int z) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                   reinterpret_cast<uint64_t>(tensor_map)),
+               "r"(x), "r"(y), "r"(z)
+               : "memory");
 }
 
 // Prefetch one 2-D box of a tensor from global memory into L2 (no data

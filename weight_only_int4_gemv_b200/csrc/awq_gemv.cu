@@ -7,16 +7,27 @@
 // The layer is bound by HBM: every packed code byte is read once and feeds
 // only M multiply-adds. Design:
 //
-// * Work unit = (row block of 16*RT output channels, one group of 128 k).
-//   Units are ordered block-major and split evenly over every warp of a grid
-//   sized to the resident capacity of the GPU (a stream-K split): all SMs
-//   stream the same number of bytes whatever N and K are.
-// * Each warp owns an S-stage ring in shared memory. Lane 0 fills a stage
-//   with TMA: one 2-D box of packed codes (16*RT rows x 64 bytes), one box
-//   of x (M rows x 128 k), and the 16*RT-long runs of scales and zero points
-//   (group-major metadata makes them contiguous), all completing on the
-//   stage's mbarrier. Units S-1 ahead of the arithmetic stay in flight
-//   without holding registers or L1 request slots.
+// * Output channels come in tiles of 16 (one MMA tile). Each CTA owns a
+//   contiguous run of whole tiles over the whole of K, so no partial sum
+//   ever leaves the SM: the CTA's 8 warps split K between them and reduce
+//   through shared memory. Tiles are spread evenly over one CTA per SM (at
+//   most one tile of difference). Only when there are fewer tiles than SMs
+//   is K also cut into slices handled by different CTAs; their fp32
+//   partials meet in a workspace and the last CTA to arrive on a tile sums
+//   them in slice order.
+// * A CTA walks its tiles in chunks of up to four (64 channels). Within a
+//   chunk, the K range goes by in stages of 8 groups, one group per warp: a
+//   unit of work is (chunk, group), 16 words x up to 64 rows of codes.
+// * The stages form one ring per CTA in shared memory, filled by TMA with a
+//   few large boxes per stage: the codes through a 3-D view of qweight that
+//   lands them group-major ([group][16 rows][16 words] per tile, so a warp's
+//   16-byte reads hit distinct banks), the 64 x 8 blocks of scales and zero
+//   points (group-major metadata), and x as [m][group][128 k]. A TMA issue
+//   can hold its thread for hundreds of cycles, so few, large copies keep
+//   that cost off the arithmetic. Each warp takes its group of a stage into
+//   registers and counts itself out of the stage; the last of the 8 warps
+//   refills the stage with the one S ahead, so no warp ever waits for
+//   another.
 // * Decode: the packed nibble order puts consecutive k pairs in the low and
 //   high halves of a word, so one LOP3 turns a word into two exact fp16
 //   integers, 1024+q for the pairs (0,1), (4,5) and 64+q for (2,3), (6,7):
@@ -26,27 +37,25 @@
 //   n dimension, two n8 tiles for M > 8). The k positions inside an MMA are
 //   a permutation of the word's k (each lane owns whole words), matched by
 //   reading x[m][8w .. 8w+7] for the same words: one 16-byte read covers two
-//   MMAs. Products are exact and accumulation is fp32. The RT row tiles are
-//   independent accumulator chains, interleaved.
+//   MMAs. Products are exact and accumulation is fp32.
 // * Offsets and scale, once per group and batch row, in fp32:
 //   sum_k x (q - z) = raw - C(m) - z S(m), with raw the MMA sum over the
 //   magic-offset values, C(m) = 1024 sum_{k: 1024 pairs} x + 64 sum_{k: 64
 //   pairs} x and S(m) = sum_k x. C and S come from two more MMAs against a
-//   constant tile (rows 0 and 1), shared by all rows of the unit. Then
-//   acc += s (raw - C - z S): the scale multiplies the group's partial sum.
-// * A row block split between warps is finished by the last warp to arrive
-//   (arrival counter per block): it sums the contributors' fp32 partials in
-//   a fixed order, so results do not depend on timing, and resets the
-//   counter for the next call. No warp ever waits on another.
+//   constant tile (rows 0 and 1). Then acc += s (raw - C - z S).
 // * Programmatic dependent launch: every CTA lets the next kernel launch as
-//   soon as it runs, and prefetches its first weight units from HBM into L2
-//   before waiting for the previous kernel (griddepcontrol.wait); loads into
-//   shared memory, workspace accesses and y stores come after the wait.
-//   Back-to-back layers overlap their launch and HBM ramp-up with the
-//   previous layer's tail. The L2 prefetch runs kPrefetchUnits ahead.
+//   soon as it runs. Before waiting for the previous kernel
+//   (griddepcontrol.wait) a CTA only prefetches its first code box into L2
+//   (always safe), or, when the caller declares the weights static
+//   (AWQ_FLAG_WEIGHTS_STATIC), already loads the codes, scales and zero
+//   points of its first S stages into its ring; x, the workspace and y are
+//   touched only after the wait. For M = 1 a CTA takes half an SM so that
+//   the next layer's CTA can sit beside it and fill its ring meanwhile.
 // * Every mbarrier wait is bounded (2 s); a warp that gives up records bit 1
-//   of the device error word, waits (bounded) for its copies in flight and
-//   leaves its rows unwritten.
+//   of the device error word, stops waiting and stops releasing stages,
+//   still takes part in its CTA's reductions (so no CTA barrier can hang),
+//   and before the CTA exits thread 0 waits (bounded) for the fills still in
+//   flight. The output is then incomplete.
 
 #include <atomic>
 
@@ -59,23 +68,35 @@ __device__ uint32_t g_awq_gemv_error = 0;
 
 namespace {
 
-constexpr int kMaxConsumers = 12;
+constexpr int kWarps = 8;                      // warps per CTA, each with its own ring
+constexpr int kThreads = 32 * kWarps;
+constexpr int kTile = 16;                      // output channels per MMA tile
+constexpr int kChunkTiles = 4;                 // tiles accumulated together
+constexpr int kChunkRows = kTile * kChunkTiles;
 constexpr int kMaxStages = 8;
-constexpr int kBarRegion = 2 * kMaxConsumers * kMaxStages * 8;   // full + empty mbarriers
-constexpr int kPrefetchUnits = 1;  // L2 prefetch distance, in units, per consumer
+constexpr int kRingOffset = 1024;              // mbarriers and counters live below the ring
+// One stage = one chunk x kWarps groups (one group per warp):
+constexpr int kTileStageBytes = kWarps * kTile * 64;    // codes of one tile: [group][16 rows][16 words]
+constexpr int kMetaStageBytes = kWarps * kChunkRows * 2;  // [group][64 rows] fp16 scales (or zeros)
+constexpr int kXStageBytesPerRow = kWarps * 128 * 2;      // x: [m][group][128 k] fp16
+constexpr int kReduceBarrier = 1;              // named barrier of the chunk reductions
+static_assert(kMaxStages * (8 + 4 + 4) + 4 <= kRingOffset, "stage bookkeeping overflows its region");
 
 struct GemvParams {
   uint16_t* y;
-  float* partials;       // [total consumers][2][16*RT*M] floats, [row][m]
-  uint32_t* counters;    // [nb]
-  int64_t units;         // nb * G
-  int M, N, K, G, nb;
-  int consumers;         // consumer warps per CTA
-  int total_consumers;   // grid * consumers
-  int stages;            // ring stages per consumer
+  float* partials;       // [ks][T * 16][M] fp32, only when ks > 1
+  uint32_t* counters;    // [T], only when ks > 1
+  int M, N, G;
+  int T;                 // tiles of 16 output channels
+  int ks;                // K slices (1: every CTA covers all of K)
+  int items;             // T * ks, slice-major: item i is tile i % T of slice i / T
+  int stages;            // ring stages per warp
   int stage_bytes;       // codes + metadata + x slice of one unit (multiple of 128)
   int x_offset;          // offset of the x slice inside a stage
-  uint32_t tx_bytes;     // bytes the TMA copies of one unit deliver
+  int pbuf_offset;       // shared-memory partial sums of the chunk reductions
+  int chunk_tiles;       // tiles per chunk (the kernel's TC)
+  int scale_offset;      // offset of the scales inside a stage (TC tiles of codes before it)
+  int early;             // weights may be read before the previous kernel completes
 };
 
 __device__ __forceinline__ uint4 lds128(const uint8_t* p) { return *reinterpret_cast<const uint4*>(p); }
@@ -94,128 +115,8 @@ __device__ __forceinline__ uint32_t word_of(const uint4& v, int i) {
   return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
 
-// First unit of consumer w in the even split of `units` over `consumers`.
-__device__ __forceinline__ int64_t range_start(int64_t units, int64_t w, int64_t consumers) {
-  return units * w / consumers;
-}
-
-template <int MT, int RT>
-__device__ __forceinline__ void store_y(const GemvParams& p, int64_t row0, int g, int t,
-                                        const float (&acc)[RT][MT][4]) {
-#pragma unroll
-  for (int rt = 0; rt < RT; ++rt) {
-    const int64_t r_lo = row0 + 16 * rt + g;
-    const int64_t r_hi = r_lo + 8;
-#pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
-      const int m0 = 8 * mt + 2 * t;
-      if (m0 < p.M) {
-        if (r_lo < p.N) p.y[int64_t(m0) * p.N + r_lo] = __half_as_ushort(__float2half_rn(acc[rt][mt][0]));
-        if (r_hi < p.N) p.y[int64_t(m0) * p.N + r_hi] = __half_as_ushort(__float2half_rn(acc[rt][mt][2]));
-      }
-      if (m0 + 1 < p.M) {
-        if (r_lo < p.N) p.y[int64_t(m0 + 1) * p.N + r_lo] = __half_as_ushort(__float2half_rn(acc[rt][mt][1]));
-        if (r_hi < p.N) p.y[int64_t(m0 + 1) * p.N + r_hi] = __half_as_ushort(__float2half_rn(acc[rt][mt][3]));
-      }
-    }
-  }
-}
-
-// Finish row block b after consumer gc summed groups [j0, j1) of it.
-// A split block's partial sums are stored compactly (the block's 16*RT rows
-// x M batch rows, [row][m]); the consumer that completes the block's group
-// count sums every contributor's values in consumer order (reproducible
-// bits), loading many contributors at once.
-template <int MT, int RT>
-__device__ __forceinline__ void finish_block(const GemvParams& p, int64_t b, int j0, int j1, int64_t gc,
-                                             int64_t first_block, int lane, int g, int t,
-                                             const float (&acc)[RT][MT][4]) {
-  const int64_t row0 = b * (16 * RT);
-  const int64_t G = p.G;
-  if (j0 == 0 && j1 == G) {
-    store_y<MT, RT>(p, row0, g, t, acc);
-    return;
-  }
-  const int M = p.M;
-  const int V = 16 * RT * M;                     // values of one partial
-  const int slot = (b == first_block) ? 0 : 1;
-  float* sp = p.partials + (gc * 2 + slot) * int64_t(V);
-#pragma unroll
-  for (int rt = 0; rt < RT; ++rt)
-#pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
-      const int m0 = 8 * mt + 2 * t;
-      const int r_lo = 16 * rt + g, r_hi = r_lo + 8;
-      if (m0 < M) {
-        __stcg(sp + r_lo * M + m0, acc[rt][mt][0]);
-        __stcg(sp + r_hi * M + m0, acc[rt][mt][2]);
-      }
-      if (m0 + 1 < M) {
-        __stcg(sp + r_lo * M + m0 + 1, acc[rt][mt][1]);
-        __stcg(sp + r_hi * M + m0 + 1, acc[rt][mt][3]);
-      }
-    }
-  __syncwarp();   // every lane's stores happen before lane 0's release below
-  uint32_t last = 0;
-  if (lane == 0) {
-    const uint32_t mine = uint32_t(j1 - j0);
-    uint32_t old;
-    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;"
-                 : "=r"(old) : "l"(p.counters + b), "r"(mine) : "memory");
-    last = (old + mine == uint32_t(G)) ? 1u : 0u;
-  }
-  last = __shfl_sync(0xffffffffu, last, 0);
-  if (!last) return;
-  // Contributors: every non-empty consumer range overlapping block b, in
-  // consumer order. Range starts floor(units * w / W) advance by
-  // floor(units / W) plus a carry, so no division happens per contributor.
-  const int64_t W = p.total_consumers;
-  const int64_t w_first = ((b * G + 1) * W - 1) / p.units;
-  const int64_t w_last = ((b * G + G) * W - 1) / p.units;
-  const int64_t q_step = p.units / W, r_step = p.units % W;
-  const int64_t bG = b * G;
-  constexpr int kChunk = 16;                     // contributors loaded at once
-  const int nv = V / 32;                         // values per lane (V = 64 M), two per pass
-  for (int v0 = 0; v0 < nv; v0 += 2) {
-    int64_t ws = range_start(p.units, w_first, W);
-    int64_t rem = (p.units * w_first) % W;
-    float acc2[2] = {0.0f, 0.0f};
-    for (int64_t w0 = w_first; w0 <= w_last; w0 += kChunk) {
-      float part[kChunk][2];
-#pragma unroll
-      for (int c = 0; c < kChunk; ++c) {
-        const int64_t w = w0 + c;
-        int64_t we = ws + q_step;                // start of range w + 1
-        int64_t rem2 = rem + r_step;
-        if (rem2 >= W) { rem2 -= W; ++we; }
-        const bool live = w <= w_last && ws < we;
-        const int s = ws >= bG ? 0 : 1;          // block b is the range's first block, or its last
-        const float* src = p.partials + (w * 2 + s) * int64_t(V);
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int v = lane + 32 * (v0 + e);
-          part[c][e] = (live && v < V) ? __ldcg(src + v) : 0.0f;
-        }
-        ws = we;
-        rem = rem2;
-      }
-#pragma unroll
-      for (int c = 0; c < kChunk; ++c) {
-        acc2[0] += part[c][0];
-        acc2[1] += part[c][1];
-      }
-    }
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int v = lane + 32 * (v0 + e);
-      if (v < V) {
-        const int row = v / M, m = v - row * M;
-        if (row0 + row < p.N)
-          p.y[int64_t(m) * p.N + row0 + row] = __half_as_ushort(__float2half_rn(acc2[e]));
-      }
-    }
-  }
-  if (lane == 0) p.counters[b] = 0u;
+__device__ __forceinline__ void named_barrier_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
 // A fragment of the constant 16x16 tile that turns two extra MMAs into the
@@ -227,307 +128,442 @@ __device__ __forceinline__ void offset_tile(int g, uint32_t& a0, uint32_t& a2) {
   a2 = g == 0 ? 0x54005400u : (g == 1 ? 0x3C003C00u : 0u);
 }
 
-template <int RT>
-struct StageLayout {
-  static constexpr int kCodeBytes = 16 * RT * 64;   // [16*RT rows][16 words]
-  static constexpr int kMetaBytes = 16 * RT * 2;    // one fp16 per row of the block
-  static constexpr int kMetaStride = (kMetaBytes + 127) / 128 * 128;
+// A run of up to kChunkTiles consecutive tiles of one K slice inside a CTA's
+// item range, with the slice's groups [gb, ge).
+struct Chunk {
+  int i;       // first item
+  int tc;      // tiles
+  int t0;      // first tile
+  int s;       // slice
+  int gb, ge;  // groups of the slice
 };
 
-// Consumer warps per CTA: 7, plus the producer, so each SM sub-partition's
-// quarter of the register file holds a whole number of warps. With one n8
-// batch tile a CTA is built to take half an SM (<= 128 registers per thread,
-// <= 113 KB of shared memory): one CTA per SM streams this layer while the
-// other half hosts the next kernel's CTA, which starts prefetching its
-// weights before this one finishes. With two batch tiles a CTA takes the
-// whole SM (255 registers per thread).
+__device__ __forceinline__ void load_chunk(const GemvParams& p, int i, int i_end, Chunk& c) {
+  c.i = i;
+  c.s = i / p.T;
+  c.t0 = i - c.s * p.T;
+  int tc = i_end - i;
+  if (tc > p.chunk_tiles) tc = p.chunk_tiles;
+  if (tc > p.T - c.t0) tc = p.T - c.t0;
+  c.tc = tc;
+  c.gb = int(int64_t(p.G) * c.s / p.ks);
+  c.ge = int(int64_t(p.G) * (c.s + 1) / p.ks);
+}
+
+// The CTA's sequence of stages: for each chunk, its groups in blocks of
+// kWarps. Every warp walks the same sequence; lane 0 of each warp also keeps
+// a second cursor S stages ahead, for the refill it may have to issue.
+// gbase < 0 once the sequence is exhausted.
+struct StageCursor {
+  Chunk c;
+  int gbase;   // first group of the stage
+  __device__ __forceinline__ bool done() const { return gbase < 0; }
+};
+
+__device__ __forceinline__ void cursor_init(const GemvParams& p, int i0, int i1, StageCursor& u) {
+  load_chunk(p, i0, i1, u.c);
+  u.gbase = u.c.gb;
+}
+
+__device__ __forceinline__ void cursor_next(const GemvParams& p, int i_end, StageCursor& u) {
+  u.gbase += kWarps;
+  if (u.gbase >= u.c.ge) {
+    const int ni = u.c.i + u.c.tc;
+    if (ni >= i_end) {
+      u.gbase = -1;
+    } else {
+      load_chunk(p, ni, i_end, u.c);
+      u.gbase = u.c.gb;
+    }
+  }
+}
+
+__device__ __forceinline__ uint32_t stage_tx_bytes(const GemvParams& p, int tc, bool zp) {
+  return uint32_t(tc * kTileStageBytes + kMetaStageBytes * (zp ? 2 : 1) + p.M * kXStageBytesPerRow);
+}
+
+// Copies of the weight part of a stage: for each tile one 3-D box of codes
+// (16 words x 16 rows x 8 groups, landing group-major), and the 64-row runs
+// of scales and zero points of the 8 groups.
+template <bool ZP>
+__device__ __forceinline__ void issue_weights(const StageCursor& u, uint8_t* st, uint64_t* bar,
+                                              const CUtensorMap* tq, const CUtensorMap* ts,
+                                              const CUtensorMap* tz, int p_scale_offset) {
+  const int r0 = u.c.t0 * kTile;
+  for (int r = 0; r < u.c.tc; ++r) tma_load_3d(st + r * kTileStageBytes, tq, 0, r0 + r * kTile, u.gbase, bar);
+  tma_load_2d(st + p_scale_offset, ts, r0, u.gbase, bar);
+  if (ZP) tma_load_2d(st + p_scale_offset + kMetaStageBytes, tz, r0, u.gbase, bar);
+}
+
+// Per-warp state of the stage pipeline.
 template <int MT>
-struct Consumers {
-  static constexpr int value = 7;
-  static constexpr int ctas_per_sm = MT == 1 ? 2 : 1;
+struct Pipe {
+  uint8_t* ring;
+  uint64_t* full;
+  uint32_t* released;
+  uint32_t* fills;
+  uint32_t* failed;
+  const CUtensorMap* tq;
+  const CUtensorMap* tx;
+  const CUtensorMap* ts;
+  const CUtensorMap* tz;
+  StageCursor pc;      // lane 0: the stage S ahead of the arithmetic
+  int slot;
+  uint32_t phase;
+  bool ok;
+  int S, i1;
+  int lane, w, g, t;
+  int xoff[MT];
+  bool xok[MT];
+  uint32_t ca0, ca2;
 };
 
-template <int MT, int RT, bool ZP>
-__global__ void __launch_bounds__(32 * (1 + Consumers<MT>::value), Consumers<MT>::ctas_per_sm)
+// The stages of one chunk: wait for a stage, take this warp's group into
+// registers, release the stage (the last warp refills it), then decode and
+// multiply into acc. All TC tile slots are computed, so the unrolled loops
+// carry no branches; in a chunk with fewer tiles the extra slots hold stale
+// shared memory and their rows are never stored.
+template <int MT, bool ZP, int TC>
+__device__ __forceinline__ void chunk_stages(const GemvParams& p, Pipe<MT>& pp, const Chunk& cc,
+                                             float (&acc)[kChunkTiles][MT][4], volatile int* abort_flag) {
+    for (int gbase = cc.gb; gbase < cc.ge; gbase += kWarps) {
+      if (pp.ok) {
+        pp.ok = __all_sync(0xffffffffu, wait_bounded(&pp.full[pp.slot], pp.phase, abort_flag, &g_awq_gemv_error, 2u));
+        if (!pp.ok && pp.lane == 0) atomicOr(pp.failed, 1u);
+      }
+      const uint8_t* st = pp.ring + pp.slot * p.stage_bytes;
+      const bool has = pp.ok && gbase + pp.w < cc.ge;   // this warp's group of the stage
+      uint4 xf[MT][4];
+      uint4 c_lo[kChunkTiles], c_hi[kChunkTiles];
+      uint32_t s2[kChunkTiles], z2[kChunkTiles];
+      if (has) {
+        // the unit's data, into registers: codes of rows pp.g and pp.g+8 of each
+        // tile; scales and zero points of the same two rows as fp16 pairs
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) xf[mt][jj] = pp.xok[mt] ? lds128(st + pp.xoff[mt] + jj * 16) : make_uint4(0, 0, 0, 0);
+        const uint8_t* cw = st + pp.w * (kTile * 64) + pp.g * 64 + pp.t * 16;
+        const uint8_t* sw = st + TC * kTileStageBytes + pp.w * 128 + pp.g * 2;
+#pragma unroll
+        for (int rt = 0; rt < TC; ++rt) {
+          c_lo[rt] = lds128(cw + rt * kTileStageBytes);
+          c_hi[rt] = lds128(cw + rt * kTileStageBytes + 8 * 64);
+          s2[rt] = uint32_t(lds16(sw + rt * 32)) | (uint32_t(lds16(sw + rt * 32 + 16)) << 16);
+          z2[rt] = ZP ? (uint32_t(lds16(sw + kMetaStageBytes + rt * 32)) |
+                         (uint32_t(lds16(sw + kMetaStageBytes + rt * 32 + 16)) << 16))
+                      : 0x48004800u;   // 8.0 in both halves
+        }
+      }
+      // Release the stage; the last of the CTA's warps to do so refills it
+      // with the stage pp.S ahead.
+      __syncwarp();
+      if (pp.lane == 0 && pp.ok) {
+        uint32_t before;
+        asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], 1;"
+                     : "=r"(before) : "r"(smem_u32(&pp.released[pp.slot])) : "memory");
+        if (before == kWarps - 1) {
+          pp.released[pp.slot] = 0u;
+          if (!pp.pc.done()) {
+            fence_proxy_async_smem();
+            uint8_t* dst = pp.ring + pp.slot * p.stage_bytes;
+            mbar_arrive_expect_tx(&pp.full[pp.slot], stage_tx_bytes(p, pp.pc.c.tc, ZP));
+            issue_weights<ZP>(pp.pc, dst, &pp.full[pp.slot], pp.tq, pp.ts, pp.tz, p.scale_offset);
+            tma_load_3d(dst + p.x_offset, pp.tx, 0, pp.pc.gbase, 0, &pp.full[pp.slot]);
+            pp.fills[pp.slot] += 1u;
+          }
+        }
+        cursor_next(p, pp.i1, pp.pc);
+      }
+
+      if (has) {
+        float grp[kChunkTiles][MT][4];
+        float cs[MT][4];
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            cs[mt][i] = 0.0f;
+#pragma unroll
+            for (int rt = 0; rt < TC; ++rt) grp[rt][mt][i] = 0.0f;
+          }
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt) {
+            mma_16816(cs[mt], pp.ca0, 0u, pp.ca2, 0u, xf[mt][jj].x, xf[mt][jj].y);
+            mma_16816(cs[mt], pp.ca0, 0u, pp.ca2, 0u, xf[mt][jj].z, xf[mt][jj].w);
+          }
+#pragma unroll
+          for (int rt = 0; rt < TC; ++rt) {
+            uint32_t plo[4], phi[4];
+            decode_word_magic(word_of(c_lo[rt], jj), plo);
+            decode_word_magic(word_of(c_hi[rt], jj), phi);
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+              mma_16816(grp[rt][mt], plo[0], phi[0], plo[1], phi[1], xf[mt][jj].x, xf[mt][jj].y);
+              mma_16816(grp[rt][mt], plo[2], phi[2], plo[3], phi[3], xf[mt][jj].z, xf[mt][jj].w);
+            }
+          }
+        }
+        // row 0 of the constant tile (lanes 0..3) holds C, row 1 (lanes 4..7) holds pp.S
+        float cm[MT][2], sm[MT][2];
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          cm[mt][0] = __shfl_sync(0xffffffffu, cs[mt][0], pp.t);
+          cm[mt][1] = __shfl_sync(0xffffffffu, cs[mt][1], pp.t);
+          sm[mt][0] = __shfl_sync(0xffffffffu, cs[mt][0], 4 + pp.t);
+          sm[mt][1] = __shfl_sync(0xffffffffu, cs[mt][1], 4 + pp.t);
+        }
+        // sum_k x (q - z) = raw - C(m) - z pp.S(m); then the group's scale
+#pragma unroll
+        for (int rt = 0; rt < TC; ++rt) {
+          const float s_lo = half_bits_to_float(uint16_t(s2[rt])), s_hi = half_bits_to_float(uint16_t(s2[rt] >> 16));
+          const float z_lo = half_bits_to_float(uint16_t(z2[rt])), z_hi = half_bits_to_float(uint16_t(z2[rt] >> 16));
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt) {
+            acc[rt][mt][0] = fmaf(s_lo, fmaf(-z_lo, sm[mt][0], grp[rt][mt][0] - cm[mt][0]), acc[rt][mt][0]);
+            acc[rt][mt][1] = fmaf(s_lo, fmaf(-z_lo, sm[mt][1], grp[rt][mt][1] - cm[mt][1]), acc[rt][mt][1]);
+            acc[rt][mt][2] = fmaf(s_hi, fmaf(-z_hi, sm[mt][0], grp[rt][mt][2] - cm[mt][0]), acc[rt][mt][2]);
+            acc[rt][mt][3] = fmaf(s_hi, fmaf(-z_hi, sm[mt][1], grp[rt][mt][3] - cm[mt][1]), acc[rt][mt][3]);
+          }
+        }
+      }
+      if (++pp.slot == pp.S) {
+        pp.slot = 0;
+        pp.phase ^= 1u;
+      }
+    }
+
+}
+
+template <int MT, bool ZP, int TC>
+__global__ void __launch_bounds__(kThreads, MT == 1 ? 2 : 1)
 gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_x,
             const __grid_constant__ CUtensorMap tmap_s, const __grid_constant__ CUtensorMap tmap_z,
             const GemvParams p) {
   extern __shared__ __align__(1024) uint8_t gemv_smem[];
-  using L = StageLayout<RT>;
-  const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
-  const int C = p.consumers;
-  const int S = p.stages;
-  const int64_t W = p.total_consumers;
-  const int64_t G = p.G;
-  const int stage_bytes = p.stage_bytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(gemv_smem);            // [consumer][stage]
-  uint64_t* empty = full + kMaxConsumers * kMaxStages;                // [consumer][stage]
-  uint8_t* rings = gemv_smem + kBarRegion;                            // consumer c: c * S stages
   // Let the next kernel in the stream (if launched as a programmatic
   // dependent) start as soon as every CTA of this one is running; it waits
   // for this grid's completion before it reads anything this grid writes.
   asm volatile("griddepcontrol.launch_dependents;");
 
+  const int lane = threadIdx.x & 31;
+  const int w = threadIdx.x >> 5;
+  const int g = lane >> 2;
+  const int t = lane & 3;
+  const int S = p.stages;
+  const int M = p.M;
+  uint64_t* full = reinterpret_cast<uint64_t*>(gemv_smem);                        // [S]
+  uint32_t* released = reinterpret_cast<uint32_t*>(gemv_smem + kMaxStages * 8);   // [S] warps done with a fill
+  uint32_t* fills = released + kMaxStages;                                        // [S] fills issued
+  uint32_t* failed = fills + kMaxStages;                                          // a warp gave up
+  uint8_t* ring = gemv_smem + kRingOffset;
+  float* pbuf = reinterpret_cast<float*>(gemv_smem + p.pbuf_offset);
+
+  const int i0 = int(int64_t(p.items) * blockIdx.x / gridDim.x);
+  const int i1 = int(int64_t(p.items) * (blockIdx.x + 1) / gridDim.x);
+
   if (threadIdx.x == 0) {
-    for (int i = 0; i < C * S; ++i) {
-      mbar_init(&full[(i / S) * kMaxStages + i % S], 1);
-      mbar_init(&empty[(i / S) * kMaxStages + i % S], 1);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      released[s] = 0u;
+      fills[s] = 0u;
     }
+    *failed = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     fence_proxy_async_smem();
   }
   __syncthreads();
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    // Lane c feeds consumer c. All lanes step through their rounds together,
-    // so round r of every consumer is issued before round r+1 and data
-    // returns roughly in the order it is consumed.
-    if (lane >= C) return;
-    const int64_t gc = int64_t(blockIdx.x) * C + lane;
-    const int64_t ub = range_start(p.units, gc, W);
-    const int64_t n = range_start(p.units, gc + 1, W) - ub;
-    if (n <= 0) return;
-    // (block, group) of the consumer's first unit; later units advance by one group
-    int64_t b0 = ub / G;
-    int j0 = int(ub - b0 * G);
-    // Before the dependency wait only L2 prefetches: they are safe even
-    // while an earlier kernel may still be writing these bytes.
-    {
-      int64_t b = b0;
-      int j = j0;
-      for (int64_t r = 0; r < n && r < kPrefetchUnits; ++r) {
-        const int r0 = int(b * (16 * RT));
-        tma_prefetch_l2_2d(&tmap_q, j * kWordsPerGroup, r0);
-        tma_prefetch_l2_2d(&tmap_s, r0, j);
-        if (ZP) tma_prefetch_l2_2d(&tmap_z, r0, j);
-        if (++j == G) { j = 0; ++b; }
+  // ---- the first S stages (weights possibly before the dependency wait)
+  StageCursor pc;   // lane 0 of every warp: the stage S ahead of the arithmetic
+  if (lane == 0) cursor_init(p, i0, i1, pc);
+  if (threadIdx.x == 0) {
+    if (p.early) {
+      StageCursor u = pc;
+      for (int s = 0; s < S && !u.done(); ++s) {
+        mbar_arrive_expect_tx(&full[s], stage_tx_bytes(p, u.c.tc, ZP));
+        issue_weights<ZP>(u, ring + s * p.stage_bytes, &full[s], &tmap_q, &tmap_s, &tmap_z, p.scale_offset);
+        cursor_next(p, i1, u);
       }
+    } else {
+      tma_prefetch_l2_3d(&tmap_q, 0, pc.c.t0 * kTile, pc.gbase);
     }
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    uint64_t* fb0 = &full[lane * kMaxStages];
-    uint64_t* eb0 = &empty[lane * kMaxStages];
-    uint8_t* ring = rings + lane * S * stage_bytes;
-    volatile int abort_flag = 0;
-    int64_t b = b0;
-    int j = j0;
-    int slot = 0;
-    uint32_t ephase = 1;   // parity of the empty phase to wait for in the slot's next reuse
-    int64_t r = 0;
-    for (; r < n; ++r) {
-      if (r >= S && !wait_bounded(&eb0[slot], ephase, &abort_flag, &g_awq_gemv_error, 2u)) break;
-      const int r0 = int(b * (16 * RT));
-      uint8_t* st = ring + slot * stage_bytes;
-      mbar_arrive_expect_tx(&fb0[slot], p.tx_bytes);
-      tma_load_2d(st, &tmap_q, j * kWordsPerGroup, r0, &fb0[slot]);
-      tma_load_2d(st + p.x_offset, &tmap_x, j * kGroup, 0, &fb0[slot]);
-      tma_load_2d(st + L::kCodeBytes, &tmap_s, r0, j, &fb0[slot]);
-      if (ZP) tma_load_2d(st + L::kCodeBytes + L::kMetaStride, &tmap_z, r0, j, &fb0[slot]);
-      if (++j == G) { j = 0; ++b; }
-      if (++slot == S) { slot = 0; ephase ^= 1u; }
+  }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (lane == 0) {
+    for (int s = 0; s < S && !pc.done(); ++s) {
+      if (w == 0) {
+        uint8_t* st = ring + s * p.stage_bytes;
+        if (!p.early) {
+          mbar_arrive_expect_tx(&full[s], stage_tx_bytes(p, pc.c.tc, ZP));
+          issue_weights<ZP>(pc, st, &full[s], &tmap_q, &tmap_s, &tmap_z, p.scale_offset);
+        }
+        tma_load_3d(st + p.x_offset, &tmap_x, 0, pc.gbase, 0, &full[s]);
+        fills[s] = 1u;
+      }
+      cursor_next(p, i1, pc);
     }
-    // Gave up: the copies already issued (the last S rounds before r) land
-    // before the CTA's shared memory can be reused.
-    if (r < n) {
-      for (int64_t q = r - S > 0 ? r - S : 0; q < r; ++q)
-        wait_teardown(&fb0[int(q % S)], uint32_t((q / S) & 1));
-    }
-    return;
   }
 
-  // -------------------------------------------------------------- consumer
-  const int cw = warp - 1;
-  const int g = lane >> 2;
-  const int t = lane & 3;
-  const int64_t gc = int64_t(blockIdx.x) * C + cw;
-  const int64_t u_begin = range_start(p.units, gc, W);
-  const int64_t u_end = range_start(p.units, gc + 1, W);
-  if (u_begin >= u_end) return;
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  uint8_t* ring = rings + cw * S * stage_bytes;
-
-  // x fragment offsets inside a stage: batch row m = 8 mt + g, chunk 4t + jj
-  int xoff[MT];
-  bool xok[MT];
+  volatile int abort_flag = 0;
+  Pipe<MT> pp;
+  pp.ring = ring;
+  pp.full = full;
+  pp.released = released;
+  pp.fills = fills;
+  pp.failed = failed;
+  pp.tq = &tmap_q;
+  pp.tx = &tmap_x;
+  pp.ts = &tmap_s;
+  pp.tz = &tmap_z;
+  pp.pc = pc;
+  pp.slot = 0;
+  pp.phase = 0;
+  pp.ok = true;
+  pp.S = S;
+  pp.i1 = i1;
+  pp.lane = lane;
+  pp.w = w;
+  pp.g = g;
+  pp.t = t;
+  // x fragment offsets inside a stage ([m][8 groups][128 k]): batch row
+  // m = 8 mt + g, this warp's group, chunk 4t + jj
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt) {
     const int m = 8 * mt + g;
-    xok[mt] = m < p.M;
-    xoff[mt] = p.x_offset + m * 256 + t * 64;
+    pp.xok[mt] = m < M;
+    pp.xoff[mt] = p.x_offset + (m * kWarps + w) * 256 + t * 64;
   }
-  uint32_t ca0, ca2;
-  offset_tile(g, ca0, ca2);
-  volatile int abort_flag = 0;
+  offset_tile(g, pp.ca0, pp.ca2);
 
-  const int64_t first_block = u_begin / G;
-  int64_t cur_b = first_block;
-  int jstart = int(u_begin - cur_b * G);
-  int64_t ub_ = cur_b;   // block of the unit being consumed
-  int jg = jstart;       // its group
-  float acc[RT][MT][4];
+  Chunk cc;
+  load_chunk(p, i0, i1, cc);
+  for (int chunk = 0;; ++chunk) {
+    const int tc = cc.tc;
+    float acc[kChunkTiles][MT][4];
 #pragma unroll
-  for (int rt = 0; rt < RT; ++rt)
+    for (int rt = 0; rt < kChunkTiles; ++rt)
 #pragma unroll
-    for (int mt = 0; mt < MT; ++mt)
+      for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) acc[rt][mt][i] = 0.0f;
+        for (int i = 0; i < 4; ++i) acc[rt][mt][i] = 0.0f;
 
-  int slot = 0;
-  uint32_t phase = 0;
-  for (int64_t u = u_begin; u < u_end; ++u) {
-    const bool got = wait_bounded(&full[cw * kMaxStages + slot], phase, &abort_flag, &g_awq_gemv_error, 2u);
-    if (!__all_sync(0xffffffffu, got)) return;   // producer gave up or timed out: rows stay unwritten
-    const int64_t b = ub_;
-    if (++jg == G) { jg = 0; ++ub_; }
-    if (b != cur_b) {
-      finish_block<MT, RT>(p, cur_b, jstart, int(G), gc, first_block, lane, g, t, acc);
-      cur_b = b;
-      jstart = 0;
-#pragma unroll
-      for (int rt = 0; rt < RT; ++rt)
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-          for (int i = 0; i < 4; ++i) acc[rt][mt][i] = 0.0f;
-    }
-    const uint8_t* st = ring + slot * stage_bytes;
+    chunk_stages<MT, ZP, TC>(p, pp, cc, acc, &abort_flag);
 
-    // x fragments and packed codes of the unit
-    uint4 xf[MT][4];
+    // ---- chunk reduction: the 8 warps' partial sums meet in shared memory
+    // ([warp][row][m], double-buffered by chunk parity) and are summed in
+    // warp order, so the result does not depend on timing.
+    float* pw = pbuf + ((chunk & 1) * kWarps + w) * (kChunkRows * M);
 #pragma unroll
-    for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-      for (int jj = 0; jj < 4; ++jj) xf[mt][jj] = xok[mt] ? lds128(st + xoff[mt] + jj * 16) : make_uint4(0, 0, 0, 0);
-    uint4 c_lo[RT], c_hi[RT];
-#pragma unroll
-    for (int rt = 0; rt < RT; ++rt) {
-      c_lo[rt] = lds128(st + (16 * rt + g) * 64 + t * 16);
-      c_hi[rt] = lds128(st + (16 * rt + 8 + g) * 64 + t * 16);
-    }
-    float grp[RT][MT][4];
-    float cs[MT][4];
-#pragma unroll
-    for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        cs[mt][i] = 0.0f;
-#pragma unroll
-        for (int rt = 0; rt < RT; ++rt) grp[rt][mt][i] = 0.0f;
-      }
-#pragma unroll
-    for (int jj = 0; jj < 4; ++jj) {
+    for (int rt = 0; rt < kChunkTiles; ++rt)
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) {
-        mma_16816(cs[mt], ca0, 0u, ca2, 0u, xf[mt][jj].x, xf[mt][jj].y);
-        mma_16816(cs[mt], ca0, 0u, ca2, 0u, xf[mt][jj].z, xf[mt][jj].w);
+        const int m0 = 8 * mt + 2 * t;
+        const int r_lo = 16 * rt + g, r_hi = r_lo + 8;
+        if (rt < tc) {
+          if (m0 < M) {
+            pw[r_lo * M + m0] = acc[rt][mt][0];
+            pw[r_hi * M + m0] = acc[rt][mt][2];
+          }
+          if (m0 + 1 < M) {
+            pw[r_lo * M + m0 + 1] = acc[rt][mt][1];
+            pw[r_hi * M + m0 + 1] = acc[rt][mt][3];
+          }
+        }
       }
+    named_barrier_sync(kReduceBarrier, kThreads);
+    const int V = kTile * tc * M;
+    const float* pb0 = pbuf + (chunk & 1) * kWarps * (kChunkRows * M);
+    const int64_t row0 = int64_t(cc.t0) * kTile;
+    for (int v = threadIdx.x; v < V; v += kThreads) {
+      float sum = 0.0f;
 #pragma unroll
-      for (int rt = 0; rt < RT; ++rt) {
-        uint32_t plo[4], phi[4];
-        decode_word_magic(word_of(c_lo[rt], jj), plo);
-        decode_word_magic(word_of(c_hi[rt], jj), phi);
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-          mma_16816(grp[rt][mt], plo[0], phi[0], plo[1], phi[1], xf[mt][jj].x, xf[mt][jj].y);
-          mma_16816(grp[rt][mt], plo[2], phi[2], plo[3], phi[3], xf[mt][jj].z, xf[mt][jj].w);
+      for (int ww = 0; ww < kWarps; ++ww) sum += pb0[ww * (kChunkRows * M) + v];
+      const int row = v / M;
+      const int m = v - row * M;
+      if (p.ks == 1) {
+        if (row0 + row < p.N) p.y[int64_t(m) * p.N + row0 + row] = __half_as_ushort(__float2half_rn(sum));
+      } else {
+        __stcg(p.partials + ((int64_t(cc.s) * p.T * kTile + row0 + row) * M + m), sum);
+      }
+    }
+    if (p.ks > 1) {
+      // Slices of a tile meet in the workspace: the CTA that brings a tile's
+      // arrival count to ks sums the ks partials in slice order.
+      __threadfence();
+      named_barrier_sync(kReduceBarrier, kThreads);
+      if (w < tc) {
+        const int tile = cc.t0 + w;
+        uint32_t last = 0;
+        if (lane == 0) {
+          uint32_t old;
+          asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
+                       : "=r"(old) : "l"(p.counters + tile) : "memory");
+          last = (old + 1 == uint32_t(p.ks)) ? 1u : 0u;
+        }
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (last) {
+          const int64_t trow = int64_t(tile) * kTile;
+          for (int v = lane; v < kTile * M; v += 32) {
+            float sum = 0.0f;
+            for (int s = 0; s < p.ks; ++s)
+              sum += __ldcg(p.partials + ((int64_t(s) * p.T * kTile + trow) * M + v));
+            const int row = v / M;
+            const int m = v - row * M;
+            if (trow + row < p.N) p.y[int64_t(m) * p.N + trow + row] = __half_as_ushort(__float2half_rn(sum));
+          }
+          if (lane == 0) p.counters[tile] = 0u;
         }
       }
     }
-    // row 0 of the constant tile (lanes 0..3) holds C, row 1 (lanes 4..7) holds S
-    float cm[MT][2], sm[MT][2];
-#pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
-      cm[mt][0] = __shfl_sync(0xffffffffu, cs[mt][0], t);
-      cm[mt][1] = __shfl_sync(0xffffffffu, cs[mt][1], t);
-      sm[mt][0] = __shfl_sync(0xffffffffu, cs[mt][0], 4 + t);
-      sm[mt][1] = __shfl_sync(0xffffffffu, cs[mt][1], 4 + t);
-    }
-    float s_lo[RT], s_hi[RT], z_lo[RT], z_hi[RT];
-#pragma unroll
-    for (int rt = 0; rt < RT; ++rt) {
-      s_lo[rt] = half_bits_to_float(lds16(st + L::kCodeBytes + (16 * rt + g) * 2));
-      s_hi[rt] = half_bits_to_float(lds16(st + L::kCodeBytes + (16 * rt + 8 + g) * 2));
-      z_lo[rt] = ZP ? half_bits_to_float(lds16(st + L::kCodeBytes + L::kMetaStride + (16 * rt + g) * 2)) : 8.0f;
-      z_hi[rt] = ZP ? half_bits_to_float(lds16(st + L::kCodeBytes + L::kMetaStride + (16 * rt + 8 + g) * 2)) : 8.0f;
-    }
-    // everything the unit needs is in registers: release the slot
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[cw * kMaxStages + slot]);
-    if (++slot == S) {
-      slot = 0;
-      phase ^= 1u;
-    }
-    // sum_k x (q - z) = raw - C(m) - z S(m); then the group's scale
-#pragma unroll
-    for (int rt = 0; rt < RT; ++rt)
-#pragma unroll
-      for (int mt = 0; mt < MT; ++mt) {
-        acc[rt][mt][0] = fmaf(s_lo[rt], fmaf(-z_lo[rt], sm[mt][0], grp[rt][mt][0] - cm[mt][0]), acc[rt][mt][0]);
-        acc[rt][mt][1] = fmaf(s_lo[rt], fmaf(-z_lo[rt], sm[mt][1], grp[rt][mt][1] - cm[mt][1]), acc[rt][mt][1]);
-        acc[rt][mt][2] = fmaf(s_hi[rt], fmaf(-z_hi[rt], sm[mt][0], grp[rt][mt][2] - cm[mt][0]), acc[rt][mt][2]);
-        acc[rt][mt][3] = fmaf(s_hi[rt], fmaf(-z_hi[rt], sm[mt][1], grp[rt][mt][3] - cm[mt][1]), acc[rt][mt][3]);
-      }
+    const int ni = cc.i + cc.tc;
+    if (ni >= i1) break;
+    load_chunk(p, ni, i1, cc);
   }
-  finish_block<MT, RT>(p, cur_b, jstart, int(u_end - cur_b * G), gc, first_block, lane, g, t, acc);
+
+  // If a warp gave up, copies may still be in flight: a slot is refilled
+  // only after every warp has taken its previous fill, so at most its latest
+  // fill is pending; thread 0 waits (bounded) for it before the CTA exits.
+  __syncthreads();
+  if (threadIdx.x == 0 && *reinterpret_cast<volatile uint32_t*>(failed)) {
+    for (int s = 0; s < S; ++s)
+      if (fills[s] > 0u) wait_teardown(&full[s], (fills[s] - 1u) & 1u);
+  }
 }
 
 // ---------------------------------------------------------------------------
-// host side: plan (variant, grid, workspace) for a shape
+// host side: plan (variant, decomposition, ring geometry, workspace) for a shape
 // ---------------------------------------------------------------------------
 using KernelFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap,
                           const GemvParams);
 
 struct Variant {
   KernelFn fn;
-  int mt, rt, consumers, id;
+  int mt, id;
 };
 
-constexpr int kNumVariants = 4;
-constexpr int kRT = 4;
+constexpr int kNumVariants = 8;
 constexpr int kSmemBudget = 232448;   // largest dynamic shared memory of one sm_100 CTA
 constexpr int kHalfSmBudget = 115712; // half of an SM's 228 KB, less the 1 KB reserved per CTA
 
-int smem_budget(const Variant& v);
-
-Variant pick_variant(int64_t M, bool zp) {
-  if (M <= 8)
-    return zp ? Variant{gemv_kernel<1, kRT, true>, 1, kRT, Consumers<1>::value, 0}
-              : Variant{gemv_kernel<1, kRT, false>, 1, kRT, Consumers<1>::value, 1};
-  return zp ? Variant{gemv_kernel<2, kRT, true>, 2, kRT, Consumers<2>::value, 2}
-            : Variant{gemv_kernel<2, kRT, false>, 2, kRT, Consumers<2>::value, 3};
+Variant pick_variant(int64_t M, bool zp, int tc) {
+  static const Variant table[kNumVariants] = {
+      {gemv_kernel<1, true, 4>, 1, 0},  {gemv_kernel<1, false, 4>, 1, 1},
+      {gemv_kernel<2, true, 4>, 2, 2},  {gemv_kernel<2, false, 4>, 2, 3},
+      {gemv_kernel<1, true, 2>, 1, 4},  {gemv_kernel<1, false, 2>, 1, 5},
+      {gemv_kernel<2, true, 2>, 2, 6},  {gemv_kernel<2, false, 2>, 2, 7}};
+  return table[(tc == 2 ? 4 : 0) + (M <= 8 ? 0 : 2) + (zp ? 0 : 1)];
 }
 
 int round128(int v) { return (v + 127) / 128 * 128; }
 
-struct StageGeometry {
-  int code_bytes, meta_stride, x_offset, stage_bytes, stages;
-  uint32_t tx_bytes;
-};
-
-StageGeometry stage_geometry(const Variant& v, int64_t M, bool zp) {
-  StageGeometry sg;
-  sg.code_bytes = 16 * v.rt * 64;
-  sg.meta_stride = round128(16 * v.rt * 2);
-  sg.x_offset = sg.code_bytes + sg.meta_stride * (zp ? 2 : 1);
-  sg.stage_bytes = round128(sg.x_offset + int(M) * 256);
-  sg.tx_bytes = uint32_t(sg.code_bytes + 16 * v.rt * 2 * (zp ? 2 : 1) + int(M) * 256);
-  int st = (smem_budget(v) - kBarRegion) / (v.consumers * sg.stage_bytes);
-  sg.stages = st > kMaxStages ? kMaxStages : st;
-  return sg;
-}
-
-int smem_budget(const Variant& v) { return v.mt == 1 ? kHalfSmBudget : kSmemBudget; }
-
 struct Plan {
   Variant v;
-  StageGeometry sg;
-  int grid;
-  int nb;
-  int smem;
-  int64_t units;
-  size_t counter_bytes;
-  size_t partial_bytes;
+  int grid, T, ks, items, tc, scale_offset;
+  int stages, stage_bytes, x_offset, pbuf_offset, smem;
+  size_t counter_bytes, partial_bytes;
 };
 
 constexpr int kMaxDevices = 64;
@@ -538,39 +574,52 @@ awq_status_t make_plan(int64_t M, int64_t N, int64_t K, bool zp, Plan& pl) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return AWQ_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return AWQ_ERR_UNSUPPORTED;
-  pl.v = pick_variant(M, zp);
-  pl.sg = stage_geometry(pl.v, M, zp);
-  if (pl.sg.stages < 2) return AWQ_ERR_UNSUPPORTED;
-  pl.smem = kBarRegion + pl.v.consumers * pl.sg.stages * pl.sg.stage_bytes;
   int sms = g_sm_count[dev].load(std::memory_order_relaxed);
   if (sms == 0) {
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return AWQ_ERR_CUDA;
     g_sm_count[dev].store(sms, std::memory_order_relaxed);
   }
+  // Decomposition: whole tiles per CTA, one CTA per SM; K slices only when
+  // there are fewer tiles than SMs.
+  const int64_t G = K / kGroup;
+  const int64_t T = (N + kTile - 1) / kTile;
+  int64_t ks = 1;
+  if (T < sms) {
+    ks = (sms + T - 1) / T;
+    if (ks > G) ks = G;
+  }
+  pl.T = int(T);
+  pl.ks = int(ks);
+  pl.items = int(T * ks);
+  pl.grid = pl.items < sms ? pl.items : sms;
+  // Chunks of 4 tiles, or of 2 when no CTA has more than 2 items: the CTA
+  // with the most items sets the kernel's time, and it then wastes no slot.
+  const int64_t most = (int64_t(pl.items) + pl.grid - 1) / pl.grid;
+  pl.tc = most <= 2 ? 2 : kChunkTiles;
+  pl.v = pick_variant(M, zp, pl.tc);
   if (!g_smem_attr[dev][pl.v.id].load(std::memory_order_acquire)) {
-    if (cudaFuncSetAttribute(pl.v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_budget(pl.v)) != cudaSuccess)
+    if (cudaFuncSetAttribute(pl.v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBudget) != cudaSuccess)
       return AWQ_ERR_CUDA;
     g_smem_attr[dev][pl.v.id].store(1, std::memory_order_release);
   }
-  const int64_t rows_per_block = 16 * pl.v.rt;
-  const int64_t G = K / kGroup;
-  pl.nb = int((N + rows_per_block - 1) / rows_per_block);
-  pl.units = int64_t(pl.nb) * G;
-  // one CTA per SM (for one batch tile it takes half the SM, leaving the
-  // other half to the next kernel); fewer when there are fewer units than
-  // consumers
-  const int64_t want = (pl.units + pl.v.consumers - 1) / pl.v.consumers;
-  pl.grid = int(want < sms ? (want > 0 ? want : 1) : sms);
-  const int64_t total = int64_t(pl.grid) * pl.v.consumers;
-  // units * consumers must fit the kernel's 64-bit split arithmetic
-  if (pl.units > 0 && total > (int64_t(1) << 62) / pl.units) return AWQ_ERR_SHAPE;
-  pl.counter_bytes = ((size_t(pl.nb) * 4 + 255) / 256) * 256;
-  // With one group per row (G == 1) every unit is a whole block and no
-  // block is ever split; otherwise consumers may share blocks. A consumer
-  // holds at most two partial blocks: the first and the last of its range,
-  // each 16*RT rows x M values.
-  pl.partial_bytes = G > 1 ? size_t(total) * 2 * size_t(16 * pl.v.rt) * size_t(M) * 4 : 0;
+  // Ring geometry: as many stages as the budget holds after the reduction buffers.
+  pl.scale_offset = pl.tc * kTileStageBytes;
+  pl.x_offset = pl.scale_offset + kMetaStageBytes * (zp ? 2 : 1);
+  pl.stage_bytes = round128(pl.x_offset + int(M) * kXStageBytesPerRow);
+  const int pbuf_bytes = 2 * kWarps * kChunkRows * int(M) * 4;
+  int budget = pl.v.mt == 1 ? kHalfSmBudget : kSmemBudget;
+  for (;;) {
+    int st = (budget - kRingOffset - pbuf_bytes) / pl.stage_bytes;
+    pl.stages = st > kMaxStages ? kMaxStages : st;
+    if (pl.stages >= 3 || budget == kSmemBudget) break;
+    budget = kSmemBudget;   // too few stages beside another CTA: take the whole SM
+  }
+  if (pl.stages < 2) return AWQ_ERR_UNSUPPORTED;
+  pl.pbuf_offset = kRingOffset + pl.stages * pl.stage_bytes;
+  pl.smem = pl.pbuf_offset + pbuf_bytes;
+  pl.counter_bytes = ks > 1 ? ((size_t(T) * 4 + 255) / 256) * 256 : 0;
+  pl.partial_bytes = ks > 1 ? size_t(ks) * size_t(T) * kTile * size_t(M) * 4 : 0;
   return AWQ_OK;
 }
 
@@ -600,7 +649,7 @@ awq_status_t gemv_workspace_bytes(int64_t M, int64_t N, int64_t K, bool zp, size
   Plan pl;
   awq_status_t st = make_plan(M, N, K, zp, pl);
   if (st != AWQ_OK) return st;
-  *bytes = pl.partial_bytes ? pl.counter_bytes + pl.partial_bytes : 0;
+  *bytes = pl.counter_bytes + pl.partial_bytes;
   return AWQ_OK;
 }
 
@@ -634,49 +683,51 @@ extern "C" awq_status_t awq_gemv(const uint16_t* x, const int32_t* qweight,
   p.y = y;
   p.counters = nullptr;
   p.partials = nullptr;
-  if (pl.partial_bytes) {
+  if (pl.ks > 1) {
     if (!workspace || workspace_bytes < pl.counter_bytes + pl.partial_bytes) return AWQ_ERR_WORKSPACE;
     if (!aligned16(workspace)) return AWQ_ERR_ALIGN;
     p.counters = static_cast<uint32_t*>(workspace);
     p.partials = reinterpret_cast<float*>(static_cast<char*>(workspace) + pl.counter_bytes);
   }
   const int G = int(K / kGroup);
-  // codes: int32 [N][K/8], box 16 words (one group) x 16*RT rows
-  // x: fp16 [M][K], box 128 k x M rows; scales / zeros: fp16 [G][N], box 16*RT x 1
+  // codes: int32 [N][K/8] viewed as {16 words, N rows, G groups} (a group
+  // steps 64 bytes, a row K/2 bytes), boxes of 16 x 16 x 8 that land
+  // group-major; x: fp16 [M][K] viewed as {128 k, G groups, M rows}, boxes of
+  // 128 x 8 x M; scales / zeros: fp16 [G][N], boxes of 64 rows x 8 groups.
   CUtensorMap tq, tx, ts, tz;
-  const uint32_t rows = uint32_t(16 * pl.v.rt);
-  if (!make_tensor_map_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_INT32, qweight, uint64_t(K / 8), uint64_t(N),
-                          uint64_t(K / 8) * 4, kWordsPerGroup, rows, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !make_tensor_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x, uint64_t(K), uint64_t(M),
-                          uint64_t(K) * 2, kGroup, uint32_t(M), CU_TENSOR_MAP_SWIZZLE_NONE) ||
+  if (!make_tensor_map_3d(&tq, CU_TENSOR_MAP_DATA_TYPE_INT32, qweight, kWordsPerGroup, uint64_t(N),
+                          uint64_t(G), uint64_t(K / 8) * 4, kWordsPerGroup * 4, kWordsPerGroup, kTile, kWarps) ||
+      !make_tensor_map_3d(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x, kGroup, uint64_t(G), uint64_t(M),
+                          kGroup * 2, uint64_t(K) * 2, kGroup, kWarps, uint32_t(M)) ||
       !make_tensor_map_2d(&ts, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, scales, uint64_t(N), uint64_t(G),
-                          uint64_t(N) * 2, rows, 1, CU_TENSOR_MAP_SWIZZLE_NONE))
+                          uint64_t(N) * 2, kChunkRows, kWarps, CU_TENSOR_MAP_SWIZZLE_NONE))
     return AWQ_ERR_CUDA;
   if (zp) {
     if (!make_tensor_map_2d(&tz, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, zeros, uint64_t(N), uint64_t(G),
-                            uint64_t(N) * 2, rows, 1, CU_TENSOR_MAP_SWIZZLE_NONE))
+                            uint64_t(N) * 2, kChunkRows, kWarps, CU_TENSOR_MAP_SWIZZLE_NONE))
       return AWQ_ERR_CUDA;
   } else {
     tz = ts;   // never read by the symmetric kernels
   }
-  p.units = pl.units;
   p.M = int(M);
   p.N = int(N);
-  p.K = int(K);
   p.G = G;
-  p.nb = pl.nb;
-  p.consumers = pl.v.consumers;
-  p.total_consumers = pl.grid * pl.v.consumers;
-  p.stages = pl.sg.stages;
-  p.stage_bytes = pl.sg.stage_bytes;
-  p.x_offset = pl.sg.x_offset;
-  p.tx_bytes = pl.sg.tx_bytes;
+  p.T = pl.T;
+  p.ks = pl.ks;
+  p.items = pl.items;
+  p.stages = pl.stages;
+  p.stage_bytes = pl.stage_bytes;
+  p.x_offset = pl.x_offset;
+  p.pbuf_offset = pl.pbuf_offset;
+  p.chunk_tiles = pl.tc;
+  p.scale_offset = pl.scale_offset;
+  p.early = (cfg.flags & AWQ_FLAG_WEIGHTS_STATIC) ? 1 : 0;
   // Programmatic dependent launch: this grid may start while the previous
   // kernel in the stream finishes; the kernel waits for it (griddepcontrol)
-  // before any load into shared memory, workspace access or store.
+  // before it touches x, the workspace or y.
   cudaLaunchConfig_t lc = {};
   lc.gridDim = dim3(pl.grid);
-  lc.blockDim = dim3(32 * (1 + pl.v.consumers));
+  lc.blockDim = dim3(kThreads);
   lc.dynamicSmemBytes = size_t(pl.smem);
   lc.stream = static_cast<cudaStream_t>(stream);
   cudaLaunchAttribute attr[1];

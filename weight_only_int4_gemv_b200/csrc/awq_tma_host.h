@@ -37,4 +37,23 @@ inline bool make_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, cons
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D tensor of dims {d0, d1, d2} (d0 contiguous) with byte strides s1, s2
+// for dims 1 and 2 (any order of magnitude: a view may step through memory
+// in a different order than the array is stored); boxes of b0 x b1 x b2
+// elements land in shared memory d0-fastest, then d1, then d2; reads past
+// the edges return 0.
+inline bool make_tensor_map_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
+                               uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1, uint64_t s2,
+                               uint32_t b0, uint32_t b1, uint32_t b2) {
+  PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+  if (!encode) return false;
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {s1, s2};
+  const cuuint32_t box[3] = {b0, b1, b2};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return encode(map, dtype, 3, const_cast<void*>(base), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace awq
