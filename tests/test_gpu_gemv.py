@@ -116,15 +116,16 @@ def test_gemv_is_deterministic_and_reuses_its_workspace():
 
 
 def test_gemv_whole_tiles_need_no_workspace():
-    """With at least one 16-channel tile per SM every CTA covers all of K for
-    its tiles: no workspace, and the call works without one."""
+    """With at least one 16-channel tile per CTA (two CTAs per SM for M <= 8)
+    every CTA covers all of K for its tiles: no workspace, and the call works
+    without one."""
     sms = torch.cuda.get_device_properties(0).multi_processor_count
-    for M, N, K in [(1, 16 * sms, 4096), (8, 4096, 14336), (16, 14336, 4096)]:
-        assert awq.awq_workspace_bytes(M, N, K, True) == 0
-    _, qweight, scales, zeros, Wd = oracle_layer(16 * sms, 1024, 0.02, 0.01, True)
+    for M, N, K in [(1, 32 * sms, 4096), (8, 32 * sms, 1024), (16, 14336, 4096), (12, 16 * sms, 4096)]:
+        assert awq.awq_workspace_bytes(M, N, K, True) == 0, (M, N, K)
+    _, qweight, scales, zeros, Wd = oracle_layer(32 * sms, 1024, 0.02, 0.01, True)
     x = activations(2, 1024, seed=7)
     y = host(awq.awq_gemv(dev(x), dev(qweight), dev(scales), dev(zeros), workspace=None))
-    assert_close(y, O.matmul_f64(x, Wd), "N = 16 x SMs")
+    assert_close(y, O.matmul_f64(x, Wd), "N = 32 x SMs")
 
 
 @pytest.mark.parametrize("zp", [True, False])

@@ -10,11 +10,12 @@
 // * Output channels come in tiles of 16 (one MMA tile). Each CTA owns a
 //   contiguous run of whole tiles over the whole of K, so no partial sum
 //   ever leaves the SM: the CTA's 8 warps split K between them and reduce
-//   through shared memory. Tiles are spread evenly over one CTA per SM (at
-//   most one tile of difference). Only when there are fewer tiles than SMs
-//   is K also cut into slices handled by different CTAs; their fp32
-//   partials meet in a workspace and the last CTA to arrive on a tile sums
-//   them in slice order.
+//   through shared memory. Tiles are spread evenly (at most one tile of
+//   difference) over two half-SM CTAs per SM for M <= 8 (16 warps hide the
+//   latency of the decode and MMA chains better than 8), one otherwise.
+//   Only when there are fewer tiles than CTAs is K also cut into slices
+//   handled by different CTAs; their fp32 partials meet in a workspace and
+//   the last CTA to arrive on a tile sums them in slice order.
 // * A CTA walks its tiles in chunks of up to four (64 channels). Within a
 //   chunk, the K range goes by in stages of 8 groups, one group per warp: a
 //   unit of work is (chunk, group), 16 words x up to 64 rows of codes.
@@ -49,8 +50,8 @@
 //   (always safe), or, when the caller declares the weights static
 //   (AWQ_FLAG_WEIGHTS_STATIC), already loads the codes, scales and zero
 //   points of its first S stages into its ring; x, the workspace and y are
-//   touched only after the wait. For M = 1 a CTA takes half an SM so that
-//   the next layer's CTA can sit beside it and fill its ring meanwhile.
+//   touched only after the wait; the next layer's CTAs take an SM's place as
+//   soon as this layer's CTAs there have finished.
 // * Every mbarrier wait is bounded (2 s); a warp that gives up records bit 1
 //   of the device error word, stops waiting and stops releasing stages,
 //   still takes part in its CTA's reductions (so no CTA barrier can hang),
@@ -580,46 +581,48 @@ awq_status_t make_plan(int64_t M, int64_t N, int64_t K, bool zp, Plan& pl) {
       return AWQ_ERR_CUDA;
     g_sm_count[dev].store(sms, std::memory_order_relaxed);
   }
-  // Decomposition: whole tiles per CTA, one CTA per SM; K slices only when
-  // there are fewer tiles than SMs.
+  // Decomposition: whole tiles per CTA over all of K, with as many CTAs as
+  // fill the GPU: two half-SM CTAs per SM for M <= 8 (16 warps hide more
+  // latency), one otherwise, or when half an SM cannot hold two stages. K is
+  // cut into slices only when there are fewer tiles than CTAs.
   const int64_t G = K / kGroup;
   const int64_t T = (N + kTile - 1) / kTile;
-  int64_t ks = 1;
-  if (T < sms) {
-    ks = (sms + T - 1) / T;
-    if (ks > G) ks = G;
+  const int pbuf_bytes = 2 * kWarps * kChunkRows * int(M) * 4;
+  for (int per_sm = M <= 8 ? 2 : 1;; --per_sm) {
+    const int64_t want = int64_t(per_sm) * sms;
+    int64_t ks = 1;
+    if (T < want) {
+      ks = (want + T - 1) / T;
+      if (ks > G) ks = G;
+    }
+    pl.T = int(T);
+    pl.ks = int(ks);
+    pl.items = int(T * ks);
+    pl.grid = int(pl.items < want ? pl.items : want);
+    // Chunks of 4 tiles, or of 2 when no CTA has more than 2 items: the CTA
+    // with the most items sets the kernel's time, and it then wastes no slot.
+    const int64_t most = (int64_t(pl.items) + pl.grid - 1) / pl.grid;
+    pl.tc = most <= 2 ? 2 : kChunkTiles;
+    // Ring geometry: as many stages as the budget holds after the reduction buffers.
+    pl.scale_offset = pl.tc * kTileStageBytes;
+    pl.x_offset = pl.scale_offset + kMetaStageBytes * (zp ? 2 : 1);
+    pl.stage_bytes = round128(pl.x_offset + int(M) * kXStageBytesPerRow);
+    const int budget = per_sm == 2 ? kHalfSmBudget : kSmemBudget;
+    const int st = (budget - kRingOffset - pbuf_bytes) / pl.stage_bytes;
+    pl.stages = st > kMaxStages ? kMaxStages : st;
+    if (pl.stages >= 2 || per_sm == 1) break;
   }
-  pl.T = int(T);
-  pl.ks = int(ks);
-  pl.items = int(T * ks);
-  pl.grid = pl.items < sms ? pl.items : sms;
-  // Chunks of 4 tiles, or of 2 when no CTA has more than 2 items: the CTA
-  // with the most items sets the kernel's time, and it then wastes no slot.
-  const int64_t most = (int64_t(pl.items) + pl.grid - 1) / pl.grid;
-  pl.tc = most <= 2 ? 2 : kChunkTiles;
+  if (pl.stages < 2) return AWQ_ERR_UNSUPPORTED;
   pl.v = pick_variant(M, zp, pl.tc);
   if (!g_smem_attr[dev][pl.v.id].load(std::memory_order_acquire)) {
     if (cudaFuncSetAttribute(pl.v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBudget) != cudaSuccess)
       return AWQ_ERR_CUDA;
     g_smem_attr[dev][pl.v.id].store(1, std::memory_order_release);
   }
-  // Ring geometry: as many stages as the budget holds after the reduction buffers.
-  pl.scale_offset = pl.tc * kTileStageBytes;
-  pl.x_offset = pl.scale_offset + kMetaStageBytes * (zp ? 2 : 1);
-  pl.stage_bytes = round128(pl.x_offset + int(M) * kXStageBytesPerRow);
-  const int pbuf_bytes = 2 * kWarps * kChunkRows * int(M) * 4;
-  int budget = pl.v.mt == 1 ? kHalfSmBudget : kSmemBudget;
-  for (;;) {
-    int st = (budget - kRingOffset - pbuf_bytes) / pl.stage_bytes;
-    pl.stages = st > kMaxStages ? kMaxStages : st;
-    if (pl.stages >= 3 || budget == kSmemBudget) break;
-    budget = kSmemBudget;   // too few stages beside another CTA: take the whole SM
-  }
-  if (pl.stages < 2) return AWQ_ERR_UNSUPPORTED;
   pl.pbuf_offset = kRingOffset + pl.stages * pl.stage_bytes;
   pl.smem = pl.pbuf_offset + pbuf_bytes;
-  pl.counter_bytes = ks > 1 ? ((size_t(T) * 4 + 255) / 256) * 256 : 0;
-  pl.partial_bytes = ks > 1 ? size_t(ks) * size_t(T) * kTile * size_t(M) * 4 : 0;
+  pl.counter_bytes = pl.ks > 1 ? ((size_t(T) * 4 + 255) / 256) * 256 : 0;
+  pl.partial_bytes = pl.ks > 1 ? size_t(pl.ks) * size_t(T) * kTile * size_t(M) * 4 : 0;
   return AWQ_OK;
 }
 
