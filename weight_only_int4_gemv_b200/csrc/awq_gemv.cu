@@ -238,7 +238,7 @@ __device__ __forceinline__ void chunk_stages(const GemvParams& p, Pipe<MT>& pp, 
       uint4 c_lo[kChunkTiles], c_hi[kChunkTiles];
       uint32_t s2[kChunkTiles], z2[kChunkTiles];
       if (has) {
-        // the unit's data, into registers: codes of rows pp.g and pp.g+8 of each
+        // the unit's data, into registers: codes of rows g and g+8 of each
         // tile; scales and zero points of the same two rows as fp16 pairs
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt)
@@ -257,7 +257,7 @@ __device__ __forceinline__ void chunk_stages(const GemvParams& p, Pipe<MT>& pp, 
         }
       }
       // Release the stage; the last of the CTA's warps to do so refills it
-      // with the stage pp.S ahead.
+      // with the stage S ahead.
       __syncwarp();
       if (pp.lane == 0 && pp.ok) {
         uint32_t before;
@@ -307,7 +307,7 @@ __device__ __forceinline__ void chunk_stages(const GemvParams& p, Pipe<MT>& pp, 
             }
           }
         }
-        // row 0 of the constant tile (lanes 0..3) holds C, row 1 (lanes 4..7) holds pp.S
+        // row 0 of the constant tile (lanes 0..3) holds C, row 1 (lanes 4..7) holds S
         float cm[MT][2], sm[MT][2];
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt) {
@@ -316,7 +316,7 @@ __device__ __forceinline__ void chunk_stages(const GemvParams& p, Pipe<MT>& pp, 
           sm[mt][0] = __shfl_sync(0xffffffffu, cs[mt][0], 4 + pp.t);
           sm[mt][1] = __shfl_sync(0xffffffffu, cs[mt][1], 4 + pp.t);
         }
-        // sum_k x (q - z) = raw - C(m) - z pp.S(m); then the group's scale
+        // sum_k x (q - z) = raw - C(m) - z S(m); then the group's scale
 #pragma unroll
         for (int rt = 0; rt < TC; ++rt) {
           const float s_lo = half_bits_to_float(uint16_t(s2[rt])), s_hi = half_bits_to_float(uint16_t(s2[rt] >> 16));
