@@ -98,6 +98,7 @@ struct GemvParams {
   int chunk_tiles;       // tiles per chunk (the kernel's TC)
   int scale_offset;      // offset of the scales inside a stage (TC tiles of codes before it)
   int early;             // weights may be read before the previous kernel completes
+  int codes4d;           // stage codes as one 4-D box (N % 16 == 0)
 };
 
 __device__ __forceinline__ uint4 lds128(const uint8_t* p) { return *reinterpret_cast<const uint4*>(p); }
@@ -183,15 +184,28 @@ __device__ __forceinline__ uint32_t stage_tx_bytes(const GemvParams& p, int tc, 
   return uint32_t(tc * kTileStageBytes + kMetaStageBytes * (zp ? 2 : 1) + p.M * kXStageBytesPerRow);
 }
 
-// Copies of the weight part of a stage: for each tile one 3-D box of codes
-// (16 words x 16 rows x 8 groups, landing group-major), and the 64-row runs
-// of scales and zero points of the 8 groups.
+// The codes of a stage as one 4-D box per tile count: a view of qweight as
+// {16 words, 16 rows, G groups, N/16 tiles} whose boxes of 16 x 16 x 8 x tc
+// land tile-major then group-major, the same layout as tc boxes of the 3-D
+// view. Used when N is a multiple of 16 (the view then covers exactly the
+// array).
+struct CodeMaps {
+  CUtensorMap by_tiles[kChunkTiles];   // box of 1, 2, 3, 4 tiles
+};
+
+// Copies of the weight part of a stage: the codes of its tiles (one 4-D box,
+// or one 3-D box of 16 words x 16 rows x 8 groups per tile, landing
+// group-major), and the 64-row runs of scales and zero points of the 8 groups.
 template <bool ZP>
 __device__ __forceinline__ void issue_weights(const StageCursor& u, uint8_t* st, uint64_t* bar,
                                               const CUtensorMap* tq, const CUtensorMap* ts,
-                                              const CUtensorMap* tz, int p_scale_offset) {
+                                              const CUtensorMap* tz, int p_scale_offset, const CodeMaps* cq) {
   const int r0 = u.c.t0 * kTile;
-  for (int r = 0; r < u.c.tc; ++r) tma_load_3d(st + r * kTileStageBytes, tq, 0, r0 + r * kTile, u.gbase, bar);
+  if (cq) {
+    tma_load_4d(st, &cq->by_tiles[u.c.tc - 1], 0, 0, u.gbase, u.c.t0, bar);
+  } else {
+    for (int r = 0; r < u.c.tc; ++r) tma_load_3d(st + r * kTileStageBytes, tq, 0, r0 + r * kTile, u.gbase, bar);
+  }
   tma_load_2d(st + p_scale_offset, ts, r0, u.gbase, bar);
   if (ZP) tma_load_2d(st + p_scale_offset + kMetaStageBytes, tz, r0, u.gbase, bar);
 }
@@ -208,6 +222,7 @@ struct Pipe {
   const CUtensorMap* tx;
   const CUtensorMap* ts;
   const CUtensorMap* tz;
+  const CodeMaps* cq;  // null: per-tile 3-D boxes
   StageCursor pc;      // lane 0: the stage S ahead of the arithmetic
   int slot;
   uint32_t phase;
@@ -269,7 +284,7 @@ __device__ __forceinline__ void chunk_stages(const GemvParams& p, Pipe<MT>& pp, 
             fence_proxy_async_smem();
             uint8_t* dst = pp.ring + pp.slot * p.stage_bytes;
             mbar_arrive_expect_tx(&pp.full[pp.slot], stage_tx_bytes(p, pp.pc.c.tc, ZP));
-            issue_weights<ZP>(pp.pc, dst, &pp.full[pp.slot], pp.tq, pp.ts, pp.tz, p.scale_offset);
+            issue_weights<ZP>(pp.pc, dst, &pp.full[pp.slot], pp.tq, pp.ts, pp.tz, p.scale_offset, pp.cq);
             tma_load_3d(dst + p.x_offset, pp.tx, 0, pp.pc.gbase, 0, &pp.full[pp.slot]);
             pp.fills[pp.slot] += 1u;
           }
@@ -342,7 +357,7 @@ template <int MT, bool ZP, int TC>
 __global__ void __launch_bounds__(kThreads, MT == 1 ? 2 : 1)
 gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_x,
             const __grid_constant__ CUtensorMap tmap_s, const __grid_constant__ CUtensorMap tmap_z,
-            const GemvParams p) {
+            const __grid_constant__ CodeMaps code_maps, const GemvParams p) {
   extern __shared__ __align__(1024) uint8_t gemv_smem[];
   // Let the next kernel in the stream (if launched as a programmatic
   // dependent) start as soon as every CTA of this one is running; it waits
@@ -385,7 +400,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
       StageCursor u = pc;
       for (int s = 0; s < S && !u.done(); ++s) {
         mbar_arrive_expect_tx(&full[s], stage_tx_bytes(p, u.c.tc, ZP));
-        issue_weights<ZP>(u, ring + s * p.stage_bytes, &full[s], &tmap_q, &tmap_s, &tmap_z, p.scale_offset);
+        issue_weights<ZP>(u, ring + s * p.stage_bytes, &full[s], &tmap_q, &tmap_s, &tmap_z, p.scale_offset, p.codes4d ? &code_maps : nullptr);
         cursor_next(p, i1, u);
       }
     } else {
@@ -399,7 +414,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
         uint8_t* st = ring + s * p.stage_bytes;
         if (!p.early) {
           mbar_arrive_expect_tx(&full[s], stage_tx_bytes(p, pc.c.tc, ZP));
-          issue_weights<ZP>(pc, st, &full[s], &tmap_q, &tmap_s, &tmap_z, p.scale_offset);
+          issue_weights<ZP>(pc, st, &full[s], &tmap_q, &tmap_s, &tmap_z, p.scale_offset, p.codes4d ? &code_maps : nullptr);
         }
         tma_load_3d(st + p.x_offset, &tmap_x, 0, pc.gbase, 0, &full[s]);
         fills[s] = 1u;
@@ -419,6 +434,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
   pp.tx = &tmap_x;
   pp.ts = &tmap_s;
   pp.tz = &tmap_z;
+  pp.cq = p.codes4d ? &code_maps : nullptr;
   pp.pc = pc;
   pp.slot = 0;
   pp.phase = 0;
@@ -538,7 +554,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
 // host side: plan (variant, decomposition, ring geometry, workspace) for a shape
 // ---------------------------------------------------------------------------
 using KernelFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap,
-                          const GemvParams);
+                          const CodeMaps, const GemvParams);
 
 struct Variant {
   KernelFn fn;
@@ -712,6 +728,19 @@ extern "C" awq_status_t awq_gemv(const uint16_t* x, const int32_t* qweight,
   } else {
     tz = ts;   // never read by the symmetric kernels
   }
+  CodeMaps cq;
+  p.codes4d = (N % kTile) == 0 ? 1 : 0;
+  for (int tc = 1; tc <= kChunkTiles; ++tc) {
+    if (p.codes4d) {
+      const uint64_t row = uint64_t(K / 8) * 4;
+      if (!make_tensor_map_4d(&cq.by_tiles[tc - 1], CU_TENSOR_MAP_DATA_TYPE_INT32, qweight, kWordsPerGroup,
+                              kTile, uint64_t(G), uint64_t(N / kTile), row, kWordsPerGroup * 4, row * kTile,
+                              kWordsPerGroup, kTile, kWarps, uint32_t(tc)))
+        return AWQ_ERR_CUDA;
+    } else {
+      cq.by_tiles[tc - 1] = tq;   // never read
+    }
+  }
   p.M = int(M);
   p.N = int(N);
   p.G = G;
@@ -738,7 +767,7 @@ extern "C" awq_status_t awq_gemv(const uint16_t* x, const int32_t* qweight,
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   lc.attrs = attr;
   lc.numAttrs = 1;
-  if (cudaLaunchKernelEx(&lc, pl.v.fn, tq, tx, ts, tz, p) != cudaSuccess) return AWQ_ERR_CUDA;
+  if (cudaLaunchKernelEx(&lc, pl.v.fn, tq, tx, ts, tz, cq, p) != cudaSuccess) return AWQ_ERR_CUDA;
   return launch_status();
 }
 

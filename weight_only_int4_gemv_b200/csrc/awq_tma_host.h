@@ -56,4 +56,21 @@ inline bool make_tensor_map_3d(CUtensorMap* map, CUtensorMapDataType dtype, cons
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 4-D tensor of dims {d0, d1, d2, d3} (d0 contiguous) with byte strides s1,
+// s2, s3 for dims 1..3; boxes of b0 x b1 x b2 x b3 elements land in shared
+// memory d0-fastest; reads past the edges return 0.
+inline bool make_tensor_map_4d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
+                               uint64_t d0, uint64_t d1, uint64_t d2, uint64_t d3, uint64_t s1,
+                               uint64_t s2, uint64_t s3, uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
+  PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+  if (!encode) return false;
+  const cuuint64_t dims[4] = {d0, d1, d2, d3};
+  const cuuint64_t strides[3] = {s1, s2, s3};
+  const cuuint32_t box[4] = {b0, b1, b2, b3};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return encode(map, dtype, 4, const_cast<void*>(base), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace awq
