@@ -546,6 +546,70 @@ def run_reference(args, dist):
     print(json.dumps(line), flush=True)
 
 
+def run_table(args):
+    """Per (shape, M) device time of awq_gemv and awq_gemm: one JSON line per
+    measurement. Weights come from make_packed_random (every code value in
+    every slot, which the kernels' time does not depend on); each shape gets
+    enough weight copies that one round of launches exceeds L2, and the
+    launches of a round are replayed back to back from a CUDA graph, as a
+    decode loop runs them."""
+    import torch
+    import weight_only_int4_gemv_b200 as awq
+    from workloads import make_packed_random
+
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    hbm_peak, tc_peak, _, peak_src = measured_peaks()
+    cases = [((4096, 4096), (1, 2, 4, 8, 16, 128, 512, 2048)),
+             ((14336, 4096), (1, 2, 4, 8, 16, 128, 512, 2048)),
+             ((4096, 14336), (1, 2, 4, 8, 16)),
+             ((8192, 8192), (1, 8, 2048)), ((28672, 8192), (1, 8, 2048)), ((8192, 28672), (1, 8, 2048))]
+    l2_bytes = 126 << 20
+    rng = np.random.default_rng(3)
+    for (N, K), Ms in cases:
+        q, s, z = [torch.from_numpy(a).to(device) for a in make_packed_random(N, K, 128, True, seed=1)]
+        wbytes = N * K // 2 + 4 * N * (K // 128)
+        copies = max(2, -(-2 * l2_bytes // wbytes))
+        packs = [(q.clone(), s.clone(), z.clone()) for _ in range(copies)]
+        del q, s, z
+        for M in Ms:
+            x = torch.from_numpy(rng.standard_normal((M, K), dtype=np.float32).astype(np.float16)).to(device)
+            y = torch.empty((M, N), dtype=torch.float16, device=device)
+            entry = "awq_gemv" if M <= awq.GEMV_MAX_M else "awq_gemm"
+            fn = awq.awq_gemv if M <= awq.GEMV_MAX_M else awq.awq_gemm
+            kw = {"weights_static": True} if M <= awq.GEMV_MAX_M else {}
+            ws = awq.alloc_workspace(M, N, K, True, device=device)
+            stream = torch.cuda.Stream(device)
+            with torch.cuda.stream(stream):
+                for qq, ss, zz in packs:
+                    fn(x, qq, ss, zz, workspace=ws, out=y, **kw)
+                torch.cuda.synchronize(device)
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    for qq, ss, zz in packs:
+                        fn(x, qq, ss, zz, workspace=ws, out=y, **kw)
+                reps = max(3, min(200, int(2e6 / (copies * max(1.0, M / 8)))))
+                for _ in range(3):
+                    g.replay()
+                torch.cuda.synchronize(device)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                for _ in range(reps):
+                    g.replay()
+                e1.record()
+                torch.cuda.synchronize(device)
+            us = e0.elapsed_time(e1) * 1e3 / (reps * copies)
+            gbs = algo_bytes(M, N, K) / (us * 1e-6) / 1e9
+            tfl = algo_flops(M, N, K) / (us * 1e-6) / 1e12
+            print(json.dumps({"entry": entry, "N": N, "K": K, "M": M, "us": round(us, 3), "GB/s": round(gbs, 1),
+                              "frac_hbm": round(gbs / hbm_peak, 4), "TFLOP/s": round(tfl, 2),
+                              "frac_tensor": round(tfl / tc_peak, 4), "peaks": peak_src,
+                              "weight_copies": copies}), flush=True)
+            del g
+        del packs
+        torch.cuda.empty_cache()
+
+
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -560,6 +624,8 @@ def parse_args(argv=None):
     ap.add_argument("--ref-rows", type=int, default=256)
     ap.add_argument("--no-gemm", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--table", action="store_true",
+                    help="instead of the bench line: per (shape, M) GEMV / GEMM times, one JSON line each")
     a = ap.parse_args(argv)
     if a.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -573,6 +639,9 @@ def main(argv=None):
     ws_, _, _ = dist_env()
     if args.impl == "reference":
         run_reference(args, None)
+        return 0
+    if args.table:
+        run_table(args)
         return 0
     dist = init_dist("nccl")
     try:
