@@ -7,25 +7,29 @@
 // For M beyond a few tens the layer is a dense contraction, so W' tiles are
 // decoded into shared memory and multiplied by tcgen05.mma with fp32
 // accumulators in tensor memory. One persistent CTA per SM walks output tiles
-// of 128 (rows of x) x 256 (output channels); K advances in blocks of 64.
+// of 256 (rows of x) x 128 (output channels); K advances in blocks of 64.
+// Each decoded 128 x 64 weight block feeds two M = 128 MMAs (the two halves
+// of the 256 rows of x), and narrow tiles give small batches more tiles to
+// spread over the SMs.
 //
 // Warp roles (448 threads):
-//   warps 0-7   decode: thread i owns row i of the 256-row weight tile; it
-//               reads the row's 32 code bytes of the k block from shared
-//               memory, decodes w' = (q - z) * s exactly as awq_dequant does
-//               (HSUB2 gives q - z exactly, HMUL2 rounds the product once),
-//               and writes 128 bytes in the 128-byte-swizzled K-major layout
-//               the tensor core reads.
-//   warps 8-11  epilogue: tcgen05.ld of the fp32 accumulator (lane = row of
+//   warps 0-7   decode: threads 2r and 2r+1 own row r of the 128-row weight
+//               tile, 32 k each; a thread reads its 16 code bytes of the k
+//               block from shared memory, decodes w' = (q - z) * s exactly as
+//               awq_dequant does (HSUB2 gives q - z exactly, HMUL2 rounds the
+//               product once), and writes 64 bytes in the 128-byte-swizzled
+//               K-major layout the tensor core reads.
+//   warps 8-11  epilogue: tcgen05.ld of the fp32 accumulators (lane = row of
 //               x), fp16 conversion, stores to y.
-//   warp 12     TMA: x tile (128 x 64 fp16, 128B swizzle) and code tile
-//               (256 rows x 32 bytes, 32B swizzle) per k block.
-//   warp 13     MMA: one thread issues 4 x tcgen05.mma (M=128, N=256, K=16)
-//               per k block, commits stage release and accumulator-ready
-//               barriers. Warp 13 also allocates and frees tensor memory.
+//   warp 12     TMA: x tile (256 x 64 fp16, 128B swizzle) and code tile
+//               (128 rows x 32 bytes, 32B swizzle) per k block.
+//   warp 13     MMA: one thread issues 2 x 4 tcgen05.mma (M=128, N=128,
+//               K=16) per k block, commits stage release and
+//               accumulator-ready barriers. Warp 13 also allocates and frees
+//               tensor memory.
 // Pipelines: 4 shared-memory stages (x + codes in, decoded W' out) and two
-// 256-column accumulators, so the epilogue of one tile overlaps the main
-// loop of the next.
+// accumulator pairs (4 x 128 TMEM columns), so the epilogue of one tile
+// overlaps the main loop of the next.
 //
 // Every mbarrier wait is bounded by a wall-clock limit. When a wait runs
 // out, the CTA records bit 0 in the device error word, every role leaves its
@@ -46,25 +50,28 @@ __device__ uint32_t g_awq_error_word = 0;
 
 namespace {
 
-constexpr int BM = 128;                 // rows of x per tile (MMA M)
-constexpr int BN = 256;                 // output channels per tile (MMA N)
+constexpr int BM = 256;                 // rows of x per tile (two MMAs of M = 128)
+constexpr int BMH = 128;                // rows of one MMA
+constexpr int BN = 128;                 // output channels per tile (MMA N)
 constexpr int BK = 64;                  // k per stage (one 128-byte swizzle row of fp16)
 constexpr int kStages = 4;
-constexpr int kDecodeWarps = BN / 32;   // 8
+constexpr int kDecodeWarps = 8;         // 2 threads per weight row
 constexpr int kEpiWarp0 = kDecodeWarps; // 8..11
 constexpr int kTmaWarp = kEpiWarp0 + 4; // 12
 constexpr int kMmaWarp = kTmaWarp + 1;  // 13
 constexpr int kGemmThreads = (kMmaWarp + 1) * 32;
-constexpr int kTmemCols = 2 * BN;       // two accumulators
+constexpr int kAccCols = 2 * BN;        // one accumulator pair (two M halves)
+constexpr int kTmemCols = 2 * kAccCols; // two pairs
+static_assert(kDecodeWarps * 32 == 2 * BN, "two decode threads per weight row");
 
-constexpr int kABytes = BM * BK * 2;        // 16 KB
-constexpr int kBBytes = BN * BK * 2;        // 32 KB
-constexpr int kCBytes = BN * (BK / 8) * 4;  // 8 KB of packed codes
+constexpr int kABytes = BM * BK * 2;        // 32 KB of x
+constexpr int kBBytes = BN * BK * 2;        // 16 KB of decoded W'
+constexpr int kCBytes = BN * (BK / 8) * 4;  // 4 KB of packed codes
 constexpr int kSmemTiles = kStages * (kABytes + kBBytes + kCBytes);
 constexpr int kSmemBytes = kSmemTiles + 1024 /*barriers*/ + 1024 /*alignment*/;
 
-// instruction descriptor: F16 x F16 -> F32, both K-major, M = 128, N = 256
-constexpr uint32_t kIdesc = (1u << 4) | (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
+// instruction descriptor: F16 x F16 -> F32, both K-major, M = 128, N = 128
+constexpr uint32_t kIdesc = (1u << 4) | (uint32_t(BN >> 3) << 17) | (uint32_t(BMH >> 4) << 24);
 
 struct SmemLayout {
   // offsets from the 1024-aligned base
@@ -182,7 +189,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
 
   if (warp < kDecodeWarps) {
     // ------------------------------------------------------------ decode
-    const int i = threadIdx.x;  // row of the weight tile
+    const int i = threadIdx.x >> 1;  // row of the weight tile
+    const int h = threadIdx.x & 1;   // which 32 k of the k block (words 4h .. 4h+3)
     int s = 0;
     uint32_t ph = 0;
     bool ok = true;
@@ -210,15 +218,15 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
           sc2 = uint32_t(sb) | (uint32_t(sb) << 16);
         }
         if (!wait_bounded(&bars->full_a[s], ph, abort, &g_awq_error_word, 1u)) { ok = false; break; }
-        // codes of row i: 32 bytes, 16-byte halves swapped on rows with bit 2 set (32B swizzle)
+        // codes of row i: 32 bytes, 16-byte halves swapped on rows with bit 2 set
+        // (32B swizzle); this thread decodes half h
         const uint8_t* crow = smem + SmemLayout::c(s) + i * 32;
         const int sw = (i >> 2) & 1;
-        const uint4 c0 = *reinterpret_cast<const uint4*>(crow + (sw << 4));
-        const uint4 c1 = *reinterpret_cast<const uint4*>(crow + ((sw ^ 1) << 4));
+        const uint4 c = *reinterpret_cast<const uint4*>(crow + ((h ^ sw) << 4));
         uint8_t* brow = smem + SmemLayout::b(s) + i * 128;
-        const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        const uint32_t words[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
-        for (int w = 0; w < 8; ++w) {
+        for (int w = 0; w < 4; ++w) {
           uint32_t pq[4];
           decode_word_qz(words[w], zb1024, zb64, pq);
           uint4 v;
@@ -226,7 +234,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
           v.y = hmul2_u32(pq[1], sc2);
           v.z = hmul2_u32(pq[2], sc2);
           v.w = hmul2_u32(pq[3], sc2);
-          *reinterpret_cast<uint4*>(brow + ((w ^ (i & 7)) << 4)) = v;
+          *reinterpret_cast<uint4*>(brow + (((4 * h + w) ^ (i & 7)) << 4)) = v;
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -245,12 +253,14 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
       const uint32_t aph = (it >> 1) & 1;
       if (!wait_bounded(&bars->tmem_full[acc], aph, abort, &g_awq_error_word, 1u)) break;
       tc_fence_after();
-      const int64_t m = int64_t(m0) + q * 32 + lane;
-      uint16_t* yrow = p.y + m * p.N;
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c8 = 0; c8 < 2 * (BN / 32); ++c8) {
+        const int hm = c8 / (BN / 32);      // which 128 rows of x
+        const int c = c8 % (BN / 32);       // which 32 output channels
+        const int64_t m = int64_t(m0) + hm * BMH + q * 32 + lane;
+        uint16_t* yrow = p.y + m * p.N;
         uint32_t r[32];
-        tc_ld_32x32b_x32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * BN + c * 32), r);
+        tc_ld_32x32b_x32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * kAccCols + hm * BN + c * 32), r);
         const int nc = n0 + c * 32;
         if (m < p.M && nc < p.N) {
           uint32_t h[16];
@@ -311,7 +321,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         const uint32_t aph = (it >> 1) & 1;
         if (!wait_bounded(&bars->tmem_empty[acc], aph ^ 1, abort, &g_awq_error_word, 1u)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + uint32_t(acc * BN);
+        const uint32_t d_tmem = tmem_base + uint32_t(acc * kAccCols);
         for (int kb = 0; kb < p.k_blocks; ++kb) {
           if (!wait_bounded(&bars->full_a[s], ph, abort, &g_awq_error_word, 1u) ||
               !wait_bounded(&bars->full_b[s], ph, abort, &g_awq_error_word, 1u)) { ok = false; break; }
@@ -319,9 +329,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
           const uint32_t a_addr = smem_u32(smem + SmemLayout::a(s));
           const uint32_t b_addr = smem_u32(smem + SmemLayout::b(s));
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k)
-            tc_mma_f16(d_tmem, sw128_desc(a_addr + k * 32), sw128_desc(b_addr + k * 32), kIdesc,
-                       (kb | k) != 0);
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t bd = sw128_desc(b_addr + k * 32);
+            tc_mma_f16(d_tmem, sw128_desc(a_addr + k * 32), bd, kIdesc, (kb | k) != 0);
+            tc_mma_f16(d_tmem + BN, sw128_desc(a_addr + BMH * 128 + k * 32), bd, kIdesc, (kb | k) != 0);
+          }
           tc_commit(&bars->empty[s]);
           if (++s == kStages) { s = 0; ph ^= 1; }
         }
