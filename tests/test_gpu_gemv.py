@@ -115,6 +115,17 @@ def test_gemv_is_deterministic_and_reuses_its_workspace():
     assert_close(ys[-1].view(np.float16), O.matmul_f64(x, Wd), "4th call")
 
 
+@pytest.mark.parametrize("M,N,K", [(1, 14336, 4096), (3, 4096, 14336), (16, 1000, 2048)])
+def test_gemv_repeated_calls_give_identical_bits(M, N, K):
+    """Partial sums meet in a fixed order (inside a CTA and across K
+    slices), so repeated calls agree bit for bit."""
+    _, qweight, scales, zeros, Wd = oracle_layer(N, K, 0.02, 0.01, True)
+    x = activations(M, K, seed=4)
+    ys = [bits(run_gemv(x, qweight, scales, zeros)[0]) for _ in range(3)]
+    assert np.array_equal(ys[0], ys[1]) and np.array_equal(ys[0], ys[2])
+    assert_close(ys[0].view(np.float16), O.matmul_f64(x, Wd), f"M={M} N={N} K={K}")
+
+
 def test_gemv_whole_tiles_need_no_workspace():
     """With at least one 16-channel tile per CTA (two CTAs per SM for M <= 8)
     every CTA covers all of K for its tiles: no workspace, and the call works

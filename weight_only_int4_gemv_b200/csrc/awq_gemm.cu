@@ -7,29 +7,30 @@
 // For M beyond a few tens the layer is a dense contraction, so W' tiles are
 // decoded into shared memory and multiplied by tcgen05.mma with fp32
 // accumulators in tensor memory. One persistent CTA per SM walks output tiles
-// of 256 (rows of x) x 128 (output channels); K advances in blocks of 64.
-// Each decoded 128 x 64 weight block feeds two M = 128 MMAs (the two halves
-// of the 256 rows of x), and narrow tiles give small batches more tiles to
-// spread over the SMs.
+// of 256 (rows of x) x 256 (output channels); K advances in blocks of 64.
+// Each decoded 256 x 64 weight block feeds two M = 128, N = 256 MMAs (the two
+// halves of the 256 rows of x). A tcgen05.mma costs about the same issue
+// time whatever its N, so the widest N (256) gives the most work per
+// instruction.
 //
-// Warp roles (448 threads):
-//   warps 0-7   decode: threads 2r and 2r+1 own row r of the 128-row weight
+// Warp roles (704 threads):
+//   warps 0-15  decode: threads 2r and 2r+1 own row r of the 256-row weight
 //               tile, 32 k each; a thread reads its 16 code bytes of the k
 //               block from shared memory, decodes w' = (q - z) * s exactly as
 //               awq_dequant does (HSUB2 gives q - z exactly, HMUL2 rounds the
 //               product once), and writes 64 bytes in the 128-byte-swizzled
 //               K-major layout the tensor core reads.
-//   warps 8-11  epilogue: tcgen05.ld of the fp32 accumulators (lane = row of
+//   warps 16-19 epilogue: tcgen05.ld of the fp32 accumulators (lane = row of
 //               x), fp16 conversion, stores to y.
-//   warp 12     TMA: x tile (256 x 64 fp16, 128B swizzle) and code tile
-//               (128 rows x 32 bytes, 32B swizzle) per k block.
-//   warp 13     MMA: one thread issues 2 x 4 tcgen05.mma (M=128, N=128,
-//               K=16) per k block, commits stage release and
-//               accumulator-ready barriers. Warp 13 also allocates and frees
-//               tensor memory.
-// Pipelines: 4 shared-memory stages (x + codes in, decoded W' out) and two
-// accumulator pairs (4 x 128 TMEM columns), so the epilogue of one tile
-// overlaps the main loop of the next.
+//   warp 20     TMA: x tile (256 x 64 fp16, 128B swizzle) and code tile
+//               (256 rows x 32 bytes, 32B swizzle) per k block.
+//   warp 21     MMA: one thread issues 2 x 4 tcgen05.mma (M=128, N=256,
+//               K=16) per k block (the upper half is skipped when it holds
+//               no rows of x), commits stage release and accumulator-ready
+//               barriers. Warp 21 also allocates and frees tensor memory.
+// Pipelines: 3 shared-memory stages (x + codes in, decoded W' out) and one
+// accumulator pair (all 512 TMEM columns): the epilogue of a tile runs
+// before the next tile's first MMA.
 //
 // Every mbarrier wait is bounded by a wall-clock limit. When a wait runs
 // out, the CTA records bit 0 in the device error word, every role leaves its
@@ -52,25 +53,26 @@ namespace {
 
 constexpr int BM = 256;                 // rows of x per tile (two MMAs of M = 128)
 constexpr int BMH = 128;                // rows of one MMA
-constexpr int BN = 128;                 // output channels per tile (MMA N)
+constexpr int BN = 256;                 // output channels per tile (MMA N)
 constexpr int BK = 64;                  // k per stage (one 128-byte swizzle row of fp16)
-constexpr int kStages = 4;
-constexpr int kDecodeWarps = 8;         // 2 threads per weight row
-constexpr int kEpiWarp0 = kDecodeWarps; // 8..11
-constexpr int kTmaWarp = kEpiWarp0 + 4; // 12
-constexpr int kMmaWarp = kTmaWarp + 1;  // 13
+constexpr int kStages = 3;
+constexpr int kDecodeWarps = 16;        // 2 threads per weight row
+constexpr int kEpiWarp0 = kDecodeWarps; // 16..19
+constexpr int kTmaWarp = kEpiWarp0 + 4; // 20
+constexpr int kMmaWarp = kTmaWarp + 1;  // 21
 constexpr int kGemmThreads = (kMmaWarp + 1) * 32;
 constexpr int kAccCols = 2 * BN;        // one accumulator pair (two M halves)
-constexpr int kTmemCols = 2 * kAccCols; // two pairs
+constexpr int kAccBufs = 1;             // the pair fills tensor memory
+constexpr int kTmemCols = kAccBufs * kAccCols;
 static_assert(kDecodeWarps * 32 == 2 * BN, "two decode threads per weight row");
 
 constexpr int kABytes = BM * BK * 2;        // 32 KB of x
-constexpr int kBBytes = BN * BK * 2;        // 16 KB of decoded W'
-constexpr int kCBytes = BN * (BK / 8) * 4;  // 4 KB of packed codes
+constexpr int kBBytes = BN * BK * 2;        // 32 KB of decoded W'
+constexpr int kCBytes = BN * (BK / 8) * 4;  // 8 KB of packed codes
 constexpr int kSmemTiles = kStages * (kABytes + kBBytes + kCBytes);
 constexpr int kSmemBytes = kSmemTiles + 1024 /*barriers*/ + 1024 /*alignment*/;
 
-// instruction descriptor: F16 x F16 -> F32, both K-major, M = 128, N = 128
+// instruction descriptor: F16 x F16 -> F32, both K-major, M = 128, N = 256
 constexpr uint32_t kIdesc = (1u << 4) | (uint32_t(BN >> 3) << 17) | (uint32_t(BMH >> 4) << 24);
 
 struct SmemLayout {
@@ -85,8 +87,8 @@ struct Bars {
   uint64_t full_a[kStages];    // TMA bytes of x + codes landed
   uint64_t full_b[kStages];    // decoded W' tile written (8 warp arrivals)
   uint64_t empty[kStages];     // MMAs that read the stage finished
-  uint64_t tmem_full[2];       // accumulator complete
-  uint64_t tmem_empty[2];      // accumulator drained (4 warp arrivals)
+  uint64_t tmem_full[kAccBufs];    // accumulator complete
+  uint64_t tmem_empty[kAccBufs];   // accumulator drained (4 warp arrivals)
   uint64_t mma_done;           // final commit before teardown
   uint32_t tmem_base;
   int abort;
@@ -167,7 +169,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
       mbar_init(&bars->full_b[s], kDecodeWarps);
       mbar_init(&bars->empty[s], 1);
     }
-    for (int a = 0; a < 2; ++a) {
+    for (int a = 0; a < kAccBufs; ++a) {
       mbar_init(&bars->tmem_full[a], 1);
       mbar_init(&bars->tmem_empty[a], 4);
     }
@@ -249,12 +251,13 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
       const int m0 = (tile % p.m_tiles) * BM;
       const int n0 = (tile / p.m_tiles) * BN;
-      const int acc = it & 1;
-      const uint32_t aph = (it >> 1) & 1;
+      const int acc = it % kAccBufs;
+      const uint32_t aph = (it / kAccBufs) & 1;
       if (!wait_bounded(&bars->tmem_full[acc], aph, abort, &g_awq_error_word, 1u)) break;
       tc_fence_after();
+      const int halves = m0 + BMH < p.M ? 2 : 1;   // the MMAs skip an upper half with no rows
 #pragma unroll 1
-      for (int c8 = 0; c8 < 2 * (BN / 32); ++c8) {
+      for (int c8 = 0; c8 < halves * (BN / 32); ++c8) {
         const int hm = c8 / (BN / 32);      // which 128 rows of x
         const int c = c8 % (BN / 32);       // which 32 output channels
         const int64_t m = int64_t(m0) + hm * BMH + q * 32 + lane;
@@ -317,11 +320,12 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
       int it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
-        const int acc = it & 1;
-        const uint32_t aph = (it >> 1) & 1;
+        const int acc = it % kAccBufs;
+        const uint32_t aph = (it / kAccBufs) & 1;
         if (!wait_bounded(&bars->tmem_empty[acc], aph ^ 1, abort, &g_awq_error_word, 1u)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + uint32_t(acc * kAccCols);
+        const bool upper = (tile % p.m_tiles) * BM + BMH < p.M;   // rows of x in the upper half
         for (int kb = 0; kb < p.k_blocks; ++kb) {
           if (!wait_bounded(&bars->full_a[s], ph, abort, &g_awq_error_word, 1u) ||
               !wait_bounded(&bars->full_b[s], ph, abort, &g_awq_error_word, 1u)) { ok = false; break; }
@@ -332,7 +336,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
           for (int k = 0; k < BK / 16; ++k) {
             const uint64_t bd = sw128_desc(b_addr + k * 32);
             tc_mma_f16(d_tmem, sw128_desc(a_addr + k * 32), bd, kIdesc, (kb | k) != 0);
-            tc_mma_f16(d_tmem + BN, sw128_desc(a_addr + BMH * 128 + k * 32), bd, kIdesc, (kb | k) != 0);
+            if (upper) tc_mma_f16(d_tmem + BN, sw128_desc(a_addr + BMH * 128 + k * 32), bd, kIdesc, (kb | k) != 0);
           }
           tc_commit(&bars->empty[s]);
           if (++s == kStages) { s = 0; ph ^= 1; }
@@ -410,8 +414,8 @@ extern "C" awq_status_t awq_gemm(const uint16_t* x, const int32_t* qweight,
     g_attr_set[dev][zi].store(1, std::memory_order_release);
   }
 
-  // x: fp16 [M][K], box 64 (k) x 128 (rows), 128-byte swizzle; rows past M read as 0.
-  // codes: int32 [N][K/8], box 8 words x 256 rows, 32-byte swizzle; rows past N read as 0.
+  // x: fp16 [M][K], box 64 (k) x 256 (rows), 128-byte swizzle; rows past M read as 0.
+  // codes: int32 [N][K/8], box 8 words x 256 rows (BN), 32-byte swizzle; rows past N read as 0.
   CUtensorMap tmap_x, tmap_q;
   if (!make_tensor_map_2d(&tmap_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x, uint64_t(K), uint64_t(M),
                           uint64_t(K) * 2, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
