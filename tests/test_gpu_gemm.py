@@ -51,7 +51,33 @@ def test_gemm_odd_n_scalar_epilogue():
     assert_close(run_gemm(x, qweight, scales, zeros), O.matmul_f64(x, Wd), "N=301")
 
 
-@pytest.mark.parametrize("N,K", [(4096, 4096), (14336, 4096)])
+@pytest.mark.parametrize("N,K,M", [(4000, 256, 1300), (2999, 256, 1300), (3000, 384, 2000)])
+def test_gemm_cta_pairs_many_tiles(N, K, M):
+    """Whole tiles on CTA pairs: 72 to 96 tiles of 256 x 256 (some pairs take
+    two, through both accumulators), ragged last row and channel tiles (the
+    second CTA of the last row tile has no rows of x), N not a multiple of 8.
+    Full compare, and bit-identical on a second call."""
+    _, qweight, scales, zeros, Wd = oracle_layer(N, K, 0.02, 0.01, True)
+    x = activations(M, K, seed=60 + M)
+    y = run_gemm(x, qweight, scales, zeros)
+    assert_close(y, O.matmul_f64(x, Wd), f"N={N} K={K} M={M}")
+    assert np.array_equal(bits(y), bits(run_gemm(x, qweight, scales, zeros)))
+
+
+@pytest.mark.parametrize("N,K,M", [(512, 4096, 200), (1024, 2048, 64), (2048, 8192, 129), (4096, 4096, 17)])
+def test_gemm_k_slices_over_a_cluster(N, K, M):
+    """Few tiles: K is split over a cluster of 4 or 8 CTAs per tile and the slices
+    are summed through distributed shared memory (M = 200 and 129: the upper
+    half of the tile is partly filled). Full compare, and bit-identical on a
+    second call."""
+    _, qweight, scales, zeros, Wd = oracle_layer(N, K, 0.02, 0.01, True)
+    x = activations(M, K, seed=50 + M)
+    y = run_gemm(x, qweight, scales, zeros)
+    assert_close(y, O.matmul_f64(x, Wd), f"N={N} K={K} M={M}")
+    assert np.array_equal(bits(y), bits(run_gemm(x, qweight, scales, zeros)))
+
+
+@pytest.mark.parametrize("N,K", [(4096, 4096), (14336, 4096), (4096, 14336)])
 def test_gemm_prefill_sampled(N, K):
     """Prefill: M in {128, 512, 2048}; sampled output channels, every row of x."""
     _, qweight, scales, zeros, Wd = oracle_layer(N, K, 0.02, 0.0, True)

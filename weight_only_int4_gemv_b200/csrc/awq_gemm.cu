@@ -65,6 +65,8 @@ constexpr int kAccCols = 2 * BN;        // one accumulator pair (two M halves)
 constexpr int kAccBufs = 1;             // the pair fills tensor memory
 constexpr int kTmemCols = kAccBufs * kAccCols;
 static_assert(kDecodeWarps * 32 == 2 * BN, "two decode threads per weight row");
+constexpr int kPartStride = BN + 4;
+constexpr int kMaxSlices = 8;           // cluster size limit of the K-split path     // fp32 per row of a K-slice partial (16-byte pad: no bank conflicts)
 
 constexpr int kABytes = BM * BK * 2;        // 32 KB of x
 constexpr int kBBytes = BN * BK * 2;        // 32 KB of decoded W'
@@ -135,6 +137,20 @@ __device__ __forceinline__ void tc_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[3
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+
+// 16 bytes of CTA `rank`'s shared memory at the offset `saddr` has in this CTA
+__device__ __forceinline__ float4 ld_dsmem_f4(uint32_t saddr, int rank) {
+  uint32_t a;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(saddr), "r"(rank));
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0,%1,%2,%3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a) : "memory");
+  return v;
+}
+
 // Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
 // 1024 bytes apart (stride byte offset), sm100 descriptor version 1.
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
@@ -142,12 +158,102 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
          (uint64_t(1) << 46) | (uint64_t(2) << 61);
 }
 
+// mbarrier.try_wait with a suspend-time hint: a thread whose phase is not yet
+// complete sleeps until it completes (or the hint runs out) instead of
+// re-polling, so waiting warps (MMA issuer, epilogue, producer) do not take
+// issue slots from the decode warps that share their scheduler.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait (same protocol as wait_bounded: 2 s limit, abort flag, error
+// bit 0) built on the sleeping try_wait.
+__device__ __forceinline__ bool wait_sleep(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  if (mbar_try_wait_sleep(bar, parity)) return true;
+  const uint64_t t0 = now_ns();
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity)) return true;
+    if (*abort) return false;
+    if (now_ns() - t0 > kWaitLimitNs) {
+      *abort = 1;
+      atomicOr(&g_awq_error_word, 1u);
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void wait_sleep_teardown(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = now_ns();
+  while (!mbar_try_wait_sleep(bar, parity) && now_ns() - t0 < kWaitLimitNs) {
+  }
+}
+
+// Scale and zero point of one weight row, loaded kMetaAhead groups before
+// their use through a register shift chain: the global-load latency (over a
+// microsecond under load) stays off the k loop, which otherwise waits for it
+// at every group.
+constexpr int kMetaAhead = 4;
+
+template <bool ZP>
+struct MetaChain {
+  const uint16_t* scol;
+  const uint16_t* zcol;
+  int64_t N;
+  int G;
+  bool valid;
+  uint16_t s0, s1, s2, s3, z0, z1, z2, z3;   // groups g .. g + 3
+
+  __device__ __forceinline__ uint16_t load(const uint16_t* col, int g) const {
+    return (valid && g < G) ? ld_nc_u16(col + int64_t(g) * N) : uint16_t(0);
+  }
+  __device__ __forceinline__ void start(int g0) {
+    s0 = load(scol, g0);
+    s1 = load(scol, g0 + 1);
+    s2 = load(scol, g0 + 2);
+    s3 = load(scol, g0 + 3);
+    if (ZP) {
+      z0 = load(zcol, g0);
+      z1 = load(zcol, g0 + 1);
+      z2 = load(zcol, g0 + 2);
+      z3 = load(zcol, g0 + 3);
+    } else {
+      z0 = z1 = z2 = z3 = 0;
+    }
+  }
+  // group g's scale and zero bits; group g + kMetaAhead is requested
+  __device__ __forceinline__ void next(int g, uint16_t& sb, uint16_t& zb) {
+    sb = s0;
+    zb = z0;
+    s0 = s1;
+    s1 = s2;
+    s2 = s3;
+    s3 = load(scol, g + kMetaAhead);
+    if (ZP) {
+      z0 = z1;
+      z1 = z2;
+      z2 = z3;
+      z3 = load(zcol, g + kMetaAhead);
+    }
+  }
+};
+
 struct GemmParams {
   uint16_t* y;
   const uint16_t* scales;
   const uint16_t* zeros;
   int M, N, K, G;
   int m_tiles, n_tiles, k_blocks;
+  int S;            // K slices per tile: 1 = persistent CTAs over whole tiles; 2, 4, 8 = one
+                    // cluster of S CTAs per tile, CTA r of the cluster taking slice r
+  int kb_per_unit;  // k blocks one CTA multiplies per tile (k_blocks / S)
 };
 
 template <bool ZP>
@@ -162,6 +268,12 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int num_tiles = p.m_tiles * p.n_tiles;
+  // work of this CTA: tiles t_first, t_first + t_step, ..., k blocks [kb0, kb1) of each
+  const bool split = p.S > 1;
+  const int t_first = split ? int(blockIdx.x) / p.S : int(blockIdx.x);
+  const int t_step = split ? num_tiles : int(gridDim.x);
+  const int kb0 = split ? (int(blockIdx.x) % p.S) * p.kb_per_unit : 0;
+  const int kb1 = kb0 + p.kb_per_unit;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -196,30 +308,28 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
     int s = 0;
     uint32_t ph = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+    for (int tile = t_first; tile < num_tiles && ok; tile += t_step) {
       const int n0 = (tile / p.m_tiles) * BN;
       const int64_t row = int64_t(n0) + i;
       const bool valid = row < p.N;
       // group-major metadata: consecutive threads read consecutive rows
-      const uint16_t* scol = p.scales + (valid ? row : 0);
-      const uint16_t* zcol = ZP ? p.zeros + (valid ? row : 0) : nullptr;
+      MetaChain<ZP> meta;
+      meta.scol = p.scales + (valid ? row : 0);
+      meta.zcol = ZP ? p.zeros + (valid ? row : 0) : nullptr;
+      meta.N = p.N;
+      meta.G = p.G;
+      meta.valid = valid;
+      meta.start(kb0 >> 1);   // kb0 is even: slices hold whole groups
       uint32_t zb1024 = 0, zb64 = 0, sc2 = 0;
-      // scale and zero of group 0, then always one group ahead
-      uint16_t s_next = valid ? ld_nc_u16(scol) : uint16_t(0);
-      uint16_t z_next = (ZP && valid) ? ld_nc_u16(zcol) : uint16_t(0);
-      for (int kb = 0; kb < p.k_blocks; ++kb) {
+      for (int kb = kb0; kb < kb1; ++kb) {
         if ((kb & 1) == 0) {  // new group of 128 k
-          const uint16_t sb = s_next;
-          const float z = ZP ? half_bits_to_float(z_next) : 8.0f;
-          const int gn = (kb >> 1) + 1;
-          if (valid && gn < p.G) {
-            s_next = ld_nc_u16(scol + int64_t(gn) * p.N);
-            if (ZP) z_next = ld_nc_u16(zcol + int64_t(gn) * p.N);
-          }
+          uint16_t sb, zbits;
+          meta.next(kb >> 1, sb, zbits);
+          const float z = ZP ? half_bits_to_float(zbits) : 8.0f;
           zero_bias_pairs(z, zb1024, zb64);
           sc2 = uint32_t(sb) | (uint32_t(sb) << 16);
         }
-        if (!wait_bounded(&bars->full_a[s], ph, abort, &g_awq_error_word, 1u)) { ok = false; break; }
+        if (!wait_sleep(&bars->full_a[s], ph, abort)) { ok = false; break; }
         // codes of row i: 32 bytes, 16-byte halves swapped on rows with bit 2 set
         // (32B swizzle); this thread decodes half h
         const uint8_t* crow = smem + SmemLayout::c(s) + i * 32;
@@ -245,15 +355,15 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
       }
     }
   } else if (warp < kEpiWarp0 + 4) {
-    // ------------------------------------------------------------ epilogue
+    // ------------------------------------------------------------ epilogue (whole tiles)
     const int q = warp - kEpiWarp0;            // TMEM lane quadrant (warp % 4)
     int it = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+    for (int tile = t_first; tile < num_tiles && !split; tile += t_step, ++it) {
       const int m0 = (tile % p.m_tiles) * BM;
       const int n0 = (tile / p.m_tiles) * BN;
       const int acc = it % kAccBufs;
       const uint32_t aph = (it / kAccBufs) & 1;
-      if (!wait_bounded(&bars->tmem_full[acc], aph, abort, &g_awq_error_word, 1u)) break;
+      if (!wait_sleep(&bars->tmem_full[acc], aph, abort)) break;
       tc_fence_after();
       const int halves = m0 + BMH < p.M ? 2 : 1;   // the MMAs skip an upper half with no rows
 #pragma unroll 1
@@ -295,11 +405,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
       bool ok = true;
       bool issued[kStages] = {};
       uint32_t issued_ph[kStages] = {};
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      for (int tile = t_first; tile < num_tiles && ok; tile += t_step) {
         const int m0 = (tile % p.m_tiles) * BM;
         const int n0 = (tile / p.m_tiles) * BN;
-        for (int kb = 0; kb < p.k_blocks; ++kb) {
-          if (!wait_bounded(&bars->empty[s], ph ^ 1, abort, &g_awq_error_word, 1u)) { ok = false; break; }
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!wait_sleep(&bars->empty[s], ph ^ 1, abort)) { ok = false; break; }
           mbar_arrive_expect_tx(&bars->full_a[s], kABytes + kCBytes);
           tma_load_2d(smem + SmemLayout::a(s), &tmap_x, kb * BK, m0, &bars->full_a[s]);
           tma_load_2d(smem + SmemLayout::c(s), &tmap_q, kb * (BK / 8), n0, &bars->full_a[s]);
@@ -319,24 +429,25 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
       uint32_t ph = 0;
       int it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
+      for (int tile = t_first; tile < num_tiles && ok; tile += t_step, ++it) {
         const int acc = it % kAccBufs;
         const uint32_t aph = (it / kAccBufs) & 1;
-        if (!wait_bounded(&bars->tmem_empty[acc], aph ^ 1, abort, &g_awq_error_word, 1u)) break;
+        if (!wait_sleep(&bars->tmem_empty[acc], aph ^ 1, abort)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + uint32_t(acc * kAccCols);
         const bool upper = (tile % p.m_tiles) * BM + BMH < p.M;   // rows of x in the upper half
-        for (int kb = 0; kb < p.k_blocks; ++kb) {
-          if (!wait_bounded(&bars->full_a[s], ph, abort, &g_awq_error_word, 1u) ||
-              !wait_bounded(&bars->full_b[s], ph, abort, &g_awq_error_word, 1u)) { ok = false; break; }
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!wait_sleep(&bars->full_a[s], ph, abort) ||
+              !wait_sleep(&bars->full_b[s], ph, abort)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + SmemLayout::a(s));
           const uint32_t b_addr = smem_u32(smem + SmemLayout::b(s));
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
             const uint64_t bd = sw128_desc(b_addr + k * 32);
-            tc_mma_f16(d_tmem, sw128_desc(a_addr + k * 32), bd, kIdesc, (kb | k) != 0);
-            if (upper) tc_mma_f16(d_tmem + BN, sw128_desc(a_addr + BMH * 128 + k * 32), bd, kIdesc, (kb | k) != 0);
+            const uint32_t accum = (kb > kb0 || k > 0) ? 1u : 0u;
+            tc_mma_f16(d_tmem, sw128_desc(a_addr + k * 32), bd, kIdesc, accum);
+            if (upper) tc_mma_f16(d_tmem + BN, sw128_desc(a_addr + BMH * 128 + k * 32), bd, kIdesc, accum);
           }
           tc_commit(&bars->empty[s]);
           if (++s == kStages) { s = 0; ph ^= 1; }
@@ -346,6 +457,81 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
       // every MMA this thread issued completes before tensor memory is freed
       tc_commit(&bars->mma_done);
       wait_teardown(&bars->mma_done, 0);
+    }
+  }
+
+  if (split) {
+    // ------------------------------------------------------------ K-slice reduction (all warps)
+    // Each CTA of the cluster holds the fp32 partial of its K slice for the
+    // tile. Per half of x: the epilogue warps copy the partial from tensor
+    // memory into this CTA's shared memory (the stage area, idle once the
+    // accumulator is complete); after a cluster barrier CTA r sums rows
+    // [r 128/S, (r+1) 128/S) of every slice's partial, in slice order (so
+    // the bits do not depend on timing), and stores them as fp16; a second
+    // barrier keeps every partial in place until all CTAs have read it.
+    const int tile = t_first;
+    const int m0 = (tile % p.m_tiles) * BM;
+    const int n0 = (tile / p.m_tiles) * BN;
+    const int halves = m0 + BMH < p.M ? 2 : 1;
+    const int rank = int(blockIdx.x) % p.S;
+    float* part = reinterpret_cast<float*>(smem);
+    const bool epi = warp >= kEpiWarp0 && warp < kEpiWarp0 + 4;
+    bool have = false;
+    if (epi) {
+      have = wait_sleep(&bars->tmem_full[0], 0u, abort);
+      tc_fence_after();
+    }
+    const int rows_per = BMH / p.S;
+    for (int hm = 0; hm < halves; ++hm) {
+      if (epi && have) {
+        const int q = warp - kEpiWarp0;
+        const int r = q * 32 + lane;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t v[32];
+          tc_ld_32x32b_x32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(hm * BN + c * 32), v);
+          float4* dst = reinterpret_cast<float4*>(part + r * kPartStride + c * 32);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            dst[e] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
+                                 __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
+        }
+      }
+      cluster_sync_all();
+      for (int idx = threadIdx.x; idx < rows_per * (BN / 4); idx += kGemmThreads) {
+        const int r = rank * rows_per + idx / (BN / 4);
+        const int c4 = idx % (BN / 4);
+        const int64_t m = int64_t(m0) + hm * BMH + r;
+        const int n = n0 + 4 * c4;
+        if (m >= p.M || n >= p.N) continue;
+        const uint32_t off = smem_u32(part + r * kPartStride + 4 * c4);
+        // all slices' loads in flight at once, then summed in slice order
+        float4 v[kMaxSlices];
+#pragma unroll
+        for (int sl = 0; sl < kMaxSlices; ++sl)
+          if (sl < p.S) v[sl] = ld_dsmem_f4(off, sl);
+        float4 acc = v[0];
+#pragma unroll
+        for (int sl = 1; sl < kMaxSlices; ++sl)
+          if (sl < p.S) {
+            acc.x += v[sl].x;
+            acc.y += v[sl].y;
+            acc.z += v[sl].z;
+            acc.w += v[sl].w;
+          }
+        const float a4[4] = {acc.x, acc.y, acc.z, acc.w};
+        uint16_t* yrow = p.y + m * p.N;
+        if (n + 4 <= p.N && (p.N & 3) == 0) {
+          const uint32_t lo = uint32_t(__half_as_ushort(__float2half_rn(a4[0]))) |
+                              (uint32_t(__half_as_ushort(__float2half_rn(a4[1]))) << 16);
+          const uint32_t hi = uint32_t(__half_as_ushort(__float2half_rn(a4[2]))) |
+                              (uint32_t(__half_as_ushort(__float2half_rn(a4[3]))) << 16);
+          *reinterpret_cast<uint2*>(yrow + n) = make_uint2(lo, hi);
+        } else {
+          for (int e = 0; e < 4 && n + e < p.N; ++e) yrow[n + e] = __half_as_ushort(__float2half_rn(a4[e]));
+        }
+      }
+      cluster_sync_all();
     }
   }
 
@@ -364,6 +550,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
 constexpr int kMaxDevices = 64;
 std::atomic<int> g_sms[kMaxDevices];
 std::atomic<int> g_attr_set[kMaxDevices][2];
+// clusters of 2, 4, 8 CTAs that fit at once: 0 = not queried yet, -1 = none, else the count
+std::atomic<int> g_clusters[kMaxDevices][2][3];
 
 }  // namespace
 
@@ -435,8 +623,62 @@ extern "C" awq_status_t awq_gemm(const uint16_t* x, const int32_t* qweight,
   p.k_blocks = int(K / BK);
   const int64_t tiles = int64_t(p.m_tiles) * p.n_tiles;
   if (tiles > (int64_t(1) << 31) - 1) return AWQ_ERR_SHAPE;
-  const int grid = int(tiles < sms ? tiles : sms);
-  kernel<<<grid, kGemmThreads, kSmemBytes, static_cast<cudaStream_t>(stream)>>>(tmap_x, tmap_q, p);
+  // Few tiles: split K over a cluster of S CTAs per tile (whole groups per
+  // slice, at least 4 k blocks each). S is chosen to minimise
+  //   waves(S) x (k blocks per slice + 8),
+  // waves(S) = ceil(tiles / clusters of S that fit at once) (S = 1: the
+  // persistent grid of one CTA per SM); the 8 k blocks stand for the pipeline
+  // fill and the epilogue / slice reduction.
+  p.S = 1;
+  if (2 * tiles <= sms) {
+    int64_t best = ((tiles + sms - 1) / sms) * (p.k_blocks + 8);
+    const int cands[3] = {2, 4, 8};
+    for (int ci = 0; ci < 3; ++ci) {
+      const int S = cands[ci];
+      if (p.G % S != 0 || p.k_blocks / S < 4) continue;
+      int fit = g_clusters[dev][zi][ci].load(std::memory_order_acquire);
+      if (fit == 0) {
+        cudaLaunchConfig_t qc = {};
+        qc.gridDim = dim3(unsigned(S));
+        qc.blockDim = dim3(kGemmThreads);
+        qc.dynamicSmemBytes = kSmemBytes;
+        cudaLaunchAttribute qa[1];
+        qa[0].id = cudaLaunchAttributeClusterDimension;
+        qa[0].val.clusterDim.x = unsigned(S);
+        qa[0].val.clusterDim.y = 1;
+        qa[0].val.clusterDim.z = 1;
+        qc.attrs = qa;
+        qc.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, kernel, &qc) != cudaSuccess) {
+          (void)cudaGetLastError();
+          n = 0;
+        }
+        fit = n > 0 ? n : -1;
+        g_clusters[dev][zi][ci].store(fit, std::memory_order_release);
+      }
+      if (fit <= 0) continue;
+      const int64_t cost = ((tiles + fit - 1) / fit) * (p.k_blocks / S + 8);
+      if (cost < best) {
+        best = cost;
+        p.S = S;
+      }
+    }
+  }
+  p.kb_per_unit = p.k_blocks / p.S;
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(unsigned(p.S > 1 ? tiles * p.S : (tiles < sms ? tiles : sms)));
+  lc.blockDim = dim3(kGemmThreads);
+  lc.dynamicSmemBytes = kSmemBytes;
+  lc.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = unsigned(p.S);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  lc.attrs = attr;
+  lc.numAttrs = p.S > 1 ? 1 : 0;
+  if (cudaLaunchKernelEx(&lc, kernel, tmap_x, tmap_q, p) != cudaSuccess) return AWQ_ERR_CUDA;
   return launch_status();
 }
 
