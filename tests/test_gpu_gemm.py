@@ -64,6 +64,17 @@ def test_gemm_cta_pairs_many_tiles(N, K, M):
     assert np.array_equal(bits(y), bits(run_gemm(x, qweight, scales, zeros)))
 
 
+def test_gemm_last_partial_wave_goes_to_k_slices():
+    """150 tiles on 148 SMs: 148 on the persistent grid, the last 2 (the
+    ragged last channel tile, both row tiles, the second only partly filled)
+    in a second launch with K split over clusters. Full compare."""
+    N, K, M = 19192, 1024, 500
+    _, qweight, scales, zeros, Wd = oracle_layer(N, K, 0.02, 0.01, True)
+    x = activations(M, K, seed=71)
+    y = run_gemm(x, qweight, scales, zeros)
+    assert_close(y, O.matmul_f64(x, Wd), f"N={N} K={K} M={M}")
+
+
 @pytest.mark.parametrize("N,K,M", [(512, 4096, 200), (1024, 2048, 64), (2048, 8192, 129), (4096, 4096, 17)])
 def test_gemm_k_slices_over_a_cluster(N, K, M):
     """Few tiles: K is split over a cluster of 4 or 8 CTAs per tile and the slices

@@ -251,6 +251,7 @@ struct GemmParams {
   const uint16_t* zeros;
   int M, N, K, G;
   int m_tiles, n_tiles, k_blocks;
+  int tile0, num_tiles;   // this launch takes tiles tile0 .. tile0 + num_tiles - 1
   int S;            // K slices per tile: 1 = persistent CTAs over whole tiles; 2, 4, 8 = one
                     // cluster of S CTAs per tile, CTA r of the cluster taking slice r
   int kb_per_unit;  // k blocks one CTA multiplies per tile (k_blocks / S)
@@ -267,7 +268,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
   volatile int* abort = &bars->abort;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int num_tiles = p.m_tiles * p.n_tiles;
+  const int num_tiles = p.num_tiles;   // tile indices below are relative to p.tile0
   // work of this CTA: tiles t_first, t_first + t_step, ..., k blocks [kb0, kb1) of each
   const bool split = p.S > 1;
   const int t_first = split ? int(blockIdx.x) / p.S : int(blockIdx.x);
@@ -309,7 +310,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
     uint32_t ph = 0;
     bool ok = true;
     for (int tile = t_first; tile < num_tiles && ok; tile += t_step) {
-      const int n0 = (tile / p.m_tiles) * BN;
+      const int n0 = ((tile + p.tile0) / p.m_tiles) * BN;
       const int64_t row = int64_t(n0) + i;
       const bool valid = row < p.N;
       // group-major metadata: consecutive threads read consecutive rows
@@ -359,8 +360,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
     const int q = warp - kEpiWarp0;            // TMEM lane quadrant (warp % 4)
     int it = 0;
     for (int tile = t_first; tile < num_tiles && !split; tile += t_step, ++it) {
-      const int m0 = (tile % p.m_tiles) * BM;
-      const int n0 = (tile / p.m_tiles) * BN;
+      const int m0 = ((tile + p.tile0) % p.m_tiles) * BM;
+      const int n0 = ((tile + p.tile0) / p.m_tiles) * BN;
       const int acc = it % kAccBufs;
       const uint32_t aph = (it / kAccBufs) & 1;
       if (!wait_sleep(&bars->tmem_full[acc], aph, abort)) break;
@@ -406,8 +407,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
       bool issued[kStages] = {};
       uint32_t issued_ph[kStages] = {};
       for (int tile = t_first; tile < num_tiles && ok; tile += t_step) {
-        const int m0 = (tile % p.m_tiles) * BM;
-        const int n0 = (tile / p.m_tiles) * BN;
+        const int m0 = ((tile + p.tile0) % p.m_tiles) * BM;
+        const int n0 = ((tile + p.tile0) / p.m_tiles) * BN;
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!wait_sleep(&bars->empty[s], ph ^ 1, abort)) { ok = false; break; }
           mbar_arrive_expect_tx(&bars->full_a[s], kABytes + kCBytes);
@@ -435,7 +436,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         if (!wait_sleep(&bars->tmem_empty[acc], aph ^ 1, abort)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + uint32_t(acc * kAccCols);
-        const bool upper = (tile % p.m_tiles) * BM + BMH < p.M;   // rows of x in the upper half
+        const bool upper = ((tile + p.tile0) % p.m_tiles) * BM + BMH < p.M;   // rows of x in the upper half
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!wait_sleep(&bars->full_a[s], ph, abort) ||
               !wait_sleep(&bars->full_b[s], ph, abort)) { ok = false; break; }
@@ -470,8 +471,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
     // the bits do not depend on timing), and stores them as fp16; a second
     // barrier keeps every partial in place until all CTAs have read it.
     const int tile = t_first;
-    const int m0 = (tile % p.m_tiles) * BM;
-    const int n0 = (tile / p.m_tiles) * BN;
+    const int m0 = ((tile + p.tile0) % p.m_tiles) * BM;
+    const int n0 = ((tile + p.tile0) / p.m_tiles) * BN;
     const int halves = m0 + BMH < p.M ? 2 : 1;
     const int rank = int(blockIdx.x) % p.S;
     float* part = reinterpret_cast<float*>(smem);
@@ -623,63 +624,81 @@ extern "C" awq_status_t awq_gemm(const uint16_t* x, const int32_t* qweight,
   p.k_blocks = int(K / BK);
   const int64_t tiles = int64_t(p.m_tiles) * p.n_tiles;
   if (tiles > (int64_t(1) << 31) - 1) return AWQ_ERR_SHAPE;
-  // Few tiles: split K over a cluster of S CTAs per tile (whole groups per
-  // slice, at least 4 k blocks each). S is chosen to minimise
+  // One launch takes tiles tile0 .. tile0 + count - 1. Few tiles: split K
+  // over a cluster of S CTAs per tile (whole groups per slice, at least 4 k
+  // blocks each). S is chosen to minimise
   //   waves(S) x (k blocks per slice + 8),
-  // waves(S) = ceil(tiles / clusters of S that fit at once) (S = 1: the
+  // waves(S) = ceil(count / clusters of S that fit at once) (S = 1: the
   // persistent grid of one CTA per SM); the 8 k blocks stand for the pipeline
   // fill and the epilogue / slice reduction.
-  p.S = 1;
-  if (2 * tiles <= sms) {
-    int64_t best = ((tiles + sms - 1) / sms) * (p.k_blocks + 8);
-    const int cands[3] = {2, 4, 8};
-    for (int ci = 0; ci < 3; ++ci) {
-      const int S = cands[ci];
-      if (p.G % S != 0 || p.k_blocks / S < 4) continue;
-      int fit = g_clusters[dev][zi][ci].load(std::memory_order_acquire);
-      if (fit == 0) {
-        cudaLaunchConfig_t qc = {};
-        qc.gridDim = dim3(unsigned(S));
-        qc.blockDim = dim3(kGemmThreads);
-        qc.dynamicSmemBytes = kSmemBytes;
-        cudaLaunchAttribute qa[1];
-        qa[0].id = cudaLaunchAttributeClusterDimension;
-        qa[0].val.clusterDim.x = unsigned(S);
-        qa[0].val.clusterDim.y = 1;
-        qa[0].val.clusterDim.z = 1;
-        qc.attrs = qa;
-        qc.numAttrs = 1;
-        int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, kernel, &qc) != cudaSuccess) {
-          (void)cudaGetLastError();
-          n = 0;
+  auto launch_part = [&](int64_t tile0, int64_t count) -> awq_status_t {
+    GemmParams q = p;
+    q.tile0 = int(tile0);
+    q.num_tiles = int(count);
+    q.S = 1;
+    if (2 * count <= sms) {
+      int64_t best = ((count + sms - 1) / sms) * (q.k_blocks + 8);
+      const int cands[3] = {2, 4, 8};
+      for (int ci = 0; ci < 3; ++ci) {
+        const int S = cands[ci];
+        if (q.G % S != 0 || q.k_blocks / S < 4) continue;
+        int fit = g_clusters[dev][zi][ci].load(std::memory_order_acquire);
+        if (fit == 0) {
+          cudaLaunchConfig_t qc = {};
+          qc.gridDim = dim3(unsigned(S));
+          qc.blockDim = dim3(kGemmThreads);
+          qc.dynamicSmemBytes = kSmemBytes;
+          cudaLaunchAttribute qa[1];
+          qa[0].id = cudaLaunchAttributeClusterDimension;
+          qa[0].val.clusterDim.x = unsigned(S);
+          qa[0].val.clusterDim.y = 1;
+          qa[0].val.clusterDim.z = 1;
+          qc.attrs = qa;
+          qc.numAttrs = 1;
+          int n = 0;
+          if (cudaOccupancyMaxActiveClusters(&n, kernel, &qc) != cudaSuccess) {
+            (void)cudaGetLastError();
+            n = 0;
+          }
+          fit = n > 0 ? n : -1;
+          g_clusters[dev][zi][ci].store(fit, std::memory_order_release);
         }
-        fit = n > 0 ? n : -1;
-        g_clusters[dev][zi][ci].store(fit, std::memory_order_release);
-      }
-      if (fit <= 0) continue;
-      const int64_t cost = ((tiles + fit - 1) / fit) * (p.k_blocks / S + 8);
-      if (cost < best) {
-        best = cost;
-        p.S = S;
+        if (fit <= 0) continue;
+        const int64_t cost = ((count + fit - 1) / fit) * (q.k_blocks / S + 8);
+        if (cost < best) {
+          best = cost;
+          q.S = S;
+        }
       }
     }
+    q.kb_per_unit = q.k_blocks / q.S;
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3(unsigned(q.S > 1 ? count * q.S : (count < sms ? count : sms)));
+    lc.blockDim = dim3(kGemmThreads);
+    lc.dynamicSmemBytes = kSmemBytes;
+    lc.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = unsigned(q.S);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    lc.attrs = attr;
+    lc.numAttrs = q.S > 1 ? 1 : 0;
+    if (cudaLaunchKernelEx(&lc, kernel, tmap_x, tmap_q, q) != cudaSuccess) return AWQ_ERR_CUDA;
+    return launch_status();
+  };
+  // Whole waves of one tile per SM stay on the persistent grid. A last partial
+  // wave of at most half the SMs goes to a second launch, where its few tiles
+  // split K over clusters instead of leaving the other SMs idle while they
+  // finish (448 tiles on 148 SMs: 3 waves + 4 tiles). The launches write
+  // disjoint tiles of y.
+  const int64_t rem = tiles % sms;
+  if (tiles > sms && rem > 0 && 2 * rem <= sms) {
+    const awq_status_t st1 = launch_part(0, tiles - rem);
+    if (st1 != AWQ_OK) return st1;
+    return launch_part(tiles - rem, rem);
   }
-  p.kb_per_unit = p.k_blocks / p.S;
-  cudaLaunchConfig_t lc = {};
-  lc.gridDim = dim3(unsigned(p.S > 1 ? tiles * p.S : (tiles < sms ? tiles : sms)));
-  lc.blockDim = dim3(kGemmThreads);
-  lc.dynamicSmemBytes = kSmemBytes;
-  lc.stream = static_cast<cudaStream_t>(stream);
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = unsigned(p.S);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  lc.attrs = attr;
-  lc.numAttrs = p.S > 1 ? 1 : 0;
-  if (cudaLaunchKernelEx(&lc, kernel, tmap_x, tmap_q, p) != cudaSuccess) return AWQ_ERR_CUDA;
-  return launch_status();
+  return launch_part(0, tiles);
 }
 
 extern "C" awq_status_t awq_device_error(uint32_t* error_word, void* stream) {
