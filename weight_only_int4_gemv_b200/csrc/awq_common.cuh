@@ -195,6 +195,45 @@ __device__ __forceinline__ void wait_teardown(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// mbarrier.try_wait with a suspend-time hint: a thread whose phase is not yet
+// complete sleeps until it completes (or the 1 ms hint runs out) instead of
+// re-polling, so waiting warps do not take issue slots from the warps that
+// share their scheduler.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u)
+      : "memory");
+  return ok != 0;
+}
+
+// wait_bounded built on the sleeping try_wait (same limit, abort flag and
+// error bit).
+__device__ __forceinline__ bool wait_sleep(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                           uint32_t* err, uint32_t err_bit) {
+  if (mbar_try_wait_sleep(bar, parity)) return true;
+  const uint64_t t0 = now_ns();
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity)) return true;
+    if (*abort) return false;
+    if (now_ns() - t0 > kWaitLimitNs) {
+      *abort = 1;
+      atomicOr(err, err_bit);
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void wait_sleep_teardown(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = now_ns();
+  while (!mbar_try_wait_sleep(bar, parity) && now_ns() - t0 < kWaitLimitNs) {
+  }
+}
+
 // 2-D tiled TMA load of one box into shared memory, completing on `bar`.
 __device__ __forceinline__ void tma_load_2d(void* dst, const void* tensor_map, int x, int y,
                                             uint64_t* bar) {

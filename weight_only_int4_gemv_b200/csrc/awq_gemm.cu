@@ -158,44 +158,6 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
          (uint64_t(1) << 46) | (uint64_t(2) << 61);
 }
 
-// mbarrier.try_wait with a suspend-time hint: a thread whose phase is not yet
-// complete sleeps until it completes (or the hint runs out) instead of
-// re-polling, so waiting warps (MMA issuer, epilogue, producer) do not take
-// issue slots from the decode warps that share their scheduler.
-__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u)
-      : "memory");
-  return ok != 0;
-}
-
-// Bounded wait (same protocol as wait_bounded: 2 s limit, abort flag, error
-// bit 0) built on the sleeping try_wait.
-__device__ __forceinline__ bool wait_sleep(uint64_t* bar, uint32_t parity, volatile int* abort) {
-  if (mbar_try_wait_sleep(bar, parity)) return true;
-  const uint64_t t0 = now_ns();
-  for (;;) {
-    if (mbar_try_wait_sleep(bar, parity)) return true;
-    if (*abort) return false;
-    if (now_ns() - t0 > kWaitLimitNs) {
-      *abort = 1;
-      atomicOr(&g_awq_error_word, 1u);
-      return false;
-    }
-  }
-}
-
-__device__ __forceinline__ void wait_sleep_teardown(uint64_t* bar, uint32_t parity) {
-  const uint64_t t0 = now_ns();
-  while (!mbar_try_wait_sleep(bar, parity) && now_ns() - t0 < kWaitLimitNs) {
-  }
-}
-
 // Scale and zero point of one weight row, loaded kMetaAhead groups before
 // their use through a register shift chain: the global-load latency (over a
 // microsecond under load) stays off the k loop, which otherwise waits for it
@@ -330,7 +292,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
           zero_bias_pairs(z, zb1024, zb64);
           sc2 = uint32_t(sb) | (uint32_t(sb) << 16);
         }
-        if (!wait_sleep(&bars->full_a[s], ph, abort)) { ok = false; break; }
+        if (!wait_sleep(&bars->full_a[s], ph, abort, &g_awq_error_word, 1u)) { ok = false; break; }
         // codes of row i: 32 bytes, 16-byte halves swapped on rows with bit 2 set
         // (32B swizzle); this thread decodes half h
         const uint8_t* crow = smem + SmemLayout::c(s) + i * 32;
@@ -364,7 +326,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
       const int n0 = ((tile + p.tile0) / p.m_tiles) * BN;
       const int acc = it % kAccBufs;
       const uint32_t aph = (it / kAccBufs) & 1;
-      if (!wait_sleep(&bars->tmem_full[acc], aph, abort)) break;
+      if (!wait_sleep(&bars->tmem_full[acc], aph, abort, &g_awq_error_word, 1u)) break;
       tc_fence_after();
       const int halves = m0 + BMH < p.M ? 2 : 1;   // the MMAs skip an upper half with no rows
 #pragma unroll 1
@@ -410,7 +372,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         const int m0 = ((tile + p.tile0) % p.m_tiles) * BM;
         const int n0 = ((tile + p.tile0) / p.m_tiles) * BN;
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!wait_sleep(&bars->empty[s], ph ^ 1, abort)) { ok = false; break; }
+          if (!wait_sleep(&bars->empty[s], ph ^ 1, abort, &g_awq_error_word, 1u)) { ok = false; break; }
           mbar_arrive_expect_tx(&bars->full_a[s], kABytes + kCBytes);
           tma_load_2d(smem + SmemLayout::a(s), &tmap_x, kb * BK, m0, &bars->full_a[s]);
           tma_load_2d(smem + SmemLayout::c(s), &tmap_q, kb * (BK / 8), n0, &bars->full_a[s]);
@@ -433,13 +395,13 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
       for (int tile = t_first; tile < num_tiles && ok; tile += t_step, ++it) {
         const int acc = it % kAccBufs;
         const uint32_t aph = (it / kAccBufs) & 1;
-        if (!wait_sleep(&bars->tmem_empty[acc], aph ^ 1, abort)) break;
+        if (!wait_sleep(&bars->tmem_empty[acc], aph ^ 1, abort, &g_awq_error_word, 1u)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + uint32_t(acc * kAccCols);
         const bool upper = ((tile + p.tile0) % p.m_tiles) * BM + BMH < p.M;   // rows of x in the upper half
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!wait_sleep(&bars->full_a[s], ph, abort) ||
-              !wait_sleep(&bars->full_b[s], ph, abort)) { ok = false; break; }
+          if (!wait_sleep(&bars->full_a[s], ph, abort, &g_awq_error_word, 1u) ||
+              !wait_sleep(&bars->full_b[s], ph, abort, &g_awq_error_word, 1u)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + SmemLayout::a(s));
           const uint32_t b_addr = smem_u32(smem + SmemLayout::b(s));
@@ -479,7 +441,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
     const bool epi = warp >= kEpiWarp0 && warp < kEpiWarp0 + 4;
     bool have = false;
     if (epi) {
-      have = wait_sleep(&bars->tmem_full[0], 0u, abort);
+      have = wait_sleep(&bars->tmem_full[0], 0u, abort, &g_awq_error_word, 1u);
       tc_fence_after();
     }
     const int rows_per = BMH / p.S;
