@@ -95,7 +95,6 @@ struct GemvParams {
   int stage_bytes;       // codes + metadata + x slice of one unit (multiple of 128)
   int x_offset;          // offset of the x slice inside a stage
   int pbuf_offset;       // shared-memory partial sums of the chunk reductions
-  int chunk_tiles;       // tiles per chunk (the kernel's TC)
   int scale_offset;      // offset of the scales inside a stage (TC tiles of codes before it)
   int early;             // weights may be read before the previous kernel completes
   int codes4d;           // stage codes as one 4-D box (N % 16 == 0)
@@ -140,12 +139,12 @@ struct Chunk {
   int gb, ge;  // groups of the slice
 };
 
-__device__ __forceinline__ void load_chunk(const GemvParams& p, int i, int i_end, Chunk& c) {
+__device__ __forceinline__ void load_chunk(const GemvParams& p, int ct, int i, int i_end, Chunk& c) {
   c.i = i;
   c.s = i / p.T;
   c.t0 = i - c.s * p.T;
   int tc = i_end - i;
-  if (tc > p.chunk_tiles) tc = p.chunk_tiles;
+  if (tc > ct) tc = ct;
   if (tc > p.T - c.t0) tc = p.T - c.t0;
   c.tc = tc;
   c.gb = int(int64_t(p.G) * c.s / p.ks);
@@ -162,19 +161,19 @@ struct StageCursor {
   __device__ __forceinline__ bool done() const { return gbase < 0; }
 };
 
-__device__ __forceinline__ void cursor_init(const GemvParams& p, int i0, int i1, StageCursor& u) {
-  load_chunk(p, i0, i1, u.c);
+__device__ __forceinline__ void cursor_init(const GemvParams& p, int ct, int i0, int i1, StageCursor& u) {
+  load_chunk(p, ct, i0, i1, u.c);
   u.gbase = u.c.gb;
 }
 
-__device__ __forceinline__ void cursor_next(const GemvParams& p, int i_end, StageCursor& u) {
+__device__ __forceinline__ void cursor_next(const GemvParams& p, int ct, int i_end, StageCursor& u) {
   u.gbase += kWarps;
   if (u.gbase >= u.c.ge) {
     const int ni = u.c.i + u.c.tc;
     if (ni >= i_end) {
       u.gbase = -1;
     } else {
-      load_chunk(p, ni, i_end, u.c);
+      load_chunk(p, ct, ni, i_end, u.c);
       u.gbase = u.c.gb;
     }
   }
@@ -260,7 +259,7 @@ __device__ __forceinline__ void chunk_stages(const GemvParams& p, Pipe<MT>& pp, 
 #pragma unroll
           for (int jj = 0; jj < 4; ++jj) xf[mt][jj] = pp.xok[mt] ? lds128(st + pp.xoff[mt] + jj * 16) : make_uint4(0, 0, 0, 0);
         const uint8_t* cw = st + pp.w * (kTile * 64) + pp.g * 64 + pp.t * 16;
-        const uint8_t* sw = st + TC * kTileStageBytes + pp.w * 128 + pp.g * 2;
+        const uint8_t* sw = st + p.scale_offset + pp.w * 128 + pp.g * 2;
 #pragma unroll
         for (int rt = 0; rt < TC; ++rt) {
           c_lo[rt] = lds128(cw + rt * kTileStageBytes);
@@ -289,7 +288,7 @@ __device__ __forceinline__ void chunk_stages(const GemvParams& p, Pipe<MT>& pp, 
             pp.fills[pp.slot] += 1u;
           }
         }
-        cursor_next(p, pp.i1, pp.pc);
+        cursor_next(p, TC, pp.i1, pp.pc);
       }
 
       if (has) {
@@ -353,16 +352,13 @@ __device__ __forceinline__ void chunk_stages(const GemvParams& p, Pipe<MT>& pp, 
 
 }
 
+// One CTA's work: items [i0, i1) in chunks of at most TC tiles.
 template <int MT, bool ZP, int TC>
-__global__ void __launch_bounds__(kThreads, MT == 1 ? 2 : 1)
-gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_x,
-            const __grid_constant__ CUtensorMap tmap_s, const __grid_constant__ CUtensorMap tmap_z,
-            const __grid_constant__ CodeMaps code_maps, const GemvParams p) {
+__device__ __forceinline__ void gemv_cta(const CUtensorMap& tmap_q, const CUtensorMap& tmap_x,
+                                         const CUtensorMap& tmap_s, const CUtensorMap& tmap_z,
+                                         const CodeMaps& code_maps, const GemvParams& p, const int i0,
+                                         const int i1) {
   extern __shared__ __align__(1024) uint8_t gemv_smem[];
-  // Let the next kernel in the stream (if launched as a programmatic
-  // dependent) start as soon as every CTA of this one is running; it waits
-  // for this grid's completion before it reads anything this grid writes.
-  asm volatile("griddepcontrol.launch_dependents;");
 
   const int lane = threadIdx.x & 31;
   const int w = threadIdx.x >> 5;
@@ -376,9 +372,6 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
   uint32_t* failed = fills + kMaxStages;                                          // a warp gave up
   uint8_t* ring = gemv_smem + kRingOffset;
   float* pbuf = reinterpret_cast<float*>(gemv_smem + p.pbuf_offset);
-
-  const int i0 = int(int64_t(p.items) * blockIdx.x / gridDim.x);
-  const int i1 = int(int64_t(p.items) * (blockIdx.x + 1) / gridDim.x);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -394,14 +387,14 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
 
   // ---- the first S stages (weights possibly before the dependency wait)
   StageCursor pc;   // lane 0 of every warp: the stage S ahead of the arithmetic
-  if (lane == 0) cursor_init(p, i0, i1, pc);
+  if (lane == 0) cursor_init(p, TC, i0, i1, pc);
   if (threadIdx.x == 0) {
     if (p.early) {
       StageCursor u = pc;
       for (int s = 0; s < S && !u.done(); ++s) {
         mbar_arrive_expect_tx(&full[s], stage_tx_bytes(p, u.c.tc, ZP));
         issue_weights<ZP>(u, ring + s * p.stage_bytes, &full[s], &tmap_q, &tmap_s, &tmap_z, p.scale_offset, p.codes4d ? &code_maps : nullptr);
-        cursor_next(p, i1, u);
+        cursor_next(p, TC, i1, u);
       }
     } else {
       tma_prefetch_l2_3d(&tmap_q, 0, pc.c.t0 * kTile, pc.gbase);
@@ -419,7 +412,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
         tma_load_3d(st + p.x_offset, &tmap_x, 0, pc.gbase, 0, &full[s]);
         fills[s] = 1u;
       }
-      cursor_next(p, i1, pc);
+      cursor_next(p, TC, i1, pc);
     }
   }
 
@@ -456,7 +449,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
   offset_tile(g, pp.ca0, pp.ca2);
 
   Chunk cc;
-  load_chunk(p, i0, i1, cc);
+  load_chunk(p, TC, i0, i1, cc);
   for (int chunk = 0;; ++chunk) {
     const int tc = cc.tc;
     float acc[kChunkTiles][MT][4];
@@ -537,7 +530,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
     }
     const int ni = cc.i + cc.tc;
     if (ni >= i1) break;
-    load_chunk(p, ni, i1, cc);
+    load_chunk(p, TC, ni, i1, cc);
   }
 
   // If a warp gave up, copies may still be in flight: a slot is refilled
@@ -548,6 +541,30 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
     for (int s = 0; s < S; ++s)
       if (fills[s] > 0u) wait_teardown(&full[s], (fills[s] - 1u) & 1u);
   }
+}
+
+template <int MT, bool ZP, int TC>
+__global__ void __launch_bounds__(kThreads, MT == 1 ? 2 : 1)
+gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_x,
+            const __grid_constant__ CUtensorMap tmap_s, const __grid_constant__ CUtensorMap tmap_z,
+            const __grid_constant__ CodeMaps code_maps, const GemvParams p) {
+  // Let the next kernel in the stream (if launched as a programmatic
+  // dependent) start as soon as every CTA of this one is running; it waits
+  // for this grid's completion before it reads anything this grid writes.
+  asm volatile("griddepcontrol.launch_dependents;");
+  const int i0 = int(int64_t(p.items) * blockIdx.x / gridDim.x);
+  const int i1 = int(int64_t(p.items) * (blockIdx.x + 1) / gridDim.x);
+  // A CTA with exactly 3 items of one K slice runs 3-tile chunks instead of
+  // padding a 4-tile chunk (896 tiles on 296 CTAs: 288 CTAs hold 3). The
+  // arithmetic of the stream phase is the limit, and the two CTAs of an SM
+  // share it, so an SM with 3 + 4 tiles finishes sooner than with 4 + 4.
+  if constexpr (TC == 4) {
+    if (i1 - i0 == 3 && i0 / p.T == (i1 - 1) / p.T) {
+      gemv_cta<MT, ZP, 3>(tmap_q, tmap_x, tmap_s, tmap_z, code_maps, p, i0, i1);
+      return;
+    }
+  }
+  gemv_cta<MT, ZP, TC>(tmap_q, tmap_x, tmap_s, tmap_z, code_maps, p, i0, i1);
 }
 
 // ---------------------------------------------------------------------------
@@ -751,7 +768,6 @@ extern "C" awq_status_t awq_gemv(const uint16_t* x, const int32_t* qweight,
   p.stage_bytes = pl.stage_bytes;
   p.x_offset = pl.x_offset;
   p.pbuf_offset = pl.pbuf_offset;
-  p.chunk_tiles = pl.tc;
   p.scale_offset = pl.scale_offset;
   p.early = (cfg.flags & AWQ_FLAG_WEIGHTS_STATIC) ? 1 : 0;
   // Programmatic dependent launch: this grid may start while the previous
