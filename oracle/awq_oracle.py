@@ -226,3 +226,43 @@ def max_abs_ratio(y: np.ndarray, y_ref: np.ndarray) -> float:
     den = np.abs(y_ref).max() if y_ref.size else 0.0
     num = np.abs(y - y_ref).max() if y_ref.size else 0.0
     return float(num / den) if den > 0 else float(num)
+
+
+# ---------------------------------------------------------------------------
+# Fused MLP input projection ("AutoAWQ" code tour, "The Quantization Flow Up
+# Close": the fuser merges the gate and up projections into one quantized MLP
+# block; "AutoAWQ" capability page: fused blocks cut launches and
+# intermediate tensors). Reading: the activation is SiLU, that of the
+# Llama-family MLP whose fuser the tour names; h = silu(gate) * up.
+# ---------------------------------------------------------------------------
+TILE_ROWS = 16   # rows per tile of the interleaved gate/up layout (documented format)
+
+
+def silu_f64(v: np.ndarray) -> np.ndarray:
+    """SiLU in float64: v * sigmoid(v) = v / (1 + exp(-v))."""
+    v = np.asarray(v, dtype=np.float64)
+    with np.errstate(over="ignore"):
+        return v / (1.0 + np.exp(-v))
+
+
+def gate_up_silu_f64(x: np.ndarray, Wg_d: np.ndarray, Wu_d: np.ndarray) -> np.ndarray:
+    """h[m, n] = silu(sum_k x[m,k] w'g[n,k]) * sum_k x[m,k] w'u[n,k], both
+    products by the plain float64 definition."""
+    return silu_f64(matmul_f64(x, Wg_d)) * matmul_f64(x, Wu_d)
+
+
+def interleave_gate_up(a_gate: np.ndarray, a_up: np.ndarray, axis: int = 0) -> np.ndarray:
+    """The fused weight layout: along ``axis`` (rows of qweight, columns of the
+    group-major scales and zeros), 16-row tiles alternate gate, up: tile 2j
+    holds gate rows 16j .. 16j+15, tile 2j+1 holds up rows 16j .. 16j+15.
+    Needs the row count to be a multiple of 16."""
+    a_gate = np.moveaxis(np.asarray(a_gate), axis, 0)
+    a_up = np.moveaxis(np.asarray(a_up), axis, 0)
+    n = a_gate.shape[0]
+    if a_up.shape != a_gate.shape or n % TILE_ROWS:
+        raise ValueError("gate and up need the same shape and a multiple of 16 rows")
+    out = np.empty((2 * n,) + a_gate.shape[1:], dtype=a_gate.dtype)
+    for j in range(n // TILE_ROWS):
+        out[2 * j * TILE_ROWS:(2 * j + 1) * TILE_ROWS] = a_gate[j * TILE_ROWS:(j + 1) * TILE_ROWS]
+        out[(2 * j + 1) * TILE_ROWS:(2 * j + 2) * TILE_ROWS] = a_up[j * TILE_ROWS:(j + 1) * TILE_ROWS]
+    return np.moveaxis(out, 0, axis)
