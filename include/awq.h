@@ -63,7 +63,7 @@
 extern "C" {
 #endif
 
-#define AWQ_ABI_VERSION 2
+#define AWQ_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define AWQ_API __attribute__((visibility("default")))
@@ -99,6 +99,21 @@ typedef struct awq_qconfig {
  * arrays, for instance in a decode loop over weights loaded once. The other
  * entry points ignore it. */
 #define AWQ_FLAG_WEIGHTS_STATIC 1u
+
+/* Fused MLP input projection ("AutoAWQ" code tour, "The Quantization Flow Up
+ * Close": the fuser merges the gate and up projections into one quantized
+ * MLP block; "AutoAWQ" capability page: fused blocks save launches and
+ * intermediate tensors). With this flag awq_gemv, awq_gemv_noalloc and
+ * awq_gemm read qweight / scales / zeros as N rows in which 16-row tiles
+ * alternate between a gate and an up projection of N/2 rows each -- tile 2j
+ * holds gate rows 16j .. 16j+15, tile 2j+1 up rows 16j .. 16j+15 (scales and
+ * zeros: the same order along their N columns); awq_interleave_gate_up
+ * builds it -- and write y[M][N/2] with
+ *   y[m][n] = fp16( silu(g) * u ),  silu(v) = v / (1 + exp(-v)),
+ * g and u the fp32 sums of gate row n and up row n (the values awq_gemv /
+ * awq_gemm would round to fp16 for those rows), silu and the product in
+ * fp32 (expf). Requires N % 32 == 0. awq_workspace_bytes takes the flag. */
+#define AWQ_FLAG_SILU_MUL 2u
 
 /* ABI version of the loaded library (AWQ_ABI_VERSION at build time). */
 AWQ_API int awq_abi_version(void);
@@ -163,7 +178,8 @@ AWQ_API awq_status_t awq_workspace_bytes(int64_t M, int64_t N, int64_t K,
  * device and shape, so results are reproducible run to run.
  * M in [1, 16]; N >= 0 and N % 8 == 0 (0: no work); K > 0, K % group_size == 0.
  * (N % 8 keeps every 8-row run of scales and zero points 16-byte aligned.)
- * cfg.flags may hold AWQ_FLAG_WEIGHTS_STATIC (see there).
+ * cfg.flags may hold AWQ_FLAG_WEIGHTS_STATIC and AWQ_FLAG_SILU_MUL (see there;
+ * with the latter y is [M][N/2]).
  * workspace: at least awq_workspace_bytes(M, N, K) bytes, zero-filled before
  * first use (see above); may be NULL when that size is 0, which is the case
  * whenever N / 16 is at least the device's SM count.
@@ -210,6 +226,7 @@ AWQ_API awq_status_t awq_gemv_noalloc(const uint16_t* x, const int32_t* qweight,
  * multiplied on the tensor cores (tcgen05, fp16 inputs, fp32 accumulation in
  * tensor memory); y = fp16 of the fp32 sum.
  * M >= 0, N >= 0 (either 0: no work); K > 0, K % group_size == 0.
+ * cfg.flags may hold AWQ_FLAG_SILU_MUL (y is then [M][N/2]).
  * Workspace as for awq_gemv.
  */
 AWQ_API awq_status_t awq_gemm(const uint16_t* x, const int32_t* qweight,
@@ -217,6 +234,21 @@ AWQ_API awq_status_t awq_gemm(const uint16_t* x, const int32_t* qweight,
                       int64_t M, int64_t N, int64_t K, awq_qconfig_t cfg,
                       uint16_t* y, void* workspace, size_t workspace_bytes,
                       void* stream);
+
+/*
+ * awq_interleave_gate_up -- build the AWQ_FLAG_SILU_MUL weight layout from
+ * a gate and an up projection packed by awq_pseudo_quantize_pack (same K,
+ * config and N rows each): qweight_out [2N][K/8], scales_out [G][2N],
+ * zeros_out [G][2N] (NULL iff symmetric) in 16-row tiles alternating gate,
+ * up. Copies only (cudaMemcpy2DAsync on `stream`); the outputs must not
+ * overlap the inputs. N >= 0 and N % 16 == 0; K > 0, K % group_size == 0.
+ */
+AWQ_API awq_status_t awq_interleave_gate_up(const int32_t* qweight_gate, const uint16_t* scales_gate,
+                                            const uint16_t* zeros_gate, const int32_t* qweight_up,
+                                            const uint16_t* scales_up, const uint16_t* zeros_up,
+                                            int64_t N, int64_t K, awq_qconfig_t cfg,
+                                            int32_t* qweight_out, uint16_t* scales_out,
+                                            uint16_t* zeros_out, void* stream);
 
 /*
  * awq_device_error -- read and clear the device-side error word of the

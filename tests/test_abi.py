@@ -41,7 +41,8 @@ def cfg(g=128, zp=1, flags=0):
 def test_header_declares_the_entry_points():
     syms = declared_symbols()
     for s in ["awq_pseudo_quantize_pack", "awq_dequant", "awq_gemv", "awq_gemm",
-              "awq_workspace_bytes", "awq_status_string", "awq_abi_version", "awq_device_error"]:
+              "awq_workspace_bytes", "awq_status_string", "awq_abi_version", "awq_device_error",
+              "awq_interleave_gate_up"]:
         assert s in syms
 
 
@@ -84,9 +85,26 @@ def test_product_validation(L, entry):
     assert _gemv(L, x=MIS, entry=entry) == ALIGN
     assert _gemv(L, y=MIS, entry=entry) == ALIGN
     assert _gemv(L, N=0, entry=entry) == OK                     # empty: no work, no CUDA call
-    assert _gemv(L, c=cfg(flags=2), entry=entry) == UNSUP       # undefined flag bits
+    assert _gemv(L, c=cfg(flags=4), entry=entry) == UNSUP       # undefined flag bits
     assert _gemv(L, c=cfg(flags=0x80000000), entry=entry) == UNSUP
     assert _gemv(L, N=0, c=cfg(flags=awq.FLAG_WEIGHTS_STATIC), entry=entry) == OK
+    # the fused gate/up layout needs whole 32-row tile pairs
+    assert _gemv(L, N=48, c=cfg(flags=awq.FLAG_SILU_MUL), entry=entry) == SHAPE
+    assert _gemv(L, N=0, c=cfg(flags=awq.FLAG_SILU_MUL), entry=entry) == OK
+
+
+def test_interleave_gate_up_validation(L):
+    f = L.awq_interleave_gate_up
+    P = ctypes.c_void_p
+    ok6 = [P(A)] * 6
+    # every case below is rejected before any CUDA call (the pointers are fake)
+    assert f(*ok6, 24, 256, cfg(), P(A), P(A), P(A), None) == SHAPE        # N % 16
+    assert f(*ok6, 32, 200, cfg(), P(A), P(A), P(A), None) == SHAPE        # K % 128
+    assert f(*ok6, 0, 256, cfg(), P(A), P(A), P(A), None) == OK            # empty
+    assert f(None, *ok6[1:], 32, 256, cfg(), P(A), P(A), P(A), None) == NULL
+    assert f(*ok6, 32, 256, cfg(), P(A), P(A), None, None) == NULL           # asym: zeros out
+    assert f(*ok6, 32, 256, cfg(zp=0), P(A), P(A), None, None) == SHAPE      # sym takes no zeros
+    assert f(*ok6, 32, 256, cfg(flags=4), P(A), P(A), P(A), None) == UNSUP
 
 
 def test_gemv_batch_range(L):

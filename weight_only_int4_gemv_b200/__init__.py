@@ -42,7 +42,7 @@ class AwqError(RuntimeError):
         self.status = status
 
 
-ABI_VERSION = 2   # awq_abi_version() of a library this binding matches
+ABI_VERSION = 3   # awq_abi_version() of a library this binding matches
 
 
 class QConfig(ctypes.Structure):
@@ -53,6 +53,7 @@ class QConfig(ctypes.Structure):
 # still running on the stream, so the GEMV may read them before the previous
 # kernel finishes (it still waits for that kernel before reading x).
 FLAG_WEIGHTS_STATIC = 1
+FLAG_SILU_MUL = 2   # rows are 16-row tiles alternating gate, up; y = silu(gate) * up, N/2 columns
 
 
 _lib = None
@@ -70,6 +71,7 @@ _SIGS = {
     "awq_gemm": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, QConfig, _P, _P, ctypes.c_size_t, _P]),
     "awq_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), _P]),
     "awq_gemv_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, QConfig, _P, _P]),
+    "awq_interleave_gate_up": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, QConfig, _P, _P, _P, _P]),
 }
 
 
@@ -160,19 +162,21 @@ def awq_dequant(qweight: torch.Tensor, scales: torch.Tensor, zeros, group_size: 
 
 
 def awq_workspace_bytes(M: int, N: int, K: int, zero_point: bool = True, group_size: int = GROUP_SIZE,
-                        device=None) -> int:
-    """Workspace bytes awq_gemv / awq_gemm need on `device` for this shape."""
+                        device=None, silu_mul: bool = False) -> int:
+    """Workspace bytes awq_gemv / awq_gemm need on `device` for this shape
+    (silu_mul: the fused gate/up layout, N = both projections' rows)."""
     n = ctypes.c_size_t(0)
     with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
-        _check("awq_workspace_bytes", lib().awq_workspace_bytes(M, N, K, _cfg(zero_point, group_size),
-                                                                ctypes.byref(n)))
+        _check("awq_workspace_bytes", lib().awq_workspace_bytes(
+            M, N, K, _cfg(zero_point, group_size, FLAG_SILU_MUL if silu_mul else 0), ctypes.byref(n)))
     return int(n.value)
 
 
-def alloc_workspace(M: int, N: int, K: int, zero_point: bool = True, device=None) -> torch.Tensor | None:
+def alloc_workspace(M: int, N: int, K: int, zero_point: bool = True, device=None,
+                    silu_mul: bool = False) -> torch.Tensor | None:
     """Zero-filled workspace for (M, N, K), or None when none is needed."""
     dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
-    nbytes = awq_workspace_bytes(M, N, K, zero_point, device=dev)
+    nbytes = awq_workspace_bytes(M, N, K, zero_point, device=dev, silu_mul=silu_mul)
     return torch.zeros(nbytes, dtype=torch.uint8, device=dev) if nbytes else None
 
 
@@ -190,7 +194,7 @@ def _product(entry: str, x, qweight, scales, zeros, workspace, out, group_size, 
                                      (zeros is not None and zeros.shape != scales.shape)):
         raise ValueError("scales / zeros must be [K/group_size, N]")
     if out is None:
-        out = torch.empty((M, N), dtype=torch.float16, device=x.device)
+        out = torch.empty((M, N // 2 if flags & FLAG_SILU_MUL else N), dtype=torch.float16, device=x.device)
     _need(out, "out", torch.float16, 2)
     ws_ptr, ws_bytes = None, 0
     if workspace is not None:
@@ -205,18 +209,24 @@ def _product(entry: str, x, qweight, scales, zeros, workspace, out, group_size, 
     return out
 
 
+def _flags(weights_static: bool = False, silu_mul: bool = False) -> int:
+    return (FLAG_WEIGHTS_STATIC if weights_static else 0) | (FLAG_SILU_MUL if silu_mul else 0)
+
+
 def awq_gemv(x, qweight, scales, zeros, workspace=None, out=None, group_size: int = GROUP_SIZE,
-             weights_static: bool = False):
+             weights_static: bool = False, silu_mul: bool = False):
     """y = x . W'^T for 1 <= M <= 16 (decode). `workspace` from alloc_workspace().
     weights_static: no work still running on the stream writes qweight, scales
     or zeros (a decode loop over loaded weights), so the kernel may start
-    streaming them before the previous kernel on the stream has finished."""
+    streaming them before the previous kernel on the stream has finished.
+    silu_mul: the weights are a fused gate/up pair (awq_interleave_gate_up);
+    y = silu(x . Wg'^T) * (x . Wu'^T), N/2 columns."""
     return _product("awq_gemv", x, qweight, scales, zeros, workspace, out, group_size,
-                    FLAG_WEIGHTS_STATIC if weights_static else 0)
+                    _flags(weights_static, silu_mul))
 
 
 def awq_gemv_noalloc(x, qweight, scales, zeros, out=None, group_size: int = GROUP_SIZE,
-                     weights_static: bool = False):
+                     weights_static: bool = False, silu_mul: bool = False):
     """awq_gemv with the library's fixed scratch array instead of a workspace,
     for callers that cannot allocate device memory when they run the layer.
     Calls on one device share the array and must not overlap on the GPU."""
@@ -230,27 +240,55 @@ def awq_gemv_noalloc(x, qweight, scales, zeros, out=None, group_size: int = GROU
     if qweight.shape[1] * 8 != K:
         raise ValueError("qweight must be [N, K/8] for x [M, K]")
     if out is None:
-        out = torch.empty((M, N), dtype=torch.float16, device=x.device)
+        out = torch.empty((M, N // 2 if silu_mul else N), dtype=torch.float16, device=x.device)
     _need(out, "out", torch.float16, 2)
     with torch.cuda.device(x.device):
         _check("awq_gemv_noalloc", lib().awq_gemv_noalloc(
             _ptr(x), _ptr(qweight), _ptr(scales), _ptr(zeros), M, N, K,
-            _cfg(zeros is not None, group_size, FLAG_WEIGHTS_STATIC if weights_static else 0),
+            _cfg(zeros is not None, group_size, _flags(weights_static, silu_mul)),
             _ptr(out), _stream(x.device)))
     return out
 
 
-def awq_gemm(x, qweight, scales, zeros, workspace=None, out=None, group_size: int = GROUP_SIZE):
-    """y = x . W'^T for any M (prefill), on the tcgen05 tensor cores."""
-    return _product("awq_gemm", x, qweight, scales, zeros, workspace, out, group_size)
+def awq_gemm(x, qweight, scales, zeros, workspace=None, out=None, group_size: int = GROUP_SIZE,
+             silu_mul: bool = False):
+    """y = x . W'^T for any M (prefill), on the tcgen05 tensor cores.
+    silu_mul: as for awq_gemv."""
+    return _product("awq_gemm", x, qweight, scales, zeros, workspace, out, group_size, _flags(False, silu_mul))
 
 
 def awq_linear(x, qweight, scales, zeros, workspace=None, out=None, group_size: int = GROUP_SIZE,
-               weights_static: bool = False):
+               weights_static: bool = False, silu_mul: bool = False):
     """The layer with the documented M threshold: awq_gemv for M <= 16, else awq_gemm."""
     entry = "awq_gemv" if x.shape[0] <= GEMV_MAX_M else "awq_gemm"
     return _product(entry, x, qweight, scales, zeros, workspace, out, group_size,
-                    FLAG_WEIGHTS_STATIC if weights_static else 0)
+                    _flags(weights_static, silu_mul))
+
+
+def awq_interleave_gate_up(qweight_gate, scales_gate, zeros_gate, qweight_up, scales_up, zeros_up,
+                           group_size: int = GROUP_SIZE):
+    """The fused gate/up weight layout (AWQ_FLAG_SILU_MUL) from two packed
+    projections of N rows each: (qweight [2N, K/8], scales [G, 2N], zeros or
+    None), 16-row tiles alternating gate, up. Device-side copies only."""
+    _need(qweight_gate, "qweight_gate", torch.int32, 2)
+    _need(qweight_up, "qweight_up", torch.int32, 2)
+    _need(scales_gate, "scales_gate", torch.float16, 2)
+    _need(scales_up, "scales_up", torch.float16, 2)
+    zp = zeros_gate is not None
+    if zp != (zeros_up is not None):
+        raise ValueError("gate and up must both have zero points or both not")
+    if qweight_gate.shape != qweight_up.shape or scales_gate.shape != scales_up.shape:
+        raise ValueError("gate and up must have the same shapes")
+    N, K = qweight_gate.shape[0], qweight_gate.shape[1] * 8
+    dev = qweight_gate.device
+    q = torch.empty((2 * N, K // 8), dtype=torch.int32, device=dev)
+    s = torch.empty((scales_gate.shape[0], 2 * N), dtype=torch.float16, device=dev)
+    z = torch.empty_like(s) if zp else None
+    with torch.cuda.device(dev):
+        _check("awq_interleave_gate_up", lib().awq_interleave_gate_up(
+            _ptr(qweight_gate), _ptr(scales_gate), _ptr(zeros_gate), _ptr(qweight_up), _ptr(scales_up),
+            _ptr(zeros_up), N, K, _cfg(zp, group_size), _ptr(q), _ptr(s), _ptr(z), _stream(dev)))
+    return q, s, z
 
 
 def awq_device_error(device=None) -> int:

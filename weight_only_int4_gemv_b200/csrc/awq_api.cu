@@ -4,7 +4,7 @@
 #include "awq_common.cuh"
 
 namespace awq {
-awq_status_t gemv_workspace_bytes(int64_t M, int64_t N, int64_t K, bool zp, size_t* bytes);
+awq_status_t gemv_workspace_bytes(int64_t M, int64_t N, int64_t K, bool zp, bool silu, size_t* bytes);
 awq_status_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, bool zp, size_t* bytes);
 }  // namespace awq
 
@@ -33,6 +33,7 @@ extern "C" awq_status_t awq_workspace_bytes(int64_t M, int64_t N, int64_t K, awq
   if (M < 0) return AWQ_ERR_SHAPE;
   *bytes = 0;
   if (M == 0 || N == 0) return AWQ_OK;
-  if (M <= 16) return gemv_workspace_bytes(M, N, K, cfg.zero_point != 0, bytes);
+  if ((cfg.flags & AWQ_FLAG_SILU_MUL) && N % 32) return AWQ_ERR_SHAPE;
+  if (M <= 16) return gemv_workspace_bytes(M, N, K, cfg.zero_point != 0, (cfg.flags & AWQ_FLAG_SILU_MUL) != 0, bytes);
   return gemm_workspace_bytes(M, N, K, cfg.zero_point != 0, bytes);
 }

@@ -20,9 +20,12 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 inline awq_status_t check_cfg(awq_qconfig_t cfg) {
   if (cfg.group_size != kGroup) return AWQ_ERR_UNSUPPORTED;
   if (cfg.zero_point != 0 && cfg.zero_point != 1) return AWQ_ERR_UNSUPPORTED;
-  if (cfg.flags & ~AWQ_FLAG_WEIGHTS_STATIC) return AWQ_ERR_UNSUPPORTED;
+  if (cfg.flags & ~(AWQ_FLAG_WEIGHTS_STATIC | AWQ_FLAG_SILU_MUL)) return AWQ_ERR_UNSUPPORTED;
   return AWQ_OK;
 }
+
+// SiLU in fp32 for the fused gate/up epilogues.
+__device__ __forceinline__ float silu_f32(float v) { return v / (1.0f + expf(-v)); }
 
 // K must hold whole groups; N >= 0. Sizes are bounded so that every row
 // offset fits comfortably in 64 bits and every per-row count in 32 bits.

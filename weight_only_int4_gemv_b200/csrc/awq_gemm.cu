@@ -151,6 +151,26 @@ __device__ __forceinline__ float4 ld_dsmem_f4(uint32_t saddr, int rank) {
   return v;
 }
 
+// Sum of the float4 at shared-memory offset `saddr` over CTAs 0 .. S-1 of
+// the cluster: all S loads in flight at once, then added in slice order (so
+// the bits do not depend on timing).
+__device__ __forceinline__ float4 sum_slices_dsmem(uint32_t saddr, int S) {
+  float4 v[kMaxSlices];
+#pragma unroll
+  for (int sl = 0; sl < kMaxSlices; ++sl)
+    if (sl < S) v[sl] = ld_dsmem_f4(saddr, sl);
+  float4 acc = v[0];
+#pragma unroll
+  for (int sl = 1; sl < kMaxSlices; ++sl)
+    if (sl < S) {
+      acc.x += v[sl].x;
+      acc.y += v[sl].y;
+      acc.z += v[sl].z;
+      acc.w += v[sl].w;
+    }
+  return acc;
+}
+
 // Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
 // 1024 bytes apart (stride byte offset), sm100 descriptor version 1.
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
@@ -214,6 +234,7 @@ struct GemmParams {
   int M, N, K, G;
   int m_tiles, n_tiles, k_blocks;
   int tile0, num_tiles;   // this launch takes tiles tile0 .. tile0 + num_tiles - 1
+  int silu;               // AWQ_FLAG_SILU_MUL: 16-channel tiles alternate gate, up; y has N / 2 columns
   int S;            // K slices per tile: 1 = persistent CTAs over whole tiles; 2, 4, 8 = one
                     // cluster of S CTAs per tile, CTA r of the cluster taking slice r
   int kb_per_unit;  // k blocks one CTA multiplies per tile (k_blocks / S)
@@ -338,7 +359,22 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         uint32_t r[32];
         tc_ld_32x32b_x32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * kAccCols + hm * BN + c * 32), r);
         const int nc = n0 + c * 32;
-        if (m < p.M && nc < p.N) {
+        if (p.silu) {
+          // columns nc .. nc+15: gate rows, nc+16 .. nc+31: the matching up rows
+          if (m < p.M && nc < p.N) {
+            uint32_t h[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float a = silu_f32(__uint_as_float(r[2 * e])) * __uint_as_float(r[16 + 2 * e]);
+              const float b = silu_f32(__uint_as_float(r[2 * e + 1])) * __uint_as_float(r[16 + 2 * e + 1]);
+              h[e] = uint32_t(__half_as_ushort(__float2half_rn(a))) |
+                     (uint32_t(__half_as_ushort(__float2half_rn(b))) << 16);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(p.y + m * (p.N / 2) + nc / 2);
+            dst[0] = make_uint4(h[0], h[1], h[2], h[3]);
+            dst[1] = make_uint4(h[4], h[5], h[6], h[7]);
+          }
+        } else if (m < p.M && nc < p.N) {
           uint32_t h[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
@@ -467,21 +503,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         const int64_t m = int64_t(m0) + hm * BMH + r;
         const int n = n0 + 4 * c4;
         if (m >= p.M || n >= p.N) continue;
-        const uint32_t off = smem_u32(part + r * kPartStride + 4 * c4);
-        // all slices' loads in flight at once, then summed in slice order
-        float4 v[kMaxSlices];
-#pragma unroll
-        for (int sl = 0; sl < kMaxSlices; ++sl)
-          if (sl < p.S) v[sl] = ld_dsmem_f4(off, sl);
-        float4 acc = v[0];
-#pragma unroll
-        for (int sl = 1; sl < kMaxSlices; ++sl)
-          if (sl < p.S) {
-            acc.x += v[sl].x;
-            acc.y += v[sl].y;
-            acc.z += v[sl].z;
-            acc.w += v[sl].w;
-          }
+        const float4 acc = sum_slices_dsmem(smem_u32(part + r * kPartStride + 4 * c4), p.S);
         const float a4[4] = {acc.x, acc.y, acc.z, acc.w};
         uint16_t* yrow = p.y + m * p.N;
         if (n + 4 <= p.N && (p.N & 3) == 0) {
@@ -539,6 +561,7 @@ extern "C" awq_status_t awq_gemm(const uint16_t* x, const int32_t* qweight,
   if (st != AWQ_OK) return st;
   if ((st = check_nk(N, K)) != AWQ_OK) return st;
   if (M < 0 || M > (int64_t(1) << 31) - 1) return AWQ_ERR_SHAPE;
+  if ((cfg.flags & AWQ_FLAG_SILU_MUL) && N % 32) return AWQ_ERR_SHAPE;
   if (M == 0 || N == 0) return AWQ_OK;
   if (!x || !qweight || !scales || !y) return AWQ_ERR_NULL;
   if (cfg.zero_point && !zeros) return AWQ_ERR_NULL;
@@ -575,6 +598,7 @@ extern "C" awq_status_t awq_gemm(const uint16_t* x, const int32_t* qweight,
     return AWQ_ERR_CUDA;
   GemmParams p;
   p.y = y;
+  p.silu = (cfg.flags & AWQ_FLAG_SILU_MUL) ? 1 : 0;
   p.scales = scales;
   p.zeros = zeros;
   p.M = int(M);
@@ -598,7 +622,7 @@ extern "C" awq_status_t awq_gemm(const uint16_t* x, const int32_t* qweight,
     q.tile0 = int(tile0);
     q.num_tiles = int(count);
     q.S = 1;
-    if (2 * count <= sms) {
+    if (2 * count <= sms && !q.silu) {   // the fused gate/up epilogue runs on whole tiles only
       int64_t best = ((count + sms - 1) / sms) * (q.k_blocks + 8);
       const int cands[3] = {2, 4, 8};
       for (int ci = 0; ci < 3; ++ci) {
@@ -655,7 +679,7 @@ extern "C" awq_status_t awq_gemm(const uint16_t* x, const int32_t* qweight,
   // finish (448 tiles on 148 SMs: 3 waves + 4 tiles). The launches write
   // disjoint tiles of y.
   const int64_t rem = tiles % sms;
-  if (tiles > sms && rem > 0 && 2 * rem <= sms) {
+  if (tiles > sms && rem > 0 && 2 * rem <= sms && !p.silu) {
     const awq_status_t st1 = launch_part(0, tiles - rem);
     if (st1 != AWQ_OK) return st1;
     return launch_part(tiles - rem, rem);

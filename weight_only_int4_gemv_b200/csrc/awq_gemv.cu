@@ -89,8 +89,10 @@ struct GemvParams {
   uint32_t* counters;    // [T], only when ks > 1
   int M, N, G;
   int T;                 // tiles of 16 output channels
+  int tpu;               // tiles per work unit: 1, or 2 (a gate tile and its up tile, AWQ_FLAG_SILU_MUL)
+  int units;             // T / tpu work units per K slice
   int ks;                // K slices (1: every CTA covers all of K)
-  int items;             // T * ks, slice-major: item i is tile i % T of slice i / T
+  int items;             // units * ks, slice-major: item i is unit i % units of slice i / units
   int stages;            // ring stages per warp
   int stage_bytes;       // codes + metadata + x slice of one unit (multiple of 128)
   int x_offset;          // offset of the x slice inside a stage
@@ -129,24 +131,28 @@ __device__ __forceinline__ void offset_tile(int g, uint32_t& a0, uint32_t& a2) {
   a2 = g == 0 ? 0x54005400u : (g == 1 ? 0x3C003C00u : 0u);
 }
 
-// A run of up to kChunkTiles consecutive tiles of one K slice inside a CTA's
-// item range, with the slice's groups [gb, ge).
+// A run of up to kChunkTiles consecutive tiles (whole units) of one K slice
+// inside a CTA's item range, with the slice's groups [gb, ge).
 struct Chunk {
   int i;       // first item
+  int nu;      // items (units)
   int tc;      // tiles
   int t0;      // first tile
   int s;       // slice
   int gb, ge;  // groups of the slice
 };
 
-__device__ __forceinline__ void load_chunk(const GemvParams& p, int ct, int i, int i_end, Chunk& c) {
+// ct: most tiles per chunk; tpu: tiles per unit (a compile-time constant at every call)
+__device__ __forceinline__ void load_chunk(const GemvParams& p, int ct, int tpu, int i, int i_end, Chunk& c) {
   c.i = i;
-  c.s = i / p.T;
-  c.t0 = i - c.s * p.T;
-  int tc = i_end - i;
-  if (tc > ct) tc = ct;
-  if (tc > p.T - c.t0) tc = p.T - c.t0;
-  c.tc = tc;
+  c.s = i / p.units;
+  const int u0 = i - c.s * p.units;
+  int nu = i_end - i;
+  if (nu > ct / tpu) nu = ct / tpu;
+  if (nu > p.units - u0) nu = p.units - u0;
+  c.nu = nu;
+  c.t0 = u0 * tpu;
+  c.tc = nu * tpu;
   c.gb = int(int64_t(p.G) * c.s / p.ks);
   c.ge = int(int64_t(p.G) * (c.s + 1) / p.ks);
 }
@@ -161,19 +167,19 @@ struct StageCursor {
   __device__ __forceinline__ bool done() const { return gbase < 0; }
 };
 
-__device__ __forceinline__ void cursor_init(const GemvParams& p, int ct, int i0, int i1, StageCursor& u) {
-  load_chunk(p, ct, i0, i1, u.c);
+__device__ __forceinline__ void cursor_init(const GemvParams& p, int ct, int tpu, int i0, int i1, StageCursor& u) {
+  load_chunk(p, ct, tpu, i0, i1, u.c);
   u.gbase = u.c.gb;
 }
 
-__device__ __forceinline__ void cursor_next(const GemvParams& p, int ct, int i_end, StageCursor& u) {
+__device__ __forceinline__ void cursor_next(const GemvParams& p, int ct, int tpu, int i_end, StageCursor& u) {
   u.gbase += kWarps;
   if (u.gbase >= u.c.ge) {
-    const int ni = u.c.i + u.c.tc;
+    const int ni = u.c.i + u.c.nu;
     if (ni >= i_end) {
       u.gbase = -1;
     } else {
-      load_chunk(p, ct, ni, i_end, u.c);
+      load_chunk(p, ct, tpu, ni, i_end, u.c);
       u.gbase = u.c.gb;
     }
   }
@@ -238,7 +244,7 @@ struct Pipe {
 // multiply into acc. All TC tile slots are computed, so the unrolled loops
 // carry no branches; in a chunk with fewer tiles the extra slots hold stale
 // shared memory and their rows are never stored.
-template <int MT, bool ZP, int TC>
+template <int MT, bool ZP, int TC, int TPU>
 __device__ __forceinline__ void chunk_stages(const GemvParams& p, Pipe<MT>& pp, const Chunk& cc,
                                              float (&acc)[kChunkTiles][MT][4], volatile int* abort_flag) {
     for (int gbase = cc.gb; gbase < cc.ge; gbase += kWarps) {
@@ -288,7 +294,7 @@ __device__ __forceinline__ void chunk_stages(const GemvParams& p, Pipe<MT>& pp, 
             pp.fills[pp.slot] += 1u;
           }
         }
-        cursor_next(p, TC, pp.i1, pp.pc);
+        cursor_next(p, TC, TPU, pp.i1, pp.pc);
       }
 
       if (has) {
@@ -352,13 +358,15 @@ __device__ __forceinline__ void chunk_stages(const GemvParams& p, Pipe<MT>& pp, 
 
 }
 
-// One CTA's work: items [i0, i1) in chunks of at most TC tiles.
-template <int MT, bool ZP, int TC>
+// One CTA's work: items [i0, i1) in chunks of at most TC tiles. SILU: the
+// fused gate/up epilogue (AWQ_FLAG_SILU_MUL; units are tile pairs).
+template <int MT, bool ZP, int TC, bool SILU>
 __device__ __forceinline__ void gemv_cta(const CUtensorMap& tmap_q, const CUtensorMap& tmap_x,
                                          const CUtensorMap& tmap_s, const CUtensorMap& tmap_z,
                                          const CodeMaps& code_maps, const GemvParams& p, const int i0,
                                          const int i1) {
   extern __shared__ __align__(1024) uint8_t gemv_smem[];
+  constexpr int TPU = SILU ? 2 : 1;   // tiles per work unit
 
   const int lane = threadIdx.x & 31;
   const int w = threadIdx.x >> 5;
@@ -387,14 +395,14 @@ __device__ __forceinline__ void gemv_cta(const CUtensorMap& tmap_q, const CUtens
 
   // ---- the first S stages (weights possibly before the dependency wait)
   StageCursor pc;   // lane 0 of every warp: the stage S ahead of the arithmetic
-  if (lane == 0) cursor_init(p, TC, i0, i1, pc);
+  if (lane == 0) cursor_init(p, TC, TPU, i0, i1, pc);
   if (threadIdx.x == 0) {
     if (p.early) {
       StageCursor u = pc;
       for (int s = 0; s < S && !u.done(); ++s) {
         mbar_arrive_expect_tx(&full[s], stage_tx_bytes(p, u.c.tc, ZP));
         issue_weights<ZP>(u, ring + s * p.stage_bytes, &full[s], &tmap_q, &tmap_s, &tmap_z, p.scale_offset, p.codes4d ? &code_maps : nullptr);
-        cursor_next(p, TC, i1, u);
+        cursor_next(p, TC, TPU, i1, u);
       }
     } else {
       tma_prefetch_l2_3d(&tmap_q, 0, pc.c.t0 * kTile, pc.gbase);
@@ -412,7 +420,7 @@ __device__ __forceinline__ void gemv_cta(const CUtensorMap& tmap_q, const CUtens
         tma_load_3d(st + p.x_offset, &tmap_x, 0, pc.gbase, 0, &full[s]);
         fills[s] = 1u;
       }
-      cursor_next(p, TC, i1, pc);
+      cursor_next(p, TC, TPU, i1, pc);
     }
   }
 
@@ -449,7 +457,7 @@ __device__ __forceinline__ void gemv_cta(const CUtensorMap& tmap_q, const CUtens
   offset_tile(g, pp.ca0, pp.ca2);
 
   Chunk cc;
-  load_chunk(p, TC, i0, i1, cc);
+  load_chunk(p, TC, TPU, i0, i1, cc);
   for (int chunk = 0;; ++chunk) {
     const int tc = cc.tc;
     float acc[kChunkTiles][MT][4];
@@ -460,7 +468,7 @@ __device__ __forceinline__ void gemv_cta(const CUtensorMap& tmap_q, const CUtens
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[rt][mt][i] = 0.0f;
 
-    chunk_stages<MT, ZP, TC>(p, pp, cc, acc, &abort_flag);
+    chunk_stages<MT, ZP, TC, TPU>(p, pp, cc, acc, &abort_flag);
 
     // ---- chunk reduction: the 8 warps' partial sums meet in shared memory
     // ([warp][row][m], double-buffered by chunk parity) and are summed in
@@ -484,53 +492,88 @@ __device__ __forceinline__ void gemv_cta(const CUtensorMap& tmap_q, const CUtens
         }
       }
     named_barrier_sync(kReduceBarrier, kThreads);
-    const int V = kTile * tc * M;
     const float* pb0 = pbuf + (chunk & 1) * kWarps * (kChunkRows * M);
     const int64_t row0 = int64_t(cc.t0) * kTile;
-    for (int v = threadIdx.x; v < V; v += kThreads) {
-      float sum = 0.0f;
+    if (TPU == 1 || p.ks > 1) {
+      const int V = kTile * tc * M;
+      for (int v = threadIdx.x; v < V; v += kThreads) {
+        float sum = 0.0f;
 #pragma unroll
-      for (int ww = 0; ww < kWarps; ++ww) sum += pb0[ww * (kChunkRows * M) + v];
-      const int row = v / M;
-      const int m = v - row * M;
-      if (p.ks == 1) {
-        if (row0 + row < p.N) p.y[int64_t(m) * p.N + row0 + row] = __half_as_ushort(__float2half_rn(sum));
-      } else {
-        __stcg(p.partials + ((int64_t(cc.s) * p.T * kTile + row0 + row) * M + m), sum);
+        for (int ww = 0; ww < kWarps; ++ww) sum += pb0[ww * (kChunkRows * M) + v];
+        const int row = v / M;
+        const int m = v - row * M;
+        if (p.ks == 1) {
+          if (row0 + row < p.N) p.y[int64_t(m) * p.N + row0 + row] = __half_as_ushort(__float2half_rn(sum));
+        } else {
+          __stcg(p.partials + ((int64_t(cc.s) * p.T * kTile + row0 + row) * M + m), sum);
+        }
+      }
+    } else if constexpr (SILU) {
+      // fused gate/up: tile 2q of the chunk holds gate rows, tile 2q + 1 the
+      // matching up rows; y has N / 2 columns
+      const int V = kTile * (tc / 2) * M;
+      for (int v = threadIdx.x; v < V; v += kThreads) {
+        const int q = v / (kTile * M);
+        const int rem = v - q * (kTile * M);   // row * M + m inside the pair
+        const int vg = 2 * q * kTile * M + rem;
+        float g = 0.0f, u = 0.0f;
+#pragma unroll
+        for (int ww = 0; ww < kWarps; ++ww) {
+          g += pb0[ww * (kChunkRows * M) + vg];
+          u += pb0[ww * (kChunkRows * M) + vg + kTile * M];
+        }
+        const int row = rem / M;
+        const int m = rem - row * M;
+        p.y[int64_t(m) * (p.N / 2) + row0 / 2 + q * kTile + row] =
+            __half_as_ushort(__float2half_rn(silu_f32(g) * u));
       }
     }
     if (p.ks > 1) {
-      // Slices of a tile meet in the workspace: the CTA that brings a tile's
+      // Slices of a unit meet in the workspace: the CTA that brings a unit's
       // arrival count to ks sums the ks partials in slice order.
       __threadfence();
       named_barrier_sync(kReduceBarrier, kThreads);
-      if (w < tc) {
-        const int tile = cc.t0 + w;
+      if (w < cc.nu) {
+        const int unit = cc.t0 / TPU + w;
         uint32_t last = 0;
         if (lane == 0) {
           uint32_t old;
           asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
-                       : "=r"(old) : "l"(p.counters + tile) : "memory");
+                       : "=r"(old) : "l"(p.counters + unit) : "memory");
           last = (old + 1 == uint32_t(p.ks)) ? 1u : 0u;
         }
         last = __shfl_sync(0xffffffffu, last, 0);
         if (last) {
-          const int64_t trow = int64_t(tile) * kTile;
-          for (int v = lane; v < kTile * M; v += 32) {
-            float sum = 0.0f;
-            for (int s = 0; s < p.ks; ++s)
-              sum += __ldcg(p.partials + ((int64_t(s) * p.T * kTile + trow) * M + v));
-            const int row = v / M;
-            const int m = v - row * M;
-            if (trow + row < p.N) p.y[int64_t(m) * p.N + trow + row] = __half_as_ushort(__float2half_rn(sum));
+          const int64_t trow = int64_t(unit) * TPU * kTile;
+          if constexpr (TPU == 1) {
+            for (int v = lane; v < kTile * M; v += 32) {
+              float sum = 0.0f;
+              for (int s = 0; s < p.ks; ++s)
+                sum += __ldcg(p.partials + ((int64_t(s) * p.T * kTile + trow) * M + v));
+              const int row = v / M;
+              const int m = v - row * M;
+              if (trow + row < p.N) p.y[int64_t(m) * p.N + trow + row] = __half_as_ushort(__float2half_rn(sum));
+            }
+          } else if constexpr (SILU) {
+            for (int v = lane; v < kTile * M; v += 32) {
+              float g = 0.0f, u = 0.0f;
+              for (int s = 0; s < p.ks; ++s) {
+                const float* ps = p.partials + (int64_t(s) * p.T * kTile + trow) * M;
+                g += __ldcg(ps + v);
+                u += __ldcg(ps + kTile * M + v);
+              }
+              const int row = v / M;
+              const int m = v - row * M;
+              p.y[int64_t(m) * (p.N / 2) + trow / 2 + row] = __half_as_ushort(__float2half_rn(silu_f32(g) * u));
+            }
           }
-          if (lane == 0) p.counters[tile] = 0u;
+          if (lane == 0) p.counters[unit] = 0u;
         }
       }
     }
-    const int ni = cc.i + cc.tc;
+    const int ni = cc.i + cc.nu;
     if (ni >= i1) break;
-    load_chunk(p, TC, ni, i1, cc);
+    load_chunk(p, TC, TPU, ni, i1, cc);
   }
 
   // If a warp gave up, copies may still be in flight: a slot is refilled
@@ -543,7 +586,7 @@ __device__ __forceinline__ void gemv_cta(const CUtensorMap& tmap_q, const CUtens
   }
 }
 
-template <int MT, bool ZP, int TC>
+template <int MT, bool ZP, int TC, bool SILU>
 __global__ void __launch_bounds__(kThreads, MT == 1 ? 2 : 1)
 gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_x,
             const __grid_constant__ CUtensorMap tmap_s, const __grid_constant__ CUtensorMap tmap_z,
@@ -558,13 +601,13 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
   // padding a 4-tile chunk (896 tiles on 296 CTAs: 288 CTAs hold 3). The
   // arithmetic of the stream phase is the limit, and the two CTAs of an SM
   // share it, so an SM with 3 + 4 tiles finishes sooner than with 4 + 4.
-  if constexpr (TC == 4) {
-    if (i1 - i0 == 3 && i0 / p.T == (i1 - 1) / p.T) {
-      gemv_cta<MT, ZP, 3>(tmap_q, tmap_x, tmap_s, tmap_z, code_maps, p, i0, i1);
+  if constexpr (TC == 4 && !SILU) {
+    if (i1 - i0 == 3 && i0 / p.units == (i1 - 1) / p.units) {
+      gemv_cta<MT, ZP, 3, false>(tmap_q, tmap_x, tmap_s, tmap_z, code_maps, p, i0, i1);
       return;
     }
   }
-  gemv_cta<MT, ZP, TC>(tmap_q, tmap_x, tmap_s, tmap_z, code_maps, p, i0, i1);
+  gemv_cta<MT, ZP, TC, SILU>(tmap_q, tmap_x, tmap_s, tmap_z, code_maps, p, i0, i1);
 }
 
 // ---------------------------------------------------------------------------
@@ -578,24 +621,28 @@ struct Variant {
   int mt, id;
 };
 
-constexpr int kNumVariants = 8;
+constexpr int kNumVariants = 16;
 constexpr int kSmemBudget = 232448;   // largest dynamic shared memory of one sm_100 CTA
 constexpr int kHalfSmBudget = 115712; // half of an SM's 228 KB, less the 1 KB reserved per CTA
 
-Variant pick_variant(int64_t M, bool zp, int tc) {
+Variant pick_variant(int64_t M, bool zp, int tc, bool silu) {
   static const Variant table[kNumVariants] = {
-      {gemv_kernel<1, true, 4>, 1, 0},  {gemv_kernel<1, false, 4>, 1, 1},
-      {gemv_kernel<2, true, 4>, 2, 2},  {gemv_kernel<2, false, 4>, 2, 3},
-      {gemv_kernel<1, true, 2>, 1, 4},  {gemv_kernel<1, false, 2>, 1, 5},
-      {gemv_kernel<2, true, 2>, 2, 6},  {gemv_kernel<2, false, 2>, 2, 7}};
-  return table[(tc == 2 ? 4 : 0) + (M <= 8 ? 0 : 2) + (zp ? 0 : 1)];
+      {gemv_kernel<1, true, 4, false>, 1, 0},  {gemv_kernel<1, false, 4, false>, 1, 1},
+      {gemv_kernel<2, true, 4, false>, 2, 2},  {gemv_kernel<2, false, 4, false>, 2, 3},
+      {gemv_kernel<1, true, 2, false>, 1, 4},  {gemv_kernel<1, false, 2, false>, 1, 5},
+      {gemv_kernel<2, true, 2, false>, 2, 6},  {gemv_kernel<2, false, 2, false>, 2, 7},
+      {gemv_kernel<1, true, 4, true>, 1, 8},   {gemv_kernel<1, false, 4, true>, 1, 9},
+      {gemv_kernel<2, true, 4, true>, 2, 10},  {gemv_kernel<2, false, 4, true>, 2, 11},
+      {gemv_kernel<1, true, 2, true>, 1, 12},  {gemv_kernel<1, false, 2, true>, 1, 13},
+      {gemv_kernel<2, true, 2, true>, 2, 14},  {gemv_kernel<2, false, 2, true>, 2, 15}};
+  return table[(silu ? 8 : 0) + (tc == 2 ? 4 : 0) + (M <= 8 ? 0 : 2) + (zp ? 0 : 1)];
 }
 
 int round128(int v) { return (v + 127) / 128 * 128; }
 
 struct Plan {
   Variant v;
-  int grid, T, ks, items, tc, scale_offset;
+  int grid, T, tpu, units, ks, items, tc, scale_offset;
   int stages, stage_bytes, x_offset, pbuf_offset, smem;
   size_t counter_bytes, partial_bytes;
 };
@@ -604,7 +651,7 @@ constexpr int kMaxDevices = 64;
 std::atomic<int> g_sm_count[kMaxDevices];
 std::atomic<int> g_smem_attr[kMaxDevices][kNumVariants];
 
-awq_status_t make_plan(int64_t M, int64_t N, int64_t K, bool zp, Plan& pl) {
+awq_status_t make_plan(int64_t M, int64_t N, int64_t K, bool zp, bool silu, Plan& pl) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return AWQ_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return AWQ_ERR_UNSUPPORTED;
@@ -620,22 +667,26 @@ awq_status_t make_plan(int64_t M, int64_t N, int64_t K, bool zp, Plan& pl) {
   // cut into slices only when there are fewer tiles than CTAs.
   const int64_t G = K / kGroup;
   const int64_t T = (N + kTile - 1) / kTile;
+  const int tpu = silu ? 2 : 1;          // a fused gate/up unit is a gate tile and its up tile
+  const int64_t U = T / tpu;
   const int pbuf_bytes = 2 * kWarps * kChunkRows * int(M) * 4;
   for (int per_sm = M <= 8 ? 2 : 1;; --per_sm) {
     const int64_t want = int64_t(per_sm) * sms;
     int64_t ks = 1;
-    if (T < want) {
-      ks = (want + T - 1) / T;
+    if (U < want) {
+      ks = (want + U - 1) / U;
       if (ks > G) ks = G;
     }
     pl.T = int(T);
+    pl.tpu = tpu;
+    pl.units = int(U);
     pl.ks = int(ks);
-    pl.items = int(T * ks);
+    pl.items = int(U * ks);
     pl.grid = int(pl.items < want ? pl.items : want);
     // Chunks of 4 tiles, or of 2 when no CTA has more than 2 items: the CTA
     // with the most items sets the kernel's time, and it then wastes no slot.
     const int64_t most = (int64_t(pl.items) + pl.grid - 1) / pl.grid;
-    pl.tc = most <= 2 ? 2 : kChunkTiles;
+    pl.tc = most * tpu <= 2 ? 2 : kChunkTiles;
     // Ring geometry: as many stages as the budget holds after the reduction buffers.
     pl.scale_offset = pl.tc * kTileStageBytes;
     pl.x_offset = pl.scale_offset + kMetaStageBytes * (zp ? 2 : 1);
@@ -646,7 +697,7 @@ awq_status_t make_plan(int64_t M, int64_t N, int64_t K, bool zp, Plan& pl) {
     if (pl.stages >= 2 || per_sm == 1) break;
   }
   if (pl.stages < 2) return AWQ_ERR_UNSUPPORTED;
-  pl.v = pick_variant(M, zp, pl.tc);
+  pl.v = pick_variant(M, zp, pl.tc, silu);
   if (!g_smem_attr[dev][pl.v.id].load(std::memory_order_acquire)) {
     if (cudaFuncSetAttribute(pl.v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBudget) != cudaSuccess)
       return AWQ_ERR_CUDA;
@@ -667,6 +718,7 @@ awq_status_t check_gemv_args(const uint16_t* x, const int32_t* qweight, const ui
   if ((st = check_nk(N, K)) != AWQ_OK) return st;
   if (M < 1 || M > 16) return AWQ_ERR_SHAPE;
   if (N % 8) return AWQ_ERR_SHAPE;
+  if ((cfg.flags & AWQ_FLAG_SILU_MUL) && N % 32) return AWQ_ERR_SHAPE;
   if (N == 0) return AWQ_OK;
   if (!x || !qweight || !scales || !y) return AWQ_ERR_NULL;
   if (cfg.zero_point && !zeros) return AWQ_ERR_NULL;
@@ -680,10 +732,10 @@ awq_status_t check_gemv_args(const uint16_t* x, const int32_t* qweight, const ui
 }  // namespace
 
 // Workspace bytes of the GEMV for (M, N, K); used by awq_workspace_bytes.
-awq_status_t gemv_workspace_bytes(int64_t M, int64_t N, int64_t K, bool zp, size_t* bytes) {
+awq_status_t gemv_workspace_bytes(int64_t M, int64_t N, int64_t K, bool zp, bool silu, size_t* bytes) {
   if (N == 0) { *bytes = 0; return AWQ_OK; }
   Plan pl;
-  awq_status_t st = make_plan(M, N, K, zp, pl);
+  awq_status_t st = make_plan(M, N, K, zp, silu, pl);
   if (st != AWQ_OK) return st;
   *bytes = pl.counter_bytes + pl.partial_bytes;
   return AWQ_OK;
@@ -714,7 +766,7 @@ extern "C" awq_status_t awq_gemv(const uint16_t* x, const int32_t* qweight,
   if (st != AWQ_OK || N == 0) return st;
   const bool zp = cfg.zero_point != 0;
   Plan pl;
-  if ((st = make_plan(M, N, K, zp, pl)) != AWQ_OK) return st;
+  if ((st = make_plan(M, N, K, zp, (cfg.flags & AWQ_FLAG_SILU_MUL) != 0, pl)) != AWQ_OK) return st;
   GemvParams p;
   p.y = y;
   p.counters = nullptr;
@@ -762,6 +814,8 @@ extern "C" awq_status_t awq_gemv(const uint16_t* x, const int32_t* qweight,
   p.N = int(N);
   p.G = G;
   p.T = pl.T;
+  p.tpu = pl.tpu;
+  p.units = pl.units;
   p.ks = pl.ks;
   p.items = pl.items;
   p.stages = pl.stages;
@@ -830,7 +884,8 @@ extern "C" awq_status_t awq_gemv_noalloc(const uint16_t* x, const int32_t* qweig
   awq_status_t st = check_gemv_args(x, qweight, scales, zeros, M, N, K, cfg, y);
   if (st != AWQ_OK || N == 0) return st;
   Plan pl;
-  if ((st = make_plan(M, N, K, cfg.zero_point != 0, pl)) != AWQ_OK) return st;
+  if ((st = make_plan(M, N, K, cfg.zero_point != 0, (cfg.flags & AWQ_FLAG_SILU_MUL) != 0, pl)) != AWQ_OK)
+    return st;
   const size_t need = pl.partial_bytes ? pl.counter_bytes + pl.partial_bytes : 0;
   if (need > kStaticScratchBytes) return AWQ_ERR_WORKSPACE;
   int dev = 0;

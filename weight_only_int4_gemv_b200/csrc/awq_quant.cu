@@ -177,3 +177,43 @@ extern "C" awq_status_t awq_dequant(const int32_t* qweight, const uint16_t* scal
     dequant_kernel<false><<<grid, 256, 0, s>>>(qweight, scales, nullptr, N, K, W_out);
   return launch_status();
 }
+
+// The AWQ_FLAG_SILU_MUL layout from a gate and an up projection: 16-row tiles
+// alternating gate, up, in qweight rows and in the N columns of the
+// group-major scales and zero points ("AutoAWQ" code tour, "The Quantization
+// Flow Up Close": gate and up merged into one MLP block). Plain 2-D copies.
+extern "C" awq_status_t awq_interleave_gate_up(const int32_t* qweight_gate, const uint16_t* scales_gate,
+                                               const uint16_t* zeros_gate, const int32_t* qweight_up,
+                                               const uint16_t* scales_up, const uint16_t* zeros_up, int64_t N,
+                                               int64_t K, awq_qconfig_t cfg, int32_t* qweight_out,
+                                               uint16_t* scales_out, uint16_t* zeros_out, void* stream) {
+  awq_status_t st = check_cfg(cfg);
+  if (st != AWQ_OK) return st;
+  if ((st = check_nk(N, K)) != AWQ_OK) return st;
+  if (N % 16) return AWQ_ERR_SHAPE;
+  if (N == 0) return AWQ_OK;
+  if (!qweight_gate || !scales_gate || !qweight_up || !scales_up || !qweight_out || !scales_out)
+    return AWQ_ERR_NULL;
+  if (cfg.zero_point && (!zeros_gate || !zeros_up || !zeros_out)) return AWQ_ERR_NULL;
+  if (!cfg.zero_point && (zeros_gate || zeros_up || zeros_out)) return AWQ_ERR_SHAPE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t tile_bytes = size_t(16) * size_t(K / 8) * 4;   // one 16-row tile of qweight
+  const size_t tiles = size_t(N / 16);
+  const size_t runs = size_t(K / kGroup) * tiles;               // 16-value runs of a [G][N] array
+  char* qo = reinterpret_cast<char*>(qweight_out);
+  if (cudaMemcpy2DAsync(qo, 2 * tile_bytes, qweight_gate, tile_bytes, tile_bytes, tiles,
+                        cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
+      cudaMemcpy2DAsync(qo + tile_bytes, 2 * tile_bytes, qweight_up, tile_bytes, tile_bytes, tiles,
+                        cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    return AWQ_ERR_CUDA;
+  const uint16_t* src_g[2] = {scales_gate, zeros_gate};
+  const uint16_t* src_u[2] = {scales_up, zeros_up};
+  uint16_t* dst[2] = {scales_out, zeros_out};
+  for (int a = 0; a < (cfg.zero_point ? 2 : 1); ++a) {
+    char* d = reinterpret_cast<char*>(dst[a]);
+    if (cudaMemcpy2DAsync(d, 64, src_g[a], 32, 32, runs, cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
+        cudaMemcpy2DAsync(d + 32, 64, src_u[a], 32, 32, runs, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+      return AWQ_ERR_CUDA;
+  }
+  return launch_status();
+}
