@@ -564,13 +564,16 @@ def run_table(args):
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
     hbm_peak, tc_peak, _, peak_src = measured_peaks()
-    cases = [((4096, 4096), (1, 2, 4, 8, 16, 128, 512, 2048)),
-             ((14336, 4096), (1, 2, 4, 8, 16, 128, 512, 2048)),
-             ((4096, 14336), (1, 2, 4, 8, 16)),
-             ((8192, 8192), (1, 8, 2048)), ((28672, 8192), (1, 8, 2048)), ((8192, 28672), (1, 8, 2048))]
+    # (N, K), batch sizes, fused gate/up (AWQ_FLAG_SILU_MUL: N = gate + up rows, y has N / 2 columns)
+    cases = [((4096, 4096), (1, 2, 4, 8, 16, 128, 512, 2048), False),
+             ((14336, 4096), (1, 2, 4, 8, 16, 128, 512, 2048), False),
+             ((28672, 4096), (1, 4, 16, 128, 2048), True),
+             ((4096, 14336), (1, 2, 4, 8, 16), False),
+             ((8192, 8192), (1, 8, 2048), False), ((28672, 8192), (1, 8, 2048), False),
+             ((8192, 28672), (1, 8, 2048), False)]
     l2_bytes = 126 << 20
     rng = np.random.default_rng(3)
-    for (N, K), Ms in cases:
+    for (N, K), Ms, silu in cases:
         q, s, z = [torch.from_numpy(a).to(device) for a in make_packed_random(N, K, 128, True, seed=1)]
         wbytes = N * K // 2 + 4 * N * (K // 128)
         copies = max(2, -(-2 * l2_bytes // wbytes))
@@ -578,11 +581,13 @@ def run_table(args):
         del q, s, z
         for M in Ms:
             x = torch.from_numpy(rng.standard_normal((M, K), dtype=np.float32).astype(np.float16)).to(device)
-            y = torch.empty((M, N), dtype=torch.float16, device=device)
-            entry = "awq_gemv" if M <= awq.GEMV_MAX_M else "awq_gemm"
+            y = torch.empty((M, N // 2 if silu else N), dtype=torch.float16, device=device)
+            entry = ("awq_gemv" if M <= awq.GEMV_MAX_M else "awq_gemm") + (" silu_mul" if silu else "")
             fn = awq.awq_gemv if M <= awq.GEMV_MAX_M else awq.awq_gemm
             kw = {"weights_static": True} if M <= awq.GEMV_MAX_M else {}
-            ws = awq.alloc_workspace(M, N, K, True, device=device)
+            if silu:
+                kw["silu_mul"] = True
+            ws = awq.alloc_workspace(M, N, K, True, device=device, silu_mul=silu)
             stream = torch.cuda.Stream(device)
             with torch.cuda.stream(stream):
                 for qq, ss, zz in packs:
@@ -603,7 +608,7 @@ def run_table(args):
                 e1.record()
                 torch.cuda.synchronize(device)
             us = e0.elapsed_time(e1) * 1e3 / (reps * copies)
-            gbs = algo_bytes(M, N, K) / (us * 1e-6) / 1e9
+            gbs = (algo_bytes(M, N, K) - (M * N if silu else 0)) / (us * 1e-6) / 1e9   # y: N/2 columns
             tfl = algo_flops(M, N, K) / (us * 1e-6) / 1e12
             print(json.dumps({"entry": entry, "N": N, "K": K, "M": M, "us": round(us, 3), "GB/s": round(gbs, 1),
                               "frac_hbm": round(gbs / hbm_peak, 4), "TFLOP/s": round(tfl, 2),

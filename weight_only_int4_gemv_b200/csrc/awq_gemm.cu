@@ -240,7 +240,7 @@ struct GemmParams {
   int kb_per_unit;  // k blocks one CTA multiplies per tile (k_blocks / S)
 };
 
-template <bool ZP>
+template <bool ZP, bool SILU>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_q,
             const GemmParams p) {
@@ -359,7 +359,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         uint32_t r[32];
         tc_ld_32x32b_x32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * kAccCols + hm * BN + c * 32), r);
         const int nc = n0 + c * 32;
-        if (p.silu) {
+        if constexpr (SILU) {
           // columns nc .. nc+15: gate rows, nc+16 .. nc+31: the matching up rows
           if (m < p.M && nc < p.N) {
             uint32_t h[8];
@@ -374,7 +374,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
             dst[0] = make_uint4(h[0], h[1], h[2], h[3]);
             dst[1] = make_uint4(h[4], h[5], h[6], h[7]);
           }
-        } else if (m < p.M && nc < p.N) {
+        } else if (m < p.M && nc < p.N) {   // (an else of the constexpr if: plain kernels only)
           uint32_t h[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
@@ -497,6 +497,26 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         }
       }
       cluster_sync_all();
+      if constexpr (SILU) {
+        // output quad j of a row: pair q = j / 4 (gate columns 32q .. 32q+15,
+        // up columns 32q+16 .. 32q+31 of the tile), columns 4 (j % 4) .. + 3
+        for (int idx = threadIdx.x; idx < rows_per * (BN / 8); idx += kGemmThreads) {
+          const int r = rank * rows_per + idx / (BN / 8);
+          const int j = idx % (BN / 8);
+          const int gc = 32 * (j >> 2) + 4 * (j & 3);
+          const int64_t m = int64_t(m0) + hm * BMH + r;
+          if (m >= p.M || n0 + gc >= p.N) continue;
+          const uint32_t offg = smem_u32(part + r * kPartStride + gc);
+          const float4 g = sum_slices_dsmem(offg, p.S);
+          const float4 u = sum_slices_dsmem(offg + 16 * 4, p.S);
+          const uint32_t lo = uint32_t(__half_as_ushort(__float2half_rn(silu_f32(g.x) * u.x))) |
+                              (uint32_t(__half_as_ushort(__float2half_rn(silu_f32(g.y) * u.y))) << 16);
+          const uint32_t hi = uint32_t(__half_as_ushort(__float2half_rn(silu_f32(g.z) * u.z))) |
+                              (uint32_t(__half_as_ushort(__float2half_rn(silu_f32(g.w) * u.w))) << 16);
+          *reinterpret_cast<uint2*>(p.y + m * (p.N / 2) + n0 / 2 + 16 * (j >> 2) + 4 * (j & 3)) =
+              make_uint2(lo, hi);
+        }
+      } else {
       for (int idx = threadIdx.x; idx < rows_per * (BN / 4); idx += kGemmThreads) {
         const int r = rank * rows_per + idx / (BN / 4);
         const int c4 = idx % (BN / 4);
@@ -516,6 +536,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
           for (int e = 0; e < 4 && n + e < p.N; ++e) yrow[n + e] = __half_as_ushort(__float2half_rn(a4[e]));
         }
       }
+      }
       cluster_sync_all();
     }
   }
@@ -534,9 +555,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
 // ---------------------------------------------------------------------------
 constexpr int kMaxDevices = 64;
 std::atomic<int> g_sms[kMaxDevices];
-std::atomic<int> g_attr_set[kMaxDevices][2];
+std::atomic<int> g_attr_set[kMaxDevices][4];   // [zero point + 2 * fused]
 // clusters of 2, 4, 8 CTAs that fit at once: 0 = not queried yet, -1 = none, else the count
-std::atomic<int> g_clusters[kMaxDevices][2][3];
+std::atomic<int> g_clusters[kMaxDevices][4][3];
 
 }  // namespace
 
@@ -579,8 +600,10 @@ extern "C" awq_status_t awq_gemm(const uint16_t* x, const int32_t* qweight,
       return AWQ_ERR_CUDA;
     g_sms[dev].store(sms, std::memory_order_relaxed);
   }
-  auto kernel = cfg.zero_point ? gemm_kernel<true> : gemm_kernel<false>;
-  const int zi = cfg.zero_point ? 1 : 0;
+  const bool silu = (cfg.flags & AWQ_FLAG_SILU_MUL) != 0;
+  auto kernel = cfg.zero_point ? (silu ? gemm_kernel<true, true> : gemm_kernel<true, false>)
+                               : (silu ? gemm_kernel<false, true> : gemm_kernel<false, false>);
+  const int zi = (cfg.zero_point ? 1 : 0) + (silu ? 2 : 0);
   if (!g_attr_set[dev][zi].load(std::memory_order_acquire)) {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
         cudaSuccess)
@@ -622,7 +645,7 @@ extern "C" awq_status_t awq_gemm(const uint16_t* x, const int32_t* qweight,
     q.tile0 = int(tile0);
     q.num_tiles = int(count);
     q.S = 1;
-    if (2 * count <= sms && !q.silu) {   // the fused gate/up epilogue runs on whole tiles only
+    if (2 * count <= sms) {
       int64_t best = ((count + sms - 1) / sms) * (q.k_blocks + 8);
       const int cands[3] = {2, 4, 8};
       for (int ci = 0; ci < 3; ++ci) {
@@ -679,7 +702,7 @@ extern "C" awq_status_t awq_gemm(const uint16_t* x, const int32_t* qweight,
   // finish (448 tiles on 148 SMs: 3 waves + 4 tiles). The launches write
   // disjoint tiles of y.
   const int64_t rem = tiles % sms;
-  if (tiles > sms && rem > 0 && 2 * rem <= sms && !p.silu) {
+  if (tiles > sms && rem > 0 && 2 * rem <= sms) {
     const awq_status_t st1 = launch_part(0, tiles - rem);
     if (st1 != AWQ_OK) return st1;
     return launch_part(tiles - rem, rem);
