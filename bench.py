@@ -568,6 +568,8 @@ def run_table(args):
     cases = [((4096, 4096), (1, 2, 4, 8, 16, 128, 512, 2048), False),
              ((14336, 4096), (1, 2, 4, 8, 16, 128, 512, 2048), False),
              ((28672, 4096), (1, 4, 16, 128, 2048), True),
+             ((6144, 4096), (1, 4, 16), False),     # q, k, v of Llama-3-8B concatenated
+             ((1024, 4096), (1, 4, 16), False),     # k or v alone
              ((4096, 14336), (1, 2, 4, 8, 16), False),
              ((8192, 8192), (1, 8, 2048), False), ((28672, 8192), (1, 8, 2048), False),
              ((8192, 28672), (1, 8, 2048), False)]

@@ -251,6 +251,24 @@ AWQ_API awq_status_t awq_interleave_gate_up(const int32_t* qweight_gate, const u
                                             uint16_t* zeros_out, void* stream);
 
 /*
+ * awq_concat_rows -- concatenate `parts` packed projections that share K and
+ * config along N ("AutoAWQ" code tour, "The Quantization Flow Up Close": the
+ * fuser concatenates the q, k and v projections through fuse_qkv), so one
+ * awq_gemv / awq_gemm computes all of them: part p's rows follow those of
+ * parts 0 .. p-1 in qweight_out [sum N][K/8], and its columns those of parts
+ * 0 .. p-1 in scales_out / zeros_out [G][sum N] (zeros NULL iff symmetric,
+ * for every part). qweights / scales / zeros are arrays of `parts` device
+ * pointers (zeros may be NULL when symmetric), Ns their row counts (host
+ * memory, read before the call returns). Copies only (cudaMemcpy2DAsync on
+ * `stream`); outputs must not overlap inputs. 1 <= parts <= 16, every
+ * N_p >= 0, K > 0, K % group_size == 0.
+ */
+AWQ_API awq_status_t awq_concat_rows(int parts, const int32_t* const* qweights, const uint16_t* const* scales,
+                                     const uint16_t* const* zeros, const int64_t* Ns, int64_t K,
+                                     awq_qconfig_t cfg, int32_t* qweight_out, uint16_t* scales_out,
+                                     uint16_t* zeros_out, void* stream);
+
+/*
  * awq_device_error -- read and clear the device-side error word of the
  * current device (synchronizes `stream`). Bit 0: a pipeline wait inside
  * awq_gemm passed its time limit (2 s) and the kernel abandoned its tiles;

@@ -42,7 +42,7 @@ def test_header_declares_the_entry_points():
     syms = declared_symbols()
     for s in ["awq_pseudo_quantize_pack", "awq_dequant", "awq_gemv", "awq_gemm",
               "awq_workspace_bytes", "awq_status_string", "awq_abi_version", "awq_device_error",
-              "awq_interleave_gate_up"]:
+              "awq_interleave_gate_up", "awq_concat_rows"]:
         assert s in syms
 
 
@@ -91,6 +91,26 @@ def test_product_validation(L, entry):
     # the fused gate/up layout needs whole 32-row tile pairs
     assert _gemv(L, N=48, c=cfg(flags=awq.FLAG_SILU_MUL), entry=entry) == SHAPE
     assert _gemv(L, N=0, c=cfg(flags=awq.FLAG_SILU_MUL), entry=entry) == OK
+
+
+def test_concat_rows_validation(L):
+    f = L.awq_concat_rows
+    P = ctypes.c_void_p
+    ptrs = (P * 2)(A, A)
+    Ns = (ctypes.c_int64 * 2)(16, 32)
+    # every case below is rejected before any CUDA call (the pointers are fake)
+    assert f(0, ptrs, ptrs, ptrs, Ns, 256, cfg(), P(A), P(A), P(A), None) == SHAPE       # no parts
+    assert f(17, ptrs, ptrs, ptrs, Ns, 256, cfg(), P(A), P(A), P(A), None) == SHAPE      # too many
+    assert f(2, ptrs, ptrs, ptrs, Ns, 200, cfg(), P(A), P(A), P(A), None) == SHAPE       # K % 128
+    assert f(2, None, ptrs, ptrs, Ns, 256, cfg(), P(A), P(A), P(A), None) == NULL
+    assert f(2, ptrs, ptrs, None, Ns, 256, cfg(), P(A), P(A), P(A), None) == NULL        # asym needs zeros
+    assert f(2, ptrs, ptrs, ptrs, Ns, 256, cfg(), P(A), P(A), None, None) == NULL        # zeros out
+    assert f(2, ptrs, ptrs, ptrs, Ns, 256, cfg(zp=0), P(A), P(A), None, None) == SHAPE   # sym: no zeros
+    assert f(2, ptrs, ptrs, ptrs, Ns, 256, cfg(flags=4), P(A), P(A), P(A), None) == UNSUP
+    zero = (ctypes.c_int64 * 2)(0, 0)
+    assert f(2, ptrs, ptrs, ptrs, zero, 256, cfg(), P(A), P(A), P(A), None) == OK       # empty
+    neg = (ctypes.c_int64 * 2)(16, -1)
+    assert f(2, ptrs, ptrs, ptrs, neg, 256, cfg(), P(A), P(A), P(A), None) == SHAPE
 
 
 def test_interleave_gate_up_validation(L):

@@ -122,3 +122,30 @@ def test_silu_mul_matches_separate_products_then_silu():
     h = host(awq.awq_gemv(x, q, s, z, silu_mul=True)).astype(np.float64)
     ref = O.gate_up_silu_f64(host(x), *[oracle_layer(N, K, 0.02, 0.0, True, sd)[4] for sd in (0, 1)])
     assert_close(h, ref, "fused vs oracle")
+
+
+@pytest.mark.parametrize("zp", [True, False])
+def test_concat_rows_is_the_concatenation(zp):
+    shapes = [(256, 512), (64, 512), (96, 512)]
+    parts = [oracle_layer(n, k, 0.02, 0.0, zp, i) for i, (n, k) in enumerate(shapes)]
+    q, s, z = awq.awq_concat_rows([(dev(p[1]), dev(p[2]), dev(p[3]) if zp else None) for p in parts])
+    assert np.array_equal(bits(q), bits(np.concatenate([p[1] for p in parts], axis=0)))
+    assert np.array_equal(bits(s), bits(np.concatenate([p[2] for p in parts], axis=1)))
+    if zp:
+        assert np.array_equal(bits(z), bits(np.concatenate([p[3] for p in parts], axis=1)))
+    else:
+        assert z is None
+
+
+def test_gemv_on_concatenated_qkv():
+    """Llama-3-8B q, k, v (4096 + 1024 + 1024 rows, K = 4096) as one GEMV: every
+    output equals the oracle's product with the concatenated W'."""
+    K = 4096
+    parts = [oracle_layer(n, K, 0.02, 0.0, True, i) for i, n in enumerate((4096, 1024, 1024))]
+    q, s, z = awq.awq_concat_rows([(dev(p[1]), dev(p[2]), dev(p[3])) for p in parts])
+    Wd = np.concatenate([p[4] for p in parts], axis=0)
+    for M in (1, 5):
+        x = activations(M, K, seed=90 + M)
+        ws = awq.alloc_workspace(M, 6144, K, True)
+        y = host(awq.awq_gemv(dev(x), q, s, z, workspace=ws))
+        assert_close(y, O.matmul_f64(x, Wd), f"qkv M={M}")

@@ -72,6 +72,8 @@ _SIGS = {
     "awq_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), _P]),
     "awq_gemv_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, QConfig, _P, _P]),
     "awq_interleave_gate_up": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, QConfig, _P, _P, _P, _P]),
+    "awq_concat_rows": (ctypes.c_int, [ctypes.c_int, ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.POINTER(_P),
+                                       ctypes.POINTER(_I64), _I64, QConfig, _P, _P, _P, _P]),
 }
 
 
@@ -298,3 +300,35 @@ def awq_device_error(device=None) -> int:
     with torch.cuda.device(dev):
         _check("awq_device_error", lib().awq_device_error(ctypes.byref(v), _stream(dev)))
     return int(v.value)
+
+
+def awq_concat_rows(parts, group_size: int = GROUP_SIZE):
+    """Concatenate packed projections [(qweight, scales, zeros or None), ...]
+    sharing K along N (q, k and v into one layer): returns (qweight
+    [sum N, K/8], scales [G, sum N], zeros or None). Device-side copies only."""
+    parts = list(parts)
+    if not parts:
+        raise ValueError("no parts")
+    zp = parts[0][2] is not None
+    K = parts[0][0].shape[1] * 8
+    for q, s, z in parts:
+        _need(q, "qweight", torch.int32, 2)
+        _need(s, "scales", torch.float16, 2)
+        if (z is not None) != zp:
+            raise ValueError("all parts must have zero points or none")
+        if q.shape[1] * 8 != K:
+            raise ValueError("all parts must share K")
+    n = len(parts)
+    Ns = (_I64 * n)(*[q.shape[0] for q, _, _ in parts])
+    qs = (_P * n)(*[q.data_ptr() for q, _, _ in parts])
+    ss = (_P * n)(*[s.data_ptr() for _, s, _ in parts])
+    zs = (_P * n)(*[(z.data_ptr() if z is not None else None) for _, _, z in parts])
+    total = sum(Ns)
+    dev = parts[0][0].device
+    q = torch.empty((total, K // 8), dtype=torch.int32, device=dev)
+    s = torch.empty((parts[0][1].shape[0], total), dtype=torch.float16, device=dev)
+    z = torch.empty_like(s) if zp else None
+    with torch.cuda.device(dev):
+        _check("awq_concat_rows", lib().awq_concat_rows(n, qs, ss, zs, Ns, K, _cfg(zp, group_size),
+                                                        _ptr(q), _ptr(s), _ptr(z), _stream(dev)))
+    return q, s, z

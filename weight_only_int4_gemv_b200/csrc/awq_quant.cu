@@ -217,3 +217,51 @@ extern "C" awq_status_t awq_interleave_gate_up(const int32_t* qweight_gate, cons
   }
   return launch_status();
 }
+
+// Projections sharing K concatenated along N (the fuser's fuse_qkv, "AutoAWQ"
+// code tour, "The Quantization Flow Up Close"). Plain 2-D copies.
+extern "C" awq_status_t awq_concat_rows(int parts, const int32_t* const* qweights, const uint16_t* const* scales,
+                                        const uint16_t* const* zeros, const int64_t* Ns, int64_t K,
+                                        awq_qconfig_t cfg, int32_t* qweight_out, uint16_t* scales_out,
+                                        uint16_t* zeros_out, void* stream) {
+  awq_status_t st = check_cfg(cfg);
+  if (st != AWQ_OK) return st;
+  if (parts < 1 || parts > 16) return AWQ_ERR_SHAPE;
+  if (!qweights || !scales || !Ns || (cfg.zero_point && !zeros)) return AWQ_ERR_NULL;
+  int64_t total = 0;
+  for (int i = 0; i < parts; ++i) {
+    if ((st = check_nk(Ns[i], K)) != AWQ_OK) return st;
+    total += Ns[i];
+  }
+  if ((st = check_nk(total, K)) != AWQ_OK) return st;
+  if (total == 0) return AWQ_OK;
+  if (!qweight_out || !scales_out) return AWQ_ERR_NULL;
+  if (cfg.zero_point && !zeros_out) return AWQ_ERR_NULL;
+  if (!cfg.zero_point && zeros_out) return AWQ_ERR_SHAPE;
+  for (int i = 0; i < parts; ++i) {
+    if (Ns[i] == 0) continue;
+    if (!qweights[i] || !scales[i]) return AWQ_ERR_NULL;
+    if (cfg.zero_point && !zeros[i]) return AWQ_ERR_NULL;
+    if (!cfg.zero_point && zeros && zeros[i]) return AWQ_ERR_SHAPE;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t row_bytes = size_t(K / 8) * 4;
+  const size_t G = size_t(K / kGroup);
+  int64_t off = 0;
+  for (int i = 0; i < parts; ++i) {
+    const int64_t n = Ns[i];
+    if (n == 0) continue;
+    if (cudaMemcpyAsync(reinterpret_cast<char*>(qweight_out) + size_t(off) * row_bytes, qweights[i],
+                        size_t(n) * row_bytes, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+      return AWQ_ERR_CUDA;
+    for (int a = 0; a < (cfg.zero_point ? 2 : 1); ++a) {
+      const uint16_t* src = a == 0 ? scales[i] : zeros[i];
+      uint16_t* dst = (a == 0 ? scales_out : zeros_out) + off;
+      if (cudaMemcpy2DAsync(dst, size_t(total) * 2, src, size_t(n) * 2, size_t(n) * 2, G,
+                            cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+        return AWQ_ERR_CUDA;
+    }
+    off += n;
+  }
+  return launch_status();
+}
