@@ -266,3 +266,77 @@ def interleave_gate_up(a_gate: np.ndarray, a_up: np.ndarray, axis: int = 0) -> n
         out[2 * j * TILE_ROWS:(2 * j + 1) * TILE_ROWS] = a_gate[j * TILE_ROWS:(j + 1) * TILE_ROWS]
         out[(2 * j + 1) * TILE_ROWS:(2 * j + 2) * TILE_ROWS] = a_up[j * TILE_ROWS:(j + 1) * TILE_ROWS]
     return np.moveaxis(out, 0, axis)
+
+
+# ---------------------------------------------------------------------------
+# Activation-aware scale search ("AutoAWQ" code tour, "The Quantization Flow
+# Up Close": the search computes a per-channel mean of normalized weights and
+# a float32 mean of activations, runs the fp16 module once as the reference,
+# and picks the candidate scaling with the lowest output error; "From Install
+# to Your First Model": duo_scaling uses both the weight and the activation
+# statistics; "The big picture": dividing an input channel of x by s and
+# multiplying the matching weight column by s leaves the output unchanged).
+#
+# Readings (the pages give no formula or grid):
+# * candidates s(alpha) = mean|x|^alpha / (mean|w^|^(1 - alpha) + 1e-4) with
+#   duo scaling, mean|x|^alpha without, for alpha = i / n_grid, i = 0 ..
+#   n_grid - 1; each floored at 1e-4 and divided by sqrt(max(s) * min(s)) so
+#   the scaled weights stay in fp16 range;
+# * w^ = |w| / (max |w| over its group of 128 in the same row), 0 for an
+#   all-zero group; mean|w^| is over the N rows;
+# * all of the statistics and candidate arithmetic in fp32;
+# * error = mean over outputs of (y_ref - y)^2, y_ref = fp16(x . W^T) (the
+#   fp16 module), y = fp16((x / s) . Q(W diag(s))'^T), x / s and W diag(s)
+#   rounded to fp16;
+# * the first minimum wins a tie.
+# ---------------------------------------------------------------------------
+SCALE_EPS = np.float32(1e-4)
+
+
+def act_mean_abs(X: np.ndarray) -> np.ndarray:
+    """mean over rows of |x[m, k]|, fp32 [K]."""
+    return np.abs(np.asarray(X).astype(np.float32)).mean(axis=0, dtype=np.float32)
+
+
+def weight_norm_mean(W: np.ndarray, group_size: int = GROUP_SIZE) -> np.ndarray:
+    """mean over rows n of |w[n, k]| / max|w[n, group of k]|, fp32 [K]."""
+    A = np.abs(_groups_f32(W, group_size))                    # [N, G, g]
+    mx = A.max(axis=2, keepdims=True)
+    Wn = np.divide(A, mx, out=np.zeros_like(A), where=mx > 0)
+    N, G, g = Wn.shape
+    return Wn.reshape(N, G * g).mean(axis=0, dtype=np.float32)
+
+
+def candidate_scales(x_mean: np.ndarray, w_mean: np.ndarray, alpha: float, duo: bool = True) -> np.ndarray:
+    """The scale vector of one grid point, fp32 [K]."""
+    a = np.float32(alpha)
+    s = np.power(x_mean.astype(np.float32), a)
+    if duo:
+        s = s / (np.power(w_mean.astype(np.float32), np.float32(1.0) - a) + SCALE_EPS)
+    s = np.maximum(s.astype(np.float32), SCALE_EPS)
+    return (s / np.sqrt(s.max() * s.min())).astype(np.float32)
+
+
+def scaled_output(W: np.ndarray, X: np.ndarray, s: np.ndarray, group_size: int = GROUP_SIZE,
+                  zero_point: bool = True) -> np.ndarray:
+    """fp16((x / s) . Q(W diag(s))'^T): the quantized module with the scale
+    folded into its weights and divided out of its input."""
+    s = s.astype(np.float32)
+    Ws = (np.asarray(W).astype(np.float32) * s[None, :]).astype(np.float16)
+    Xs = (np.asarray(X).astype(np.float32) / s[None, :]).astype(np.float16)
+    codes, sc, z = pseudo_quantize(Ws, group_size, zero_point)
+    return matmul_f64(Xs, dequant(codes, sc, z, group_size)).astype(np.float16)
+
+
+def search_scale(W: np.ndarray, X: np.ndarray, group_size: int = GROUP_SIZE, zero_point: bool = True,
+                 n_grid: int = 20, duo: bool = True):
+    """(best scales fp32 [K], losses [n_grid] float64, best index)."""
+    y_ref = matmul_f64(X, W).astype(np.float16).astype(np.float64)
+    x_mean, w_mean = act_mean_abs(X), weight_norm_mean(W, group_size)
+    losses = np.empty(n_grid)
+    for i in range(n_grid):
+        s = candidate_scales(x_mean, w_mean, i / n_grid, duo)
+        y = scaled_output(W, X, s, group_size, zero_point).astype(np.float64)
+        losses[i] = np.mean((y_ref - y) ** 2)
+    best = int(np.argmin(losses))
+    return candidate_scales(x_mean, w_mean, best / n_grid, duo), losses, best
