@@ -63,7 +63,7 @@
 extern "C" {
 #endif
 
-#define AWQ_ABI_VERSION 3
+#define AWQ_ABI_VERSION 4
 
 #if defined(__GNUC__)
 #define AWQ_API __attribute__((visibility("default")))
@@ -267,6 +267,43 @@ AWQ_API awq_status_t awq_concat_rows(int parts, const int32_t* const* qweights, 
                                      const uint16_t* const* zeros, const int64_t* Ns, int64_t K,
                                      awq_qconfig_t cfg, int32_t* qweight_out, uint16_t* scales_out,
                                      uint16_t* zeros_out, void* stream);
+
+/*
+ * awq_search_scale -- activation-aware per-input-channel scale search.
+ * ("AutoAWQ" code tour, "The Quantization Flow Up Close": a per-channel mean
+ * of normalized weights and a float32 mean of activations, the fp16 module
+ * run once as the reference, the candidate scaling with the lowest output
+ * error kept; "From Install to Your First Model": duo_scaling.)
+ * With x_mean[k] = mean_m |X[m][k]| and w_mean[k] = mean_n |W[n][k]| /
+ * max|W[n][group of k]| (fp32), grid point i (alpha = i / n_grid) tries
+ *   s = max(x_mean^alpha / (w_mean^(1 - alpha) + 1e-4), 1e-4)  (duo != 0)
+ *   s = max(x_mean^alpha, 1e-4)                                 (duo == 0)
+ * divided by sqrt(max s * min s); its loss is the mean over outputs of
+ * (fp16(X . W^T) - fp16((X / s) . Q(W diag(s))'^T))^2, Q the quantizer of
+ * awq_pseudo_quantize_pack and the product that of awq_gemv / awq_gemm,
+ * X / s and W diag(s) rounded to fp16. losses_out [n_grid] (device fp32)
+ * receives the losses, scales_out [K] (device fp32) the scales of the first
+ * minimum. To use them: quantize W diag(s) (awq_apply_scale, then
+ * awq_pseudo_quantize_pack) and divide the layer's input by s upstream.
+ * W [N][K], X [Ms][K] fp16 device; N >= 1, N % 8 == 0, K % group_size == 0,
+ * 1 <= Ms <= 2^24, 1 <= n_grid <= 64, cfg.flags == 0.
+ * workspace: awq_search_scale_workspace_bytes(N, K, Ms, cfg) bytes of device
+ * memory, 16-byte aligned, contents irrelevant. Stream-ordered, no host
+ * synchronization; same inputs give the same bits.
+ */
+AWQ_API awq_status_t awq_search_scale_workspace_bytes(int64_t N, int64_t K, int64_t Ms, awq_qconfig_t cfg,
+                                                      size_t* bytes);
+AWQ_API awq_status_t awq_search_scale(const uint16_t* W, int64_t N, int64_t K, const uint16_t* X, int64_t Ms,
+                                      awq_qconfig_t cfg, int n_grid, int duo, float* scales_out,
+                                      float* losses_out, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * awq_apply_scale -- W_out[n][k] = fp16(W[n][k] * s[k]) (fp32 product, one
+ * rounding): the weights of a layer whose input will be divided by s.
+ * W, W_out [N][K] fp16 device, s [K] fp32 device. N >= 0, K > 0.
+ */
+AWQ_API awq_status_t awq_apply_scale(const uint16_t* W, const float* s, int64_t N, int64_t K, uint16_t* W_out,
+                                     void* stream);
 
 /*
  * awq_device_error -- read and clear the device-side error word of the

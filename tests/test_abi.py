@@ -42,7 +42,8 @@ def test_header_declares_the_entry_points():
     syms = declared_symbols()
     for s in ["awq_pseudo_quantize_pack", "awq_dequant", "awq_gemv", "awq_gemm",
               "awq_workspace_bytes", "awq_status_string", "awq_abi_version", "awq_device_error",
-              "awq_interleave_gate_up", "awq_concat_rows"]:
+              "awq_interleave_gate_up", "awq_concat_rows", "awq_search_scale",
+              "awq_search_scale_workspace_bytes", "awq_apply_scale"]:
         assert s in syms
 
 
@@ -111,6 +112,34 @@ def test_concat_rows_validation(L):
     assert f(2, ptrs, ptrs, ptrs, zero, 256, cfg(), P(A), P(A), P(A), None) == OK       # empty
     neg = (ctypes.c_int64 * 2)(16, -1)
     assert f(2, ptrs, ptrs, ptrs, neg, 256, cfg(), P(A), P(A), P(A), None) == SHAPE
+
+
+def test_search_scale_validation(L):
+    P = ctypes.c_void_p
+    n = ctypes.c_size_t(0)
+    ws = L.awq_search_scale_workspace_bytes
+    assert ws(64, 256, 8, cfg(), None) == NULL
+    assert ws(60, 256, 8, cfg(), ctypes.byref(n)) == SHAPE          # N % 8
+    assert ws(64, 200, 8, cfg(), ctypes.byref(n)) == SHAPE          # K % 128
+    assert ws(64, 256, 0, cfg(), ctypes.byref(n)) == SHAPE          # no calibration rows
+    assert ws(64, 256, 8, cfg(flags=1), ctypes.byref(n)) == UNSUP    # no flags
+    # the size depends on the device's SM count: without a GPU the query reports CUDA
+    st = ws(64, 256, 8, cfg(), ctypes.byref(n))
+    assert st in (OK, CUDA) and (st == CUDA or n.value > 0)
+    f = L.awq_search_scale
+    big = 1 << 30
+    # every case below is rejected before any CUDA call (the pointers are fake)
+    assert f(P(A), 64, 256, P(A), 8, cfg(), 0, 1, P(A), P(A), P(A), big, None) == SHAPE      # n_grid
+    assert f(P(A), 64, 256, P(A), 8, cfg(), 65, 1, P(A), P(A), P(A), big, None) == SHAPE
+    assert f(None, 64, 256, P(A), 8, cfg(), 10, 1, P(A), P(A), P(A), big, None) == NULL
+    assert f(P(A), 64, 256, P(A), 8, cfg(), 10, 1, P(A), P(A), None, big, None) == NULL
+    assert f(P(MIS), 64, 256, P(A), 8, cfg(), 10, 1, P(A), P(A), P(A), big, None) == ALIGN
+    if st == OK:   # (on a GPU machine) a workspace one short of the need is refused before any launch
+        assert f(P(A), 64, 256, P(A), 8, cfg(), 10, 1, P(A), P(A), P(A), n.value - 16, None) == WS
+    ap = L.awq_apply_scale
+    assert ap(P(A), P(A), 0, 256, P(A), None) == OK
+    assert ap(None, P(A), 8, 256, P(A), None) == NULL
+    assert ap(P(A), P(A), -1, 256, P(A), None) == SHAPE
 
 
 def test_interleave_gate_up_validation(L):

@@ -42,7 +42,7 @@ class AwqError(RuntimeError):
         self.status = status
 
 
-ABI_VERSION = 3   # awq_abi_version() of a library this binding matches
+ABI_VERSION = 4   # awq_abi_version() of a library this binding matches
 
 
 class QConfig(ctypes.Structure):
@@ -74,6 +74,10 @@ _SIGS = {
     "awq_interleave_gate_up": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, QConfig, _P, _P, _P, _P]),
     "awq_concat_rows": (ctypes.c_int, [ctypes.c_int, ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.POINTER(_P),
                                        ctypes.POINTER(_I64), _I64, QConfig, _P, _P, _P, _P]),
+    "awq_search_scale_workspace_bytes": (ctypes.c_int, [_I64, _I64, _I64, QConfig, ctypes.POINTER(ctypes.c_size_t)]),
+    "awq_search_scale": (ctypes.c_int, [_P, _I64, _I64, _P, _I64, QConfig, ctypes.c_int, ctypes.c_int, _P, _P, _P,
+                                        ctypes.c_size_t, _P]),
+    "awq_apply_scale": (ctypes.c_int, [_P, _P, _I64, _I64, _P, _P]),
 }
 
 
@@ -332,3 +336,42 @@ def awq_concat_rows(parts, group_size: int = GROUP_SIZE):
         _check("awq_concat_rows", lib().awq_concat_rows(n, qs, ss, zs, Ns, K, _cfg(zp, group_size),
                                                         _ptr(q), _ptr(s), _ptr(z), _stream(dev)))
     return q, s, z
+
+
+def awq_search_scale(W: torch.Tensor, X: torch.Tensor, zero_point: bool = True, n_grid: int = 20,
+                     duo: bool = True, group_size: int = GROUP_SIZE):
+    """Activation-aware scale search for the layer W [N, K] on calibration
+    inputs X [Ms, K]: returns (scales fp32 [K] of the lowest-error grid point,
+    losses fp32 [n_grid]). All on the device (see awq.h)."""
+    _need(W, "W", torch.float16, 2)
+    _need(X, "X", torch.float16, 2)
+    N, K = W.shape
+    Ms = X.shape[0]
+    if X.shape[1] != K:
+        raise ValueError("X must be [Ms, K] for W [N, K]")
+    cfg = _cfg(zero_point, group_size)
+    n = ctypes.c_size_t(0)
+    with torch.cuda.device(W.device):
+        _check("awq_search_scale_workspace_bytes",
+               lib().awq_search_scale_workspace_bytes(N, K, Ms, cfg, ctypes.byref(n)))
+        ws = torch.empty(n.value, dtype=torch.uint8, device=W.device)
+        scales = torch.empty(K, dtype=torch.float32, device=W.device)
+        losses = torch.empty(n_grid, dtype=torch.float32, device=W.device)
+        _check("awq_search_scale", lib().awq_search_scale(
+            _ptr(W), N, K, _ptr(X), Ms, cfg, n_grid, 1 if duo else 0, _ptr(scales), _ptr(losses), _ptr(ws),
+            n.value, _stream(W.device)))
+    return scales, losses
+
+
+def awq_apply_scale(W: torch.Tensor, scales: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """fp16(W[n, k] * s[k]): the weights of a layer whose input is divided by s."""
+    _need(W, "W", torch.float16, 2)
+    _need(scales, "scales", torch.float32, 1)
+    N, K = W.shape
+    if scales.shape[0] != K:
+        raise ValueError("scales must be [K]")
+    if out is None:
+        out = torch.empty_like(W)
+    with torch.cuda.device(W.device):
+        _check("awq_apply_scale", lib().awq_apply_scale(_ptr(W), _ptr(scales), N, K, _ptr(out), _stream(W.device)))
+    return out
