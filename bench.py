@@ -375,8 +375,10 @@ def run_native(args, dist):
     e2e = run_e2e(awq, torch, device, stream, layers, shapes, M, args, dist, step_bytes)
 
     gemm = None
+    search = None
     if ws_ == 1 and not args.no_gemm:
         gemm = run_gemm_prefill(awq, torch, device, tc_peak, peak_src, args)
+        search = run_scale_search(awq, torch, device)
 
     cpu = None
     if ws_ == 1 and rank == 0 and not args.no_cpu:
@@ -429,6 +431,8 @@ def run_native(args, dist):
         }
         if gemm is not None:
             line["prefill_gemm"] = gemm
+        if search is not None:
+            line["scale_search"] = search
         print(json.dumps(line), flush=True)
 
 
@@ -471,6 +475,29 @@ def run_e2e(awq, torch, device, stream, layers, shapes, M, args, dist, step_byte
             "d2h_bytes_per_step": d2h, "steps": steps,
             "note": "effective HBM GB/s of the same algorithmic bytes, time includes the copies and a "
                     "host synchronize per step"}
+
+
+def run_scale_search(awq, torch, device):
+    """awq_search_scale on gate_proj 14336x4096 with 512 calibration tokens
+    (the pages' max_calib_seq_len) of synthetic activations whose 1 % salient
+    channels are 10x larger, a 20-point grid: one warm call, device time."""
+    N, K, Ms, n_grid = 14336, 4096, 512, 20
+    W = torch.from_numpy(make_weight(N, K, 0.02, 0.0, seed=0)).to(device)
+    rng = np.random.default_rng(2)
+    X = rng.standard_normal((Ms, K), dtype=np.float32)
+    X[:, rng.choice(K, K // 100, replace=False)] *= 10.0
+    X = torch.from_numpy(X.astype(np.float16)).to(device)
+    awq.awq_search_scale(W, X, n_grid=n_grid)
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    _, losses = awq.awq_search_scale(W, X, n_grid=n_grid)
+    e1.record()
+    torch.cuda.synchronize(device)
+    losses = losses.cpu().numpy().astype(np.float64)
+    best = int(np.argmin(losses))
+    return {"workload": "gate_proj 14336x4096, 512 calibration tokens, 20 grid points", "ms": round(e0.elapsed_time(e1), 3),
+            "best_alpha": best / n_grid, "loss_best_over_alpha0": round(float(losses[best] / losses[0]), 4)}
 
 
 def run_gemm_prefill(awq, torch, device, tc_peak, peak_src, args):
