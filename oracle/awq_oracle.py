@@ -340,3 +340,44 @@ def search_scale(W: np.ndarray, X: np.ndarray, group_size: int = GROUP_SIZE, zer
         losses[i] = np.mean((y_ref - y) ** 2)
     best = int(np.argmin(losses))
     return candidate_scales(x_mean, w_mean, best / n_grid, duo), losses, best
+
+
+# ---------------------------------------------------------------------------
+# Clip search ("AutoAWQ" code tour, "The Quantization Flow Up Close": the
+# clipping pass shrinks extreme values group by group where that lowers the
+# output error; apply_clip switches it). Readings (the pages give no grid or
+# criterion formula):
+# * ratio grid r_i = 1 - max_shrink * i / n_grid, i = 0 .. n_grid - 1;
+# * a group of row n is clipped to [-t, t], t = r * max|w| of the group (fp32),
+#   and the clipped values rounded to fp16, then quantized as usual;
+# * error of (row n, group j) = sum over calibration rows m of
+#   (x[m, group j] . (w - w'))^2 = d^T (X_j^T X_j) d, d = w - w' in float64;
+# * per (row, group) the first ratio with the lowest error wins.
+# ---------------------------------------------------------------------------
+def clip_groups(W: np.ndarray, ratios: np.ndarray, group_size: int = GROUP_SIZE) -> np.ndarray:
+    """fp16 W clipped per (row, group) to [-t, t], t = ratio * max|w| of the
+    group; ratios [G, N] (group-major, as the scales)."""
+    A = _groups_f32(W, group_size)                                   # [N, G, g]
+    t = np.abs(A).max(axis=2) * np.asarray(ratios, np.float32).T     # [N, G] fp32
+    C = np.clip(A, -t[:, :, None], t[:, :, None]).astype(np.float16)
+    return C.reshape(np.asarray(W).shape)
+
+
+def search_clip(W: np.ndarray, X: np.ndarray, group_size: int = GROUP_SIZE, zero_point: bool = True,
+                n_grid: int = 20, max_shrink: float = 0.5):
+    """(best ratios fp32 [G, N], errors float64 [n_grid, G, N])."""
+    N, K = np.asarray(W).shape
+    G = K // group_size
+    Xg = np.asarray(X).astype(np.float64).reshape(-1, G, group_size)
+    gram = np.einsum("mja,mjb->jab", Xg, Xg)                         # [G, g, g]
+    Wf = np.asarray(W).astype(np.float64).reshape(N, G, group_size)
+    errs = np.empty((n_grid, G, N))
+    for i in range(n_grid):
+        r = np.float32(1.0) - np.float32(max_shrink) * np.float32(i) / np.float32(n_grid)
+        Wc = clip_groups(W, np.full((G, N), r, np.float32), group_size)
+        codes, sc, z = pseudo_quantize(Wc, group_size, zero_point)
+        D = Wf - dequant(codes, sc, z, group_size).astype(np.float64).reshape(N, G, group_size)
+        errs[i] = np.einsum("nja,jab,njb->jn", D, gram, D)
+    best = np.argmin(errs, axis=0)                                    # first minimum
+    ratios = (np.float32(1.0) - np.float32(max_shrink) * best.astype(np.float32) / np.float32(n_grid))
+    return ratios.astype(np.float32), errs
