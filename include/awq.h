@@ -63,7 +63,7 @@
 extern "C" {
 #endif
 
-#define AWQ_ABI_VERSION 4
+#define AWQ_ABI_VERSION 5
 
 #if defined(__GNUC__)
 #define AWQ_API __attribute__((visibility("default")))
@@ -304,6 +304,37 @@ AWQ_API awq_status_t awq_search_scale(const uint16_t* W, int64_t N, int64_t K, c
  */
 AWQ_API awq_status_t awq_apply_scale(const uint16_t* W, const float* s, int64_t N, int64_t K, uint16_t* W_out,
                                      void* stream);
+
+/*
+ * awq_search_clip -- per (row, group) clipping-ratio search.
+ * ("AutoAWQ" code tour, "The Quantization Flow Up Close": the clipping pass
+ * shrinks extreme weights group by group where that lowers the output error;
+ * apply_clip switches it.) For row n and group j, grid point i tries
+ * r = 1 - max_shrink * i / n_grid (fp32): the group is clipped to [-t, t],
+ * t = r * max|w| of the group (fp32), the values rounded to fp16 and
+ * quantized as by awq_pseudo_quantize_pack; the error is d^T G_j d with
+ * d = w - w' (fp32) and G_j = X_j^T X_j (fp32) the Gram matrix of the
+ * calibration inputs over the group's input channels. ratios_out [G][N]
+ * (device fp32, group-major like the scales) receives the first ratio with
+ * the lowest error. To use them: awq_apply_clip, then
+ * awq_pseudo_quantize_pack. W [N][K], X [Ms][K] fp16 device; N >= 1,
+ * N % 8 == 0, K % group_size == 0, 1 <= Ms <= 2^24, 1 <= n_grid <= 64,
+ * 0 <= max_shrink < 1, cfg.flags == 0. workspace:
+ * awq_search_clip_workspace_bytes(K) bytes (the Gram matrices), 16-byte
+ * aligned, contents irrelevant. Stream-ordered; same inputs, same bits.
+ */
+AWQ_API awq_status_t awq_search_clip_workspace_bytes(int64_t K, size_t* bytes);
+AWQ_API awq_status_t awq_search_clip(const uint16_t* W, int64_t N, int64_t K, const uint16_t* X, int64_t Ms,
+                                     awq_qconfig_t cfg, int n_grid, float max_shrink, float* ratios_out,
+                                     void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * awq_apply_clip -- W_out = W with each (row n, group j) clipped to [-t, t],
+ * t = ratios[j][n] * max|w| of the group (fp32), rounded to fp16.
+ * W, W_out [N][K] fp16 device (16-byte aligned), ratios [G][N] fp32 device.
+ */
+AWQ_API awq_status_t awq_apply_clip(const uint16_t* W, const float* ratios, int64_t N, int64_t K,
+                                    uint16_t* W_out, void* stream);
 
 /*
  * awq_device_error -- read and clear the device-side error word of the

@@ -43,7 +43,8 @@ def test_header_declares_the_entry_points():
     for s in ["awq_pseudo_quantize_pack", "awq_dequant", "awq_gemv", "awq_gemm",
               "awq_workspace_bytes", "awq_status_string", "awq_abi_version", "awq_device_error",
               "awq_interleave_gate_up", "awq_concat_rows", "awq_search_scale",
-              "awq_search_scale_workspace_bytes", "awq_apply_scale"]:
+              "awq_search_scale_workspace_bytes", "awq_apply_scale", "awq_search_clip",
+              "awq_search_clip_workspace_bytes", "awq_apply_clip"]:
         assert s in syms
 
 
@@ -140,6 +141,27 @@ def test_search_scale_validation(L):
     assert ap(P(A), P(A), 0, 256, P(A), None) == OK
     assert ap(None, P(A), 8, 256, P(A), None) == NULL
     assert ap(P(A), P(A), -1, 256, P(A), None) == SHAPE
+
+
+def test_search_clip_validation(L):
+    P = ctypes.c_void_p
+    n = ctypes.c_size_t(0)
+    assert L.awq_search_clip_workspace_bytes(200, ctypes.byref(n)) == SHAPE
+    assert L.awq_search_clip_workspace_bytes(256, ctypes.byref(n)) == OK and n.value == 2 * 128 * 128 * 4
+    f = L.awq_search_clip
+    big = 1 << 30
+    # every case below is rejected before any CUDA call (the pointers are fake)
+    assert f(P(A), 64, 256, P(A), 8, cfg(), 0, ctypes.c_float(0.5), P(A), P(A), big, None) == SHAPE
+    assert f(P(A), 64, 256, P(A), 8, cfg(), 10, ctypes.c_float(1.0), P(A), P(A), big, None) == SHAPE
+    assert f(P(A), 64, 256, P(A), 8, cfg(), 10, ctypes.c_float(-0.1), P(A), P(A), big, None) == SHAPE
+    assert f(P(A), 60, 256, P(A), 8, cfg(), 10, ctypes.c_float(0.5), P(A), P(A), big, None) == SHAPE
+    assert f(None, 64, 256, P(A), 8, cfg(), 10, ctypes.c_float(0.5), P(A), P(A), big, None) == NULL
+    assert f(P(A), 64, 256, P(A), 8, cfg(), 10, ctypes.c_float(0.5), P(A), P(A), n.value - 4, None) == WS
+    assert f(P(A), 64, 256, P(A), 8, cfg(flags=2), 10, ctypes.c_float(0.5), P(A), P(A), big, None) == UNSUP
+    ap = L.awq_apply_clip
+    assert ap(P(A), P(A), 0, 256, P(A), None) == OK
+    assert ap(P(A), P(A), 8, 200, P(A), None) == SHAPE
+    assert ap(P(MIS), P(A), 8, 256, P(A), None) == ALIGN
 
 
 def test_interleave_gate_up_validation(L):

@@ -42,7 +42,7 @@ class AwqError(RuntimeError):
         self.status = status
 
 
-ABI_VERSION = 4   # awq_abi_version() of a library this binding matches
+ABI_VERSION = 5   # awq_abi_version() of a library this binding matches
 
 
 class QConfig(ctypes.Structure):
@@ -78,6 +78,10 @@ _SIGS = {
     "awq_search_scale": (ctypes.c_int, [_P, _I64, _I64, _P, _I64, QConfig, ctypes.c_int, ctypes.c_int, _P, _P, _P,
                                         ctypes.c_size_t, _P]),
     "awq_apply_scale": (ctypes.c_int, [_P, _P, _I64, _I64, _P, _P]),
+    "awq_search_clip_workspace_bytes": (ctypes.c_int, [_I64, ctypes.POINTER(ctypes.c_size_t)]),
+    "awq_search_clip": (ctypes.c_int, [_P, _I64, _I64, _P, _I64, QConfig, ctypes.c_int, ctypes.c_float, _P, _P,
+                                       ctypes.c_size_t, _P]),
+    "awq_apply_clip": (ctypes.c_int, [_P, _P, _I64, _I64, _P, _P]),
 }
 
 
@@ -374,4 +378,38 @@ def awq_apply_scale(W: torch.Tensor, scales: torch.Tensor, out: torch.Tensor | N
         out = torch.empty_like(W)
     with torch.cuda.device(W.device):
         _check("awq_apply_scale", lib().awq_apply_scale(_ptr(W), _ptr(scales), N, K, _ptr(out), _stream(W.device)))
+    return out
+
+
+def awq_search_clip(W: torch.Tensor, X: torch.Tensor, zero_point: bool = True, n_grid: int = 20,
+                    max_shrink: float = 0.5, group_size: int = GROUP_SIZE) -> torch.Tensor:
+    """Clipping-ratio search for W [N, K] on calibration inputs X [Ms, K]:
+    returns the ratios fp32 [K/group_size, N] (see awq.h)."""
+    _need(W, "W", torch.float16, 2)
+    _need(X, "X", torch.float16, 2)
+    N, K = W.shape
+    if X.shape[1] != K:
+        raise ValueError("X must be [Ms, K] for W [N, K]")
+    n = ctypes.c_size_t(0)
+    with torch.cuda.device(W.device):
+        _check("awq_search_clip_workspace_bytes", lib().awq_search_clip_workspace_bytes(K, ctypes.byref(n)))
+        ws = torch.empty(n.value, dtype=torch.uint8, device=W.device)
+        ratios = torch.empty((K // group_size, N), dtype=torch.float32, device=W.device)
+        _check("awq_search_clip", lib().awq_search_clip(
+            _ptr(W), N, K, _ptr(X), X.shape[0], _cfg(zero_point, group_size), n_grid, float(max_shrink),
+            _ptr(ratios), _ptr(ws), n.value, _stream(W.device)))
+    return ratios
+
+
+def awq_apply_clip(W: torch.Tensor, ratios: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """W with each (row, group) clipped to ratio * max|w| of the group (fp16)."""
+    _need(W, "W", torch.float16, 2)
+    _need(ratios, "ratios", torch.float32, 2)
+    N, K = W.shape
+    if ratios.shape != (K // GROUP_SIZE, N):
+        raise ValueError("ratios must be [K/128, N]")
+    if out is None:
+        out = torch.empty_like(W)
+    with torch.cuda.device(W.device):
+        _check("awq_apply_clip", lib().awq_apply_clip(_ptr(W), _ptr(ratios), N, K, _ptr(out), _stream(W.device)))
     return out

@@ -24,6 +24,45 @@ inline awq_status_t check_cfg(awq_qconfig_t cfg) {
   return AWQ_OK;
 }
 
+// Group quantization parameters, one warp per (row, group), four weights per
+// lane in any lane order ("AutoAWQ" code tour, "The Quantization Flow Up
+// Close": each group is rounded against its scale and zero point). IEEE fp32
+// with explicit round-to-nearest intrinsics, so the bits do not depend on
+// contraction flags:
+//   asymmetric: s = fp16(max((max w - min w) / 15, 1e-5)), z = clamp(-rint(min w / s), 0, 15)
+//   symmetric:  s = fp16(max(max|w| / 7, 1e-5)), z = 8
+// sf is the fp32 value of the fp16 scale.
+template <bool ZP>
+__device__ __forceinline__ void group_quant_params(const float (&w)[4], float& sf, float& zf) {
+  if (ZP) {
+    float mx = fmaxf(fmaxf(w[0], w[1]), fmaxf(w[2], w[3]));
+    float mn = fminf(fminf(w[0], w[1]), fminf(w[2], w[3]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    }
+    const float s32 = fmaxf(__fdiv_rn(__fsub_rn(mx, mn), 15.0f), 1e-5f);
+    sf = __half2float(__float2half_rn(s32));
+    zf = fminf(fmaxf(-rintf(__fdiv_rn(mn, sf)), 0.0f), 15.0f);
+  } else {
+    float a = fmaxf(fmaxf(fabsf(w[0]), fabsf(w[1])), fmaxf(fabsf(w[2]), fabsf(w[3])));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    const float s32 = fmaxf(__fdiv_rn(a, 7.0f), 1e-5f);
+    sf = __half2float(__float2half_rn(s32));
+    zf = 8.0f;
+  }
+}
+
+// The code of one weight under (sf, zf): clamp(rint(w / s) + z, 0, 15)
+// (symmetric: clamp(rint(w / s), -8, 7) + 8, the same value with z = 8).
+template <bool ZP>
+__device__ __forceinline__ int group_quant_code(float w, float sf, float zf) {
+  if (ZP) return int(fminf(fmaxf(__fadd_rn(rintf(__fdiv_rn(w, sf)), zf), 0.0f), 15.0f));
+  return int(fminf(fmaxf(rintf(__fdiv_rn(w, sf)), -8.0f), 7.0f)) + 8;
+}
+
 // SiLU in fp32 for the fused gate/up epilogues.
 __device__ __forceinline__ float silu_f32(float v) { return v / (1.0f + expf(-v)); }
 

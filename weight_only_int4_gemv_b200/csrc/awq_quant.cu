@@ -41,32 +41,10 @@ quantize_pack_kernel(const uint16_t* __restrict__ W, int64_t N, int64_t K,
     w[3] = half_bits_to_float(uint16_t(raw.y >> 16));
 
     int q[4];
-    float sf;
-    float zf = 0.0f;
-    if (ZP) {
-      float mx = fmaxf(fmaxf(w[0], w[1]), fmaxf(w[2], w[3]));
-      float mn = fminf(fminf(w[0], w[1]), fminf(w[2], w[3]));
+    float sf, zf;
+    group_quant_params<ZP>(w, sf, zf);
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-      }
-      const float s32 = fmaxf(__fdiv_rn(__fsub_rn(mx, mn), 15.0f), 1e-5f);
-      sf = __half2float(__float2half_rn(s32));
-      zf = fminf(fmaxf(-rintf(__fdiv_rn(mn, sf)), 0.0f), 15.0f);
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        q[i] = int(fminf(fmaxf(__fadd_rn(rintf(__fdiv_rn(w[i], sf)), zf), 0.0f), 15.0f));
-    } else {
-      float a = fmaxf(fmaxf(fabsf(w[0]), fabsf(w[1])), fmaxf(fabsf(w[2]), fabsf(w[3])));
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-      const float s32 = fmaxf(__fdiv_rn(a, 7.0f), 1e-5f);
-      sf = __half2float(__float2half_rn(s32));
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        q[i] = int(fminf(fmaxf(rintf(__fdiv_rn(w[i], sf)), -8.0f), 7.0f)) + 8;
-    }
+    for (int i = 0; i < 4; ++i) q[i] = group_quant_code<ZP>(w[i], sf, zf);
 
     // k offset o of the word goes to slot (o even ? o/2 : 4 + o/2).
     // Even lane: offsets 0..3 -> slots 0,4,1,5; odd lane: offsets 4..7 -> slots 2,6,3,7.

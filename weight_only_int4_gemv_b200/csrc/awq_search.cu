@@ -215,6 +215,135 @@ __global__ void loss_finish_kernel(const double* __restrict__ partial, int64_t c
   }
 }
 
+// ---------------------------------------------------------------------------
+// Clip search ("AutoAWQ" code tour, "The Quantization Flow Up Close": the
+// clipping pass shrinks extreme weights group by group where that lowers the
+// output error). For row n and group j, grid point i tries the ratio
+// r = 1 - max_shrink * i / n_grid: the group is clipped to [-t, t], t = r *
+// max|w| (fp32), the clipped values rounded to fp16 and quantized as by
+// awq_pseudo_quantize_pack; the error is d^T G_j d, d = w - w' and G_j =
+// X_j^T X_j the Gram matrix of the calibration inputs over the group's 128
+// input channels. The first ratio with the lowest error wins.
+// ---------------------------------------------------------------------------
+constexpr int kGramPad = kGroup + 1;   // row stride of a Gram matrix in shared memory (no bank conflicts)
+constexpr int kClipRowsPerBlock = 64;
+
+// G_j[a][b] = sum_m x[m][128 j + a] x[m][128 j + b] in fp32, rows of x in
+// order. One block per group; thread (a, half) owns 64 entries of row a.
+__global__ void __launch_bounds__(256) gram_kernel(const uint16_t* __restrict__ X, int64_t Ms, int64_t K,
+                                                   float* __restrict__ gram) {
+  __shared__ float xs[32][kGroup + 1];
+  const int j = blockIdx.x;
+  const int a = threadIdx.x >> 1;
+  const int b0 = (threadIdx.x & 1) * 64;
+  float acc[64];
+#pragma unroll
+  for (int b = 0; b < 64; ++b) acc[b] = 0.0f;
+  for (int64_t m0 = 0; m0 < Ms; m0 += 32) {
+    for (int i = threadIdx.x; i < 32 * kGroup; i += 256) {
+      const int r = i >> 7, c = i & 127;
+      xs[r][c] = (m0 + r < Ms) ? h2f(X[(m0 + r) * K + int64_t(j) * kGroup + c]) : 0.0f;
+    }
+    __syncthreads();
+    for (int r = 0; r < 32; ++r) {
+      const float xa = xs[r][a];
+#pragma unroll
+      for (int b = 0; b < 64; ++b) acc[b] = fmaf(xa, xs[r][b0 + b], acc[b]);
+    }
+    __syncthreads();
+  }
+  float* out = gram + (int64_t(j) * kGroup + a) * kGroup + b0;
+#pragma unroll
+  for (int b = 0; b < 64; ++b) out[b] = acc[b];
+}
+
+__device__ __forceinline__ float clip_ratio(int i, int n_grid, float max_shrink) {
+  return __fsub_rn(1.0f, __fdiv_rn(__fmul_rn(max_shrink, float(i)), float(n_grid)));
+}
+
+// Block: one group j (its Gram matrix in shared memory) x 64 rows; warp: one
+// row at a time, lane l holding k = l + 32 i of the group.
+template <bool ZP>
+__global__ void __launch_bounds__(256) clip_search_kernel(const uint16_t* __restrict__ W, int64_t N, int64_t K,
+                                                          const float* __restrict__ gram, int n_grid,
+                                                          float max_shrink, float* __restrict__ ratios) {
+  extern __shared__ float clip_smem[];
+  float* gs = clip_smem;                                          // [128][129]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float* dbuf = clip_smem + kGroup * kGramPad + warp * kGroup;    // [128] per warp
+  const int j = blockIdx.x;
+  for (int i = threadIdx.x; i < kGroup * kGroup; i += 256)
+    gs[(i >> 7) * kGramPad + (i & 127)] = gram[int64_t(j) * kGroup * kGroup + i];
+  __syncthreads();
+  const int64_t n_end = (int64_t(blockIdx.y) + 1) * kClipRowsPerBlock < N ? (int64_t(blockIdx.y) + 1) * kClipRowsPerBlock : N;
+  for (int64_t n = int64_t(blockIdx.y) * kClipRowsPerBlock + warp; n < n_end; n += 8) {
+    float w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w[i] = h2f(W[n * K + int64_t(j) * kGroup + lane + 32 * i]);
+    float amax = fmaxf(fmaxf(fabsf(w[0]), fabsf(w[1])), fmaxf(fabsf(w[2]), fabsf(w[3])));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    float best_err = 0.0f;
+    int best = 0;
+    for (int it = 0; it < n_grid; ++it) {
+      const float t = __fmul_rn(amax, clip_ratio(it, n_grid, max_shrink));
+      float wc[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) wc[i] = h2f(f2h(fminf(fmaxf(w[i], -t), t)));
+      float sf, zf;
+      group_quant_params<ZP>(wc, sf, zf);
+      float d[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int q = group_quant_code<ZP>(wc[i], sf, zf);
+        const float wq = h2f(f2h(__fmul_rn(__fsub_rn(float(q), zf), sf)));
+        d[i] = __fsub_rn(w[i], wq);
+        dbuf[lane + 32 * i] = d[i];
+      }
+      __syncwarp();
+      float v[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      for (int b = 0; b < kGroup; ++b) {
+        const float db = dbuf[b];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[i] = fmaf(gs[(lane + 32 * i) * kGramPad + b], db, v[i]);
+      }
+      float e = d[0] * v[0] + d[1] * v[1] + d[2] * v[2] + d[3] * v[3];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
+      e = __shfl_sync(0xffffffffu, e, 0);   // one value for the whole warp
+      if (it == 0 || e < best_err) {
+        best_err = e;
+        best = it;
+      }
+      __syncwarp();
+    }
+    if (lane == 0) ratios[int64_t(j) * N + n] = clip_ratio(best, n_grid, max_shrink);
+  }
+}
+
+// W_out = W clipped per (row, group) to [-t, t], t = ratio[j][n] * max|w|,
+// values rounded to fp16. One warp per (row, group), four weights per lane.
+__global__ void __launch_bounds__(256) apply_clip_kernel(const uint16_t* __restrict__ W,
+                                                         const float* __restrict__ ratios, int64_t N, int64_t K,
+                                                         uint16_t* __restrict__ W_out) {
+  const int lane = threadIdx.x & 31;
+  const int64_t G = K / kGroup, units = N * G;
+  const int64_t nwarps = (int64_t(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t u = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; u < units; u += nwarps) {
+    const int64_t n = u / G, j = u - n * G;
+    const int64_t base = n * K + j * kGroup + lane * 4;
+    float w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w[i] = h2f(W[base + i]);
+    float amax = fmaxf(fmaxf(fabsf(w[0]), fabsf(w[1])), fmaxf(fabsf(w[2]), fabsf(w[3])));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float t = __fmul_rn(amax, ratios[j * N + n]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) W_out[base + i] = f2h(fminf(fmaxf(w[i], -t), t));
+  }
+}
+
 size_t align256(size_t v) { return (v + 255) / 256 * 256; }
 
 struct SearchLayout {
@@ -338,5 +467,55 @@ extern "C" awq_status_t awq_apply_scale(const uint16_t* W, const float* s, int64
   if (N == 0) return AWQ_OK;
   if (!W || !s || !W_out) return AWQ_ERR_NULL;
   scale_columns_kernel<<<148 * 8, 256, 0, static_cast<cudaStream_t>(stream)>>>(W, s, N, K, 1, W_out);
+  return launch_status();
+}
+
+extern "C" awq_status_t awq_search_clip_workspace_bytes(int64_t K, size_t* bytes) {
+  if (!bytes) return AWQ_ERR_NULL;
+  if (K <= 0 || K % kGroup) return AWQ_ERR_SHAPE;
+  *bytes = size_t(K / kGroup) * kGroup * kGroup * 4;
+  return AWQ_OK;
+}
+
+extern "C" awq_status_t awq_search_clip(const uint16_t* W, int64_t N, int64_t K, const uint16_t* X, int64_t Ms,
+                                        awq_qconfig_t cfg, int n_grid, float max_shrink, float* ratios_out,
+                                        void* workspace, size_t workspace_bytes, void* stream) {
+  awq_status_t st = check_search_args(N, K, Ms, cfg);
+  if (st != AWQ_OK) return st;
+  if (n_grid < 1 || n_grid > kMaxGrid || !(max_shrink >= 0.0f && max_shrink < 1.0f)) return AWQ_ERR_SHAPE;
+  if (!W || !X || !ratios_out || !workspace) return AWQ_ERR_NULL;
+  if (!aligned16(workspace)) return AWQ_ERR_ALIGN;
+  const size_t need = size_t(K / kGroup) * kGroup * kGroup * 4;
+  if (workspace_bytes < need) return AWQ_ERR_WORKSPACE;
+  float* gram = static_cast<float*>(workspace);
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const unsigned G = unsigned(K / kGroup);
+  gram_kernel<<<G, 256, 0, cs>>>(X, Ms, K, gram);
+  const size_t smem = size_t(kGroup * kGramPad + 8 * kGroup) * 4;
+  const dim3 grid(G, unsigned((N + kClipRowsPerBlock - 1) / kClipRowsPerBlock));
+  if (cfg.zero_point) {
+    if (cudaFuncSetAttribute(clip_search_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+        cudaSuccess)
+      return AWQ_ERR_CUDA;
+    clip_search_kernel<true><<<grid, 256, smem, cs>>>(W, N, K, gram, n_grid, max_shrink, ratios_out);
+  } else {
+    if (cudaFuncSetAttribute(clip_search_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+        cudaSuccess)
+      return AWQ_ERR_CUDA;
+    clip_search_kernel<false><<<grid, 256, smem, cs>>>(W, N, K, gram, n_grid, max_shrink, ratios_out);
+  }
+  return launch_status();
+}
+
+extern "C" awq_status_t awq_apply_clip(const uint16_t* W, const float* ratios, int64_t N, int64_t K,
+                                       uint16_t* W_out, void* stream) {
+  if (N < 0 || K <= 0 || K % kGroup) return AWQ_ERR_SHAPE;
+  if (N == 0) return AWQ_OK;
+  if (!W || !ratios || !W_out) return AWQ_ERR_NULL;
+  if (!aligned16(W) || !aligned16(W_out)) return AWQ_ERR_ALIGN;
+  const int64_t units = N * (K / kGroup);
+  const int64_t blocks = (units + 7) / 8;
+  apply_clip_kernel<<<unsigned(blocks < 148 * 16 ? blocks : 148 * 16), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      W, ratios, N, K, W_out);
   return launch_status();
 }
