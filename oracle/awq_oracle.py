@@ -25,7 +25,7 @@ Sources (cited by page title and section):
   of x by a constant and multiplying the matching weight column by it leaves
   the layer output unchanged (used as a pin on the matmul, not here).
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
 
 * Asymmetric scale/zero follow the plain per-group min/max affine rule on
   the levels 0..15; the range is not widened to include 0.
