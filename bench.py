@@ -263,8 +263,9 @@ def cpu_baseline(shapes, M: int, budget_s: float = 10.0, rows: int = 1024):
 class DecodeLayer:
     """One layer copy: packed weights of each shape plus its x / y buffers."""
 
-    def __init__(self, packed, xs, ys, workspaces):
+    def __init__(self, packed, xs, ys, workspaces, x_all, y_all):
         self.packed, self.xs, self.ys, self.ws = packed, xs, ys, workspaces
+        self.x_all, self.y_all = x_all, y_all   # the xs / ys are contiguous views of these
 
 
 def build_decode(awq, torch, device, shapes, M: int, n_layers: int, zp: bool):
@@ -291,11 +292,19 @@ def build_decode(awq, torch, device, shapes, M: int, n_layers: int, zp: bool):
     layers = []
     for _ in range(n_layers):
         packed = [(q.clone(), s.clone(), z.clone() if z is not None else None) for q, s, z in base]
-        xs = [torch.from_numpy(rng.standard_normal((M, sh.K), dtype=np.float32).astype(np.float16)).to(device)
-              for sh in shapes]
-        ys = [torch.empty((M, sh.N), dtype=torch.float16, device=device) for sh in shapes]
+        # each layer's inputs (outputs) are consecutive views of one buffer, so the
+        # end-to-end leg moves them with one copy each way
+        x_all = torch.from_numpy(np.concatenate(
+            [rng.standard_normal((M, sh.K), dtype=np.float32).astype(np.float16).ravel() for sh in shapes])).to(device)
+        y_all = torch.empty(sum(M * sh.N for sh in shapes), dtype=torch.float16, device=device)
+        xs, ys, ox, oy = [], [], 0, 0
+        for sh in shapes:
+            xs.append(x_all[ox:ox + M * sh.K].view(M, sh.K))
+            ys.append(y_all[oy:oy + M * sh.N].view(M, sh.N))
+            ox += M * sh.K
+            oy += M * sh.N
         wss = [awq.alloc_workspace(M, sh.N, sh.K, zp, device=device) for sh in shapes]
-        layers.append(DecodeLayer(packed, xs, ys, wss))
+        layers.append(DecodeLayer(packed, xs, ys, wss, x_all, y_all))
     return layers, {"ms": round(quant_ms, 4), "GB/s": round(quant_bytes / (quant_ms * 1e-3) / 1e9, 1)}
 
 
@@ -438,23 +447,22 @@ def run_native(args, dist):
 
 def run_e2e(awq, torch, device, stream, layers, shapes, M, args, dist, step_bytes):
     """Same metric through the Python API with host buffers: every step copies
-    its x from pinned host memory and reads its y back into pinned host
-    memory, then synchronizes."""
+    its inputs (all projections' x, one pinned buffer) to the device, runs the
+    GEMVs, reads all their y back into pinned host memory, then synchronizes."""
     steps = max(1, min(args.steps, args.e2e_steps))
-    hx = [torch.empty((M, sh.K), dtype=torch.float16).pin_memory() for sh in shapes]
-    hy = [torch.empty((M, sh.N), dtype=torch.float16).pin_memory() for sh in shapes]
-    for i in range(len(shapes)):
-        hx[i].copy_(layers[0].xs[i].cpu())
-    h2d = sum(t.numel() * 2 for t in hx)
-    d2h = sum(t.numel() * 2 for t in hy)
+    hx = torch.empty_like(layers[0].x_all, device="cpu").pin_memory()
+    hy = torch.empty_like(layers[0].y_all, device="cpu").pin_memory()
+    hx.copy_(layers[0].x_all.cpu())
+    h2d = hx.numel() * 2
+    d2h = hy.numel() * 2
     n = len(layers)
 
     def step(s):
         L = layers[s % n]
+        L.x_all.copy_(hx, non_blocking=True)
         for i in range(len(shapes)):
-            L.xs[i].copy_(hx[i], non_blocking=True)
             awq.awq_gemv(L.xs[i], *L.packed[i], workspace=L.ws[i], out=L.ys[i], weights_static=True)
-            hy[i].copy_(L.ys[i], non_blocking=True)
+        hy.copy_(L.y_all, non_blocking=True)
         torch.cuda.current_stream(device).synchronize()
 
     with torch.cuda.stream(stream):

@@ -112,12 +112,19 @@ def _check(fn: str, st: int):
         raise AwqError(fn, st, lib().awq_status_string(st).decode())
 
 
+_CFGS = {}
+
+
 def _cfg(zero_point: bool, group_size: int, flags: int = 0) -> QConfig:
-    return QConfig(group_size, 1 if zero_point else 0, flags)
+    key = (bool(zero_point), group_size, flags)
+    c = _CFGS.get(key)
+    if c is None:
+        c = _CFGS[key] = QConfig(group_size, 1 if zero_point else 0, flags)
+    return c
 
 
 def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    return None if t is None else t.data_ptr()
 
 
 def _stream(device) -> ctypes.c_void_p:
@@ -210,12 +217,16 @@ def _product(entry: str, x, qweight, scales, zeros, workspace, out, group_size, 
     if workspace is not None:
         if not workspace.is_cuda or not workspace.is_contiguous():
             raise ValueError("workspace must be a contiguous CUDA tensor")
-        ws_ptr, ws_bytes = _ptr(workspace), workspace.numel() * workspace.element_size()
-    with torch.cuda.device(x.device):
-        fn = getattr(lib(), entry)
-        _check(entry, fn(_ptr(x), _ptr(qweight), _ptr(scales), _ptr(zeros), M, N, K,
-                         _cfg(zeros is not None, group_size, flags), _ptr(out), ws_ptr, ws_bytes,
-                         _stream(x.device)))
+        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    fn = getattr(lib(), entry)
+    dev = x.device
+    args = (_ptr(x), qweight.data_ptr(), scales.data_ptr(), _ptr(zeros), M, N, K,
+            _cfg(zeros is not None, group_size, flags), out.data_ptr(), ws_ptr, ws_bytes)
+    if dev.index == torch.cuda.current_device():   # no device switch needed (the common case)
+        _check(entry, fn(*args, torch.cuda.current_stream().cuda_stream))
+    else:
+        with torch.cuda.device(dev):
+            _check(entry, fn(*args, torch.cuda.current_stream(dev).cuda_stream))
     return out
 
 
