@@ -300,7 +300,8 @@ AWQ_API awq_status_t awq_search_scale(const uint16_t* W, int64_t N, int64_t K, c
 /*
  * awq_apply_scale -- W_out[n][k] = fp16(W[n][k] * s[k]) (fp32 product, one
  * rounding): the weights of a layer whose input will be divided by s.
- * W, W_out [N][K] fp16 device, s [K] fp32 device. N >= 0, K > 0.
+ * W, W_out [N][K] fp16 device (16-byte aligned), s [K] fp32 device.
+ * N >= 0, K > 0, K % 8 == 0.
  */
 AWQ_API awq_status_t awq_apply_scale(const uint16_t* W, const float* s, int64_t N, int64_t K, uint16_t* W_out,
                                      void* stream);

@@ -174,14 +174,23 @@ __global__ void __launch_bounds__(1024) candidate_kernel(const float* __restrict
   for (int64_t k = threadIdx.x; k < K; k += blockDim.x) s[k] = s[k] / norm;
 }
 
-// out[r][k] = fp16(in[r][k] * s[k]) (mul = 1) or fp16(in[r][k] / s[k]) (mul = 0)
+// out[r][k] = fp16(in[r][k] * s[k]) (mul = 1) or fp16(in[r][k] / s[k]) (mul = 0),
+// eight consecutive values (one 16-byte load and store) per thread; K % 8 == 0.
 __global__ void scale_columns_kernel(const uint16_t* __restrict__ in, const float* __restrict__ s, int64_t rows,
                                      int64_t K, int mul, uint16_t* __restrict__ out) {
-  const int64_t total = rows * K;
-  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += int64_t(gridDim.x) * blockDim.x) {
-    const float v = h2f(in[i]);
-    const float sk = s[i % K];
-    out[i] = f2h(mul ? v * sk : v / sk);
+  const int64_t vecs = rows * K / 8;
+  for (int64_t v = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; v < vecs; v += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t k0 = (v * 8) % K;
+    const uint4 raw = reinterpret_cast<const uint4*>(in)[v];
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float a = h2f(uint16_t(w[e] & 0xFFFF)), b = h2f(uint16_t(w[e] >> 16));
+      const float sa = s[k0 + 2 * e], sb = s[k0 + 2 * e + 1];
+      o[e] = uint32_t(f2h(mul ? a * sa : a / sa)) | (uint32_t(f2h(mul ? b * sb : b / sb)) << 16);
+    }
+    reinterpret_cast<uint4*>(out)[v] = make_uint4(o[0], o[1], o[2], o[3]);
   }
 }
 
@@ -465,7 +474,9 @@ extern "C" awq_status_t awq_apply_scale(const uint16_t* W, const float* s, int64
                                         void* stream) {
   if (N < 0 || K <= 0) return AWQ_ERR_SHAPE;
   if (N == 0) return AWQ_OK;
+  if (K % 8) return AWQ_ERR_SHAPE;
   if (!W || !s || !W_out) return AWQ_ERR_NULL;
+  if (!aligned16(W) || !aligned16(W_out)) return AWQ_ERR_ALIGN;
   scale_columns_kernel<<<148 * 8, 256, 0, static_cast<cudaStream_t>(stream)>>>(W, s, N, K, 1, W_out);
   return launch_status();
 }
