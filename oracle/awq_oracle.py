@@ -381,3 +381,44 @@ def search_clip(W: np.ndarray, X: np.ndarray, group_size: int = GROUP_SIZE, zero
     best = np.argmin(errs, axis=0)                                    # first minimum
     ratios = (np.float32(1.0) - np.float32(max_shrink) * best.astype(np.float32) / np.float32(n_grid))
     return ratios.astype(np.float32), errs
+
+
+# ---------------------------------------------------------------------------
+# Packed zero points ("AWQ > Implementation", "Understanding the Quantization
+# Structure": a quantized layer holds ``qweight``, ``scales`` and ``qzeros``;
+# its 4-bit values are stored eight per int32).
+#
+# Readings (the pages name ``qzeros`` but give neither its axis nor its nibble
+# order):
+# * qzeros is group-major like the scales, [G, N/8]: word w of group row j
+#   covers output channels n = 8w .. 8w+7, and nibble i (bits 4i..4i+3) holds
+#   n = 8w + i (the plain order: unlike the codes, no decode trick depends on
+#   it);
+# * a zero point that is not an integer in 0..15 is rounded to the nearest
+#   integer (ties to even) and clamped to 0..15; NaN becomes 0.
+# ---------------------------------------------------------------------------
+def pack_zeros(zeros: np.ndarray) -> np.ndarray:
+    """fp16 zero points [G, N] -> int32 qzeros [G, N/8] (N % 8 == 0)."""
+    z = np.asarray(zeros).astype(np.float32)
+    G, N = z.shape
+    if N % 8:
+        raise ValueError("N must be a multiple of 8")
+    z = np.where(np.isnan(z), np.float32(0.0), z)
+    q = np.clip(np.rint(z), 0, LEVELS).astype(np.uint32).reshape(G, N // 8, 8)
+    word = np.zeros((G, N // 8), dtype=np.uint32)
+    for i in range(8):
+        word |= q[:, :, i] << np.uint32(4 * i)
+    return word.view(np.int32)
+
+
+def unpack_zeros(qzeros: np.ndarray) -> np.ndarray:
+    """Inverse of :func:`pack_zeros`: int32 [G, N/8] -> fp16 zero points [G, N]."""
+    qzeros = np.asarray(qzeros)
+    if qzeros.dtype != np.int32:
+        raise TypeError("qzeros must be int32")
+    G, W = qzeros.shape
+    word = qzeros.view(np.uint32)
+    out = np.zeros((G, W, 8), dtype=np.float16)
+    for i in range(8):
+        out[:, :, i] = ((word >> np.uint32(4 * i)) & np.uint32(0xF)).astype(np.float16)
+    return out.reshape(G, W * 8)
