@@ -599,19 +599,24 @@ def run_table(args):
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
     hbm_peak, tc_peak, _, peak_src = measured_peaks()
-    # (N, K), batch sizes, fused gate/up (AWQ_FLAG_SILU_MUL: N = gate + up rows, y has N / 2 columns)
-    cases = [((4096, 4096), (1, 2, 4, 8, 16, 128, 512, 2048), False),
-             ((14336, 4096), (1, 2, 4, 8, 16, 128, 512, 2048), False),
-             ((28672, 4096), (1, 4, 16, 128, 2048), True),
-             ((6144, 4096), (1, 4, 16), False),     # q, k, v of Llama-3-8B concatenated
-             ((1024, 4096), (1, 4, 16), False),     # k or v alone
-             ((4096, 14336), (1, 2, 4, 8, 16), False),
-             ((8192, 8192), (1, 8, 2048), False), ((28672, 8192), (1, 8, 2048), False),
-             ((8192, 28672), (1, 8, 2048), False)]
+    # (N, K), batch sizes, fused gate/up (AWQ_FLAG_SILU_MUL: N = gate + up rows, y has N / 2 columns),
+    # packed zero points (AWQ_FLAG_PACKED_ZEROS, GEMV only)
+    cases = [((4096, 4096), (1, 2, 4, 8, 16, 128, 512, 2048), False, False),
+             ((14336, 4096), (1, 2, 4, 8, 16, 128, 512, 2048), False, False),
+             ((28672, 4096), (1, 4, 16, 128, 2048), True, False),
+             ((6144, 4096), (1, 4, 16), False, False),     # q, k, v of Llama-3-8B concatenated
+             ((1024, 4096), (1, 4, 16), False, False),     # k or v alone
+             ((4096, 14336), (1, 2, 4, 8, 16), False, False),
+             ((8192, 8192), (1, 8, 2048), False, False), ((28672, 8192), (1, 8, 2048), False, False),
+             ((8192, 28672), (1, 8, 2048), False, False),
+             ((4096, 4096), (1, 4, 16), False, True), ((14336, 4096), (1, 4, 16), False, True),
+             ((4096, 14336), (1, 4, 16), False, True), ((28672, 4096), (1, 4, 16), True, True)]
     l2_bytes = 126 << 20
     rng = np.random.default_rng(3)
-    for (N, K), Ms, silu in cases:
+    for (N, K), Ms, silu, packed in cases:
         q, s, z = [torch.from_numpy(a).to(device) for a in make_packed_random(N, K, 128, True, seed=1)]
+        if packed:
+            z = awq.awq_pack_zeros(z)
         wbytes = N * K // 2 + 4 * N * (K // 128)
         copies = max(2, -(-2 * l2_bytes // wbytes))
         packs = [(q.clone(), s.clone(), z.clone()) for _ in range(copies)]
@@ -619,7 +624,8 @@ def run_table(args):
         for M in Ms:
             x = torch.from_numpy(rng.standard_normal((M, K), dtype=np.float32).astype(np.float16)).to(device)
             y = torch.empty((M, N // 2 if silu else N), dtype=torch.float16, device=device)
-            entry = ("awq_gemv" if M <= awq.GEMV_MAX_M else "awq_gemm") + (" silu_mul" if silu else "")
+            entry = (("awq_gemv" if M <= awq.GEMV_MAX_M else "awq_gemm") + (" silu_mul" if silu else "") +
+                     (" packed_zeros" if packed else ""))
             fn = awq.awq_gemv if M <= awq.GEMV_MAX_M else awq.awq_gemm
             kw = {"weights_static": True} if M <= awq.GEMV_MAX_M else {}
             if silu:
@@ -645,7 +651,9 @@ def run_table(args):
                 e1.record()
                 torch.cuda.synchronize(device)
             us = e0.elapsed_time(e1) * 1e3 / (reps * copies)
-            gbs = (algo_bytes(M, N, K) - (M * N if silu else 0)) / (us * 1e-6) / 1e9   # y: N/2 columns
+            # y: N/2 columns with silu_mul; packed zero points: 4 bits instead of 16 per (row, group)
+            nbytes = algo_bytes(M, N, K) - (M * N if silu else 0) - (3 * N * (K // 128) // 2 if packed else 0)
+            gbs = nbytes / (us * 1e-6) / 1e9
             tfl = algo_flops(M, N, K) / (us * 1e-6) / 1e12
             print(json.dumps({"entry": entry, "N": N, "K": K, "M": M, "us": round(us, 3), "GB/s": round(gbs, 1),
                               "frac_hbm": round(gbs / hbm_peak, 4), "TFLOP/s": round(tfl, 2),

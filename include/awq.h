@@ -63,7 +63,7 @@
 extern "C" {
 #endif
 
-#define AWQ_ABI_VERSION 5
+#define AWQ_ABI_VERSION 6
 
 #if defined(__GNUC__)
 #define AWQ_API __attribute__((visibility("default")))
@@ -115,6 +115,21 @@ typedef struct awq_qconfig {
  * fp32 (expf). Requires N % 32 == 0. awq_workspace_bytes takes the flag. */
 #define AWQ_FLAG_SILU_MUL 2u
 
+/* Packed zero points ("AWQ > Implementation", "Understanding the Quantization
+ * Structure": a quantized layer holds qweight, scales and qzeros, its 4-bit
+ * values stored eight per int32). With this flag the `zeros` argument of
+ * awq_gemv, awq_gemv_noalloc and awq_dequant points to int32
+ * qzeros[K/128][N/8] instead of fp16 zeros[K/128][N]: word w of group row j
+ * holds the zero points of output channels 8w .. 8w+7 of that group, channel
+ * 8w+i in bits 4i .. 4i+3 (awq_pack_zeros writes it from the fp16 array).
+ * Results are identical to the fp16 form of the same zero points. Needs
+ * zero_point = 1 (else AWQ_ERR_UNSUPPORTED); N % 32 == 0 for awq_gemv and
+ * awq_gemv_noalloc (a group row of qzeros is then whole 16-byte runs), N % 8
+ * == 0 for awq_dequant (else AWQ_ERR_SHAPE). awq_workspace_bytes takes it for
+ * M <= 16. Every other entry point, awq_gemm included, returns
+ * AWQ_ERR_UNSUPPORTED for it (awq_unpack_zeros restores the fp16 form). */
+#define AWQ_FLAG_PACKED_ZEROS 4u
+
 /* ABI version of the loaded library (AWQ_ABI_VERSION at build time). */
 AWQ_API int awq_abi_version(void);
 
@@ -152,10 +167,27 @@ AWQ_API awq_status_t awq_pseudo_quantize_pack(const uint16_t* W, int64_t N, int6
  * w'[n][k] = fp16((q - z) * s), one rounding to nearest even ((q - z) * s is
  * exact in fp32), z = 8 for symmetric. Bit-exact.
  * N >= 0, K > 0, K % group_size == 0; zeros NULL iff symmetric.
+ * cfg.flags may hold AWQ_FLAG_PACKED_ZEROS (zeros is then int32 qzeros).
  */
 AWQ_API awq_status_t awq_dequant(const int32_t* qweight, const uint16_t* scales,
                          const uint16_t* zeros, int64_t N, int64_t K,
                          awq_qconfig_t cfg, uint16_t* W_out, void* stream);
+
+/*
+ * awq_pack_zeros -- fp16 zero points [G][N] (as awq_pseudo_quantize_pack
+ * writes them) -> int32 qzeros [G][N/8] in the AWQ_FLAG_PACKED_ZEROS layout.
+ * Each value is rounded to the nearest integer (ties to even) and clamped to
+ * 0..15 (NaN -> 0); the quantizer's zero points are integers 0..15 already.
+ * G >= 0, N >= 0, N % 8 == 0 (either 0: no work); zeros and qzeros
+ * device pointers, 16-byte aligned, caller-owned. One kernel on `stream`.
+ *
+ * awq_unpack_zeros -- the inverse: qzeros [G][N/8] -> fp16 zeros [G][N]
+ * holding the integers 0..15. Same limits.
+ */
+AWQ_API awq_status_t awq_pack_zeros(const uint16_t* zeros, int64_t G, int64_t N,
+                                    int32_t* qzeros, void* stream);
+AWQ_API awq_status_t awq_unpack_zeros(const int32_t* qzeros, int64_t G, int64_t N,
+                                      uint16_t* zeros, void* stream);
 
 /*
  * awq_workspace_bytes -- bytes of workspace awq_gemv / awq_gemm need for
@@ -178,8 +210,8 @@ AWQ_API awq_status_t awq_workspace_bytes(int64_t M, int64_t N, int64_t K,
  * device and shape, so results are reproducible run to run.
  * M in [1, 16]; N >= 0 and N % 8 == 0 (0: no work); K > 0, K % group_size == 0.
  * (N % 8 keeps every 8-row run of scales and zero points 16-byte aligned.)
- * cfg.flags may hold AWQ_FLAG_WEIGHTS_STATIC and AWQ_FLAG_SILU_MUL (see there;
- * with the latter y is [M][N/2]).
+ * cfg.flags may hold AWQ_FLAG_WEIGHTS_STATIC, AWQ_FLAG_SILU_MUL and
+ * AWQ_FLAG_PACKED_ZEROS (see there; with AWQ_FLAG_SILU_MUL y is [M][N/2]).
  * workspace: at least awq_workspace_bytes(M, N, K) bytes, zero-filled before
  * first use (see above); may be NULL when that size is 0, which is the case
  * whenever N / 16 is at least the device's SM count.

@@ -10,6 +10,7 @@ import os
 import re
 
 import pytest
+import torch
 
 import weight_only_int4_gemv_b200 as awq
 
@@ -44,7 +45,7 @@ def test_header_declares_the_entry_points():
               "awq_workspace_bytes", "awq_status_string", "awq_abi_version", "awq_device_error",
               "awq_interleave_gate_up", "awq_concat_rows", "awq_search_scale",
               "awq_search_scale_workspace_bytes", "awq_apply_scale", "awq_search_clip",
-              "awq_search_clip_workspace_bytes", "awq_apply_clip"]:
+              "awq_search_clip_workspace_bytes", "awq_apply_clip", "awq_pack_zeros", "awq_unpack_zeros"]:
         assert s in syms
 
 
@@ -87,7 +88,7 @@ def test_product_validation(L, entry):
     assert _gemv(L, x=MIS, entry=entry) == ALIGN
     assert _gemv(L, y=MIS, entry=entry) == ALIGN
     assert _gemv(L, N=0, entry=entry) == OK                     # empty: no work, no CUDA call
-    assert _gemv(L, c=cfg(flags=4), entry=entry) == UNSUP       # undefined flag bits
+    assert _gemv(L, c=cfg(flags=8), entry=entry) == UNSUP       # undefined flag bits
     assert _gemv(L, c=cfg(flags=0x80000000), entry=entry) == UNSUP
     assert _gemv(L, N=0, c=cfg(flags=awq.FLAG_WEIGHTS_STATIC), entry=entry) == OK
     # the fused gate/up layout needs whole 32-row tile pairs
@@ -200,6 +201,49 @@ def test_quantize_and_dequant_validation(L):
     assert d(P(A), P(A), P(A), 8, 256, cfg(g=32), P(A), None) == UNSUP
     assert d(P(A), P(A), P(A), 8, 256, cfg(), P(MIS), None) == ALIGN
     assert d(P(A), P(A), P(A), 0, 256, cfg(), P(A), None) == OK
+
+
+def test_packed_zeros_validation(L):
+    PZ = awq.FLAG_PACKED_ZEROS
+    assert PZ == int(re.search(r"#define AWQ_FLAG_PACKED_ZEROS (\d+)u", open(HEADER).read()).group(1))
+    P = ctypes.c_void_p
+    # every case below is rejected (or has no work) before any CUDA call (the pointers are fake)
+    for entry in ("awq_gemv", "awq_gemv_noalloc"):
+        f = getattr(L, entry)
+        args = lambda N, c, z=A: (P(A), P(A), P(A), P(z) if z else None, 1, N, 256, c, P(A))
+        tail = (None, 0, None) if entry == "awq_gemv" else (None,)
+        assert f(*args(64, cfg(zp=0, flags=PZ), z=0), *tail) == UNSUP     # packed zeros need zero_point = 1
+        assert f(*args(48, cfg(flags=PZ)), *tail) == SHAPE                # N % 32
+        assert f(*args(0, cfg(flags=PZ)), *tail) == OK                    # empty
+        assert f(*args(64, cfg(flags=PZ), z=0), *tail) == NULL
+        assert f(*args(64, cfg(flags=PZ), z=MIS), *tail) == ALIGN
+    assert _gemv(L, c=cfg(flags=PZ), entry="awq_gemm") == UNSUP          # the GEMM reads fp16 zero points only
+    n = ctypes.c_size_t(7)
+    assert L.awq_workspace_bytes(32, 64, 256, cfg(flags=PZ), ctypes.byref(n)) == UNSUP
+    assert L.awq_workspace_bytes(1, 48, 256, cfg(flags=PZ), ctypes.byref(n)) == SHAPE
+    assert L.awq_workspace_bytes(1, 0, 256, cfg(flags=PZ), ctypes.byref(n)) == OK and n.value == 0
+    d = L.awq_dequant
+    assert d(P(A), P(A), P(A), 12, 256, cfg(flags=PZ), P(A), None) == SHAPE     # N % 8
+    assert d(P(A), P(A), None, 8, 256, cfg(zp=0, flags=PZ), P(A), None) == UNSUP
+    assert d(P(A), P(A), P(MIS), 8, 256, cfg(flags=PZ), P(A), None) == ALIGN
+    assert d(P(A), P(A), P(A), 0, 256, cfg(flags=PZ), P(A), None) == OK
+    for f in (L.awq_pack_zeros, L.awq_unpack_zeros):
+        assert f(P(A), 2, 12, P(A), None) == SHAPE       # N % 8
+        assert f(P(A), -1, 16, P(A), None) == SHAPE
+        assert f(P(A), 2, -8, P(A), None) == SHAPE
+        assert f(P(A), 0, 16, P(A), None) == OK          # empty
+        assert f(P(A), 2, 0, None, None) == OK
+        assert f(None, 2, 16, P(A), None) == NULL
+        assert f(P(A), 2, 16, None, None) == NULL
+        assert f(P(MIS), 2, 16, P(A), None) == ALIGN
+        assert f(P(A), 2, 16, P(MIS), None) == ALIGN
+    # entry points that copy or write zero points take the fp16 form only
+    assert L.awq_pseudo_quantize_pack(P(A), 8, 256, cfg(flags=PZ), P(A), P(A), P(A), None) == UNSUP
+
+
+def test_binding_packed_zeros_shapes():
+    with pytest.raises(ValueError):
+        awq.awq_pack_zeros(torch.zeros(2, 16, dtype=torch.float16))     # not a CUDA tensor
 
 
 def test_workspace_query_validation(L):

@@ -25,6 +25,7 @@ __all__ = [
     "LIB_PATH", "AwqError", "lib", "GROUP_SIZE",
     "awq_pseudo_quantize_pack", "awq_dequant", "awq_workspace_bytes",
     "awq_gemv", "awq_gemm", "awq_device_error", "awq_linear", "GEMV_MAX_M", "awq_gemv_noalloc",
+    "awq_pack_zeros", "awq_unpack_zeros",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libawq_b200.so")
@@ -42,7 +43,7 @@ class AwqError(RuntimeError):
         self.status = status
 
 
-ABI_VERSION = 5   # awq_abi_version() of a library this binding matches
+ABI_VERSION = 6   # awq_abi_version() of a library this binding matches
 
 
 class QConfig(ctypes.Structure):
@@ -54,6 +55,7 @@ class QConfig(ctypes.Structure):
 # kernel finishes (it still waits for that kernel before reading x).
 FLAG_WEIGHTS_STATIC = 1
 FLAG_SILU_MUL = 2   # rows are 16-row tiles alternating gate, up; y = silu(gate) * up, N/2 columns
+FLAG_PACKED_ZEROS = 4   # zeros is int32 qzeros [K/128, N/8], eight 4-bit zero points per word
 
 
 _lib = None
@@ -71,6 +73,8 @@ _SIGS = {
     "awq_gemm": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, QConfig, _P, _P, ctypes.c_size_t, _P]),
     "awq_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), _P]),
     "awq_gemv_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, QConfig, _P, _P]),
+    "awq_pack_zeros": (ctypes.c_int, [_P, _I64, _I64, _P, _P]),
+    "awq_unpack_zeros": (ctypes.c_int, [_P, _I64, _I64, _P, _P]),
     "awq_interleave_gate_up": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, QConfig, _P, _P, _P, _P]),
     "awq_concat_rows": (ctypes.c_int, [ctypes.c_int, ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.POINTER(_P),
                                        ctypes.POINTER(_I64), _I64, QConfig, _P, _P, _P, _P]),
@@ -142,6 +146,52 @@ def _need(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int):
         raise ValueError(f"{name} must be a contiguous {ndim}-d tensor")
 
 
+def _zeros_flag(zeros, N: int, K: int, group_size: int) -> int:
+    """Check the zero points' form: fp16 [K/g, N], or int32 qzeros [K/g, N/8]
+    (AWQ_FLAG_PACKED_ZEROS, returned as the flag to pass)."""
+    if zeros is None:
+        return 0
+    if isinstance(zeros, torch.Tensor) and zeros.dtype == torch.int32:
+        _need(zeros, "zeros", torch.int32, 2)
+        if group_size == GROUP_SIZE and (N % 8 or zeros.shape != (K // group_size, N // 8)):
+            raise ValueError("packed zeros must be int32 [K/group_size, N/8]")
+        return FLAG_PACKED_ZEROS
+    _need(zeros, "zeros", torch.float16, 2)
+    if group_size == GROUP_SIZE and zeros.shape != (K // group_size, N):
+        raise ValueError("scales / zeros must be [K/group_size, N]")
+    return 0
+
+
+def awq_pack_zeros(zeros: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """fp16 zero points [G, N] -> int32 qzeros [G, N/8] (eight 4-bit values per
+    word, channel 8w+i in bits 4i..4i+3), the AWQ_FLAG_PACKED_ZEROS form that
+    awq_gemv and awq_dequant accept in place of the fp16 array."""
+    _need(zeros, "zeros", torch.float16, 2)
+    G, N = zeros.shape
+    if out is None:
+        out = torch.empty((G, N // 8), dtype=torch.int32, device=zeros.device)
+    _need(out, "out", torch.int32, 2)
+    if out.shape != (G, N // 8):
+        raise ValueError("out must be int32 [G, N/8]")
+    with torch.cuda.device(zeros.device):
+        _check("awq_pack_zeros", lib().awq_pack_zeros(_ptr(zeros), G, N, _ptr(out), _stream(zeros.device)))
+    return out
+
+
+def awq_unpack_zeros(qzeros: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """int32 qzeros [G, N/8] -> fp16 zero points [G, N] (the integers 0..15)."""
+    _need(qzeros, "qzeros", torch.int32, 2)
+    G, N = qzeros.shape[0], qzeros.shape[1] * 8
+    if out is None:
+        out = torch.empty((G, N), dtype=torch.float16, device=qzeros.device)
+    _need(out, "out", torch.float16, 2)
+    if out.shape != (G, N):
+        raise ValueError("out must be fp16 [G, N]")
+    with torch.cuda.device(qzeros.device):
+        _check("awq_unpack_zeros", lib().awq_unpack_zeros(_ptr(qzeros), G, N, _ptr(out), _stream(qzeros.device)))
+    return out
+
+
 def awq_pseudo_quantize_pack(W: torch.Tensor, zero_point: bool = True, group_size: int = GROUP_SIZE):
     """Quantize fp16 W[N, K] and pack it: returns (qweight, scales, zeros or None)."""
     _need(W, "W", torch.float16, 2)
@@ -162,18 +212,16 @@ def awq_dequant(qweight: torch.Tensor, scales: torch.Tensor, zeros, group_size: 
     """Decode packed weights to fp16 W'[N, K] (bit-exact)."""
     _need(qweight, "qweight", torch.int32, 2)
     _need(scales, "scales", torch.float16, 2)
-    if zeros is not None:
-        _need(zeros, "zeros", torch.float16, 2)
     N, K = qweight.shape[0], qweight.shape[1] * 8
-    if group_size == GROUP_SIZE and (scales.shape != (K // group_size, N) or
-                                     (zeros is not None and zeros.shape != scales.shape)):
+    zflag = _zeros_flag(zeros, N, K, group_size)
+    if group_size == GROUP_SIZE and scales.shape != (K // group_size, N):
         raise ValueError("scales / zeros must be [K/group_size, N]")
     if out is None:
         out = torch.empty((N, K), dtype=torch.float16, device=qweight.device)
     _need(out, "out", torch.float16, 2)
     with torch.cuda.device(qweight.device):
         _check("awq_dequant", lib().awq_dequant(
-            _ptr(qweight), _ptr(scales), _ptr(zeros), N, K, _cfg(zeros is not None, group_size),
+            _ptr(qweight), _ptr(scales), _ptr(zeros), N, K, _cfg(zeros is not None, group_size, zflag),
             _ptr(out), _stream(qweight.device)))
     return out
 
@@ -201,14 +249,12 @@ def _product(entry: str, x, qweight, scales, zeros, workspace, out, group_size, 
     _need(x, "x", torch.float16, 2)
     _need(qweight, "qweight", torch.int32, 2)
     _need(scales, "scales", torch.float16, 2)
-    if zeros is not None:
-        _need(zeros, "zeros", torch.float16, 2)
     M, K = x.shape
     N = qweight.shape[0]
     if qweight.shape[1] * 8 != K:
         raise ValueError("qweight must be [N, K/8] for x [M, K]")
-    if group_size == GROUP_SIZE and (scales.shape != (K // group_size, N) or
-                                     (zeros is not None and zeros.shape != scales.shape)):
+    flags |= _zeros_flag(zeros, N, K, group_size)
+    if group_size == GROUP_SIZE and scales.shape != (K // group_size, N):
         raise ValueError("scales / zeros must be [K/group_size, N]")
     if out is None:
         out = torch.empty((M, N // 2 if flags & FLAG_SILU_MUL else N), dtype=torch.float16, device=x.device)
@@ -241,7 +287,9 @@ def awq_gemv(x, qweight, scales, zeros, workspace=None, out=None, group_size: in
     or zeros (a decode loop over loaded weights), so the kernel may start
     streaming them before the previous kernel on the stream has finished.
     silu_mul: the weights are a fused gate/up pair (awq_interleave_gate_up);
-    y = silu(x . Wg'^T) * (x . Wu'^T), N/2 columns."""
+    y = silu(x . Wg'^T) * (x . Wu'^T), N/2 columns.
+    zeros may be fp16 [K/128, N] or int32 qzeros [K/128, N/8] from
+    awq_pack_zeros (N % 32 == 0); y is the same."""
     return _product("awq_gemv", x, qweight, scales, zeros, workspace, out, group_size,
                     _flags(weights_static, silu_mul))
 
@@ -254,19 +302,18 @@ def awq_gemv_noalloc(x, qweight, scales, zeros, out=None, group_size: int = GROU
     _need(x, "x", torch.float16, 2)
     _need(qweight, "qweight", torch.int32, 2)
     _need(scales, "scales", torch.float16, 2)
-    if zeros is not None:
-        _need(zeros, "zeros", torch.float16, 2)
     M, K = x.shape
     N = qweight.shape[0]
     if qweight.shape[1] * 8 != K:
         raise ValueError("qweight must be [N, K/8] for x [M, K]")
+    zflag = _zeros_flag(zeros, N, K, group_size)
     if out is None:
         out = torch.empty((M, N // 2 if silu_mul else N), dtype=torch.float16, device=x.device)
     _need(out, "out", torch.float16, 2)
     with torch.cuda.device(x.device):
         _check("awq_gemv_noalloc", lib().awq_gemv_noalloc(
             _ptr(x), _ptr(qweight), _ptr(scales), _ptr(zeros), M, N, K,
-            _cfg(zeros is not None, group_size, _flags(weights_static, silu_mul)),
+            _cfg(zeros is not None, group_size, _flags(weights_static, silu_mul) | zflag),
             _ptr(out), _stream(x.device)))
     return out
 

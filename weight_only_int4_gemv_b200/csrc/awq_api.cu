@@ -4,7 +4,7 @@
 #include "awq_common.cuh"
 
 namespace awq {
-awq_status_t gemv_workspace_bytes(int64_t M, int64_t N, int64_t K, bool zp, bool silu, size_t* bytes);
+awq_status_t gemv_workspace_bytes(int64_t M, int64_t N, int64_t K, int zp, bool silu, size_t* bytes);
 awq_status_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, bool zp, size_t* bytes);
 }  // namespace awq
 
@@ -27,13 +27,16 @@ extern "C" awq_status_t awq_workspace_bytes(int64_t M, int64_t N, int64_t K, awq
                                             size_t* bytes) {
   using namespace awq;
   if (!bytes) return AWQ_ERR_NULL;
-  awq_status_t st = check_cfg(cfg);
+  awq_status_t st = check_cfg(cfg, true);
   if (st != AWQ_OK) return st;
   if ((st = check_nk(N, K)) != AWQ_OK) return st;
   if (M < 0) return AWQ_ERR_SHAPE;
+  // packed zero points are read by the GEMV only
+  if ((cfg.flags & AWQ_FLAG_PACKED_ZEROS) && M > 16) return AWQ_ERR_UNSUPPORTED;
   *bytes = 0;
   if (M == 0 || N == 0) return AWQ_OK;
   if ((cfg.flags & AWQ_FLAG_SILU_MUL) && N % 32) return AWQ_ERR_SHAPE;
-  if (M <= 16) return gemv_workspace_bytes(M, N, K, cfg.zero_point != 0, (cfg.flags & AWQ_FLAG_SILU_MUL) != 0, bytes);
+  if ((cfg.flags & AWQ_FLAG_PACKED_ZEROS) && N % 32) return AWQ_ERR_SHAPE;
+  if (M <= 16) return gemv_workspace_bytes(M, N, K, zero_mode(cfg), (cfg.flags & AWQ_FLAG_SILU_MUL) != 0, bytes);
   return gemm_workspace_bytes(M, N, K, cfg.zero_point != 0, bytes);
 }

@@ -17,11 +17,20 @@ constexpr int kWordsPerGroup = kGroup / 8;
 // ---------------------------------------------------------------------------
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-inline awq_status_t check_cfg(awq_qconfig_t cfg) {
+// packed_zeros: the entry point reads AWQ_FLAG_PACKED_ZEROS zero points
+// (the others reject the flag).
+inline awq_status_t check_cfg(awq_qconfig_t cfg, bool packed_zeros = false) {
   if (cfg.group_size != kGroup) return AWQ_ERR_UNSUPPORTED;
   if (cfg.zero_point != 0 && cfg.zero_point != 1) return AWQ_ERR_UNSUPPORTED;
-  if (cfg.flags & ~(AWQ_FLAG_WEIGHTS_STATIC | AWQ_FLAG_SILU_MUL)) return AWQ_ERR_UNSUPPORTED;
+  const uint32_t known = AWQ_FLAG_WEIGHTS_STATIC | AWQ_FLAG_SILU_MUL | (packed_zeros ? AWQ_FLAG_PACKED_ZEROS : 0u);
+  if (cfg.flags & ~known) return AWQ_ERR_UNSUPPORTED;
+  if ((cfg.flags & AWQ_FLAG_PACKED_ZEROS) && !cfg.zero_point) return AWQ_ERR_UNSUPPORTED;
   return AWQ_OK;
+}
+
+// 0 symmetric, 1 fp16 zero points, 2 packed zero points (after check_cfg).
+inline int zero_mode(awq_qconfig_t cfg) {
+  return cfg.zero_point ? ((cfg.flags & AWQ_FLAG_PACKED_ZEROS) ? 2 : 1) : 0;
 }
 
 // Group quantization parameters, one warp per (row, group), four weights per

@@ -80,6 +80,12 @@ constexpr int kRingOffset = 1024;              // mbarriers and counters live be
 constexpr int kTileStageBytes = kWarps * kTile * 64;    // codes of one tile: [group][16 rows][16 words]
 constexpr int kMetaStageBytes = kWarps * kChunkRows * 2;  // [group][64 rows] fp16 scales (or zeros)
 constexpr int kXStageBytesPerRow = kWarps * 128 * 2;      // x: [m][group][128 k] fp16
+// Packed zero points (AWQ_FLAG_PACKED_ZEROS): a stage holds, per group, the
+// 8 qzeros words of a 4-tile chunk from a 16-byte-aligned start word (2 words
+// before an odd first tile), rounded up to whole 16-byte runs: 12 words.
+constexpr int kPackedZeroWords = 12;
+constexpr int kPackedZeroStageBytes = kWarps * kPackedZeroWords * 4;
+static_assert(kPackedZeroStageBytes % 128 == 0, "x must stay 128-byte aligned in a stage");
 constexpr int kReduceBarrier = 1;              // named barrier of the chunk reductions
 static_assert(kMaxStages * (8 + 4 + 4) + 4 <= kRingOffset, "stage bookkeeping overflows its region");
 
@@ -185,9 +191,21 @@ __device__ __forceinline__ void cursor_next(const GemvParams& p, int ct, int tpu
   }
 }
 
-__device__ __forceinline__ uint32_t stage_tx_bytes(const GemvParams& p, int tc, bool zp) {
-  return uint32_t(tc * kTileStageBytes + kMetaStageBytes * (zp ? 2 : 1) + p.M * kXStageBytesPerRow);
+template <bool ZP, bool PZ>
+__device__ __forceinline__ uint32_t stage_tx_bytes(const GemvParams& p, int tc) {
+  return uint32_t(tc * kTileStageBytes + kMetaStageBytes + (ZP ? (PZ ? kPackedZeroStageBytes : kMetaStageBytes) : 0) +
+                  p.M * kXStageBytesPerRow);
 }
+
+// Two integers 0..15 in the halves of v -> the same two values as fp16:
+// 0x6400 | q is exactly 1024 + q, less 1024.
+__device__ __forceinline__ uint32_t small_ints_to_half2(uint32_t v) {
+  uint32_t r;
+  asm("sub.f16x2 %0, %1, %2;" : "=r"(r) : "r"(v | 0x64006400u), "r"(0x64006400u));
+  return r;
+}
+
+__device__ __forceinline__ uint2 lds64(const uint8_t* p) { return *reinterpret_cast<const uint2*>(p); }
 
 // The codes of a stage as one 4-D box per tile count: a view of qweight as
 // {16 words, 16 rows, G groups, N/16 tiles} whose boxes of 16 x 16 x 8 x tc
@@ -200,8 +218,10 @@ struct CodeMaps {
 
 // Copies of the weight part of a stage: the codes of its tiles (one 4-D box,
 // or one 3-D box of 16 words x 16 rows x 8 groups per tile, landing
-// group-major), and the 64-row runs of scales and zero points of the 8 groups.
-template <bool ZP>
+// group-major), and the 64-row runs of scales and zero points of the 8 groups
+// (packed zero points: 12 words x 8 groups from word 2 t0 rounded down to a
+// multiple of 4, so the box starts on a 16-byte boundary).
+template <bool ZP, bool PZ>
 __device__ __forceinline__ void issue_weights(const StageCursor& u, uint8_t* st, uint64_t* bar,
                                               const CUtensorMap* tq, const CUtensorMap* ts,
                                               const CUtensorMap* tz, int p_scale_offset, const CodeMaps* cq) {
@@ -212,7 +232,10 @@ __device__ __forceinline__ void issue_weights(const StageCursor& u, uint8_t* st,
     for (int r = 0; r < u.c.tc; ++r) tma_load_3d(st + r * kTileStageBytes, tq, 0, r0 + r * kTile, u.gbase, bar);
   }
   tma_load_2d(st + p_scale_offset, ts, r0, u.gbase, bar);
-  if (ZP) tma_load_2d(st + p_scale_offset + kMetaStageBytes, tz, r0, u.gbase, bar);
+  if (ZP) {
+    if (PZ) tma_load_2d(st + p_scale_offset + kMetaStageBytes, tz, (2 * u.c.t0) & ~3, u.gbase, bar);
+    else tma_load_2d(st + p_scale_offset + kMetaStageBytes, tz, r0, u.gbase, bar);
+  }
 }
 
 // Per-warp state of the stage pipeline.
@@ -234,6 +257,7 @@ struct Pipe {
   bool ok;
   int S, i1;
   int lane, w, g, t;
+  int zsh;             // 4 g: this lane's nibble in a packed zero-point word
   int xoff[MT];
   bool xok[MT];
   uint32_t ca0, ca2;
@@ -244,7 +268,7 @@ struct Pipe {
 // multiply into acc. All TC tile slots are computed, so the unrolled loops
 // carry no branches; in a chunk with fewer tiles the extra slots hold stale
 // shared memory and their rows are never stored.
-template <int MT, bool ZP, int TC, int TPU>
+template <int MT, bool ZP, bool PZ, int TC, int TPU>
 __device__ __forceinline__ void chunk_stages(const GemvParams& p, Pipe<MT>& pp, const Chunk& cc,
                                              float (&acc)[kChunkTiles][MT][4], volatile int* abort_flag) {
     for (int gbase = cc.gb; gbase < cc.ge; gbase += kWarps) {
@@ -266,14 +290,22 @@ __device__ __forceinline__ void chunk_stages(const GemvParams& p, Pipe<MT>& pp, 
           for (int jj = 0; jj < 4; ++jj) xf[mt][jj] = pp.xok[mt] ? lds128(st + pp.xoff[mt] + jj * 16) : make_uint4(0, 0, 0, 0);
         const uint8_t* cw = st + pp.w * (kTile * 64) + pp.g * 64 + pp.t * 16;
         const uint8_t* sw = st + p.scale_offset + pp.w * 128 + pp.g * 2;
+        // packed zero points: rows g and g + 8 of tile rt are nibble g of
+        // words 2 rt and 2 rt + 1 past the chunk's first word
+        const uint8_t* zw = st + p.scale_offset + kMetaStageBytes + pp.w * (kPackedZeroWords * 4) + (cc.t0 & 1) * 8;
 #pragma unroll
         for (int rt = 0; rt < TC; ++rt) {
           c_lo[rt] = lds128(cw + rt * kTileStageBytes);
           c_hi[rt] = lds128(cw + rt * kTileStageBytes + 8 * 64);
           s2[rt] = uint32_t(lds16(sw + rt * 32)) | (uint32_t(lds16(sw + rt * 32 + 16)) << 16);
-          z2[rt] = ZP ? (uint32_t(lds16(sw + kMetaStageBytes + rt * 32)) |
-                         (uint32_t(lds16(sw + kMetaStageBytes + rt * 32 + 16)) << 16))
-                      : 0x48004800u;   // 8.0 in both halves
+          if constexpr (PZ) {
+            const uint2 zz = lds64(zw + rt * 8);
+            z2[rt] = small_ints_to_half2(((zz.x >> pp.zsh) & 0xFu) | (((zz.y >> pp.zsh) & 0xFu) << 16));
+          } else {
+            z2[rt] = ZP ? (uint32_t(lds16(sw + kMetaStageBytes + rt * 32)) |
+                           (uint32_t(lds16(sw + kMetaStageBytes + rt * 32 + 16)) << 16))
+                        : 0x48004800u;   // 8.0 in both halves
+          }
         }
       }
       // Release the stage; the last of the CTA's warps to do so refills it
@@ -288,8 +320,8 @@ __device__ __forceinline__ void chunk_stages(const GemvParams& p, Pipe<MT>& pp, 
           if (!pp.pc.done()) {
             fence_proxy_async_smem();
             uint8_t* dst = pp.ring + pp.slot * p.stage_bytes;
-            mbar_arrive_expect_tx(&pp.full[pp.slot], stage_tx_bytes(p, pp.pc.c.tc, ZP));
-            issue_weights<ZP>(pp.pc, dst, &pp.full[pp.slot], pp.tq, pp.ts, pp.tz, p.scale_offset, pp.cq);
+            mbar_arrive_expect_tx(&pp.full[pp.slot], stage_tx_bytes<ZP, PZ>(p, pp.pc.c.tc));
+            issue_weights<ZP, PZ>(pp.pc, dst, &pp.full[pp.slot], pp.tq, pp.ts, pp.tz, p.scale_offset, pp.cq);
             tma_load_3d(dst + p.x_offset, pp.tx, 0, pp.pc.gbase, 0, &pp.full[pp.slot]);
             pp.fills[pp.slot] += 1u;
           }
@@ -359,8 +391,9 @@ __device__ __forceinline__ void chunk_stages(const GemvParams& p, Pipe<MT>& pp, 
 }
 
 // One CTA's work: items [i0, i1) in chunks of at most TC tiles. SILU: the
-// fused gate/up epilogue (AWQ_FLAG_SILU_MUL; units are tile pairs).
-template <int MT, bool ZP, int TC, bool SILU>
+// fused gate/up epilogue (AWQ_FLAG_SILU_MUL; units are tile pairs). PZ:
+// packed zero points (AWQ_FLAG_PACKED_ZEROS, asymmetric only).
+template <int MT, bool ZP, bool PZ, int TC, bool SILU>
 __device__ __forceinline__ void gemv_cta(const CUtensorMap& tmap_q, const CUtensorMap& tmap_x,
                                          const CUtensorMap& tmap_s, const CUtensorMap& tmap_z,
                                          const CodeMaps& code_maps, const GemvParams& p, const int i0,
@@ -400,8 +433,8 @@ __device__ __forceinline__ void gemv_cta(const CUtensorMap& tmap_q, const CUtens
     if (p.early) {
       StageCursor u = pc;
       for (int s = 0; s < S && !u.done(); ++s) {
-        mbar_arrive_expect_tx(&full[s], stage_tx_bytes(p, u.c.tc, ZP));
-        issue_weights<ZP>(u, ring + s * p.stage_bytes, &full[s], &tmap_q, &tmap_s, &tmap_z, p.scale_offset, p.codes4d ? &code_maps : nullptr);
+        mbar_arrive_expect_tx(&full[s], stage_tx_bytes<ZP, PZ>(p, u.c.tc));
+        issue_weights<ZP, PZ>(u, ring + s * p.stage_bytes, &full[s], &tmap_q, &tmap_s, &tmap_z, p.scale_offset, p.codes4d ? &code_maps : nullptr);
         cursor_next(p, TC, TPU, i1, u);
       }
     } else {
@@ -414,8 +447,8 @@ __device__ __forceinline__ void gemv_cta(const CUtensorMap& tmap_q, const CUtens
       if (w == 0) {
         uint8_t* st = ring + s * p.stage_bytes;
         if (!p.early) {
-          mbar_arrive_expect_tx(&full[s], stage_tx_bytes(p, pc.c.tc, ZP));
-          issue_weights<ZP>(pc, st, &full[s], &tmap_q, &tmap_s, &tmap_z, p.scale_offset, p.codes4d ? &code_maps : nullptr);
+          mbar_arrive_expect_tx(&full[s], stage_tx_bytes<ZP, PZ>(p, pc.c.tc));
+          issue_weights<ZP, PZ>(pc, st, &full[s], &tmap_q, &tmap_s, &tmap_z, p.scale_offset, p.codes4d ? &code_maps : nullptr);
         }
         tma_load_3d(st + p.x_offset, &tmap_x, 0, pc.gbase, 0, &full[s]);
         fills[s] = 1u;
@@ -446,6 +479,7 @@ __device__ __forceinline__ void gemv_cta(const CUtensorMap& tmap_q, const CUtens
   pp.w = w;
   pp.g = g;
   pp.t = t;
+  pp.zsh = 4 * g;
   // x fragment offsets inside a stage ([m][8 groups][128 k]): batch row
   // m = 8 mt + g, this warp's group, chunk 4t + jj
 #pragma unroll
@@ -468,7 +502,7 @@ __device__ __forceinline__ void gemv_cta(const CUtensorMap& tmap_q, const CUtens
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[rt][mt][i] = 0.0f;
 
-    chunk_stages<MT, ZP, TC, TPU>(p, pp, cc, acc, &abort_flag);
+    chunk_stages<MT, ZP, PZ, TC, TPU>(p, pp, cc, acc, &abort_flag);
 
     // ---- chunk reduction: the 8 warps' partial sums meet in shared memory
     // ([warp][row][m], double-buffered by chunk parity) and are summed in
@@ -586,7 +620,7 @@ __device__ __forceinline__ void gemv_cta(const CUtensorMap& tmap_q, const CUtens
   }
 }
 
-template <int MT, bool ZP, int TC, bool SILU>
+template <int MT, bool ZP, bool PZ, int TC, bool SILU>
 __global__ void __launch_bounds__(kThreads, MT == 1 ? 2 : 1)
 gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_x,
             const __grid_constant__ CUtensorMap tmap_s, const __grid_constant__ CUtensorMap tmap_z,
@@ -603,11 +637,11 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
   // share it, so an SM with 3 + 4 tiles finishes sooner than with 4 + 4.
   if constexpr (TC == 4 && !SILU) {
     if (i1 - i0 == 3 && i0 / p.units == (i1 - 1) / p.units) {
-      gemv_cta<MT, ZP, 3, false>(tmap_q, tmap_x, tmap_s, tmap_z, code_maps, p, i0, i1);
+      gemv_cta<MT, ZP, PZ, 3, false>(tmap_q, tmap_x, tmap_s, tmap_z, code_maps, p, i0, i1);
       return;
     }
   }
-  gemv_cta<MT, ZP, TC, SILU>(tmap_q, tmap_x, tmap_s, tmap_z, code_maps, p, i0, i1);
+  gemv_cta<MT, ZP, PZ, TC, SILU>(tmap_q, tmap_x, tmap_s, tmap_z, code_maps, p, i0, i1);
 }
 
 // ---------------------------------------------------------------------------
@@ -621,20 +655,26 @@ struct Variant {
   int mt, id;
 };
 
-constexpr int kNumVariants = 16;
+constexpr int kNumVariants = 24;
 constexpr int kSmemBudget = 232448;   // largest dynamic shared memory of one sm_100 CTA
 constexpr int kHalfSmBudget = 115712; // half of an SM's 228 KB, less the 1 KB reserved per CTA
 
-Variant pick_variant(int64_t M, bool zp, int tc, bool silu) {
+// zp: 0 symmetric, 1 fp16 zero points, 2 packed zero points
+Variant pick_variant(int64_t M, int zp, int tc, bool silu) {
   static const Variant table[kNumVariants] = {
-      {gemv_kernel<1, true, 4, false>, 1, 0},  {gemv_kernel<1, false, 4, false>, 1, 1},
-      {gemv_kernel<2, true, 4, false>, 2, 2},  {gemv_kernel<2, false, 4, false>, 2, 3},
-      {gemv_kernel<1, true, 2, false>, 1, 4},  {gemv_kernel<1, false, 2, false>, 1, 5},
-      {gemv_kernel<2, true, 2, false>, 2, 6},  {gemv_kernel<2, false, 2, false>, 2, 7},
-      {gemv_kernel<1, true, 4, true>, 1, 8},   {gemv_kernel<1, false, 4, true>, 1, 9},
-      {gemv_kernel<2, true, 4, true>, 2, 10},  {gemv_kernel<2, false, 4, true>, 2, 11},
-      {gemv_kernel<1, true, 2, true>, 1, 12},  {gemv_kernel<1, false, 2, true>, 1, 13},
-      {gemv_kernel<2, true, 2, true>, 2, 14},  {gemv_kernel<2, false, 2, true>, 2, 15}};
+      {gemv_kernel<1, true, false, 4, false>, 1, 0},  {gemv_kernel<1, false, false, 4, false>, 1, 1},
+      {gemv_kernel<2, true, false, 4, false>, 2, 2},  {gemv_kernel<2, false, false, 4, false>, 2, 3},
+      {gemv_kernel<1, true, false, 2, false>, 1, 4},  {gemv_kernel<1, false, false, 2, false>, 1, 5},
+      {gemv_kernel<2, true, false, 2, false>, 2, 6},  {gemv_kernel<2, false, false, 2, false>, 2, 7},
+      {gemv_kernel<1, true, false, 4, true>, 1, 8},   {gemv_kernel<1, false, false, 4, true>, 1, 9},
+      {gemv_kernel<2, true, false, 4, true>, 2, 10},  {gemv_kernel<2, false, false, 4, true>, 2, 11},
+      {gemv_kernel<1, true, false, 2, true>, 1, 12},  {gemv_kernel<1, false, false, 2, true>, 1, 13},
+      {gemv_kernel<2, true, false, 2, true>, 2, 14},  {gemv_kernel<2, false, false, 2, true>, 2, 15},
+      {gemv_kernel<1, true, true, 4, false>, 1, 16},  {gemv_kernel<2, true, true, 4, false>, 2, 17},
+      {gemv_kernel<1, true, true, 2, false>, 1, 18},  {gemv_kernel<2, true, true, 2, false>, 2, 19},
+      {gemv_kernel<1, true, true, 4, true>, 1, 20},   {gemv_kernel<2, true, true, 4, true>, 2, 21},
+      {gemv_kernel<1, true, true, 2, true>, 1, 22},   {gemv_kernel<2, true, true, 2, true>, 2, 23}};
+  if (zp == 2) return table[16 + (silu ? 4 : 0) + (tc == 2 ? 2 : 0) + (M <= 8 ? 0 : 1)];
   return table[(silu ? 8 : 0) + (tc == 2 ? 4 : 0) + (M <= 8 ? 0 : 2) + (zp ? 0 : 1)];
 }
 
@@ -651,7 +691,8 @@ constexpr int kMaxDevices = 64;
 std::atomic<int> g_sm_count[kMaxDevices];
 std::atomic<int> g_smem_attr[kMaxDevices][kNumVariants];
 
-awq_status_t make_plan(int64_t M, int64_t N, int64_t K, bool zp, bool silu, Plan& pl) {
+// zp: 0 symmetric, 1 fp16 zero points, 2 packed zero points
+awq_status_t make_plan(int64_t M, int64_t N, int64_t K, int zp, bool silu, Plan& pl) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return AWQ_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return AWQ_ERR_UNSUPPORTED;
@@ -689,7 +730,7 @@ awq_status_t make_plan(int64_t M, int64_t N, int64_t K, bool zp, bool silu, Plan
     pl.tc = most * tpu <= 2 ? 2 : kChunkTiles;
     // Ring geometry: as many stages as the budget holds after the reduction buffers.
     pl.scale_offset = pl.tc * kTileStageBytes;
-    pl.x_offset = pl.scale_offset + kMetaStageBytes * (zp ? 2 : 1);
+    pl.x_offset = pl.scale_offset + kMetaStageBytes + (zp == 2 ? kPackedZeroStageBytes : zp ? kMetaStageBytes : 0);
     pl.stage_bytes = round128(pl.x_offset + int(M) * kXStageBytesPerRow);
     const int budget = per_sm == 2 ? kHalfSmBudget : kSmemBudget;
     const int st = (budget - kRingOffset - pbuf_bytes) / pl.stage_bytes;
@@ -713,12 +754,16 @@ awq_status_t make_plan(int64_t M, int64_t N, int64_t K, bool zp, bool silu, Plan
 awq_status_t check_gemv_args(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
                              const uint16_t* zeros, int64_t M, int64_t N, int64_t K,
                              awq_qconfig_t cfg, uint16_t* y) {
-  awq_status_t st = check_cfg(cfg);
+  awq_status_t st = check_cfg(cfg, true);
   if (st != AWQ_OK) return st;
   if ((st = check_nk(N, K)) != AWQ_OK) return st;
   if (M < 1 || M > 16) return AWQ_ERR_SHAPE;
   if (N % 8) return AWQ_ERR_SHAPE;
   if ((cfg.flags & AWQ_FLAG_SILU_MUL) && N % 32) return AWQ_ERR_SHAPE;
+  if (cfg.flags & AWQ_FLAG_PACKED_ZEROS) {
+    if (!cfg.zero_point) return AWQ_ERR_UNSUPPORTED;
+    if (N % 32) return AWQ_ERR_SHAPE;   // a group row of qzeros is N/2 bytes, whole 16-byte runs
+  }
   if (N == 0) return AWQ_OK;
   if (!x || !qweight || !scales || !y) return AWQ_ERR_NULL;
   if (cfg.zero_point && !zeros) return AWQ_ERR_NULL;
@@ -732,7 +777,7 @@ awq_status_t check_gemv_args(const uint16_t* x, const int32_t* qweight, const ui
 }  // namespace
 
 // Workspace bytes of the GEMV for (M, N, K); used by awq_workspace_bytes.
-awq_status_t gemv_workspace_bytes(int64_t M, int64_t N, int64_t K, bool zp, bool silu, size_t* bytes) {
+awq_status_t gemv_workspace_bytes(int64_t M, int64_t N, int64_t K, int zp, bool silu, size_t* bytes) {
   if (N == 0) { *bytes = 0; return AWQ_OK; }
   Plan pl;
   awq_status_t st = make_plan(M, N, K, zp, silu, pl);
@@ -764,7 +809,7 @@ extern "C" awq_status_t awq_gemv(const uint16_t* x, const int32_t* qweight,
                                  void* workspace, size_t workspace_bytes, void* stream) {
   awq_status_t st = check_gemv_args(x, qweight, scales, zeros, M, N, K, cfg, y);
   if (st != AWQ_OK || N == 0) return st;
-  const bool zp = cfg.zero_point != 0;
+  const int zp = zero_mode(cfg);
   Plan pl;
   if ((st = make_plan(M, N, K, zp, (cfg.flags & AWQ_FLAG_SILU_MUL) != 0, pl)) != AWQ_OK) return st;
   GemvParams p;
@@ -781,7 +826,8 @@ extern "C" awq_status_t awq_gemv(const uint16_t* x, const int32_t* qweight,
   // codes: int32 [N][K/8] viewed as {16 words, N rows, G groups} (a group
   // steps 64 bytes, a row K/2 bytes), boxes of 16 x 16 x 8 that land
   // group-major; x: fp16 [M][K] viewed as {128 k, G groups, M rows}, boxes of
-  // 128 x 8 x M; scales / zeros: fp16 [G][N], boxes of 64 rows x 8 groups.
+  // 128 x 8 x M; scales / zeros: fp16 [G][N], boxes of 64 rows x 8 groups;
+  // packed zero points: int32 [G][N/8], boxes of 12 words x 8 groups.
   CUtensorMap tq, tx, ts, tz;
   if (!make_tensor_map_3d(&tq, CU_TENSOR_MAP_DATA_TYPE_INT32, qweight, kWordsPerGroup, uint64_t(N),
                           uint64_t(G), uint64_t(K / 8) * 4, kWordsPerGroup * 4, kWordsPerGroup, kTile, kWarps) ||
@@ -790,7 +836,11 @@ extern "C" awq_status_t awq_gemv(const uint16_t* x, const int32_t* qweight,
       !make_tensor_map_2d(&ts, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, scales, uint64_t(N), uint64_t(G),
                           uint64_t(N) * 2, kChunkRows, kWarps, CU_TENSOR_MAP_SWIZZLE_NONE))
     return AWQ_ERR_CUDA;
-  if (zp) {
+  if (zp == 2) {
+    if (!make_tensor_map_2d(&tz, CU_TENSOR_MAP_DATA_TYPE_INT32, zeros, uint64_t(N / 8), uint64_t(G),
+                            uint64_t(N) / 2, kPackedZeroWords, kWarps, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return AWQ_ERR_CUDA;
+  } else if (zp) {
     if (!make_tensor_map_2d(&tz, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, zeros, uint64_t(N), uint64_t(G),
                             uint64_t(N) * 2, kChunkRows, kWarps, CU_TENSOR_MAP_SWIZZLE_NONE))
       return AWQ_ERR_CUDA;
@@ -884,7 +934,7 @@ extern "C" awq_status_t awq_gemv_noalloc(const uint16_t* x, const int32_t* qweig
   awq_status_t st = check_gemv_args(x, qweight, scales, zeros, M, N, K, cfg, y);
   if (st != AWQ_OK || N == 0) return st;
   Plan pl;
-  if ((st = make_plan(M, N, K, cfg.zero_point != 0, (cfg.flags & AWQ_FLAG_SILU_MUL) != 0, pl)) != AWQ_OK)
+  if ((st = make_plan(M, N, K, zero_mode(cfg), (cfg.flags & AWQ_FLAG_SILU_MUL) != 0, pl)) != AWQ_OK)
     return st;
   const size_t need = pl.partial_bytes ? pl.counter_bytes + pl.partial_bytes : 0;
   if (need > kStaticScratchBytes) return AWQ_ERR_WORKSPACE;

@@ -64,12 +64,51 @@ quantize_pack_kernel(const uint16_t* __restrict__ W, int64_t N, int64_t K,
   }
 }
 
+// Zero points fp16 [G][N] <-> packed int32 [G][N/8]: word i holds the values
+// 8i .. 8i+7 of the flat array, value 8i + c in bits 4c .. 4c+3. Packing
+// rounds to the nearest integer (ties to even) and clamps to 0..15 (NaN -> 0).
+__global__ void __launch_bounds__(256)
+pack_zeros_kernel(const uint16_t* __restrict__ zeros, int64_t words, int32_t* __restrict__ qzeros) {
+  const int64_t stride = int64_t(gridDim.x) * blockDim.x;
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < words; i += stride) {
+    const uint4 v = *reinterpret_cast<const uint4*>(zeros + i * 8);
+    const uint32_t h[4] = {v.x, v.y, v.z, v.w};
+    uint32_t word = 0;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const float f = half_bits_to_float(uint16_t(h[c >> 1] >> (16 * (c & 1))));
+      const float q = fminf(fmaxf(rintf(f), 0.0f), 15.0f);   // fmaxf(NaN, 0) = 0
+      word |= uint32_t(q) << (4 * c);
+    }
+    qzeros[i] = int32_t(word);
+  }
+}
+
+__global__ void __launch_bounds__(256)
+unpack_zeros_kernel(const int32_t* __restrict__ qzeros, int64_t words, uint16_t* __restrict__ zeros) {
+  const int64_t stride = int64_t(gridDim.x) * blockDim.x;
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < words; i += stride) {
+    const uint32_t word = uint32_t(qzeros[i]);
+    uint32_t h[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) h[c] = __half_as_ushort(__uint2half_rn((word >> (4 * c)) & 0xFu));
+    uint4 v;
+    v.x = h[0] | (h[1] << 16);
+    v.y = h[2] | (h[3] << 16);
+    v.z = h[4] | (h[5] << 16);
+    v.w = h[6] | (h[7] << 16);
+    *reinterpret_cast<uint4*>(zeros + i * 8) = v;
+  }
+}
+
 // One thread per packed word: eight fp16 outputs written as one 16-byte store.
 // w' = fp16((q - z) * s): the fp32 product is exact, so one rounding.
-template <bool ZP>
+// ZP: 0 symmetric (z = 8), 1 fp16 zero points [G][N], 2 packed zero points
+// int32 [G][N/8] (channel n in bits 4 (n % 8) of word n / 8).
+template <int ZP>
 __global__ void __launch_bounds__(256)
 dequant_kernel(const int32_t* __restrict__ qweight, const uint16_t* __restrict__ scales,
-               const uint16_t* __restrict__ zeros, int64_t N, int64_t K,
+               const void* __restrict__ zeros, int64_t N, int64_t K,
                uint16_t* __restrict__ out) {
   const int64_t wpr = K / 8;
   const int64_t words = N * wpr;
@@ -77,9 +116,13 @@ dequant_kernel(const int32_t* __restrict__ qweight, const uint16_t* __restrict__
   for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < words; i += stride) {
     const int64_t n = i / wpr;
     const int64_t wi = i - n * wpr;
-    const int64_t g = ((wi * 8) / kGroup) * N + n;   // group-major metadata
+    const int64_t j = (wi * 8) / kGroup;
+    const int64_t g = j * N + n;   // group-major metadata
     const float sf = half_bits_to_float(scales[g]);
-    const float zf = ZP ? half_bits_to_float(zeros[g]) : 8.0f;
+    float zf = 8.0f;
+    if (ZP == 1) zf = half_bits_to_float(static_cast<const uint16_t*>(zeros)[g]);
+    if (ZP == 2)
+      zf = float((uint32_t(static_cast<const int32_t*>(zeros)[j * (N / 8) + n / 8]) >> (4 * (n % 8))) & 0xFu);
     const uint32_t word = uint32_t(qweight[i]);
     uint32_t h[8];
 #pragma unroll
@@ -137,9 +180,10 @@ extern "C" awq_status_t awq_pseudo_quantize_pack(const uint16_t* W, int64_t N, i
 extern "C" awq_status_t awq_dequant(const int32_t* qweight, const uint16_t* scales,
                                     const uint16_t* zeros, int64_t N, int64_t K,
                                     awq_qconfig_t cfg, uint16_t* W_out, void* stream) {
-  awq_status_t st = check_cfg(cfg);
+  awq_status_t st = check_cfg(cfg, true);
   if (st != AWQ_OK) return st;
   if ((st = check_nk(N, K)) != AWQ_OK) return st;
+  if ((cfg.flags & AWQ_FLAG_PACKED_ZEROS) && N % 8) return AWQ_ERR_SHAPE;
   if (N == 0) return AWQ_OK;
   if (!qweight || !scales || !W_out) return AWQ_ERR_NULL;
   if (cfg.zero_point && !zeros) return AWQ_ERR_NULL;
@@ -149,10 +193,33 @@ extern "C" awq_status_t awq_dequant(const int32_t* qweight, const uint16_t* scal
   const int64_t words = N * (K / 8);
   const int grid = grid_for(words, 1, 256);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cfg.zero_point)
-    dequant_kernel<true><<<grid, 256, 0, s>>>(qweight, scales, zeros, N, K, W_out);
-  else
-    dequant_kernel<false><<<grid, 256, 0, s>>>(qweight, scales, nullptr, N, K, W_out);
+  switch (zero_mode(cfg)) {
+    case 2: dequant_kernel<2><<<grid, 256, 0, s>>>(qweight, scales, zeros, N, K, W_out); break;
+    case 1: dequant_kernel<1><<<grid, 256, 0, s>>>(qweight, scales, zeros, N, K, W_out); break;
+    default: dequant_kernel<0><<<grid, 256, 0, s>>>(qweight, scales, nullptr, N, K, W_out); break;
+  }
+  return launch_status();
+}
+
+extern "C" awq_status_t awq_pack_zeros(const uint16_t* zeros, int64_t G, int64_t N, int32_t* qzeros,
+                                       void* stream) {
+  if (G < 0 || N < 0 || N % 8 || G > (int64_t(1) << 30) || N > (int64_t(1) << 31) - 1) return AWQ_ERR_SHAPE;
+  if (G == 0 || N == 0) return AWQ_OK;
+  if (!zeros || !qzeros) return AWQ_ERR_NULL;
+  if (!aligned16(zeros) || !aligned16(qzeros)) return AWQ_ERR_ALIGN;
+  const int64_t words = G * (N / 8);
+  pack_zeros_kernel<<<grid_for(words, 1, 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(zeros, words, qzeros);
+  return launch_status();
+}
+
+extern "C" awq_status_t awq_unpack_zeros(const int32_t* qzeros, int64_t G, int64_t N, uint16_t* zeros,
+                                         void* stream) {
+  if (G < 0 || N < 0 || N % 8 || G > (int64_t(1) << 30) || N > (int64_t(1) << 31) - 1) return AWQ_ERR_SHAPE;
+  if (G == 0 || N == 0) return AWQ_OK;
+  if (!zeros || !qzeros) return AWQ_ERR_NULL;
+  if (!aligned16(zeros) || !aligned16(qzeros)) return AWQ_ERR_ALIGN;
+  const int64_t words = G * (N / 8);
+  unpack_zeros_kernel<<<grid_for(words, 1, 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(qzeros, words, zeros);
   return launch_status();
 }
 
