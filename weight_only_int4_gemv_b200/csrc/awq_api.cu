@@ -16,7 +16,9 @@ extern "C" const char* awq_status_string(awq_status_t status) {
     case AWQ_ERR_NULL: return "a required pointer is NULL";
     case AWQ_ERR_SHAPE: return "a size is out of range or inconsistent";
     case AWQ_ERR_ALIGN: return "a device pointer is not 16-byte aligned";
-    case AWQ_ERR_UNSUPPORTED: return "configuration not supported (group size must be 128)";
+    case AWQ_ERR_UNSUPPORTED:
+      return "configuration not supported (group size other than 128, zero_point not 0 or 1, an undefined "
+             "flag, or a flag this entry point does not take)";
     case AWQ_ERR_CUDA: return "the CUDA runtime reported an error";
     case AWQ_ERR_WORKSPACE: return "workspace missing or too small";
   }
