@@ -353,30 +353,49 @@ def run_native(args, dist):
     step_flops = sum(algo_flops(M, sh.N, sh.K) for sh in shapes)
     stream = torch.cuda.Stream(device)
 
-    # one CUDA graph per layer copy holding only its GEMV launches, so the
-    # programmatic-dependent-launch edges between consecutive GEMVs survive
+    # CUDA graphs hold only GEMV launches, so the programmatic-dependent-launch
+    # edges between consecutive GEMVs survive capture: one graph per layer copy,
+    # and one over all layer copies in order (a whole model pass, as a decode
+    # loop would capture it), whose edges also link one layer to the next.
+    # Runs of whole passes replay the latter; other steps the per-layer graphs.
+    def run_layer(L):
+        for i in range(len(shapes)):
+            awq.awq_gemv(L.xs[i], *L.packed[i], workspace=L.ws[i], out=L.ys[i], weights_static=True)
+
     graphs = []
     with torch.cuda.stream(stream):
         for L in layers:     # warm the plan caches outside capture
-            for i in range(len(shapes)):
-                awq.awq_gemv(L.xs[i], *L.packed[i], workspace=L.ws[i], out=L.ys[i], weights_static=True)
+            run_layer(L)
         torch.cuda.synchronize(device)
         for L in layers:
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
-                for i in range(len(shapes)):
-                    awq.awq_gemv(L.xs[i], *L.packed[i], workspace=L.ws[i], out=L.ys[i], weights_static=True)
+                run_layer(L)
             graphs.append(g)
+        model_graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(model_graph, stream=stream):
+            for L in layers:
+                run_layer(L)
     torch.cuda.synchronize(device)
+    n = len(graphs)
+
+    def replay_steps(first: int, count: int):
+        """Steps first .. first+count-1; step s runs layer copy s % n."""
+        s, end = first, first + count
+        while s < end:
+            if s % n == 0 and end - s >= n:
+                model_graph.replay()
+                s += n
+            else:
+                graphs[s % n].replay()
+                s += 1
 
     def barrier():
         if dist is not None:
             dist.barrier()
 
-    n = len(graphs)
     with torch.cuda.stream(stream):
-        for s in range(args.warmup):
-            graphs[s % n].replay()
+        replay_steps(0, args.warmup)
     torch.cuda.synchronize(device)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(device.index if device.index is not None else 0)
@@ -385,8 +404,7 @@ def run_native(args, dist):
     with sampler:
         with torch.cuda.stream(stream):
             t0.record()
-            for s in range(args.steps):
-                graphs[(args.warmup + s) % n].replay()
+            replay_steps(args.warmup, args.steps)
             t1.record()
         torch.cuda.synchronize(device)
     barrier()
@@ -438,6 +456,8 @@ def run_native(args, dist):
                 "weights_static": "AWQ_FLAG_WEIGHTS_STATIC set: weights are loaded once, so each GEMV may "
                                   "start streaming them before the previous kernel on the stream finishes",
                 "step": "one layer: one GEMV per listed projection",
+                "graphs": f"runs of {args.layers} steps replay one CUDA graph of all {args.layers} layer "
+                          "copies (a model pass); other steps replay one graph per layer copy",
                 "l2": f"inputs larger than L2: steps rotate over {args.layers} layer copies "
                       f"({args.layers * step_bytes / 1e9:.2f} GB of packed weights)",
                 "parallelism": f"replicas x{ws_}",
