@@ -282,6 +282,22 @@ def cpu_baseline(shapes, M: int, budget_s: float = 10.0, rows: int = 1024):
 # ----------------------------------------------------------------------------
 # native arm
 # ----------------------------------------------------------------------------
+def replay_schedule(first: int, count: int, n: int):
+    """Graph replays for steps first .. first+count-1, where step s runs layer
+    copy s % n: ("pass", 0) replays the graph of all n copies (steps s .. s+n-1,
+    s a multiple of n), ("layer", i) the graph of copy i alone. Covers exactly
+    `count` steps, in order."""
+    out, s, end = [], first, first + count
+    while s < end:
+        if s % n == 0 and end - s >= n:
+            out.append(("pass", 0))
+            s += n
+        else:
+            out.append(("layer", s % n))
+            s += 1
+    return out
+
+
 class DecodeLayer:
     """One layer copy: packed weights of each shape plus its x / y buffers."""
 
@@ -380,15 +396,8 @@ def run_native(args, dist):
     n = len(graphs)
 
     def replay_steps(first: int, count: int):
-        """Steps first .. first+count-1; step s runs layer copy s % n."""
-        s, end = first, first + count
-        while s < end:
-            if s % n == 0 and end - s >= n:
-                model_graph.replay()
-                s += n
-            else:
-                graphs[s % n].replay()
-                s += 1
+        for kind, i in replay_schedule(first, count, n):
+            (model_graph if kind == "pass" else graphs[i]).replay()
 
     def barrier():
         if dist is not None:
