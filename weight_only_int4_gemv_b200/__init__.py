@@ -327,7 +327,9 @@ def awq_gemm(x, qweight, scales, zeros, workspace=None, out=None, group_size: in
 
 def awq_linear(x, qweight, scales, zeros, workspace=None, out=None, group_size: int = GROUP_SIZE,
                weights_static: bool = False, silu_mul: bool = False):
-    """The layer with the documented M threshold: awq_gemv for M <= 16, else awq_gemm."""
+    """The layer with the documented M threshold: awq_gemv for M <= 16, else awq_gemm.
+    Packed zero points (int32 qzeros) are read by awq_gemv only: for M > 16 pass
+    the fp16 form (awq_unpack_zeros), or the call raises AWQ_ERR_UNSUPPORTED."""
     entry = "awq_gemv" if x.shape[0] <= GEMV_MAX_M else "awq_gemm"
     return _product(entry, x, qweight, scales, zeros, workspace, out, group_size,
                     _flags(weights_static, silu_mul))
