@@ -2,6 +2,8 @@
 as the identity, the Gram form of the output error against the direct
 product, and that the search helps on groups with an outlier."""
 
+import os
+
 import numpy as np
 
 from oracle import awq_oracle as O
@@ -44,3 +46,28 @@ def test_search_clips_outlier_groups():
     assert np.mean(ratios[0] < 1.0) > 0.9                  # group 0 is clipped for almost every row
     best = errs.min(axis=0)
     assert np.all(best <= errs[0]) and best[0].sum() < 0.5 * errs[0, 0].sum()
+
+
+def test_clip_grid_hand_worked(golden_dir):
+    """The ratio grid of search_clip against the case worked by hand in
+    search_readings_worked.txt: with n_grid = 4 and max_shrink = 1/2 the grid
+    is 1, 7/8, 3/4, 5/8, and ratio 3/4 puts every weight that matters exactly
+    on the quantization grid (error 0), so every row picks it."""
+    row = None
+    with open(os.path.join(golden_dir, "search_readings_worked.txt")) as f:
+        for line in f:
+            parts = line.split()
+            if parts and parts[0] == "clip":
+                row = parts[1:]
+    n_grid, shrink, outlier, best_i, best_r = int(row[0]), float(row[1]), float(row[2]), int(row[3]), float(row[4])
+    rng = np.random.default_rng(8)
+    N = 16
+    W = (rng.integers(-7, 8, (N, 128)) / 16.0).astype(np.float16)
+    W[:, 0], W[:, 1] = outlier, -outlier
+    X = rng.standard_normal((256, 128)).astype(np.float16)
+    X[:, :2] = 0.0
+    ratios, errs = O.search_clip(W, X, n_grid=n_grid, max_shrink=shrink)
+    assert errs.shape == (n_grid, 1, N)
+    assert np.all(errs[best_i] == 0.0)
+    assert np.all(np.delete(errs, best_i, axis=0) > 0.0)
+    assert np.all(ratios == np.float32(best_r))

@@ -3,6 +3,8 @@ statistics against hand-worked values, the candidate normalisation, the
 alpha = 0 point against plain quantization, the scale invariance it relies
 on, and that the search helps on inputs with salient channels."""
 
+import os
+
 import numpy as np
 
 from oracle import awq_oracle as O
@@ -67,3 +69,54 @@ def test_search_beats_plain_quantization_on_salient_channels():
     plain = O.search_scale(W, X, n_grid=1, duo=False)[1][0]     # alpha = 0, no duo: s = 1
     assert best > 0 and losses[best] == losses.min()
     assert losses[best] < 0.8 * plain
+
+
+def _golden_rows(golden_dir, kind):
+    rows = []
+    with open(os.path.join(golden_dir, "search_readings_worked.txt")) as f:
+        for line in f:
+            parts = line.split()
+            if parts and parts[0] == kind:
+                rows.append(parts[1:])
+    return rows
+
+
+def test_candidates_hand_worked(golden_dir):
+    """candidate_scales against the values worked by hand in
+    search_readings_worked.txt: four channels whose activation and weight
+    statistics are powers of two, at alpha = 1/4 and 1/2, with and without
+    duo scaling. The alpha = 1/4 rows tell the activation exponent alpha from
+    1 - alpha and the weight exponent 1 - alpha from alpha; the duo rows tell
+    dividing by the weight statistic from multiplying by it."""
+    xm = np.array([16.0, 4.0, 1.0, 0.0625], dtype=np.float32)
+    wm = np.array([0.0625, 1.0, 0.25, 1.0], dtype=np.float32)
+    rows = _golden_rows(golden_dir, "candidates")
+    assert len(rows) == 4
+    for alpha, duo, *vals in rows:
+        s = O.candidate_scales(xm, wm, float(alpha), bool(int(duo)))
+        np.testing.assert_allclose(s, np.array(vals, dtype=np.float64), rtol=2e-6,
+                                   err_msg=f"alpha={alpha} duo={duo}")
+
+
+def test_candidate_ratios_do_not_depend_on_the_normalisation():
+    """Between two channels with the same weight statistic the scales differ
+    by exactly (x_i / x_j)^alpha, whatever the normaliser: 16 against 1 at
+    alpha = 1/4 gives 2."""
+    xm = np.array([16.0, 1.0, 3.0], dtype=np.float32)
+    wm = np.array([0.5, 0.5, 0.2], dtype=np.float32)
+    for duo in (False, True):
+        s = O.candidate_scales(xm, wm, 0.25, duo)
+        assert abs(float(s[0]) / float(s[1]) - 2.0) < 1e-6
+
+
+def test_loss_hand_worked(golden_dir):
+    """search_scale's loss at one grid point against the mean square worked by
+    hand (5/8192); a mean absolute difference would give 3/128."""
+    (w0, w1, w2, x0, x1, num, den), = _golden_rows(golden_dir, "loss")
+    W = np.zeros((1, 128), dtype=np.float16)
+    W[0, :3] = [float(w0), float(w1), float(w2)]
+    X = np.zeros((2, 128), dtype=np.float16)
+    X[0, 2], X[1, 2] = float(x0), float(x1)
+    _, losses, best = O.search_scale(W, X, n_grid=1, duo=False)
+    assert best == 0 and losses.shape == (1,)
+    assert losses[0] == int(num) / int(den)
