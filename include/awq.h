@@ -238,8 +238,10 @@ AWQ_API awq_status_t awq_gemv(const uint16_t* x, const int32_t* qweight,
  * cudaFree or any allocating routine. It enqueues a cudaMemsetAsync of the
  * array's counter region and then the GEMV kernel, both on `stream`.
  * The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress) with that device current and caches it; make that
- * first call before any stream capture. All calls on a device share the
+ * (cudaGetSymbolAddress) with that device current and caches it with the
+ * device's current context (a new context after cudaDeviceReset is looked
+ * up again, by its first call); make that first call before any stream
+ * capture. All calls on a device share the
  * array: calls that may overlap on the GPU (different streams, or
  * concurrent host threads) race and must be serialized by the caller.
  */

@@ -259,3 +259,71 @@ def test_binding_refuses_cpu_tensors():
     x = torch.zeros(1, 256, dtype=torch.float16)
     with pytest.raises(ValueError, match="CUDA"):
         awq.awq_gemv(x, torch.zeros(8, 32, dtype=torch.int32), torch.zeros(8, 2, dtype=torch.float16), None)
+
+
+def _layer(M=2, N=64, K=256, device="cpu", packed=False):
+    x = torch.zeros(M, K, dtype=torch.float16, device=device)
+    q = torch.zeros(N, K // 8, dtype=torch.int32, device=device)
+    s = torch.zeros(K // 128, N, dtype=torch.float16, device=device)
+    z = (torch.zeros(K // 128, N // 8, dtype=torch.int32, device=device) if packed
+         else torch.zeros(K // 128, N, dtype=torch.float16, device=device))
+    return x, q, s, z
+
+
+def test_binding_validation_accepts_a_consistent_layer():
+    x, q, s, z = _layer()
+    assert awq.validate_product(x, q, s, z) == (2, 64, 256, 0)
+    assert awq.validate_product(x, q, s, None) == (2, 64, 256, 0)
+    out = torch.zeros(2, 32, dtype=torch.float16)
+    assert awq.validate_product(x, q, s, z, out, flags=awq.FLAG_SILU_MUL)[3] == awq.FLAG_SILU_MUL
+    xp, qp, sp, zp = _layer(packed=True)
+    assert awq.validate_product(xp, qp, sp, zp)[3] == awq.FLAG_PACKED_ZEROS
+
+
+def test_binding_validation_rejects_wrong_out_shape():
+    """An `out` smaller than [M, N] would be written past its end."""
+    x, q, s, z = _layer()
+    for shape in [(2, 32), (1, 64), (2, 65), (64, 2)]:
+        with pytest.raises(ValueError, match="out must be"):
+            awq.validate_product(x, q, s, z, torch.zeros(*shape, dtype=torch.float16))
+    with pytest.raises(ValueError, match="out must be"):      # silu_mul: [M, N/2]
+        awq.validate_product(x, q, s, z, torch.zeros(2, 64, dtype=torch.float16), flags=awq.FLAG_SILU_MUL)
+
+
+def test_binding_validation_rejects_wrong_metadata_shapes():
+    x, q, s, z = _layer()
+    with pytest.raises(ValueError, match="scales"):
+        awq.validate_product(x, q, torch.zeros(1, 64, dtype=torch.float16), z)     # undersized scales
+    with pytest.raises(ValueError):
+        awq.validate_product(x, q, s, torch.zeros(2, 32, dtype=torch.float16))      # undersized zeros
+    with pytest.raises(ValueError):
+        awq.validate_product(x, q, s, torch.zeros(2, 4, dtype=torch.int32))        # undersized qzeros
+    with pytest.raises(ValueError, match="qweight"):
+        awq.validate_product(x, torch.zeros(64, 16, dtype=torch.int32), s, z)
+
+
+def test_binding_validation_rejects_operands_on_another_device():
+    """Operands on different devices would make the kernel read another
+    device's memory; the 'meta' device stands in for a second device here."""
+    x, q, s, z = _layer()
+    xm, qm, sm, zm = _layer(device="meta")
+    out_m = torch.zeros(2, 64, dtype=torch.float16, device="meta")
+    for args in [(x, qm, s, z), (x, q, sm, z), (x, q, s, zm)]:
+        with pytest.raises(ValueError, match="device"):
+            awq.validate_product(*args)
+    with pytest.raises(ValueError, match="device"):
+        awq.validate_product(x, q, s, z, out_m)
+    with pytest.raises(ValueError, match="device"):
+        awq.validate_product(x, q, s, z, workspace=torch.zeros(16, dtype=torch.uint8, device="meta"))
+
+
+def test_noalloc_binding_runs_the_same_checks():
+    """awq_gemv_noalloc goes through the same validation as awq_gemv: with a
+    CUDA-less x it stops at the device check, and its shape checks are those
+    of validate_product (exercised above)."""
+    import inspect
+    src = inspect.getsource(awq.awq_gemv_noalloc)
+    assert "validate_product(" in src
+    x, q, s, z = _layer()
+    with pytest.raises(ValueError, match="CUDA"):
+        awq.awq_gemv_noalloc(x, q, torch.zeros(1, 64, dtype=torch.float16), z)

@@ -70,8 +70,39 @@ def test_noalloc_array_covers_every_shape():
     cap = int(m.group(1)) << int(m.group(2))
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     worst = 0
-    for M in (1, 8, 16):
+    for M in (1, 8, 9, 16):
         for N in (8, 16, 120, 1000, 16 * sms - 8, 16 * sms, 4096, 28672):
             for K in (128, 4096, 28672, 1 << 20):
                 worst = max(worst, awq.awq_workspace_bytes(M, N, K, True))
+                worst = max(worst, awq.awq_workspace_bytes(M, N, K, False))
+                if N % 32 == 0:
+                    # the fused gate/up layout (units of two tiles) and packed zero points
+                    for silu, packed in [(True, False), (False, True), (True, True)]:
+                        worst = max(worst, awq.awq_workspace_bytes(M, N, K, True, silu_mul=silu,
+                                                                   packed_zeros=packed))
     assert 0 < worst <= cap
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("M,packed", [(1, False), (8, True), (16, True)])
+def test_noalloc_fused_gate_up_and_packed_zeros(M, packed):
+    """The fused SiLU epilogue and packed zero points through the fixed array:
+    gate + up of 512 rows each (2N = 1024, fewer tiles than SMs, so K is split
+    across CTAs and the partials go through the array), bit for bit against
+    awq_gemv with a caller workspace on two calls in a row."""
+    N, K = 512, 4096
+    _, qg, sg, zg, _ = oracle_layer(N, K, 0.02, 0.01, True, seed=11)
+    _, qu, su, zu, _ = oracle_layer(N, K, 0.02, 0.01, True, seed=12)
+    q, s, z = awq.awq_interleave_gate_up(dev(qg), dev(sg), dev(zg), dev(qu), dev(su), dev(zu))
+    if packed:
+        z = awq.awq_pack_zeros(z)
+    x = dev(activations(M, K, seed=3))
+    ws = awq.alloc_workspace(M, 2 * N, K, True, silu_mul=True, packed_zeros=packed)
+    assert ws is not None      # the shape does split K
+    ref = host(awq.awq_gemv(x, q, s, z, workspace=ws, silu_mul=True))
+    torch.cuda.synchronize()
+    for call in range(2):
+        y = torch.full((M, N), float("nan"), dtype=torch.float16, device="cuda")
+        awq.awq_gemv_noalloc(x, q, s, z, out=y, silu_mul=True)
+        torch.cuda.synchronize()
+        assert np.array_equal(bits(host(y)), bits(ref)), f"call {call}"

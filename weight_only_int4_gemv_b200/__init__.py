@@ -25,7 +25,7 @@ __all__ = [
     "LIB_PATH", "AwqError", "lib", "GROUP_SIZE",
     "awq_pseudo_quantize_pack", "awq_dequant", "awq_workspace_bytes",
     "awq_gemv", "awq_gemm", "awq_device_error", "awq_linear", "GEMV_MAX_M", "awq_gemv_noalloc",
-    "awq_pack_zeros", "awq_unpack_zeros",
+    "awq_pack_zeros", "awq_unpack_zeros", "validate_product",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libawq_b200.so")
@@ -135,15 +135,32 @@ def _stream(device) -> ctypes.c_void_p:
     return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
 
 
-def _need(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int):
+def _form(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int):
+    """Type, dtype, rank and contiguity of one operand (no device check)."""
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
-    if not t.is_cuda:
-        raise ValueError(f"{name} must be a CUDA tensor (no CPU path exists)")
     if t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
     if t.dim() != ndim or not t.is_contiguous():
         raise ValueError(f"{name} must be a contiguous {ndim}-d tensor")
+
+
+def _need(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int):
+    if isinstance(t, torch.Tensor) and not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (no CPU path exists)")
+    _form(t, name, dtype, ndim)
+
+
+def _same_device(ref: torch.Tensor, **tensors):
+    """Every given tensor (None skipped) must sit on ref's device."""
+    for name, t in tensors.items():
+        if t is not None and t.device != ref.device:
+            raise ValueError(f"{name} is on {t.device}, expected {ref.device}: operands must share a device")
+
+
+def _out_shape(out: torch.Tensor, shape):
+    if tuple(out.shape) != tuple(shape):
+        raise ValueError(f"out must be {list(shape)}, got {list(out.shape)}")
 
 
 def _zeros_flag(zeros, N: int, K: int, group_size: int) -> int:
@@ -152,11 +169,11 @@ def _zeros_flag(zeros, N: int, K: int, group_size: int) -> int:
     if zeros is None:
         return 0
     if isinstance(zeros, torch.Tensor) and zeros.dtype == torch.int32:
-        _need(zeros, "zeros", torch.int32, 2)
+        _form(zeros, "zeros", torch.int32, 2)
         if group_size == GROUP_SIZE and (N % 8 or zeros.shape != (K // group_size, N // 8)):
             raise ValueError("packed zeros must be int32 [K/group_size, N/8]")
         return FLAG_PACKED_ZEROS
-    _need(zeros, "zeros", torch.float16, 2)
+    _form(zeros, "zeros", torch.float16, 2)
     if group_size == GROUP_SIZE and zeros.shape != (K // group_size, N):
         raise ValueError("scales / zeros must be [K/group_size, N]")
     return 0
@@ -173,6 +190,7 @@ def awq_pack_zeros(zeros: torch.Tensor, out: torch.Tensor | None = None) -> torc
     _need(out, "out", torch.int32, 2)
     if out.shape != (G, N // 8):
         raise ValueError("out must be int32 [G, N/8]")
+    _same_device(zeros, out=out)
     with torch.cuda.device(zeros.device):
         _check("awq_pack_zeros", lib().awq_pack_zeros(_ptr(zeros), G, N, _ptr(out), _stream(zeros.device)))
     return out
@@ -187,6 +205,7 @@ def awq_unpack_zeros(qzeros: torch.Tensor, out: torch.Tensor | None = None) -> t
     _need(out, "out", torch.float16, 2)
     if out.shape != (G, N):
         raise ValueError("out must be fp16 [G, N]")
+    _same_device(qzeros, out=out)
     with torch.cuda.device(qzeros.device):
         _check("awq_unpack_zeros", lib().awq_unpack_zeros(_ptr(qzeros), G, N, _ptr(out), _stream(qzeros.device)))
     return out
@@ -219,6 +238,8 @@ def awq_dequant(qweight: torch.Tensor, scales: torch.Tensor, zeros, group_size: 
     if out is None:
         out = torch.empty((N, K), dtype=torch.float16, device=qweight.device)
     _need(out, "out", torch.float16, 2)
+    _out_shape(out, (N, K))
+    _same_device(qweight, scales=scales, zeros=zeros, out=out)
     with torch.cuda.device(qweight.device):
         _check("awq_dequant", lib().awq_dequant(
             _ptr(qweight), _ptr(scales), _ptr(zeros), N, K, _cfg(zeros is not None, group_size, zflag),
@@ -227,28 +248,37 @@ def awq_dequant(qweight: torch.Tensor, scales: torch.Tensor, zeros, group_size: 
 
 
 def awq_workspace_bytes(M: int, N: int, K: int, zero_point: bool = True, group_size: int = GROUP_SIZE,
-                        device=None, silu_mul: bool = False) -> int:
+                        device=None, silu_mul: bool = False, packed_zeros: bool = False) -> int:
     """Workspace bytes awq_gemv / awq_gemm need on `device` for this shape
-    (silu_mul: the fused gate/up layout, N = both projections' rows)."""
+    (silu_mul: the fused gate/up layout, N = both projections' rows;
+    packed_zeros: int32 qzeros, GEMV only)."""
     n = ctypes.c_size_t(0)
+    flags = (FLAG_SILU_MUL if silu_mul else 0) | (FLAG_PACKED_ZEROS if packed_zeros else 0)
     with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
         _check("awq_workspace_bytes", lib().awq_workspace_bytes(
-            M, N, K, _cfg(zero_point, group_size, FLAG_SILU_MUL if silu_mul else 0), ctypes.byref(n)))
+            M, N, K, _cfg(zero_point, group_size, flags), ctypes.byref(n)))
     return int(n.value)
 
 
 def alloc_workspace(M: int, N: int, K: int, zero_point: bool = True, device=None,
-                    silu_mul: bool = False) -> torch.Tensor | None:
+                    silu_mul: bool = False, packed_zeros: bool = False) -> torch.Tensor | None:
     """Zero-filled workspace for (M, N, K), or None when none is needed."""
     dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
-    nbytes = awq_workspace_bytes(M, N, K, zero_point, device=dev, silu_mul=silu_mul)
+    nbytes = awq_workspace_bytes(M, N, K, zero_point, device=dev, silu_mul=silu_mul, packed_zeros=packed_zeros)
     return torch.zeros(nbytes, dtype=torch.uint8, device=dev) if nbytes else None
 
 
-def _product(entry: str, x, qweight, scales, zeros, workspace, out, group_size, flags=0):
-    _need(x, "x", torch.float16, 2)
-    _need(qweight, "qweight", torch.int32, 2)
-    _need(scales, "scales", torch.float16, 2)
+def validate_product(x, qweight, scales, zeros, out=None, workspace=None, group_size: int = GROUP_SIZE,
+                     flags: int = 0):
+    """The host-side checks every product entry point runs before it calls the
+    library: dtypes, ranks, contiguity, the shapes of qweight [N, K/8],
+    scales [K/g, N], zeros (fp16 [K/g, N] or int32 [K/g, N/8]) and out
+    ([M, N], or [M, N/2] with FLAG_SILU_MUL), and that every operand sits on
+    x's device. Touches no device. Returns (M, N, K, flags) with the packed
+    zero-point flag added when zeros is int32."""
+    _form(x, "x", torch.float16, 2)
+    _form(qweight, "qweight", torch.int32, 2)
+    _form(scales, "scales", torch.float16, 2)
     M, K = x.shape
     N = qweight.shape[0]
     if qweight.shape[1] * 8 != K:
@@ -256,13 +286,28 @@ def _product(entry: str, x, qweight, scales, zeros, workspace, out, group_size, 
     flags |= _zeros_flag(zeros, N, K, group_size)
     if group_size == GROUP_SIZE and scales.shape != (K // group_size, N):
         raise ValueError("scales / zeros must be [K/group_size, N]")
+    if out is not None:
+        _form(out, "out", torch.float16, 2)
+        want = (M, N // 2 if flags & FLAG_SILU_MUL else N)
+        if tuple(out.shape) != want:
+            raise ValueError(f"out must be [{want[0]}, {want[1]}], got {list(out.shape)}")
+    if workspace is not None:
+        if not isinstance(workspace, torch.Tensor) or not workspace.is_contiguous():
+            raise ValueError("workspace must be a contiguous tensor")
+    for name, t in (("qweight", qweight), ("scales", scales), ("zeros", zeros), ("out", out),
+                    ("workspace", workspace)):
+        if t is not None and t.device != x.device:
+            raise ValueError(f"{name} is on {t.device}, x on {x.device}: every operand must be on x's device")
+    return M, N, K, flags
+
+
+def _product(entry: str, x, qweight, scales, zeros, workspace, out, group_size, flags=0):
+    _need(x, "x", torch.float16, 2)
+    M, N, K, flags = validate_product(x, qweight, scales, zeros, out, workspace, group_size, flags)
     if out is None:
         out = torch.empty((M, N // 2 if flags & FLAG_SILU_MUL else N), dtype=torch.float16, device=x.device)
-    _need(out, "out", torch.float16, 2)
     ws_ptr, ws_bytes = None, 0
     if workspace is not None:
-        if not workspace.is_cuda or not workspace.is_contiguous():
-            raise ValueError("workspace must be a contiguous CUDA tensor")
         ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
     fn = getattr(lib(), entry)
     dev = x.device
@@ -300,21 +345,14 @@ def awq_gemv_noalloc(x, qweight, scales, zeros, out=None, group_size: int = GROU
     for callers that cannot allocate device memory when they run the layer.
     Calls on one device share the array and must not overlap on the GPU."""
     _need(x, "x", torch.float16, 2)
-    _need(qweight, "qweight", torch.int32, 2)
-    _need(scales, "scales", torch.float16, 2)
-    M, K = x.shape
-    N = qweight.shape[0]
-    if qweight.shape[1] * 8 != K:
-        raise ValueError("qweight must be [N, K/8] for x [M, K]")
-    zflag = _zeros_flag(zeros, N, K, group_size)
+    M, N, K, flags = validate_product(x, qweight, scales, zeros, out, None, group_size,
+                                      _flags(weights_static, silu_mul))
     if out is None:
         out = torch.empty((M, N // 2 if silu_mul else N), dtype=torch.float16, device=x.device)
-    _need(out, "out", torch.float16, 2)
     with torch.cuda.device(x.device):
         _check("awq_gemv_noalloc", lib().awq_gemv_noalloc(
             _ptr(x), _ptr(qweight), _ptr(scales), _ptr(zeros), M, N, K,
-            _cfg(zeros is not None, group_size, _flags(weights_static, silu_mul) | zflag),
-            _ptr(out), _stream(x.device)))
+            _cfg(zeros is not None, group_size, flags), _ptr(out), _stream(x.device)))
     return out
 
 
@@ -413,6 +451,7 @@ def awq_search_scale(W: torch.Tensor, X: torch.Tensor, zero_point: bool = True, 
     Ms = X.shape[0]
     if X.shape[1] != K:
         raise ValueError("X must be [Ms, K] for W [N, K]")
+    _same_device(W, X=X)
     cfg = _cfg(zero_point, group_size)
     n = ctypes.c_size_t(0)
     with torch.cuda.device(W.device):
@@ -436,6 +475,9 @@ def awq_apply_scale(W: torch.Tensor, scales: torch.Tensor, out: torch.Tensor | N
         raise ValueError("scales must be [K]")
     if out is None:
         out = torch.empty_like(W)
+    _need(out, "out", torch.float16, 2)
+    _out_shape(out, (N, K))
+    _same_device(W, scales=scales, out=out)
     with torch.cuda.device(W.device):
         _check("awq_apply_scale", lib().awq_apply_scale(_ptr(W), _ptr(scales), N, K, _ptr(out), _stream(W.device)))
     return out
@@ -450,6 +492,7 @@ def awq_search_clip(W: torch.Tensor, X: torch.Tensor, zero_point: bool = True, n
     N, K = W.shape
     if X.shape[1] != K:
         raise ValueError("X must be [Ms, K] for W [N, K]")
+    _same_device(W, X=X)
     n = ctypes.c_size_t(0)
     with torch.cuda.device(W.device):
         _check("awq_search_clip_workspace_bytes", lib().awq_search_clip_workspace_bytes(K, ctypes.byref(n)))
@@ -470,6 +513,9 @@ def awq_apply_clip(W: torch.Tensor, ratios: torch.Tensor, out: torch.Tensor | No
         raise ValueError("ratios must be [K/128, N]")
     if out is None:
         out = torch.empty_like(W)
+    _need(out, "out", torch.float16, 2)
+    _out_shape(out, (N, K))
+    _same_device(W, ratios=ratios, out=out)
     with torch.cuda.device(W.device):
         _check("awq_apply_clip", lib().awq_apply_clip(_ptr(W), _ptr(ratios), N, K, _ptr(out), _stream(W.device)))
     return out

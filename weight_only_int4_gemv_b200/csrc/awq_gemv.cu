@@ -59,6 +59,7 @@
 //   flight. The output is then incomplete.
 
 #include <atomic>
+#include <mutex>
 
 #include "awq_common.cuh"
 #include "awq_tma_host.h"
@@ -907,20 +908,46 @@ constexpr size_t kStaticScratchBytes = AWQ_GEMV_STATIC_WORKSPACE_BYTES;
 // a device share it.
 static __device__ __align__(256) uint8_t g_gemv_scratch[kStaticScratchBytes];
 
-std::atomic<uintptr_t> g_scratch_addr[kMaxDevices];
+// The cached device address of g_gemv_scratch per device, with the context it
+// was looked up in: a context that is torn down and created again (for
+// example after cudaDeviceReset) maps the array elsewhere.
+struct ScratchCache {
+  std::mutex lock;
+  CUcontext ctx = nullptr;
+  uintptr_t addr = 0;
+};
+ScratchCache g_scratch[kMaxDevices];
+
+PFN_cuCtxGetCurrent_v4000 ctx_getter() {
+  static PFN_cuCtxGetCurrent_v4000 fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<PFN_cuCtxGetCurrent_v4000>(nullptr);
+    return reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f);
+  }();
+  return fn;
+}
 
 // Device address of g_gemv_scratch on the current device. In host code the
-// array's name is only a host-side stand-in, so the address is looked up once
-// per device (with that device current) and cached.
+// array's name is only a host-side stand-in, so the address is looked up
+// (with that device current) and cached per device and context.
 awq_status_t scratch_address(int dev, void** out) {
-  uintptr_t a = g_scratch_addr[dev].load(std::memory_order_acquire);
-  if (a == 0) {
+  PFN_cuCtxGetCurrent_v4000 get = ctx_getter();
+  CUcontext ctx = nullptr;
+  if (!get || get(&ctx) != CUDA_SUCCESS) return AWQ_ERR_CUDA;
+  ScratchCache& c = g_scratch[dev];
+  std::lock_guard<std::mutex> g(c.lock);
+  if (ctx == nullptr || c.addr == 0 || c.ctx != ctx) {
+    // the lookup also makes the device's primary context current if it was not
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_gemv_scratch) != cudaSuccess || p == nullptr) return AWQ_ERR_CUDA;
-    a = reinterpret_cast<uintptr_t>(p);
-    g_scratch_addr[dev].store(a, std::memory_order_release);
+    if (get(&ctx) != CUDA_SUCCESS || ctx == nullptr) return AWQ_ERR_CUDA;
+    c.addr = reinterpret_cast<uintptr_t>(p);
+    c.ctx = ctx;
   }
-  *out = reinterpret_cast<void*>(a);
+  *out = reinterpret_cast<void*>(c.addr);
   return AWQ_OK;
 }
 
