@@ -47,6 +47,7 @@ METRIC = "W4A16 GEMV/GEMM TFLOP/s and effective HBM GB/s (fraction of roofline),
 HBM_FALLBACK_GBS = 6650.0
 TENSOR_FALLBACK_TFLOPS = 1590.0
 GEMV_PROFILE = os.path.join(ROOT, "profiles", "awq_gemv_llama3_8b_decode_m1.md")
+CHAIN_PROFILE = os.path.join(ROOT, "profiles", "awq_gemv_chain_llama3_8b_decode_m1.md")
 GEMM_PROFILE = os.path.join(ROOT, "profiles", "awq_gemm_prefill_m2048.md")
 
 
@@ -282,34 +283,31 @@ def cpu_baseline(shapes, M: int, budget_s: float = 10.0, rows: int = 1024):
 # ----------------------------------------------------------------------------
 # native arm
 # ----------------------------------------------------------------------------
-def replay_schedule(first: int, count: int, n: int):
-    """Graph replays for steps first .. first+count-1, where step s runs layer
-    copy s % n: ("pass", 0) replays the graph of all n copies (steps s .. s+n-1,
-    s a multiple of n), ("layer", i) the graph of copy i alone. Covers exactly
-    `count` steps, in order."""
-    out, s, end = [], first, first + count
-    while s < end:
-        if s % n == 0 and end - s >= n:
-            out.append(("pass", 0))
-            s += n
-        else:
-            out.append(("layer", s % n))
-            s += 1
-    return out
+def chain_sources(shapes):
+    """Per layer of a decode step, the earlier layer whose output is its input
+    (-1: the step's input): the most recent earlier layer with as many output
+    channels as this layer has input channels. For the Llama-3-8B layer:
+    q_proj on the step's input, gate_proj and up_proj on q_proj's output,
+    down_proj on up_proj's output."""
+    src = []
+    for i, sh in enumerate(shapes):
+        j = next((j for j in range(i - 1, -1, -1) if shapes[j].N == sh.K), -1)
+        src.append(j)
+    return src
 
 
 class DecodeLayer:
-    """One layer copy: packed weights of each shape plus its x / y buffers."""
+    """One layer copy: packed weights of each shape, the step's input x and
+    its prepared chain call (outputs and workspace allocated)."""
 
-    def __init__(self, packed, xs, ys, workspaces, x_all, y_all):
-        self.packed, self.xs, self.ys, self.ws = packed, xs, ys, workspaces
-        self.x_all, self.y_all = x_all, y_all   # the xs / ys are contiguous views of these
+    def __init__(self, packed, x, chain, per_gemv):
+        self.packed, self.x, self.chain, self.per_gemv = packed, x, chain, per_gemv
 
 
 def build_decode(awq, torch, device, shapes, M: int, n_layers: int, zp: bool):
     """Quantize each shape on the GPU (recipe W, seed 0; the second, warm call
     is timed), then clone the packed tensors into n_layers copies at distinct
-    addresses."""
+    addresses, each with its own input and a prepared chain call."""
     base, quant_ms, quant_bytes = [], 0.0, 0
     for sh in shapes:
         W = torch.from_numpy(make_weight(sh.N, sh.K, 0.02, 0.01, seed=0)).to(device)
@@ -327,22 +325,22 @@ def build_decode(awq, torch, device, shapes, M: int, n_layers: int, zp: bool):
         base.append((q, s, z))
         del W
     rng = np.random.default_rng(1)
+    src = chain_sources(shapes)
     layers = []
     for _ in range(n_layers):
         packed = [(q.clone(), s.clone(), z.clone() if z is not None else None) for q, s, z in base]
-        # each layer's inputs (outputs) are consecutive views of one buffer, so the
-        # end-to-end leg moves them with one copy each way
-        x_all = torch.from_numpy(np.concatenate(
-            [rng.standard_normal((M, sh.K), dtype=np.float32).astype(np.float16).ravel() for sh in shapes])).to(device)
-        y_all = torch.empty(sum(M * sh.N for sh in shapes), dtype=torch.float16, device=device)
-        xs, ys, ox, oy = [], [], 0, 0
-        for sh in shapes:
-            xs.append(x_all[ox:ox + M * sh.K].view(M, sh.K))
-            ys.append(y_all[oy:oy + M * sh.N].view(M, sh.N))
-            ox += M * sh.K
-            oy += M * sh.N
+        x = torch.from_numpy(rng.standard_normal((M, shapes[0].K), dtype=np.float32).astype(np.float16)).to(device)
+        specs = [dict(x=x if src[i] < 0 else None, x_from=src[i], qweight=q, scales=s, zeros=z)
+                 for i, (q, s, z) in enumerate(packed)]
+        chain = awq.GemvChain(M, specs, weights_static=True)
+        # the same products as separate awq_gemv launches (for --per-gemv)
         wss = [awq.alloc_workspace(M, sh.N, sh.K, zp, device=device) for sh in shapes]
-        layers.append(DecodeLayer(packed, xs, ys, wss, x_all, y_all))
+
+        def per_gemv(chain=chain, packed=packed, wss=wss, x=x):
+            for i in range(len(packed)):
+                xin = x if src[i] < 0 else chain.outputs[src[i]]
+                awq.awq_gemv(xin, *packed[i], workspace=wss[i], out=chain.outputs[i], weights_static=True)
+        layers.append(DecodeLayer(packed, x, chain, per_gemv))
     return layers, {"ms": round(quant_ms, 4), "GB/s": round(quant_bytes / (quant_ms * 1e-3) / 1e9, 1)}
 
 
@@ -368,43 +366,37 @@ def run_native(args, dist):
     step_bytes = sum(algo_bytes(M, sh.N, sh.K, zp) for sh in shapes)
     step_flops = sum(algo_flops(M, sh.N, sh.K) for sh in shapes)
     stream = torch.cuda.Stream(device)
+    n = len(layers)
+    launches_per_step = len(shapes) if args.per_gemv else 1
 
-    # CUDA graphs hold only GEMV launches, so the programmatic-dependent-launch
-    # edges between consecutive GEMVs survive capture: one graph per layer copy,
-    # and one over all layer copies in order (a whole model pass, as a decode
-    # loop would capture it), whose edges also link one layer to the next.
-    # Runs of whole passes replay the latter; other steps the per-layer graphs.
-    def run_layer(L):
-        for i in range(len(shapes)):
-            awq.awq_gemv(L.xs[i], *L.packed[i], workspace=L.ws[i], out=L.ys[i], weights_static=True)
+    def step(i):
+        L = layers[i % n]
+        L.per_gemv() if args.per_gemv else L.chain()
 
-    graphs = []
+    # Each run of steps is replayed from one CUDA graph holding exactly those
+    # steps (step i on layer copy i % n), so consecutive launches stay linked
+    # by programmatic dependent launch whatever the number of steps.
+    def capture(first, count):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(first, first + count):
+                step(i)
+        return g
+
     with torch.cuda.stream(stream):
-        for L in layers:     # warm the plan caches outside capture
-            run_layer(L)
-        torch.cuda.synchronize(device)
-        for L in layers:
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                run_layer(L)
-            graphs.append(g)
-        model_graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(model_graph, stream=stream):
-            for L in layers:
-                run_layer(L)
+        for i in range(n):            # warm the plan caches outside capture
+            step(i)
     torch.cuda.synchronize(device)
-    n = len(graphs)
-
-    def replay_steps(first: int, count: int):
-        for kind, i in replay_schedule(first, count, n):
-            (model_graph if kind == "pass" else graphs[i]).replay()
+    g_warm = capture(0, args.warmup)
+    g_timed = capture(args.warmup, args.steps)
+    torch.cuda.synchronize(device)
 
     def barrier():
         if dist is not None:
             dist.barrier()
 
     with torch.cuda.stream(stream):
-        replay_steps(0, args.warmup)
+        g_warm.replay()
     torch.cuda.synchronize(device)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(device.index if device.index is not None else 0)
@@ -413,16 +405,18 @@ def run_native(args, dist):
     with sampler:
         with torch.cuda.stream(stream):
             t0.record()
-            replay_steps(args.warmup, args.steps)
+            g_timed.replay()
             t1.record()
         torch.cuda.synchronize(device)
     barrier()
     elapsed_s = t0.elapsed_time(t1) * 1e-3
+    dev_err = awq.awq_device_error(device)
+    del g_warm, g_timed
 
-    # Every launch in the timed region is a GEMV and consecutive launches
-    # overlap (programmatic dependent launch), so the kernel's average launch
-    # duration is the timed region over the launches in it.
-    n_launch = args.steps * len(shapes)
+    # Every launch in the timed region is one of this library's products and
+    # consecutive launches overlap (programmatic dependent launch), so the
+    # kernel's average launch duration is the timed region over its launches.
+    n_launch = args.steps * launches_per_step
     mean_launch_s = elapsed_s / n_launch
     kernel_gbs = step_bytes * args.steps / elapsed_s / 1e9
 
@@ -443,8 +437,10 @@ def run_native(args, dist):
         cpu = cpu_baseline(shapes, M, budget_s=args.cpu_seconds)
 
     if rank == 0:
-        gemv_src = os.path.join(ROOT, "weight_only_int4_gemv_b200", "csrc", "awq_gemv.cu")
-        traffic = profile_traffic(GEMV_PROFILE, gemv_src)
+        src_file = "awq_gemv.cu" if args.per_gemv else "awq_gemv_chain.cu"
+        kern_src = os.path.join(ROOT, "weight_only_int4_gemv_b200", "csrc", src_file)
+        traffic = profile_traffic(GEMV_PROFILE if args.per_gemv else CHAIN_PROFILE, kern_src)
+        deps = chain_sources(shapes)
         line = {
             "metric": METRIC,
             "value": round(value, 2),
@@ -460,13 +456,16 @@ def run_native(args, dist):
             "data": "synthetic (seeded N(0,0.02) weights, 1% salient input channels x10, N(0,1) x; no checkpoint)",
             "config": {
                 "workload": f"{args.workload}_m{M}",
-                "layers": [f"{sh.name} {sh.N}x{sh.K}" for sh in shapes],
+                "layers": [f"{sh.name} {sh.N}x{sh.K}" + (f" (x = {shapes[d].name} output)" if d >= 0 else " (x = step input)")
+                           for sh, d in zip(shapes, deps)],
                 "M": M, "group_size": 128, "zero_point": zp,
-                "weights_static": "AWQ_FLAG_WEIGHTS_STATIC set: weights are loaded once, so each GEMV may "
+                "weights_static": "AWQ_FLAG_WEIGHTS_STATIC set: weights are loaded once, so a launch may "
                                   "start streaming them before the previous kernel on the stream finishes",
-                "step": "one layer: one GEMV per listed projection",
-                "graphs": f"runs of {args.layers} steps replay one CUDA graph of all {args.layers} layer "
-                          "copies (a model pass); other steps replay one graph per layer copy",
+                "step": ("one layer: one awq_gemv launch per listed projection" if args.per_gemv else
+                         "one layer: one awq_gemv_chain launch of the listed projections, each reading its "
+                         "input only after the projection it comes from is complete"),
+                "graphs": "the warm-up steps and the timed steps are each replayed from one CUDA graph "
+                          "holding exactly those steps",
                 "l2": f"inputs larger than L2: steps rotate over {args.layers} layer copies "
                       f"({args.layers * step_bytes / 1e9:.2f} GB of packed weights)",
                 "parallelism": f"replicas x{ws_}",
@@ -476,17 +475,19 @@ def run_native(args, dist):
                 "bound": "hbm", "achieved": round(kernel_gbs, 1), "peak": hbm_peak, "unit": "GB/s",
                 "frac": round(kernel_gbs / hbm_peak, 4),
                 "traffic": traffic, "peak_source": peak_src,
-                "kernel": "awq_gemv (gemv_kernel<1, true>: M tile 1, asymmetric)",
+                "kernel": ("awq_gemv (gemv_kernel, M tile 1, asymmetric)" if args.per_gemv else
+                           "awq_gemv_chain (chain_kernel<1, 1>: M = 1, fp16 zero points)"),
                 "launches_timed": n_launch,
-                "algorithmic_bytes_per_launch": round(step_bytes / len(shapes)),
+                "algorithmic_bytes_per_launch": round(step_bytes / launches_per_step),
                 "mean_launch_us": round(1e6 * mean_launch_s, 3),
                 "duration_source": "CUDA events around the timed steps on the launch stream / launches",
                 "frac_of_nominal_8TBs": round(kernel_gbs / 8000.0, 4),
             },
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": args.steps * len(shapes),
+            "gpu_launches": n_launch,
             "clocks": sampler.summary(),
+            "device_error": dev_err,
             "quantize": quant,
         }
         if gemm is not None:
@@ -498,22 +499,22 @@ def run_native(args, dist):
 
 def run_e2e(awq, torch, device, stream, layers, shapes, M, args, dist, step_bytes):
     """Same metric through the Python API with host buffers: every step copies
-    its inputs (all projections' x, one pinned buffer) to the device, runs the
-    GEMVs, reads all their y back into pinned host memory, then synchronizes."""
+    its input x from pinned host memory to the device, runs the layer (the
+    prepared chain call), reads the layer's result (the last projection's
+    output) back into pinned host memory, then synchronizes."""
     steps = max(1, min(args.steps, args.e2e_steps))
-    hx = torch.empty_like(layers[0].x_all, device="cpu").pin_memory()
-    hy = torch.empty_like(layers[0].y_all, device="cpu").pin_memory()
-    hx.copy_(layers[0].x_all.cpu())
+    hx = torch.empty_like(layers[0].x, device="cpu").pin_memory()
+    hy = torch.empty_like(layers[0].chain.outputs[-1], device="cpu").pin_memory()
+    hx.copy_(layers[0].x.cpu())
     h2d = hx.numel() * 2
     d2h = hy.numel() * 2
     n = len(layers)
 
     def step(s):
         L = layers[s % n]
-        L.x_all.copy_(hx, non_blocking=True)
-        for i in range(len(shapes)):
-            awq.awq_gemv(L.xs[i], *L.packed[i], workspace=L.ws[i], out=L.ys[i], weights_static=True)
-        hy.copy_(L.y_all, non_blocking=True)
+        L.x.copy_(hx, non_blocking=True)
+        L.per_gemv() if args.per_gemv else L.chain()
+        hy.copy_(L.chain.outputs[-1], non_blocking=True)
         torch.cuda.current_stream(device).synchronize()
 
     with torch.cuda.stream(stream):
@@ -743,7 +744,7 @@ def run_table(args):
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=64)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--workload", choices=["llama3_8b_decode", "decode_sweep"], default="llama3_8b_decode")
@@ -754,6 +755,8 @@ def parse_args(argv=None):
     ap.add_argument("--ref-rows", type=int, default=256)
     ap.add_argument("--no-gemm", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--per-gemv", action="store_true",
+                    help="run each projection as its own awq_gemv launch instead of one awq_gemv_chain per step")
     ap.add_argument("--table", action="store_true",
                     help="instead of the bench line: per (shape, M) GEMV / GEMM times, one JSON line each")
     a = ap.parse_args(argv)

@@ -63,7 +63,7 @@
 extern "C" {
 #endif
 
-#define AWQ_ABI_VERSION 6
+#define AWQ_ABI_VERSION 7
 
 #if defined(__GNUC__)
 #define AWQ_API __attribute__((visibility("default")))
@@ -252,6 +252,72 @@ AWQ_API awq_status_t awq_gemv_noalloc(const uint16_t* x, const int32_t* qweight,
                                       uint16_t* y, void* stream);
 
 /*
+ * awq_gemv_chain -- several decode products in one launch, where a layer's
+ * input may be the output of an earlier layer of the same call.
+ * ("AutoAWQ" code tour, "The big picture": the GEMV kernel for single-token
+ * decoding; "AutoAWQ" capability page, WQLinear paragraph: the INT4 layer is
+ * bound by memory at small batch, and fused-blocks paragraph: fused blocks
+ * save launches.)
+ *
+ * For l = 0 .. n_layers - 1, in order:
+ *   layers[l].y[M][N_l] = layers[l].x[M][K_l] . W_l'^T
+ * with the arithmetic, results and flags of awq_gemv (AWQ_FLAG_SILU_MUL:
+ * y is [M][N_l/2]). The results are bit-identical to n_layers awq_gemv
+ * calls made in order on the same stream whenever each layer's split of K
+ * is the same (it is whenever N_l / 16 is at least twice the SM count).
+ * The launch streams the weights of all layers back to back; a layer's x
+ * is read only after the layer it comes from is complete.
+ *
+ * x_from = -1: x is ready when the call starts (written by earlier work on
+ * the stream). x_from = d (0 <= d < l): x is layer d's y of this call; x
+ * must then equal layers[d].y and K_l the column count of that y.
+ * A layer's y must not overlap any other layer's x or y, except as the x
+ * of the layers that name it in x_from.
+ * 1 <= n_layers <= AWQ_CHAIN_MAX_LAYERS; 1 <= M <= 16; per layer: N >= 8,
+ * N % 8 == 0 (N % 32 with AWQ_FLAG_SILU_MUL or AWQ_FLAG_PACKED_ZEROS);
+ * K % 128 == 0; every layer has the same zero-point form (symmetric, fp16
+ * zeros or packed zeros); pointers 16-byte aligned. The weights may be read
+ * before the kernel launched just before this one on the stream has
+ * finished only if every layer carries AWQ_FLAG_WEIGHTS_STATIC.
+ * layers: host memory, read before the call returns.
+ * workspace: at least awq_gemv_chain_workspace_bytes() bytes of device
+ * memory, zero-filled before its first use; every call that completes (also
+ * one whose waits gave up, see awq_device_error) leaves it zero-filled.
+ * Calls that may run concurrently need separate workspaces.
+ * Every CTA of the launch must be resident at once (the grid is sized from
+ * the occupancy of the kernel on this device): do not run other kernels
+ * concurrently on the same device that could hold SMs for a long time, or
+ * the dependency waits reach their time limit and the call gives up
+ * (reported by awq_device_error, bit 2).
+ */
+#define AWQ_CHAIN_MAX_LAYERS 8
+typedef struct awq_gemv_layer {
+  const uint16_t* x;        /* [M][K] fp16 */
+  const int32_t* qweight;   /* [N][K/8] */
+  const uint16_t* scales;   /* [K/128][N] fp16 */
+  const uint16_t* zeros;    /* [K/128][N] fp16, int32 [K/128][N/8] with
+                               AWQ_FLAG_PACKED_ZEROS, or NULL (symmetric) */
+  uint16_t* y;              /* [M][N] fp16 ([M][N/2] with AWQ_FLAG_SILU_MUL) */
+  int64_t N, K;
+  awq_qconfig_t cfg;
+  int32_t x_from;           /* -1, or the index of the layer whose y x is */
+} awq_gemv_layer_t;
+
+AWQ_API awq_status_t awq_gemv_chain_workspace_bytes(const awq_gemv_layer_t* layers, int n_layers,
+                                                    int64_t M, size_t* bytes);
+AWQ_API awq_status_t awq_gemv_chain(const awq_gemv_layer_t* layers, int n_layers, int64_t M,
+                                    void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * awq_debug_set_wait_limit_ns -- test hook: the time limit after which a
+ * pipeline wait inside awq_gemv_chain gives up (0 restores the default of
+ * 2 s; at most 2 s). Copies already in flight are always waited for with
+ * the full limit. Synchronizes `stream`. The pages have no counterpart; it
+ * exists so that tests can make a wait run out without a fault.
+ */
+AWQ_API awq_status_t awq_debug_set_wait_limit_ns(uint64_t ns, void* stream);
+
+/*
  * awq_gemm -- y[M][N] = x[M][K] . W'^T for any M >= 1 (prefill).
  * ("AutoAWQ" code tour, "The big picture": the GEMM variant for batched
  * requests; "AWQ Quantization Support", "Integration with Forward Pass":
@@ -375,7 +441,8 @@ AWQ_API awq_status_t awq_apply_clip(const uint16_t* W, const float* ratios, int6
  * awq_device_error -- read and clear the device-side error word of the
  * current device (synchronizes `stream`). Bit 0: a pipeline wait inside
  * awq_gemm passed its time limit (2 s) and the kernel abandoned its tiles;
- * bit 1: the same inside awq_gemv. The output is then incomplete. 0 means
+ * bit 1: the same inside awq_gemv; bit 2: a pipeline or dependency wait
+ * inside awq_gemv_chain. The output is then incomplete. 0 means
  * no error was recorded. No kernel traps: a wait that gives up records the
  * bit, lets its copies in flight land, frees what it holds and returns.
  */

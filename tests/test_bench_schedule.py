@@ -1,36 +1,32 @@
-"""The decode bench's graph replay schedule: exactly the requested steps, in
-layer order, with whole model passes only where they start on a pass."""
+"""The decode bench's step structure: which projection of a layer reads which
+one's output (host logic, no GPU)."""
 import os
 import sys
-
-import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 import bench  # noqa: E402
+from workloads import LLAMA3_8B_DECODE, WORKLOADS, LayerShape  # noqa: E402
 
 
-def _expand(schedule, n):
-    steps = []
-    for kind, i in schedule:
-        steps.extend(range(n) if kind == "pass" else [i])
-    return steps
+def test_llama3_8b_layer_dependencies():
+    # q_proj on the step input; gate_proj and up_proj on q_proj's output;
+    # down_proj on up_proj's output
+    assert bench.chain_sources(LLAMA3_8B_DECODE) == [-1, 0, 0, 2]
 
 
-@pytest.mark.parametrize("first,count,n", [(0, 64, 32), (64, 3000, 32), (3, 40, 32), (1, 2, 32),
-                                           (64, 20, 32), (5, 100, 7), (0, 0, 4), (31, 33, 32), (0, 1, 1)])
-def test_schedule_covers_exactly_the_steps_in_order(first, count, n):
-    sched = bench.replay_schedule(first, count, n)
-    assert _expand(sched, n) == [s % n for s in range(first, first + count)]
+def test_sweep_and_unrelated_shapes():
+    assert bench.chain_sources(WORKLOADS["decode_sweep"].shapes) == [-1, 0]
+    shapes = (LayerShape("a", 256, 512), LayerShape("b", 128, 1024), LayerShape("c", 64, 256))
+    assert bench.chain_sources(shapes) == [-1, -1, 0]
 
 
-def test_schedule_uses_whole_passes_where_it_can():
-    sched = bench.replay_schedule(64, 3000, 32)
-    passes = sum(1 for k, _ in sched if k == "pass")
-    assert passes == 3000 // 32          # 64 is a pass boundary; the last 24 steps are single layers
-    assert all(k == "layer" for k, _ in sched[passes:])
-    # a run that starts mid-pass finishes that pass layer by layer first
-    sched = bench.replay_schedule(30, 40, 32)
-    assert sched[:2] == [("layer", 30), ("layer", 31)] and sched[2] == ("pass", 0)
+def test_every_source_feeds_a_matching_width():
+    for wl in WORKLOADS.values():
+        src = bench.chain_sources(wl.shapes)
+        for i, d in enumerate(src):
+            assert d < i
+            if d >= 0:
+                assert wl.shapes[d].N == wl.shapes[i].K

@@ -118,9 +118,9 @@ def test_silu_mul_matches_separate_products_then_silu():
     fp16 rounding at the end (GEMV, whole tiles)."""
     N, K = 14336, 4096
     q, s, z, _, _ = fused_layer(N, K, True)
-    x = dev(activations(1, K, seed=77))
-    h = host(awq.awq_gemv(x, q, s, z, silu_mul=True)).astype(np.float64)
-    ref = O.gate_up_silu_f64(host(x), *[oracle_layer(N, K, 0.02, 0.0, True, sd)[4] for sd in (0, 1)])
+    xh = activations(1, K, seed=77)
+    h = host(awq.awq_gemv(dev(xh), q, s, z, silu_mul=True)).astype(np.float64)
+    ref = O.gate_up_silu_f64(xh, *[oracle_layer(N, K, 0.02, 0.0, True, sd)[4] for sd in (0, 1)])
     assert_close(h, ref, "fused vs oracle")
 
 

@@ -25,7 +25,8 @@ __all__ = [
     "LIB_PATH", "AwqError", "lib", "GROUP_SIZE",
     "awq_pseudo_quantize_pack", "awq_dequant", "awq_workspace_bytes",
     "awq_gemv", "awq_gemm", "awq_device_error", "awq_linear", "GEMV_MAX_M", "awq_gemv_noalloc",
-    "awq_pack_zeros", "awq_unpack_zeros", "validate_product",
+    "awq_pack_zeros", "awq_unpack_zeros", "validate_product", "GemvChain", "awq_gemv_chain",
+    "CHAIN_MAX_LAYERS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libawq_b200.so")
@@ -43,7 +44,7 @@ class AwqError(RuntimeError):
         self.status = status
 
 
-ABI_VERSION = 6   # awq_abi_version() of a library this binding matches
+ABI_VERSION = 7   # awq_abi_version() of a library this binding matches
 
 
 class QConfig(ctypes.Structure):
@@ -57,6 +58,15 @@ FLAG_WEIGHTS_STATIC = 1
 FLAG_SILU_MUL = 2   # rows are 16-row tiles alternating gate, up; y = silu(gate) * up, N/2 columns
 FLAG_PACKED_ZEROS = 4   # zeros is int32 qzeros [K/128, N/8], eight 4-bit zero points per word
 
+
+class GemvLayer(ctypes.Structure):
+    """awq_gemv_layer_t: one layer of an awq_gemv_chain call."""
+    _fields_ = [("x", ctypes.c_void_p), ("qweight", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("zeros", ctypes.c_void_p), ("y", ctypes.c_void_p), ("N", ctypes.c_int64),
+                ("K", ctypes.c_int64), ("cfg", QConfig), ("x_from", ctypes.c_int32)]
+
+
+CHAIN_MAX_LAYERS = 8
 
 _lib = None
 _lock = threading.Lock()
@@ -86,6 +96,10 @@ _SIGS = {
     "awq_search_clip": (ctypes.c_int, [_P, _I64, _I64, _P, _I64, QConfig, ctypes.c_int, ctypes.c_float, _P, _P,
                                        ctypes.c_size_t, _P]),
     "awq_apply_clip": (ctypes.c_int, [_P, _P, _I64, _I64, _P, _P]),
+    "awq_gemv_chain_workspace_bytes": (ctypes.c_int, [ctypes.POINTER(GemvLayer), ctypes.c_int, _I64,
+                                                      ctypes.POINTER(ctypes.c_size_t)]),
+    "awq_gemv_chain": (ctypes.c_int, [ctypes.POINTER(GemvLayer), ctypes.c_int, _I64, _P, ctypes.c_size_t, _P]),
+    "awq_debug_set_wait_limit_ns": (ctypes.c_int, [ctypes.c_uint64, _P]),
 }
 
 
@@ -519,3 +533,92 @@ def awq_apply_clip(W: torch.Tensor, ratios: torch.Tensor, out: torch.Tensor | No
     with torch.cuda.device(W.device):
         _check("awq_apply_clip", lib().awq_apply_clip(_ptr(W), _ptr(ratios), N, K, _ptr(out), _stream(W.device)))
     return out
+
+
+class GemvChain:
+    """A prepared awq_gemv_chain call: several decode products in one launch,
+    where a layer's input may be an earlier layer's output.
+
+    layers: a list of dicts with keys
+      qweight, scales, zeros  the packed layer (zeros None: symmetric; int32:
+                              packed zero points, the same form for every layer)
+      x                       fp16 [M, K] input, or None when x_from >= 0
+      x_from                  -1 (default), or the index of the earlier layer
+                              whose output is this layer's input
+      silu_mul                fused gate/up layout (output N/2 columns)
+      out                     optional fp16 output tensor
+    The outputs (self.outputs) and a zero-filled workspace are allocated here;
+    calling the object enqueues the launch on the current stream. The layer
+    descriptors are built once, so repeated calls cost one library call.
+    weights_static: no work still running on the stream writes the weights,
+    so the launch may start streaming them before the previous kernel on the
+    stream has finished."""
+
+    def __init__(self, M: int, layers, weights_static: bool = False, device=None):
+        layers = list(layers)
+        n = len(layers)
+        if not 1 <= n <= CHAIN_MAX_LAYERS:
+            raise ValueError(f"a chain has 1 .. {CHAIN_MAX_LAYERS} layers")
+        self.M = int(M)
+        self.outputs = []
+        self._keep = []
+        arr = (GemvLayer * n)()
+        dev = None
+        for l, d in enumerate(layers):
+            q, sc, z = d["qweight"], d["scales"], d.get("zeros")
+            x_from = int(d.get("x_from", -1))
+            silu = bool(d.get("silu_mul", False))
+            if x_from >= 0:
+                if not 0 <= x_from < l:
+                    raise ValueError(f"layer {l}: x_from must name an earlier layer")
+                x = self.outputs[x_from]
+            else:
+                x = d["x"]
+            _need(x, f"layers[{l}].x", torch.float16, 2)
+            if x.shape[0] != self.M:
+                raise ValueError(f"layer {l}: x has {x.shape[0]} rows, the chain M = {self.M}")
+            flags = (FLAG_WEIGHTS_STATIC if weights_static else 0) | (FLAG_SILU_MUL if silu else 0)
+            _, N, K, flags = validate_product(x, q, sc, z, d.get("out"), None, GROUP_SIZE, flags)
+            if dev is None:
+                dev = x.device
+            elif x.device != dev:
+                raise ValueError(f"layer {l} is on {x.device}, the chain on {dev}")
+            out = d.get("out")
+            if out is None:
+                out = torch.empty((self.M, N // 2 if silu else N), dtype=torch.float16, device=x.device)
+            self.outputs.append(out)
+            self._keep += [x, q, sc, z, out]
+            arr[l] = GemvLayer(x.data_ptr(), q.data_ptr(), sc.data_ptr(), _ptr(z), out.data_ptr(), N, K,
+                               _cfg(z is not None, GROUP_SIZE, flags), x_from)
+        self.device = dev if device is None else torch.device(device)
+        self._arr, self._n = arr, n
+        nbytes = ctypes.c_size_t(0)
+        with torch.cuda.device(self.device):
+            _check("awq_gemv_chain_workspace_bytes",
+                   lib().awq_gemv_chain_workspace_bytes(arr, n, self.M, ctypes.byref(nbytes)))
+        self.workspace = torch.zeros(max(int(nbytes.value), 16), dtype=torch.uint8, device=self.device)
+        self._ws = (self.workspace.data_ptr(), self.workspace.numel())
+
+    def __call__(self):
+        if self.device.index == torch.cuda.current_device():
+            st = lib().awq_gemv_chain(self._arr, self._n, self.M, self._ws[0], self._ws[1],
+                                      torch.cuda.current_stream().cuda_stream)
+        else:
+            with torch.cuda.device(self.device):
+                st = lib().awq_gemv_chain(self._arr, self._n, self.M, self._ws[0], self._ws[1],
+                                          torch.cuda.current_stream(self.device).cuda_stream)
+        _check("awq_gemv_chain", st)
+        return self.outputs
+
+
+def awq_gemv_chain(M: int, layers, weights_static: bool = False):
+    """One awq_gemv_chain call (see GemvChain); returns the layers' outputs."""
+    return GemvChain(M, layers, weights_static)()
+
+
+def awq_debug_set_wait_limit_ns(ns: int, device=None):
+    """Test hook: the time limit of awq_gemv_chain's pipeline waits (0: the
+    default 2 s). Synchronizes the device's current stream."""
+    dev = device if device is not None else torch.cuda.current_device()
+    with torch.cuda.device(dev):
+        _check("awq_debug_set_wait_limit_ns", lib().awq_debug_set_wait_limit_ns(int(ns), _stream(dev)))

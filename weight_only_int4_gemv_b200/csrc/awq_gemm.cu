@@ -562,6 +562,7 @@ std::atomic<int> g_clusters[kMaxDevices][4][3];
 }  // namespace
 
 awq_status_t gemv_take_error(uint32_t* word, cudaStream_t s);
+awq_status_t chain_take_error(uint32_t* word, cudaStream_t s);
 
 awq_status_t gemm_workspace_bytes(int64_t, int64_t, int64_t, bool, size_t* bytes) {
   *bytes = 0;
@@ -724,6 +725,8 @@ extern "C" awq_status_t awq_device_error(uint32_t* error_word, void* stream) {
   if (cudaStreamSynchronize(s) != cudaSuccess) return AWQ_ERR_CUDA;
   awq_status_t st = gemv_take_error(&gemv_word, s);
   if (st != AWQ_OK) return st;
-  *error_word = gemm_word | gemv_word;
+  uint32_t chain_word = 0;
+  if ((st = chain_take_error(&chain_word, s)) != AWQ_OK) return st;
+  *error_word = gemm_word | gemv_word | chain_word;
   return AWQ_OK;
 }
