@@ -296,18 +296,69 @@ def chain_sources(shapes):
     return src
 
 
-class DecodeLayer:
-    """One layer copy: packed weights of each shape, the step's input x and
-    its prepared chain call (outputs and workspace allocated)."""
+class DecodeModel:
+    """n layer copies of the decode layer: packed weights of each shape and
+    one output buffer per projection. Step s runs copy s % n; its first
+    projection reads the last projection's output of the step before (copy
+    (s - 1) % n), as a decode pass feeds each layer the previous one's
+    output. Launches carry up to `per_launch` consecutive steps."""
 
-    def __init__(self, packed, x, chain, per_gemv):
-        self.packed, self.x, self.chain, self.per_gemv = packed, x, chain, per_gemv
+    def __init__(self, awq, torch, packed, ys, shapes, M, per_launch):
+        self.awq, self.torch = awq, torch
+        self.packed, self.ys, self.shapes, self.M = packed, ys, shapes, M
+        self.n = len(packed)
+        self.per_launch = per_launch
+        self.src = chain_sources(shapes)
+        self._chains = {}
+
+    def step_input(self, c):
+        return self.ys[(c - 1) % self.n][-1]
+
+    def chain(self, start, count):
+        """The prepared awq_gemv_chain call of steps start .. start + count - 1."""
+        key = (start % self.n, count)
+        ch = self._chains.get(key)
+        if ch is None:
+            nl = len(self.shapes)
+            specs = []
+            for j in range(count):
+                c = (start + j) % self.n
+                for i, (q, s, z) in enumerate(self.packed[c]):
+                    if i == 0:
+                        xs = dict(x=self.step_input(c)) if j == 0 else dict(x_from=nl * (j - 1) + nl - 1)
+                    else:
+                        xs = dict(x_from=nl * j + self.src[i])
+                    specs.append(dict(xs, qweight=q, scales=s, zeros=z, out=self.ys[c][i]))
+            ch = self._chains[key] = self.awq.GemvChain(self.M, specs, weights_static=True)
+        return ch
+
+    def launches(self, first, count):
+        """(start, count) of the launches that run steps first .. first + count - 1."""
+        out, s = [], first
+        while s < first + count:
+            k = min(self.per_launch, first + count - s)
+            out.append((s, k))
+            s += k
+        return out
+
+    def run_steps_chain(self, first, count):
+        for s, k in self.launches(first, count):
+            self.chain(s, k)()
+
+    def run_steps_per_gemv(self, first, count, workspaces):
+        awq = self.awq
+        for s in range(first, first + count):
+            c = s % self.n
+            for i, (q, sc, z) in enumerate(self.packed[c]):
+                x = self.step_input(c) if i == 0 else self.ys[c][self.src[i]]
+                awq.awq_gemv(x, q, sc, z, workspace=workspaces[i], out=self.ys[c][i], weights_static=True)
 
 
 def build_decode(awq, torch, device, shapes, M: int, n_layers: int, zp: bool):
     """Quantize each shape on the GPU (recipe W, seed 0; the second, warm call
     is timed), then clone the packed tensors into n_layers copies at distinct
-    addresses, each with its own input and a prepared chain call."""
+    addresses, each with its own output buffers (seeded N(0,1) values, so the
+    first steps read finite inputs)."""
     base, quant_ms, quant_bytes = [], 0.0, 0
     for sh in shapes:
         W = torch.from_numpy(make_weight(sh.N, sh.K, 0.02, 0.01, seed=0)).to(device)
@@ -324,24 +375,17 @@ def build_decode(awq, torch, device, shapes, M: int, n_layers: int, zp: bool):
         quant_bytes += 2 * sh.N * sh.K + algo_bytes(0, sh.N, sh.K, zp)
         base.append((q, s, z))
         del W
+    if shapes[-1].N != shapes[0].K:
+        raise SystemExit("a decode step's last projection must feed its first")
     rng = np.random.default_rng(1)
-    src = chain_sources(shapes)
-    layers = []
+    packed, ys = [], []
     for _ in range(n_layers):
-        packed = [(q.clone(), s.clone(), z.clone() if z is not None else None) for q, s, z in base]
-        x = torch.from_numpy(rng.standard_normal((M, shapes[0].K), dtype=np.float32).astype(np.float16)).to(device)
-        specs = [dict(x=x if src[i] < 0 else None, x_from=src[i], qweight=q, scales=s, zeros=z)
-                 for i, (q, s, z) in enumerate(packed)]
-        chain = awq.GemvChain(M, specs, weights_static=True)
-        # the same products as separate awq_gemv launches (for --per-gemv)
-        wss = [awq.alloc_workspace(M, sh.N, sh.K, zp, device=device) for sh in shapes]
-
-        def per_gemv(chain=chain, packed=packed, wss=wss, x=x):
-            for i in range(len(packed)):
-                xin = x if src[i] < 0 else chain.outputs[src[i]]
-                awq.awq_gemv(xin, *packed[i], workspace=wss[i], out=chain.outputs[i], weights_static=True)
-        layers.append(DecodeLayer(packed, x, chain, per_gemv))
-    return layers, {"ms": round(quant_ms, 4), "GB/s": round(quant_bytes / (quant_ms * 1e-3) / 1e9, 1)}
+        packed.append([(q.clone(), s.clone(), z.clone() if z is not None else None) for q, s, z in base])
+        ys.append([torch.from_numpy(rng.standard_normal((M, sh.N), dtype=np.float32).astype(np.float16)).to(device)
+                   for sh in shapes])
+    per_launch = max(1, awq.CHAIN_MAX_LAYERS // len(shapes))
+    model = DecodeModel(awq, torch, packed, ys, shapes, M, per_launch)
+    return model, {"ms": round(quant_ms, 4), "GB/s": round(quant_bytes / (quant_ms * 1e-3) / 1e9, 1)}
 
 
 def run_native(args, dist):
@@ -362,30 +406,32 @@ def run_native(args, dist):
     if M > awq.GEMV_MAX_M:
         raise SystemExit("the decode bench runs the GEMV path; use --workload llama3_8b_decode or decode_sweep")
 
-    layers, quant = build_decode(awq, torch, device, shapes, M, args.layers, zp)
+    model, quant = build_decode(awq, torch, device, shapes, M, args.layers, zp)
     step_bytes = sum(algo_bytes(M, sh.N, sh.K, zp) for sh in shapes)
     step_flops = sum(algo_flops(M, sh.N, sh.K) for sh in shapes)
     stream = torch.cuda.Stream(device)
-    n = len(layers)
-    launches_per_step = len(shapes) if args.per_gemv else 1
+    wss = [awq.alloc_workspace(M, sh.N, sh.K, zp, device=device) for sh in shapes]
 
-    def step(i):
-        L = layers[i % n]
-        L.per_gemv() if args.per_gemv else L.chain()
+    def run_steps(first, count):
+        if args.per_gemv:
+            model.run_steps_per_gemv(first, count, wss)
+        else:
+            model.run_steps_chain(first, count)
 
-    # Each run of steps is replayed from one CUDA graph holding exactly those
-    # steps (step i on layer copy i % n), so consecutive launches stay linked
+    def n_launches(first, count):
+        return count * len(shapes) if args.per_gemv else len(model.launches(first, count))
+
+    # The warm-up steps and the timed steps are each replayed from one CUDA
+    # graph holding exactly those steps, so consecutive launches stay linked
     # by programmatic dependent launch whatever the number of steps.
     def capture(first, count):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
-            for i in range(first, first + count):
-                step(i)
+            run_steps(first, count)
         return g
 
     with torch.cuda.stream(stream):
-        for i in range(n):            # warm the plan caches outside capture
-            step(i)
+        run_steps(0, args.warmup + args.steps)   # prepares every chain and plan outside capture
     torch.cuda.synchronize(device)
     g_warm = capture(0, args.warmup)
     g_timed = capture(args.warmup, args.steps)
@@ -416,7 +462,7 @@ def run_native(args, dist):
     # Every launch in the timed region is one of this library's products and
     # consecutive launches overlap (programmatic dependent launch), so the
     # kernel's average launch duration is the timed region over its launches.
-    n_launch = args.steps * launches_per_step
+    n_launch = n_launches(args.warmup, args.steps)
     mean_launch_s = elapsed_s / n_launch
     kernel_gbs = step_bytes * args.steps / elapsed_s / 1e9
 
@@ -424,7 +470,7 @@ def run_native(args, dist):
     value = total_bytes / max_s / 1e9
 
     # end to end through the public API: pinned host x in, pinned host y out, every step
-    e2e = run_e2e(awq, torch, device, stream, layers, shapes, M, args, dist, step_bytes)
+    e2e = run_e2e(awq, torch, device, stream, model, shapes, M, args, dist, step_bytes)
 
     gemm = None
     search = None
@@ -461,9 +507,13 @@ def run_native(args, dist):
                 "M": M, "group_size": 128, "zero_point": zp,
                 "weights_static": "AWQ_FLAG_WEIGHTS_STATIC set: weights are loaded once, so a launch may "
                                   "start streaming them before the previous kernel on the stream finishes",
-                "step": ("one layer: one awq_gemv launch per listed projection" if args.per_gemv else
-                         "one layer: one awq_gemv_chain launch of the listed projections, each reading its "
-                         "input only after the projection it comes from is complete"),
+                "step": "one layer: the listed projections, each reading its input only after the projection "
+                        "it comes from is complete; a step's first projection reads the previous step's last "
+                        "output",
+                "launch": ("one awq_gemv launch per projection" if args.per_gemv else
+                           f"one awq_gemv_chain launch per {model.per_launch} consecutive steps "
+                           f"({model.per_launch * len(shapes)} projections; a shorter last launch when the step "
+                           "count is not a multiple)"),
                 "graphs": "the warm-up steps and the timed steps are each replayed from one CUDA graph "
                           "holding exactly those steps",
                 "l2": f"inputs larger than L2: steps rotate over {args.layers} layer copies "
@@ -478,7 +528,7 @@ def run_native(args, dist):
                 "kernel": ("awq_gemv (gemv_kernel, M tile 1, asymmetric)" if args.per_gemv else
                            "awq_gemv_chain (chain_kernel<1, 1>: M = 1, fp16 zero points)"),
                 "launches_timed": n_launch,
-                "algorithmic_bytes_per_launch": round(step_bytes / launches_per_step),
+                "algorithmic_bytes_per_launch": round(step_bytes * args.steps / n_launch),
                 "mean_launch_us": round(1e6 * mean_launch_s, 3),
                 "duration_source": "CUDA events around the timed steps on the launch stream / launches",
                 "frac_of_nominal_8TBs": round(kernel_gbs / 8000.0, 4),
@@ -497,24 +547,27 @@ def run_native(args, dist):
         print(json.dumps(line), flush=True)
 
 
-def run_e2e(awq, torch, device, stream, layers, shapes, M, args, dist, step_bytes):
+def run_e2e(awq, torch, device, stream, model, shapes, M, args, dist, step_bytes):
     """Same metric through the Python API with host buffers: every step copies
-    its input x from pinned host memory to the device, runs the layer (the
-    prepared chain call), reads the layer's result (the last projection's
-    output) back into pinned host memory, then synchronizes."""
+    its input x from pinned host memory to the device, runs the layer (one
+    prepared chain call of that step), reads the layer's result (the last
+    projection's output) back into pinned host memory, then synchronizes."""
     steps = max(1, min(args.steps, args.e2e_steps))
-    hx = torch.empty_like(layers[0].x, device="cpu").pin_memory()
-    hy = torch.empty_like(layers[0].chain.outputs[-1], device="cpu").pin_memory()
-    hx.copy_(layers[0].x.cpu())
+    hx = torch.empty_like(model.step_input(0), device="cpu").pin_memory()
+    hy = torch.empty_like(model.ys[0][-1], device="cpu").pin_memory()
+    hx.copy_(model.step_input(0).cpu())
     h2d = hx.numel() * 2
     d2h = hy.numel() * 2
-    n = len(layers)
+    wss = [awq.alloc_workspace(M, sh.N, sh.K, True, device=device) for sh in shapes]
 
     def step(s):
-        L = layers[s % n]
-        L.x.copy_(hx, non_blocking=True)
-        L.per_gemv() if args.per_gemv else L.chain()
-        hy.copy_(L.chain.outputs[-1], non_blocking=True)
+        c = s % model.n
+        model.step_input(c).copy_(hx, non_blocking=True)
+        if args.per_gemv:
+            model.run_steps_per_gemv(s, 1, wss)
+        else:
+            model.chain(s, 1)()
+        hy.copy_(model.ys[c][-1], non_blocking=True)
         torch.cuda.current_stream(device).synchronize()
 
     with torch.cuda.stream(stream):
@@ -534,7 +587,7 @@ def run_e2e(awq, torch, device, stream, layers, shapes, M, args, dist, step_byte
     return {"value": round(total / max_s / 1e9, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": steps,
             "note": "effective HBM GB/s of the same algorithmic bytes, time includes the copies and a "
-                    "host synchronize per step"}
+                    "host synchronize per step (one launch per step)"}
 
 
 def run_scale_search(awq, torch, device):

@@ -193,9 +193,10 @@ AWQ_API awq_status_t awq_unpack_zeros(const int32_t* qzeros, int64_t G, int64_t 
  * awq_workspace_bytes -- bytes of workspace awq_gemv / awq_gemm need for
  * (M, N, K) on the current device. *bytes is 0 when none is needed.
  * The workspace holds split-K partial sums and arrival counters. It must be
- * zero-filled before its first use; every call that completes leaves it
- * zero-filled again, so one memset at allocation suffices. Calls that may
- * run concurrently need separate workspaces.
+ * zero-filled before its first use; every call that completes brings the
+ * counters back to zero (the partial sums need no clearing), so one memset
+ * at allocation suffices. Calls that may run concurrently need separate
+ * workspaces.
  */
 AWQ_API awq_status_t awq_workspace_bytes(int64_t M, int64_t N, int64_t K,
                                  awq_qconfig_t cfg, size_t* bytes);
@@ -282,7 +283,8 @@ AWQ_API awq_status_t awq_gemv_noalloc(const uint16_t* x, const int32_t* qweight,
  * layers: host memory, read before the call returns.
  * workspace: at least awq_gemv_chain_workspace_bytes() bytes of device
  * memory, zero-filled before its first use; every call that completes (also
- * one whose waits gave up, see awq_device_error) leaves it zero-filled.
+ * one whose waits gave up, see awq_device_error) brings its counters back to
+ * zero, so one memset at allocation suffices.
  * Calls that may run concurrently need separate workspaces.
  * Every CTA of the launch must be resident at once (the grid is sized from
  * the occupancy of the kernel on this device): do not run other kernels
@@ -290,7 +292,7 @@ AWQ_API awq_status_t awq_gemv_noalloc(const uint16_t* x, const int32_t* qweight,
  * the dependency waits reach their time limit and the call gives up
  * (reported by awq_device_error, bit 2).
  */
-#define AWQ_CHAIN_MAX_LAYERS 8
+#define AWQ_CHAIN_MAX_LAYERS 32
 typedef struct awq_gemv_layer {
   const uint16_t* x;        /* [M][K] fp16 */
   const int32_t* qweight;   /* [N][K/8] */

@@ -30,3 +30,13 @@ def test_every_source_feeds_a_matching_width():
             assert d < i
             if d >= 0:
                 assert wl.shapes[d].N == wl.shapes[i].K
+
+
+def test_launches_cover_the_steps_in_order():
+    m = bench.DecodeModel(None, None, [None] * 32, [None] * 32, LLAMA3_8B_DECODE, 1, 8)
+    for first, count in [(0, 20), (64, 2000), (5, 3), (3, 8), (0, 1)]:
+        ls = m.launches(first, count)
+        steps = [s for a, k in ls for s in range(a, a + k)]
+        assert steps == list(range(first, first + count))
+        assert all(1 <= k <= 8 for _, k in ls)
+        assert all(k == 8 for _, k in ls[:-1])

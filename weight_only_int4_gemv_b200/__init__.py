@@ -66,7 +66,7 @@ class GemvLayer(ctypes.Structure):
                 ("K", ctypes.c_int64), ("cfg", QConfig), ("x_from", ctypes.c_int32)]
 
 
-CHAIN_MAX_LAYERS = 8
+CHAIN_MAX_LAYERS = 32
 
 _lib = None
 _lock = threading.Lock()

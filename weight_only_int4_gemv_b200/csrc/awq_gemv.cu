@@ -578,6 +578,7 @@ __device__ __forceinline__ void gemv_cta(const CUtensorMap& tmap_q, const CUtens
           last = (old + 1 == uint32_t(p.ks)) ? 1u : 0u;
         }
         last = __shfl_sync(0xffffffffu, last, 0);
+        __syncwarp();   // lane 0's acquire orders the warp's partial reads
         if (last) {
           const int64_t trow = int64_t(unit) * TPU * kTile;
           if constexpr (TPU == 1) {

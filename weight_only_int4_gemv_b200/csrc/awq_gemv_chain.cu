@@ -57,6 +57,9 @@
 
 #include <atomic>
 #include <cstring>
+#include <mutex>
+#include <utility>
+#include <vector>
 
 namespace awq {
 
@@ -72,7 +75,7 @@ constexpr int kCW = 8;                          // consumer warps
 constexpr int kThreads = (kCW + 1) * 32;        // + one producer warp
 constexpr int kTile = 16;                       // output channels per MMA tile
 constexpr int kMaxTC = 4;                       // tiles per chunk
-constexpr int kMaxLayers = 8;
+constexpr int kMaxLayers = AWQ_CHAIN_MAX_LAYERS;
 constexpr int kMaxStages = 8;
 constexpr int kHeader = 1024;                   // barriers and flags below the ring
 constexpr int kTileBytes = kCW * 1024;          // codes of one tile: [group][16 rows][16 words]
@@ -181,6 +184,21 @@ __device__ __forceinline__ bool mbar_try_wait_u32(uint32_t bar, uint32_t parity)
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint: a thread whose phase is not complete
+// sleeps until it completes or the hint (ns) runs out, instead of spinning
+// and taking issue slots from the warps that share its scheduler.
+__device__ __forceinline__ bool mbar_sleep_wait(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
   uint32_t v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -211,16 +229,33 @@ struct Chunk {
   int i, nu, tc, t0, s, gb, ge;
 };
 
-// The CTA's items of a layer: q = items / grid each, and one more for the r
-// = items % grid CTAs from `rot` on (cyclically), so that consecutive
-// independent layers hand their leftover items to different CTAs.
+// The items (units of one K slice) of a layer that CTA position b (of
+// `grid`) takes. Without K slices: q = units / grid each, one more for the
+// first units % grid positions. With ks slices: slice s goes to positions
+// [ceil(s grid / ks), ceil((s + 1) grid / ks)), which share its units the
+// same way, so that no CTA straddles two slices. Items are slice-major
+// (item = slice * units + unit). The same arithmetic runs on the host.
+__host__ __device__ __forceinline__ void split_items(int units, int ks, int grid, int b, int& i0, int& i1) {
+  int s = 0, b0 = 0, n = grid;
+  if (ks > 1) {
+    s = int(int64_t(b) * ks / grid);
+    b0 = int((int64_t(s) * grid + ks - 1) / ks);
+    n = int((int64_t(s + 1) * grid + ks - 1) / ks) - b0;
+  }
+  const int j = b - b0;
+  const int q = units / n, r = units - q * n;
+  const int u0 = j * q + (j < r ? j : r);
+  i0 = s * units + u0;
+  i1 = i0 + q + (j < r ? 1 : 0);
+}
+
+// The CTA's items of a layer, its position rotated by `rot` so that
+// consecutive independent layers hand their leftover items to different CTAs.
 __device__ __forceinline__ void item_range(const LayerDesc& L, int& i0, int& i1) {
   const int grid = int(gridDim.x);
   int b = int(blockIdx.x) - L.rot;
   if (b < 0) b += grid;
-  const int q = L.items / grid, r = L.items - q * grid;
-  i0 = b * q + (b < r ? b : r);
-  i1 = i0 + q + (b < r ? 1 : 0);
+  split_items(L.units, L.ks, grid, b, i0, i1);
 }
 
 __device__ __forceinline__ void load_chunk(const LayerDesc& L, int i, int i_end, Chunk& c) {
@@ -405,6 +440,7 @@ chain_kernel(const __grid_constant__ ChainParams p) {
   const int warp = int(threadIdx.x) >> 5;
   const int lane = int(threadIdx.x) & 31;
   const unsigned long long limit = g_awq_chain_wait_limit_ns;
+  const uint32_t hint = limit < 20000ull ? uint32_t(limit) : 20000u;   // sleep of one wait step, ns
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -467,6 +503,11 @@ chain_kernel(const __grid_constant__ ChainParams p) {
         if (progress) {
           t_idle = 0;
           continue;
+        }
+        if (sx == sw && !cw.done(p.n_layers)) {
+          // nothing to do until the next slot frees: sleep on its barrier
+          const int slot = sw % S;
+          mbar_sleep_wait(empty0 + 8 * slot, uint32_t((sw / S) + 1) & 1u, hint);
         }
         if (*abort_flag) {
           gave_up = true;
@@ -531,12 +572,12 @@ chain_kernel(const __grid_constant__ ChainParams p) {
         for (int gbase = cc.gb; gbase < cc.ge; gbase += kCW) {
           const uint32_t full = full0 + 8 * slot;
           if (live) {
-            bool ok = mbar_try_wait_u32(full, phase);
+            bool ok = mbar_sleep_wait(full, phase, hint);
             if (!ok) {
               const uint64_t t0 = now_ns();
-              for (uint32_t it = 1; !ok; ++it) {
-                ok = mbar_try_wait_u32(full, phase);
-                if (!ok && (it & 31) == 0) {
+              while (!ok) {
+                ok = mbar_sleep_wait(full, phase, hint);
+                if (!ok) {
                   if (*abort_flag) break;
                   if (now_ns() - t0 > limit) {
                     *abort_flag = 1;
@@ -618,8 +659,9 @@ chain_kernel(const __grid_constant__ ChainParams p) {
         }
         if (L.ks > 1) {
           // slices of a unit meet in the workspace: the CTA whose arrival
-          // brings a unit's count to ks sums the ks partials in slice order
-          __threadfence();
+          // brings a unit's count to ks sums the ks partials in slice order.
+          // The barrier orders every consumer's partial stores before the
+          // arrivals, whose release makes them visible at GPU scope.
           consumer_sync();
           if (w < cc.nu) {
             const int unit = cc.t0 / L.tpu + w;
@@ -631,6 +673,7 @@ chain_kernel(const __grid_constant__ ChainParams p) {
               last = (old + 1 == uint32_t(L.ks)) ? 1u : 0u;
             }
             last = __shfl_sync(0xffffffffu, last, 0);
+            __syncwarp();   // lane 0's acquire orders the warp's partial reads
             if (last) {
               const int64_t trow = int64_t(unit) * L.tpu * kTile;
               if (L.tpu == 1) {
@@ -663,11 +706,7 @@ chain_kernel(const __grid_constant__ ChainParams p) {
       }
       // This CTA is done with layer l: release its y stores (and fixups) to
       // the producers that wait for the layer.
-      if (threadIdx.x == 0) {
-        asm volatile("fence.proxy.async.global;" ::: "memory");
-        __threadfence();
-        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(p.done + l) : "memory");
-      }
+      if (threadIdx.x == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(p.done + l) : "memory");
     }
   }
   __syncthreads();
@@ -745,6 +784,67 @@ awq_status_t check_layer(const awq_gemv_layer_t* L, int l, const awq_gemv_layer_
   return AWQ_OK;
 }
 
+// Cost of the busiest CTA when a layer of `units` units (tpu tiles each) and
+// G groups is cut into ks K slices over `grid` CTAs, in tile-group units: each
+// stage of kCW groups costs its tiles x groups, but never less than that of
+// three tiles (a stage of one or two tiles has too little independent work
+// to hide the latency of its decode-and-multiply chains), plus a fixed cost
+// per stage, per chunk (the reduction) and per chunk of a split layer
+// (partials and the arrival).
+int64_t split_cost(int units, int tpu, int G, int ks, int grid) {
+  constexpr int64_t kMinTiles = 3, kStageCost = 2, kChunkCost = 4, kSplitCost = 6;
+  int64_t worst = 0;
+  for (int b = 0; b < grid; ++b) {
+    int i0, i1;
+    split_items(units, ks, grid, b, i0, i1);
+    int64_t c = 0;
+    for (int i = i0; i < i1;) {
+      const int sl = i / units, u0 = i - sl * units;
+      int nu = i1 - i;
+      if (nu > kMaxTC / tpu) nu = kMaxTC / tpu;
+      if (nu > units - u0) nu = units - u0;
+      const int64_t g = int64_t(G) * (sl + 1) / ks - int64_t(G) * sl / ks;
+      const int64_t tc = nu * tpu;
+      // a stage takes as long as a full one whatever its group count (one group per warp)
+      c += ((g + kCW - 1) / kCW) * ((tc > kMinTiles ? tc : kMinTiles) * kCW + kStageCost) + kChunkCost +
+           (ks > 1 ? kSplitCost : 0);
+      i += nu;
+    }
+    if (c > worst) worst = c;
+  }
+  return worst;
+}
+
+// K slices for a layer: the candidate whose busiest CTA costs least (ties:
+// fewer slices). Cached per (units, tpu, G, grid): the choice is a few
+// hundred thousand steps of host arithmetic.
+int pick_ks(int units, int tpu, int G, int grid) {
+  struct Key {
+    int units, tpu, G, grid;
+  };
+  static std::mutex lock;
+  static std::vector<std::pair<Key, int>> cache;
+  {
+    std::lock_guard<std::mutex> g(lock);
+    for (const auto& e : cache)
+      if (e.first.units == units && e.first.tpu == tpu && e.first.G == G && e.first.grid == grid) return e.second;
+  }
+  int best = 1;
+  int64_t best_cost = split_cost(units, tpu, G, 1, grid);
+  const int cands[] = {2, 3, 4, 5, 6, 7, 8, 10, 12, 14, 16, 24, 32};
+  for (int ks : cands) {
+    if (ks > G || ks > grid) break;
+    const int64_t c = split_cost(units, tpu, G, ks, grid);
+    if (c < best_cost) {
+      best_cost = c;
+      best = ks;
+    }
+  }
+  std::lock_guard<std::mutex> g(lock);
+  if (cache.size() < 4096) cache.push_back({Key{units, tpu, G, grid}, best});
+  return best;
+}
+
 awq_status_t make_chain_plan(const awq_gemv_layer_t* layers, int n, int64_t M, ChainPlan& pl) {
   if (!layers) return AWQ_ERR_NULL;
   if (n < 1 || n > kMaxLayers) return AWQ_ERR_SHAPE;
@@ -801,13 +901,9 @@ awq_status_t make_chain_plan(const awq_gemv_layer_t* layers, int n, int64_t M, C
     lp.T = int((L.N + kTile - 1) / kTile);
     lp.tpu = (L.cfg.flags & AWQ_FLAG_SILU_MUL) ? 2 : 1;
     lp.units = lp.T / lp.tpu;
-    int64_t ks = 1;
-    if (lp.units < pl.grid) {
-      ks = (pl.grid + lp.units - 1) / lp.units;
-      if (ks > G) ks = G;
-    }
-    lp.ks = int(ks);
-    lp.items = int(int64_t(lp.units) * ks);
+    const int ks = pick_ks(lp.units, lp.tpu, int(G), pl.grid);
+    lp.ks = ks;
+    lp.items = lp.units * ks;
     // A layer that reads the output of a layer of the current level starts a
     // new level. Within a level, each layer's leftover items go to the CTAs
     // after those that took the previous layers' leftovers.
@@ -816,7 +912,7 @@ awq_status_t make_chain_plan(const awq_gemv_layer_t* layers, int n, int64_t M, C
       extra = 0;
     }
     lp.rot = int(extra % pl.grid);
-    extra += lp.items % pl.grid;
+    if (lp.ks == 1) extra += lp.units % pl.grid;
     if (lp.ks > 1) {
       lp.counter_off = off;
       off += align256(size_t(lp.units) * 4);
