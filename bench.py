@@ -421,22 +421,23 @@ def run_native(args, dist):
     def n_launches(first, count):
         return count * len(shapes) if args.per_gemv else len(model.launches(first, count))
 
-    # The warm-up steps and the timed steps are replayed from one CUDA graph
-    # holding exactly those steps, with the two timing events recorded inside
-    # it between the warm-up steps and the timed ones and after the last: the
-    # timed steps run exactly as in a longer run (consecutive launches linked
-    # by programmatic dependent launch), and the graph's own launch is not
-    # part of the timed region.
+    # The warm-up steps and the timed steps are each replayed from one CUDA
+    # graph holding exactly those steps, so consecutive launches stay linked
+    # by programmatic dependent launch whatever the number of steps (only the
+    # first launch of the timed graph cannot overlap the launch before it).
+    def capture(first, count):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            run_steps(first, count)
+        return g
+
     with torch.cuda.stream(stream):
         run_steps(0, args.warmup + args.steps)   # prepares every chain and plan outside capture
     torch.cuda.synchronize(device)
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=stream):
-        run_steps(0, args.warmup)
-        t0.record(stream)
-        run_steps(args.warmup, args.steps)
-        t1.record(stream)
+    g_warm = capture(0, args.warmup)
+    g_timed = capture(args.warmup, args.steps)
+    with torch.cuda.stream(stream):
+        g_timed.replay()                           # untimed: first replay of the instantiated graph
     torch.cuda.synchronize(device)
 
     def barrier():
@@ -444,19 +445,22 @@ def run_native(args, dist):
             dist.barrier()
 
     with torch.cuda.stream(stream):
-        graph.replay()                            # untimed: first replay of the instantiated graph
+        g_warm.replay()
     torch.cuda.synchronize(device)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(device.index if device.index is not None else 0)
     barrier()
     torch.cuda.synchronize(device)
     with sampler:
         with torch.cuda.stream(stream):
-            graph.replay()
+            t0.record()
+            g_timed.replay()
+            t1.record()
         torch.cuda.synchronize(device)
     barrier()
     elapsed_s = t0.elapsed_time(t1) * 1e-3
     dev_err = awq.awq_device_error(device)
-    del graph
+    del g_warm, g_timed
 
     # Every launch in the timed region is one of this library's products and
     # consecutive launches overlap (programmatic dependent launch), so the
@@ -513,9 +517,8 @@ def run_native(args, dist):
                            f"one awq_gemv_chain launch per {model.per_launch} consecutive steps "
                            f"({model.per_launch * len(shapes)} projections; a shorter last launch when the step "
                            "count is not a multiple)"),
-                "graphs": "the warm-up steps and the timed steps are replayed from one CUDA graph holding "
-                          "exactly those steps; the timing events are recorded inside it (after the warm-up "
-                          "steps and after the last step); the graph is replayed once untimed first",
+                "graphs": "the warm-up steps and the timed steps are each replayed from one CUDA graph "
+                          "holding exactly those steps (the timed graph is replayed once untimed first)",
                 "l2": f"inputs larger than L2: steps rotate over {args.layers} layer copies "
                       f"({args.layers * step_bytes / 1e9:.2f} GB of packed weights)",
                 "parallelism": f"replicas x{ws_}",
