@@ -710,37 +710,45 @@ def run_table(args):
     torch.cuda.set_device(device)
     hbm_peak, tc_peak, _, peak_src = measured_peaks()
     # (N, K), batch sizes, fused gate/up (AWQ_FLAG_SILU_MUL: N = gate + up rows, y has N / 2 columns),
-    # packed zero points (AWQ_FLAG_PACKED_ZEROS, GEMV only)
-    cases = [((4096, 4096), (1, 2, 4, 8, 16, 128, 512, 2048), False, False),
-             ((14336, 4096), (1, 2, 4, 8, 16, 128, 512, 2048), False, False),
-             ((28672, 4096), (1, 4, 16, 128, 2048), True, False),
-             ((6144, 4096), (1, 4, 16), False, False),     # q, k, v of Llama-3-8B concatenated
-             ((1024, 4096), (1, 4, 16), False, False),     # k or v alone
-             ((4096, 14336), (1, 2, 4, 8, 16), False, False),
-             ((8192, 8192), (1, 8, 2048), False, False), ((28672, 8192), (1, 8, 2048), False, False),
-             ((8192, 28672), (1, 8, 2048), False, False),
-             ((4096, 4096), (1, 4, 16), False, True), ((14336, 4096), (1, 4, 16), False, True),
-             ((4096, 14336), (1, 4, 16), False, True), ((28672, 4096), (1, 4, 16), True, True)]
+    # packed zero points (AWQ_FLAG_PACKED_ZEROS, GEMV only), zero points (False: symmetric)
+    mid = (16, 24, 32, 48, 64, 96, 128)   # around the GEMV / GEMM crossover
+    cases = [((4096, 4096), (1, 2, 4, 8, 16, 128, 512, 2048), False, False, True),
+             ((14336, 4096), (1, 2, 4, 8, 16, 128, 512, 2048), False, False, True),
+             ((4096, 4096), mid[1:], False, False, True), ((14336, 4096), mid[1:], False, False, True),
+             ((28672, 4096), (1, 4, 16, 128, 2048), True, False, True),
+             ((6144, 4096), (1, 4, 16), False, False, True),     # q, k, v of Llama-3-8B concatenated
+             ((1024, 4096), (1, 4, 16), False, False, True),     # k or v alone
+             ((4096, 14336), (1, 2, 4, 8, 16), False, False, True),
+             ((14336, 4096), (1, 2, 4, 8, 16), False, False, False),   # symmetric
+             ((4096, 14336), (1, 2, 4, 8, 16), False, False, False),
+             ((8192, 8192), (1, 8, 2048), False, False, True), ((28672, 8192), (1, 8, 2048), False, False, True),
+             ((8192, 28672), (1, 8, 2048), False, False, True),
+             ((4096, 4096), (1, 4, 16), False, True, True), ((14336, 4096), (1, 4, 16), False, True, True),
+             ((4096, 14336), (1, 4, 16), False, True, True), ((28672, 4096), (1, 4, 16), True, True, True)]
+    only = os.environ.get("AWQ_TABLE_CASES")   # optional comma-separated case indices
+    if only:
+        cases = [cases[int(i)] for i in only.split(",")]
     l2_bytes = 126 << 20
     rng = np.random.default_rng(3)
-    for (N, K), Ms, silu, packed in cases:
-        q, s, z = [torch.from_numpy(a).to(device) for a in make_packed_random(N, K, 128, True, seed=1)]
+    for (N, K), Ms, silu, packed, zp in cases:
+        q, s, z = [torch.from_numpy(a).to(device) if a is not None else None
+                   for a in make_packed_random(N, K, 128, zp, seed=1)]
         if packed:
             z = awq.awq_pack_zeros(z)
-        wbytes = N * K // 2 + 4 * N * (K // 128)
+        wbytes = N * K // 2 + (4 if zp else 2) * N * (K // 128)
         copies = max(2, -(-2 * l2_bytes // wbytes))
-        packs = [(q.clone(), s.clone(), z.clone()) for _ in range(copies)]
+        packs = [(q.clone(), s.clone(), z.clone() if z is not None else None) for _ in range(copies)]
         del q, s, z
         for M in Ms:
             x = torch.from_numpy(rng.standard_normal((M, K), dtype=np.float32).astype(np.float16)).to(device)
             y = torch.empty((M, N // 2 if silu else N), dtype=torch.float16, device=device)
             entry = (("awq_gemv" if M <= awq.GEMV_MAX_M else "awq_gemm") + (" silu_mul" if silu else "") +
-                     (" packed_zeros" if packed else ""))
+                     (" packed_zeros" if packed else "") + ("" if zp else " symmetric"))
             fn = awq.awq_gemv if M <= awq.GEMV_MAX_M else awq.awq_gemm
             kw = {"weights_static": True} if M <= awq.GEMV_MAX_M else {}
             if silu:
                 kw["silu_mul"] = True
-            ws = awq.alloc_workspace(M, N, K, True, device=device, silu_mul=silu)
+            ws = awq.alloc_workspace(M, N, K, zp, device=device, silu_mul=silu, packed_zeros=packed)
             stream = torch.cuda.Stream(device)
             with torch.cuda.stream(stream):
                 for qq, ss, zz in packs:
@@ -782,7 +790,7 @@ def run_table(args):
                     del gh
             us = cold_ms * 1e3 / (reps * copies)
             # y: N/2 columns with silu_mul; packed zero points: 4 bits instead of 16 per (row, group)
-            nbytes = algo_bytes(M, N, K) - (M * N if silu else 0) - (3 * N * (K // 128) // 2 if packed else 0)
+            nbytes = algo_bytes(M, N, K, zp) - (M * N if silu else 0) - (3 * N * (K // 128) // 2 if packed else 0)
             gbs = nbytes / (us * 1e-6) / 1e9
             tfl = algo_flops(M, N, K) / (us * 1e-6) / 1e12
             print(json.dumps({"entry": entry, "N": N, "K": K, "M": M, "us": round(us, 3), "GB/s": round(gbs, 1),

@@ -21,6 +21,8 @@
 
 #include <cuda_fp16.h>
 
+#include <atomic>
+
 #include "awq_common.cuh"
 
 
@@ -389,6 +391,19 @@ awq_status_t search_layout(int64_t N, int64_t K, int64_t Ms, awq_qconfig_t cfg, 
   return AWQ_OK;
 }
 
+// SM count of the current device (cached per device; 148 on B200 if the query fails).
+int device_sms() {
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  int v = cache[dev].load(std::memory_order_relaxed);
+  if (v == 0) {
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) return 148;
+    cache[dev].store(v, std::memory_order_relaxed);
+  }
+  return v;
+}
+
 awq_status_t check_search_args(int64_t N, int64_t K, int64_t Ms, awq_qconfig_t cfg) {
   awq_status_t st = check_cfg(cfg);
   if (st != AWQ_OK) return st;
@@ -453,7 +468,7 @@ extern "C" awq_status_t awq_search_scale(const uint16_t* W, int64_t N, int64_t K
                                                                                                    y_ref);
   if ((st = launch_status()) != AWQ_OK) return st;
   const int64_t outs = Ms * N;
-  const int sgrid = 148 * 8;
+  const int sgrid = device_sms() * 8;   // grid-stride column scaling: eight CTAs per SM
   for (int i = 0; i < n_grid; ++i) {
     candidate_kernel<<<1, 1024, 0, cs>>>(x_mean, w_mean, K, n_grid, i, losses_out, duo, s);
     scale_columns_kernel<<<sgrid, 256, 0, cs>>>(W, s, N, K, 1, w_s);
@@ -477,7 +492,7 @@ extern "C" awq_status_t awq_apply_scale(const uint16_t* W, const float* s, int64
   if (K % 8) return AWQ_ERR_SHAPE;
   if (!W || !s || !W_out) return AWQ_ERR_NULL;
   if (!aligned16(W) || !aligned16(W_out)) return AWQ_ERR_ALIGN;
-  scale_columns_kernel<<<148 * 8, 256, 0, static_cast<cudaStream_t>(stream)>>>(W, s, N, K, 1, W_out);
+  scale_columns_kernel<<<device_sms() * 8, 256, 0, static_cast<cudaStream_t>(stream)>>>(W, s, N, K, 1, W_out);
   return launch_status();
 }
 
@@ -526,7 +541,8 @@ extern "C" awq_status_t awq_apply_clip(const uint16_t* W, const float* ratios, i
   if (!aligned16(W) || !aligned16(W_out)) return AWQ_ERR_ALIGN;
   const int64_t units = N * (K / kGroup);
   const int64_t blocks = (units + 7) / 8;
-  apply_clip_kernel<<<unsigned(blocks < 148 * 16 ? blocks : 148 * 16), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+  const int64_t cap = int64_t(device_sms()) * 16;
+  apply_clip_kernel<<<unsigned(blocks < cap ? blocks : cap), 256, 0, static_cast<cudaStream_t>(stream)>>>(
       W, ratios, N, K, W_out);
   return launch_status();
 }
