@@ -137,3 +137,43 @@ def test_gemm_empty_batch():
     y = awq.awq_gemm(torch.empty((0, 512), dtype=torch.float16, device="cuda"), dev(qweight), dev(scales),
                      dev(zeros))
     assert y.shape == (0, 512)
+
+
+@pytest.mark.parametrize("zp", [True, False])
+@pytest.mark.parametrize("N,K", [(14336, 4096), (4096, 4096), (6144, 4096), (4096, 14336)])
+def test_gemm_small_batches_around_the_crossover(N, K, zp):
+    """Prefill batches between the GEMV range and a full 256-row tile of x
+    (M = 17 .. 128, and 160 / 256 on both sides of one x tile), where the
+    product may take 128-channel tiles: every output of sampled channels
+    against the float64 oracle, both zero-point variants, and the same bits
+    on a second call."""
+    W = make_weight(N, K, 0.02, 0.01, seed=21)
+    codes, scales, zeros = O.pseudo_quantize(W, 128, zp)
+    qweight = O.pack(codes)
+    rows = sample_rows(N, 256, seed=N)
+    Wd = O.dequant(codes[rows], scales[:, rows], zeros[:, rows] if zp else None, 128)
+    q, s, z = dev(qweight), dev(scales), dev(zeros) if zp else None
+    for M in (17, 24, 32, 48, 64, 96, 128, 160, 256):
+        xh = activations(M, K, seed=M)
+        x = dev(xh)
+        y = awq.awq_gemm(x, q, s, z)
+        y2 = awq.awq_gemm(x, q, s, z)
+        torch.cuda.synchronize()
+        assert_close(host(y)[:, rows], O.matmul_f64(xh, Wd), f"N={N} K={K} M={M} zp={zp}")
+        assert np.array_equal(bits(y), bits(y2)), f"M={M}: second call differs"
+
+
+@pytest.mark.parametrize("M", [24, 96, 128])
+def test_gemm_small_batches_fused_gate_up(M):
+    """The fused SiLU epilogue on 128-channel tiles (8 gate/up tile pairs per
+    256 channels, 4 per 128): against the float64 oracle of silu(gate) * up."""
+    N, K = 5632, 2048
+    Wg = make_weight(N, K, 0.02, 0.0, seed=31)
+    Wu = make_weight(N, K, 0.02, 0.0, seed=32)
+    cg, sg, zg = O.pseudo_quantize(Wg, 128, True)
+    cu, su, zu = O.pseudo_quantize(Wu, 128, True)
+    q, s, z = awq.awq_interleave_gate_up(dev(O.pack(cg)), dev(sg), dev(zg), dev(O.pack(cu)), dev(su), dev(zu))
+    xh = activations(M, K, seed=5)
+    y = host(awq.awq_gemm(dev(xh), q, s, z, silu_mul=True))
+    ref = O.gate_up_silu_f64(xh, O.dequant(cg, sg, zg, 128), O.dequant(cu, su, zu, 128))
+    assert_close(y, ref, f"fused M={M}")
