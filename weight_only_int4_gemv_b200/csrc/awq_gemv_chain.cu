@@ -471,10 +471,13 @@ chain_kernel(const __grid_constant__ ChainParams p) {
       }
       asm volatile("griddepcontrol.wait;" ::: "memory");
       const uint32_t target = gridDim.x;
-      uint64_t t_idle = 0;          // start of the current stretch without progress
+      // Starts of the two waits the producer can be in (0: not waiting): for
+      // the layer that the next x copy comes from, and for a free slot. A
+      // wait longer than the limit gives up.
+      uint64_t t_x = 0, t_slot = 0;
       bool gave_up = false;
       while (!cx.done(p.n_layers)) {
-        bool progress = false;
+        bool progress = false, slot_busy = false, x_blocked = false;
         if (!cw.done(p.n_layers)) {
           const int slot = sw % S;
           if (sw < S || mbar_test_wait(empty0 + 8 * slot, uint32_t((sw / S) + 1) & 1u)) {
@@ -482,6 +485,8 @@ chain_kernel(const __grid_constant__ ChainParams p) {
             cursor_next(p, cw);
             ++sw;
             progress = true;
+          } else {
+            slot_busy = true;
           }
         }
         if (sx < sw) {
@@ -498,13 +503,11 @@ chain_kernel(const __grid_constant__ ChainParams p) {
             cursor_next(p, cx);
             ++sx;
             progress = true;
+          } else {
+            x_blocked = true;
           }
         }
-        if (progress) {
-          t_idle = 0;
-          continue;
-        }
-        if (sx == sw && !cw.done(p.n_layers)) {
+        if (!progress && sx == sw && slot_busy) {
           // nothing to do until the next slot frees: sleep on its barrier
           const int slot = sw % S;
           mbar_sleep_wait(empty0 + 8 * slot, uint32_t((sw / S) + 1) & 1u, hint);
@@ -514,9 +517,11 @@ chain_kernel(const __grid_constant__ ChainParams p) {
           break;
         }
         const uint64_t now = now_ns();
-        if (t_idle == 0) {
-          t_idle = now;
-        } else if (now - t_idle > limit) {
+        if (!x_blocked) t_x = 0;
+        else if (t_x == 0) t_x = now;
+        if (!slot_busy) t_slot = 0;
+        else if (t_slot == 0) t_slot = now;
+        if ((t_x && now - t_x > limit) || (t_slot && now - t_slot > limit)) {
           *abort_flag = 1;
           atomicOr(&g_awq_chain_error, kErrBit);
           gave_up = true;
