@@ -24,7 +24,9 @@
 //   rotate the CTA order so that their leftover tiles land on different
 //   CTAs.
 // * Warp roles: one producer warp (one thread) issues every TMA copy; eight
-//   consumer warps decode and multiply. A stage of the ring is one chunk of
+//   consumer warps decode and multiply; one release warp (one thread)
+//   publishes the CTA's completed layers, so that no consumer waits for the
+//   acknowledgement of its stores. A stage of the ring is one chunk of
 //   up to four tiles x eight groups (one group per consumer warp): codes,
 //   scales, zero points and the matching slice of x. Consumers wait on the
 //   stage's "full" barrier, compute, and arrive on its "empty" barrier; the
@@ -33,6 +35,9 @@
 //   issued as soon as a slot frees up, but the copy of its x only once every
 //   CTA has counted itself done with layer d (a per-layer counter, released
 //   after the CTA's y stores and acquired by the producer before the copy).
+// * Schedule: each CTA's share of every layer (items, K slice, groups) and
+//   the layer fields the loops read are computed once at kernel start into a
+//   table in shared memory; the kernel parameters hold the tensor maps.
 // * Arithmetic (per consumer warp, one group of every tile of the stage):
 //   the packed nibble order puts consecutive k pairs in the low and high
 //   halves of a word, so one LOP3 with an fp16 magic number yields two exact
@@ -72,12 +77,16 @@ __device__ unsigned long long g_awq_chain_wait_limit_ns = kWaitLimitNs;
 namespace {
 
 constexpr int kCW = 8;                          // consumer warps
-constexpr int kThreads = (kCW + 1) * 32;        // + one producer warp
+constexpr int kProducerWarp = kCW;
+constexpr int kReleaseWarp = kCW + 1;
+constexpr int kThreads = (kCW + 2) * 32;        // + the producer and release warps
 constexpr int kTile = 16;                       // output channels per MMA tile
 constexpr int kMaxTC = 4;                       // tiles per chunk
 constexpr int kMaxLayers = AWQ_CHAIN_MAX_LAYERS;
 constexpr int kMaxStages = 8;
-constexpr int kHeader = 1024;                   // barriers and flags below the ring
+constexpr int kMaxHeader = 2048;                // barriers, flags and the layer table below the ring
+constexpr int kFlagsOff = kMaxStages * 16;      // abort flag, then the count of layers the consumers finished
+constexpr int kTableOff = 256;                  // LayerRun[n_layers]
 constexpr int kTileBytes = kCW * 1024;          // codes of one tile: [group][16 rows][16 words]
 constexpr int kScaleOff = kMaxTC * kTileBytes;  // scales: [group][64 rows] fp16
 constexpr int kMetaBytes = kCW * 64 * 2;
@@ -89,7 +98,7 @@ constexpr int kConsumerBarrier = 1;             // named barrier of the consumer
 constexpr uint32_t kErrBit = 4u;
 constexpr uint32_t kCodesBoxBytes = kTileBytes;
 
-static_assert(kMaxStages * 16 + 64 <= kHeader, "stage bookkeeping overflows its region");
+static_assert(kFlagsOff + 8 <= kTableOff, "stage bookkeeping overflows its region");
 static_assert(kXOff % 1024 == 0, "x must start 1024-aligned inside a stage");
 
 struct alignas(64) LayerDesc {
@@ -109,6 +118,33 @@ struct alignas(64) LayerDesc {
   int rot;             // CTA rotation of this layer's item ranges
   int silu;
 };
+
+// This CTA's share of one layer and the layer fields its loops read, filled
+// at kernel start (kernel parameters are read through the constant cache,
+// which misses for a table of 32 layer descriptors; shared memory does not).
+struct LayerRun {
+  int i0, i1;          // items of the CTA
+  int s;               // their K slice (a CTA never straddles two)
+  int gb, ge;          // the slice's groups
+  int units;
+  int N;
+  int info;            // tpu (bits 0-1), silu (bit 2), ks (bits 8-15), x_from + 1 (bits 16-23)
+  uint16_t* y;
+  float* partials;
+  uint32_t* counters;
+};
+static_assert(sizeof(LayerRun) == 56, "layer table entry");
+static_assert(kTableOff + kMaxLayers * sizeof(LayerRun) <= kMaxHeader, "layer table overflows the header");
+
+// Bytes below the ring: the table of n layers, rounded up to the ring's 1024-byte alignment.
+__host__ __device__ constexpr int header_bytes(int n) {
+  return (kTableOff + n * int(sizeof(LayerRun)) + 1023) / 1024 * 1024;
+}
+
+__host__ __device__ __forceinline__ int run_tpu(const LayerRun& r) { return r.info & 3; }
+__host__ __device__ __forceinline__ int run_silu(const LayerRun& r) { return (r.info >> 2) & 1; }
+__host__ __device__ __forceinline__ int run_ks(const LayerRun& r) { return (r.info >> 8) & 0xff; }
+__host__ __device__ __forceinline__ int run_x_from(const LayerRun& r) { return ((r.info >> 16) & 0xff) - 1; }
 
 struct ChainParams {
   LayerDesc layer[kMaxLayers];
@@ -236,11 +272,12 @@ struct Chunk {
 // same way, so that no CTA straddles two slices. Items are slice-major
 // (item = slice * units + unit). The same arithmetic runs on the host.
 __host__ __device__ __forceinline__ void split_items(int units, int ks, int grid, int b, int& i0, int& i1) {
+  // grid <= 2048 CTAs and ks <= 32 slices: the products fit in 32 bits
   int s = 0, b0 = 0, n = grid;
   if (ks > 1) {
-    s = int(int64_t(b) * ks / grid);
-    b0 = int((int64_t(s) * grid + ks - 1) / ks);
-    n = int((int64_t(s + 1) * grid + ks - 1) / ks) - b0;
+    s = b * ks / grid;
+    b0 = (s * grid + ks - 1) / ks;
+    n = ((s + 1) * grid + ks - 1) / ks - b0;
   }
   const int j = b - b0;
   const int q = units / n, r = units - q * n;
@@ -258,59 +295,72 @@ __device__ __forceinline__ void item_range(const LayerDesc& L, int& i0, int& i1)
   split_items(L.units, L.ks, grid, b, i0, i1);
 }
 
-__device__ __forceinline__ void load_chunk(const LayerDesc& L, int i, int i_end, Chunk& c) {
+// The CTA's share of layer l (thread-parallel at kernel start).
+__device__ __forceinline__ void fill_run(const LayerDesc& L, LayerRun& r) {
+  item_range(L, r.i0, r.i1);
+  r.s = r.i0 < r.i1 ? r.i0 / L.units : 0;
+  r.gb = L.G * r.s / L.ks;            // G < 2^25, ks <= 32
+  r.ge = L.G * (r.s + 1) / L.ks;
+  r.units = L.units;
+  r.N = L.N;
+  r.info = L.tpu | (L.silu << 2) | (L.ks << 8) | ((L.x_from + 1) << 16);
+  r.y = L.y;
+  r.partials = L.partials;
+  r.counters = L.counters;
+}
+
+__device__ __forceinline__ void load_chunk(const LayerRun& R, int i, Chunk& c) {
+  const int tpu = run_tpu(R);
   c.i = i;
-  c.s = i / L.units;
-  const int u0 = i - c.s * L.units;
-  int nu = i_end - i;
-  const int cap = kMaxTC / L.tpu;
+  c.s = R.s;
+  const int u0 = i - R.s * R.units;
+  int nu = R.i1 - i;
+  const int cap = kMaxTC / tpu;
   if (nu > cap) nu = cap;
-  if (nu > L.units - u0) nu = L.units - u0;
+  if (nu > R.units - u0) nu = R.units - u0;
   c.nu = nu;
-  c.t0 = u0 * L.tpu;
-  c.tc = nu * L.tpu;
-  c.gb = int(int64_t(L.G) * c.s / L.ks);
-  c.ge = int(int64_t(L.G) * (c.s + 1) / L.ks);
+  c.t0 = u0 * tpu;
+  c.tc = nu * tpu;
+  c.gb = R.gb;
+  c.ge = R.ge;
 }
 
 // Flat cursor over (layer, chunk, stage) for the producer.
 struct Cursor {
-  int l, i1;
+  int l;
   Chunk c;
   int gbase;
   __device__ __forceinline__ bool done(int n) const { return l >= n; }
 };
 
-__device__ __forceinline__ void cursor_layer(const ChainParams& p, Cursor& u) {
+__device__ __forceinline__ void cursor_layer(const ChainParams& p, const LayerRun* runs, Cursor& u) {
   // from layer u.l on, the first layer with items for this CTA
   for (; u.l < p.n_layers; ++u.l) {
-    int i0, i1;
-    item_range(p.layer[u.l], i0, i1);
-    if (i0 < i1) {
-      u.i1 = i1;
-      load_chunk(p.layer[u.l], i0, i1, u.c);
+    const LayerRun& R = runs[u.l];
+    if (R.i0 < R.i1) {
+      load_chunk(R, R.i0, u.c);
       u.gbase = u.c.gb;
       return;
     }
   }
 }
 
-__device__ __forceinline__ void cursor_init(const ChainParams& p, Cursor& u) {
+__device__ __forceinline__ void cursor_init(const ChainParams& p, const LayerRun* runs, Cursor& u) {
   u.l = 0;
-  cursor_layer(p, u);
+  cursor_layer(p, runs, u);
 }
 
-__device__ __forceinline__ void cursor_next(const ChainParams& p, Cursor& u) {
+__device__ __forceinline__ void cursor_next(const ChainParams& p, const LayerRun* runs, Cursor& u) {
   u.gbase += kCW;
   if (u.gbase < u.c.ge) return;
   const int ni = u.c.i + u.c.nu;
-  if (ni < u.i1) {
-    load_chunk(p.layer[u.l], ni, u.i1, u.c);
+  if (ni < runs[u.l].i1) {
+    load_chunk(runs[u.l], ni, u.c);
     u.gbase = u.c.gb;
     return;
   }
   ++u.l;
-  cursor_layer(p, u);
+  cursor_layer(p, runs, u);
 }
 
 template <int ZM>
@@ -426,7 +476,7 @@ __device__ __forceinline__ void stage_compute(uint32_t st, int w, int g, int t, 
 // the kernel
 // ---------------------------------------------------------------------------
 template <int MB, int ZM>
-__global__ void __launch_bounds__(kThreads, MB <= 8 ? 2 : 1)
+__global__ void __launch_bounds__(kThreads, MB == 1 ? 2 : 1)
 chain_kernel(const __grid_constant__ ChainParams p) {
   constexpr int MT = MB > 8 ? 2 : 1;
   asm volatile("griddepcontrol.launch_dependents;");
@@ -434,8 +484,11 @@ chain_kernel(const __grid_constant__ ChainParams p) {
   const uint32_t sbase = smem_u32(smem);
   const uint32_t full0 = sbase;                        // [S] mbarriers
   const uint32_t empty0 = sbase + kMaxStages * 8;      // [S] mbarriers
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kMaxStages * 16);
-  const uint32_t ring = sbase + kHeader;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kFlagsOff);
+  // layers the consumers have finished (written by consumer thread 0, read by the release warp)
+  const uint32_t layers_done = sbase + kFlagsOff + 4;
+  LayerRun* runs = reinterpret_cast<LayerRun*>(smem + kTableOff);
+  const uint32_t ring = sbase + header_bytes(p.n_layers);
   const int S = p.stages;
   const int warp = int(threadIdx.x) >> 5;
   const int lane = int(threadIdx.x) & 31;
@@ -448,16 +501,18 @@ chain_kernel(const __grid_constant__ ChainParams p) {
       asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(empty0 + 8 * s), "r"(kCW));
     }
     *abort_flag = 0;
+    asm volatile("st.shared.u32 [%0], 0;" ::"r"(layers_done) : "memory");
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     fence_proxy_async_smem();
   }
+  for (int l = int(threadIdx.x); l < p.n_layers; l += int(blockDim.x)) fill_run(p.layer[l], runs[l]);
   __syncthreads();
 
-  if (warp == kCW) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       Cursor cw, cx;
-      cursor_init(p, cw);
+      cursor_init(p, runs, cw);
       cx = cw;
       int sw = 0, sx = 0;           // stages whose weights / x have been issued
       uint32_t ready = 0;           // layers whose x may be read
@@ -466,7 +521,7 @@ chain_kernel(const __grid_constant__ ChainParams p) {
       if (p.early) {
         for (; sw < S && !cw.done(p.n_layers); ++sw) {
           issue_weights<ZM>(p, cw, ring + sw * p.stage_bytes, full0 + 8 * sw);
-          cursor_next(p, cw);
+          cursor_next(p, runs, cw);
         }
       }
       asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -482,7 +537,7 @@ chain_kernel(const __grid_constant__ ChainParams p) {
           const int slot = sw % S;
           if (sw < S || mbar_test_wait(empty0 + 8 * slot, uint32_t((sw / S) + 1) & 1u)) {
             issue_weights<ZM>(p, cw, ring + slot * p.stage_bytes, full0 + 8 * slot);
-            cursor_next(p, cw);
+            cursor_next(p, runs, cw);
             ++sw;
             progress = true;
           } else {
@@ -492,7 +547,7 @@ chain_kernel(const __grid_constant__ ChainParams p) {
         if (sx < sw) {
           const int l = cx.l;
           if (!((ready >> l) & 1u)) {
-            if (ld_acquire_gpu(p.done + p.layer[l].x_from) >= target) {
+            if (ld_acquire_gpu(p.done + run_x_from(runs[l])) >= target) {
               asm volatile("fence.proxy.async.global;" ::: "memory");
               ready |= 1u << l;
             }
@@ -500,7 +555,7 @@ chain_kernel(const __grid_constant__ ChainParams p) {
           if ((ready >> l) & 1u) {
             const int slot = sx % S;
             issue_x(p, cx, ring + slot * p.stage_bytes, full0 + 8 * slot);
-            cursor_next(p, cx);
+            cursor_next(p, runs, cx);
             ++sx;
             progress = true;
           } else {
@@ -534,7 +589,7 @@ chain_kernel(const __grid_constant__ ChainParams p) {
         for (; sx < sw; ++sx) {
           const int slot = sx % S;
           issue_x(p, cx, ring + slot * p.stage_bytes, full0 + 8 * slot);
-          cursor_next(p, cx);
+          cursor_next(p, runs, cx);
         }
       }
       // every copy issued must land before the CTA exits: the last phase
@@ -546,6 +601,38 @@ chain_kernel(const __grid_constant__ ChainParams p) {
         const uint64_t t0 = now_ns();
         while (!mbar_try_wait_u32(full0 + 8 * slot, par) && now_ns() - t0 < kWaitLimitNs) {
         }
+      }
+    }
+    __syncwarp();
+  } else if (warp == kReleaseWarp) {
+    // ------------------------------------------------------------ release
+    // Publishes each layer once the consumers have finished it: their
+    // stores are ordered before consumer thread 0's release of the count
+    // (named barrier), this thread acquires the count, and its gpu-scope
+    // release of the layer's done counter covers them.
+    if (lane == 0) {
+      // the previous launch's last CTA resets the counters: wait for it
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      uint64_t t0 = 0;
+      for (int l = 0; l < p.n_layers;) {
+        uint32_t n;
+        asm volatile("ld.acquire.cta.shared.u32 %0, [%1];" : "=r"(n) : "r"(layers_done) : "memory");
+        if (n > uint32_t(l)) {
+          for (; l < int(n); ++l) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(p.done + l) : "memory");
+          t0 = 0;
+          continue;
+        }
+        const uint64_t now = now_ns();
+        if (t0 == 0) {
+          t0 = now;
+        } else if (now - t0 > kWaitLimitNs) {
+          // the consumers count every layer even after giving up, so this
+          // is reached only if they stopped: let the others give up too
+          *abort_flag = 1;
+          atomicOr(&g_awq_chain_error, kErrBit);
+          break;
+        }
+        __nanosleep(64);
       }
     }
     __syncwarp();
@@ -561,12 +648,14 @@ chain_kernel(const __grid_constant__ ChainParams p) {
     uint32_t phase = 0;
     bool live = true;
     for (int l = 0; l < p.n_layers; ++l) {
-      const LayerDesc& L = p.layer[l];
-      int i0, i1;
-      item_range(L, i0, i1);
-      for (int i = i0; i < i1;) {
+      const LayerRun& R = runs[l];
+      const int i1 = R.i1;
+      const int ks = run_ks(R), tpu = run_tpu(R), silu = run_silu(R), N = R.N;
+      const int T = R.units * tpu;
+      uint16_t* const y = R.y;
+      for (int i = R.i0; i < i1;) {
         Chunk cc;
-        load_chunk(L, i, i1, cc);
+        load_chunk(R, i, cc);
         float acc[kMaxTC][MT][4];
 #pragma unroll
         for (int rt = 0; rt < kMaxTC; ++rt)
@@ -629,7 +718,7 @@ chain_kernel(const __grid_constant__ ChainParams p) {
         consumer_sync();
         const int64_t row0 = int64_t(cc.t0) * kTile;
         const int tid = int(threadIdx.x);
-        if (!L.silu || L.ks > 1) {
+        if (!silu || ks > 1) {
           const int V = kTile * cc.tc * M;
           for (int v = tid; v < V; v += kCW * 32) {
             float sum = 0.0f;
@@ -637,10 +726,10 @@ chain_kernel(const __grid_constant__ ChainParams p) {
             for (int ww = 0; ww < kCW; ++ww) sum += lds_f32(pbuf + uint32_t(ww * 64 * M + v) * 4);
             const int row = v / M;
             const int m = v - row * M;
-            if (L.ks == 1) {
-              if (row0 + row < L.N) L.y[int64_t(m) * L.N + row0 + row] = __half_as_ushort(__float2half_rn(sum));
+            if (ks == 1) {
+              if (row0 + row < N) y[int64_t(m) * N + row0 + row] = __half_as_ushort(__float2half_rn(sum));
             } else {
-              __stcg(L.partials + ((int64_t(cc.s) * L.T * kTile + row0 + row) * M + m), sum);
+              __stcg(R.partials + ((int64_t(cc.s) * T * kTile + row0 + row) * M + m), sum);
             }
           }
         } else {
@@ -658,60 +747,60 @@ chain_kernel(const __grid_constant__ ChainParams p) {
             }
             const int row = rem / M;
             const int m = rem - row * M;
-            L.y[int64_t(m) * (L.N / 2) + row0 / 2 + q * kTile + row] =
+            y[int64_t(m) * (N / 2) + row0 / 2 + q * kTile + row] =
                 __half_as_ushort(__float2half_rn(silu_f32(gs) * us));
           }
         }
-        if (L.ks > 1) {
+        if (ks > 1) {
           // slices of a unit meet in the workspace: the CTA whose arrival
           // brings a unit's count to ks sums the ks partials in slice order.
           // The barrier orders every consumer's partial stores before the
           // arrivals, whose release makes them visible at GPU scope.
           consumer_sync();
           if (w < cc.nu) {
-            const int unit = cc.t0 / L.tpu + w;
+            const int unit = cc.t0 / tpu + w;
             uint32_t last = 0;
             if (lane == 0) {
               uint32_t old;
               asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
-                           : "=r"(old) : "l"(L.counters + unit) : "memory");
-              last = (old + 1 == uint32_t(L.ks)) ? 1u : 0u;
+                           : "=r"(old) : "l"(R.counters + unit) : "memory");
+              last = (old + 1 == uint32_t(ks)) ? 1u : 0u;
             }
             last = __shfl_sync(0xffffffffu, last, 0);
             __syncwarp();   // lane 0's acquire orders the warp's partial reads
             if (last) {
-              const int64_t trow = int64_t(unit) * L.tpu * kTile;
-              if (L.tpu == 1) {
+              const int64_t trow = int64_t(unit) * tpu * kTile;
+              if (tpu == 1) {
                 for (int v = lane; v < kTile * M; v += 32) {
                   float sum = 0.0f;
-                  for (int s = 0; s < L.ks; ++s) sum += __ldcg(L.partials + ((int64_t(s) * L.T * kTile + trow) * M + v));
+                  for (int s = 0; s < ks; ++s) sum += __ldcg(R.partials + ((int64_t(s) * T * kTile + trow) * M + v));
                   const int row = v / M;
                   const int m = v - row * M;
-                  if (trow + row < L.N) L.y[int64_t(m) * L.N + trow + row] = __half_as_ushort(__float2half_rn(sum));
+                  if (trow + row < N) y[int64_t(m) * N + trow + row] = __half_as_ushort(__float2half_rn(sum));
                 }
               } else {
                 for (int v = lane; v < kTile * M; v += 32) {
                   float gs = 0.0f, us = 0.0f;
-                  for (int s = 0; s < L.ks; ++s) {
-                    const float* ps = L.partials + (int64_t(s) * L.T * kTile + trow) * M;
+                  for (int s = 0; s < ks; ++s) {
+                    const float* ps = R.partials + (int64_t(s) * T * kTile + trow) * M;
                     gs += __ldcg(ps + v);
                     us += __ldcg(ps + kTile * M + v);
                   }
                   const int row = v / M;
                   const int m = v - row * M;
-                  L.y[int64_t(m) * (L.N / 2) + trow / 2 + row] = __half_as_ushort(__float2half_rn(silu_f32(gs) * us));
+                  y[int64_t(m) * (N / 2) + trow / 2 + row] = __half_as_ushort(__float2half_rn(silu_f32(gs) * us));
                 }
               }
-              if (lane == 0) L.counters[unit] = 0u;
+              if (lane == 0) R.counters[unit] = 0u;
             }
           }
         }
         consumer_sync();   // pbuf is reused by the next chunk; the layer's stores are done
         i += cc.nu;
       }
-      // This CTA is done with layer l: release its y stores (and fixups) to
-      // the producers that wait for the layer.
-      if (threadIdx.x == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(p.done + l) : "memory");
+      // This CTA is done with layer l (the chunk's last barrier ordered every
+      // consumer's stores before this point): the release warp publishes it.
+      if (threadIdx.x == 0) asm volatile("st.release.cta.shared.u32 [%0], %1;" ::"r"(layers_done), "r"(l + 1) : "memory");
     }
   }
   __syncthreads();
@@ -880,13 +969,13 @@ awq_status_t make_chain_plan(const awq_gemv_layer_t* layers, int n, int64_t M, C
   int per_sm = 2;
   for (;; --per_sm) {
     const int budget = per_sm == 2 ? kHalfSmBudget : kSmemBudget;
-    int st = (budget - kHeader - pbuf_bytes) / pl.stage_bytes;
+    int st = (budget - header_bytes(n) - pbuf_bytes) / pl.stage_bytes;
     if (st > kMaxStages) st = kMaxStages;
     pl.stages = st;
     if (st >= 3 || per_sm == 1) break;
   }
   if (pl.stages < 2) return AWQ_ERR_UNSUPPORTED;
-  pl.pbuf_offset = kHeader + pl.stages * pl.stage_bytes;
+  pl.pbuf_offset = header_bytes(n) + pl.stages * pl.stage_bytes;
   pl.smem = pl.pbuf_offset + pbuf_bytes;
   int occ = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, pl.fn, kThreads, size_t(pl.smem)) != cudaSuccess)
