@@ -266,8 +266,9 @@ AWQ_API awq_status_t awq_gemv_noalloc(const uint16_t* x, const int32_t* qweight,
  * y is [M][N_l/2]). The results are bit-identical to n_layers awq_gemv
  * calls made in order on the same stream whenever each layer's split of K
  * is the same (it is whenever N_l / 16 is at least twice the SM count).
- * The launch streams the weights of all layers back to back; a layer's x
- * is read only after the layer it comes from is complete.
+ * The launch streams the weights of all layers back to back; a layer that
+ * reads an earlier layer's output takes its x from a copy of that output in
+ * the workspace and uses each value only once it has been written.
  *
  * x_from = -1: x is ready when the call starts (written by earlier work on
  * the stream). x_from = d (0 <= d < l): x is layer d's y of this call; x
@@ -282,9 +283,12 @@ AWQ_API awq_status_t awq_gemv_noalloc(const uint16_t* x, const int32_t* qweight,
  * finished only if every layer carries AWQ_FLAG_WEIGHTS_STATIC.
  * layers: host memory, read before the call returns.
  * workspace: at least awq_gemv_chain_workspace_bytes() bytes of device
- * memory, zero-filled before its first use; every call that completes (also
- * one whose waits gave up, see awq_device_error) brings its counters back to
- * zero, so one memset at allocation suffices.
+ * memory, zero-filled before its first use and then kept for calls with the
+ * same layers (shapes, flags, x_from; the pointers may change) and not
+ * written by anything else: between calls it holds a launch count and the
+ * half of the output-copy region that the next call reads, zeroed (every
+ * call that completes, also one whose waits gave up, leaves it so). A call
+ * with other layers needs its own workspace, or this one zero-filled again.
  * Calls that may run concurrently need separate workspaces.
  * Every CTA of the launch must be resident at once (the grid is sized from
  * the occupancy of the kernel on this device): do not run other kernels

@@ -138,10 +138,10 @@ def test_chain_every_batch_size_small_layers():
 
 
 def test_chain_repeated_calls_and_graph_replay():
-    """The workspace counters return to zero after each call: repeated calls,
+    """The workspace is left ready for the next call: repeated calls,
     and a CUDA graph of two chained launches replayed twice, give the eager
-    bits (a counter left over would skip or repeat a K-slice sum, or release
-    a layer's input too early)."""
+    bits (a counter left over would skip or repeat a K-slice sum; an output
+    copy left from the previous call would be read as this call's input)."""
     shapes = [(2048, 2048, -1), (2048, 2048, 0), (8192, 2048, 1), (2048, 8192, 2)]
     ls = [oracle_layer(N, K, 0.02, 0.01, True, seed=90 + i) for i, (N, K, _) in enumerate(shapes)]
     M = 2
@@ -218,3 +218,38 @@ def test_chain_wait_gives_up_and_recovers():
     refs = _oracle_chain(xh, [(layer[4], xf) for layer, (_, _, xf) in zip(ls, shapes)])
     for i, (y, ref) in enumerate(zip(ys, refs)):
         assert_close(host(y), ref, f"after recovery layer {i}")
+
+
+def test_chains_taking_turns_on_one_workspace():
+    """Two chains of different layers on one workspace, each call after the
+    first of a chain made on a freshly zeroed workspace (the contract when
+    the layers change), and a chain called twice in a row on it: every call
+    gives the bits of the same chain on a workspace of its own."""
+    M = 1
+    shapes_a = [(4096, 2048, -1), (2048, 4096, 0), (4096, 2048, 1)]
+    shapes_b = [(1024, 4096, -1), (8192, 1024, 0), (4096, 8192, 1), (4096, 4096, 2)]
+    chains = []
+    for shapes, seed in ((shapes_a, 120), (shapes_b, 130)):
+        specs = []
+        for i, (N, K, xf) in enumerate(shapes):
+            q, s_, z = _packed(oracle_layer(N, K, 0.02, 0.01, True, seed=seed + i), True)
+            specs.append(dict(x=dev(activations(M, K, seed=seed)) if xf < 0 else None, x_from=xf,
+                              qweight=q, scales=s_, zeros=z))
+        chains.append(specs)
+    own = [awq.GemvChain(M, sp, weights_static=True) for sp in chains]
+    for c in own:
+        c()
+    torch.cuda.synchronize()
+    ref = [[bits(y).copy() for y in c.outputs] for c in own]
+    need = max(c.workspace.numel() for c in own)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    shared = [awq.GemvChain(M, sp, weights_static=True, workspace=ws) for sp in chains]
+    for k, which in enumerate([0, 0, 1, 1, 1, 0, 1]):
+        if k > 0 and which != [0, 0, 1, 1, 1, 0, 1][k - 1]:
+            ws.zero_()
+        c = shared[which]
+        c()
+        torch.cuda.synchronize()
+        for i, y in enumerate(c.outputs):
+            assert np.array_equal(bits(y), ref[which][i]), f"call {k} (chain {which}) layer {i}"
+    assert awq.awq_device_error() == 0

@@ -547,14 +547,17 @@ class GemvChain:
                               whose output is this layer's input
       silu_mul                fused gate/up layout (output N/2 columns)
       out                     optional fp16 output tensor
-    The outputs (self.outputs) and a zero-filled workspace are allocated here;
-    calling the object enqueues the launch on the current stream. The layer
-    descriptors are built once, so repeated calls cost one library call.
+    The outputs (self.outputs) and a zero-filled workspace are allocated here
+    (workspace: a uint8 device tensor to use instead; it must be zero-filled
+    before the first call of this chain and then serve no other chain, or be
+    zero-filled again in between); calling the object enqueues the launch on
+    the current stream. The layer descriptors are built once, so repeated
+    calls cost one library call.
     weights_static: no work still running on the stream writes the weights,
     so the launch may start streaming them before the previous kernel on the
     stream has finished."""
 
-    def __init__(self, M: int, layers, weights_static: bool = False, device=None):
+    def __init__(self, M: int, layers, weights_static: bool = False, device=None, workspace=None):
         layers = list(layers)
         n = len(layers)
         if not 1 <= n <= CHAIN_MAX_LAYERS:
@@ -596,7 +599,15 @@ class GemvChain:
         with torch.cuda.device(self.device):
             _check("awq_gemv_chain_workspace_bytes",
                    lib().awq_gemv_chain_workspace_bytes(arr, n, self.M, ctypes.byref(nbytes)))
-        self.workspace = torch.zeros(max(int(nbytes.value), 16), dtype=torch.uint8, device=self.device)
+        if workspace is None:
+            workspace = torch.zeros(max(int(nbytes.value), 16), dtype=torch.uint8, device=self.device)
+        else:
+            _need(workspace, "workspace", torch.uint8, 1)
+            if workspace.device != self.device:
+                raise ValueError(f"workspace is on {workspace.device}, the chain on {self.device}")
+            if workspace.numel() < int(nbytes.value):
+                raise ValueError(f"workspace has {workspace.numel()} bytes, the chain needs {int(nbytes.value)}")
+        self.workspace = workspace
         self._ws = (self.workspace.data_ptr(), self.workspace.numel())
 
     def __call__(self):

@@ -24,17 +24,23 @@
 //   rotate the CTA order so that their leftover tiles land on different
 //   CTAs.
 // * Warp roles: one producer warp (one thread) issues every TMA copy; eight
-//   consumer warps decode and multiply; one release warp (one thread)
-//   publishes the CTA's completed layers, so that no consumer waits for the
-//   acknowledgement of its stores. A stage of the ring is one chunk of
+//   consumer warps decode and multiply. A stage of the ring is one chunk of
 //   up to four tiles x eight groups (one group per consumer warp): codes,
 //   scales, zero points and the matching slice of x. Consumers wait on the
 //   stage's "full" barrier, compute, and arrive on its "empty" barrier; the
 //   producer refills a slot once its empty barrier completes.
 // * Dependencies: a layer whose x is the y of layer d has its weight copies
-//   issued as soon as a slot frees up, but the copy of its x only once every
-//   CTA has counted itself done with layer d (a per-layer counter, released
-//   after the CTA's y stores and acquired by the producer before the copy).
+//   issued as soon as a slot frees up; its x comes from an exchange copy of
+//   d's output in the workspace, in which every 16-bit value is stored as
+//   its bit pattern plus one, so that 0 means "not written by this launch".
+//   Each consumer warp loads its own group of x one stage ahead (plain loads
+//   into registers), and before the stage checks that no value is 0,
+//   reloading until all are written; it then stores the decoded values into
+//   the stage's x region. No counter, fence or flag sits between the last
+//   store of layer d and the first use of its values. The exchange region
+//   has two halves used by alternate launches (the parity of a launch count
+//   kept in the workspace); each launch zeroes its share of the half the
+//   previous launch used.
 // * Schedule: each CTA's share of every layer (items, K slice, groups) and
 //   the layer fields the loops read are computed once at kernel start into a
 //   table in shared memory; the kernel parameters hold the tensor maps.
@@ -51,11 +57,10 @@
 //   of its own batch columns. Then acc += s (raw - C - z S).
 // * Every wait is bounded. A wait that gives up records bit 2 of the device
 //   error word and raises the CTA's abort flag; the CTA then walks the rest
-//   of its schedule without waiting or computing (so every named barrier,
-//   arrival counter and done counter is still reached), the producer issues
-//   the activation copies still missing from stages whose weights it issued
-//   (so every armed phase completes) and waits, bounded, for all copies in
-//   flight before the CTA exits. The output is then incomplete.
+//   of its schedule without waiting or computing (so every named barrier and
+//   arrival counter is still reached, and every output is still written),
+//   and the producer waits, bounded, for all copies in flight before the
+//   CTA exits. The output is then incomplete.
 
 #include "awq_common.cuh"
 #include "awq_tma_host.h"
@@ -77,15 +82,13 @@ __device__ unsigned long long g_awq_chain_wait_limit_ns = kWaitLimitNs;
 namespace {
 
 constexpr int kCW = 8;                          // consumer warps
-constexpr int kProducerWarp = kCW;
-constexpr int kReleaseWarp = kCW + 1;
-constexpr int kThreads = (kCW + 2) * 32;        // + the producer and release warps
+constexpr int kThreads = (kCW + 1) * 32;        // + one producer warp
 constexpr int kTile = 16;                       // output channels per MMA tile
 constexpr int kMaxTC = 4;                       // tiles per chunk
 constexpr int kMaxLayers = AWQ_CHAIN_MAX_LAYERS;
 constexpr int kMaxStages = 8;
 constexpr int kMaxHeader = 2048;                // barriers, flags and the layer table below the ring
-constexpr int kFlagsOff = kMaxStages * 16;      // abort flag, then the count of layers the consumers finished
+constexpr int kFlagsOff = kMaxStages * 16;      // abort flag
 constexpr int kTableOff = 256;                  // LayerRun[n_layers]
 constexpr int kTileBytes = kCW * 1024;          // codes of one tile: [group][16 rows][16 words]
 constexpr int kScaleOff = kMaxTC * kTileBytes;  // scales: [group][64 rows] fp16
@@ -107,8 +110,10 @@ struct alignas(64) LayerDesc {
   CUtensorMap ts;      // scales: {N, G}, box {64, kCW}
   CUtensorMap tz;      // zeros: {N, G} box {64, kCW}, or packed {N/8 words, G} box {12, kCW}
   uint16_t* y;
-  float* partials;     // [ks][T * 16][M], only when ks > 1
-  uint32_t* counters;  // [units], only when ks > 1
+  uint32_t partial_off;  // workspace offset of the partials [ks][T * 16][M] (ks > 1)
+  uint32_t counter_off;  // workspace offset of the arrival counters [units] (ks > 1)
+  uint32_t ll_off;       // offset of the exchange copy [M][N or N/2] in each half (source layers)
+  int source;            // a later layer reads this layer's output
   int N, G, T;
   int tpu;             // tiles per unit: 1, or 2 (gate tile + up tile, fused SiLU epilogue)
   int units;           // T / tpu
@@ -123,15 +128,15 @@ struct alignas(64) LayerDesc {
 // at kernel start (kernel parameters are read through the constant cache,
 // which misses for a table of 32 layer descriptors; shared memory does not).
 struct LayerRun {
-  int i0, i1;          // items of the CTA
-  int s;               // their K slice (a CTA never straddles two)
+  int i0, i1;          // items of the CTA (all in one K slice)
   int gb, ge;          // the slice's groups
   int units;
   int N;
-  int info;            // tpu (bits 0-1), silu (bit 2), ks (bits 8-15), x_from + 1 (bits 16-23)
+  int G;
+  int info;            // tpu (bits 0-1), silu (bit 2), source (bit 3), ks (bits 8-15), x_from + 1 (bits 16-23)
   uint16_t* y;
-  float* partials;
-  uint32_t* counters;
+  uint32_t partial_off, counter_off, ll_off;
+  int next;            // the next layer with items for this CTA (n_layers: none)
 };
 static_assert(sizeof(LayerRun) == 56, "layer table entry");
 static_assert(kTableOff + kMaxLayers * sizeof(LayerRun) <= kMaxHeader, "layer table overflows the header");
@@ -143,12 +148,20 @@ __host__ __device__ constexpr int header_bytes(int n) {
 
 __host__ __device__ __forceinline__ int run_tpu(const LayerRun& r) { return r.info & 3; }
 __host__ __device__ __forceinline__ int run_silu(const LayerRun& r) { return (r.info >> 2) & 1; }
+__host__ __device__ __forceinline__ int run_source(const LayerRun& r) { return (r.info >> 3) & 1; }
 __host__ __device__ __forceinline__ int run_ks(const LayerRun& r) { return (r.info >> 8) & 0xff; }
 __host__ __device__ __forceinline__ int run_x_from(const LayerRun& r) { return ((r.info >> 16) & 0xff) - 1; }
 
+// Control words at the start of the workspace.
+constexpr int kExitWord = 0;     // CTAs done with the call (the last one resets it)
+constexpr int kEpochWord = 1;    // launches completed on this workspace: its parity picks the exchange half
+constexpr int kControlBytes = 256;
+
 struct ChainParams {
   LayerDesc layer[kMaxLayers];
-  uint32_t* done;      // [n_layers] CTAs done with each layer; done[kMaxLayers]: CTAs done with the call
+  char* ws;            // workspace: control words, split-K partials and counters, the exchange region
+  uint32_t ll_base;    // offset of the exchange region (two halves of ll_half bytes)
+  uint32_t ll_half;
   int n_layers, M, stages, stage_bytes, pbuf_offset, early;
 };
 
@@ -235,10 +248,27 @@ __device__ __forceinline__ bool mbar_sleep_wait(uint32_t bar, uint32_t parity, u
   return ok != 0;
 }
 
-__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
-  uint32_t v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+// The exchange copy of a layer's output: each fp16 value v is stored as
+// v + 1 (the pattern 0xFFFF, a NaN that the conversion never produces, is
+// first replaced by the canonical NaN 0x7FFF), so that 0 marks a value not
+// written by this launch. Stores and loads are relaxed at gpu scope: a value
+// is either 0 or complete (16-bit accesses are single-copy atomic), so a
+// reader needs no ordering, only to see every value of its slice non-zero.
+__device__ __forceinline__ void ll_put(char* base, int64_t idx, uint16_t h) {
+  const uint16_t e = uint16_t((h == 0xFFFFu ? 0x7FFFu : h) + 1u);
+  asm volatile("st.relaxed.gpu.global.u16 [%0], %1;" ::"l"(base + idx * 2), "h"(e) : "memory");
+}
+__device__ __forceinline__ uint2 ll_get2(const char* a) {
+  uint2 v;
+  asm volatile("ld.relaxed.gpu.global.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(a) : "memory");
   return v;
+}
+__device__ __forceinline__ bool ll_complete(uint2 v) { return (__vcmpeq2(v.x, 0u) | __vcmpeq2(v.y, 0u)) == 0u; }
+__device__ __forceinline__ uint2 ll_decode(uint2 v) {
+  return make_uint2(__vsub2(v.x, 0x00010001u), __vsub2(v.y, 0x00010001u));
+}
+__device__ __forceinline__ void sts64(uint32_t a, uint2 v) {
+  asm volatile("st.shared.v2.u32 [%0], {%1,%2};" ::"r"(a), "r"(v.x), "r"(v.y) : "memory");
 }
 
 __device__ __forceinline__ void tma_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z, uint32_t bar) {
@@ -298,22 +328,24 @@ __device__ __forceinline__ void item_range(const LayerDesc& L, int& i0, int& i1)
 // The CTA's share of layer l (thread-parallel at kernel start).
 __device__ __forceinline__ void fill_run(const LayerDesc& L, LayerRun& r) {
   item_range(L, r.i0, r.i1);
-  r.s = r.i0 < r.i1 ? r.i0 / L.units : 0;
-  r.gb = L.G * r.s / L.ks;            // G < 2^25, ks <= 32
-  r.ge = L.G * (r.s + 1) / L.ks;
+  const int s = r.i0 < r.i1 ? r.i0 / L.units : 0;
+  r.gb = L.G * s / L.ks;            // G < 2^25, ks <= 32
+  r.ge = L.G * (s + 1) / L.ks;
   r.units = L.units;
   r.N = L.N;
-  r.info = L.tpu | (L.silu << 2) | (L.ks << 8) | ((L.x_from + 1) << 16);
+  r.G = L.G;
+  r.info = L.tpu | (L.silu << 2) | (L.source << 3) | (L.ks << 8) | ((L.x_from + 1) << 16);
   r.y = L.y;
-  r.partials = L.partials;
-  r.counters = L.counters;
+  r.partial_off = L.partial_off;
+  r.counter_off = L.counter_off;
+  r.ll_off = L.ll_off;
 }
 
 __device__ __forceinline__ void load_chunk(const LayerRun& R, int i, Chunk& c) {
   const int tpu = run_tpu(R);
   c.i = i;
-  c.s = R.s;
-  const int u0 = i - R.s * R.units;
+  c.s = i / R.units;
+  const int u0 = i - c.s * R.units;
   int nu = R.i1 - i;
   const int cap = kMaxTC / tpu;
   if (nu > cap) nu = cap;
@@ -374,10 +406,14 @@ __device__ __forceinline__ uint32_t weight_bytes(int tc) {
 // points (packed: 12 words from word 2 t0 rounded down to a multiple of 4,
 // a 16-byte boundary).
 template <int ZM>
-__device__ __forceinline__ void issue_weights(const ChainParams& p, const Cursor& u, uint32_t st, uint32_t bar) {
+__device__ __forceinline__ void issue_weights(const ChainParams& p, const LayerRun* runs, const Cursor& u, uint32_t st,
+                                              uint32_t bar) {
   const LayerDesc& L = p.layer[u.l];
+  // the x of a layer that reads an earlier layer's output comes from the
+  // consumers, not from a copy
+  const uint32_t xb = run_x_from(runs[u.l]) < 0 ? uint32_t(p.M) * kXRowBytes : 0u;
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar),
-               "r"(weight_bytes<ZM>(u.c.tc) + uint32_t(p.M) * kXRowBytes)
+               "r"(weight_bytes<ZM>(u.c.tc) + xb)
                : "memory");
   const int r0 = u.c.t0 * kTile;
   for (int r = 0; r < u.c.tc; ++r) tma_3d(st + r * kTileBytes, &L.tq, 0, r0 + r * kTile, u.gbase, bar);
@@ -388,6 +424,35 @@ __device__ __forceinline__ void issue_weights(const ChainParams& p, const Cursor
 
 __device__ __forceinline__ void issue_x(const ChainParams& p, const Cursor& u, uint32_t st, uint32_t bar) {
   tma_3d(st + kXOff, &p.layer[u.l].tx, 0, u.gbase, 0, bar);
+}
+
+// ---------------------------------------------------------------------------
+// consumer: x of a layer that reads an earlier layer's output (this warp's
+// group of the stage, 4 values per lane of each batch row, from the exchange
+// copy [M][K] of the source layer, K = this layer's input width)
+// ---------------------------------------------------------------------------
+template <int MB>
+__device__ __forceinline__ void load_x(uint2 (&px)[MB], const LayerRun* runs, const char* xch, int l, int gbase,
+                                       int w, int lane, int M) {
+  const size_t K = size_t(runs[l].G) * kGroup;
+  const char* a = xch + runs[run_x_from(runs[l])].ll_off + (size_t(gbase + w) * kGroup + 4 * lane) * 2;
+#pragma unroll
+  for (int m = 0; m < MB; ++m)
+    if (m < M) px[m] = ll_get2(a + size_t(m) * K * 2);
+}
+
+template <int MB>
+__device__ __forceinline__ bool x_complete(const uint2 (&px)[MB], int M) {
+  bool got = true;
+#pragma unroll
+  for (int m = 0; m < MB; ++m)
+    if (m < M) got = got && ll_complete(px[m]);
+  return __all_sync(0xffffffffu, got);
+}
+
+// Whether this warp needs exchange x for the stage of layer l starting at group gbase.
+__device__ __forceinline__ bool x_needed(const ChainParams& p, const LayerRun* runs, int l, int gbase, int w) {
+  return l < p.n_layers && run_x_from(runs[l]) >= 0 && gbase + w < runs[l].ge;
 }
 
 // ---------------------------------------------------------------------------
@@ -485,8 +550,6 @@ chain_kernel(const __grid_constant__ ChainParams p) {
   const uint32_t full0 = sbase;                        // [S] mbarriers
   const uint32_t empty0 = sbase + kMaxStages * 8;      // [S] mbarriers
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kFlagsOff);
-  // layers the consumers have finished (written by consumer thread 0, read by the release warp)
-  const uint32_t layers_done = sbase + kFlagsOff + 4;
   LayerRun* runs = reinterpret_cast<LayerRun*>(smem + kTableOff);
   const uint32_t ring = sbase + header_bytes(p.n_layers);
   const int S = p.stages;
@@ -494,6 +557,7 @@ chain_kernel(const __grid_constant__ ChainParams p) {
   const int lane = int(threadIdx.x) & 31;
   const unsigned long long limit = g_awq_chain_wait_limit_ns;
   const uint32_t hint = limit < 20000ull ? uint32_t(limit) : 20000u;   // sleep of one wait step, ns
+  uint32_t* const ctl = reinterpret_cast<uint32_t*>(p.ws);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -501,95 +565,59 @@ chain_kernel(const __grid_constant__ ChainParams p) {
       asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(empty0 + 8 * s), "r"(kCW));
     }
     *abort_flag = 0;
-    asm volatile("st.shared.u32 [%0], 0;" ::"r"(layers_done) : "memory");
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     fence_proxy_async_smem();
   }
   for (int l = int(threadIdx.x); l < p.n_layers; l += int(blockDim.x)) fill_run(p.layer[l], runs[l]);
   __syncthreads();
+  for (int l = int(threadIdx.x); l < p.n_layers; l += int(blockDim.x)) {
+    int n = l + 1;
+    while (n < p.n_layers && runs[n].i0 >= runs[n].i1) ++n;
+    runs[l].next = n;
+  }
+  __syncthreads();
 
-  if (warp == kProducerWarp) {
+  if (warp == kCW) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      Cursor cw, cx;
+      Cursor cw;
       cursor_init(p, runs, cw);
-      cx = cw;
-      int sw = 0, sx = 0;           // stages whose weights / x have been issued
-      uint32_t ready = 0;           // layers whose x may be read
-      for (int l = 0; l < p.n_layers; ++l)
-        if (p.layer[l].x_from < 0) ready |= 1u << l;
+      Cursor cx = cw;               // stages whose weights were issued before the wait
+      int sw = 0;                   // stages issued
       if (p.early) {
         for (; sw < S && !cw.done(p.n_layers); ++sw) {
-          issue_weights<ZM>(p, cw, ring + sw * p.stage_bytes, full0 + 8 * sw);
+          issue_weights<ZM>(p, runs, cw, ring + sw * p.stage_bytes, full0 + 8 * sw);
           cursor_next(p, runs, cw);
         }
       }
       asm volatile("griddepcontrol.wait;" ::: "memory");
-      const uint32_t target = gridDim.x;
-      // Starts of the two waits the producer can be in (0: not waiting): for
-      // the layer that the next x copy comes from, and for a free slot. A
-      // wait longer than the limit gives up.
-      uint64_t t_x = 0, t_slot = 0;
-      bool gave_up = false;
-      while (!cx.done(p.n_layers)) {
-        bool progress = false, slot_busy = false, x_blocked = false;
-        if (!cw.done(p.n_layers)) {
-          const int slot = sw % S;
-          if (sw < S || mbar_test_wait(empty0 + 8 * slot, uint32_t((sw / S) + 1) & 1u)) {
-            issue_weights<ZM>(p, cw, ring + slot * p.stage_bytes, full0 + 8 * slot);
-            cursor_next(p, runs, cw);
-            ++sw;
-            progress = true;
-          } else {
-            slot_busy = true;
-          }
+      // x of those stages (layers whose x is an input of the call)
+      for (int j = 0; j < sw; ++j) {
+        if (run_x_from(runs[cx.l]) < 0) issue_x(p, cx, ring + j * p.stage_bytes, full0 + 8 * j);
+        cursor_next(p, runs, cx);
+      }
+      uint64_t t_slot = 0;          // start of the wait for a free slot (0: not waiting)
+      while (!cw.done(p.n_layers)) {
+        const int slot = sw % S;
+        if (sw < S || mbar_test_wait(empty0 + 8 * slot, uint32_t((sw / S) + 1) & 1u)) {
+          const uint32_t st = ring + slot * p.stage_bytes;
+          issue_weights<ZM>(p, runs, cw, st, full0 + 8 * slot);
+          if (run_x_from(runs[cw.l]) < 0) issue_x(p, cw, st, full0 + 8 * slot);
+          cursor_next(p, runs, cw);
+          ++sw;
+          t_slot = 0;
+          continue;
         }
-        if (sx < sw) {
-          const int l = cx.l;
-          if (!((ready >> l) & 1u)) {
-            if (ld_acquire_gpu(p.done + run_x_from(runs[l])) >= target) {
-              asm volatile("fence.proxy.async.global;" ::: "memory");
-              ready |= 1u << l;
-            }
-          }
-          if ((ready >> l) & 1u) {
-            const int slot = sx % S;
-            issue_x(p, cx, ring + slot * p.stage_bytes, full0 + 8 * slot);
-            cursor_next(p, runs, cx);
-            ++sx;
-            progress = true;
-          } else {
-            x_blocked = true;
-          }
-        }
-        if (!progress && sx == sw && slot_busy) {
-          // nothing to do until the next slot frees: sleep on its barrier
-          const int slot = sw % S;
-          mbar_sleep_wait(empty0 + 8 * slot, uint32_t((sw / S) + 1) & 1u, hint);
-        }
-        if (*abort_flag) {
-          gave_up = true;
-          break;
-        }
+        // nothing to do until the slot frees: sleep on its barrier
+        mbar_sleep_wait(empty0 + 8 * slot, uint32_t((sw / S) + 1) & 1u, hint);
+        if (*abort_flag) break;
         const uint64_t now = now_ns();
-        if (!x_blocked) t_x = 0;
-        else if (t_x == 0) t_x = now;
-        if (!slot_busy) t_slot = 0;
-        else if (t_slot == 0) t_slot = now;
-        if ((t_x && now - t_x > limit) || (t_slot && now - t_slot > limit)) {
+        if (t_slot == 0) {
+          t_slot = now;
+        } else if (now - t_slot > limit) {
           *abort_flag = 1;
           atomicOr(&g_awq_chain_error, kErrBit);
-          gave_up = true;
           break;
-        }
-      }
-      if (gave_up) {
-        // every armed stage still missing its x gets it (from wherever x
-        // points now) so that every armed phase completes
-        for (; sx < sw; ++sx) {
-          const int slot = sx % S;
-          issue_x(p, cx, ring + slot * p.stage_bytes, full0 + 8 * slot);
-          cursor_next(p, runs, cx);
         }
       }
       // every copy issued must land before the CTA exits: the last phase
@@ -604,38 +632,6 @@ chain_kernel(const __grid_constant__ ChainParams p) {
       }
     }
     __syncwarp();
-  } else if (warp == kReleaseWarp) {
-    // ------------------------------------------------------------ release
-    // Publishes each layer once the consumers have finished it: their
-    // stores are ordered before consumer thread 0's release of the count
-    // (named barrier), this thread acquires the count, and its gpu-scope
-    // release of the layer's done counter covers them.
-    if (lane == 0) {
-      // the previous launch's last CTA resets the counters: wait for it
-      asm volatile("griddepcontrol.wait;" ::: "memory");
-      uint64_t t0 = 0;
-      for (int l = 0; l < p.n_layers;) {
-        uint32_t n;
-        asm volatile("ld.acquire.cta.shared.u32 %0, [%1];" : "=r"(n) : "r"(layers_done) : "memory");
-        if (n > uint32_t(l)) {
-          for (; l < int(n); ++l) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(p.done + l) : "memory");
-          t0 = 0;
-          continue;
-        }
-        const uint64_t now = now_ns();
-        if (t0 == 0) {
-          t0 = now;
-        } else if (now - t0 > kWaitLimitNs) {
-          // the consumers count every layer even after giving up, so this
-          // is reached only if they stopped: let the others give up too
-          *abort_flag = 1;
-          atomicOr(&g_awq_chain_error, kErrBit);
-          break;
-        }
-        __nanosleep(64);
-      }
-    }
-    __syncwarp();
   } else {
     // ------------------------------------------------------------ consumers
     asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -644,15 +640,36 @@ chain_kernel(const __grid_constant__ ChainParams p) {
     const int t = lane & 3;
     const int M = p.M;
     const uint32_t pbuf = sbase + p.pbuf_offset;       // [warp][64 rows][M] fp32
+    // The exchange half of this launch, and this CTA's share of the other
+    // half to zero for the next launch (the previous launch, which used it,
+    // has completed: griddepcontrol.wait above).
+    const uint32_t parity = ctl[kEpochWord] & 1u;
+    char* const xch = p.ws + p.ll_base + size_t(parity) * p.ll_half;
+    {
+      uint4* o = reinterpret_cast<uint4*>(p.ws + p.ll_base + size_t(parity ^ 1u) * p.ll_half);
+      const uint32_t n16 = p.ll_half / 16;
+      const uint32_t per = (n16 + gridDim.x - 1) / gridDim.x;
+      const uint32_t b = blockIdx.x * per;
+      const uint32_t e = b + per < n16 ? b + per : n16;
+      for (uint32_t k = b + threadIdx.x; k < e; k += kCW * 32) o[k] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    // x of a stage that reads an earlier layer's output: this warp's group,
+    // 4 values per lane of each batch row, loaded one stage ahead
+    uint2 px[MB];
+    {
+      // the first stage's x
+      int l0 = 0;
+      while (l0 < p.n_layers && runs[l0].i0 >= runs[l0].i1) ++l0;
+      if (x_needed(p, runs, l0, runs[l0 < p.n_layers ? l0 : 0].gb, w))
+        load_x<MB>(px, runs, xch, l0, runs[l0].gb, w, lane, M);
+    }
     int slot = 0;
     uint32_t phase = 0;
     bool live = true;
     for (int l = 0; l < p.n_layers; ++l) {
       const LayerRun& R = runs[l];
       const int i1 = R.i1;
-      const int ks = run_ks(R), tpu = run_tpu(R), silu = run_silu(R), N = R.N;
-      const int T = R.units * tpu;
-      uint16_t* const y = R.y;
+      const bool dep = run_x_from(R) >= 0;
       for (int i = R.i0; i < i1;) {
         Chunk cc;
         load_chunk(R, i, cc);
@@ -664,7 +681,9 @@ chain_kernel(const __grid_constant__ ChainParams p) {
 #pragma unroll
             for (int k = 0; k < 4; ++k) acc[rt][mt][k] = 0.0f;
         for (int gbase = cc.gb; gbase < cc.ge; gbase += kCW) {
+          const uint32_t st = ring + slot * p.stage_bytes;
           const uint32_t full = full0 + 8 * slot;
+          const bool mine = gbase + w < cc.ge;
           if (live) {
             bool ok = mbar_sleep_wait(full, phase, hint);
             if (!ok) {
@@ -682,10 +701,47 @@ chain_kernel(const __grid_constant__ ChainParams p) {
               }
             }
             live = __all_sync(0xffffffffu, ok);
+            if (live && dep && mine) {
+              // the layer's x: every value written by this launch, else
+              // reload until it is (bounded; the decisions are warp-uniform)
+              if (!x_complete<MB>(px, M)) {
+                const uint64_t t0 = now_ns();
+                for (;;) {
+                  load_x<MB>(px, runs, xch, l, gbase, w, lane, M);
+                  if (x_complete<MB>(px, M)) break;
+                  const bool late = now_ns() - t0 > limit;
+                  if (__any_sync(0xffffffffu, late || *abort_flag != 0)) {
+                    if (lane == 0 && late) {
+                      *abort_flag = 1;
+                      atomicOr(&g_awq_chain_error, kErrBit);
+                    }
+                    live = false;
+                    break;
+                  }
+                }
+              }
+              if (live) {
+#pragma unroll
+                for (int m = 0; m < MB; ++m)
+                  if (m < M) sts64(st + kXOff + uint32_t(m) * kXRowBytes + w * 256 + lane * 8, ll_decode(px[m]));
+                __syncwarp();
+              }
+            }
           }
           if (live) {
-            if (gbase + w < cc.ge)
-              stage_compute<MB, ZM>(ring + slot * p.stage_bytes, w, g, t, cc.tc, M, (cc.t0 & 1) * 8, acc);
+            // the next stage's x: the next groups of this chunk, the next
+            // chunk of this layer (same slice, so the same first group), or
+            // the first stage of the next layer with items
+            int nl = l, ng = gbase + kCW;
+            if (ng >= cc.ge) {
+              ng = cc.gb;
+              if (i + cc.nu >= i1) {
+                nl = R.next;
+                ng = nl < p.n_layers ? runs[nl].gb : 0;
+              }
+            }
+            if (x_needed(p, runs, nl, ng, w)) load_x<MB>(px, runs, xch, nl, ng, w, lane, M);
+            if (mine) stage_compute<MB, ZM>(st, w, g, t, cc.tc, M, (cc.t0 & 1) * 8, acc);
             __syncwarp();
             if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(empty0 + 8 * slot) : "memory");
           }
@@ -716,6 +772,16 @@ chain_kernel(const __grid_constant__ ChainParams p) {
           }
         }
         consumer_sync();
+        // the layer's fields, read here (from the table) rather than kept in
+        // registers through the stage loop
+        const int ks = run_ks(R), tpu = run_tpu(R), silu = run_silu(R), N = R.N;
+        const int T = R.units * tpu;
+        const bool src = run_source(R) != 0;
+        const int W = silu ? N / 2 : N;        // output columns
+        uint16_t* const y = R.y;
+        char* const xout = xch + R.ll_off;
+        float* const partials = reinterpret_cast<float*>(p.ws + R.partial_off);
+        uint32_t* const counters = reinterpret_cast<uint32_t*>(p.ws + R.counter_off);
         const int64_t row0 = int64_t(cc.t0) * kTile;
         const int tid = int(threadIdx.x);
         if (!silu || ks > 1) {
@@ -727,9 +793,13 @@ chain_kernel(const __grid_constant__ ChainParams p) {
             const int row = v / M;
             const int m = v - row * M;
             if (ks == 1) {
-              if (row0 + row < N) y[int64_t(m) * N + row0 + row] = __half_as_ushort(__float2half_rn(sum));
+              if (row0 + row < N) {
+                const uint16_t h = __half_as_ushort(__float2half_rn(sum));
+                y[int64_t(m) * N + row0 + row] = h;
+                if (src) ll_put(xout, int64_t(m) * W + row0 + row, h);
+              }
             } else {
-              __stcg(R.partials + ((int64_t(cc.s) * T * kTile + row0 + row) * M + m), sum);
+              __stcg(partials + ((int64_t(cc.s) * T * kTile + row0 + row) * M + m), sum);
             }
           }
         } else {
@@ -747,8 +817,9 @@ chain_kernel(const __grid_constant__ ChainParams p) {
             }
             const int row = rem / M;
             const int m = rem - row * M;
-            y[int64_t(m) * (N / 2) + row0 / 2 + q * kTile + row] =
-                __half_as_ushort(__float2half_rn(silu_f32(gs) * us));
+            const uint16_t h = __half_as_ushort(__float2half_rn(silu_f32(gs) * us));
+            y[int64_t(m) * W + row0 / 2 + q * kTile + row] = h;
+            if (src) ll_put(xout, int64_t(m) * W + row0 / 2 + q * kTile + row, h);
           }
         }
         if (ks > 1) {
@@ -763,7 +834,7 @@ chain_kernel(const __grid_constant__ ChainParams p) {
             if (lane == 0) {
               uint32_t old;
               asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
-                           : "=r"(old) : "l"(R.counters + unit) : "memory");
+                           : "=r"(old) : "l"(counters + unit) : "memory");
               last = (old + 1 == uint32_t(ks)) ? 1u : 0u;
             }
             last = __shfl_sync(0xffffffffu, last, 0);
@@ -773,45 +844,48 @@ chain_kernel(const __grid_constant__ ChainParams p) {
               if (tpu == 1) {
                 for (int v = lane; v < kTile * M; v += 32) {
                   float sum = 0.0f;
-                  for (int s = 0; s < ks; ++s) sum += __ldcg(R.partials + ((int64_t(s) * T * kTile + trow) * M + v));
+                  for (int s = 0; s < ks; ++s) sum += __ldcg(partials + ((int64_t(s) * T * kTile + trow) * M + v));
                   const int row = v / M;
                   const int m = v - row * M;
-                  if (trow + row < N) y[int64_t(m) * N + trow + row] = __half_as_ushort(__float2half_rn(sum));
+                  if (trow + row < N) {
+                    const uint16_t h = __half_as_ushort(__float2half_rn(sum));
+                    y[int64_t(m) * N + trow + row] = h;
+                    if (src) ll_put(xout, int64_t(m) * W + trow + row, h);
+                  }
                 }
               } else {
                 for (int v = lane; v < kTile * M; v += 32) {
                   float gs = 0.0f, us = 0.0f;
                   for (int s = 0; s < ks; ++s) {
-                    const float* ps = R.partials + (int64_t(s) * T * kTile + trow) * M;
+                    const float* ps = partials + (int64_t(s) * T * kTile + trow) * M;
                     gs += __ldcg(ps + v);
                     us += __ldcg(ps + kTile * M + v);
                   }
                   const int row = v / M;
                   const int m = v - row * M;
-                  y[int64_t(m) * (N / 2) + trow / 2 + row] = __half_as_ushort(__float2half_rn(silu_f32(gs) * us));
+                  const uint16_t h = __half_as_ushort(__float2half_rn(silu_f32(gs) * us));
+                  y[int64_t(m) * W + trow / 2 + row] = h;
+                  if (src) ll_put(xout, int64_t(m) * W + trow / 2 + row, h);
                 }
               }
-              if (lane == 0) R.counters[unit] = 0u;
+              if (lane == 0) counters[unit] = 0u;
             }
           }
         }
-        consumer_sync();   // pbuf is reused by the next chunk; the layer's stores are done
+        consumer_sync();   // pbuf is reused by the next chunk
         i += cc.nu;
       }
-      // This CTA is done with layer l (the chunk's last barrier ordered every
-      // consumer's stores before this point): the release warp publishes it.
-      if (threadIdx.x == 0) asm volatile("st.release.cta.shared.u32 [%0], %1;" ::"r"(layers_done), "r"(l + 1) : "memory");
     }
   }
   __syncthreads();
-  // The last CTA out resets the per-layer counters for the next call.
+  // The last CTA out resets the exit counter and counts the launch (the
+  // parity of the count picks the exchange half of the next launch).
   if (threadIdx.x == 0) {
     uint32_t old;
-    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
-                 : "=r"(old) : "l"(p.done + kMaxLayers) : "memory");
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(ctl + kExitWord) : "memory");
     if (old + 1 == gridDim.x) {
-      for (int l = 0; l < p.n_layers; ++l) p.done[l] = 0u;
-      p.done[kMaxLayers] = 0u;
+      ctl[kExitWord] = 0u;
+      ctl[kEpochWord] += 1u;
     }
   }
 }
@@ -842,12 +916,15 @@ std::atomic<int> g_attr_set[kMaxDevices][kNumVariants];
 struct LayerPlan {
   int T, tpu, units, ks, items, rot;
   size_t counter_off, partial_off;   // workspace offsets (ks > 1)
+  int source;                        // a later layer reads this layer's output
+  size_t ll_off;                     // its exchange copy, within each half
 };
 
 struct ChainPlan {
   ChainFn fn;
   int id, grid, stages, stage_bytes, pbuf_offset, smem;
   LayerPlan lp[kMaxLayers];
+  size_t ll_base, ll_half;           // the exchange region: two halves
   size_t ws_bytes;
 };
 
@@ -985,7 +1062,7 @@ awq_status_t make_chain_plan(const awq_gemv_layer_t* layers, int n, int64_t M, C
   pl.grid = per_sm * sms;
   // Per layer: whole tiles per CTA over all of K, K slices only when a
   // layer has fewer units than CTAs (as a one-layer launch would).
-  size_t off = align256(size_t(kMaxLayers + 1) * 4);   // per-layer done counters + the exit counter
+  size_t off = kControlBytes;   // exit counter, launch count
   int level_start = 0;
   int64_t extra = 0;
   for (int l = 0; l < n; ++l) {
@@ -1015,8 +1092,26 @@ awq_status_t make_chain_plan(const awq_gemv_layer_t* layers, int n, int64_t M, C
     } else {
       lp.counter_off = lp.partial_off = 0;
     }
+    lp.source = 0;
+    lp.ll_off = 0;
   }
+  // The exchange region: a copy of the output of every layer that a later
+  // layer reads, in each of two halves.
+  size_t half = 0;
+  for (int l = 0; l < n; ++l)
+    if (layers[l].x_from >= 0) pl.lp[layers[l].x_from].source = 1;
+  for (int l = 0; l < n; ++l) {
+    if (!pl.lp[l].source) continue;
+    const int64_t W = (layers[l].cfg.flags & AWQ_FLAG_SILU_MUL) ? layers[l].N / 2 : layers[l].N;
+    pl.lp[l].ll_off = half;
+    half += align256(size_t(M) * size_t(W) * 2);
+  }
+  pl.ll_base = off;
+  pl.ll_half = half;
+  off += 2 * half;
   pl.ws_bytes = off;
+  // offsets travel to the kernel as 32-bit values
+  if (pl.ws_bytes > size_t(0xFFFFFFFFu)) return AWQ_ERR_SHAPE;
   return AWQ_OK;
 }
 
@@ -1085,8 +1180,10 @@ extern "C" awq_status_t awq_gemv_chain(const awq_gemv_layer_t* layers, int n_lay
       D.tz = D.ts;   // never read
     }
     D.y = A.y;
-    D.partials = lp.ks > 1 ? reinterpret_cast<float*>(ws + lp.partial_off) : nullptr;
-    D.counters = lp.ks > 1 ? reinterpret_cast<uint32_t*>(ws + lp.counter_off) : nullptr;
+    D.partial_off = uint32_t(lp.partial_off);
+    D.counter_off = uint32_t(lp.counter_off);
+    D.ll_off = uint32_t(lp.ll_off);
+    D.source = lp.source;
     D.N = int(A.N);
     D.G = int(G);
     D.T = lp.T;
@@ -1099,7 +1196,9 @@ extern "C" awq_status_t awq_gemv_chain(const awq_gemv_layer_t* layers, int n_lay
     D.silu = (A.cfg.flags & AWQ_FLAG_SILU_MUL) ? 1 : 0;
     early = early && (A.cfg.flags & AWQ_FLAG_WEIGHTS_STATIC);
   }
-  p.done = reinterpret_cast<uint32_t*>(ws);
+  p.ws = ws;
+  p.ll_base = uint32_t(pl.ll_base);
+  p.ll_half = uint32_t(pl.ll_half);
   p.n_layers = n_layers;
   p.M = int(M);
   p.stages = pl.stages;
