@@ -110,8 +110,7 @@ struct alignas(64) LayerDesc {
   CUtensorMap ts;      // scales: {N, G}, box {64, kCW}
   CUtensorMap tz;      // zeros: {N, G} box {64, kCW}, or packed {N/8 words, G} box {12, kCW}
   uint16_t* y;
-  uint32_t partial_off;  // workspace offset of the partials [ks][T * 16][M] (ks > 1)
-  uint32_t counter_off;  // workspace offset of the arrival counters [units] (ks > 1)
+  uint32_t partial_off;  // workspace offset of the tagged partials [ks - 1][T * 16][M] (ks > 1)
   uint32_t ll_off;       // offset of the exchange copy [M][N or N/2] in each half (source layers)
   int source;            // a later layer reads this layer's output
   int N, G, T;
@@ -135,8 +134,9 @@ struct LayerRun {
   int G;
   int info;            // tpu (bits 0-1), silu (bit 2), source (bit 3), ks (bits 8-15), x_from + 1 (bits 16-23)
   uint16_t* y;
-  uint32_t partial_off, counter_off, ll_off;
+  uint32_t partial_off, ll_off;
   int next;            // the next layer with items for this CTA (n_layers: none)
+  int pad;
 };
 static_assert(sizeof(LayerRun) == 56, "layer table entry");
 static_assert(kTableOff + kMaxLayers * sizeof(LayerRun) <= kMaxHeader, "layer table overflows the header");
@@ -159,7 +159,7 @@ constexpr int kControlBytes = 256;
 
 struct ChainParams {
   LayerDesc layer[kMaxLayers];
-  char* ws;            // workspace: control words, split-K partials and counters, the exchange region
+  char* ws;            // workspace: control words, split-K partials, the exchange region
   uint32_t ll_base;    // offset of the exchange region (two halves of ll_half bytes)
   uint32_t ll_half;
   int n_layers, M, stages, stage_bytes, pbuf_offset, early;
@@ -267,6 +267,58 @@ __device__ __forceinline__ bool ll_complete(uint2 v) { return (__vcmpeq2(v.x, 0u
 __device__ __forceinline__ uint2 ll_decode(uint2 v) {
   return make_uint2(__vsub2(v.x, 0x00010001u), __vsub2(v.y, 0x00010001u));
 }
+// Partial sums of the K slices of a unit: 64-bit relaxed stores of (a tag,
+// the float's bits), the tag being the launch count plus one (a zero-filled
+// workspace holds tag 0), so that a reader sees a value of this launch whole
+// or not at all, with no fence between store and use.
+__device__ __forceinline__ void put_tagged(unsigned long long* a, uint32_t tag, float v) {
+  const unsigned long long x = (static_cast<unsigned long long>(tag) << 32) | __float_as_uint(v);
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(a), "l"(x) : "memory");
+}
+__device__ __forceinline__ unsigned long long get_tagged(const unsigned long long* a) {
+  unsigned long long x;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(x) : "l"(a) : "memory");
+  return x;
+}
+
+// The sum over the K slices of one value of a unit: the tagged partials of
+// slices 0 .. ks-2 (stride ss apart), each waited for (bounded) until it
+// carries this launch's tag, in slice order, then the caller's own sum (the
+// last slice). Loads are issued four at a time. Kept out of line: it runs
+// once per value at the end of a chunk, and inlined it would take registers
+// from the stage loop.
+__device__ __noinline__ float slice_sum(const unsigned long long* partials, int64_t ss, int ks, int64_t idx,
+                                        uint32_t tag, float own, volatile int* abort_flag,
+                                        unsigned long long limit) {
+  float sum = 0.0f;
+  for (int s0 = 0; s0 < ks - 1; s0 += 4) {
+    unsigned long long x[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (s0 + j < ks - 1) x[j] = get_tagged(partials + (int64_t(s0 + j) * ss + idx));
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (s0 + j < ks - 1) {
+        if (uint32_t(x[j] >> 32) != tag) {
+          const unsigned long long* a = partials + (int64_t(s0 + j) * ss + idx);
+          const uint64_t t0 = now_ns();
+          for (;;) {
+            x[j] = get_tagged(a);
+            if (uint32_t(x[j] >> 32) == tag || *abort_flag) break;
+            if (now_ns() - t0 > limit) {
+              *abort_flag = 1;
+              atomicOr(&g_awq_chain_error, kErrBit);
+              break;
+            }
+          }
+        }
+        sum += __uint_as_float(uint32_t(x[j]));
+      }
+    }
+  }
+  return sum + own;
+}
+
 __device__ __forceinline__ void sts64(uint32_t a, uint2 v) {
   asm volatile("st.shared.v2.u32 [%0], {%1,%2};" ::"r"(a), "r"(v.x), "r"(v.y) : "memory");
 }
@@ -337,7 +389,6 @@ __device__ __forceinline__ void fill_run(const LayerDesc& L, LayerRun& r) {
   r.info = L.tpu | (L.silu << 2) | (L.source << 3) | (L.ks << 8) | ((L.x_from + 1) << 16);
   r.y = L.y;
   r.partial_off = L.partial_off;
-  r.counter_off = L.counter_off;
   r.ll_off = L.ll_off;
 }
 
@@ -643,7 +694,9 @@ chain_kernel(const __grid_constant__ ChainParams p) {
     // The exchange half of this launch, and this CTA's share of the other
     // half to zero for the next launch (the previous launch, which used it,
     // has completed: griddepcontrol.wait above).
-    const uint32_t parity = ctl[kEpochWord] & 1u;
+    const uint32_t epoch = ctl[kEpochWord];
+    const uint32_t parity = epoch & 1u;
+    const uint32_t tag = epoch + 1u;    // of this launch's partials (a zero-filled workspace holds tag 0)
     char* const xch = p.ws + p.ll_base + size_t(parity) * p.ll_half;
     {
       uint4* o = reinterpret_cast<uint4*>(p.ws + p.ll_base + size_t(parity ^ 1u) * p.ll_half);
@@ -780,11 +833,23 @@ chain_kernel(const __grid_constant__ ChainParams p) {
         const int W = silu ? N / 2 : N;        // output columns
         uint16_t* const y = R.y;
         char* const xout = xch + R.ll_off;
-        float* const partials = reinterpret_cast<float*>(p.ws + R.partial_off);
-        uint32_t* const counters = reinterpret_cast<uint32_t*>(p.ws + R.counter_off);
+        unsigned long long* const partials = reinterpret_cast<unsigned long long*>(p.ws + R.partial_off);
         const int64_t row0 = int64_t(cc.t0) * kTile;
         const int tid = int(threadIdx.x);
-        if (!silu || ks > 1) {
+        // With K slices, every slice but the last stores its sums tagged
+        // with the launch count; the CTA of the last slice waits for each
+        // to carry this launch's tag and adds them in slice order, its own
+        // sum last (the order of a sum over the slices from 0).
+        const bool reducer = ks > 1 && cc.s == ks - 1;
+        if (ks > 1 && !reducer) {
+          const int V = kTile * cc.tc * M;
+          for (int v = tid; v < V; v += kCW * 32) {
+            float own = 0.0f;
+#pragma unroll
+            for (int ww = 0; ww < kCW; ++ww) own += lds_f32(pbuf + uint32_t(ww * 64 * M + v) * 4);
+            put_tagged(partials + ((int64_t(cc.s) * T * kTile + row0) * M + v), tag, own);
+          }
+        } else if (!silu) {
           const int V = kTile * cc.tc * M;
           for (int v = tid; v < V; v += kCW * 32) {
             float sum = 0.0f;
@@ -792,14 +857,11 @@ chain_kernel(const __grid_constant__ ChainParams p) {
             for (int ww = 0; ww < kCW; ++ww) sum += lds_f32(pbuf + uint32_t(ww * 64 * M + v) * 4);
             const int row = v / M;
             const int m = v - row * M;
-            if (ks == 1) {
-              if (row0 + row < N) {
-                const uint16_t h = __half_as_ushort(__float2half_rn(sum));
-                y[int64_t(m) * N + row0 + row] = h;
-                if (src) ll_put(xout, int64_t(m) * W + row0 + row, h);
-              }
-            } else {
-              __stcg(partials + ((int64_t(cc.s) * T * kTile + row0 + row) * M + m), sum);
+            if (reducer) sum = slice_sum(partials, int64_t(T) * kTile * M, ks, (row0 + row) * M + m, tag, sum, abort_flag, limit);
+            if (row0 + row < N) {
+              const uint16_t h = __half_as_ushort(__float2half_rn(sum));
+              y[int64_t(m) * N + row0 + row] = h;
+              if (src) ll_put(xout, int64_t(m) * W + row0 + row, h);
             }
           }
         } else {
@@ -815,61 +877,16 @@ chain_kernel(const __grid_constant__ ChainParams p) {
               gs += lds_f32(pbuf + uint32_t(ww * 64 * M + vg) * 4);
               us += lds_f32(pbuf + uint32_t(ww * 64 * M + vg + kTile * M) * 4);
             }
+            if (reducer) {
+              const int64_t ss = int64_t(T) * kTile * M;
+              gs = slice_sum(partials, ss, ks, (row0 + 2 * q * kTile) * M + rem, tag, gs, abort_flag, limit);
+              us = slice_sum(partials, ss, ks, (row0 + (2 * q + 1) * kTile) * M + rem, tag, us, abort_flag, limit);
+            }
             const int row = rem / M;
             const int m = rem - row * M;
             const uint16_t h = __half_as_ushort(__float2half_rn(silu_f32(gs) * us));
             y[int64_t(m) * W + row0 / 2 + q * kTile + row] = h;
             if (src) ll_put(xout, int64_t(m) * W + row0 / 2 + q * kTile + row, h);
-          }
-        }
-        if (ks > 1) {
-          // slices of a unit meet in the workspace: the CTA whose arrival
-          // brings a unit's count to ks sums the ks partials in slice order.
-          // The barrier orders every consumer's partial stores before the
-          // arrivals, whose release makes them visible at GPU scope.
-          consumer_sync();
-          if (w < cc.nu) {
-            const int unit = cc.t0 / tpu + w;
-            uint32_t last = 0;
-            if (lane == 0) {
-              uint32_t old;
-              asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
-                           : "=r"(old) : "l"(counters + unit) : "memory");
-              last = (old + 1 == uint32_t(ks)) ? 1u : 0u;
-            }
-            last = __shfl_sync(0xffffffffu, last, 0);
-            __syncwarp();   // lane 0's acquire orders the warp's partial reads
-            if (last) {
-              const int64_t trow = int64_t(unit) * tpu * kTile;
-              if (tpu == 1) {
-                for (int v = lane; v < kTile * M; v += 32) {
-                  float sum = 0.0f;
-                  for (int s = 0; s < ks; ++s) sum += __ldcg(partials + ((int64_t(s) * T * kTile + trow) * M + v));
-                  const int row = v / M;
-                  const int m = v - row * M;
-                  if (trow + row < N) {
-                    const uint16_t h = __half_as_ushort(__float2half_rn(sum));
-                    y[int64_t(m) * N + trow + row] = h;
-                    if (src) ll_put(xout, int64_t(m) * W + trow + row, h);
-                  }
-                }
-              } else {
-                for (int v = lane; v < kTile * M; v += 32) {
-                  float gs = 0.0f, us = 0.0f;
-                  for (int s = 0; s < ks; ++s) {
-                    const float* ps = partials + (int64_t(s) * T * kTile + trow) * M;
-                    gs += __ldcg(ps + v);
-                    us += __ldcg(ps + kTile * M + v);
-                  }
-                  const int row = v / M;
-                  const int m = v - row * M;
-                  const uint16_t h = __half_as_ushort(__float2half_rn(silu_f32(gs) * us));
-                  y[int64_t(m) * W + trow / 2 + row] = h;
-                  if (src) ll_put(xout, int64_t(m) * W + trow / 2 + row, h);
-                }
-              }
-              if (lane == 0) counters[unit] = 0u;
-            }
           }
         }
         consumer_sync();   // pbuf is reused by the next chunk
@@ -915,7 +932,7 @@ std::atomic<int> g_attr_set[kMaxDevices][kNumVariants];
 
 struct LayerPlan {
   int T, tpu, units, ks, items, rot;
-  size_t counter_off, partial_off;   // workspace offsets (ks > 1)
+  size_t partial_off;                // workspace offset (ks > 1)
   int source;                        // a later layer reads this layer's output
   size_t ll_off;                     // its exchange copy, within each half
 };
@@ -1085,12 +1102,10 @@ awq_status_t make_chain_plan(const awq_gemv_layer_t* layers, int n, int64_t M, C
     lp.rot = int(extra % pl.grid);
     if (lp.ks == 1) extra += lp.units % pl.grid;
     if (lp.ks > 1) {
-      lp.counter_off = off;
-      off += align256(size_t(lp.units) * 4);
       lp.partial_off = off;
-      off += align256(size_t(lp.ks) * size_t(lp.T) * kTile * size_t(M) * 4);
+      off += align256(size_t(lp.ks - 1) * size_t(lp.T) * kTile * size_t(M) * 8);
     } else {
-      lp.counter_off = lp.partial_off = 0;
+      lp.partial_off = 0;
     }
     lp.source = 0;
     lp.ll_off = 0;
@@ -1181,7 +1196,6 @@ extern "C" awq_status_t awq_gemv_chain(const awq_gemv_layer_t* layers, int n_lay
     }
     D.y = A.y;
     D.partial_off = uint32_t(lp.partial_off);
-    D.counter_off = uint32_t(lp.counter_off);
     D.ll_off = uint32_t(lp.ll_off);
     D.source = lp.source;
     D.N = int(A.N);
