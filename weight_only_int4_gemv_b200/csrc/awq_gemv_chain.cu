@@ -977,10 +977,13 @@ awq_status_t check_layer(const awq_gemv_layer_t* L, int l, const awq_gemv_layer_
 // stage of kCW groups costs its tiles x groups, but never less than that of
 // three tiles (a stage of one or two tiles has too little independent work
 // to hide the latency of its decode-and-multiply chains), plus a fixed cost
-// per stage, per chunk (the reduction) and per chunk of a split layer
-// (partials and the arrival).
+// per stage (waits, barriers), per chunk (the reduction through shared
+// memory, the output stores) and per chunk of a split layer (the tagged
+// partials). The constants are fitted to B200 timings of the Llama-3-8B
+// decode step (4 slices for its 4096-row layers, none for the 14336-row
+// ones).
 int64_t split_cost(int units, int tpu, int G, int ks, int grid) {
-  constexpr int64_t kMinTiles = 3, kStageCost = 2, kChunkCost = 4, kSplitCost = 6;
+  constexpr int64_t kMinTiles = 3, kStageCost = 10, kChunkCost = 20, kSplitCost = 6;
   int64_t worst = 0;
   for (int b = 0; b < grid; ++b) {
     int i0, i1;
