@@ -127,9 +127,12 @@ COMMON_SRC = os.path.join(ROOT, "weight_only_int4_gemv_b200", "csrc", "awq_commo
 
 def source_sha(path: str) -> str:
     """First 16 hex digits of the SHA-256 of a kernel's .cu file followed by
-    the device helpers it includes, so a profile goes stale when either changes."""
+    the kernel body it includes (awq_gemm_body.cuh, for the GEMM) and the
+    device helpers, so a profile goes stale when any of them changes."""
     h = hashlib.sha256()
-    for p in (path, COMMON_SRC):
+    body = os.path.join(os.path.dirname(path), "awq_gemm_body.cuh")
+    parts = (path, body, COMMON_SRC) if path.endswith("awq_gemm.cu") else (path, COMMON_SRC)
+    for p in parts:
         with open(p, "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
