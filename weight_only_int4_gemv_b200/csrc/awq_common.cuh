@@ -72,8 +72,12 @@ __device__ __forceinline__ int group_quant_code(float w, float sf, float zf) {
   return int(fminf(fmaxf(rintf(__fdiv_rn(w, sf)), -8.0f), 7.0f)) + 8;
 }
 
-// SiLU in fp32 for the fused gate/up epilogues.
-__device__ __forceinline__ float silu_f32(float v) { return v / (1.0f + expf(-v)); }
+// SiLU in fp32 for the fused gate/up epilogues: v / (1 + e^-v) with the
+// fast exponential and division intrinsics (relative error a few fp32 ulp,
+// far below the fp16 rounding of the output; large negative v gives 0, NaN
+// stays NaN). The exact library forms cost tens of instructions and enough
+// registers to spill the GEMM's epilogue warps.
+__device__ __forceinline__ float silu_f32(float v) { return __fdividef(v, 1.0f + __expf(-v)); }
 
 // K must hold whole groups; N >= 0. Sizes are bounded so that every row
 // offset fits comfortably in 64 bits and every per-row count in 32 bits.

@@ -84,6 +84,15 @@ __device__ __forceinline__ void tc_mma_f16(uint32_t d_tmem, uint64_t a_desc, uin
       : "memory");
 }
 
+// 32 lanes x 8 consecutive fp32 columns
+__device__ __forceinline__ void tc_ld_32x32b_x8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
 // 32 lanes x 32 consecutive fp32 columns
 __device__ __forceinline__ void tc_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
@@ -131,6 +140,29 @@ __device__ __forceinline__ float4 sum_slices_dsmem(uint32_t saddr, int S) {
       acc.w += v[sl].w;
     }
   return acc;
+}
+
+// Two such sums at once (the gate and up values of the fused epilogue), in
+// the same slice order, two slices per step so that no more than eight
+// float4 loads are live (all slices of both at once would spill).
+__device__ __forceinline__ void sum_slices_dsmem2(uint32_t sa, uint32_t sb, int S, float4& a, float4& b) {
+  a = ld_dsmem_f4(sa, 0);
+  b = ld_dsmem_f4(sb, 0);
+#pragma unroll 1
+  for (int sl = 1; sl < S; sl += 2) {
+    const float4 a1 = ld_dsmem_f4(sa, sl), b1 = ld_dsmem_f4(sb, sl);
+    float4 a2 = make_float4(0.f, 0.f, 0.f, 0.f), b2 = a2;
+    if (sl + 1 < S) {
+      a2 = ld_dsmem_f4(sa, sl + 1);
+      b2 = ld_dsmem_f4(sb, sl + 1);
+    }
+    a.x += a1.x; a.y += a1.y; a.z += a1.z; a.w += a1.w;
+    b.x += b1.x; b.y += b1.y; b.z += b1.z; b.w += b1.w;
+    if (sl + 1 < S) {
+      a.x += a2.x; a.y += a2.y; a.z += a2.z; a.w += a2.w;
+      b.x += b2.x; b.y += b2.y; b.z += b2.z; b.w += b2.w;
+    }
+  }
 }
 
 // Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
@@ -318,39 +350,48 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         const int c = c8 % (BN / 32);       // which 32 output channels
         const int64_t m = int64_t(m0) + hm * BMH + q * 32 + lane;
         uint16_t* yrow = p.y + m * p.N;
-        uint32_t r[32];
-        tc_ld_32x32b_x32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * kAccCols + hm * BN + c * 32), r);
+        const uint32_t tcol = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * kAccCols + hm * BN + c * 32);
         const int nc = n0 + c * 32;
         if constexpr (SILU) {
-          // columns nc .. nc+15: gate rows, nc+16 .. nc+31: the matching up rows
-          if (m < p.M && nc < p.N) {
-            uint32_t h[8];
+          // columns nc .. nc+15: gate rows, nc+16 .. nc+31: the matching up
+          // rows; eight of each at a time (fewer live registers)
+#pragma unroll 1
+          for (int hh = 0; hh < 2; ++hh) {
+            uint32_t gr[8], ur[8];
+            tc_ld_32x32b_x8(tcol + hh * 8, gr);
+            tc_ld_32x32b_x8(tcol + 16 + hh * 8, ur);
+            if (m < p.M && nc < p.N) {
+              uint32_t h[4];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const float a = silu_f32(__uint_as_float(r[2 * e])) * __uint_as_float(r[16 + 2 * e]);
-              const float b = silu_f32(__uint_as_float(r[2 * e + 1])) * __uint_as_float(r[16 + 2 * e + 1]);
-              h[e] = uint32_t(__half_as_ushort(__float2half_rn(a))) |
-                     (uint32_t(__half_as_ushort(__float2half_rn(b))) << 16);
+              for (int e = 0; e < 4; ++e) {
+                const float a = silu_f32(__uint_as_float(gr[2 * e])) * __uint_as_float(ur[2 * e]);
+                const float b = silu_f32(__uint_as_float(gr[2 * e + 1])) * __uint_as_float(ur[2 * e + 1]);
+                h[e] = uint32_t(__half_as_ushort(__float2half_rn(a))) |
+                       (uint32_t(__half_as_ushort(__float2half_rn(b))) << 16);
+              }
+              reinterpret_cast<uint4*>(p.y + m * (p.N / 2) + nc / 2)[hh] = make_uint4(h[0], h[1], h[2], h[3]);
             }
-            uint4* dst = reinterpret_cast<uint4*>(p.y + m * (p.N / 2) + nc / 2);
-            dst[0] = make_uint4(h[0], h[1], h[2], h[3]);
-            dst[1] = make_uint4(h[4], h[5], h[6], h[7]);
           }
-        } else if (m < p.M && nc < p.N) {   // (an else of the constexpr if: plain kernels only)
-          uint32_t h[16];
+        } else {
+          // (tcgen05.ld is warp-collective: every lane loads, whatever its row)
+          uint32_t r[32];
+          tc_ld_32x32b_x32(tcol, r);
+          if (m < p.M && nc < p.N) {
+            uint32_t h[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const uint32_t lo = __half_as_ushort(__float2half_rn(__uint_as_float(r[2 * e])));
-            const uint32_t hi = __half_as_ushort(__float2half_rn(__uint_as_float(r[2 * e + 1])));
-            h[e] = lo | (hi << 16);
-          }
-          if (nc + 32 <= p.N && (p.N & 7) == 0) {
-            uint4* dst = reinterpret_cast<uint4*>(yrow + nc);
+            for (int e = 0; e < 16; ++e) {
+              const uint32_t lo = __half_as_ushort(__float2half_rn(__uint_as_float(r[2 * e])));
+              const uint32_t hi = __half_as_ushort(__float2half_rn(__uint_as_float(r[2 * e + 1])));
+              h[e] = lo | (hi << 16);
+            }
+            if (nc + 32 <= p.N && (p.N & 7) == 0) {
+              uint4* dst = reinterpret_cast<uint4*>(yrow + nc);
 #pragma unroll
-            for (int v = 0; v < 4; ++v) dst[v] = make_uint4(h[4 * v], h[4 * v + 1], h[4 * v + 2], h[4 * v + 3]);
-          } else {
-            for (int e = 0; e < 32 && nc + e < p.N; ++e)
-              yrow[nc + e] = uint16_t((h[e >> 1] >> ((e & 1) * 16)) & 0xFFFF);
+              for (int v = 0; v < 4; ++v) dst[v] = make_uint4(h[4 * v], h[4 * v + 1], h[4 * v + 2], h[4 * v + 3]);
+            } else {
+              for (int e = 0; e < 32 && nc + e < p.N; ++e)
+                yrow[nc + e] = uint16_t((h[e >> 1] >> ((e & 1) * 16)) & 0xFFFF);
+            }
           }
         }
       }
@@ -469,8 +510,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
           const int64_t m = int64_t(m0) + hm * BMH + r;
           if (m >= p.M || n0 + gc >= p.N) continue;
           const uint32_t offg = smem_u32(part + r * kPartStride + gc);
-          const float4 g = sum_slices_dsmem(offg, p.S);
-          const float4 u = sum_slices_dsmem(offg + 16 * 4, p.S);
+          float4 g, u;
+          sum_slices_dsmem2(offg, offg + 16 * 4, p.S, g, u);
           const uint32_t lo = uint32_t(__half_as_ushort(__float2half_rn(silu_f32(g.x) * u.x))) |
                               (uint32_t(__half_as_ushort(__float2half_rn(silu_f32(g.y) * u.y))) << 16);
           const uint32_t hi = uint32_t(__half_as_ushort(__float2half_rn(silu_f32(g.z) * u.z))) |
