@@ -20,25 +20,52 @@ constexpr int kQuantThreads = 256;
 
 // One warp per (row, group) unit. Lane l holds k = 4l .. 4l+3 of the group:
 // a coalesced 256-byte read per warp, min/max by butterfly shuffles, and
-// the packed word of k = 8w .. 8w+7 assembled from lanes 2w and 2w+1.
-template <bool ZP>
+// the packed word of k = 8w .. 8w+7 assembled from lanes 2w and 2w+1. A warp
+// reads the groups of kUnitsAhead units before working on the first, so that
+// several reads are in flight per warp. SCALED: the weights are first
+// multiplied by a per-input-channel factor and rounded to fp16, exactly as
+// awq_apply_scale writes them (the scale search quantizes W diag(s) without
+// storing it).
+constexpr int kUnitsAhead = 4;
+
+template <bool ZP, bool SCALED>
 __global__ void __launch_bounds__(kQuantThreads)
-quantize_pack_kernel(const uint16_t* __restrict__ W, int64_t N, int64_t K,
+quantize_pack_kernel(const uint16_t* __restrict__ W, const float* __restrict__ colscale, int64_t N, int64_t K,
                      int32_t* __restrict__ qweight, uint16_t* __restrict__ scales,
                      uint16_t* __restrict__ zeros) {
   const int lane = threadIdx.x & 31;
   const int64_t G = K / kGroup;
   const int64_t units = N * G;
   const int64_t nwarps = (int64_t(gridDim.x) * blockDim.x) >> 5;
-  for (int64_t u = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; u < units; u += nwarps) {
+  for (int64_t u0 = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; u0 < units; u0 += kUnitsAhead * nwarps) {
+  uint2 raws[kUnitsAhead];
+#pragma unroll
+  for (int a = 0; a < kUnitsAhead; ++a) {
+    const int64_t u = u0 + a * nwarps;
+    if (u < units) {
+      const int64_t n = u / G, j = u - n * G;
+      raws[a] = *reinterpret_cast<const uint2*>(W + n * K + j * kGroup + lane * 4);
+    }
+  }
+#pragma unroll
+  for (int a = 0; a < kUnitsAhead; ++a) {
+    const int64_t u = u0 + a * nwarps;
+    if (u >= units) break;
     const int64_t n = u / G;
     const int64_t j = u - n * G;
-    const uint2 raw = *reinterpret_cast<const uint2*>(W + n * K + j * kGroup + lane * 4);
+    const uint2 raw = raws[a];
     float w[4];
     w[0] = half_bits_to_float(uint16_t(raw.x & 0xFFFF));
     w[1] = half_bits_to_float(uint16_t(raw.x >> 16));
     w[2] = half_bits_to_float(uint16_t(raw.y & 0xFFFF));
     w[3] = half_bits_to_float(uint16_t(raw.y >> 16));
+    if (SCALED) {
+      const float4 cs = *reinterpret_cast<const float4*>(colscale + j * kGroup + lane * 4);
+      w[0] = half_bits_to_float(__half_as_ushort(__float2half_rn(__fmul_rn(w[0], cs.x))));
+      w[1] = half_bits_to_float(__half_as_ushort(__float2half_rn(__fmul_rn(w[1], cs.y))));
+      w[2] = half_bits_to_float(__half_as_ushort(__float2half_rn(__fmul_rn(w[2], cs.z))));
+      w[3] = half_bits_to_float(__half_as_ushort(__float2half_rn(__fmul_rn(w[3], cs.w))));
+    }
 
     int q[4];
     float sf, zf;
@@ -61,6 +88,7 @@ quantize_pack_kernel(const uint16_t* __restrict__ W, int64_t N, int64_t K,
       scales[j * N + n] = __half_as_ushort(__float2half_rn(sf));
       if (ZP) zeros[j * N + n] = __half_as_ushort(__int2half_rn(int(zf)));
     }
+  }
   }
 }
 
@@ -150,6 +178,29 @@ int grid_for(int64_t work_items, int threads_per_item, int threads_per_block) {
 }
 
 }  // namespace
+
+// W diag(colscale) (colscale null: W) quantized and packed as by
+// awq_pseudo_quantize_pack; arguments already checked by the caller.
+awq_status_t quantize_pack_scaled(const uint16_t* W, const float* colscale, int64_t N, int64_t K, awq_qconfig_t cfg,
+                                  int32_t* qweight, uint16_t* scales, uint16_t* zeros, void* stream) {
+  const int64_t units = N * (K / kGroup);
+  if (units == 0) return AWQ_OK;
+  const int grid = grid_for((units + kUnitsAhead - 1) / kUnitsAhead, 32, kQuantThreads);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (colscale) {
+    if (cfg.zero_point)
+      quantize_pack_kernel<true, true><<<grid, kQuantThreads, 0, s>>>(W, colscale, N, K, qweight, scales, zeros);
+    else
+      quantize_pack_kernel<false, true><<<grid, kQuantThreads, 0, s>>>(W, colscale, N, K, qweight, scales, nullptr);
+  } else {
+    if (cfg.zero_point)
+      quantize_pack_kernel<true, false><<<grid, kQuantThreads, 0, s>>>(W, nullptr, N, K, qweight, scales, zeros);
+    else
+      quantize_pack_kernel<false, false><<<grid, kQuantThreads, 0, s>>>(W, nullptr, N, K, qweight, scales, nullptr);
+  }
+  return launch_status();
+}
+
 }  // namespace awq
 
 using namespace awq;
@@ -167,14 +218,7 @@ extern "C" awq_status_t awq_pseudo_quantize_pack(const uint16_t* W, int64_t N, i
   if (!cfg.zero_point && zeros) return AWQ_ERR_SHAPE;
   if (!aligned16(W) || !aligned16(qweight) || !aligned16(scales) || (zeros && !aligned16(zeros)))
     return AWQ_ERR_ALIGN;
-  const int64_t units = N * (K / kGroup);
-  const int grid = grid_for(units, 32, kQuantThreads);
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cfg.zero_point)
-    quantize_pack_kernel<true><<<grid, kQuantThreads, 0, s>>>(W, N, K, qweight, scales, zeros);
-  else
-    quantize_pack_kernel<false><<<grid, kQuantThreads, 0, s>>>(W, N, K, qweight, scales, nullptr);
-  return launch_status();
+  return quantize_pack_scaled(W, nullptr, N, K, cfg, qweight, scales, zeros, stream);
 }
 
 extern "C" awq_status_t awq_dequant(const int32_t* qweight, const uint16_t* scales,

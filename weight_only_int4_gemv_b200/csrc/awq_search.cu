@@ -11,10 +11,11 @@
 // For every grid point alpha = i / n_grid the candidate
 //   s = max(mean|x|^alpha / (mean|w^|^(1 - alpha) + 1e-4), 1e-4)   (duo)
 //   s = max(mean|x|^alpha, 1e-4)                                  (no duo)
-// is divided by sqrt(max s * min s); W diag(s) is quantized by
-// awq_pseudo_quantize_pack, (x / s) is multiplied by it with awq_gemv /
-// awq_gemm, and the loss is the mean of (y_ref - y)^2 over the outputs, y_ref
-// = fp16(x . W^T). Every step runs on the device in stream order; the best
+// is divided by sqrt(max s * min s); W diag(s) (rounded to fp16) is quantized
+// by the quantizer of awq_pseudo_quantize_pack reading W and s directly, (x /
+// s) is multiplied by it with awq_gemv / awq_gemm, and the loss is the mean
+// of (y_ref - y)^2 over the outputs, y_ref = fp16(x . W^T) on the tensor
+// cores. Every step runs on the device in stream order; the best
 // grid point (first minimum) is picked on the device too, so the call makes
 // no host synchronization. Sums are taken in a fixed order: same inputs, same
 // bits.
@@ -27,6 +28,11 @@
 
 
 namespace awq {
+
+// the quantizer with a per-input-channel factor (awq_quant.cu)
+awq_status_t quantize_pack_scaled(const uint16_t* W, const float* colscale, int64_t N, int64_t K, awq_qconfig_t cfg,
+                                  int32_t* qweight, uint16_t* scales, uint16_t* zeros, void* stream);
+
 namespace {
 
 constexpr float kScaleEps = 1e-4f;
@@ -78,44 +84,108 @@ __global__ void weight_norm_finish_kernel(const float* __restrict__ partial, int
   out[k] = sum / float(N);
 }
 
-// y_ref[m][n] = fp16(sum_k x[m][k] w[n][k]) in fp32: 64 x 64 output tiles,
-// 256 threads of 4 x 4 outputs, k in steps of 32 through shared memory.
-__global__ void __launch_bounds__(256) reference_product_kernel(const uint16_t* __restrict__ X,
-                                                                const uint16_t* __restrict__ W, int64_t Ms,
-                                                                int64_t N, int64_t K, uint16_t* __restrict__ y) {
-  __shared__ float xs[64][33];
-  __shared__ float ws[64][33];
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  const int64_t m0 = int64_t(blockIdx.y) * 64, n0 = int64_t(blockIdx.x) * 64;
-  float acc[4][4] = {};
-  for (int64_t k0 = 0; k0 < K; k0 += 32) {
-    for (int i = threadIdx.x; i < 64 * 32; i += 256) {
-      const int r = i >> 5, c = i & 31;
-      xs[r][c] = (m0 + r < Ms) ? h2f(X[(m0 + r) * K + k0 + c]) : 0.0f;
-      ws[r][c] = (n0 + r < N) ? h2f(W[(n0 + r) * K + k0 + c]) : 0.0f;
+// y_ref[m][n] = fp16(sum_k x[m][k] w[n][k]) with fp32 accumulation on the
+// tensor cores (mma.sync m16n8k16, fp16 operands): 128 x 128 output tiles,
+// 8 warps of 64 (m) x 32 (n), k in steps of 32 through a two-stage
+// cp.async ring. Shared rows are 64 bytes (32 halves); the 16-byte chunk c of
+// row r sits at chunk c ^ ((r >> 1) & 3), so that the eight rows an ldmatrix
+// reads fall in eight different bank groups. Rows past Ms or N are read as
+// zeros (cp.async with no source bytes).
+constexpr int kRefBM = 128, kRefBN = 128, kRefBK = 32, kRefThreads = 256;
+
+__device__ __forceinline__ uint32_t ref_swz(int row, int chunk) {
+  return uint32_t(row * 64 + ((chunk ^ ((row >> 1) & 3)) << 4));
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
+               : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t a, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(a));
+}
+
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__global__ void __launch_bounds__(kRefThreads) reference_product_kernel(const uint16_t* __restrict__ X,
+                                                                        const uint16_t* __restrict__ W, int64_t Ms,
+                                                                        int64_t N, int64_t K,
+                                                                        uint16_t* __restrict__ y) {
+  __shared__ __align__(128) uint8_t sm[2][2][kRefBM * kRefBK * 2];   // [stage][x, w][128 rows x 64 B]
+  const int tid = int(threadIdx.x), lane = tid & 31, warp = tid >> 5;
+  const int wm = warp >> 2, wn = warp & 3;            // warp tile: rows 64 wm.., columns 32 wn..
+  const int64_t m0 = int64_t(blockIdx.y) * kRefBM, n0 = int64_t(blockIdx.x) * kRefBN;
+  const uint32_t base = static_cast<uint32_t>(__cvta_generic_to_shared(sm));
+  constexpr uint32_t kTileBytes = kRefBM * kRefBK * 2;
+
+  // one stage: 128 rows x 4 chunks of x and of w, two chunks of each per thread
+  auto load = [&](int stage, int64_t k0) {
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int idx = tid + e * kRefThreads, row = idx >> 2, chunk = idx & 3;
+      const int64_t xm = m0 + row, wn_ = n0 + row;
+      const uint32_t sx = base + uint32_t(stage) * 2 * kTileBytes + ref_swz(row, chunk);
+      cp_async16(sx, X + (xm < Ms ? xm : 0) * K + k0 + chunk * 8, xm < Ms);
+      cp_async16(sx + kTileBytes, W + (wn_ < N ? wn_ : 0) * K + k0 + chunk * 8, wn_ < N);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+
+  float acc[4][4][4] = {};
+  const int nk = int(K / kRefBK);
+  load(0, 0);
+  for (int kb = 0; kb < nk; ++kb) {
+    if (kb + 1 < nk) {
+      load((kb + 1) & 1, int64_t(kb + 1) * kRefBK);
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    } else {
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
     }
     __syncthreads();
-#pragma unroll 8
-    for (int c = 0; c < 32; ++c) {
-      float a[4], b[4];
+    const uint32_t sx = base + uint32_t(kb & 1) * 2 * kTileBytes, sw = sx + kTileBytes;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        a[i] = xs[ty * 4 + i][c];
-        b[i] = ws[tx * 4 + i][c];
+    for (int kk = 0; kk < 2; ++kk) {           // two k16 steps per stage
+      uint32_t a[4][4], b[4][2];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {            // A: rows 64 wm + 16 i + (lane % 16), k half lane / 16
+        const int row = wm * 64 + i * 16 + (lane & 15);
+        ldsm_x4(sx + ref_swz(row, kk * 2 + (lane >> 4)), a[i][0], a[i][1], a[i][2], a[i][3]);
+      }
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {            // B: two n8 tiles per ldmatrix.x4
+        const int row = wn * 32 + j * 16 + (lane & 7) + ((lane >> 4) << 3);
+        ldsm_x4(sw + ref_swz(row, kk * 2 + ((lane >> 3) & 1)), b[2 * j][0], b[2 * j][1], b[2 * j + 1][0],
+                b[2 * j + 1][1]);
       }
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+        for (int jn = 0; jn < 4; ++jn) mma16816(acc[i][jn], a[i], b[jn][0], b[jn][1]);
     }
     __syncthreads();
   }
+  const int g = lane >> 2, t = lane & 3;
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int64_t m = m0 + ty * 4 + i, n = n0 + tx * 4 + j;
-      if (m < Ms && n < N) y[m * N + n] = f2h(acc[i][j]);
+    for (int jn = 0; jn < 4; ++jn) {
+      const int64_t n = n0 + wn * 32 + jn * 8 + 2 * t;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int64_t m = m0 + wm * 64 + i * 16 + g + 8 * h;
+        if (m < Ms && n < N)   // N % 8 == 0: n + 1 < N too
+          *reinterpret_cast<uint32_t*>(y + m * N + n) =
+              uint32_t(f2h(acc[i][jn][2 * h])) | (uint32_t(f2h(acc[i][jn][2 * h + 1])) << 16);
+      }
     }
 }
 
@@ -358,7 +428,7 @@ __global__ void __launch_bounds__(256) apply_clip_kernel(const uint16_t* __restr
 size_t align256(size_t v) { return (v + 255) / 256 * 256; }
 
 struct SearchLayout {
-  size_t x_mean, w_mean, w_part, s, loss_part, y_ref, y_q, w_s, x_s, qweight, scales, zeros, prod_ws, total;
+  size_t x_mean, w_mean, w_part, s, loss_part, y_ref, y_q, x_s, qweight, scales, zeros, prod_ws, total;
 };
 
 awq_status_t search_layout(int64_t N, int64_t K, int64_t Ms, awq_qconfig_t cfg, SearchLayout& L) {
@@ -381,7 +451,6 @@ awq_status_t search_layout(int64_t N, int64_t K, int64_t Ms, awq_qconfig_t cfg, 
   L.loss_part = take(size_t(kLossBlocks) * 8);
   L.y_ref = take(size_t(Ms) * size_t(N) * 2);
   L.y_q = take(size_t(Ms) * size_t(N) * 2);
-  L.w_s = take(size_t(N) * size_t(K) * 2);
   L.x_s = take(size_t(Ms) * size_t(K) * 2);
   L.qweight = take(size_t(N) * size_t(K / 8) * 4);
   L.scales = take(G * size_t(N) * 2);
@@ -449,7 +518,6 @@ extern "C" awq_status_t awq_search_scale(const uint16_t* W, int64_t N, int64_t K
   double* loss_part = reinterpret_cast<double*>(ws + L.loss_part);
   uint16_t* y_ref = reinterpret_cast<uint16_t*>(ws + L.y_ref);
   uint16_t* y_q = reinterpret_cast<uint16_t*>(ws + L.y_q);
-  uint16_t* w_s = reinterpret_cast<uint16_t*>(ws + L.w_s);
   uint16_t* x_s = reinterpret_cast<uint16_t*>(ws + L.x_s);
   int32_t* qweight = reinterpret_cast<int32_t*>(ws + L.qweight);
   uint16_t* qscales = reinterpret_cast<uint16_t*>(ws + L.scales);
@@ -464,17 +532,17 @@ extern "C" awq_status_t awq_search_scale(const uint16_t* W, int64_t N, int64_t K
   act_mean_abs_kernel<<<kb, 256, 0, cs>>>(X, Ms, K, x_mean);
   weight_norm_partial_kernel<<<dim3(unsigned(K / 128), kWRowSplit), 128, 0, cs>>>(W, N, K, w_part);
   weight_norm_finish_kernel<<<kb, 256, 0, cs>>>(w_part, N, K, w_mean);
-  reference_product_kernel<<<dim3(unsigned((N + 63) / 64), unsigned((Ms + 63) / 64)), 256, 0, cs>>>(X, W, Ms, N, K,
-                                                                                                   y_ref);
+  reference_product_kernel<<<dim3(unsigned((N + kRefBN - 1) / kRefBN), unsigned((Ms + kRefBM - 1) / kRefBM)),
+                             kRefThreads, 0, cs>>>(X, W, Ms, N, K, y_ref);
   if ((st = launch_status()) != AWQ_OK) return st;
   const int64_t outs = Ms * N;
   const int sgrid = device_sms() * 8;   // grid-stride column scaling: eight CTAs per SM
   for (int i = 0; i < n_grid; ++i) {
     candidate_kernel<<<1, 1024, 0, cs>>>(x_mean, w_mean, K, n_grid, i, losses_out, duo, s);
-    scale_columns_kernel<<<sgrid, 256, 0, cs>>>(W, s, N, K, 1, w_s);
     scale_columns_kernel<<<sgrid, 256, 0, cs>>>(X, s, Ms, K, 0, x_s);
     if ((st = launch_status()) != AWQ_OK) return st;
-    if ((st = awq_pseudo_quantize_pack(w_s, N, K, cfg, qweight, qscales, qzeros, stream)) != AWQ_OK) return st;
+    // W diag(s) is quantized straight from W (never stored)
+    if ((st = quantize_pack_scaled(W, s, N, K, cfg, qweight, qscales, qzeros, stream)) != AWQ_OK) return st;
     st = Ms <= 16 ? awq_gemv(x_s, qweight, qscales, qzeros, Ms, N, K, cfg, y_q, prod_ws, prod_bytes, stream)
                   : awq_gemm(x_s, qweight, qscales, qzeros, Ms, N, K, cfg, y_q, prod_ws, prod_bytes, stream);
     if (st != AWQ_OK) return st;
