@@ -557,7 +557,10 @@ def run_e2e(awq, torch, device, stream, model, shapes, M, args, dist, step_bytes
     """Same metric through the Python API with host buffers: every step copies
     its input x from pinned host memory to the device, runs the layer (one
     prepared chain call of that step), reads the layer's result (the last
-    projection's output) back into pinned host memory, then synchronizes."""
+    projection's output) back into pinned host memory, then synchronizes.
+    By default the three operations of a step are replayed from one CUDA
+    graph per layer copy (as a serving loop would run them); --e2e-eager
+    issues them one by one."""
     steps = max(1, min(args.steps, args.e2e_steps))
     hx = torch.empty_like(model.step_input(0), device="cpu").pin_memory()
     hy = torch.empty_like(model.ys[0][-1], device="cpu").pin_memory()
@@ -576,9 +579,25 @@ def run_e2e(awq, torch, device, stream, model, shapes, M, args, dist, step_bytes
         hy.copy_(model.ys[c][-1], non_blocking=True)
         torch.cuda.current_stream(device).synchronize()
 
+    graphs = []
     with torch.cuda.stream(stream):
         for s in range(max(min(args.warmup, 20), model.n)):   # every layer copy's chain is prepared
             step(s)
+        if not args.e2e_eager and not args.per_gemv:
+            for c in range(model.n):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    model.step_input(c).copy_(hx, non_blocking=True)
+                    model.chain(c, 1)()
+                    hy.copy_(model.ys[c][-1], non_blocking=True)
+                graphs.append(g)
+
+            def step(s):   # noqa: F811 (the graph form of the same step)
+                graphs[s % model.n].replay()
+                torch.cuda.current_stream(device).synchronize()
+
+            for s in range(model.n):
+                step(s)
         if dist is not None:
             dist.barrier()
         torch.cuda.synchronize(device)
@@ -593,7 +612,9 @@ def run_e2e(awq, torch, device, stream, model, shapes, M, args, dist, step_bytes
     return {"value": round(total / max_s / 1e9, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": steps,
             "note": "effective HBM GB/s of the same algorithmic bytes, time includes the copies and a "
-                    "host synchronize per step (one launch per step)"}
+                    "host synchronize per step (one launch per step" +
+                    (", issued one by one)" if args.e2e_eager or args.per_gemv else
+                     "; copy in, launch and copy out replayed from one CUDA graph per step)")}
 
 
 def run_scale_search(awq, torch, device):
@@ -817,6 +838,8 @@ def parse_args(argv=None):
     ap.add_argument("--workload", choices=["llama3_8b_decode", "decode_sweep"], default="llama3_8b_decode")
     ap.add_argument("--layers", type=int, default=32, help="layer copies the steps rotate over")
     ap.add_argument("--e2e-steps", type=int, default=500)
+    ap.add_argument("--e2e-eager", action="store_true",
+                    help="e2e: issue each step's copies and launch one by one instead of replaying a graph")
     ap.add_argument("--gemm-steps", type=int, default=100)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-rows", type=int, default=256)
