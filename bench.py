@@ -827,6 +827,54 @@ def run_table(args):
             del g
         del packs
         torch.cuda.empty_cache()
+    if not only:
+        run_table_chain(awq, torch, device, hbm_peak, peak_src)
+
+
+def run_table_chain(awq, torch, device, hbm_peak, peak_src):
+    """The Llama-3-8B decode step (the bench's data flow: gate/up on q's
+    output, down on up's, the next q on down's) through awq_gemv_chain at
+    M = 1 .. 16, asymmetric and symmetric: 8 steps per launch over 8 layer
+    copies (0.8 GB of packed weights), 64 steps replayed from one CUDA graph.
+    One JSON line per (M, variant) with the time per step."""
+    from workloads import make_packed_random
+    shapes = LLAMA3_8B_DECODE
+    stream = torch.cuda.Stream(device)
+    for zp in (True, False):
+        base = [[torch.from_numpy(a).to(device) if a is not None else None
+                 for a in make_packed_random(sh.N, sh.K, 128, zp, seed=1)] for sh in shapes]
+        n = 8
+        packed = [[tuple(t.clone() if t is not None else None for t in b) for b in base] for _ in range(n)]
+        for M in (1, 2, 4, 8, 16):
+            rng = np.random.default_rng(M)
+            ys = [[torch.from_numpy(rng.standard_normal((M, sh.N), dtype=np.float32).astype(np.float16) * 0.01)
+                   .to(device) for sh in shapes] for _ in range(n)]
+            model = DecodeModel(awq, torch, packed, ys, shapes, M, awq.CHAIN_MAX_LAYERS // len(shapes))
+            steps = 64
+            with torch.cuda.stream(stream):
+                model.run_steps_chain(0, steps)
+            torch.cuda.synchronize(device)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                model.run_steps_chain(0, steps)
+            ts = []
+            for _ in range(4):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                with torch.cuda.stream(stream):
+                    g.replay()
+                e1.record(stream)
+                torch.cuda.synchronize(device)
+                ts.append(e0.elapsed_time(e1) * 1e3 / steps)
+            us = float(np.median(ts[1:]))
+            nbytes = sum(algo_bytes(M, sh.N, sh.K, zp) for sh in shapes)
+            gbs = nbytes / (us * 1e-6) / 1e9
+            print(json.dumps({"entry": "awq_gemv_chain llama3_8b step" + ("" if zp else " symmetric"), "M": M,
+                              "us_per_step": round(us, 3), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm_peak, 4),
+                              "peaks": peak_src, "device_error": awq.awq_device_error()}), flush=True)
+            del g, model
+        del packed, base
+        torch.cuda.empty_cache()
 
 
 def parse_args(argv=None):

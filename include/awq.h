@@ -112,7 +112,9 @@ typedef struct awq_qconfig {
  *   y[m][n] = fp16( silu(g) * u ),  silu(v) = v / (1 + exp(-v)),
  * g and u the fp32 sums of gate row n and up row n (the values awq_gemv /
  * awq_gemm would round to fp16 for those rows), silu and the product in
- * fp32 (expf). Requires N % 32 == 0. awq_workspace_bytes takes the flag. */
+ * fp32 with the fast exponential and division intrinsics (within a few fp32
+ * ulp of the exact silu). Requires N % 32 == 0. awq_workspace_bytes takes
+ * the flag. */
 #define AWQ_FLAG_SILU_MUL 2u
 
 /* Packed zero points ("AWQ > Implementation", "Understanding the Quantization
@@ -122,12 +124,14 @@ typedef struct awq_qconfig {
  * qzeros[K/128][N/8] instead of fp16 zeros[K/128][N]: word w of group row j
  * holds the zero points of output channels 8w .. 8w+7 of that group, channel
  * 8w+i in bits 4i .. 4i+3 (awq_pack_zeros writes it from the fp16 array).
- * Results are identical to the fp16 form of the same zero points. Needs
- * zero_point = 1 (else AWQ_ERR_UNSUPPORTED); N % 32 == 0 for awq_gemv and
- * awq_gemv_noalloc (a group row of qzeros is then whole 16-byte runs), N % 8
- * == 0 for awq_dequant (else AWQ_ERR_SHAPE). awq_workspace_bytes takes it for
- * M <= 16. Every other entry point, awq_gemm included, returns
- * AWQ_ERR_UNSUPPORTED for it (awq_unpack_zeros restores the fp16 form). */
+ * Results are identical to the fp16 form of the same zero points. The GEMV
+ * reads the packed words directly; awq_gemm unpacks them into its workspace
+ * first (G x N x 2 bytes, which awq_workspace_bytes counts for M > 16). Needs
+ * zero_point = 1 (else AWQ_ERR_UNSUPPORTED); N % 32 == 0 for awq_gemv,
+ * awq_gemv_noalloc and awq_gemm (a group row of qzeros is then whole 16-byte
+ * runs), N % 8 == 0 for awq_dequant (else AWQ_ERR_SHAPE). Every other entry
+ * point returns AWQ_ERR_UNSUPPORTED for it (awq_unpack_zeros restores the
+ * fp16 form). */
 #define AWQ_FLAG_PACKED_ZEROS 4u
 
 /* ABI version of the loaded library (AWQ_ABI_VERSION at build time). */
@@ -332,8 +336,10 @@ AWQ_API awq_status_t awq_debug_set_wait_limit_ns(uint64_t ns, void* stream);
  * multiplied on the tensor cores (tcgen05, fp16 inputs, fp32 accumulation in
  * tensor memory); y = fp16 of the fp32 sum.
  * M >= 0, N >= 0 (either 0: no work); K > 0, K % group_size == 0.
- * cfg.flags may hold AWQ_FLAG_SILU_MUL (y is then [M][N/2]).
- * Workspace as for awq_gemv.
+ * cfg.flags may hold AWQ_FLAG_SILU_MUL (y is then [M][N/2]) and
+ * AWQ_FLAG_PACKED_ZEROS (see there).
+ * Workspace as for awq_gemv: awq_workspace_bytes(M, N, K, cfg) bytes, 0
+ * (NULL allowed) unless the zero points are packed.
  */
 AWQ_API awq_status_t awq_gemm(const uint16_t* x, const int32_t* qweight,
                       const uint16_t* scales, const uint16_t* zeros,

@@ -217,9 +217,17 @@ def test_packed_zeros_validation(L):
         assert f(*args(0, cfg(flags=PZ)), *tail) == OK                    # empty
         assert f(*args(64, cfg(flags=PZ), z=0), *tail) == NULL
         assert f(*args(64, cfg(flags=PZ), z=MIS), *tail) == ALIGN
-    assert _gemv(L, c=cfg(flags=PZ), entry="awq_gemm") == UNSUP          # the GEMM reads fp16 zero points only
+    # the GEMM unpacks packed zero points into its workspace: none given, or too small
+    assert _gemv(L, M=32, c=cfg(flags=PZ), entry="awq_gemm") == WS
+    g = L.awq_gemm
+    assert g(P(A), P(A), P(A), P(A), 32, 64, 256, cfg(flags=PZ), P(A), P(A), 255, None) == WS
+    assert g(P(A), P(A), P(A), P(A), 32, 64, 256, cfg(flags=PZ), P(A), P(MIS), 256, None) == ALIGN
+    assert _gemv(L, M=32, N=48, c=cfg(flags=PZ), entry="awq_gemm") == SHAPE   # N % 32
+    assert _gemv(L, M=32, c=cfg(zp=0, flags=PZ), z=0, entry="awq_gemm") == UNSUP
     n = ctypes.c_size_t(7)
-    assert L.awq_workspace_bytes(32, 64, 256, cfg(flags=PZ), ctypes.byref(n)) == UNSUP
+    # M > 16: the fp16 copy of the zero points, G x N x 2 bytes
+    assert L.awq_workspace_bytes(32, 64, 256, cfg(flags=PZ), ctypes.byref(n)) == OK and n.value == 2 * 64 * 2
+    assert L.awq_workspace_bytes(32, 64, 256, cfg(), ctypes.byref(n)) == OK and n.value == 0
     assert L.awq_workspace_bytes(1, 48, 256, cfg(flags=PZ), ctypes.byref(n)) == SHAPE
     assert L.awq_workspace_bytes(1, 0, 256, cfg(flags=PZ), ctypes.byref(n)) == OK and n.value == 0
     d = L.awq_dequant

@@ -1,8 +1,9 @@
 """GPU parity of the packed zero points (AWQ_FLAG_PACKED_ZEROS, int32 qzeros
 [G][N/8]): awq_pack_zeros / awq_unpack_zeros bit for bit against the oracle,
 awq_dequant with packed zero points bit for bit against the oracle's
-dequantization, and awq_gemv with packed zero points against the float64
-oracle and bit for bit against the same call with the fp16 zero points."""
+dequantization, and awq_gemv and awq_gemm with packed zero points against
+the float64 oracle and bit for bit against the same call with the fp16 zero
+points."""
 
 import numpy as np
 import pytest
@@ -118,8 +119,43 @@ def test_gemv_packed_zeros_noalloc_and_fused_gate_up():
         assert_close(host(h4), O.gate_up_silu_f64(xm, Wg, Wu), f"fused packed M={M}")
 
 
-def test_gemm_refuses_packed_zeros():
+@pytest.mark.parametrize("M,N,K,silu", [(17, 256, 512, False), (128, 4096, 4096, False), (300, 1024, 2048, False),
+                                       (2048, 512, 1024, False), (96, 2048, 1024, True)])
+def test_gemm_with_packed_zeros_matches_fp16_zeros(M, N, K, silu):
+    """awq_gemm with int32 qzeros (unpacked into the workspace by the call)
+    gives the bits of the same call with the fp16 zero points, and stays
+    within the oracle's tolerance; with the fused gate/up layout too."""
+    if silu:
+        half = N // 2
+        _, qg, sg, zg, Wg = oracle_layer(half, K, 0.02, 0.01, True, seed=41)
+        _, qu, su, zu, Wu = oracle_layer(half, K, 0.02, 0.01, True, seed=42)
+        q, s, z = awq.awq_interleave_gate_up(dev(qg), dev(sg), dev(zg), dev(qu), dev(su), dev(zu))
+    else:
+        _, qweight, scales, zeros, Wd = oracle_layer(N, K, 0.02, 0.01, True, seed=M)
+        q, s, z = dev(qweight), dev(scales), dev(zeros)
+    qz = awq.awq_pack_zeros(z)
+    xh = activations(M, K, seed=M + 1)
+    x = dev(xh)
+    ws16 = awq.alloc_workspace(M, N, K, True, silu_mul=silu)
+    ws4 = awq.alloc_workspace(M, N, K, True, silu_mul=silu, packed_zeros=True)
+    assert ws4 is not None and ws4.numel() >= (K // 128) * N * 2
+    y16 = awq.awq_gemm(x, q, s, z, workspace=ws16, silu_mul=silu)
+    y4 = awq.awq_gemm(x, q, s, qz, workspace=ws4, silu_mul=silu)
+    torch.cuda.synchronize()
+    assert np.array_equal(bits(y4), bits(y16))
+    if silu:
+        assert_close(host(y4), O.gate_up_silu_f64(xh, Wg, Wu), f"fused packed gemm M={M}")
+    else:
+        rows = sample_rows(N, 512, seed=M)
+        assert_close(host(y4)[:, rows], O.matmul_f64(xh, Wd[rows]), f"packed gemm M={M}")
+    # awq_linear takes either form at any M
+    yl = awq.awq_linear(x, q, s, qz, workspace=ws4, silu_mul=silu)
+    torch.cuda.synchronize()
+    assert np.array_equal(bits(yl), bits(y16))
+
+
+def test_gemm_packed_zeros_without_room_is_refused():
     _, qweight, scales, zeros, _ = oracle_layer(256, 512, 0.02, 0.01, True)
     x = dev(activations(32, 512))
-    with pytest.raises(awq.AwqError, match="UNSUPPORTED"):
+    with pytest.raises(awq.AwqError, match="WORKSPACE"):
         awq.awq_gemm(x, dev(qweight), dev(scales), dev(O.pack_zeros(zeros)))

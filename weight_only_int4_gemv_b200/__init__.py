@@ -265,7 +265,7 @@ def awq_workspace_bytes(M: int, N: int, K: int, zero_point: bool = True, group_s
                         device=None, silu_mul: bool = False, packed_zeros: bool = False) -> int:
     """Workspace bytes awq_gemv / awq_gemm need on `device` for this shape
     (silu_mul: the fused gate/up layout, N = both projections' rows;
-    packed_zeros: int32 qzeros, GEMV only)."""
+    packed_zeros: int32 qzeros; the GEMM unpacks them into its workspace)."""
     n = ctypes.c_size_t(0)
     flags = (FLAG_SILU_MUL if silu_mul else 0) | (FLAG_PACKED_ZEROS if packed_zeros else 0)
     with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
@@ -373,15 +373,17 @@ def awq_gemv_noalloc(x, qweight, scales, zeros, out=None, group_size: int = GROU
 def awq_gemm(x, qweight, scales, zeros, workspace=None, out=None, group_size: int = GROUP_SIZE,
              silu_mul: bool = False):
     """y = x . W'^T for any M (prefill), on the tcgen05 tensor cores.
-    silu_mul: as for awq_gemv."""
+    silu_mul: as for awq_gemv. zeros may be fp16 [K/128, N] or int32 qzeros
+    [K/128, N/8] (N % 32 == 0; the workspace then holds their fp16 form:
+    alloc_workspace(..., packed_zeros=True))."""
     return _product("awq_gemm", x, qweight, scales, zeros, workspace, out, group_size, _flags(False, silu_mul))
 
 
 def awq_linear(x, qweight, scales, zeros, workspace=None, out=None, group_size: int = GROUP_SIZE,
                weights_static: bool = False, silu_mul: bool = False):
     """The layer with the documented M threshold: awq_gemv for M <= 16, else awq_gemm.
-    Packed zero points (int32 qzeros) are read by awq_gemv only: for M > 16 pass
-    the fp16 form (awq_unpack_zeros), or the call raises AWQ_ERR_UNSUPPORTED."""
+    Either zero-point form; with packed zero points at M > 16 the workspace
+    must come from alloc_workspace(..., packed_zeros=True)."""
     entry = "awq_gemv" if x.shape[0] <= GEMV_MAX_M else "awq_gemm"
     return _product(entry, x, qweight, scales, zeros, workspace, out, group_size,
                     _flags(weights_static, silu_mul))

@@ -33,12 +33,13 @@ extern "C" awq_status_t awq_workspace_bytes(int64_t M, int64_t N, int64_t K, awq
   if (st != AWQ_OK) return st;
   if ((st = check_nk(N, K)) != AWQ_OK) return st;
   if (M < 0) return AWQ_ERR_SHAPE;
-  // packed zero points are read by the GEMV only
-  if ((cfg.flags & AWQ_FLAG_PACKED_ZEROS) && M > 16) return AWQ_ERR_UNSUPPORTED;
   *bytes = 0;
   if (M == 0 || N == 0) return AWQ_OK;
   if ((cfg.flags & AWQ_FLAG_SILU_MUL) && N % 32) return AWQ_ERR_SHAPE;
   if ((cfg.flags & AWQ_FLAG_PACKED_ZEROS) && N % 32) return AWQ_ERR_SHAPE;
   if (M <= 16) return gemv_workspace_bytes(M, N, K, zero_mode(cfg), (cfg.flags & AWQ_FLAG_SILU_MUL) != 0, bytes);
-  return gemm_workspace_bytes(M, N, K, cfg.zero_point != 0, bytes);
+  if ((st = gemm_workspace_bytes(M, N, K, cfg.zero_point != 0, bytes)) != AWQ_OK) return st;
+  // the GEMM reads packed zero points through an fp16 copy in the workspace
+  if (cfg.flags & AWQ_FLAG_PACKED_ZEROS) *bytes += size_t(K / kGroup) * size_t(N) * 2;
+  return AWQ_OK;
 }

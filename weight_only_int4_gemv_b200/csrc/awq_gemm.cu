@@ -90,13 +90,13 @@ extern "C" awq_status_t awq_gemm(const uint16_t* x, const int32_t* qweight,
                                  const uint16_t* scales, const uint16_t* zeros, int64_t M,
                                  int64_t N, int64_t K, awq_qconfig_t cfg, uint16_t* y,
                                  void* workspace, size_t workspace_bytes, void* stream) {
-  (void)workspace;
-  (void)workspace_bytes;
-  awq_status_t st = check_cfg(cfg);
+  awq_status_t st = check_cfg(cfg, true);
   if (st != AWQ_OK) return st;
   if ((st = check_nk(N, K)) != AWQ_OK) return st;
   if (M < 0 || M > (int64_t(1) << 31) - 1) return AWQ_ERR_SHAPE;
   if ((cfg.flags & AWQ_FLAG_SILU_MUL) && N % 32) return AWQ_ERR_SHAPE;
+  const bool packed = (cfg.flags & AWQ_FLAG_PACKED_ZEROS) != 0;
+  if (packed && N % 32) return AWQ_ERR_SHAPE;
   if (M == 0 || N == 0) return AWQ_OK;
   if (!x || !qweight || !scales || !y) return AWQ_ERR_NULL;
   if (cfg.zero_point && !zeros) return AWQ_ERR_NULL;
@@ -104,6 +104,18 @@ extern "C" awq_status_t awq_gemm(const uint16_t* x, const int32_t* qweight,
   if (!aligned16(x) || !aligned16(qweight) || !aligned16(scales) || !aligned16(y) ||
       (zeros && !aligned16(zeros)))
     return AWQ_ERR_ALIGN;
+  if (packed) {
+    // Packed zero points: unpacked into the workspace (fp16 [K/128][N], the
+    // values the fp16 form holds), then the same product as with that form.
+    const int64_t G = K / kGroup;
+    const size_t need = size_t(G) * size_t(N) * 2;
+    if (!workspace || workspace_bytes < need) return AWQ_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return AWQ_ERR_ALIGN;
+    uint16_t* z16 = static_cast<uint16_t*>(workspace);
+    if ((st = awq_unpack_zeros(reinterpret_cast<const int32_t*>(zeros), G, N, z16, stream)) != AWQ_OK) return st;
+    zeros = z16;
+    cfg.flags &= ~AWQ_FLAG_PACKED_ZEROS;
+  }
 
   // The tile shape with the lowest estimated time (ties: the wider tiles).
   // Beyond 256 rows of x the 256-channel tiles always win (measured).
