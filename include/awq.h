@@ -288,7 +288,7 @@ AWQ_API awq_status_t awq_gemv_noalloc(const uint16_t* x, const int32_t* qweight,
  * layers: host memory, read before the call returns.
  * workspace: at least awq_gemv_chain_workspace_bytes() bytes of device
  * memory, zero-filled before its first use and then kept for calls with the
- * same layers (shapes, flags, x_from; the pointers may change) and not
+ * same M and layers (shapes, flags, x_from; the pointers may change) and not
  * written by anything else: between calls it holds a launch count and the
  * half of the output-copy region that the next call reads, zeroed (every
  * call that completes, also one whose waits gave up, leaves it so). A call
