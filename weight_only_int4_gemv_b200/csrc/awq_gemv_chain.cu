@@ -104,6 +104,16 @@ constexpr uint32_t kCodesBoxBytes = kTileBytes;
 static_assert(kFlagsOff + 8 <= kTableOff, "stage bookkeeping overflows its region");
 static_assert(kXOff % 1024 == 0, "x must start 1024-aligned inside a stage");
 
+// Stage geometry for chunks of up to TCAP tiles: codes [TCAP][group][16 rows]
+// [16 words], then scales, zero points and x. The batch tiles of 2 and 4
+// rows use two-tile stages, so that two CTAs of at least three stages share
+// an SM; the others use four-tile stages (the constants above).
+template <int TCAP> __host__ __device__ constexpr uint32_t scale_off() { return uint32_t(TCAP * kTileBytes); }
+template <int TCAP> __host__ __device__ constexpr uint32_t zero_off() { return scale_off<TCAP>() + kMetaBytes; }
+template <int TCAP> __host__ __device__ constexpr uint32_t x_off() { return zero_off<TCAP>() + kMetaBytes; }
+template <int MB> __host__ __device__ constexpr int tile_cap() { return MB == 2 || MB == 4 ? 2 : kMaxTC; }
+static_assert(x_off<2>() % 1024 == 0 && x_off<kMaxTC>() == uint32_t(kXOff), "stage geometry");
+
 struct alignas(64) LayerDesc {
   CUtensorMap tq;      // codes: {16 words, N rows, G groups}, box {16, 16, kCW}
   CUtensorMap tx;      // x: {128, G, M}, box {128, kCW, M}
@@ -392,13 +402,14 @@ __device__ __forceinline__ void fill_run(const LayerDesc& L, LayerRun& r) {
   r.ll_off = L.ll_off;
 }
 
+template <int TCAP>
 __device__ __forceinline__ void load_chunk(const LayerRun& R, int i, Chunk& c) {
   const int tpu = run_tpu(R);
   c.i = i;
   c.s = i / R.units;
   const int u0 = i - c.s * R.units;
   int nu = R.i1 - i;
-  const int cap = kMaxTC / tpu;
+  const int cap = TCAP / tpu;
   if (nu > cap) nu = cap;
   if (nu > R.units - u0) nu = R.units - u0;
   c.nu = nu;
@@ -416,34 +427,37 @@ struct Cursor {
   __device__ __forceinline__ bool done(int n) const { return l >= n; }
 };
 
+template <int TCAP>
 __device__ __forceinline__ void cursor_layer(const ChainParams& p, const LayerRun* runs, Cursor& u) {
   // from layer u.l on, the first layer with items for this CTA
   for (; u.l < p.n_layers; ++u.l) {
     const LayerRun& R = runs[u.l];
     if (R.i0 < R.i1) {
-      load_chunk(R, R.i0, u.c);
+      load_chunk<TCAP>(R, R.i0, u.c);
       u.gbase = u.c.gb;
       return;
     }
   }
 }
 
+template <int TCAP>
 __device__ __forceinline__ void cursor_init(const ChainParams& p, const LayerRun* runs, Cursor& u) {
   u.l = 0;
-  cursor_layer(p, runs, u);
+  cursor_layer<TCAP>(p, runs, u);
 }
 
+template <int TCAP>
 __device__ __forceinline__ void cursor_next(const ChainParams& p, const LayerRun* runs, Cursor& u) {
   u.gbase += kCW;
   if (u.gbase < u.c.ge) return;
   const int ni = u.c.i + u.c.nu;
   if (ni < runs[u.l].i1) {
-    load_chunk(runs[u.l], ni, u.c);
+    load_chunk<TCAP>(runs[u.l], ni, u.c);
     u.gbase = u.c.gb;
     return;
   }
   ++u.l;
-  cursor_layer(p, runs, u);
+  cursor_layer<TCAP>(p, runs, u);
 }
 
 template <int ZM>
@@ -456,7 +470,7 @@ __device__ __forceinline__ uint32_t weight_bytes(int tc) {
 // the weight copies: codes tile by tile, the 64-row runs of scales and zero
 // points (packed: 12 words from word 2 t0 rounded down to a multiple of 4,
 // a 16-byte boundary).
-template <int ZM>
+template <int ZM, int TCAP>
 __device__ __forceinline__ void issue_weights(const ChainParams& p, const LayerRun* runs, const Cursor& u, uint32_t st,
                                               uint32_t bar) {
   const LayerDesc& L = p.layer[u.l];
@@ -468,13 +482,14 @@ __device__ __forceinline__ void issue_weights(const ChainParams& p, const LayerR
                : "memory");
   const int r0 = u.c.t0 * kTile;
   for (int r = 0; r < u.c.tc; ++r) tma_3d(st + r * kTileBytes, &L.tq, 0, r0 + r * kTile, u.gbase, bar);
-  tma_2d(st + kScaleOff, &L.ts, r0, u.gbase, bar);
-  if (ZM == 2) tma_2d(st + kZeroOff, &L.tz, (2 * u.c.t0) & ~3, u.gbase, bar);
-  if (ZM == 1) tma_2d(st + kZeroOff, &L.tz, r0, u.gbase, bar);
+  tma_2d(st + scale_off<TCAP>(), &L.ts, r0, u.gbase, bar);
+  if (ZM == 2) tma_2d(st + zero_off<TCAP>(), &L.tz, (2 * u.c.t0) & ~3, u.gbase, bar);
+  if (ZM == 1) tma_2d(st + zero_off<TCAP>(), &L.tz, r0, u.gbase, bar);
 }
 
+template <int TCAP>
 __device__ __forceinline__ void issue_x(const ChainParams& p, const Cursor& u, uint32_t st, uint32_t bar) {
-  tma_3d(st + kXOff, &p.layer[u.l].tx, 0, u.gbase, 0, bar);
+  tma_3d(st + x_off<TCAP>(), &p.layer[u.l].tx, 0, u.gbase, 0, bar);
 }
 
 // ---------------------------------------------------------------------------
@@ -511,7 +526,8 @@ __device__ __forceinline__ bool x_needed(const ChainParams& p, const LayerRun* r
 // ---------------------------------------------------------------------------
 template <int MB, int ZM>
 __device__ __forceinline__ void stage_compute(uint32_t st, int w, int g, int t, int tc, int M, int zoff,
-                                              float (&acc)[kMaxTC][MB > 8 ? 2 : 1][4]) {
+                                              float (&acc)[tile_cap<MB>()][MB > 8 ? 2 : 1][4]) {
+  constexpr int TCAP = tile_cap<MB>();
   constexpr int MT = MB > 8 ? 2 : 1;
   constexpr bool ODD = MB > 1;        // batch columns 2t + 1 exist
   // x fragments: batch row m = 8 mt + g, this warp's group, k = 32 t .. 32 t + 31
@@ -519,7 +535,7 @@ __device__ __forceinline__ void stage_compute(uint32_t st, int w, int g, int t, 
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt) {
     const int m = 8 * mt + g;
-    const uint32_t xa = st + kXOff + uint32_t(m) * kXRowBytes + w * 256 + t * 64;
+    const uint32_t xa = st + x_off<TCAP>() + uint32_t(m) * kXRowBytes + w * 256 + t * 64;
 #pragma unroll
     for (int jj = 0; jj < 4; ++jj) xf[mt][jj] = (MB == 1 ? g == 0 : m < M) ? lds128(xa + jj * 16) : make_uint4(0, 0, 0, 0);
   }
@@ -538,9 +554,9 @@ __device__ __forceinline__ void stage_compute(uint32_t st, int w, int g, int t, 
     }
   }
   const uint32_t cbase = st + w * 1024 + g * 64 + t * 16;
-  const uint32_t sbase = st + kScaleOff + w * 128 + g * 2;
+  const uint32_t sbase = st + scale_off<TCAP>() + w * 128 + g * 2;
 #pragma unroll
-  for (int rt = 0; rt < kMaxTC; ++rt) {
+  for (int rt = 0; rt < TCAP; ++rt) {
     if (rt < tc) {
       const uint4 c_lo = lds128(cbase + rt * kTileBytes);
       const uint4 c_hi = lds128(cbase + rt * kTileBytes + 512);
@@ -568,7 +584,7 @@ __device__ __forceinline__ void stage_compute(uint32_t st, int w, int g, int t, 
       } else if constexpr (ZM == 2) {
         // rows g and g + 8 of tile rt: nibble g of words 2 rt and 2 rt + 1
         // past the chunk's first word (zoff: 8 bytes when t0 is odd)
-        const uint2 zz = lds64(st + kZeroOff + w * (kPackedZeroWords * 4) + zoff + rt * 8);
+        const uint2 zz = lds64(st + zero_off<TCAP>() + w * (kPackedZeroWords * 4) + zoff + rt * 8);
         z_lo = float((zz.x >> (4 * g)) & 0xFu);
         z_hi = float((zz.y >> (4 * g)) & 0xFu);
       } else {
@@ -592,9 +608,10 @@ __device__ __forceinline__ void stage_compute(uint32_t st, int w, int g, int t, 
 // the kernel
 // ---------------------------------------------------------------------------
 template <int MB, int ZM>
-__global__ void __launch_bounds__(kThreads, MB == 1 ? 2 : 1)
+__global__ void __launch_bounds__(kThreads, MB <= 4 ? 2 : 1)
 chain_kernel(const __grid_constant__ ChainParams p) {
   constexpr int MT = MB > 8 ? 2 : 1;
+  constexpr int TCAP = tile_cap<MB>();
   asm volatile("griddepcontrol.launch_dependents;");
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
@@ -632,29 +649,29 @@ chain_kernel(const __grid_constant__ ChainParams p) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       Cursor cw;
-      cursor_init(p, runs, cw);
+      cursor_init<TCAP>(p, runs, cw);
       Cursor cx = cw;               // stages whose weights were issued before the wait
       int sw = 0;                   // stages issued
       if (p.early) {
         for (; sw < S && !cw.done(p.n_layers); ++sw) {
-          issue_weights<ZM>(p, runs, cw, ring + sw * p.stage_bytes, full0 + 8 * sw);
-          cursor_next(p, runs, cw);
+          issue_weights<ZM, TCAP>(p, runs, cw, ring + sw * p.stage_bytes, full0 + 8 * sw);
+          cursor_next<TCAP>(p, runs, cw);
         }
       }
       asm volatile("griddepcontrol.wait;" ::: "memory");
       // x of those stages (layers whose x is an input of the call)
       for (int j = 0; j < sw; ++j) {
-        if (run_x_from(runs[cx.l]) < 0) issue_x(p, cx, ring + j * p.stage_bytes, full0 + 8 * j);
-        cursor_next(p, runs, cx);
+        if (run_x_from(runs[cx.l]) < 0) issue_x<TCAP>(p, cx, ring + j * p.stage_bytes, full0 + 8 * j);
+        cursor_next<TCAP>(p, runs, cx);
       }
       uint64_t t_slot = 0;          // start of the wait for a free slot (0: not waiting)
       while (!cw.done(p.n_layers)) {
         const int slot = sw % S;
         if (sw < S || mbar_test_wait(empty0 + 8 * slot, uint32_t((sw / S) + 1) & 1u)) {
           const uint32_t st = ring + slot * p.stage_bytes;
-          issue_weights<ZM>(p, runs, cw, st, full0 + 8 * slot);
-          if (run_x_from(runs[cw.l]) < 0) issue_x(p, cw, st, full0 + 8 * slot);
-          cursor_next(p, runs, cw);
+          issue_weights<ZM, TCAP>(p, runs, cw, st, full0 + 8 * slot);
+          if (run_x_from(runs[cw.l]) < 0) issue_x<TCAP>(p, cw, st, full0 + 8 * slot);
+          cursor_next<TCAP>(p, runs, cw);
           ++sw;
           t_slot = 0;
           continue;
@@ -725,10 +742,10 @@ chain_kernel(const __grid_constant__ ChainParams p) {
       const bool dep = run_x_from(R) >= 0;
       for (int i = R.i0; i < i1;) {
         Chunk cc;
-        load_chunk(R, i, cc);
-        float acc[kMaxTC][MT][4];
+        load_chunk<TCAP>(R, i, cc);
+        float acc[TCAP][MT][4];
 #pragma unroll
-        for (int rt = 0; rt < kMaxTC; ++rt)
+        for (int rt = 0; rt < TCAP; ++rt)
 #pragma unroll
           for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
@@ -776,7 +793,7 @@ chain_kernel(const __grid_constant__ ChainParams p) {
               if (live) {
 #pragma unroll
                 for (int m = 0; m < MB; ++m)
-                  if (m < M) sts64(st + kXOff + uint32_t(m) * kXRowBytes + w * 256 + lane * 8, ll_decode(px[m]));
+                  if (m < M) sts64(st + x_off<TCAP>() + uint32_t(m) * kXRowBytes + w * 256 + lane * 8, ll_decode(px[m]));
                 __syncwarp();
               }
             }
@@ -807,7 +824,7 @@ chain_kernel(const __grid_constant__ ChainParams p) {
         // ([warp][row][m]) and are summed in warp order (deterministic)
         const uint32_t pw = pbuf + uint32_t(w * 64 * M) * 4;
 #pragma unroll
-        for (int rt = 0; rt < kMaxTC; ++rt) {
+        for (int rt = 0; rt < TCAP; ++rt) {
           if (rt < cc.tc) {
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
@@ -912,7 +929,7 @@ chain_kernel(const __grid_constant__ ChainParams p) {
 // ---------------------------------------------------------------------------
 using ChainFn = void (*)(const ChainParams);
 
-constexpr int kNumVariants = 9;     // batch tile {1, 8, 16} x zero points {sym, fp16, packed}
+constexpr int kNumVariants = 15;    // batch tile {1, 2, 4, 8, 16} x zero points {sym, fp16, packed}
 constexpr int kSmemBudget = 232448;
 constexpr int kHalfSmBudget = 115712;
 constexpr int kMaxDevices = 64;
@@ -921,8 +938,10 @@ ChainFn pick(int64_t M, int zm, int& id) {
   static const ChainFn table[kNumVariants] = {
       chain_kernel<1, 0>, chain_kernel<1, 1>, chain_kernel<1, 2>,
       chain_kernel<8, 0>, chain_kernel<8, 1>, chain_kernel<8, 2>,
-      chain_kernel<16, 0>, chain_kernel<16, 1>, chain_kernel<16, 2>};
-  const int mb = M == 1 ? 0 : M <= 8 ? 1 : 2;
+      chain_kernel<16, 0>, chain_kernel<16, 1>, chain_kernel<16, 2>,
+      chain_kernel<2, 0>,  chain_kernel<2, 1>,  chain_kernel<2, 2>,
+      chain_kernel<4, 0>,  chain_kernel<4, 1>,  chain_kernel<4, 2>};
+  const int mb = M == 1 ? 0 : M == 2 ? 3 : M <= 4 ? 4 : M <= 8 ? 1 : 2;
   id = mb * 3 + zm;
   return table[id];
 }
@@ -939,7 +958,7 @@ struct LayerPlan {
 
 struct ChainPlan {
   ChainFn fn;
-  int id, grid, stages, stage_bytes, pbuf_offset, smem;
+  int id, grid, stages, stage_bytes, pbuf_offset, smem, tcap;
   LayerPlan lp[kMaxLayers];
   size_t ll_base, ll_half;           // the exchange region: two halves
   size_t ws_bytes;
@@ -982,7 +1001,7 @@ awq_status_t check_layer(const awq_gemv_layer_t* L, int l, const awq_gemv_layer_
 // partials). The constants are fitted to B200 timings of the Llama-3-8B
 // decode step (4 slices for its 4096-row layers, none for the 14336-row
 // ones).
-int64_t split_cost(int units, int tpu, int G, int ks, int grid) {
+int64_t split_cost(int units, int tpu, int G, int ks, int grid, int tcap) {
   constexpr int64_t kMinTiles = 3, kStageCost = 10, kChunkCost = 20, kSplitCost = 6;
   int64_t worst = 0;
   for (int b = 0; b < grid; ++b) {
@@ -992,7 +1011,7 @@ int64_t split_cost(int units, int tpu, int G, int ks, int grid) {
     for (int i = i0; i < i1;) {
       const int sl = i / units, u0 = i - sl * units;
       int nu = i1 - i;
-      if (nu > kMaxTC / tpu) nu = kMaxTC / tpu;
+      if (nu > tcap / tpu) nu = tcap / tpu;
       if (nu > units - u0) nu = units - u0;
       const int64_t g = int64_t(G) * (sl + 1) / ks - int64_t(G) * sl / ks;
       const int64_t tc = nu * tpu;
@@ -1009,30 +1028,32 @@ int64_t split_cost(int units, int tpu, int G, int ks, int grid) {
 // K slices for a layer: the candidate whose busiest CTA costs least (ties:
 // fewer slices). Cached per (units, tpu, G, grid): the choice is a few
 // hundred thousand steps of host arithmetic.
-int pick_ks(int units, int tpu, int G, int grid) {
+int pick_ks(int units, int tpu, int G, int grid, int tcap) {
   struct Key {
-    int units, tpu, G, grid;
+    int units, tpu, G, grid, tcap;
   };
   static std::mutex lock;
   static std::vector<std::pair<Key, int>> cache;
   {
     std::lock_guard<std::mutex> g(lock);
     for (const auto& e : cache)
-      if (e.first.units == units && e.first.tpu == tpu && e.first.G == G && e.first.grid == grid) return e.second;
+      if (e.first.units == units && e.first.tpu == tpu && e.first.G == G && e.first.grid == grid &&
+          e.first.tcap == tcap)
+        return e.second;
   }
   int best = 1;
-  int64_t best_cost = split_cost(units, tpu, G, 1, grid);
+  int64_t best_cost = split_cost(units, tpu, G, 1, grid, tcap);
   const int cands[] = {2, 3, 4, 5, 6, 7, 8, 10, 12, 14, 16, 24, 32};
   for (int ks : cands) {
     if (ks > G || ks > grid) break;
-    const int64_t c = split_cost(units, tpu, G, ks, grid);
+    const int64_t c = split_cost(units, tpu, G, ks, grid, tcap);
     if (c < best_cost) {
       best_cost = c;
       best = ks;
     }
   }
   std::lock_guard<std::mutex> g(lock);
-  if (cache.size() < 4096) cache.push_back({Key{units, tpu, G, grid}, best});
+  if (cache.size() < 4096) cache.push_back({Key{units, tpu, G, grid, tcap}, best});
   return best;
 }
 
@@ -1061,7 +1082,9 @@ awq_status_t make_chain_plan(const awq_gemv_layer_t* layers, int n, int64_t M, C
   }
   // Ring geometry: two CTAs per SM when each still holds three stages,
   // else one CTA per SM with the whole shared memory.
-  pl.stage_bytes = kXOff + int(M) * kXRowBytes;
+  // batch tiles of 2 and 4 rows: two-tile stages (see tile_cap)
+  pl.tcap = (M == 2 || M == 3 || M == 4) ? tile_cap<2>() : kMaxTC;
+  pl.stage_bytes = int(pl.tcap == 2 ? x_off<2>() : x_off<kMaxTC>()) + int(M) * kXRowBytes;
   const int pbuf_bytes = kCW * 64 * int(M) * 4;
   int per_sm = 2;
   for (;; --per_sm) {
@@ -1092,7 +1115,7 @@ awq_status_t make_chain_plan(const awq_gemv_layer_t* layers, int n, int64_t M, C
     lp.T = int((L.N + kTile - 1) / kTile);
     lp.tpu = (L.cfg.flags & AWQ_FLAG_SILU_MUL) ? 2 : 1;
     lp.units = lp.T / lp.tpu;
-    const int ks = pick_ks(lp.units, lp.tpu, int(G), pl.grid);
+    const int ks = pick_ks(lp.units, lp.tpu, int(G), pl.grid, pl.tcap);
     lp.ks = ks;
     lp.items = lp.units * ks;
     // A layer that reads the output of a layer of the current level starts a
