@@ -63,7 +63,7 @@
 extern "C" {
 #endif
 
-#define AWQ_ABI_VERSION 7
+#define AWQ_ABI_VERSION 8
 
 #if defined(__GNUC__)
 #define AWQ_API __attribute__((visibility("default")))

@@ -44,7 +44,7 @@ class AwqError(RuntimeError):
         self.status = status
 
 
-ABI_VERSION = 7   # awq_abi_version() of a library this binding matches
+ABI_VERSION = 8   # awq_abi_version() of a library this binding matches
 
 
 class QConfig(ctypes.Structure):
